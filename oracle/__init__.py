@@ -1,0 +1,218 @@
+"""fp64 CPU oracle of the sparse top-k MoE layer forward pass -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of ``bench.py`` may
+import this package.  The CUDA library and its Python binding never import it, and the two share no
+code; the only thing both sides see is the seeded input generator (``synth``), which holds no MoE
+arithmetic.
+
+The arithmetic lives in ``moe_oracle.c`` (plain loops in double, each function citing the page and
+section it follows).  This wrapper only marshals numpy arrays through ctypes and composes the
+documented steps:
+
+  route      -> logits, logsumexp, softmax, top-k (logit desc, index asc), renormalised weights
+  losses     -> Switch aux loss E*sum f*P (pre-drop counts / (T*k)), z-loss mean(lse^2)
+  dispatch   -> capacity ceil(CF*T*k/E) or unlimited; slot-major then token-order ranks; rows
+  forward    -> out[t] = sum over kept slots of w * FFN_e(x_t)
+
+Parity status of each function is recorded in the test-suite pins (``tests/test_oracle_pins.py``);
+every function here is pinned there against closed forms, library routines or brute force.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libmoe_oracle.so")
+_lib = None
+
+F32, BF16 = 0, 1
+_DT = {"f32": F32, "bf16": BF16}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain -O2, IEEE semantics kept: no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    i64, vp, c_int, dbl = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_double
+    lib.oracle_gelu.argtypes = [dbl]
+    lib.oracle_gelu.restype = dbl
+    lib.oracle_capacity.argtypes = [dbl, i64, i64, i64]
+    lib.oracle_capacity.restype = i64
+    lib.oracle_route.argtypes = [i64, i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.oracle_route.restype = None
+    lib.oracle_losses.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp]
+    lib.oracle_losses.restype = None
+    lib.oracle_dispatch.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.oracle_dispatch.restype = i64
+    lib.oracle_expert_rows.argtypes = [i64, i64, c_int, vp, vp, vp, vp, vp, i64, vp, vp, vp, c_int]
+    lib.oracle_expert_rows.restype = None
+    lib.oracle_forward_tokens.argtypes = [i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp,
+                                          c_int]
+    lib.oracle_forward_tokens.restype = None
+    lib.oracle_max_threads.argtypes = []
+    lib.oracle_max_threads.restype = c_int
+    lib.oracle_set_threads.argtypes = [c_int]
+    lib.oracle_set_threads.restype = None
+    _lib = lib
+    return lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data
+
+
+def _c(a, dtype=None):
+    a = np.ascontiguousarray(a) if dtype is None else np.ascontiguousarray(a, dtype=dtype)
+    return a
+
+
+def max_threads() -> int:
+    return _load().oracle_max_threads()
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def gelu(u: float) -> float:
+    return _load().oracle_gelu(float(u))
+
+
+def capacity(cf: float, T: int, k: int, E: int):
+    """Per-expert capacity, or None when unlimited (CF = +inf)."""
+    c = _load().oracle_capacity(float(cf), T, k, E)
+    return None if c < 0 else int(c)
+
+
+@dataclass
+class Routing:
+    logits: np.ndarray  # [T,E] f64
+    lse: np.ndarray  # [T] f64
+    p: np.ndarray  # [T,E] f64
+    topk_idx: np.ndarray  # [T,k] int32
+    topk_w: np.ndarray  # [T,k] f64
+    margin: np.ndarray  # [T] f64: smallest adjacent gap among the top-(k+1) logits
+
+
+def route(x, Wg, bg, k: int, dtype: str) -> Routing:
+    x, Wg, bg = _c(x), _c(Wg), _c(bg)
+    T, H = x.shape
+    E = Wg.shape[1]
+    logits = np.empty((T, E), np.float64)
+    lse = np.empty(T, np.float64)
+    p = np.empty((T, E), np.float64)
+    idx = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float64)
+    margin = np.empty(T, np.float64)
+    _load().oracle_route(T, H, E, k, _DT[dtype], _p(x), _p(Wg), _p(bg), _p(logits), _p(lse), _p(p), _p(idx),
+                         _p(w), _p(margin))
+    return Routing(logits, lse, p, idx, w, margin)
+
+
+def losses(p, lse, topk_idx):
+    p, lse, idx = _c(p, np.float64), _c(lse, np.float64), _c(topk_idx, np.int32)
+    T, E = p.shape if p.ndim == 2 else (0, 0)
+    k = idx.shape[1] if idx.ndim == 2 else 0
+    aux = np.zeros(1, np.float64)
+    z = np.zeros(1, np.float64)
+    _load().oracle_losses(T, E, k, _p(p), _p(lse), _p(idx), _p(aux), _p(z))
+    return float(aux[0]), float(z[0])
+
+
+@dataclass
+class Dispatch:
+    cap: int | None
+    cnt_pre: np.ndarray  # [E] int32
+    expert_counts: np.ndarray  # [E] int32
+    offsets: np.ndarray  # [E+1] int32
+    dropped: np.ndarray  # [T,k] uint8
+    row_of: np.ndarray  # [T,k] int32
+    row_token: np.ndarray  # [kept] int32
+    row_slot: np.ndarray  # [kept] int32
+
+    @property
+    def kept(self) -> int:
+        return int(self.offsets[-1])
+
+
+def dispatch(topk_idx, E: int, cf: float) -> Dispatch:
+    idx = _c(topk_idx, np.int32)
+    T, k = idx.shape
+    cap = capacity(cf, T, k, E)
+    cnt_pre = np.empty(E, np.int32)
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    dropped = np.empty((T, k), np.uint8)
+    row_of = np.empty((T, k), np.int32)
+    row_token = np.full(max(T * k, 1), -1, np.int32)
+    row_slot = np.full(max(T * k, 1), -1, np.int32)
+    kept = _load().oracle_dispatch(T, E, k, -1 if cap is None else cap, _p(idx), _p(cnt_pre), _p(counts),
+                                   _p(offsets), _p(dropped), _p(row_of), _p(row_token), _p(row_slot))
+    return Dispatch(cap, cnt_pre, counts, offsets, dropped, row_of, row_token[:kept].copy(),
+                    row_slot[:kept].copy())
+
+
+def expert_rows(x, W1, b1, W2, b2, tokens, experts, dtype: str, nthreads: int = 0) -> np.ndarray:
+    """y[i] = FFN_{experts[i]}(x[tokens[i]]) in double."""
+    x, W1, b1, W2, b2 = _c(x), _c(W1), _c(b1), _c(W2), _c(b2)
+    tokens, experts = _c(tokens, np.int32), _c(experts, np.int32)
+    E, H, F = W1.shape
+    n = tokens.shape[0]
+    y = np.empty((n, H), np.float64)
+    _load().oracle_expert_rows(H, F, _DT[dtype], _p(x), _p(W1), _p(b1), _p(W2), _p(b2), n, _p(tokens),
+                               _p(experts), _p(y), int(nthreads))
+    return y
+
+
+def forward_tokens(x, W1, b1, W2, b2, topk_idx, topk_w, dropped, tokens, dtype: str,
+                   nthreads: int = 0) -> np.ndarray:
+    """out[i] = sum over kept slots of w * FFN(x[tokens[i]]) in double, for the listed tokens."""
+    x, W1, b1, W2, b2 = _c(x), _c(W1), _c(b1), _c(W2), _c(b2)
+    idx, w = _c(topk_idx, np.int32), _c(topk_w, np.float64)
+    drp = None if dropped is None else _c(dropped, np.uint8)
+    tokens = _c(tokens, np.int32)
+    E, H, F = W1.shape
+    k = idx.shape[1]
+    n = tokens.shape[0]
+    out = np.empty((n, H), np.float64)
+    _load().oracle_forward_tokens(H, F, k, _DT[dtype], _p(x), _p(W1), _p(b1), _p(W2), _p(b2), _p(idx), _p(w),
+                                  _p(drp), n, _p(tokens), _p(out), int(nthreads))
+    return out
+
+
+@dataclass
+class Forward:
+    routing: Routing
+    aux: float
+    z: float
+    disp: Dispatch
+    out: np.ndarray | None  # [len(tokens), H] f64
+    tokens: np.ndarray
+
+
+def forward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=None, nthreads: int = 0) -> Forward:
+    """Whole layer: routing and dispatch over all tokens, FFN + combine for ``tokens`` (default: all)."""
+    r = route(x, Wg, bg, k, dtype)
+    aux, z = losses(r.p, r.lse, r.topk_idx)
+    d = dispatch(r.topk_idx, Wg.shape[1], cf)
+    T = x.shape[0]
+    tokens = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
+    out = forward_tokens(x, W1, b1, W2, b2, r.topk_idx, r.topk_w, d.dropped, tokens, dtype, nthreads)
+    return Forward(r, aux, z, d, out, tokens)

@@ -1,0 +1,356 @@
+"""Pins of the fp64 oracle against facts fixed outside the oracle itself (CPU only).
+
+Each pin checks the oracle against something other than its own code: textbook constants, closed
+forms that follow from the MoE definitions on the pages ("MoE Training: Mixture of Experts":
+Quick Start MoELayer; Core Concepts 2 Routing, 3 Load Balancing, 4 Expert Parallelism; Best
+Practices 2 Capacity Factor; Advanced Patterns Mixtral block), library routines (numpy fp64
+matmul, scipy logsumexp / softmax / erf / normal CDF), invariants and brute force on tiny inputs.
+Every pin is chosen so that a plausible slip in the oracle (a dropped bias, a transposed operand, a
+wrong sign, a wrong order of drops) fails it; ``test_planted_mistakes_are_caught`` demonstrates this
+on copies of the inputs.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+from scipy import special, stats
+
+import oracle
+import synth
+
+RNG_SEED = 1234
+
+
+def _rand_layer(T, H, E, F, seed, dtype="f32", bias_std=0.1):
+    cfg = synth.LayerConfig("t", T=T, H=H, E=E, k=1, F=F, CF=math.inf, dtype=dtype, seed=seed, bias_std=bias_std)
+    inp = synth.make_inputs(cfg)
+    # non-zero gate bias so a dropped bias term is visible
+    inp.bg = synth.normal(seed, 99, (E,), 0.0, 0.5, dtype)
+    return inp
+
+
+def _f64(a, dtype):
+    return synth.as_f64(a, dtype)
+
+
+# ---------------------------------------------------------------- GELU ---------------------------
+
+def test_gelu_textbook_values():
+    # GELU(u) = u * Phi(u); Phi at 0.5, 1, 2 from standard normal tables
+    assert oracle.gelu(0.0) == 0.0
+    assert oracle.gelu(1.0) == pytest.approx(0.8413447460685429, abs=1e-15)
+    assert oracle.gelu(-1.0) == pytest.approx(-(1 - 0.8413447460685429), abs=1e-15)
+    assert oracle.gelu(2.0) == pytest.approx(2 * 0.9772498680518208, abs=1e-15)
+    assert oracle.gelu(0.5) == pytest.approx(0.5 * 0.6914624612740131, abs=1e-15)
+    assert oracle.gelu(40.0) == 40.0
+    assert oracle.gelu(-40.0) == pytest.approx(0.0, abs=1e-300)
+
+
+def test_gelu_matches_normal_cdf():
+    for u in np.linspace(-8, 8, 161):
+        assert oracle.gelu(u) == pytest.approx(u * stats.norm.cdf(u), rel=1e-14, abs=1e-15)
+
+
+# ---------------------------------------------------------------- router -------------------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_route_logits_lse_softmax_vs_library(dtype):
+    inp = _rand_layer(T=37, H=24, E=7, F=8, seed=11, dtype=dtype)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, k=3, dtype=dtype)
+    x, Wg, bg = _f64(inp.x, dtype), _f64(inp.Wg, dtype), _f64(inp.bg, dtype)
+    logits = x @ Wg + bg
+    np.testing.assert_allclose(r.logits, logits, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r.lse, special.logsumexp(logits, axis=1), rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(r.p, special.softmax(logits, axis=1), rtol=1e-12, atol=1e-15)
+
+
+def test_route_topk_brute_force_and_renorm():
+    """Over every k-subset, the chosen set is the unique one whose worst member beats every
+    non-member under (logit desc, index asc); slots are in that order; weights are p renormalised."""
+    inp = _rand_layer(T=64, H=16, E=6, F=8, seed=5)
+    for k in (1, 2, 3, 6):
+        r = oracle.route(inp.x, inp.Wg, inp.bg, k=k, dtype="f32")
+        for t in range(64):
+            lg = r.logits[t]
+            key = lambda e: (lg[e], -e)  # noqa: E731
+            winners = [set(S) for S in itertools.combinations(range(6), k)
+                       if all(key(a) > key(b) for a in S for b in set(range(6)) - set(S))]
+            assert len(winners) == 1
+            assert set(r.topk_idx[t].tolist()) == winners[0]
+            ks = [key(e) for e in r.topk_idx[t]]
+            assert ks == sorted(ks, reverse=True)
+            psel = special.softmax(lg)[r.topk_idx[t]]
+            np.testing.assert_allclose(r.topk_w[t], psel / psel.sum(), rtol=1e-13)
+            assert r.topk_w[t].sum() == pytest.approx(1.0, abs=1e-14)
+
+
+def test_route_tie_break_lower_index_and_uniform_closed_form():
+    """Wg = 0, bg = 0: all logits equal -> p = 1/E, top-k = {0..k-1}, w = 1/k, lse = ln E."""
+    T, H, E, k = 9, 5, 8, 3
+    x = synth.normal(3, 1, (T, H))
+    Wg = np.zeros((H, E), np.float32)
+    bg = np.zeros(E, np.float32)
+    r = oracle.route(x, Wg, bg, k, "f32")
+    assert (r.topk_idx == np.arange(k)[None, :]).all()
+    np.testing.assert_allclose(r.topk_w, 1.0 / k, rtol=1e-15)
+    np.testing.assert_allclose(r.p, 1.0 / E, rtol=1e-15)
+    np.testing.assert_allclose(r.lse, math.log(E), rtol=1e-15)
+    assert (r.margin == 0).all()
+
+
+def test_route_k1_weight_is_one():
+    inp = _rand_layer(T=20, H=8, E=5, F=8, seed=8)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, 1, "f32")
+    assert (r.topk_w == 1.0).all()
+    assert (r.topk_idx[:, 0] == np.argmax(r.logits, axis=1)).all()  # Switch argmax routing
+
+
+def test_route_margin():
+    inp = _rand_layer(T=30, H=8, E=6, F=8, seed=9)
+    k = 2
+    r = oracle.route(inp.x, inp.Wg, inp.bg, k, "f32")
+    s = -np.sort(-r.logits, axis=1)
+    np.testing.assert_allclose(r.margin, np.min(s[:, :k] - s[:, 1:k + 1], axis=1), rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------- losses -------------------------
+
+def test_losses_uniform_closed_form():
+    """Equal logits: f and P uniform -> aux = 1 exactly; z = (ln E)^2; constant c -> (c + ln E)^2."""
+    T, H, E, k = 16, 4, 8, 2
+    x = synth.normal(4, 1, (T, H))
+    r = oracle.route(x, np.zeros((H, E), np.float32), np.zeros(E, np.float32), k, "f32")
+    # with ties every token picks {0,1}: f is not uniform -- use k = E to get uniform f
+    r8 = oracle.route(x, np.zeros((H, E), np.float32), np.zeros(E, np.float32), E, "f32")
+    aux, z = oracle.losses(r8.p, r8.lse, r8.topk_idx)
+    assert aux == pytest.approx(1.0, abs=1e-15)
+    assert z == pytest.approx(math.log(E) ** 2, rel=1e-15)
+    # f one-hot-ish on {0,1} (each 1/2), P uniform 1/E -> aux = E * (1/2*1/E + 1/2*1/E) = 1
+    aux2, _ = oracle.losses(r.p, r.lse, r.topk_idx)
+    assert aux2 == pytest.approx(1.0, abs=1e-15)
+    c = 2.5
+    rc = oracle.route(x, np.zeros((H, E), np.float32), np.full(E, c, np.float32), k, "f32")
+    _, zc = oracle.losses(rc.p, rc.lse, rc.topk_idx)
+    assert zc == pytest.approx((c + math.log(E)) ** 2, rel=1e-14)
+
+
+def test_losses_worked_example_two_experts():
+    """H=1, x=1, Wg=[[1,0]]: both tokens have logits (1,0) -> p=(e/(e+1), 1/(e+1)), both pick expert 0.
+    f=(1,0), P=p -> aux = 2 e/(e+1); z = ln(e+1)^2."""
+    x = np.ones((2, 1), np.float32)
+    Wg = np.array([[1.0, 0.0]], np.float32)
+    r = oracle.route(x, Wg, np.zeros(2, np.float32), 1, "f32")
+    aux, z = oracle.losses(r.p, r.lse, r.topk_idx)
+    e = math.e
+    assert aux == pytest.approx(2 * e / (e + 1), rel=1e-15)
+    assert z == pytest.approx(math.log(e + 1) ** 2, rel=1e-15)
+
+
+def test_losses_one_hot_limit_equals_E():
+    """f and P both concentrated on one expert -> aux -> E (upper bound)."""
+    T, H, E, k = 10, 3, 6, 1
+    x = synth.normal(6, 1, (T, H))
+    bg = np.zeros(E, np.float32)
+    bg[2] = 60.0
+    r = oracle.route(x, np.zeros((H, E), np.float32), bg, k, "f32")
+    aux, _ = oracle.losses(r.p, r.lse, r.topk_idx)
+    assert aux == pytest.approx(E, rel=1e-20 + 1e-12)
+    assert aux <= E
+
+
+def test_losses_bound_and_permutation_invariance():
+    inp = _rand_layer(T=50, H=12, E=5, F=8, seed=21)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, 2, "f32")
+    aux, z = oracle.losses(r.p, r.lse, r.topk_idx)
+    assert 0 < aux <= 5
+    perm = np.random.default_rng(RNG_SEED).permutation(50)
+    aux2, z2 = oracle.losses(r.p[perm], r.lse[perm], r.topk_idx[perm])
+    assert aux2 == pytest.approx(aux, rel=1e-14) and z2 == pytest.approx(z, rel=1e-14)
+
+
+def test_losses_empty_batch():
+    aux, z = oracle.losses(np.zeros((0, 4)), np.zeros(0), np.zeros((0, 2), np.int32))
+    assert aux == 0.0 and z == 0.0
+
+
+# ---------------------------------------------------------------- capacity / dispatch ------------
+
+def test_capacity_values():
+    assert oracle.capacity(1.25, 8192, 1, 128) == 80
+    assert oracle.capacity(math.inf, 8192, 1, 128) is None
+    assert oracle.capacity(1.0, 10, 1, 3) == 4  # ceil(10/3)
+    assert oracle.capacity(2.0, 256, 2, 4) == 256
+    assert oracle.capacity(1.25, 4096, 2, 8) == 1280
+
+
+def _check_dispatch_invariants(idx, E, d):
+    T, k = idx.shape
+    cap = d.cap
+    drops = int(d.dropped.sum())
+    assert d.expert_counts.sum() == T * k - drops
+    assert (d.cnt_pre == np.bincount(idx.ravel(), minlength=E)).all()
+    if cap is not None:
+        assert (d.expert_counts <= cap).all()
+        assert (d.expert_counts == np.minimum(d.cnt_pre, cap)).all()
+    else:
+        assert drops == 0
+    assert (np.diff(d.offsets) == d.expert_counts).all() and d.offsets[0] == 0
+    # rows are a bijection onto the kept assignments
+    kept = [(t, s) for t in range(T) for s in range(k) if not d.dropped[t, s]]
+    assert sorted(zip(d.row_token.tolist(), d.row_slot.tolist())) == sorted(kept)
+    for t, s in kept:
+        r = d.row_of[t, s]
+        assert d.row_token[r] == t and d.row_slot[r] == s
+        assert d.offsets[idx[t, s]] <= r < d.offsets[idx[t, s] + 1]
+    assert (d.row_of[d.dropped == 1] == -1).all()
+    # stability: inside each expert's segment rows go (slot, token) increasing
+    for e in range(E):
+        seg = list(zip(d.row_slot[d.offsets[e]:d.offsets[e + 1]], d.row_token[d.offsets[e]:d.offsets[e + 1]]))
+        assert seg == sorted(seg)
+    # the kept set of each expert is the first `cap` of its assignments in (slot, token) order
+    for e in range(E):
+        order = [(s, t) for s in range(k) for t in range(T) if idx[t, s] == e]
+        keep = order if cap is None else order[:cap]
+        assert sorted(keep) == sorted((s, t) for (s, t) in order if not d.dropped[t, s])
+
+
+@pytest.mark.parametrize("k,cf", [(1, 1.25), (2, 1.25), (2, 1.0), (3, 0.5), (2, math.inf), (1, 100.0)])
+def test_dispatch_invariants_random(k, cf):
+    rng = np.random.default_rng(k * 100 + int(min(cf, 99) * 10))
+    T, E = 97, 6
+    # skewed assignments: distinct experts per token, expert 0 popular
+    idx = np.empty((T, k), np.int32)
+    for t in range(T):
+        p = np.array([6, 3, 2, 1, 1, 1], float)
+        idx[t] = rng.choice(E, size=k, replace=False, p=p / p.sum())
+    d = oracle.dispatch(idx, E, cf)
+    _check_dispatch_invariants(idx, E, d)
+
+
+def test_dispatch_closed_form_same_expert():
+    """Wg = 0 with distinct bg: every token picks the same expert (k=1); with CF=1.25 exactly
+    cap = ceil(1.25*T/E) tokens -- the first cap in token order -- are kept."""
+    T, H, E = 40, 4, 8
+    x = synth.normal(7, 1, (T, H))
+    bg = np.linspace(-1, 1, E).astype(np.float32)  # expert E-1 wins
+    r = oracle.route(x, np.zeros((H, E), np.float32), bg, 1, "f32")
+    assert (r.topk_idx[:, 0] == E - 1).all()
+    d = oracle.dispatch(r.topk_idx, E, 1.25)
+    cap = math.ceil(1.25 * T / E)
+    assert d.cap == cap == 7
+    assert d.expert_counts[E - 1] == cap and d.expert_counts[:E - 1].sum() == 0
+    assert (d.dropped[:cap, 0] == 0).all() and (d.dropped[cap:, 0] == 1).all()
+    assert d.row_token.tolist() == list(range(cap))
+
+
+def test_dispatch_slot_major_drop_order():
+    """Slot 0 of every token is placed before any slot 1: with cap=2 and tokens (0:[a,b], 1:[b,a],
+    2:[a,b]) expert a keeps t0s0, t2s0 and drops t1s1; expert b keeps t1s0, t0s1 and drops t2s1."""
+    idx = np.array([[0, 1], [1, 0], [0, 1]], np.int32)
+    d = oracle.dispatch(idx, 2, cf=2 * 2 / (3 * 2))  # ceil(CF*T*k/E) = ceil(0.6667*6/2) = 2
+    assert d.cap == 2
+    assert d.dropped.tolist() == [[0, 0], [0, 1], [0, 1]]
+    assert d.row_token.tolist() == [0, 2, 1, 0]
+    assert d.row_slot.tolist() == [0, 0, 0, 1]
+
+
+def test_dispatch_empty():
+    d = oracle.dispatch(np.zeros((0, 2), np.int32), 4, math.inf)
+    assert d.kept == 0 and (d.expert_counts == 0).all()
+
+
+# ---------------------------------------------------------------- FFN / combine -----------------
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_expert_rows_vs_numpy_matmul(dtype):
+    inp = _rand_layer(T=11, H=24, E=3, F=40, seed=31, dtype=dtype)
+    tokens = np.array([0, 3, 10, 3, 7], np.int32)
+    experts = np.array([2, 0, 1, 1, 2], np.int32)
+    y = oracle.expert_rows(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, tokens, experts, dtype)
+    x, W1, b1, W2, b2 = (_f64(a, dtype) for a in (inp.x, inp.W1, inp.b1, inp.W2, inp.b2))
+    for i, (t, e) in enumerate(zip(tokens, experts)):
+        u = x[t] @ W1[e] + b1[e]
+        g = u * stats.norm.cdf(u)
+        ref = g @ W2[e] + b2[e]
+        np.testing.assert_allclose(y[i], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_identical_experts_equal_dense_ffn():
+    """All experts share weights and the k weights sum to 1 -> layer output = one dense FFN."""
+    T, H, E, F, k = 23, 16, 5, 32, 2
+    inp = _rand_layer(T=T, H=H, E=1, F=F, seed=41)
+    W1 = np.repeat(inp.W1, E, 0)
+    b1 = np.repeat(inp.b1, E, 0)
+    W2 = np.repeat(inp.W2, E, 0)
+    b2 = np.repeat(inp.b2, E, 0)
+    Wg = synth.normal(41, 50, (H, E), 0, 0.3)
+    bg = synth.normal(41, 51, (E,), 0, 0.3)
+    f = oracle.forward(inp.x, Wg, bg, W1, b1, W2, b2, k, math.inf, "f32")
+    x = inp.x.astype(np.float64)
+    u = x @ inp.W1[0].astype(np.float64) + inp.b1[0]
+    dense = (u * stats.norm.cdf(u)) @ inp.W2[0].astype(np.float64) + inp.b2[0]
+    np.testing.assert_allclose(f.out, dense, rtol=1e-11, atol=1e-12)
+
+
+def test_k_equals_E_is_dense_softmax_mixture():
+    T, H, E, F = 19, 12, 4, 20
+    inp = _rand_layer(T=T, H=H, E=E, F=F, seed=43)
+    f = oracle.forward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, E, math.inf, "f32")
+    x = inp.x.astype(np.float64)
+    p = special.softmax(x @ inp.Wg.astype(np.float64) + inp.bg, axis=1)
+    ref = np.zeros((T, H))
+    for e in range(E):
+        u = x @ inp.W1[e].astype(np.float64) + inp.b1[e]
+        ref += p[:, e:e + 1] * ((u * stats.norm.cdf(u)) @ inp.W2[e].astype(np.float64) + inp.b2[e])
+    np.testing.assert_allclose(f.out, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_forward_drops_contribute_nothing():
+    """CF small enough to drop: out[t] = sum over kept slots only; all-dropped tokens are zero."""
+    T, H, E, F, k = 40, 8, 4, 16, 2
+    inp = _rand_layer(T=T, H=H, E=E, F=F, seed=47)
+    f = oracle.forward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, k, 0.25, "f32")
+    assert f.disp.dropped.sum() > 0
+    allk = oracle.forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, f.routing.topk_idx, f.routing.topk_w, None,
+                                 np.arange(T), "f32")
+    ys = {}
+    for t in range(T):
+        ys[t] = oracle.expert_rows(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, np.array([t, t]), f.routing.topk_idx[t],
+                                   "f32")
+        ref = sum(f.routing.topk_w[t, s] * ys[t][s] for s in range(k) if not f.disp.dropped[t, s])
+        ref = np.zeros(H) if isinstance(ref, int) else ref
+        np.testing.assert_allclose(f.out[t], ref, rtol=1e-13, atol=1e-14)
+        full = sum(f.routing.topk_w[t, s] * ys[t][s] for s in range(k))
+        np.testing.assert_allclose(allk[t], full, rtol=1e-13, atol=1e-14)
+    all_dropped = np.where(f.disp.dropped.all(axis=1))[0]
+    assert len(all_dropped) > 0
+    assert (f.out[all_dropped] == 0).all()
+
+
+def test_forward_token_subset_matches_full():
+    T, H, E, F, k = 30, 8, 4, 12, 2
+    inp = _rand_layer(T=T, H=H, E=E, F=F, seed=53)
+    full = oracle.forward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, k, 1.0, "f32")
+    sub = np.array([29, 0, 13], np.int32)
+    part = oracle.forward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, k, 1.0, "f32", tokens=sub)
+    np.testing.assert_array_equal(part.out, full.out[sub])
+
+
+# ---------------------------------------------------------------- planted mistakes ---------------
+
+def test_planted_mistakes_are_caught():
+    """Mistakes planted in a Python restatement's inputs (not in the oracle) show the pins have teeth:
+    a transposed gate, a dropped gate bias and a flipped drop order each change the checked values."""
+    inp = _rand_layer(T=37, H=24, E=7, F=8, seed=11)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, 3, "f32")
+    x, Wg, bg = inp.x.astype(np.float64), inp.Wg.astype(np.float64), inp.bg.astype(np.float64)
+    assert not np.allclose(r.logits, x @ Wg)  # dropped bias is visible
+    Wsq = synth.normal(2, 2, (7, 7))
+    r2 = oracle.route(synth.normal(2, 3, (5, 7)), Wsq, np.zeros(7, np.float32), 2, "f32")
+    xs = synth.normal(2, 3, (5, 7)).astype(np.float64)
+    assert not np.allclose(r2.logits, xs @ Wsq.T.astype(np.float64))  # transposed gate is visible
+    idx = np.array([[0, 1], [1, 0], [0, 1]], np.int32)
+    d = oracle.dispatch(idx, 2, 2 * 2 / 6)
+    token_major_drop = [[0, 0], [1, 0], [0, 1]]  # what token-major order would give
+    assert d.dropped.tolist() != token_major_drop
