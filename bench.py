@@ -1,0 +1,396 @@
+"""Benchmark of the sparse top-k MoE layer forward pass on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+Workload: the Mixtral-shaped layer (T=4096 tokens, H=4096, E=8 experts, top-2, F=14336, GELU FFN
+with biases, dropless; bf16 storage, fp32 accumulation), synthetic seeded inputs.  A step is one
+whole forward pass (router, permutation, both grouped GEMMs with the fused combine) through the
+C-ABI call moe_forward; inputs are resident in HBM when the timed region starts.  The expert
+weights (1.88 GB) stream through L2 every step, so the inputs are larger than L2 and no flush is
+needed.  ``e2e`` times moe_forward_host: per step it copies x from pinned host memory to the device
+and out back to pinned host memory.  With N GPUs (torchrun), every rank runs its own replica on its
+own batch (no data-path collective; the layer shards by tokens), timing is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded token sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer fwd tokens/sec (Mixtral shape, 1 B200); grouped-GEMM % of BF16 peak"
+
+
+def workload_config(cfg: synth.LayerConfig) -> str:
+    cf = "dropless" if math.isinf(cfg.CF) else f"CF={cfg.CF}"
+    return (f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} F={cfg.F} {cf}, GELU FFN with biases, "
+            f"{cfg.dtype} storage / fp32 accumulate")
+
+
+def alg_flops(cfg: synth.LayerConfig, kept: int) -> float:
+    """4*H*F per kept assignment (two GEMMs) + 2*T*H*E for the gate."""
+    return 4.0 * cfg.H * cfg.F * kept + 2.0 * cfg.T * cfg.H * cfg.E
+
+
+def alg_bytes(cfg: synth.LayerConfig, touched_experts: int) -> float:
+    es = 2 if cfg.dtype == "bf16" else 4
+    w = touched_experts * (2 * cfg.H * cfg.F + cfg.F + cfg.H) * es
+    return w + cfg.T * cfg.H * es + cfg.T * cfg.H * 4 + cfg.H * cfg.E * es
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.gpu_id:
+            cmd.insert(1, f"--id={self.gpu_id}")
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+                power.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        thr = max(power) * 0.5 if power else 0
+        loaded = [s for s, p in zip(sm, power) if p >= thr] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ------------------------------------------------------------------------------------------------
+def cpu_oracle_rate(cfg: synth.LayerConfig, inp: synth.LayerInputs, budget_s: float, max_tokens: int = 4096):
+    """Tokens/s of the fp64 oracle (routing + dispatch + FFN + combine) on a leading token sample,
+    growing the sample until one run lasts at least budget_s / 3."""
+    import oracle
+
+    oracle.build()
+    threads = oracle.max_threads()
+    n = 2
+    best = None
+    spent = 0.0
+    while True:
+        t0 = time.perf_counter()
+        oracle.forward(inp.x[:n], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+        dt = time.perf_counter() - t0
+        spent += dt
+        best = (n, dt)
+        if dt >= budget_s / 3 or n >= max_tokens or spent + 2.2 * dt > budget_s:
+            break
+        n *= 2
+    n, dt = best
+    return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {n} tokens of the {cfg.name} workload as one layer call (routing, dispatch, "
+                      f"expert FFN, combine in fp64), {dt:.2f} s"}
+
+
+def run_reference(args, cfg):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+
+    inp = synth.make_inputs(cfg)
+    oracle.build()
+    threads = oracle.max_threads()
+    # calibrate tokens per step so the whole run stays within about two minutes
+    t0 = time.perf_counter()
+    oracle.forward(inp.x[:1], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+    t1 = time.perf_counter() - t0
+    per_step = 120.0 / max(1, args.steps + args.warmup)
+    S = int(max(1, min(cfg.T, per_step / max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        oracle.forward(inp.x[:S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        lo = (i * S) % max(1, cfg.T - S + 1)
+        oracle.forward(inp.x[lo:lo + S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+    dt = time.perf_counter() - t0
+    value = S * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_config(cfg), "global_batch": S, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{S} tokens per step of the {cfg.name} workload (fp64 oracle, OpenMP)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------------------------
+def _upload(arr, dtype):
+    import torch
+
+    if dtype == "bf16":
+        return torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32)).cuda()
+
+
+def run_ours_impl(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_23_b200 as moe
+    from sparse_mixture_experts_23_b200 import build as moe_build
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=180), device_id=torch.device("cuda", local))
+        if rank == 0:
+            moe_build.build()
+        dist.barrier()
+    else:
+        moe_build.build()
+    moe.load_library()
+
+    inp = synth.make_inputs(cfg)
+    if rank > 0:  # each replica routes its own batch through the same layer weights
+        inp.x = synth.x_batch(cfg, rank)
+    dev = {n: _upload(a, cfg.dtype) for n, a in inp.arrays().items()}
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype)
+    buf = moe.MoEBuffers(shape, dev)
+    stream = torch.cuda.current_stream()
+    peaks = load_peaks()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        uuid = None
+    sampler = ClockSampler(uuid if rank == 0 else None)
+
+    def sync_all():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        buf.forward()
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.5)  # let the sampler take its first reading
+    # ---------------- timed region: K whole forward passes -----------------------------------
+    sync_all()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        buf.forward()
+    ev1.record(stream)
+    sync_all()
+    launches_per_step = moe.moe_last_launch_count()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_step = ms_total / args.steps
+    value = world * cfg.T * args.steps / (ms_total / 1000.0)
+
+    # ---------------- per-kernel timing (same stream, CUDA events, inputs > L2) ---------------
+    reps = max(args.steps, 20)
+
+    def time_calls(fn) -> float:
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
+    ms_ffn = time_calls(lambda: buf.expert_ffn(True))
+    ms_route = time_calls(buf.route)
+    ms_permute = time_calls(buf.permute)
+    buf.forward()
+    torch.cuda.synchronize()
+    counts = buf.expert_counts.cpu().numpy()
+    kept = int(counts.sum())
+    touched = int((counts > 0).sum())
+    drops = int(buf.dropped.cpu().numpy().sum())
+    losses = buf.losses.cpu().numpy()
+
+    # ---------------- e2e: host buffers through moe_forward_host ----------------------------
+    es = 2 if cfg.dtype == "bf16" else 4
+    x_host = torch.from_numpy(np.ascontiguousarray(inp.x).view(np.int16 if es == 2 else np.float32))
+    if es == 2:
+        x_host = x_host.view(torch.bfloat16)
+    x_host = x_host.pin_memory()
+    out_host = torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
+    for _ in range(2):
+        buf.forward_host(x_host, out_host)
+    sync_all()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        buf.forward_host(x_host, out_host)
+    e1.record(stream)
+    sync_all()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * cfg.T * args.steps / (ms_e2e / 1000.0)
+
+    clocks = sampler.stop() if rank == 0 else None
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    ffn_flops = 4.0 * cfg.H * cfg.F * kept
+    tflops = ffn_flops / (ms_ffn / 1000.0) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    router_bytes = cfg.T * cfg.H * es + cfg.H * cfg.E * es + cfg.T * cfg.k * 8
+    # permute: read the kept x rows, write them to x_perm, clear out (fp32), index traffic
+    permute_bytes = kept * cfg.H * es * 2 + cfg.T * cfg.H * 4 + cfg.T * cfg.k * 8
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get(cfg.name, {}).get("grouped_gemm_bytes_per_launch")
+        except Exception:
+            traffic = None
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_rate(cfg, inp, budget_s=args.cpu_budget)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": workload_config(cfg), "global_batch": world * cfg.T, "seq_len": None,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: the expert weights (%.2f GB) stream every step" %
+                         (cfg.E * 2 * cfg.H * cfg.F * es / 1e9)},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                     "traffic": traffic,
+                     "kernel": "grouped GEMM pair (GEMM1 bias+GELU, GEMM2 scale+combine), one moe_expert_ffn call",
+                     "peak_source": f"{peaks['source']} bf16 sustained"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": cfg.T * cfg.H * es,
+                "d2h_bytes_per_step": cfg.T * cfg.H * 4},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "kernels": {
+            "ffn_ms": ms_ffn, "route_ms": ms_route, "permute_ms": ms_permute,
+            "ffn_tflops": tflops, "ffn_frac_burst_peak": tflops / peaks["bf16_tflops"],
+            "route_gbs": router_bytes / (ms_route / 1000.0) / 1e9,
+            "permute_gbs": permute_bytes / (ms_permute / 1000.0) / 1e9,
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+            "layer_roofline_ms": 1000 * max(alg_flops(cfg, kept) / (peaks["bf16_tflops"] * 1e12),
+                                            alg_bytes(cfg, touched) / (peaks["hbm_gbs"] * 1e9)),
+        },
+        "layer": {"kept": kept, "dropped": drops, "touched_experts": touched, "aux_loss": float(losses[0]),
+                  "z_loss": float(losses[1]), "expert_counts_min_max": [int(counts.min()), int(counts.max())]},
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="mixtral", choices=list(synth.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
+    for dim in ("T", "H", "E", "k", "F"):
+        ap.add_argument(f"--{dim}", type=int, default=None, help=f"override {dim} of the workload (profiling)")
+    args = ap.parse_args()
+    cfg = synth.CONFIGS[args.config]
+    over = {d: getattr(args, d) for d in ("T", "H", "E", "k", "F") if getattr(args, d) is not None}
+    if over:
+        cfg = cfg.with_(name=cfg.name + "[" + ",".join(f"{d}={v}" for d, v in over.items()) + "]", **over)
+    if args.impl == "reference":
+        run_reference(args, cfg)
+    else:
+        run_ours_impl(args, cfg)
+
+
+if __name__ == "__main__":
+    main()

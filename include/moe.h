@@ -1,0 +1,198 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse top-k Mixture-of-Experts layer forward pass.
+ *
+ * The layer (web page "MoE Training: Mixture of Experts", Quick Start "Basic MoE Architecture",
+ * class MoELayer; Core Concepts 2-4; Advanced Patterns "Mixtral 8x7B Architecture") maps
+ * x[T,H] to out[T,H] in four steps, each one entry point below:
+ *
+ *   moe_route       gate logits = x.Wg + bg, softmax, top-k, renormalised top-k weights,
+ *                   Switch load-balancing loss and router z-loss           (Core Concepts 2, 3)
+ *   moe_permute     per-expert counts, capacity, drop order, stable permutation of token rows
+ *                   into expert-contiguous segments                        (Core Concepts 4;
+ *                                                                           Best Practices 2)
+ *   moe_expert_ffn  per-expert Linear(H,F) -> GELU -> Linear(F,H) as two grouped GEMMs
+ *                   (Quick Start expert FFN), optionally with the weighted combine fused in
+ *   moe_combine     out[t] = sum over kept slots of w[t,s] * y[row(t,s)]     (Quick Start
+ *                                                          "output[mask] += score * output";
+ *                                                          Mixtral block index_add_)
+ *   moe_forward     the four chained on one stream (fused combine)
+ *
+ * Conventions shared by every entry point
+ *  - All tensors are row-major and contiguous.  Every pointer in moe_io_t is a DEVICE pointer
+ *    owned by the caller; the library never allocates device memory and never frees it.
+ *  - Storage dtype (moe_shape_t.dtype) applies to x, Wg, bg, W1, b1, W2, b2: MOE_DTYPE_F32 or
+ *    MOE_DTYPE_BF16.  Accumulation is fp32 everywhere.  out, topk_w and the losses are fp32.
+ *  - All work is asynchronous on the given stream (0 = legacy default stream).  No entry point
+ *    synchronises except moe_get_device_status.
+ *  - Arguments are validated on the host before anything is launched:
+ *      MOE_ERR_INVALID_ARG  null shape/io/workspace pointer, a needed io pointer that is null, a
+ *                           device pointer of x/Wg/W1/W2/out/workspace not 16-byte aligned,
+ *                           T < 0, H/E/F/k <= 0, k > E, k > 8, E > 256, capacity_factor <= 0 or
+ *                           NaN, unknown dtype
+ *      MOE_ERR_UNSUPPORTED  bf16 with H or F not a multiple of 64; f32 with H or F not a multiple
+ *                           of 4; T*k*max(H,F) beyond 2^31 elements
+ *      MOE_ERR_WORKSPACE    ws_bytes < moe_workspace_size(shape)
+ *      MOE_ERR_CUDA         a launch or driver call failed (the CUDA error is not cleared)
+ *    On any error nothing has been launched by that call.
+ *  - The workspace is a caller-allocated device buffer of moe_workspace_size() bytes, 256-byte
+ *    aligned, whose first 256 bytes (the device error word) must be zero before its first use
+ *    (e.g. cudaMemsetAsync(ws, 0, 256, stream)); afterwards the library keeps them.  It carries state from moe_route to moe_permute to moe_expert_ffn to moe_combine, so
+ *    one workspace serves one layer invocation at a time; calls on distinct workspaces are
+ *    independent and may run concurrently on different streams.
+ *  - T = 0 is valid: every entry point returns MOE_OK; moe_route writes aux_loss = z_loss = 0 and
+ *    moe_permute writes expert_counts = 0.
+ *  - Device-side waits (pipeline barriers in the tensor-core kernels) are bounded.  A wait that
+ *    runs out records an error word in the workspace and the kernel returns early;
+ *    moe_get_device_status() reports it as MOE_ERR_TIMEOUT.  No kernel traps.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,
+  MOE_ERR_UNSUPPORTED = 2,
+  MOE_ERR_WORKSPACE = 3,
+  MOE_ERR_CUDA = 4,
+  MOE_ERR_TIMEOUT = 5
+} moe_status_t;
+
+typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
+
+/* Problem statement.  capacity_factor = +INFINITY means dropless.  Per-expert capacity is
+ * ceil(capacity_factor * T * k / E) evaluated in double ("MoE Training" page, Core Concepts 4 and
+ * Best Practices 2 give capacity = tokens * CF / E; k counts the assignments of top-k routing). */
+typedef struct {
+  int32_t T;              /* tokens (batch * sequence), >= 0 */
+  int32_t H;              /* hidden size */
+  int32_t E;              /* experts, 1..256 */
+  int32_t F;              /* FFN width of each expert */
+  int32_t k;              /* experts per token, 1..min(E, 8) */
+  double capacity_factor; /* > 0; +INFINITY = no capacity limit */
+  moe_dtype_t dtype;      /* storage type of x and all weights */
+} moe_shape_t;
+
+/* Caller-owned device buffers.  Layouts (row-major):
+ *   x[T,H] Wg[H,E] bg[E] W1[E,H,F] b1[E,F] W2[E,F,H] b2[E,H]       storage dtype, read only
+ *   out[T,H]           fp32  layer output
+ *   topk_idx[T,k]      int32 chosen experts, slot s = rank s by (logit desc, expert index asc)
+ *   topk_w[T,k]        fp32  softmax probabilities of the chosen experts divided by their sum
+ *                            (pre-drop values; dropped slots keep their weight here)
+ *   expert_counts[E]   int32 kept assignments per expert (after capacity)
+ *   dropped[T,k]       uint8 1 = assignment dropped by capacity
+ *   aux_loss, z_loss   fp32 scalars: E*sum_e f_e*P_e and mean_t logsumexp_t^2, no coefficients */
+typedef struct {
+  const void* x;
+  const void* Wg;
+  const void* bg;
+  const void* W1;
+  const void* b1;
+  const void* W2;
+  const void* b2;
+  float* out;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* expert_counts;
+  uint8_t* dropped;
+  float* aux_loss;
+  float* z_loss;
+} moe_io_t;
+
+/* Pointers into a workspace, for inspection of the intermediate stages. */
+typedef struct {
+  int32_t* status;     /* device error word (0 = ok) */
+  int32_t* offsets;    /* [E+1] exclusive prefix sum of expert_counts; offsets[E] = kept rows */
+  int32_t* cnt_pre;    /* [E] assignments per expert before capacity */
+  int32_t* row_of;     /* [T,k] row of assignment (t,s) in x_perm, -1 if dropped */
+  int32_t* row_token;  /* [T*k] token of each row (rows >= offsets[E] unused) */
+  int32_t* row_slot;   /* [T*k] slot of each row */
+  void* x_perm;        /* [T*k, H] storage dtype: x rows grouped by expert, (slot, token) order */
+  void* h;             /* [T*k, F] storage dtype: GELU(x_perm . W1[e] + b1[e]) */
+  float* y;            /* [T*k, H] fp32: h . W2[e] + b2[e] (only written when the combine is not fused) */
+  size_t bytes;        /* total workspace size */
+} moe_ws_view_t;
+
+/* Workspace bytes for a shape; 0 if the shape is invalid.  Host only, pure. */
+MOE_API size_t moe_workspace_size(const moe_shape_t* shape);
+
+/* Pointers to each stage buffer inside `ws` for `shape`.  Host only, pure. */
+MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, moe_ws_view_t* view);
+
+/* Router ("MoE Training" page, Quick Start MoELayer.forward: gate, softmax, topk, renormalise;
+ * Core Concepts 3: load_balancing_loss, router_z_loss).
+ * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws). */
+MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Dispatch (Core Concepts 4 "capacity_factor", "drop_tokens"; Best Practices 2; Advanced Patterns
+ * Mixtral block gather by expert).  Assignments are visited slot-major then by token; an
+ * assignment is kept iff fewer than `capacity` earlier assignments went to its expert.
+ * Reads x, topk_idx.  Writes expert_counts, dropped, the row maps and x_perm in ws, and clears
+ * out[T,H] to zero (the fused combine accumulates into it). */
+MOE_API moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* Expert FFN (Quick Start expert: Linear(H, F) -> GELU(erf) -> Linear(F, H), with biases) as two
+ * grouped GEMMs over the expert segments of x_perm.  bf16: tcgen05 tensor cores, h stored bf16;
+ * f32: CUDA cores, h stored f32.  fuse_combine != 0: out[t] += topk_w[t,s]*(h.W2[e] + b2[e]) for
+ * every kept row (out must hold zeros from moe_permute); at most k fp32 adds reach each element,
+ * so for k <= 2 the result does not depend on their order.  fuse_combine == 0: y in ws is
+ * written instead and out is untouched.  Reads W1, b1, W2, b2, topk_w and the ws state of
+ * moe_permute. */
+MOE_API moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                            int fuse_combine, cudaStream_t stream);
+
+/* Combine from a materialised y (Quick Start "output[mask] += expert_scores * expert_output"):
+ * out[t] = sum over kept slots s, in slot order, of topk_w[t,s] * y[row_of(t,s)]; tokens with
+ * every slot dropped get zeros.  Overwrites out.  Use after moe_expert_ffn(fuse_combine = 0). */
+MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream. */
+MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* The same forward pass for callers whose activations live in host memory: copies x_host
+ * (T*H elements of the storage dtype) to io->x, runs moe_forward, and copies io->out back to
+ * out_host (T*H fp32), all asynchronously on `stream` (pinned host memory makes the copies
+ * asynchronous).  io->x must be a writable device buffer.  Does not synchronise. */
+MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_io_t* io, const void* x_host,
+                              float* out_host, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the workspace's device error word.
+ * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out) or MOE_ERR_CUDA. */
+MOE_API moe_status_t moe_get_device_status(void* ws, cudaStream_t stream);
+
+/* Bound on device-side waits, in GPU clock cycles (default 2e9, about one second).  Applies to
+ * launches made after the call.  Values <= 0 restore the default. */
+MOE_API void moe_set_wait_limit(long long cycles);
+
+/* Launches one block that waits on a pipeline barrier nothing will ever complete, with the
+ * current wait bound; it must come back with the error word set.  For testing the timeout path. */
+MOE_API moe_status_t moe_debug_timeout_probe(void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Number of kernels the last moe_* call launched on the host thread (for launch accounting). */
+MOE_API int moe_last_launch_count(void);
+
+MOE_API const char* moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

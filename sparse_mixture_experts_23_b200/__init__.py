@@ -1,0 +1,226 @@
+"""Python binding of the B200 sparse top-k MoE forward library (``libmoe.so``, C ABI in include/moe.h).
+
+This module only marshals arguments: it mirrors the C structs with ctypes and calls the entry
+points by the same names.  Every step of the layer runs in the CUDA kernels of ``libmoe.so``;
+there is no Python or CPU fallback, and loading fails loudly when the library is missing.
+PyTorch is used by ``MoEBuffers`` only to allocate device memory and to hand over its stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
+DTYPES = {"f32": MOE_DTYPE_F32, "bf16": MOE_DTYPE_BF16}
+
+ENTRY_POINTS = (
+    "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+    "moe_forward", "moe_forward_host", "moe_get_device_status", "moe_set_wait_limit", "moe_debug_timeout_probe",
+    "moe_last_launch_count", "moe_status_string",
+)
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32), ("F", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_double), ("dtype", ctypes.c_int)]
+
+
+class IO(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("x", "Wg", "bg", "W1", "b1", "W2", "b2", "out", "topk_idx", "topk_w",
+                                               "expert_counts", "dropped", "aux_loss", "z_loss")]
+
+
+class WsView(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("status", "offsets", "cnt_pre", "row_of", "row_token", "row_slot",
+                                               "x_perm", "h", "y")] + [("bytes", ctypes.c_size_t)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load ``libmoe.so``; raises if it has not been built (run ``sparse_mixture_experts_23_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"CUDA library not built: {path} is missing (python -m sparse_mixture_experts_23_b200.build)")
+    lib = ctypes.CDLL(path)
+    P, vp, sz, st = ctypes.POINTER, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    lib.moe_workspace_size.argtypes = [P(Shape)]
+    lib.moe_workspace_size.restype = sz
+    lib.moe_workspace_layout.argtypes = [P(Shape), vp, P(WsView)]
+    lib.moe_workspace_layout.restype = st
+    for name in ("moe_route", "moe_permute", "moe_combine", "moe_forward"):
+        fn = getattr(lib, name)
+        fn.argtypes = [P(Shape), P(IO), vp, sz, vp]
+        fn.restype = st
+    lib.moe_expert_ffn.argtypes = [P(Shape), P(IO), vp, sz, ctypes.c_int, vp]
+    lib.moe_expert_ffn.restype = st
+    lib.moe_forward_host.argtypes = [P(Shape), P(IO), vp, vp, vp, sz, vp]
+    lib.moe_forward_host.restype = st
+    lib.moe_get_device_status.argtypes = [vp, vp]
+    lib.moe_get_device_status.restype = st
+    lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
+    lib.moe_set_wait_limit.restype = None
+    lib.moe_debug_timeout_probe.argtypes = [vp, sz, vp]
+    lib.moe_debug_timeout_probe.restype = st
+    lib.moe_last_launch_count.argtypes = []
+    lib.moe_last_launch_count.restype = ctypes.c_int
+    lib.moe_status_string.argtypes = [st]
+    lib.moe_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().moe_status_string(status).decode()
+
+
+def make_shape(T: int, H: int, E: int, k: int, F: int, capacity_factor: float = math.inf, dtype: str = "bf16") -> Shape:
+    return Shape(T, H, E, F, k, float(capacity_factor), DTYPES[dtype])
+
+
+def _check(status: int, where: str) -> int:
+    if status != MOE_OK:
+        raise MoEError(status, where)
+    return status
+
+
+# ---- thin wrappers, same names as the C ABI; pointers are ints, streams are cudaStream_t ints ----
+
+def moe_workspace_size(shape: Shape) -> int:
+    return load_library().moe_workspace_size(ctypes.byref(shape))
+
+
+def moe_workspace_layout(shape: Shape, ws: int) -> WsView:
+    v = WsView()
+    _check(load_library().moe_workspace_layout(ctypes.byref(shape), ws, ctypes.byref(v)), "moe_workspace_layout")
+    return v
+
+
+def moe_route(shape, io, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_route(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, stream)
+
+
+def moe_permute(shape, io, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_permute(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, stream)
+
+
+def moe_expert_ffn(shape, io, ws, ws_bytes, fuse_combine=1, stream=0) -> int:
+    return load_library().moe_expert_ffn(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, int(fuse_combine), stream)
+
+
+def moe_combine(shape, io, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_combine(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, stream)
+
+
+def moe_forward(shape, io, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_forward(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, stream)
+
+
+def moe_forward_host(shape, io, x_host, out_host, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_forward_host(ctypes.byref(shape), ctypes.byref(io), x_host, out_host, ws, ws_bytes,
+                                           stream)
+
+
+def moe_get_device_status(ws, stream=0) -> int:
+    return load_library().moe_get_device_status(ws, stream)
+
+
+def moe_set_wait_limit(cycles: int) -> None:
+    load_library().moe_set_wait_limit(int(cycles))
+
+
+def moe_debug_timeout_probe(ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_debug_timeout_probe(ws, ws_bytes, stream)
+
+
+def moe_last_launch_count() -> int:
+    return load_library().moe_last_launch_count()
+
+
+class MoEBuffers:
+    """Device buffers of one layer invocation, allocated with PyTorch (plumbing only).
+
+    ``inputs`` maps x, Wg, bg, W1, b1, W2, b2 to device tensors of the storage dtype (bf16 as
+    torch.bfloat16, f32 as torch.float32).  Outputs and the workspace are allocated here.
+    """
+
+    def __init__(self, shape: Shape, inputs: dict, device="cuda"):
+        import torch
+
+        self.shape = shape
+        T, H, E, k = shape.T, shape.H, shape.E, shape.k
+        self.inputs = inputs
+        self.out = torch.empty((T, H), dtype=torch.float32, device=device)
+        self.topk_idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.topk_w = torch.empty((T, k), dtype=torch.float32, device=device)
+        self.expert_counts = torch.empty((E,), dtype=torch.int32, device=device)
+        self.dropped = torch.empty((T, k), dtype=torch.uint8, device=device)
+        self.losses = torch.empty((2,), dtype=torch.float32, device=device)
+        self.ws_bytes = moe_workspace_size(shape)
+        if self.ws_bytes == 0:
+            raise MoEError(MOE_ERR_INVALID_ARG, "moe_workspace_size")
+        self.ws = torch.empty((self.ws_bytes,), dtype=torch.uint8, device=device)
+        self.ws[:256].zero_()  # the device error word starts cleared
+        self.io = self.make_io()
+
+    def make_io(self) -> IO:
+        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        i = self.inputs
+        return IO(p(i.get("x")), p(i.get("Wg")), p(i.get("bg")), p(i.get("W1")), p(i.get("b1")), p(i.get("W2")),
+                  p(i.get("b2")), p(self.out), p(self.topk_idx), p(self.topk_w), p(self.expert_counts),
+                  p(self.dropped), self.losses.data_ptr(), self.losses.data_ptr() + 4)
+
+    def set_input(self, name: str, tensor) -> None:
+        self.inputs[name] = tensor
+        self.io = self.make_io()
+
+    @property
+    def ws_ptr(self) -> int:
+        return self.ws.data_ptr()
+
+    def view(self) -> WsView:
+        return moe_workspace_layout(self.shape, self.ws_ptr)
+
+    @staticmethod
+    def stream() -> int:
+        import torch
+
+        return torch.cuda.current_stream().cuda_stream
+
+    def route(self):
+        return _check(moe_route(self.shape, self.io, self.ws_ptr, self.ws_bytes, self.stream()), "moe_route")
+
+    def permute(self):
+        return _check(moe_permute(self.shape, self.io, self.ws_ptr, self.ws_bytes, self.stream()), "moe_permute")
+
+    def expert_ffn(self, fuse_combine=True):
+        return _check(moe_expert_ffn(self.shape, self.io, self.ws_ptr, self.ws_bytes, int(fuse_combine), self.stream()),
+                      "moe_expert_ffn")
+
+    def combine(self):
+        return _check(moe_combine(self.shape, self.io, self.ws_ptr, self.ws_bytes, self.stream()), "moe_combine")
+
+    def forward(self):
+        return _check(moe_forward(self.shape, self.io, self.ws_ptr, self.ws_bytes, self.stream()), "moe_forward")
+
+    def forward_host(self, x_host, out_host):
+        """x_host / out_host: pinned CPU tensors (storage dtype / float32)."""
+        return _check(moe_forward_host(self.shape, self.io, x_host.data_ptr(), out_host.data_ptr(), self.ws_ptr,
+                                       self.ws_bytes, self.stream()), "moe_forward_host")
+
+    def device_status(self) -> int:
+        return moe_get_device_status(self.ws_ptr, self.stream())

@@ -1,0 +1,548 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (sm_100a: TMA + tcgen05.mma + TMEM).
+//
+// Expert FFN of the MoE layer ("MoE Training: Mixture of Experts" page, Quick Start expert
+// Linear(H, 4H) -> GELU -> Linear(4H, H); Advanced Patterns Mixtral block: gather rows by expert,
+// scale by the routing weight, index_add_ back to token order) over variable-length expert
+// segments of the permuted rows:
+//   GEMM1 (EPI_GELU):     h[r, n]   = bf16( GELU( sum_k x_perm[r,k] W1[e,k,n] + b1[e,n] ) )
+//   GEMM2 (EPI_COMBINE):  out[t, n] += w(t,s) * ( sum_k h[r,k] W2[e,k,n] + b2[e,n] ),  t,s = row r's
+//   GEMM2 (EPI_STORE_Y):  y[r, n]   = sum_k h[r,k] W2[e,k,n] + b2[e,n]
+//
+// Design (one persistent CTA per SM, 192 threads):
+//   warp 0      TMA producer: A tile [128 rows x 64 k] (K-major, 128B swizzle) and B tile
+//               [64 k x BN n] (weights are stored n-contiguous, i.e. MN-major, 128B swizzle, loaded
+//               as BN/64 boxes of 64x64) into a kStages-deep shared-memory ring.
+//   warp 1      allocates 2*BN TMEM columns (two fp32 accumulators), one elected lane issues
+//               tcgen05.mma kind::f16 (M=128, N=BN, K=16, bf16 x bf16 -> fp32) and tcgen05.commit
+//               to release smem stages and to hand a finished accumulator to the epilogue.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns per step (each thread owns one row),
+//               fused bias + GELU -> bf16 store, or bias + gate-weight scale + vector fp32 red.add
+//               into out (at most k adds per element, so k <= 2 is order independent).
+// Tiles run expert-major, then n-tile, then m-tile, so the CTAs in flight share one expert's
+// weight columns and activation rows through L2.  Rows past an expert's segment inside its last
+// m-tile are computed on whatever the buffer holds there and masked in the epilogue.
+// Every mbarrier wait is bounded: a wait that runs out sets the workspace error word, raises a
+// CTA-wide abort flag, and the CTA drains its in-flight copies / MMAs (bounded) and exits.
+// No TMA multicast is used anywhere.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // one 128-byte swizzle row of bf16
+constexpr int kThreads = 192;
+
+enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2 };
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kABytes = BM * BK * 2;
+  static constexpr int kBBytes = BK * BN * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;
+  // smem: [align pad][A stages][B stages][barriers][tmem slot, abort][offsets, tile prefix]
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kStages + 4 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kOffsOff = kMiscOff + 16;
+  static constexpr int kSmemBytes = 1024 + kOffsOff + 2 * 260 * 4;
+  // instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16 MN-major, M=128, N=BN
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                                     ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+};
+
+struct GemmArgs {
+  const int32_t* offsets;
+  int E, N, K;
+  const __nv_bfloat16* bias;
+  __nv_bfloat16* h_out;
+  float* out;
+  float* y;
+  const int32_t* row_token;
+  const int32_t* row_slot;
+  const float* topk_w;
+  int k;
+  int32_t* status;
+  long long wait_limit;
+};
+
+// ------------------------------------------------------------------ PTX wrappers ----------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait. Returns false when the CTA is aborting or the bound ran out (then it aborts).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit, volatile int* abort_flag,
+                                          int32_t* status, int code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit) {
+      *abort_flag = 1;
+      atomicCAS(status, 0, code);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot), "r"(ncols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Shared-memory matrix descriptors (tcgen05 "matrix descriptor" format, version 1 for sm_100):
+// bits 0-13 start>>4, 16-29 leading byte offset>>4, 32-45 stride byte offset>>4, 46-47 version=1,
+// 49-51 base offset (0: atoms 1024-aligned), 61-63 layout (2 = 128-byte swizzle).
+// A, K-major 128B swizzle: rows of 128 bytes, 8-row atoms 1024 B apart (SBO); LBO unused (16 B).
+__device__ __forceinline__ uint64_t desc_a_kmajor(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// B, MN-major 128B swizzle: each k row holds 64 n values (128 B); 8 k rows form a 1024 B atom
+// (SBO = 1024 between k groups); the next 64 n values sit one whole 64x64 box further (LBO).
+__device__ __forceinline__ uint64_t desc_b_mnmajor(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((BK * 128) >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// tile -> (expert, m tile inside the expert, n tile); prefix[e] = tiles of experts < e
+__device__ __forceinline__ void decode_tile(int tile, const int* prefix, const int* offs, int E, int NT, int& e,
+                                            int& m_local, int& n_idx, int& row0, int& rows) {
+  int lo = 0, hi = E;  // find the last e with prefix[e] <= tile (skips empty experts)
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= tile) lo = mid;
+    else hi = mid;
+  }
+  e = lo;
+  const int cnt = offs[e + 1] - offs[e];
+  const int mt = (cnt + BM - 1) / BM;
+  const int local = tile - prefix[e];
+  n_idx = local / mt;
+  m_local = local % mt;
+  row0 = offs[e] + m_local * BM;
+  rows = min(BM, cnt - m_local * BM);
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  int* offs = reinterpret_cast<int*>(smem + C::kOffsOff);
+  int* prefix = offs + 260;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = g.E, NT = g.N / BN, KB = g.K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  for (int i = threadIdx.x; i <= E; i += kThreads) offs[i] = g.offsets[i];
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      prefix[e] = run;
+      run += ((offs[e + 1] - offs[e] + BM - 1) / BM) * NT;
+    }
+    prefix[E] = run;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = prefix[E];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer -----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, m_local, n_idx, row0, rows;
+        decode_tile(tile, prefix, offs, E, NT, e, m_local, n_idx, row0, rows);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = sbase + stage * C::kABytes;
+          const uint32_t b_dst = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          armed[stage] = (int)phase;
+          tma_load_2d(a_dst, &tmA, kb * BK, row0, full_bar(stage));
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_3d(b_dst + j * (BK * 128), &tmB, n_idx * BN + j * 64, kb * BK, e, full_bar(stage));
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok || *abort_flag) {
+        // drain: every armed stage's copies must land before the CTA exits
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed[s] >= 0) {
+            volatile int dummy = 0;
+            mbar_wait(full_bar(s), (uint32_t)armed[s], g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer -------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+        if (!mbar_wait(tempty_bar(buf), tphase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status, kDevTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = sbase + stage * C::kABytes;
+          const uint32_t b_addr = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            mma_bf16(d_tmem, desc_a_kmajor(a_addr + kk * 32), desc_b_mnmajor(b_addr + kk * 16 * 128), C::kIdesc,
+                     (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit(empty_bar(stage));
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar(buf));
+      }
+      if ((!ok || *abort_flag) && issued) {
+        // drain: MMAs still running must finish before TMEM is released
+        mma_commit(drain_bar);
+        volatile int dummy = 0;
+        mbar_wait(drain_bar, 0, g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5) --------
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int r_in_tile = quarter * 32 + lane;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      int e, m_local, n_idx, row0, rows;
+      decode_tile(tile, prefix, offs, E, NT, e, m_local, n_idx, row0, rows);
+      const int buf = it & 1;
+      const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+      // every lane waits; the warp leaves together if any lane gave up (tcgen05.ld is warp-wide)
+      const bool got = mbar_wait(tfull_bar(buf), tphase, g.wait_limit, abort_flag, g.status, kDevTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const bool row_ok = r_in_tile < rows;
+      const int grow = row0 + r_in_tile;
+      float wgt = 0.f;
+      int tok = 0;
+      if (EPI == EPI_COMBINE && row_ok) {
+        tok = g.row_token[grow];
+        wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
+      }
+      const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
+        const int n0 = n_idx * BN + c * 32;
+        if (row_ok) {
+          float v[32];
+          const uint4* bp = reinterpret_cast<const uint4*>(brow + n0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 bb = __ldg(bp + q);
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              float2 f = __bfloat1622float2(b2[u]);
+              v[q * 8 + 2 * u] = __uint_as_float(r[q * 8 + 2 * u]) + f.x;
+              v[q * 8 + 2 * u + 1] = __uint_as_float(r[q * 8 + 2 * u + 1]) + f.y;
+            }
+          }
+          if (EPI == EPI_GELU) {
+            uint4* dst = reinterpret_cast<uint4*>(g.h_out + (size_t)grow * g.N + n0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint4 o;
+              o.x = pack_bf16(gelu_erf(v[q * 8 + 0]), gelu_erf(v[q * 8 + 1]));
+              o.y = pack_bf16(gelu_erf(v[q * 8 + 2]), gelu_erf(v[q * 8 + 3]));
+              o.z = pack_bf16(gelu_erf(v[q * 8 + 4]), gelu_erf(v[q * 8 + 5]));
+              o.w = pack_bf16(gelu_erf(v[q * 8 + 6]), gelu_erf(v[q * 8 + 7]));
+              dst[q] = o;
+            }
+          } else if (EPI == EPI_COMBINE) {
+            float* dst = g.out + (size_t)tok * g.N + n0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              red_add_v4(dst + 4 * q, wgt * v[4 * q], wgt * v[4 * q + 1], wgt * v[4 * q + 2], wgt * v[4 * q + 3]);
+          } else {
+            float4* dst = reinterpret_cast<float4*>(g.y + (size_t)grow * g.N + n0);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// One thread waits on a barrier that nothing completes; the bound must end it.
+__global__ void timeout_probe_kernel(int32_t* status, long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    mbar_wait(smem_u32(&bar), 0, limit, &abort_flag, status, kDevTimeoutProbe);
+  }
+}
+
+// ------------------------------------------------------------------ host side -------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// A operand: [rows, K] bf16 row-major; box = 64 k x 128 rows
+bool make_map_a(CUtensorMap* m, const void* base, int rows, int K) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {BK, BM};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// B operand: [E, K, N] bf16 (n contiguous); box = 64 n x 64 k x 1 expert
+bool make_map_b(CUtensorMap* m, const void* base, int E, int K, int N) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)K, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)N * 2, (cuuint64_t)K * N * 2};
+  cuuint32_t box[3] = {64, BK, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI>
+cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid, cudaStream_t st) {
+  auto kern = grouped_gemm_kernel<BN, EPI>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  kern<<<grid, kThreads, Cfg<BN>::kSmemBytes, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid,
+                      cudaStream_t st) {
+  if (N % 256 == 0) return launch_one<256, EPI>(ma, mb, g, grid, st);
+  if (N % 128 == 0) return launch_one<128, EPI>(ma, mb, g, grid, st);
+  return launch_one<64, EPI>(ma, mb, g, grid, st);
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches) {
+  CUtensorMap ma1, mb1, ma2, mb2;
+  if (!make_map_a(&ma1, a.x_perm, a.rows_cap, a.H) || !make_map_b(&mb1, a.W1, a.E, a.H, a.F) ||
+      !make_map_a(&ma2, a.h, a.rows_cap, a.F) || !make_map_b(&mb2, a.W2, a.E, a.F, a.H))
+    return cudaErrorInvalidValue;
+  const int grid = a.num_sms > 0 ? a.num_sms : 148;
+
+  GemmArgs g1{};
+  g1.offsets = a.offsets;
+  g1.E = a.E;
+  g1.N = a.F;
+  g1.K = a.H;
+  g1.bias = reinterpret_cast<const __nv_bfloat16*>(a.b1);
+  g1.h_out = reinterpret_cast<__nv_bfloat16*>(a.h);
+  g1.k = a.k;
+  g1.status = a.status;
+  g1.wait_limit = a.wait_limit;
+  cudaError_t err = launch_bn<EPI_GELU>(a.F, ma1, mb1, g1, grid, st);
+  if (err != cudaSuccess) return err;
+  ++*launches;
+
+  GemmArgs g2 = g1;
+  g2.N = a.H;
+  g2.K = a.F;
+  g2.bias = reinterpret_cast<const __nv_bfloat16*>(a.b2);
+  g2.h_out = nullptr;
+  g2.out = a.out;
+  g2.y = a.y;
+  g2.row_token = a.row_token;
+  g2.row_slot = a.row_slot;
+  g2.topk_w = a.topk_w;
+  if (a.fuse_combine)
+    err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, g2, grid, st);
+  else
+    err = launch_bn<EPI_STORE_Y>(a.H, ma2, mb2, g2, grid, st);
+  if (err != cudaSuccess) return err;
+  ++*launches;
+  return cudaSuccess;
+}
+
+cudaError_t launch_timeout_probe(int32_t* status, long long limit, cudaStream_t st) {
+  timeout_probe_kernel<<<1, 32, 0, st>>>(status, limit);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,396 @@
+// Host side of the C ABI declared in include/moe.h: argument validation, workspace layout and
+// the launch sequence of each stage on the caller's stream.  No allocation, no synchronisation
+// (except moe_get_device_status).
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "moe_internal.cuh"
+
+namespace moe {
+
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+WsLayout ws_layout(const moe_shape_t& s) {
+  WsLayout L{};
+  const size_t T = (size_t)s.T, E = (size_t)s.E, k = (size_t)s.k;
+  const size_t es = s.dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  L.nblk = (int)((T + kChunk - 1) / kChunk);
+  const size_t nblk = (size_t)L.nblk;
+  const size_t rows = T * k;
+  size_t o = 0;
+  L.status = o;
+  o = align256(o + 16);
+  L.offsets = o;
+  o = align256(o + (E + 1) * 4);
+  L.cnt_pre = o;
+  o = align256(o + E * 4);
+  L.chunk_hist = o;
+  o = align256(o + k * nblk * E * 4);
+  L.chunk_base = o;
+  o = align256(o + k * nblk * E * 4);
+  L.loss_part = o;
+  o = align256(o + nblk * (E + 1) * 4);
+  L.row_of = o;
+  o = align256(o + rows * 4);
+  L.row_token = o;
+  o = align256(o + rows * 4);
+  L.row_slot = o;
+  o = align256(o + rows * 4);
+  L.x_perm = o;
+  o = align256(o + rows * (size_t)s.H * es);
+  L.h = o;
+  o = align256(o + rows * (size_t)s.F * es);
+  L.y = o;
+  o = align256(o + rows * (size_t)s.H * 4);
+  L.total = o;
+  return L;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+namespace {
+
+thread_local int g_launches = 0;
+long long g_wait_limit = 2000000000LL;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t check_shape(const moe_shape_t* s) {
+  if (s == nullptr) return MOE_ERR_INVALID_ARG;
+  if (s->T < 0 || s->H <= 0 || s->E <= 0 || s->F <= 0 || s->k <= 0) return MOE_ERR_INVALID_ARG;
+  if (s->k > s->E || s->k > 8 || s->E > 256) return MOE_ERR_INVALID_ARG;
+  if (!(s->capacity_factor > 0.0)) return MOE_ERR_INVALID_ARG;  // also rejects NaN
+  if (s->dtype != MOE_DTYPE_F32 && s->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if (s->dtype == MOE_DTYPE_BF16 && (s->H % 64 != 0 || s->F % 64 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (s->dtype == MOE_DTYPE_F32 && (s->H % 4 != 0 || s->F % 4 != 0)) return MOE_ERR_UNSUPPORTED;
+  const long long rows = (long long)s->T * s->k;
+  const long long widest = s->H > s->F ? s->H : s->F;
+  if (rows * widest >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+long long capacity_of(const moe_shape_t* s) {
+  if (isinf(s->capacity_factor)) return -1;
+  double c = ceil(s->capacity_factor * (double)s->T * (double)s->k / (double)s->E);
+  if (c >= (double)((long long)s->T * s->k)) return -1;  // never binding
+  return (long long)c;
+}
+
+moe_status_t check_ws(const moe_shape_t* s, const void* ws, size_t ws_bytes) {
+  if (ws == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(*s).total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------- stage bodies (validated) -------
+moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, bool emit_hist) {
+  const WsLayout L = ws_layout(*s);
+  if (s->T == 0) {
+    ++g_launches;
+    return cuda_status(launch_zero_outputs(nullptr, 0, io->aux_loss, io->z_loss, st));
+  }
+  RouterArgs r{};
+  r.x = io->x;
+  r.Wg = io->Wg;
+  r.bg = io->bg;
+  r.T = s->T;
+  r.H = s->H;
+  r.E = s->E;
+  r.k = s->k;
+  r.topk_idx = io->topk_idx;
+  r.topk_w = io->topk_w;
+  r.loss_part = at<float>(ws, L.loss_part);
+  r.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+  (void)emit_hist;
+  cudaError_t err = launch_router(r, s->dtype, st);
+  ++g_launches;
+  if (err != cudaSuccess) return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int do_losses, int do_dispatch) {
+  const WsLayout L = ws_layout(*s);
+  ReduceArgs a{};
+  a.T = s->T;
+  a.E = s->E;
+  a.k = s->k;
+  a.nblk = L.nblk;
+  a.cap = capacity_of(s);
+  a.loss_part = at<float>(ws, L.loss_part);
+  a.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+  a.chunk_base = at<int32_t>(ws, L.chunk_base);
+  a.cnt_pre = at<int32_t>(ws, L.cnt_pre);
+  a.expert_counts = io->expert_counts;
+  a.offsets = at<int32_t>(ws, L.offsets);
+  a.aux_loss = io->aux_loss;
+  a.z_loss = io->z_loss;
+  a.do_losses = do_losses;
+  a.do_dispatch = do_dispatch;
+  return a;
+}
+
+moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(*s);
+  ScatterArgs a{};
+  a.x = io->x;
+  a.T = s->T;
+  a.H = s->H;
+  a.E = s->E;
+  a.k = s->k;
+  a.nblk = L.nblk;
+  a.esize = s->dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  a.cap = capacity_of(s);
+  a.topk_idx = io->topk_idx;
+  a.chunk_base = at<int32_t>(ws, L.chunk_base);
+  a.offsets = at<int32_t>(ws, L.offsets);
+  a.dropped = io->dropped;
+  a.row_of = at<int32_t>(ws, L.row_of);
+  a.row_token = at<int32_t>(ws, L.row_token);
+  a.row_slot = at<int32_t>(ws, L.row_slot);
+  a.x_perm = at<void>(ws, L.x_perm);
+  a.out = io->out;
+  ++g_launches;
+  return cuda_status(launch_scatter(a, st));
+}
+
+moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse, cudaStream_t st) {
+  const WsLayout L = ws_layout(*s);
+  FfnArgs a{};
+  a.T = s->T;
+  a.H = s->H;
+  a.E = s->E;
+  a.F = s->F;
+  a.k = s->k;
+  a.rows_cap = s->T * s->k;
+  a.offsets = at<int32_t>(ws, L.offsets);
+  a.row_token = at<int32_t>(ws, L.row_token);
+  a.row_slot = at<int32_t>(ws, L.row_slot);
+  a.topk_w = io->topk_w;
+  a.x_perm = at<void>(ws, L.x_perm);
+  a.W1 = io->W1;
+  a.b1 = io->b1;
+  a.W2 = io->W2;
+  a.b2 = io->b2;
+  a.h = at<void>(ws, L.h);
+  a.y = at<float>(ws, L.y);
+  a.out = io->out;
+  a.fuse_combine = fuse;
+  a.status = at<int32_t>(ws, L.status);
+  a.wait_limit = g_wait_limit;
+  a.num_sms = num_sms();
+  cudaError_t err = s->dtype == MOE_DTYPE_BF16 ? launch_ffn_bf16_sm100(a, st, &g_launches) : launch_ffn_f32(a, st, &g_launches);
+  return cuda_status(err);
+}
+
+bool null_any(std::initializer_list<const void*> ps) {
+  for (const void* p : ps)
+    if (p == nullptr) return true;
+  return false;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_shape_t* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return ws_layout(*shape).total;
+}
+
+moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, moe_ws_view_t* view) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (ws == nullptr || view == nullptr) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*shape);
+  view->status = at<int32_t>(ws, L.status);
+  view->offsets = at<int32_t>(ws, L.offsets);
+  view->cnt_pre = at<int32_t>(ws, L.cnt_pre);
+  view->row_of = at<int32_t>(ws, L.row_of);
+  view->row_token = at<int32_t>(ws, L.row_token);
+  view->row_slot = at<int32_t>(ws, L.row_slot);
+  view->x_perm = at<void>(ws, L.x_perm);
+  view->h = at<void>(ws, L.h);
+  view->y = at<float>(ws, L.y);
+  view->bytes = L.total;
+  return MOE_OK;
+}
+
+moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  g_launches = 0;
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (io == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (null_any({io->aux_loss, io->z_loss})) return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) return do_route(shape, io, ws, stream, true);
+  if (null_any({io->x, io->Wg, io->bg, io->topk_idx, io->topk_w})) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(io->x) || !aligned16(io->Wg)) return MOE_ERR_INVALID_ARG;
+  if ((st = do_route(shape, io, ws, stream, true)) != MOE_OK) return st;
+  ++g_launches;
+  return cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 0), stream));
+}
+
+moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  g_launches = 0;
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (io == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (null_any({io->expert_counts})) return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) {
+    ++g_launches;
+    return cuda_status(launch_zero_outputs(io->expert_counts, shape->E, nullptr, nullptr, stream));
+  }
+  if (null_any({io->x, io->topk_idx, io->dropped, io->out})) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(io->x) || !aligned16(io->out)) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*shape);
+  ++g_launches;
+  if ((st = cuda_status(launch_hist(io->topk_idx, shape->T, shape->E, shape->k, L.nblk, at<int32_t>(ws, L.chunk_hist),
+                                    stream))) != MOE_OK)
+    return st;
+  ++g_launches;
+  if ((st = cuda_status(launch_reduce(reduce_args(shape, io, ws, 0, 1), stream))) != MOE_OK) return st;
+  return do_scatter(shape, io, ws, stream);
+}
+
+moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, int fuse_combine,
+                            cudaStream_t stream) {
+  g_launches = 0;
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (io == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  if (null_any({io->W1, io->b1, io->W2, io->b2, io->topk_w})) return MOE_ERR_INVALID_ARG;
+  if (fuse_combine && io->out == nullptr) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(io->W1) || !aligned16(io->W2) || !aligned16(io->b1) || !aligned16(io->b2) ||
+      (fuse_combine && !aligned16(io->out)))
+    return MOE_ERR_INVALID_ARG;
+  return do_ffn(shape, io, ws, fuse_combine ? 1 : 0, stream);
+}
+
+moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  g_launches = 0;
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (io == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (shape->T == 0) return MOE_OK;
+  if (null_any({io->out, io->topk_w})) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(io->out)) return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*shape);
+  ++g_launches;
+  return cuda_status(launch_combine(at<float>(ws, L.y), at<int32_t>(ws, L.row_of), io->topk_w, shape->T, shape->H,
+                                    shape->k, io->out, stream));
+}
+
+moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  g_launches = 0;
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (io == nullptr) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (null_any({io->aux_loss, io->z_loss, io->expert_counts})) return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) {
+    ++g_launches;
+    return cuda_status(launch_zero_outputs(io->expert_counts, shape->E, io->aux_loss, io->z_loss, stream));
+  }
+  if (null_any({io->x, io->Wg, io->bg, io->W1, io->b1, io->W2, io->b2, io->out, io->topk_idx, io->topk_w,
+                io->dropped}))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(io->x) || !aligned16(io->Wg) || !aligned16(io->W1) || !aligned16(io->W2) || !aligned16(io->out) ||
+      !aligned16(io->b1) || !aligned16(io->b2))
+    return MOE_ERR_INVALID_ARG;
+  int n = 0;
+  // router emits the chunk histograms itself, so one reduction serves losses and dispatch
+  if ((st = do_route(shape, io, ws, stream, true)) != MOE_OK) return st;
+  n += g_launches;
+  ++n;
+  if ((st = cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 1), stream))) != MOE_OK) return st;
+  g_launches = 0;
+  if ((st = do_scatter(shape, io, ws, stream)) != MOE_OK) return st;
+  n += g_launches;
+  g_launches = 0;
+  st = do_ffn(shape, io, ws, 1, stream);
+  g_launches += n;
+  return st;
+}
+
+moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_io_t* io, const void* x_host, float* out_host,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (io == nullptr || x_host == nullptr || out_host == nullptr || io->x == nullptr || io->out == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  const size_t es = shape->dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  const size_t n = (size_t)shape->T * shape->H;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
+  if (n > 0 && cudaMemcpyAsync(const_cast<void*>(io->x), x_host, n * es, cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  st = moe_forward(shape, io, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  if (n > 0 && cudaMemcpyAsync(out_host, io->out, n * 4, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status_t moe_get_device_status(void* ws, cudaStream_t stream) {
+  if (ws == nullptr) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t word = 0;
+  if (cudaMemcpy(&word, ws, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (word != 0) {
+    const int32_t zero = 0;
+    if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_ERR_TIMEOUT;
+  }
+  return MOE_OK;
+}
+
+void moe_set_wait_limit(long long cycles) { g_wait_limit = cycles > 0 ? cycles : 2000000000LL; }
+
+moe_status_t moe_debug_timeout_probe(void* ws, size_t ws_bytes, cudaStream_t stream) {
+  g_launches = 0;
+  if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  ++g_launches;
+  return cuda_status(launch_timeout_probe(reinterpret_cast<int32_t*>(ws), g_wait_limit, stream));
+}
+
+int moe_last_launch_count(void) { return g_launches; }
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+// Internal declarations shared by the kernels and the host C-ABI of the MoE forward library.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr int kChunk = 32;          // tokens per router chunk; also one warp in the permute ranks
+constexpr int kRouterThreads = 256; // router block
+constexpr int kRouterHC = 32;       // H columns per router pipeline stage
+constexpr int kRouterStages = 4;
+
+// Device error codes written to the workspace status word (first writer wins).
+enum DevError : int {
+  kDevOk = 0,
+  kDevTimeoutProducer = 0x101,
+  kDevTimeoutMma = 0x102,
+  kDevTimeoutEpilogue = 0x103,
+  kDevTimeoutProbe = 0x104,
+  kDevTimeoutDrain = 0x105,
+};
+
+// Workspace sections (byte offsets from the workspace base, 256-aligned).
+struct WsLayout {
+  size_t status, offsets, cnt_pre, chunk_hist, chunk_base, loss_part, row_of, row_token, row_slot, x_perm, h, y,
+      total;
+  int nblk;  // router chunks = ceil(T / kChunk)
+};
+
+WsLayout ws_layout(const moe_shape_t& s);
+
+struct RouterArgs {
+  const void* x;
+  const void* Wg;
+  const void* bg;
+  int T, H, E, k;
+  int32_t* topk_idx;
+  float* topk_w;
+  float* loss_part;    // [nblk][E+1]: sum_t p[t,e] (E values) then sum_t lse_t^2
+  int32_t* chunk_hist; // [k][nblk][E] or null
+};
+
+struct ReduceArgs {
+  int T, E, k, nblk;
+  long long cap;  // < 0: unlimited
+  const float* loss_part;
+  int32_t* chunk_hist;  // [k][nblk][E]
+  int32_t* chunk_base;  // [k][nblk][E] out: first rank of each chunk's assignments in its expert
+  int32_t* cnt_pre;     // [E]
+  int32_t* expert_counts;
+  int32_t* offsets;     // [E+1]
+  float* aux_loss;
+  float* z_loss;
+  int do_losses, do_dispatch;
+};
+
+struct ScatterArgs {
+  const void* x;
+  int T, H, E, k, nblk, esize;
+  long long cap;
+  const int32_t* topk_idx;
+  const int32_t* chunk_base;
+  const int32_t* offsets;
+  uint8_t* dropped;
+  int32_t* row_of;
+  int32_t* row_token;
+  int32_t* row_slot;
+  void* x_perm;
+  float* out;  // cleared for this chunk's tokens (slot 0 blocks); may be null
+};
+
+struct FfnArgs {
+  int T, H, E, F, k;
+  int rows_cap;  // T*k: height of x_perm / h / y
+  const int32_t* offsets;
+  const int32_t* row_token;
+  const int32_t* row_slot;
+  const float* topk_w;
+  const void* x_perm;
+  const void* W1;
+  const void* b1;
+  const void* W2;
+  const void* b2;
+  void* h;
+  float* y;
+  float* out;
+  int fuse_combine;
+  int32_t* status;
+  long long wait_limit;
+  int num_sms;
+};
+
+cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st);
+cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, cudaStream_t st);
+cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);
+cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
+cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);
+cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t st, int* launches);
+cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches);
+cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int T, int H, int k, float* out,
+                           cudaStream_t st);
+cudaError_t launch_timeout_probe(int32_t* status, long long limit, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,92 @@
+"""Helpers shared by the GPU parity tests: upload seeded inputs, run the CUDA stages through the C ABI,
+and the tolerance rules used against the oracle.
+
+Tolerances (written here once, used by every parity test):
+  * integer outputs (top-k indices, counts, drop flags, row maps): bit-exact, except tokens whose
+    oracle logit margin (smallest gap among the top-(k+1) logits) is below NEAR_TIE; those are
+    excluded from the index comparison and counted;
+  * fp32 path: normwise relative error max|d| / max|ref| <= 1e-4 per output tensor;
+  * bf16-input / fp32-accumulate path: max|d| <= 2e-2 * RMS(ref) per output tensor;
+  * topk_w (fp32 from fp32 logits): max relative error 1e-4; losses: relative error 1e-3.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+import synth
+
+NEAR_TIE = 1e-4
+TOL_F32 = 1e-4
+TOL_BF16_RMS = 2e-2
+TOL_W = 1e-4
+TOL_LOSS = 1e-3
+
+
+def torch_dtype(dtype: str):
+    import torch
+
+    return torch.bfloat16 if dtype == "bf16" else torch.float32
+
+
+def to_device(arr: np.ndarray, dtype: str, device="cuda"):
+    import torch
+
+    if dtype == "bf16":
+        t = torch.from_numpy(np.ascontiguousarray(arr).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(arr, dtype=np.float32))
+    return t.to(device)
+
+
+def upload(inp: synth.LayerInputs, device="cuda") -> dict:
+    return {name: to_device(a, inp.cfg.dtype, device) for name, a in inp.arrays().items()}
+
+
+def shape_of(cfg: synth.LayerConfig):
+    import sparse_mixture_experts_23_b200 as moe
+
+    return moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype)
+
+
+def from_device_bits(t, dtype: str) -> np.ndarray:
+    """Storage-dtype tensor -> numpy in the oracle's input convention (bf16 as uint16 bits)."""
+    import torch
+
+    if dtype == "bf16":
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def normwise_rel(a: np.ndarray, ref: np.ndarray) -> float:
+    den = float(np.max(np.abs(ref))) if ref.size else 0.0
+    return float(np.max(np.abs(a - ref))) / den if den > 0 else float(np.max(np.abs(a - ref), initial=0.0))
+
+
+def rms_rel(a: np.ndarray, ref: np.ndarray) -> float:
+    rms = math.sqrt(float(np.mean(np.square(ref)))) if ref.size else 0.0
+    d = float(np.max(np.abs(a - ref), initial=0.0))
+    return d / rms if rms > 0 else d
+
+
+def out_error(a: np.ndarray, ref: np.ndarray, dtype: str, rows=None) -> tuple[float, float]:
+    """(error, tolerance) under the rule for the storage dtype.
+
+    ``rows`` (boolean mask) restricts both the error and the reference scale to the output rows
+    that received at least one expert output: rows whose every slot was dropped are zero by
+    definition, are checked for exact zeros separately, and would otherwise shrink RMS(ref)."""
+    if rows is not None:
+        a, ref = a[rows], ref[rows]
+    if dtype == "f32":
+        return normwise_rel(a, ref), TOL_F32
+    return rms_rel(a, ref), TOL_BF16_RMS
+
+
+def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
+    if T <= n:
+        return np.arange(T, dtype=np.int32)
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, T // 2, T - 2, T - 1]
+    rest = rng.choice(np.arange(2, T - 2), size=n - len(fixed), replace=False)
+    return np.unique(np.concatenate([fixed, rest])).astype(np.int32)

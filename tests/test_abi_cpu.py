@@ -1,0 +1,149 @@
+"""The C-ABI library loads, exports every symbol its header declares, and validates arguments on the
+host before touching the GPU (these calls return before any CUDA work, so they run without a GPU)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_23_b200 as moe
+from sparse_mixture_experts_23_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.load_library()
+
+
+def header_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = header_symbols()
+    for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward", "moe_workspace_size"):
+        assert name in syms
+    assert sorted(moe.ENTRY_POINTS) == syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_no_torch_types_in_signatures():
+    text = open(HEADER).read()
+    assert "torch" not in text.lower().replace("pytorch", "") and "at::" not in text and "Tensor" not in text
+
+
+def _shape(**kw):
+    d = dict(T=256, H=64, E=4, k=2, F=256, capacity_factor=math.inf, dtype="f32")
+    d.update(kw)
+    return moe.make_shape(d["T"], d["H"], d["E"], d["k"], d["F"], d["capacity_factor"], d["dtype"])
+
+
+FAKE = 1 << 20  # a 256-aligned non-null "device" address; never dereferenced by these calls
+
+
+def _io(**over):
+    io = moe.IO(*([FAKE] * 14))
+    for k, v in over.items():
+        setattr(io, k, v)
+    return io
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(T=-1), moe.MOE_ERR_INVALID_ARG),
+    (dict(H=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(E=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=0), moe.MOE_ERR_INVALID_ARG),
+    (dict(k=5), moe.MOE_ERR_INVALID_ARG),        # k > E
+    (dict(E=300, k=2), moe.MOE_ERR_INVALID_ARG),  # E > 256
+    (dict(E=16, k=9), moe.MOE_ERR_INVALID_ARG),   # k > 8
+    (dict(capacity_factor=0.0), moe.MOE_ERR_INVALID_ARG),
+    (dict(capacity_factor=-1.0), moe.MOE_ERR_INVALID_ARG),
+    (dict(capacity_factor=float("nan")), moe.MOE_ERR_INVALID_ARG),
+    (dict(dtype="bf16", H=96), moe.MOE_ERR_UNSUPPORTED),
+    (dict(dtype="bf16", F=100), moe.MOE_ERR_UNSUPPORTED),
+    (dict(H=66), moe.MOE_ERR_UNSUPPORTED),
+])
+def test_shape_validation(lib, bad, code):
+    s = _shape(**bad)
+    assert moe.moe_workspace_size(s) == 0
+    for fn in (moe.moe_route, moe.moe_permute, moe.moe_combine, moe.moe_forward):
+        assert fn(s, _io(), FAKE, 1 << 40) == code
+    assert moe.moe_expert_ffn(s, _io(), FAKE, 1 << 40, 1) == code
+
+
+def test_bad_dtype_enum(lib):
+    s = _shape()
+    s.dtype = 7
+    assert moe.moe_forward(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_workspace_errors(lib):
+    s = _shape()
+    n = moe.moe_workspace_size(s)
+    assert n > 0 and n % 256 == 0
+    assert moe.moe_forward(s, _io(), FAKE, n - 1) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_forward(s, _io(), None, n) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_forward(s, _io(), FAKE + 16, n) == moe.MOE_ERR_INVALID_ARG  # not 256-aligned
+
+
+@pytest.mark.parametrize("field", ["x", "Wg", "bg", "W1", "b1", "W2", "b2", "out", "topk_idx", "topk_w",
+                                   "expert_counts", "dropped", "aux_loss", "z_loss"])
+def test_null_pointers_rejected(lib, field):
+    s = _shape()
+    n = moe.moe_workspace_size(s)
+    assert moe.moe_forward(s, _io(**{field: None}), FAKE, n) == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("field", ["x", "Wg", "W1", "W2", "out"])
+def test_misaligned_pointers_rejected(lib, field):
+    s = _shape()
+    n = moe.moe_workspace_size(s)
+    assert moe.moe_forward(s, _io(**{field: FAKE + 4}), FAKE, n) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_null_shape_and_io(lib):
+    s = _shape()
+    L = moe.load_library()
+    assert L.moe_forward(None, ctypes.byref(_io()), FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_forward(ctypes.byref(s), None, FAKE, 1 << 30, None) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_size(None) == 0
+
+
+def test_workspace_layout_is_pure_and_ordered(lib):
+    s = _shape(T=100, H=128, E=8, k=2, F=512, dtype="bf16")
+    n = moe.moe_workspace_size(s)
+    v = moe.moe_workspace_layout(s, FAKE)
+    assert v.bytes == n
+    ptrs = [v.status, v.offsets, v.cnt_pre, v.row_of, v.row_token, v.row_slot, v.x_perm, v.h, v.y]
+    assert ptrs == sorted(ptrs) and all(p % 256 == 0 for p in ptrs)
+    assert v.status == FAKE
+    rows = 100 * 2
+    assert v.h - v.x_perm >= rows * 128 * 2 and v.y - v.h >= rows * 512 * 2
+    assert FAKE + n - v.y >= rows * 128 * 4
+
+
+def test_status_strings(lib):
+    assert moe.status_string(moe.MOE_OK) == "ok"
+    assert "workspace" in moe.status_string(moe.MOE_ERR_WORKSPACE)
+    assert "timed out" in moe.status_string(moe.MOE_ERR_TIMEOUT)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    import sparse_mixture_experts_23_b200 as m
+    saved = m._lib
+    try:
+        m._lib = None
+        with pytest.raises(RuntimeError, match="not built"):
+            m.load_library(str(tmp_path / "nope.so"))
+    finally:
+        m._lib = saved

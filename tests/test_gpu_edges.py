@@ -1,0 +1,226 @@
+"""Edge cases of the CUDA path, each checked against the oracle: empty batch, ragged token counts,
+odd expert counts, every N-tile width of the tensor-core kernel, empty experts, heavy capacity drops
+(tokens with every slot dropped), maximum E and k, the unfused combine, the host-buffer entry point,
+run-to-run determinism and the bounded device wait."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from moe_testlib import NEAR_TIE, TOL_LOSS, out_error, shape_of, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def _lib():
+    import sparse_mixture_experts_23_b200 as moe
+    from sparse_mixture_experts_23_b200 import build as moe_build
+
+    moe_build.build()
+    return moe
+
+
+def _cfg(name, T, H, E, k, F, CF, dtype, seed, **kw):
+    return synth.LayerConfig(name, T=T, H=H, E=E, k=k, F=F, CF=CF, dtype=dtype, seed=seed, **kw)
+
+
+def _run_forward(cfg, inp=None, bg_override=None):
+    import torch
+
+    moe = _lib()
+    inp = inp or synth.make_inputs(cfg)
+    if bg_override is not None:
+        inp.bg = synth.to_storage(bg_override, cfg.dtype)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf.forward()
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+    r = dict(inp=inp, buf=buf, out=buf.out.cpu().numpy(), topk_idx=buf.topk_idx.cpu().numpy(),
+             topk_w=buf.topk_w.cpu().numpy(), dropped=buf.dropped.cpu().numpy(),
+             counts=buf.expert_counts.cpu().numpy(), losses=buf.losses.cpu().numpy())
+    return r
+
+
+def _check_against_oracle(cfg, r):
+    inp = r["inp"]
+    ref = oracle.route(inp.x, inp.Wg, inp.bg, cfg.k, cfg.dtype)
+    ok = ref.margin >= NEAR_TIE
+    assert (r["topk_idx"][ok] == ref.topk_idx[ok]).all()
+    d = oracle.dispatch(r["topk_idx"], cfg.E, cfg.CF)
+    assert (r["dropped"] == d.dropped).all()
+    assert (r["counts"] == d.expert_counts).all()
+    aux, z = oracle.losses(ref.p, ref.lse, r["topk_idx"])
+    assert abs(r["losses"][0] - aux) <= TOL_LOSS * abs(aux)
+    assert abs(r["losses"][1] - z) <= TOL_LOSS * abs(z)
+    toks = np.arange(cfg.T, dtype=np.int32)
+    want = oracle.forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, r["topk_idx"],
+                                 r["topk_w"].astype(np.float64), r["dropped"], toks, cfg.dtype)
+    live = ~r["dropped"].astype(bool).all(axis=1)
+    err, tol = out_error(r["out"].astype(np.float64), want, cfg.dtype, rows=live)
+    assert err <= tol, (err, tol)
+    assert (r["out"][~live] == 0).all()
+    return d
+
+
+@pytest.mark.parametrize("cfg", [
+    # ragged T (not a multiple of 32), odd E, k=3, F=192 -> 64-wide N tiles, H=128 -> 128-wide N tiles
+    _cfg("ragged_bf16", 100, 128, 6, 3, 192, 1.0, "bf16", 21),
+    # fp32 path with small odd sizes
+    _cfg("ragged_f32", 77, 20, 5, 2, 12, math.inf, "f32", 22),
+    # maximum E and k
+    _cfg("maxE_bf16", 64, 64, 256, 8, 64, math.inf, "bf16", 23),
+    # k = 1 Switch routing with drops, 256-wide N tiles
+    _cfg("switch_small", 300, 256, 16, 1, 512, 1.25, "bf16", 24),
+    # one token
+    _cfg("one_token", 1, 64, 4, 2, 64, math.inf, "bf16", 25),
+    # segments longer than one 128-row tile and a ragged tail in several experts
+    _cfg("long_segments", 1000, 128, 3, 2, 256, math.inf, "bf16", 26),
+], ids=lambda c: c.name)
+def test_small_shapes_end_to_end(cfg):
+    r = _run_forward(cfg)
+    _check_against_oracle(cfg, r)
+
+
+def test_empty_experts():
+    cfg = _cfg("empty_experts", 200, 128, 8, 2, 128, math.inf, "bf16", 31)
+    bg = np.zeros(8)
+    bg[4:] = -30.0  # experts 4..7 are never chosen
+    r = _run_forward(cfg, bg_override=bg)
+    d = _check_against_oracle(cfg, r)
+    assert (d.expert_counts[4:] == 0).all()
+
+
+def test_heavy_drops_and_all_dropped_tokens():
+    cfg = _cfg("drops", 256, 64, 4, 2, 128, 0.125, "bf16", 32)  # cap = ceil(0.125*256*2/4) = 16
+    bg = np.array([3.0, 2.5, -5.0, -5.0])  # everyone wants experts 0 and 1
+    r = _run_forward(cfg, bg_override=bg)
+    d = _check_against_oracle(cfg, r)
+    assert d.cap == 16
+    all_dropped = r["dropped"].all(axis=1)
+    assert all_dropped.sum() > 100
+    assert (r["out"][all_dropped] == 0).all()
+
+
+def test_empty_batch():
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("empty", 0, 64, 4, 2, 64, math.inf, "bf16", 33)
+    dev = {n: torch.zeros(1, dtype=torch.bfloat16, device="cuda") for n in ("x", "Wg", "bg", "W1", "b1", "W2", "b2")}
+    buf = moe.MoEBuffers(shape_of(cfg), dev)
+    buf.expert_counts.fill_(7)
+    buf.losses.fill_(5.0)
+    buf.forward()
+    torch.cuda.synchronize()
+    assert (buf.expert_counts.cpu().numpy() == 0).all()
+    assert (buf.losses.cpu().numpy() == 0).all()
+    for fn in (buf.route, buf.permute, buf.combine):
+        fn()
+    buf.expert_ffn(True)
+    torch.cuda.synchronize()
+
+
+def test_unfused_combine_matches_fused():
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("unfused", 333, 256, 8, 2, 512, 1.25, "bf16", 34)
+    inp = synth.make_inputs(cfg)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf.forward()
+    torch.cuda.synchronize()
+    fused = buf.out.cpu().numpy().copy()
+    buf.out.fill_(float("nan"))
+    buf.route()
+    buf.permute()
+    buf.expert_ffn(fuse_combine=False)
+    buf.out.fill_(float("nan"))  # combine must overwrite every element
+    buf.combine()
+    torch.cuda.synchronize()
+    unfused = buf.out.cpu().numpy()
+    assert np.isfinite(unfused).all()
+    np.testing.assert_allclose(unfused, fused, rtol=1e-5, atol=1e-6)
+    toks = np.arange(cfg.T, dtype=np.int32)
+    want = oracle.forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, buf.topk_idx.cpu().numpy(),
+                                 buf.topk_w.cpu().numpy().astype(np.float64), buf.dropped.cpu().numpy(), toks,
+                                 cfg.dtype)
+    err, tol = out_error(unfused.astype(np.float64), want, cfg.dtype)
+    assert err <= tol
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_deterministic_bitwise(dtype):
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("det", 512, 128, 8, 2, 256, math.inf, dtype, 35)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(synth.make_inputs(cfg)))
+    outs = []
+    for _ in range(3):
+        buf.forward()
+        torch.cuda.synchronize()
+        outs.append((buf.out.cpu().numpy().copy(), buf.losses.cpu().numpy().copy()))
+    for o, l in outs[1:]:
+        assert np.array_equal(o, outs[0][0]) and np.array_equal(l, outs[0][1])
+
+
+def test_forward_host_buffers():
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("host", 128, 128, 4, 2, 256, math.inf, "bf16", 36)
+    inp = synth.make_inputs(cfg)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf.forward()
+    torch.cuda.synchronize()
+    ref = buf.out.cpu().numpy().copy()
+    x2 = synth.x_batch(cfg, 1)
+    x_host = torch.from_numpy(x2.view(np.int16)).view(torch.bfloat16).pin_memory()
+    out_host = torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
+    buf.inputs["x"].zero_()
+    buf.forward_host(x_host, out_host)
+    torch.cuda.synchronize()
+    inp2 = synth.make_inputs(cfg)
+    inp2.x = x2
+    r = oracle.forward(inp2.x, inp2.Wg, inp2.bg, inp2.W1, inp2.b1, inp2.W2, inp2.b2, cfg.k, cfg.CF, cfg.dtype)
+    err, tol = out_error(out_host.numpy().astype(np.float64), r.out, cfg.dtype)
+    assert err <= tol
+    assert not np.array_equal(out_host.numpy(), ref)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    import torch
+
+    moe = _lib()
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    moe.moe_set_wait_limit(2_000_000)  # ~1 ms
+    try:
+        assert moe.moe_debug_timeout_probe(ws.data_ptr(), 256, stream) == moe.MOE_OK
+        assert moe.moe_get_device_status(ws.data_ptr(), stream) == moe.MOE_ERR_TIMEOUT
+        assert moe.moe_get_device_status(ws.data_ptr(), stream) == moe.MOE_OK  # cleared
+    finally:
+        moe.moe_set_wait_limit(0)
+    # the context is still usable
+    cfg = _cfg("after_timeout", 64, 64, 4, 2, 64, math.inf, "bf16", 37)
+    r = _run_forward(cfg)
+    _check_against_oracle(cfg, r)
+
+
+def test_stream_ordering_on_side_stream():
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("side", 256, 128, 8, 2, 256, math.inf, "bf16", 38)
+    inp = synth.make_inputs(cfg)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        buf.forward()
+    s.synchronize()
+    r = dict(inp=inp, out=buf.out.cpu().numpy(), topk_idx=buf.topk_idx.cpu().numpy(),
+             topk_w=buf.topk_w.cpu().numpy(), dropped=buf.dropped.cpu().numpy(),
+             counts=buf.expert_counts.cpu().numpy(), losses=buf.losses.cpu().numpy())
+    _check_against_oracle(cfg, r)
