@@ -63,7 +63,7 @@ def load_peaks() -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms while running."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -76,7 +76,7 @@ class ClockSampler:
         self.thread = None
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.gpu_id:
             cmd.insert(1, f"--id={self.gpu_id}")
         try:
@@ -129,6 +129,31 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def replica_inputs(cfg: synth.LayerConfig, rank: int, with_weights: bool = True) -> synth.LayerInputs:
+    """Inputs of one data-parallel replica: the shared layer weights and this rank's own batch."""
+    inp = synth.make_inputs(cfg, with_weights=with_weights)
+    if rank > 0:
+        inp.x = synth.x_batch(cfg, rank)
+    return inp
+
+
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """Slowest rank's value (timings are reported as the max over ranks)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(world: int, tokens_per_rank: int, steps: int, ms_total_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (ms_total_max / 1000.0)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -221,9 +246,7 @@ def run_ours_impl(args, cfg):
         moe_build.build()
     moe.load_library()
 
-    inp = synth.make_inputs(cfg)
-    if rank > 0:  # each replica routes its own batch through the same layer weights
-        inp.x = synth.x_batch(cfg, rank)
+    inp = replica_inputs(cfg, rank)
     dev = {n: _upload(a, cfg.dtype) for n, a in inp.arrays().items()}
     shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype)
     buf = moe.MoEBuffers(shape, dev)
@@ -242,13 +265,6 @@ def run_ours_impl(args, cfg):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         buf.forward()
     if rank == 0:
@@ -262,13 +278,14 @@ def run_ours_impl(args, cfg):
         buf.forward()
     ev1.record(stream)
     sync_all()
+    clocks = sampler.stop() if rank == 0 else None
     launches_per_step = moe.moe_last_launch_count()
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, "cuda")
     ms_step = ms_total / args.steps
-    value = world * cfg.T * args.steps / (ms_total / 1000.0)
+    value = aggregate_rate(world, cfg.T, args.steps, ms_total)
 
     # ---------------- per-kernel timing (same stream, CUDA events, inputs > L2) ---------------
-    reps = max(args.steps, 20)
+    reps = min(max(args.steps, 20), 200)
 
     def time_calls(fn) -> float:
         for _ in range(2):
@@ -309,10 +326,9 @@ def run_ours_impl(args, cfg):
         buf.forward_host(x_host, out_host)
     e1.record(stream)
     sync_all()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * cfg.T * args.steps / (ms_e2e / 1000.0)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+    e2e_value = aggregate_rate(world, cfg.T, args.steps, ms_e2e)
 
-    clocks = sampler.stop() if rank == 0 else None
     if rank != 0:
         if world > 1:
             dist.barrier()
@@ -373,7 +389,7 @@ def run_ours_impl(args, cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="mixtral", choices=list(synth.CONFIGS))
