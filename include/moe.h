@@ -139,6 +139,22 @@ MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, mo
 MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* moe_route without a workspace, for callers that cannot allocate device memory: code running
+ * inside another runtime's fixed device-memory pool, serving paths that forbid any device
+ * allocation after start-up, plugins whose host framework owns every allocation.  The pages
+ * have no counterpart; it exists for these callers only.
+ * Same inputs, outputs, validation and results as moe_route.  The router's scratch (per-block
+ * sums and per-chunk histograms) lives in a 1 MiB array built into the library, which every GPU
+ * that loads the library keeps until the process exits.  It needs
+ *   align256(ceil(T/32)*(E+1)*4) + align256(k*ceil(T/32)*E*4) + align256(E*4) <= 1 MiB
+ * (for example T = 16384 with E = 64, k = 2 uses 395 KB); larger shapes return MOE_ERR_WORKSPACE
+ * before anything is launched.  No device memory is allocated or freed, by this call or by any
+ * routine it calls.  The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress, with the device current); make that first call before any stream
+ * capture.  Every call, on every stream, shares the one array and leaves the last call's contents
+ * in it: calls that overlap on the GPU race, so serialise them (one stream, or events). */
+MOE_API moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream);
+
 /* Dispatch (Core Concepts 4 "capacity_factor", "drop_tokens"; Best Practices 2; Advanced Patterns
  * Mixtral block gather by expert).  Assignments are visited slot-major then by token; an
  * assignment is kept iff fewer than `capacity` earlier assignments went to its expert.

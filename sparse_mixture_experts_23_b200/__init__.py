@@ -21,7 +21,7 @@ DTYPES = {"f32": MOE_DTYPE_F32, "bf16": MOE_DTYPE_BF16}
 ENTRY_POINTS = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_forward_host", "moe_get_device_status", "moe_set_wait_limit", "moe_debug_timeout_probe",
-    "moe_last_launch_count", "moe_status_string",
+    "moe_last_launch_count", "moe_status_string", "moe_route_noalloc",
 )
 
 
@@ -66,6 +66,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         fn = getattr(lib, name)
         fn.argtypes = [P(Shape), P(IO), vp, sz, vp]
         fn.restype = st
+    lib.moe_route_noalloc.argtypes = [P(Shape), P(IO), vp]
+    lib.moe_route_noalloc.restype = st
     lib.moe_expert_ffn.argtypes = [P(Shape), P(IO), vp, sz, ctypes.c_int, vp]
     lib.moe_expert_ffn.restype = st
     lib.moe_forward_host.argtypes = [P(Shape), P(IO), vp, vp, vp, sz, vp]
@@ -112,6 +114,10 @@ def moe_workspace_layout(shape: Shape, ws: int) -> WsView:
 
 def moe_route(shape, io, ws, ws_bytes, stream=0) -> int:
     return load_library().moe_route(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, stream)
+
+
+def moe_route_noalloc(shape, io, stream=0) -> int:
+    return load_library().moe_route_noalloc(ctypes.byref(shape), ctypes.byref(io), stream)
 
 
 def moe_permute(shape, io, ws, ws_bytes, stream=0) -> int:

@@ -1,0 +1,125 @@
+// moe_route_noalloc: the router stage for callers that cannot allocate device memory.
+//
+// Some callers cannot hand this library a workspace: code that runs inside another runtime's
+// fixed device-memory pool with no room to carve from, latency-critical serving paths where any
+// device allocation is forbidden once the process is up, and plugins whose host framework owns
+// every allocation.  For them this entry point runs the same router kernels as moe_route, but
+// keeps the router's scratch (per-block softmax sums, lse^2 sums and per-chunk expert
+// histograms) in a fixed array compiled into the library instead of in a caller workspace.
+//
+// The array is a file-scope __device__ object, so every GPU that loads the library holds it
+// until the process exits.  Host code must not use the array's name as a device address: it only
+// names a host-side stand-in.  The device address is looked up once per device, with that device
+// current, by cudaGetSymbolAddress, and handed to the kernels as a plain pointer.
+#include <mutex>
+
+#include "moe_internal.cuh"
+
+namespace {
+
+constexpr size_t kScratchBytes = 1u << 20;  // 1 MiB
+__device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mutex;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// Device address of g_route_scratch on the current device; looked up on first use per device.
+cudaError_t scratch_for_current_device(void** out) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_route_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+// Scratch layout for a shape: router partials [nblk][E+1] fp32, chunk histograms [k][nblk][E]
+// int32, per-expert totals [E] int32, each section 256-byte aligned.
+size_t scratch_bytes(const moe_shape_t* s, size_t* hist_off, size_t* cnt_off) {
+  const size_t nblk = ((size_t)s->T + moe::kChunk - 1) / moe::kChunk;
+  const size_t part = align256(nblk * ((size_t)s->E + 1) * 4);
+  const size_t hist = align256((size_t)s->k * nblk * (size_t)s->E * 4);
+  *hist_off = part;
+  *cnt_off = part + hist;
+  return part + hist + align256((size_t)s->E * 4);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream) {
+  if (shape == nullptr || io == nullptr) return MOE_ERR_INVALID_ARG;
+  // same argument rules as moe_route, checked through a zero-size workspace probe of the shape
+  if (moe_workspace_size(shape) == 0) {
+    if (shape->T < 0 || shape->H <= 0 || shape->E <= 0 || shape->F <= 0 || shape->k <= 0 || shape->k > shape->E ||
+        shape->k > 8 || shape->E > 256 || !(shape->capacity_factor > 0.0) ||
+        (shape->dtype != MOE_DTYPE_F32 && shape->dtype != MOE_DTYPE_BF16))
+      return MOE_ERR_INVALID_ARG;
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (io->aux_loss == nullptr || io->z_loss == nullptr) return MOE_ERR_INVALID_ARG;
+  size_t hist_off = 0, cnt_off = 0;
+  if (scratch_bytes(shape, &hist_off, &cnt_off) > kScratchBytes)
+    return MOE_ERR_WORKSPACE;  // shape too large for the built-in scratch
+  if (shape->T == 0) return moe::launch_zero_outputs(nullptr, 0, io->aux_loss, io->z_loss, stream) == cudaSuccess
+                                ? MOE_OK
+                                : MOE_ERR_CUDA;
+  if (io->x == nullptr || io->Wg == nullptr || io->bg == nullptr || io->topk_idx == nullptr || io->topk_w == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(io->x) & 15u) || (reinterpret_cast<uintptr_t>(io->Wg) & 15u))
+    return MOE_ERR_INVALID_ARG;
+
+  void* base = nullptr;
+  if (scratch_for_current_device(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  const int nblk = (shape->T + moe::kChunk - 1) / moe::kChunk;
+  float* loss_part = static_cast<float*>(base);
+  int32_t* chunk_hist = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + hist_off);
+  int32_t* cnt_pre = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + cnt_off);
+  // Every element the kernels read from the scratch is written earlier in the same call (each
+  // router block writes its whole partial row and histogram rows; the reduction writes the
+  // per-expert totals before reading them), so nothing needs clearing between calls.
+  moe::RouterArgs r{};
+  r.x = io->x;
+  r.Wg = io->Wg;
+  r.bg = io->bg;
+  r.T = shape->T;
+  r.H = shape->H;
+  r.E = shape->E;
+  r.k = shape->k;
+  r.topk_idx = io->topk_idx;
+  r.topk_w = io->topk_w;
+  r.loss_part = loss_part;
+  r.chunk_hist = chunk_hist;
+  if (moe::launch_router(r, shape->dtype, stream) != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe::ReduceArgs a{};
+  a.T = shape->T;
+  a.E = shape->E;
+  a.k = shape->k;
+  a.nblk = nblk;
+  a.cap = -1;
+  a.loss_part = loss_part;
+  a.chunk_hist = chunk_hist;
+  a.chunk_base = nullptr;
+  a.cnt_pre = cnt_pre;
+  a.expert_counts = nullptr;
+  a.offsets = nullptr;
+  a.aux_loss = io->aux_loss;
+  a.z_loss = io->z_loss;
+  a.do_losses = 1;
+  a.do_dispatch = 0;
+  return moe::launch_reduce(a, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // extern "C"
