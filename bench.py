@@ -67,7 +67,7 @@ class ClockSampler:
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_power_cap,power.limit,temperature.gpu")
 
     def __init__(self, gpu_id: str | None):
         self.gpu_id = gpu_id
@@ -101,7 +101,7 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
-        sm, smax, power, reasons = [], [], [], set()
+        sm, smax, power, reasons, plimit, temp = [], [], [], set(), [], []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -116,12 +116,19 @@ class ClockSampler:
             for n, v in zip(names, parts[4:8]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
+            try:
+                plimit.append(float(parts[8]))
+                temp.append(float(parts[9]))
+            except (ValueError, IndexError):
+                pass
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         thr = max(power) * 0.5 if power else 0
         loaded = [s for s, p in zip(sm, power) if p >= thr] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm), "power_w_max": max(power) if power else None}
+                "samples": len(sm), "power_w_max": max(power) if power else None,
+                "power_w_median": statistics.median(power) if power else None,
+                "power_limit_w": max(plimit) if plimit else None, "temp_c_max": max(temp) if temp else None}
 
 
 def dist_env():
@@ -288,15 +295,31 @@ def run_ours_impl(args, cfg):
     reps = min(max(args.steps, 20), 200)
 
     def time_calls(fn) -> float:
+        """Average device time of one call: `reps` calls captured in a CUDA graph and replayed, so
+        host-side launch cost does not enter (plain back-to-back calls when capture fails)."""
         for _ in range(2):
             fn()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize()
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for _ in range(reps):
+                    fn()
+            g.replay()
+            torch.cuda.synchronize()
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            del g
+        except Exception:
+            torch.cuda.synchronize()
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
         return a.elapsed_time(b) / reps
 
     ms_ffn = time_calls(lambda: buf.expert_ffn(True))

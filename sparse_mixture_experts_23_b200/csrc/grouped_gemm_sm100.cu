@@ -8,14 +8,15 @@
 //   GEMM2 (EPI_COMBINE):  out[t, n] += w(t,s) * ( sum_k h[r,k] W2[e,k,n] + b2[e,n] ),  t,s = row r's
 //   GEMM2 (EPI_STORE_Y):  y[r, n]   = sum_k h[r,k] W2[e,k,n] + b2[e,n]
 //
-// Design (one persistent CTA per SM, 192 threads):
+// Design (one persistent CTA per SM, 320 threads):
 //   warp 0      TMA producer: A tile [128 rows x 64 k] (K-major, 128B swizzle) and B tile
 //               [64 k x BN n] (weights are stored n-contiguous, i.e. MN-major, 128B swizzle, loaded
 //               as BN/64 boxes of 64x64) into a kStages-deep shared-memory ring.
 //   warp 1      allocates 2*BN TMEM columns (two fp32 accumulators), one elected lane issues
 //               tcgen05.mma kind::f16 (M=128, N=BN, K=16, bf16 x bf16 -> fp32) and tcgen05.commit
 //               to release smem stages and to hand a finished accumulator to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns per step (each thread owns one row),
+//   warps 2..9  epilogue: tcgen05.ld 32 lanes x 32 columns per step (each thread owns one row; two
+//               warps share each TMEM lane quarter and split the tile's columns),
 //               fused bias + GELU -> bf16 store, or bias + gate-weight scale + vector fp32 red.add
 //               into out (at most k adds per element, so k <= 2 is order independent).
 // Tiles run expert-major, then n-tile, then m-tile, so the CTAs in flight share one expert's
@@ -23,11 +24,12 @@
 // m-tile are computed on whatever the buffer holds there and masked in the epilogue.
 // Every mbarrier wait is bounded: a wait that runs out sets the workspace error word, raises a
 // CTA-wide abort flag, and the CTA drains its in-flight copies / MMAs (bounded) and exits.
-// No TMA multicast is used anywhere.
+// Every TMA load brings one CTA its own tile; no load is shared across the CTAs of a cluster.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <stdlib.h>
 
 #include "moe_internal.cuh"
 
@@ -37,13 +39,19 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BK = 64;  // one 128-byte swizzle row of bf16
-constexpr int kThreads = 192;
+#ifndef MOE_EPI_WARPS
+#define MOE_EPI_WARPS 4
+#endif
+constexpr int kEpiWarps = MOE_EPI_WARPS;  // 4 or 8: one or two warps per TMEM lane quarter
+constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kStgStride = 36;                     // floats per staged row (32 + 4: 16-byte rows, spread banks)
+constexpr int kStgWarpBytes = 32 * kStgStride * 4;  // one warp's 32 x 32 fp32 staging tile
 
 enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2 };
 
 template <int BN>
 struct Cfg {
-  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int kStages = BN == 256 ? 3 : (BN == 128 ? 5 : 6);
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = BK * BN * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -53,7 +61,9 @@ struct Cfg {
   static constexpr int kNumBars = 2 * kStages + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kOffsOff = kMiscOff + 16;
-  static constexpr int kSmemBytes = 1024 + kOffsOff + 2 * 260 * 4;
+  static constexpr int kStgOff = (kOffsOff + 2 * 260 * 4 + 127) & ~127;  // per-warp epilogue staging tiles
+  static constexpr int kSmemBytes = 1024 + kStgOff + kEpiWarps * kStgWarpBytes;
+  static_assert(kStgOff % 16 == 0 && kSmemBytes <= 232448, "shared-memory plan");
   // instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16 MN-major, M=128, N=BN
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                      ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
@@ -180,6 +190,68 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 }
 
+// ---- CTA-pair (cta_group::2) helpers --------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+// address of the same shared-memory offset in CTA `rank` of this cluster
+__device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+}
+// TMA into this CTA's shared memory, completion bytes counted on a barrier of either CTA of the pair
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
+      "%4}], [%5];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot), "r"(ncols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// arrive (once the pair's prior MMAs complete) on the barrier at this offset in both CTAs of the pair
+__device__ __forceinline__ void mma_commit_both(uint32_t bar) {
+  const uint16_t both = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster"
+      ".multicast::cluster.b64 [%0], %1;\n" ::"r"(bar),
+      "h"(both)
+      : "memory");
+}
+// arrive (once the pair's prior MMAs complete) on the barrier at cluster address `bar`
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
@@ -211,6 +283,43 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, const i
   rows = min(BM, cnt - m_local * BM);
 }
 
+// Epilogue of one 32 x 32 accumulator chunk of a warp (lane i holds row i of the chunk in r[]).
+// The chunk goes through the warp's shared staging tile so that, after the transpose, lane j owns
+// column j and every global store or reduction writes one contiguous row segment:
+//   EPI_GELU:    h[grow_i, n0 + j]   = bf16(GELU(acc + b1[n0 + j]))       (64 B per row)
+//   EPI_COMBINE: out[tok_i, n0 + j] += w_i * (acc + b2[n0 + j])           (128 B per row, fp32 red)
+//   EPI_STORE_Y: y[grow_i, n0 + j]   = acc + b2[n0 + j]                   (128 B per row)
+// Rows i >= nrows (past the expert's segment) are skipped.  grow_i = grow0 + i.
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t (&r)[32], float* stg, int lane,
+                                               int grow0, int nrows, int my_tok, float my_w, const __nv_bfloat16* brow,
+                                               int n0) {
+  float4* mine = reinterpret_cast<float4*>(stg + lane * kStgStride);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    mine[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                          __uint_as_float(r[4 * q + 3]));
+  __syncwarp();
+  const float bj = __bfloat162float(brow[n0 + lane]);
+  const int nr = nrows < 32 ? nrows : 32;
+  if (EPI == EPI_GELU) {
+    for (int i = 0; i < nr; ++i) {
+      const float v = stg[i * kStgStride + lane] + bj;
+      g.h_out[(size_t)(grow0 + i) * g.N + n0 + lane] = __float2bfloat16_rn(gelu_erf(v));
+    }
+  } else if (EPI == EPI_COMBINE) {
+    for (int i = 0; i < nr; ++i) {
+      const int tok = __shfl_sync(0xffffffffu, my_tok, i);
+      const float w = __shfl_sync(0xffffffffu, my_w, i);
+      const float v = stg[i * kStgStride + lane] + bj;
+      atomicAdd(g.out + (size_t)tok * g.N + n0 + lane, w * v);
+    }
+  } else {
+    for (int i = 0; i < nr; ++i) g.y[(size_t)(grow0 + i) * g.N + n0 + lane] = stg[i * kStgStride + lane] + bj;
+  }
+  __syncwarp();
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
@@ -231,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int E = g.E, NT = g.N / BN, KB = g.K / BK;
+  float* stg = reinterpret_cast<float*>(smem + C::kStgOff + (warp >= 2 ? warp - 2 : 0) * kStgWarpBytes);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -239,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 4);
+      mbar_init(tempty_bar(b), kEpiWarps);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -354,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5) --------
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int half = (warp - 2) >> 2;  // which half of the tile's columns this warp handles
     const int r_in_tile = quarter * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
@@ -374,47 +485,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
       }
       const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
+      const int wrows = rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      constexpr int kChunks = BN / 32 / (kEpiWarps / 4);  // 32-column chunks per epilogue warp
+      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
-        const int n0 = n_idx * BN + c * 32;
-        if (row_ok) {
-          float v[32];
-          const uint4* bp = reinterpret_cast<const uint4*>(brow + n0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 bb = __ldg(bp + q);
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              float2 f = __bfloat1622float2(b2[u]);
-              v[q * 8 + 2 * u] = __uint_as_float(r[q * 8 + 2 * u]) + f.x;
-              v[q * 8 + 2 * u + 1] = __uint_as_float(r[q * 8 + 2 * u + 1]) + f.y;
-            }
-          }
-          if (EPI == EPI_GELU) {
-            uint4* dst = reinterpret_cast<uint4*>(g.h_out + (size_t)grow * g.N + n0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint4 o;
-              o.x = pack_bf16(gelu_erf(v[q * 8 + 0]), gelu_erf(v[q * 8 + 1]));
-              o.y = pack_bf16(gelu_erf(v[q * 8 + 2]), gelu_erf(v[q * 8 + 3]));
-              o.z = pack_bf16(gelu_erf(v[q * 8 + 4]), gelu_erf(v[q * 8 + 5]));
-              o.w = pack_bf16(gelu_erf(v[q * 8 + 6]), gelu_erf(v[q * 8 + 7]));
-              dst[q] = o;
-            }
-          } else if (EPI == EPI_COMBINE) {
-            float* dst = g.out + (size_t)tok * g.N + n0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              red_add_v4(dst + 4 * q, wgt * v[4 * q], wgt * v[4 * q + 1], wgt * v[4 * q + 2], wgt * v[4 * q + 3]);
-          } else {
-            float4* dst = reinterpret_cast<float4*>(g.y + (size_t)grow * g.N + n0);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          }
-        }
+        if (wrows > 0) epilogue_chunk<EPI>(g, r, stg, lane, row0 + quarter * 32, wrows, tok, wgt, brow, n_idx * BN + c * 32);
       }
       tc_fence_before();
       __syncwarp();
@@ -424,9 +501,268 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  __syncwarp();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// CTA-pair variant: a cluster of 2 CTAs on one TPC computes a 256 x 256 tile with
+// tcgen05.mma.cta_group::2 (M=256, N=256, K=16).  Each CTA loads its own 128 rows of A and its
+// own 128 columns of B (so each SM streams half of B), and each CTA's TMEM receives the fp32
+// accumulator of its 128 rows.  Shared-memory traffic per FLOP falls by a third against the
+// single-CTA 128 x 256 tile, which is what lets the tensor pipe run near its rate.
+//   leader (rank 0): arms the full barriers with both CTAs' bytes, issues the MMAs, commits to
+//                    the empty / accumulator-full barriers of both CTAs;
+//   both CTAs:       TMA producer (completion counted on the leader's full barrier), epilogue
+//                    on their own rows (released to the leader's accumulator-empty barrier).
+struct PairCfg {
+  static constexpr int kTileM = 256, kTileN = 256;
+  static constexpr int kHalfN = 128;  // B columns held by each CTA
+  static constexpr int kSubK = 2;     // 64-wide K sub-blocks per pipeline stage
+  static constexpr int kStageK = kSubK * BK;
+#ifndef MOE_PAIR_STAGES
+#define MOE_PAIR_STAGES 3
+#endif
+  static constexpr int kStages = MOE_PAIR_STAGES;
+  static constexpr int kASubBytes = BM * BK * 2;       // 16 KB: 128 rows x 64 k
+  static constexpr int kBSubBytes = BK * kHalfN * 2;   // 16 KB: 64 k x 128 columns (two 64x64 boxes)
+  static constexpr int kABytes = kSubK * kASubBytes;   // 32 KB
+  static constexpr int kBBytes = kSubK * kBSubBytes;   // 32 KB
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * kTileN;
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kStages + 4 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kOffsOff = kMiscOff + 16;
+  static constexpr int kStgOff = (kOffsOff + 2 * 260 * 4 + 127) & ~127;
+  static constexpr int kSmemBytes = 1024 + kStgOff + kEpiWarps * kStgWarpBytes;
+  static_assert(kStgOff % 16 == 0 && kSmemBytes <= 232448, "shared-memory plan");
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                                     ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+};
+
+__device__ __forceinline__ void decode_tile_m(int tile, const int* prefix, const int* offs, int E, int NT, int tile_m,
+                                              int& e, int& m_local, int& n_idx, int& row0, int& rows) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= tile) lo = mid;
+    else hi = mid;
+  }
+  e = lo;
+  const int cnt = offs[e + 1] - offs[e];
+  const int mt = (cnt + tile_m - 1) / tile_m;
+  const int local = tile - prefix[e];
+  n_idx = local / mt;
+  m_local = local % mt;
+  row0 = offs[e] + m_local * tile_m;
+  rows = min(tile_m, cnt - m_local * tile_m);
+}
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                             GemmArgs g) {
+  using C = PairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  int* offs = reinterpret_cast<int*>(smem + C::kOffsOff);
+  int* prefix = offs + 260;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* stg = reinterpret_cast<float*>(smem + C::kStgOff + (warp >= 2 ? warp - 2 : 0) * kStgWarpBytes);
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const int E = g.E, NT = g.N / C::kTileN, KB = g.K / C::kStageK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 2 * kEpiWarps);  // every epilogue warp of both CTAs of the pair
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  for (int i = threadIdx.x; i <= E; i += kThreads) offs[i] = g.offsets[i];
+  if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int e = 0; e < E; ++e) {
+      prefix[e] = run;
+      run += ((offs[e + 1] - offs[e] + C::kTileM - 1) / C::kTileM) * NT;
+    }
+    prefix[E] = run;
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers are initialised before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = prefix[E];
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs) -----
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
+      bool ok = true;
+      for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
+        int e, m_local, n_idx, row0, rows;
+        decode_tile_m(tile, prefix, offs, E, NT, C::kTileM, e, m_local, n_idx, row0, rows);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = sbase + stage * C::kABytes;
+          const uint32_t b_dst = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
+          if (leader) {
+            mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
+            armed[stage] = (int)phase;
+          }
+          const uint32_t fb = peer_addr(full_bar(stage), 0);
+#pragma unroll
+          for (int sk = 0; sk < C::kSubK; ++sk) {
+            const int k0 = kb * C::kStageK + sk * BK;
+            tma_load_2d_pair(a_dst + sk * C::kASubBytes, &tmA, k0, row0 + BM * (int)rank, fb);
+#pragma unroll
+            for (int j = 0; j < C::kHalfN / 64; ++j)
+              tma_load_3d_pair(b_dst + sk * C::kBSubBytes + j * (BK * 128), &tmB,
+                               n_idx * C::kTileN + C::kHalfN * (int)rank + j * 64, k0, e, fb);
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (leader && (!ok || *abort_flag)) {
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed[s] >= 0) {
+            volatile int dummy = 0;
+            mbar_wait(full_bar(s), (uint32_t)armed[s], g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only) -----
+    if (leader && lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = cluster_id; tile < total && ok; tile += nclusters, ++it) {
+        const int buf = it & 1;
+        const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+        if (!mbar_wait(tempty_bar(buf), tphase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kTileN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status, kDevTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = sbase + stage * C::kABytes;
+          const uint32_t b_addr = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
+#pragma unroll
+          for (int kk = 0; kk < C::kStageK / 16; ++kk) {
+            const int sk = kk / (BK / 16), ks = kk % (BK / 16);
+            mma_bf16_pair(d_tmem, desc_a_kmajor(a_addr + sk * C::kASubBytes + ks * 32),
+                          desc_b_mnmajor(b_addr + sk * C::kBSubBytes + ks * 16 * 128), C::kIdesc,
+                          (kb | kk) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit_both(empty_bar(stage));  // frees this stage in both CTAs once its MMAs are done
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_both(tfull_bar(buf));
+      }
+      if ((!ok || *abort_flag) && issued) {
+        mma_commit_pair(drain_bar);
+        volatile int dummy = 0;
+        mbar_wait(drain_bar, 0, g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5, both) --
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int r_in_tile = quarter * 32 + lane;
+    const uint32_t tempty_leader0 = peer_addr(tempty_bar(0), 0);
+    const uint32_t tempty_leader1 = peer_addr(tempty_bar(1), 0);
+    int it = 0;
+    for (int tile = cluster_id; tile < total; tile += nclusters, ++it) {
+      int e, m_local, n_idx, row0, rows;
+      decode_tile_m(tile, prefix, offs, E, NT, C::kTileM, e, m_local, n_idx, row0, rows);
+      const int buf = it & 1;
+      const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+      const bool got = mbar_wait(tfull_bar(buf), tphase, g.wait_limit, abort_flag, g.status, kDevTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int my_rows = rows - BM * (int)rank;  // rows of this tile held by this CTA (may be <= 0)
+      const bool row_ok = r_in_tile < my_rows;
+      const int grow = row0 + BM * (int)rank + r_in_tile;
+      float wgt = 0.f;
+      int tok = 0;
+      if (EPI == EPI_COMBINE && row_ok) {
+        tok = g.row_token[grow];
+        wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
+      }
+      const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
+      const int wrows = my_rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
+#pragma unroll 1
+      constexpr int kChunks = C::kTileN / 32 / (kEpiWarps / 4);
+      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::kTileN + c * 32), r);
+        if (wrows > 0)
+          epilogue_chunk<EPI>(g, r, stg, lane, row0 + BM * (int)rank + quarter * 32, wrows, tok, wgt, brow,
+                              n_idx * C::kTileN + c * 32);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync_all();  // neither CTA frees TMEM or exits while the pair still uses it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
   }
 }
 
@@ -453,6 +789,17 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   }
   return fn;
+}
+
+// CTA-pair tiles are the default for N divisible by 256; MOE_GEMM_PAIR=0 in the environment selects
+// the single-CTA kernel instead (kept for comparison and as the path for other widths).
+bool pair_mode_enabled() {
+  static int mode = -1;
+  if (mode < 0) {
+    const char* v = getenv("MOE_GEMM_PAIR");
+    mode = (v != nullptr && v[0] == '0') ? 0 : 1;
+  }
+  return mode == 1;
 }
 
 // A operand: [rows, K] bf16 row-major; box = 64 k x 128 rows
@@ -484,15 +831,25 @@ bool make_map_b(CUtensorMap* m, const void* base, int E, int K, int N) {
 template <int BN, int EPI>
 cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid, cudaStream_t st) {
   auto kern = grouped_gemm_kernel<BN, EPI>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes);
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(kern), Cfg<BN>::kSmemBytes);
   if (err != cudaSuccess) return err;
   kern<<<grid, kThreads, Cfg<BN>::kSmemBytes, st>>>(ma, mb, g);
   return cudaGetLastError();
 }
 
 template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid, cudaStream_t st) {
+  auto kern = grouped_gemm_pair_kernel<EPI>;
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(kern), PairCfg::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  kern<<<grid & ~1, kThreads, PairCfg::kSmemBytes, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
+template <int EPI>
 cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid,
                       cudaStream_t st) {
+  if (N % 256 == 0 && g.K % PairCfg::kStageK == 0 && pair_mode_enabled()) return launch_pair<EPI>(ma, mb, g, grid, st);
   if (N % 256 == 0) return launch_one<256, EPI>(ma, mb, g, grid, st);
   if (N % 128 == 0) return launch_one<128, EPI>(ma, mb, g, grid, st);
   return launch_one<64, EPI>(ma, mb, g, grid, st);

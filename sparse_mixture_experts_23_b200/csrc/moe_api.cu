@@ -5,11 +5,38 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+#include <vector>
+
 #include "moe_internal.cuh"
 
 namespace moe {
 
 static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
+  struct Entry {
+    const void* kernel;
+    int device;
+    int bytes;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> done;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(mu);
+  for (Entry& en : done)
+    if (en.kernel == kernel && en.device == dev) {
+      if (en.bytes >= bytes) return cudaSuccess;
+      err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (err == cudaSuccess) en.bytes = bytes;
+      return err;
+    }
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess) done.push_back({kernel, dev, bytes});
+  return err;
+}
 
 WsLayout ws_layout(const moe_shape_t& s) {
   WsLayout L{};

@@ -93,6 +93,10 @@ struct FfnArgs {
   int num_sms;
 };
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the current device; the
+// driver call is made once per (kernel, device) and size, so repeated launches cost nothing.
+cudaError_t ensure_smem_limit(const void* kernel, int bytes);
+
 cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st);
 cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, cudaStream_t st);
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);

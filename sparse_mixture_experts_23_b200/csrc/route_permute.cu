@@ -10,6 +10,7 @@
 #include <cuda_bf16.h>
 #include <float.h>
 #include <math.h>
+#include <stdlib.h>
 
 #include "moe_internal.cuh"
 
@@ -61,13 +62,124 @@ __host__ __device__ inline RouterSmem router_smem(int E, int esize) {
   return s;
 }
 
+// Softmax, top-k, renormalisation and the block's loss partials from logits[32][epad] in shared
+// memory (bias already added).  256 threads: warp w handles the chunk's tokens w, w+8, w+16, w+24.
+// psum: [8][epad] floats, hist: [k][E] ints, zw: [8] floats, all shared.
+__device__ void router_finish(const RouterArgs& a, const float* logits, int epad, float* psum, int* hist, float* zw) {
+  const int E = a.E, T = a.T, k = a.k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int blk = blockIdx.x;
+  const int t0 = blk * kChunk;
+  for (int i = tid; i < k * E; i += kRouterThreads) hist[i] = 0;
+  for (int i = tid; i < 8 * epad; i += kRouterThreads) psum[i] = 0.f;
+  __syncthreads();
+
+  const int NJ = (E + 31) / 32;  // <= 8
+  float pacc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) pacc[j] = 0.f;
+  float zacc = 0.f;
+  for (int r = 0; r < 4; ++r) {
+    int tl = warp + 8 * r;
+    int t = t0 + tl;
+    if (t >= T) break;
+    float lv[8];
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      int e = lane + 32 * j;
+      lv[j] = (j < NJ && e < E) ? logits[tl * epad + e] : -INFINITY;
+      m = fmaxf(m, lv[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s += (j < NJ && lane + 32 * j < E) ? expf(lv[j] - m) : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float inv_s = 1.f / s;
+    const float lse = m + logf(s);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (j < NJ && lane + 32 * j < E) pacc[j] += expf(lv[j] - m) * inv_s;
+    zacc += lse * lse;
+
+    // top-k: k rounds of a warp arg-max with ties to the lower index
+    unsigned taken = 0;
+    float psel_sum = 0.f;
+    float my_p = 0.f;
+    int my_e = -1;
+    for (int rr = 0; rr < k; ++rr) {
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        int e = lane + 32 * j;
+        if (j < NJ && e < E && !((taken >> j) & 1u)) {
+          if (lv[j] > bv || (lv[j] == bv && e < be)) {
+            bv = lv[j];
+            be = e;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      float pv = expf(bv - m) * inv_s;
+      psel_sum += pv;
+      if (lane == rr) {
+        my_p = pv;
+        my_e = be;
+      }
+    }
+    if (lane < k) {
+      a.topk_idx[(size_t)t * k + lane] = my_e;
+      a.topk_w[(size_t)t * k + lane] = my_p / psel_sum;
+      if (a.chunk_hist) atomicAdd(&hist[lane * E + my_e], 1);
+    }
+  }
+  // per-warp partial sums -> smem; then fixed-order sums across warps
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    int e = lane + 32 * j;
+    if (j < NJ && e < E) psum[warp * epad + e] = pacc[j];
+  }
+  if (lane == 0) zw[warp] = zacc;  // every lane holds the same per-warp sum of lse^2
+  __syncthreads();
+  for (int e = tid; e < E; e += kRouterThreads) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += psum[w * epad + e];
+    a.loss_part[(size_t)blk * (E + 1) + e] = s;
+  }
+  if (tid == 0) {
+    float s = 0.f;
+    for (int w = 0; w < 8; ++w) s += zw[w];
+    a.loss_part[(size_t)blk * (E + 1) + E] = s;
+  }
+  if (a.chunk_hist) {
+    const int nblk = gridDim.x;
+    for (int i = tid; i < k * E; i += kRouterThreads) {
+      int s = i / E, e = i % E;
+      a.chunk_hist[((size_t)s * nblk + blk) * E + e] = hist[i];
+    }
+  }
+}
+
 template <typename TIn>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const int E = a.E, H = a.H, T = a.T, k = a.k;
+  const int E = a.E, H = a.H, T = a.T;
   constexpr int esize = sizeof(TIn);
   const RouterSmem L = router_smem(E, esize);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int blk = blockIdx.x;
   const int t0 = blk * kChunk;
   const TIn* x = reinterpret_cast<const TIn*>(a.x);
@@ -194,111 +306,457 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   }
   __syncthreads();
 
-  // ---- softmax, top-k, renormalisation, loss partials: warp w handles tokens w, w+8, w+16, w+24 ----
-  float* psum = reinterpret_cast<float*>(smem + L.psum);
-  int* hist = reinterpret_cast<int*>(smem + L.misc);
-  float* zw = reinterpret_cast<float*>(smem + L.misc + 8 * 256 * 4);
-  for (int i = tid; i < k * E; i += kRouterThreads) hist[i] = 0;
-  for (int i = tid; i < 8 * L.epad; i += kRouterThreads) psum[i] = 0.f;
+  router_finish(a, logits, L.epad, reinterpret_cast<float*>(smem + L.psum), reinterpret_cast<int*>(smem + L.misc),
+                reinterpret_cast<float*>(smem + L.misc + 8 * 256 * 4));
+}
+
+// Streaming router for bf16 with few experts (E <= 16): memory-bound, so the gate weights stay in
+// shared memory and each warp streams 4 token rows from HBM with 16-byte loads (lane l reads
+// 16-byte chunks l, l+32, ...).  Wg is stored in groups of 8 rows padded by 16 bytes so that the
+// 32 lanes, which read rows 8 apart, spread over all banks.
+template <int EP>
+struct StreamSmem {
+  static constexpr int kGroupBytes = 8 * EP * 2 + 16;  // 8 Wg rows of EP bf16 + pad
+  static __host__ __device__ int wg_bytes(int H) { return (H / 8) * kGroupBytes; }
+  static __host__ __device__ int logits_off(int H) { return (wg_bytes(H) + 15) & ~15; }
+  static __host__ __device__ int psum_off(int H) { return logits_off(H) + kChunk * EP * 4; }
+  static __host__ __device__ int misc_off(int H) { return psum_off(H) + 8 * EP * 4; }
+  static __host__ __device__ int total(int H) { return misc_off(H) + (8 * 256 + 64) * 4; }
+};
+
+template <int EP>
+__global__ void __launch_bounds__(kRouterThreads) router_stream_kernel(RouterArgs a) {
+  using S = StreamSmem<EP>;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int E = a.E, H = a.H, T = a.T;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const __nv_bfloat16* Wg = reinterpret_cast<const __nv_bfloat16*>(a.Wg);
+  // stage Wg [H][E] -> padded groups of 8 rows x EP columns (zero for e >= E)
+  if (E == EP && EP >= 8) {
+    // whole rows as 16-byte vectors, all loads of a thread issued before its stores
+    constexpr int VPR = EP / 8;  // 16-byte vectors per row
+    const uint4* src = reinterpret_cast<const uint4*>(Wg);
+    const int nvec = H * VPR;
+    for (int i0 = tid; i0 < nvec; i0 += kRouterThreads * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kRouterThreads;
+        v[u] = i < nvec ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kRouterThreads;
+        if (i < nvec) {
+          const int h = i / VPR, q = i % VPR;
+          *reinterpret_cast<uint4*>(smem + (h >> 3) * S::kGroupBytes + ((h & 7) * EP + 8 * q) * 2) = v[u];
+        }
+      }
+    }
+  } else {
+    for (int i = tid; i < H * EP; i += kRouterThreads) {
+      const int h = i / EP, e = i % EP;
+      __nv_bfloat16 v = e < E ? Wg[(size_t)h * E + e] : __float2bfloat16(0.f);
+      *reinterpret_cast<__nv_bfloat16*>(smem + (h >> 3) * S::kGroupBytes + ((h & 7) * EP + e) * 2) = v;
+    }
+  }
   __syncthreads();
 
-  const int NJ = (E + 31) / 32;  // <= 8
-  float pacc[8];
+  const int tl0 = warp * 4;  // this warp's 4 tokens inside the chunk
+  const int t0 = blockIdx.x * kChunk + tl0;
+  const int nch = H / 8;  // 16-byte chunks per row
+  const uint4* xr[4];
+  bool valid[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) pacc[j] = 0.f;
-  float zacc = 0.f;
-  for (int r = 0; r < 4; ++r) {
-    int tl = warp + 8 * r;
-    int t = t0 + tl;
-    if (t >= T) break;
-    float lv[8];
-    float m = -INFINITY;
+  for (int i = 0; i < 4; ++i) {
+    valid[i] = t0 + i < T;
+    xr[i] = reinterpret_cast<const uint4*>(a.x) + (size_t)(valid[i] ? t0 + i : 0) * nch;
+  }
+  float acc[4][EP];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      int e = lane + 32 * j;
-      lv[j] = (j < NJ && e < E) ? logits[tl * L.epad + e] : -INFINITY;
-      m = fmaxf(m, lv[j]);
-    }
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s += (j < NJ && lane + 32 * j < E) ? expf(lv[j] - m) : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    const float inv_s = 1.f / s;
-    const float lse = m + logf(s);
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (j < NJ && lane + 32 * j < E) pacc[j] += expf(lv[j] - m) * inv_s;
-    zacc += lse * lse;
+    for (int e = 0; e < EP; ++e) acc[i][e] = 0.f;
 
-    // top-k: k rounds of a warp arg-max with ties to the lower index
-    unsigned taken = 0;
-    float psel_sum = 0.f;
-    float my_p = 0.f;
-    int my_e = -1;
-    for (int rr = 0; rr < k; ++rr) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
+  constexpr int U = EP <= 8 ? 4 : 2;  // chunks per lane in flight per token
+  for (int c0 = lane; c0 < nch; c0 += 32 * U) {
+    uint4 xv[U][4];
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = c0 + 32 * u;
+        xv[u][i] = (valid[i] && c < nch) ? __ldcs(xr[i] + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c >= nch) break;
+      const unsigned char* grp = smem + c * S::kGroupBytes;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        int e = lane + 32 * j;
-        if (j < NJ && e < E && !((taken >> j) & 1u)) {
-          if (lv[j] > bv || (lv[j] == bv && e < be)) {
-            bv = lv[j];
-            be = e;
+        float w[EP];
+        if (EP >= 8) {
+#pragma unroll
+          for (int q = 0; q < EP / 8; ++q) {  // 16-byte reads: conflict-free with the padded groups
+            const uint4 wv = *reinterpret_cast<const uint4*>(grp + (j * EP + 8 * q) * 2);
+            const uint32_t ws4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ws4[r]));
+              w[8 * q + 2 * r] = f.x;
+              w[8 * q + 2 * r + 1] = f.y;
+            }
           }
+        } else {
+          const uint2 wv = *reinterpret_cast<const uint2*>(grp + j * EP * 2);
+          const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.x));
+          const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wv.y));
+          w[0] = lo.x;
+          w[1] = lo.y;
+          w[2] = hi.x;
+          w[3] = hi.y;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t word = (&xv[u][i].x)[j >> 1];
+          const float xf = __uint_as_float((j & 1) ? (word & 0xffff0000u) : (word << 16));
+#pragma unroll
+          for (int e = 0; e < EP; ++e) acc[i][e] = fmaf(xf, w[e], acc[i][e]);
         }
       }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      float pv = expf(bv - m) * inv_s;
-      psel_sum += pv;
-      if (lane == rr) {
-        my_p = pv;
-        my_e = be;
-      }
-    }
-    if (lane < k) {
-      a.topk_idx[(size_t)t * k + lane] = my_e;
-      a.topk_w[(size_t)t * k + lane] = my_p / psel_sum;
-      if (a.chunk_hist) atomicAdd(&hist[lane * E + my_e], 1);
     }
   }
-  // per-warp partial sums -> smem; then fixed-order sums across warps
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    int e = lane + 32 * j;
-    if (j < NJ && e < E) psum[warp * L.epad + e] = pacc[j];
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < EP; ++e)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc[i][e] += __shfl_xor_sync(0xffffffffu, acc[i][e], o);
+
+  float* logits = reinterpret_cast<float*>(smem + S::logits_off(H));
+  if (lane == 0) {
+    const __nv_bfloat16* bg = reinterpret_cast<const __nv_bfloat16*>(a.bg);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < EP; ++e) logits[(tl0 + i) * EP + e] = acc[i][e] + (e < E ? __bfloat162float(bg[e]) : 0.f);
   }
-  if (lane == 0) zw[warp] = zacc;  // every lane holds the same per-warp sum of lse^2
   __syncthreads();
-  for (int e = tid; e < E; e += kRouterThreads) {
-    float s = 0.f;
-    for (int w = 0; w < 8; ++w) s += psum[w * L.epad + e];
-    a.loss_part[(size_t)blk * (E + 1) + e] = s;
-  }
-  if (tid == 0) {
-    float s = 0.f;
-    for (int w = 0; w < 8; ++w) s += zw[w];
-    a.loss_part[(size_t)blk * (E + 1) + E] = s;
-  }
-  if (a.chunk_hist) {
-    const int nblk = gridDim.x;
-    for (int i = tid; i < k * E; i += kRouterThreads) {
-      int s = i / E, e = i % E;
-      a.chunk_hist[((size_t)s * nblk + blk) * E + e] = hist[i];
+  router_finish(a, logits, EP, reinterpret_cast<float*>(smem + S::psum_off(H)), reinterpret_cast<int*>(smem + S::misc_off(H)),
+                reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4));
+}
+
+// Tensor-core router for bf16 with E a multiple of 8: the gate GEMM [32 tokens x H] x [H x E] of
+// one chunk on mma.sync m16n8k16 (bf16 products are exact in fp32, accumulation in fp32), so the
+// kernel stays bound by reading x from HBM for any expert count.  x and Wg tiles of HC columns of
+// H stream through a 3-stage cp.async ring (rows padded to an odd number of 16-byte units so the
+// ldmatrix row reads hit distinct banks); fragments come from ldmatrix, Wg's (k, n) tile via .trans.
+// With fewer than 8 n-tiles the warps split K and their partials are added in a fixed order.
+struct MmaRouterPlan {
+  int ep8, nt8, ks, hc, xs, ws, stage, logits, red, psum, misc, total;
+};
+
+__host__ __device__ inline MmaRouterPlan mma_router_plan(int E, int H) {
+  MmaRouterPlan p;
+  p.ep8 = (E + 7) & ~7;
+  p.nt8 = p.ep8 / 8;
+  p.ks = p.nt8 >= 8 ? 1 : 8 / p.nt8;
+  int wunits = p.ep8 / 8;
+  if ((wunits & 1) == 0) ++wunits;
+  p.ws = wunits * 16;
+  p.hc = 64;
+  for (int hc = 512; hc >= 64; hc >>= 1) {
+    const int xs = hc * 2 + 16;
+    if (3 * (32 * xs + hc * p.ws) <= 150 * 1024 && hc <= H) {
+      p.hc = hc;
+      break;
     }
   }
+  p.xs = p.hc * 2 + 16;
+  p.stage = 32 * p.xs + p.hc * p.ws;
+  p.logits = 3 * p.stage;
+  p.red = p.logits + 32 * p.ep8 * 4;
+  p.psum = p.red + (p.ks > 1 ? p.ks * 32 * p.ep8 * 4 : 0);
+  p.misc = p.psum + 8 * p.ep8 * 4;
+  p.total = p.misc + (8 * 256 + 64) * 4;
+  return p;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                          uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__global__ void __launch_bounds__(kRouterThreads) router_mma_kernel(RouterArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int E = a.E, H = a.H, T = a.T;
+  const MmaRouterPlan P = mma_router_plan(E, H);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = blockIdx.x * kChunk;
+  const unsigned char* xg = reinterpret_cast<const unsigned char*>(a.x);
+  const unsigned char* wg = reinterpret_cast<const unsigned char*>(a.Wg);
+  const int ntiles = (H + P.hc - 1) / P.hc;
+  const int xchunks = P.hc / 8;    // 16-byte chunks per x row per stage
+  const int wchunks = E / 8;       // 16-byte chunks per Wg row (E % 8 == 0)
+
+  auto load_stage = [&](int tile, int stage) {
+    unsigned char* xs = smem + stage * P.stage;
+    unsigned char* ws = xs + 32 * P.xs;
+    const int h0 = tile * P.hc;
+    const int hl = min(P.hc, H - h0);
+    for (int i = tid; i < 32 * xchunks; i += kRouterThreads) {
+      const int r = i / xchunks, c = i % xchunks;
+      const int t = t0 + r;
+      const bool ok = t < T && c * 8 < hl;
+      const void* src = ok ? (const void*)(xg + ((size_t)t * H + h0 + c * 8) * 2) : (const void*)xg;
+      cp_async16(xs + r * P.xs + c * 16, src, ok ? 16 : 0);
+    }
+    for (int i = tid; i < P.hc * wchunks; i += kRouterThreads) {
+      const int r = i / wchunks, c = i % wchunks;
+      const bool ok = r < hl;
+      const void* src = ok ? (const void*)(wg + ((size_t)(h0 + r) * E + c * 8) * 2) : (const void*)wg;
+      cp_async16(ws + r * P.ws + c * 16, src, ok ? 16 : 0);
+    }
+  };
+
+  // warp's n-tiles and K share
+  const int my_ks = P.ks > 1 ? warp / P.nt8 : 0;
+  const bool active = P.ks > 1 ? (warp < P.ks * P.nt8) : true;
+  float acc[4][2][4];  // [n-tile slot][m-tile][fragment]
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[j][m][q] = 0.f;
+
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    if (s < ntiles) load_stage(s, s);
+    cp_async_commit();
+  }
+  for (int tile = 0; tile < ntiles; ++tile) {
+    cp_async_wait<1>();
+    __syncthreads();
+    if (tile + 2 < ntiles) load_stage(tile + 2, (tile + 2) % 3);
+    cp_async_commit();
+    const uint32_t xs = (uint32_t)__cvta_generic_to_shared(smem + (tile % 3) * P.stage);
+    const uint32_t ws = xs + 32 * P.xs;
+    const int ksteps = min(P.hc, H - tile * P.hc) / 16;
+    if (active) {
+      for (int kk = my_ks; kk < ksteps; kk += P.ks) {
+        uint32_t af[2][4];
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const int row = m * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int col = kk * 16 + (lane >> 4) * 8;
+          ldsm_x4(xs + row * P.xs + col * 2, af[m][0], af[m][1], af[m][2], af[m][3]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int nt = P.ks > 1 ? (j == 0 ? warp % P.nt8 : -1) : warp + 8 * j;
+          if (nt < 0 || nt >= P.nt8) continue;
+          uint32_t b0, b1;
+          const int krow = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldsm_x2_trans(ws + krow * P.ws + nt * 16, b0, b1);
+#pragma unroll
+          for (int m = 0; m < 2; ++m) mma_16816(acc[j][m], af[m][0], af[m][1], af[m][2], af[m][3], b0, b1);
+        }
+      }
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();
+
+  // fragments -> logits[32][ep8] (+ bias); K-split partials added in warp order
+  float* logits = reinterpret_cast<float*>(smem + P.logits);
+  float* red = reinterpret_cast<float*>(smem + P.red);
+  const __nv_bfloat16* bg = reinterpret_cast<const __nv_bfloat16*>(a.bg);
+  const int g = lane >> 2, t4 = lane & 3;
+  if (active) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int nt = P.ks > 1 ? (j == 0 ? warp % P.nt8 : -1) : warp + 8 * j;
+      if (nt < 0 || nt >= P.nt8) continue;
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = m * 16 + g + (q >= 2 ? 8 : 0);
+          const int col = nt * 8 + t4 * 2 + (q & 1);
+          if (P.ks > 1) red[(my_ks * 32 + row) * P.ep8 + col] = acc[j][m][q];
+          else logits[row * P.ep8 + col] = acc[j][m][q] + (col < E ? __bfloat162float(bg[col]) : 0.f);
+        }
+    }
+  }
+  if (P.ks > 1) {
+    __syncthreads();
+    for (int o = tid; o < 32 * P.ep8; o += kRouterThreads) {
+      float v = 0.f;
+      for (int q = 0; q < P.ks; ++q) v += red[q * 32 * P.ep8 + o];
+      const int col = o % P.ep8;
+      logits[o] = v + (col < E ? __bfloat162float(bg[col]) : 0.f);
+    }
+  }
+  __syncthreads();
+  router_finish(a, logits, P.ep8, reinterpret_cast<float*>(smem + P.psum), reinterpret_cast<int*>(smem + P.misc),
+                reinterpret_cast<float*>(smem + P.misc + 8 * 256 * 4));
+}
+
+// Register-direct tensor-core router for bf16 with E = 8, 16 or 32 (gate weights resident in
+// shared memory): lanes load 16-byte vectors of x straight from HBM, deeply unrolled, and feed
+// them to mma.sync m16n8k16 without staging.  Lane (g = lane/4, t = lane%4) loads the 8 columns
+// [8t, 8t+8) of a 32-column block for token rows g and g+8; the sum over h does not depend on its
+// order, so the fragments use a permuted k (virtual pair {2t, 2t+1} <-> columns {8t, 8t+1},
+// {2t+8, 2t+9} <-> {8t+2, 8t+3} in the first MMA; columns 8t+4..8t+7 in the second) and the
+// matching Wg^T vector (row e, columns 8t..8t+7) supplies both B fragments.  Warps split H and
+// their partial logits are added in warp order.
+template <int NT8>
+struct DirectSmem {
+  static constexpr int E = NT8 * 8;
+  static __host__ __device__ int row_bytes(int H) { return H * 2 + 16; }  // Wg^T row, padded
+  static __host__ __device__ int red_off(int H) { return E * row_bytes(H); }
+  static __host__ __device__ int logits_off(int H) { return red_off(H) + 8 * 32 * E * 4; }
+  static __host__ __device__ int psum_off(int H) { return logits_off(H) + 32 * E * 4; }
+  static __host__ __device__ int misc_off(int H) { return psum_off(H) + 8 * E * 4; }
+  static __host__ __device__ int total(int H) { return misc_off(H) + (8 * 256 + 64) * 4; }
+};
+
+template <int NT8>
+__global__ void __launch_bounds__(kRouterThreads) router_direct_kernel(RouterArgs a) {
+  using S = DirectSmem<NT8>;
+  constexpr int E = S::E;
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int H = a.H, T = a.T;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int RB = S::row_bytes(H);
+
+  const int t0 = blockIdx.x * kChunk;
+  const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+  const int rowvec = H / 8;  // 16-byte vectors per token row
+  // this lane's token rows: m-tile m, row g (+8)
+  int rows[4];
+  bool rvalid[4];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+      const int t = t0 + 16 * m + g + 8 * hi;
+      rvalid[2 * m + hi] = t < T;
+      rows[2 * m + hi] = t < T ? t : 0;
+    }
+  float acc[2][NT8][4];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < NT8; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[m][n][q] = 0.f;
+
+  const int nblk32 = H / 32 / 8;  // 32-column blocks per warp
+  const int b0 = warp * nblk32;
+  constexpr int U = 4;
+  auto load_x = [&](uint4 (&xr)[U][4], int bb) {
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int blk = b0 + bb + u;
+        xr[u][r] = (rvalid[r] && bb + u < nblk32) ? __ldcs(xv + (size_t)rows[r] * rowvec + blk * 4 + t4)
+                                                  : make_uint4(0, 0, 0, 0);
+      }
+  };
+  uint4 xr[U][4];
+  load_x(xr, 0);  // first x loads go out before the gate weights are staged
+
+  // Wg [H][E] -> Wg^T [E][H] (bf16) in shared memory; each thread issues all its loads first
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.Wg);
+    const int nvec = H * E / 8;
+    for (int i0 = tid; i0 < nvec; i0 += kRouterThreads * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kRouterThreads;
+        v[u] = i < nvec ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kRouterThreads;
+        if (i < nvec) {
+          const int h = (i * 8) / E, e0 = (i * 8) % E;
+          const uint16_t* pv = reinterpret_cast<const uint16_t*>(&v[u]);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) *reinterpret_cast<uint16_t*>(smem + (e0 + q) * RB + h * 2) = pv[q];
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  auto compute = [&](const uint4 (&xr)[U][4], int bb) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (bb + u >= nblk32) break;
+      const int h0 = (b0 + bb + u) * 32;
+#pragma unroll
+      for (int n = 0; n < NT8; ++n) {
+        const uint4 w = *reinterpret_cast<const uint4*>(smem + (n * 8 + g) * RB + (h0 + 8 * t4) * 2);
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const uint4 xa = xr[u][2 * m], xb = xr[u][2 * m + 1];
+          mma_16816(acc[m][n], xa.x, xb.x, xa.y, xb.y, w.x, w.y);
+          mma_16816(acc[m][n], xa.z, xb.z, xa.w, xb.w, w.z, w.w);
+        }
+      }
+    }
+  };
+  // two register groups alternate: the next group's loads are in flight while one is computed
+  uint4 xr2[U][4];
+  for (int bb = 0; bb < nblk32; bb += 2 * U) {
+    if (bb + U < nblk32) load_x(xr2, bb + U);
+    compute(xr, bb);
+    if (bb + 2 * U < nblk32) load_x(xr, bb + 2 * U);
+    if (bb + U < nblk32) compute(xr2, bb + U);
+  }
+  // per-warp partials -> shared, then a fixed-order sum over warps (+ bias)
+  float* red = reinterpret_cast<float*>(smem + S::red_off(H));
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < NT8; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = 16 * m + g + (q >= 2 ? 8 : 0);
+        const int col = n * 8 + t4 * 2 + (q & 1);
+        red[(warp * 32 + row) * E + col] = acc[m][n][q];
+      }
+  __syncthreads();
+  float* logits = reinterpret_cast<float*>(smem + S::logits_off(H));
+  const __nv_bfloat16* bg = reinterpret_cast<const __nv_bfloat16*>(a.bg);
+  for (int o = tid; o < 32 * E; o += kRouterThreads) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w * 32 * E + o];
+    logits[o] = v + __bfloat162float(bg[o % E]);
+  }
+  __syncthreads();
+  router_finish(a, logits, E, reinterpret_cast<float*>(smem + S::psum_off(H)), reinterpret_cast<int*>(smem + S::misc_off(H)),
+                reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4));
 }
 
 // Per-chunk, per-slot expert histogram from a given topk_idx (standalone permute).
@@ -325,6 +783,8 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
   __shared__ int cnt_s[256];
   __shared__ double term[256];
   __shared__ float zred[32];
+  __shared__ float pf[1024];
+  __shared__ float zf[1024];
   const int tid = threadIdx.x, E = a.E;
   const int C = a.k * a.nblk;  // chunks in (slot, token-chunk) order
   const int G = 1024 / E;      // groups of chunks
@@ -368,18 +828,33 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
     a.offsets[E] = run;
   }
   if (a.do_losses) {
-    // P_e: fixed-order sum over router blocks; z: lane-strided then a fixed shuffle tree
-    if (tid < E) {
-      float P = 0.f;
-      for (int b = 0; b < a.nblk; ++b) P += a.loss_part[(size_t)b * (E + 1) + tid];
-      term[tid] = ((double)cnt_s[tid] / ((double)a.T * a.k)) * ((double)P / (double)a.T);
+    // P_e: thread (g, e) sums a fixed range of router blocks, then the group sums are added in
+    // group order; z: thread-strided sums then a fixed tree.  Same order on every run.
+    {
+      const int b0 = in ? (int)((long long)a.nblk * g / G) : 0;
+      const int b1 = in ? (int)((long long)a.nblk * (g + 1) / G) : 0;
+      float ps = 0.f;
+      for (int b = b0; b < b1; ++b) ps += a.loss_part[(size_t)b * (E + 1) + e];
+      if (in) pf[g * E + e] = ps;
+      float zs = 0.f;
+      for (int b = tid; b < a.nblk; b += 1024) zs += a.loss_part[(size_t)b * (E + 1) + E];
+      zf[tid] = zs;
+    }
+    __syncthreads();
+    for (int w = 512; w >= 32; w >>= 1) {
+      if (tid < w) zf[tid] += zf[tid + w];
+      __syncthreads();
     }
     if (tid < 32) {
-      float z = 0.f;
-      for (int b = tid; b < a.nblk; b += 32) z += a.loss_part[(size_t)b * (E + 1) + E];
+      float z = zf[tid];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       if (tid == 0) zred[0] = z;
+    }
+    if (tid < E) {
+      float P = 0.f;
+      for (int q = 0; q < G; ++q) P += pf[q * E + tid];
+      term[tid] = ((double)cnt_s[tid] / ((double)a.T * a.k)) * ((double)P / (double)a.T);
     }
     __syncthreads();
     if (tid == 0) {
@@ -495,17 +970,69 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 }  // namespace
 
+// MOE_ROUTER_MMA=0 in the environment selects the CUDA-core routers instead (for comparison).
+bool router_mma_disabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MOE_ROUTER_MMA");
+    v = (e != nullptr && e[0] == '0') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+template <int EP>
+cudaError_t launch_stream(const RouterArgs& a, int nblk, cudaStream_t st) {
+  const int bytes = StreamSmem<EP>::total(a.H);
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(router_stream_kernel<EP>), bytes);
+  if (err != cudaSuccess) return err;
+  router_stream_kernel<EP><<<nblk, kRouterThreads, bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st) {
   const int nblk = (a.T + kChunk - 1) / kChunk;
+  // bf16, E in {8, 16, 32}, Wg^T fits in shared memory: register-direct tensor-core stream over x
+  if (dtype == MOE_DTYPE_BF16 && (a.E == 8 || a.E == 16 || a.E == 32) && a.H % 256 == 0 && !router_mma_disabled()) {
+    const int bytes = a.E == 8 ? DirectSmem<1>::total(a.H) : (a.E == 16 ? DirectSmem<2>::total(a.H) : DirectSmem<4>::total(a.H));
+    if (bytes <= 200 * 1024) {
+      const void* kern = a.E == 8 ? reinterpret_cast<const void*>(router_direct_kernel<1>)
+                                  : (a.E == 16 ? reinterpret_cast<const void*>(router_direct_kernel<2>)
+                                               : reinterpret_cast<const void*>(router_direct_kernel<4>));
+      cudaError_t err = ensure_smem_limit(kern, bytes);
+      if (err != cudaSuccess) return err;
+      if (a.E == 8) router_direct_kernel<1><<<nblk, kRouterThreads, bytes, st>>>(a);
+      else if (a.E == 16) router_direct_kernel<2><<<nblk, kRouterThreads, bytes, st>>>(a);
+      else router_direct_kernel<4><<<nblk, kRouterThreads, bytes, st>>>(a);
+      return cudaGetLastError();
+    }
+  }
+  // bf16 with E a multiple of 8: tensor-core gate tile staged through shared memory
+  if (dtype == MOE_DTYPE_BF16 && a.E % 8 == 0 && a.H % 64 == 0 && !router_mma_disabled()) {
+    const MmaRouterPlan P = mma_router_plan(a.E, a.H);
+    cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(router_mma_kernel), P.total);
+    if (err != cudaSuccess) return err;
+    router_mma_kernel<<<nblk, kRouterThreads, P.total, st>>>(a);
+    return cudaGetLastError();
+  }
+  // other small expert counts: the gate is a weight-resident stream over x (HBM bound)
+  if (dtype == MOE_DTYPE_BF16 && a.E <= 16 && a.H % 8 == 0) {
+    const int ep = a.E <= 4 ? 4 : (a.E <= 8 ? 8 : 16);
+    const int bytes = ep == 4 ? StreamSmem<4>::total(a.H) : (ep == 8 ? StreamSmem<8>::total(a.H) : StreamSmem<16>::total(a.H));
+    if (bytes <= 200 * 1024) {
+      if (ep == 4) return launch_stream<4>(a, nblk, st);
+      if (ep == 8) return launch_stream<8>(a, nblk, st);
+      return launch_stream<16>(a, nblk, st);
+    }
+  }
   const int esize = dtype == MOE_DTYPE_BF16 ? 2 : 4;
   const RouterSmem L = router_smem(a.E, esize);
   cudaError_t err;
   if (dtype == MOE_DTYPE_BF16) {
-    err = cudaFuncSetAttribute(router_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+    err = ensure_smem_limit(reinterpret_cast<const void*>(router_kernel<__nv_bfloat16>), L.total);
     if (err != cudaSuccess) return err;
     router_kernel<__nv_bfloat16><<<nblk, kRouterThreads, L.total, st>>>(a);
   } else {
-    err = cudaFuncSetAttribute(router_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, L.total);
+    err = ensure_smem_limit(reinterpret_cast<const void*>(router_kernel<float>), L.total);
     if (err != cudaSuccess) return err;
     router_kernel<float><<<nblk, kRouterThreads, L.total, st>>>(a);
   }
