@@ -45,7 +45,8 @@ constexpr int BK = 64;  // one 128-byte swizzle row of bf16
 constexpr int kEpiWarps = MOE_EPI_WARPS;  // 4 or 8: one or two warps per TMEM lane quarter
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kStgStride = 36;                     // floats per staged row (32 + 4: 16-byte rows, spread banks)
-constexpr int kStgWarpBytes = 32 * kStgStride * 4;  // one warp's 32 x 32 fp32 staging tile
+constexpr int kStgWarpBytes = 5 * 1024;  // one warp's staging tile: 32 x 32 fp32 (padded rows) or a
+                                          // 1024-aligned 32 x 64 bf16 box in 128-byte swizzle
 
 enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2 };
 
@@ -136,6 +137,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
 }
+// TMA store of a shared-memory box to global memory, tracked by this thread's bulk groups
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];\n" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -252,17 +265,7 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
-}
-
 __device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
 
 // tile -> (expert, m tile inside the expert, n tile); prefix[e] = tiles of experts < e
 __device__ __forceinline__ void decode_tile(int tile, const int* prefix, const int* offs, int E, int NT, int& e,
@@ -318,6 +321,61 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t
     for (int i = 0; i < nr; ++i) g.y[(size_t)(grow0 + i) * g.N + n0 + lane] = stg[i * kStgStride + lane] + bj;
   }
   __syncwarp();
+}
+
+// GEMM1 epilogue of a 64-column group of a warp's 32 rows (lane i owns row i): bias + GELU, bf16,
+// written into the warp's staging box in the 128-byte swizzle a TMA store expects (16-byte piece
+// j of row i sits at piece j ^ (i % 8)), then stored with one TMA instruction.  Only used when all
+// 32 rows lie inside the expert's segment, so the box never touches the next expert's rows.
+__device__ __forceinline__ void epilogue_gelu_box(const CUtensorMap* tmC, const uint32_t (&r0)[32],
+                                                  const uint32_t (&r1)[32], uint8_t* stg, int lane,
+                                                  const __nv_bfloat16* brow, int n0, int grow0) {
+  if (lane == 0) bulk_wait_read0();  // the previous box has left the staging buffer
+  __syncwarp();
+  uint8_t* row = stg + lane * 128;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t* src = j < 4 ? &r0[8 * j] : &r1[8 * (j - 4)];
+    const uint4 bb = __ldg(reinterpret_cast<const uint4*>(brow + n0 + 8 * j));
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(b2[u]);
+      const __nv_bfloat162 v =
+          __floats2bfloat162_rn(gelu_erf(__uint_as_float(src[2 * u]) + f.x), gelu_erf(__uint_as_float(src[2 * u + 1]) + f.y));
+      w[u] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  fence_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmC, smem_u32(stg), n0, grow0);
+    bulk_commit();
+  }
+}
+
+// The same values written row by row from registers (rows past the segment are skipped).
+__device__ __forceinline__ void epilogue_gelu_rows(const GemmArgs& g, const uint32_t (&r0)[32], const uint32_t (&r1)[32],
+                                                   int lane, int nrows, const __nv_bfloat16* brow, int n0, int grow0) {
+  if (lane >= nrows) return;
+  uint4* dst = reinterpret_cast<uint4*>(g.h_out + (size_t)(grow0 + lane) * g.N + n0);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t* src = j < 4 ? &r0[8 * j] : &r1[8 * (j - 4)];
+    const uint4 bb = __ldg(reinterpret_cast<const uint4*>(brow + n0 + 8 * j));
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(b2[u]);
+      const __nv_bfloat162 v =
+          __floats2bfloat162_rn(gelu_erf(__uint_as_float(src[2 * u]) + f.x), gelu_erf(__uint_as_float(src[2 * u + 1]) + f.y));
+      w[u] = *reinterpret_cast<const uint32_t*>(&v);
+    }
+    dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 template <int BN, int EPI>
@@ -486,8 +544,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
       const int wrows = rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
-#pragma unroll 1
       constexpr int kChunks = BN / 32 / (kEpiWarps / 4);  // 32-column chunks per epilogue warp
+#pragma unroll 1
       for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
@@ -537,9 +595,9 @@ struct PairCfg {
   static constexpr int kNumBars = 2 * kStages + 4 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kOffsOff = kMiscOff + 16;
-  static constexpr int kStgOff = (kOffsOff + 2 * 260 * 4 + 127) & ~127;
+  static constexpr int kStgOff = (kOffsOff + 2 * 260 * 4 + 1023) & ~1023;
   static constexpr int kSmemBytes = 1024 + kStgOff + kEpiWarps * kStgWarpBytes;
-  static_assert(kStgOff % 16 == 0 && kSmemBytes <= 232448, "shared-memory plan");
+  static_assert(kStgOff % 1024 == 0 && kSmemBytes <= 232448, "shared-memory plan");
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                      ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
 };
@@ -565,7 +623,7 @@ __device__ __forceinline__ void decode_tile_m(int tile, const int* prefix, const
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                             GemmArgs g) {
+                             const __grid_constant__ CUtensorMap tmC, GemmArgs g) {
   using C = PairCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -741,19 +799,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
       const int wrows = my_rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
-#pragma unroll 1
+      const int wrow0 = row0 + BM * (int)rank + quarter * 32;
       constexpr int kChunks = C::kTileN / 32 / (kEpiWarps / 4);
-      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::kTileN + c * 32), r);
-        if (wrows > 0)
-          epilogue_chunk<EPI>(g, r, stg, lane, row0 + BM * (int)rank + quarter * 32, wrows, tok, wgt, brow,
-                              n_idx * C::kTileN + c * 32);
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::kTileN);
+      if (EPI == EPI_GELU) {
+#pragma unroll 1
+        for (int c = half * kChunks; c < (half + 1) * kChunks; c += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(taddr + c * 32, r0);
+          tmem_ld32(taddr + (c + 1) * 32, r1);
+          const int n0 = n_idx * C::kTileN + c * 32;
+          if (wrows >= 32) epilogue_gelu_box(&tmC, r0, r1, reinterpret_cast<uint8_t*>(stg), lane, brow, n0, wrow0);
+          else if (wrows > 0) epilogue_gelu_rows(g, r0, r1, lane, wrows, brow, n0, wrow0);
+        }
+      } else {
+#pragma unroll 1
+        for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          if (wrows > 0) epilogue_chunk<EPI>(g, r, stg, lane, wrow0, wrows, tok, wgt, brow, n_idx * C::kTileN + c * 32);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
     }
+    if (EPI == EPI_GELU && lane == 0) bulk_wait0();  // this warp's h boxes are written before exit
   }
 
   tc_fence_before();
@@ -791,8 +862,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-// CTA-pair tiles are the default for N divisible by 256; MOE_GEMM_PAIR=0 in the environment selects
-// the single-CTA kernel instead (kept for comparison and as the path for other widths).
+// CTA-pair tiles are used for N divisible by 256 and K by 128 when segments are long enough;
+// MOE_GEMM_PAIR=0 in the environment selects the single-CTA kernel everywhere (for comparison).
 bool pair_mode_enabled() {
   static int mode = -1;
   if (mode < 0) {
@@ -813,6 +884,19 @@ bool make_map_a(CUtensorMap* m, const void* base, int rows, int K) {
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// GEMM1 output h: [rows, N] bf16 row-major; stores of 64 columns x 32 rows, 128-byte swizzle
+bool make_map_store(CUtensorMap* m, void* base, int rows, int N) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 // B operand: [E, K, N] bf16 (n contiguous); box = 64 n x 64 k x 1 expert
@@ -838,18 +922,24 @@ cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmA
 }
 
 template <int EPI>
-cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid, cudaStream_t st) {
+cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmArgs& g, int grid,
+                        cudaStream_t st) {
   auto kern = grouped_gemm_pair_kernel<EPI>;
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(kern), PairCfg::kSmemBytes);
   if (err != cudaSuccess) return err;
-  kern<<<grid & ~1, kThreads, PairCfg::kSmemBytes, st>>>(ma, mb, g);
+  kern<<<grid & ~1, kThreads, PairCfg::kSmemBytes, st>>>(ma, mb, mc, g);
   return cudaGetLastError();
 }
 
+// 256-row CTA-pair tiles pay off when experts hold at least a full pair tile on average; with
+// shorter segments (many experts, or few tokens) most of a 256-row tile would be padding, and the
+// 128-row single-CTA tiles waste half as much.  The host sees only the expected rows per expert
+// (T*k/E); the actual counts stay on the device.
 template <int EPI>
-cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid,
-                      cudaStream_t st) {
-  if (N % 256 == 0 && g.K % PairCfg::kStageK == 0 && pair_mode_enabled()) return launch_pair<EPI>(ma, mb, g, grid, st);
+cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmArgs& g,
+                      int grid, long long avg_rows, cudaStream_t st) {
+  if (N % 256 == 0 && g.K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled())
+    return launch_pair<EPI>(ma, mb, mc, g, grid, st);
   if (N % 256 == 0) return launch_one<256, EPI>(ma, mb, g, grid, st);
   if (N % 128 == 0) return launch_one<128, EPI>(ma, mb, g, grid, st);
   return launch_one<64, EPI>(ma, mb, g, grid, st);
@@ -858,9 +948,10 @@ cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const
 }  // namespace
 
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches) {
-  CUtensorMap ma1, mb1, ma2, mb2;
+  CUtensorMap ma1, mb1, ma2, mb2, mc1;
   if (!make_map_a(&ma1, a.x_perm, a.rows_cap, a.H) || !make_map_b(&mb1, a.W1, a.E, a.H, a.F) ||
-      !make_map_a(&ma2, a.h, a.rows_cap, a.F) || !make_map_b(&mb2, a.W2, a.E, a.F, a.H))
+      !make_map_a(&ma2, a.h, a.rows_cap, a.F) || !make_map_b(&mb2, a.W2, a.E, a.F, a.H) ||
+      !make_map_store(&mc1, a.h, a.rows_cap, a.F))
     return cudaErrorInvalidValue;
   const int grid = a.num_sms > 0 ? a.num_sms : 148;
 
@@ -874,7 +965,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.k = a.k;
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
-  cudaError_t err = launch_bn<EPI_GELU>(a.F, ma1, mb1, g1, grid, st);
+  const long long avg_rows = (long long)a.T * a.k / a.E;
+  cudaError_t err = launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st);
   if (err != cudaSuccess) return err;
   ++*launches;
 
@@ -889,9 +981,9 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g2.row_slot = a.row_slot;
   g2.topk_w = a.topk_w;
   if (a.fuse_combine)
-    err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, g2, grid, st);
+    err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st);
   else
-    err = launch_bn<EPI_STORE_Y>(a.H, ma2, mb2, g2, grid, st);
+    err = launch_bn<EPI_STORE_Y>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st);
   if (err != cudaSuccess) return err;
   ++*launches;
   return cudaSuccess;

@@ -332,9 +332,13 @@ __global__ void __launch_bounds__(kRouterThreads) router_stream_kernel(RouterArg
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const __nv_bfloat16* Wg = reinterpret_cast<const __nv_bfloat16*>(a.Wg);
   // stage Wg [H][E] -> padded groups of 8 rows x EP columns (zero for e >= E)
-  if (E == EP && EP >= 8) {
+  bool staged = false;
+  if constexpr (EP >= 8) {
+    staged = E == EP;
+  }
+  if (staged) {
     // whole rows as 16-byte vectors, all loads of a thread issued before its stores
-    constexpr int VPR = EP / 8;  // 16-byte vectors per row
+    constexpr int VPR = EP >= 8 ? EP / 8 : 1;  // 16-byte vectors per row
     const uint4* src = reinterpret_cast<const uint4*>(Wg);
     const int nvec = H * VPR;
     for (int i0 = tid; i0 < nvec; i0 += kRouterThreads * 8) {
@@ -396,7 +400,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_stream_kernel(RouterArg
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float w[EP];
-        if (EP >= 8) {
+        if constexpr (EP >= 8) {
 #pragma unroll
           for (int q = 0; q < EP / 8; ++q) {  // 16-byte reads: conflict-free with the padded groups
             const uint4 wv = *reinterpret_cast<const uint4*>(grp + (j * EP + 8 * q) * 2);
@@ -797,15 +801,32 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
   for (int c = c0; c < c1; ++c) s += a.chunk_hist[(size_t)c * E + e];
   if (in) gsum[g * E + e] = s;
   __syncthreads();
-  if (tid < E) {
-    int run = 0;
-    for (int q = 0; q < G; ++q) {
-      int v = gsum[q * E + tid];
-      gsum[q * E + tid] = run;
-      run += v;
+  // exclusive scan of the G group sums of each expert: warp w scans experts w, w+32, ...; lane l
+  // owns a contiguous run of groups, then a shuffle scan across the lanes (exact integer sums)
+  {
+    const int warp = tid >> 5, lane = tid & 31;
+    const int gpl = (G + 31) / 32;  // groups per lane
+    for (int ee = warp; ee < E; ee += 32) {
+      const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
+      int local = 0;
+      for (int q = q0; q < q1; ++q) local += gsum[q * E + ee];
+      int incl = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int run = incl - local;
+      for (int q = q0; q < q1; ++q) {
+        const int v = gsum[q * E + ee];
+        gsum[q * E + ee] = run;
+        run += v;
+      }
+      if (lane == 31) {
+        cnt_s[ee] = incl;
+        a.cnt_pre[ee] = incl;
+      }
     }
-    cnt_s[tid] = run;
-    a.cnt_pre[tid] = run;
   }
   __syncthreads();
   if (a.do_dispatch && in) {
@@ -851,10 +872,19 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
       for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
       if (tid == 0) zred[0] = z;
     }
-    if (tid < E) {
-      float P = 0.f;
-      for (int q = 0; q < G; ++q) P += pf[q * E + tid];
-      term[tid] = ((double)cnt_s[tid] / ((double)a.T * a.k)) * ((double)P / (double)a.T);
+    // P_e: warp w reduces experts w, w+32, ...: lane l sums its contiguous groups, then a fixed
+    // shuffle tree (the same order on every run)
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      const int gpl = (G + 31) / 32;
+      for (int ee = warp; ee < E; ee += 32) {
+        const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
+        float P = 0.f;
+        for (int q = q0; q < q1; ++q) P += pf[q * E + ee];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) P += __shfl_xor_sync(0xffffffffu, P, o);
+        if (lane == 0) term[ee] = ((double)cnt_s[ee] / ((double)a.T * a.k)) * ((double)P / (double)a.T);
+      }
     }
     __syncthreads();
     if (tid == 0) {

@@ -77,6 +77,8 @@ def _check_against_oracle(cfg, r):
     _cfg("one_token", 1, 64, 4, 2, 64, math.inf, "bf16", 25),
     # segments longer than one 128-row tile and a ragged tail in several experts
     _cfg("long_segments", 1000, 128, 3, 2, 256, math.inf, "bf16", 26),
+    # CTA-pair tiles in both GEMMs (N divisible by 256, K by 128), ragged tails, capacity drops
+    _cfg("pair_tiles", 1500, 256, 4, 2, 512, 1.1, "bf16", 27),
 ], ids=lambda c: c.name)
 def test_small_shapes_end_to_end(cfg):
     r = _run_forward(cfg)
@@ -122,11 +124,12 @@ def test_empty_batch():
     torch.cuda.synchronize()
 
 
-def test_unfused_combine_matches_fused():
+@pytest.mark.parametrize("E", [8, 2])  # 83 rows per expert (single-CTA tiles) / 333 (CTA-pair tiles)
+def test_unfused_combine_matches_fused(E):
     import torch
 
     moe = _lib()
-    cfg = _cfg("unfused", 333, 256, 8, 2, 512, 1.25, "bf16", 34)
+    cfg = _cfg("unfused", 333, 256, E, 2, 512, 1.25, "bf16", 34)
     inp = synth.make_inputs(cfg)
     buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
     buf.forward()
@@ -150,12 +153,12 @@ def test_unfused_combine_matches_fused():
     assert err <= tol
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_deterministic_bitwise(dtype):
+@pytest.mark.parametrize("dtype,E", [("f32", 8), ("bf16", 8), ("bf16", 2)])
+def test_deterministic_bitwise(dtype, E):
     import torch
 
     moe = _lib()
-    cfg = _cfg("det", 512, 128, 8, 2, 256, math.inf, dtype, 35)
+    cfg = _cfg("det", 512, 128, E, 2, 256, math.inf, dtype, 35)
     buf = moe.MoEBuffers(shape_of(cfg), upload(synth.make_inputs(cfg)))
     outs = []
     for _ in range(3):
