@@ -600,6 +600,9 @@ struct PairCfg {
   static_assert(kStgOff % 1024 == 0 && kSmemBytes <= 232448, "shared-memory plan");
   static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
                                      ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+  // half tile (M = 128 over the pair, 64 rows per CTA) for an expert's last <= 128 rows
+  static constexpr uint32_t kIdescHalf = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
+                                         ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)((kTileM / 2) >> 4) << 24);
 };
 
 __device__ __forceinline__ void decode_tile_m(int tile, const int* prefix, const int* offs, int E, int NT, int tile_m,
@@ -689,6 +692,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
         int e, m_local, n_idx, row0, rows;
         decode_tile_m(tile, prefix, offs, E, NT, C::kTileM, e, m_local, n_idx, row0, rows);
+        const int cta_rows = rows <= C::kTileM / 2 ? C::kTileM / 4 : C::kTileM / 2;  // rows per CTA: 64 or 128
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutProducer)) {
             ok = false;
@@ -704,7 +708,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int sk = 0; sk < C::kSubK; ++sk) {
             const int k0 = kb * C::kStageK + sk * BK;
-            tma_load_2d_pair(a_dst + sk * C::kASubBytes, &tmA, k0, row0 + BM * (int)rank, fb);
+            tma_load_2d_pair(a_dst + sk * C::kASubBytes, &tmA, k0, row0 + cta_rows * (int)rank, fb);
 #pragma unroll
             for (int j = 0; j < C::kHalfN / 64; ++j)
               tma_load_3d_pair(b_dst + sk * C::kBSubBytes + j * (BK * 128), &tmB,
@@ -735,6 +739,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int tile = cluster_id; tile < total && ok; tile += nclusters, ++it) {
         const int buf = it & 1;
         const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+        int e_, m_l, n_i, r0_, rows;
+        decode_tile_m(tile, prefix, offs, E, NT, C::kTileM, e_, m_l, n_i, r0_, rows);
+        const uint32_t idesc = rows <= C::kTileM / 2 ? C::kIdescHalf : C::kIdesc;
         if (!mbar_wait(tempty_bar(buf), tphase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutMma)) {
           ok = false;
           break;
@@ -753,7 +760,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < C::kStageK / 16; ++kk) {
             const int sk = kk / (BK / 16), ks = kk % (BK / 16);
             mma_bf16_pair(d_tmem, desc_a_kmajor(a_addr + sk * C::kASubBytes + ks * 32),
-                          desc_b_mnmajor(b_addr + sk * C::kBSubBytes + ks * 16 * 128), C::kIdesc,
+                          desc_b_mnmajor(b_addr + sk * C::kBSubBytes + ks * 16 * 128), idesc,
                           (kb | kk) != 0 ? 1u : 0u);
           }
           issued = true;
@@ -776,7 +783,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (warps 2..5, both) --
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
-    const int r_in_tile = quarter * 32 + lane;
     const uint32_t tempty_leader0 = peer_addr(tempty_bar(0), 0);
     const uint32_t tempty_leader1 = peer_addr(tempty_bar(1), 0);
     int it = 0;
@@ -788,9 +794,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const bool got = mbar_wait(tfull_bar(buf), tphase, g.wait_limit, abort_flag, g.status, kDevTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
-      const int my_rows = rows - BM * (int)rank;  // rows of this tile held by this CTA (may be <= 0)
-      const bool row_ok = r_in_tile < my_rows;
-      const int grow = row0 + BM * (int)rank + r_in_tile;
+      // Full tile: this CTA's 128 rows in TMEM lanes 0..127, 256 columns.  Half tile (M = 128 over the
+      // pair): this CTA's 64 rows x 256 columns sit in 128 TMEM columns, lanes 0..63 holding columns
+      // 0..127 and lanes 64..127 columns 128..255 -- so lane quarter q has rows 32*(q%2).. and
+      // columns 128*(q/2)..
+      const bool hm = rows <= C::kTileM / 2;
+      const int cta_rows = hm ? C::kTileM / 4 : C::kTileM / 2;
+      const int qr = hm ? (quarter & 1) : quarter;  // 32-row block of this warp inside the CTA's rows
+      const int colbase = hm ? (quarter >> 1) * (C::kTileN / 2) : 0;
+      const int my_rows = min(rows - cta_rows * (int)rank, cta_rows);  // may be <= 0
+      const int r_in = qr * 32 + lane;
+      const bool row_ok = r_in < my_rows;
+      const int grow = row0 + cta_rows * (int)rank + r_in;
       float wgt = 0.f;
       int tok = 0;
       if (EPI == EPI_COMBINE && row_ok) {
@@ -798,26 +813,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
       }
       const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
-      const int wrows = my_rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
-      const int wrow0 = row0 + BM * (int)rank + quarter * 32;
-      constexpr int kChunks = C::kTileN / 32 / (kEpiWarps / 4);
+      const int wrows = my_rows - qr * 32;  // rows of this warp's 32 that lie inside the segment
+      const int wrow0 = row0 + cta_rows * (int)rank + qr * 32;
+      const int nch = (hm ? C::kTileN / 64 : C::kTileN / 32) / (kEpiWarps / 4);  // 32-column chunks per warp
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::kTileN);
       if (EPI == EPI_GELU) {
 #pragma unroll 1
-        for (int c = half * kChunks; c < (half + 1) * kChunks; c += 2) {
+        for (int c = half * nch; c < (half + 1) * nch; c += 2) {
           uint32_t r0[32], r1[32];
           tmem_ld32(taddr + c * 32, r0);
           tmem_ld32(taddr + (c + 1) * 32, r1);
-          const int n0 = n_idx * C::kTileN + c * 32;
+          const int n0 = n_idx * C::kTileN + colbase + c * 32;
           if (wrows >= 32) epilogue_gelu_box(&tmC, r0, r1, reinterpret_cast<uint8_t*>(stg), lane, brow, n0, wrow0);
           else if (wrows > 0) epilogue_gelu_rows(g, r0, r1, lane, wrows, brow, n0, wrow0);
         }
       } else {
 #pragma unroll 1
-        for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
+        for (int c = half * nch; c < (half + 1) * nch; ++c) {
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
-          if (wrows > 0) epilogue_chunk<EPI>(g, r, stg, lane, wrow0, wrows, tok, wgt, brow, n_idx * C::kTileN + c * 32);
+          if (wrows > 0)
+            epilogue_chunk<EPI>(g, r, stg, lane, wrow0, wrows, tok, wgt, brow, n_idx * C::kTileN + colbase + c * 32);
         }
       }
       tc_fence_before();

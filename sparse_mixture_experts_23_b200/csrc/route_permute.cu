@@ -930,11 +930,12 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* pv = reinterpret_cast<uint4*>(a.x_perm);
   const int total = kChunk * nvec;
-  for (int i = tid; i < total; i += 256 * 4) {
-    uint4 v[4];
-    int rr[4];
+  constexpr int U = 8;  // 16-byte loads in flight per thread
+  for (int i = tid; i < total; i += 256 * U) {
+    uint4 v[U];
+    int rr[U];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
       int idx = i + u * 256;
       rr[u] = -1;
       if (idx < total) {
@@ -947,7 +948,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < U; ++u) {
       if (rr[u] >= 0) {
         int idx = rr[u];
         int r = idx / nvec, c = idx % nvec;
