@@ -34,6 +34,7 @@ _lib = None
 
 F32, BF16 = 0, 1
 _DT = {"f32": F32, "bf16": BF16}
+ACT = {"gelu": 0, "silu": 1}
 
 
 def build(force: bool = False) -> str:
@@ -53,6 +54,8 @@ def _load():
     i64, vp, c_int, dbl = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_double
     lib.oracle_gelu.argtypes = [dbl]
     lib.oracle_gelu.restype = dbl
+    lib.oracle_silu.argtypes = [dbl]
+    lib.oracle_silu.restype = dbl
     lib.oracle_capacity.argtypes = [dbl, i64, i64, i64]
     lib.oracle_capacity.restype = i64
     lib.oracle_route.argtypes = [i64, i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -61,10 +64,10 @@ def _load():
     lib.oracle_losses.restype = None
     lib.oracle_dispatch.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.oracle_dispatch.restype = i64
-    lib.oracle_expert_rows.argtypes = [i64, i64, c_int, vp, vp, vp, vp, vp, i64, vp, vp, vp, c_int]
+    lib.oracle_expert_rows.argtypes = [i64, i64, c_int, c_int, vp, vp, vp, vp, vp, i64, vp, vp, vp, c_int]
     lib.oracle_expert_rows.restype = None
-    lib.oracle_forward_tokens.argtypes = [i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp,
-                                          c_int]
+    lib.oracle_forward_tokens.argtypes = [i64, i64, i64, c_int, c_int, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp,
+                                          vp, c_int]
     lib.oracle_forward_tokens.restype = None
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
@@ -95,6 +98,15 @@ def gelu(u: float) -> float:
     return _load().oracle_gelu(float(u))
 
 
+def silu(u: float) -> float:
+    return _load().oracle_silu(float(u))
+
+
+def _opt(a):
+    """Optional bias: None stays None (NULL pointer, i.e. zeros)."""
+    return None if a is None else _c(a)
+
+
 def capacity(cf: float, T: int, k: int, E: int):
     """Per-expert capacity, or None when unlimited (CF = +inf)."""
     c = _load().oracle_capacity(float(cf), T, k, E)
@@ -112,7 +124,7 @@ class Routing:
 
 
 def route(x, Wg, bg, k: int, dtype: str) -> Routing:
-    x, Wg, bg = _c(x), _c(Wg), _c(bg)
+    x, Wg, bg = _c(x), _c(Wg), _opt(bg)
     T, H = x.shape
     E = Wg.shape[1]
     logits = np.empty((T, E), np.float64)
@@ -169,22 +181,22 @@ def dispatch(topk_idx, E: int, cf: float) -> Dispatch:
                     row_slot[:kept].copy())
 
 
-def expert_rows(x, W1, b1, W2, b2, tokens, experts, dtype: str, nthreads: int = 0) -> np.ndarray:
-    """y[i] = FFN_{experts[i]}(x[tokens[i]]) in double."""
-    x, W1, b1, W2, b2 = _c(x), _c(W1), _c(b1), _c(W2), _c(b2)
+def expert_rows(x, W1, b1, W2, b2, tokens, experts, dtype: str, nthreads: int = 0, act: str = "gelu") -> np.ndarray:
+    """y[i] = FFN_{experts[i]}(x[tokens[i]]) in double; b1/b2 may be None (no bias)."""
+    x, W1, b1, W2, b2 = _c(x), _c(W1), _opt(b1), _c(W2), _opt(b2)
     tokens, experts = _c(tokens, np.int32), _c(experts, np.int32)
     E, H, F = W1.shape
     n = tokens.shape[0]
     y = np.empty((n, H), np.float64)
-    _load().oracle_expert_rows(H, F, _DT[dtype], _p(x), _p(W1), _p(b1), _p(W2), _p(b2), n, _p(tokens),
+    _load().oracle_expert_rows(H, F, _DT[dtype], ACT[act], _p(x), _p(W1), _p(b1), _p(W2), _p(b2), n, _p(tokens),
                                _p(experts), _p(y), int(nthreads))
     return y
 
 
 def forward_tokens(x, W1, b1, W2, b2, topk_idx, topk_w, dropped, tokens, dtype: str,
-                   nthreads: int = 0) -> np.ndarray:
+                   nthreads: int = 0, act: str = "gelu") -> np.ndarray:
     """out[i] = sum over kept slots of w * FFN(x[tokens[i]]) in double, for the listed tokens."""
-    x, W1, b1, W2, b2 = _c(x), _c(W1), _c(b1), _c(W2), _c(b2)
+    x, W1, b1, W2, b2 = _c(x), _c(W1), _opt(b1), _c(W2), _opt(b2)
     idx, w = _c(topk_idx, np.int32), _c(topk_w, np.float64)
     drp = None if dropped is None else _c(dropped, np.uint8)
     tokens = _c(tokens, np.int32)
@@ -192,8 +204,8 @@ def forward_tokens(x, W1, b1, W2, b2, topk_idx, topk_w, dropped, tokens, dtype: 
     k = idx.shape[1]
     n = tokens.shape[0]
     out = np.empty((n, H), np.float64)
-    _load().oracle_forward_tokens(H, F, k, _DT[dtype], _p(x), _p(W1), _p(b1), _p(W2), _p(b2), _p(idx), _p(w),
-                                  _p(drp), n, _p(tokens), _p(out), int(nthreads))
+    _load().oracle_forward_tokens(H, F, k, _DT[dtype], ACT[act], _p(x), _p(W1), _p(b1), _p(W2), _p(b2), _p(idx),
+                                  _p(w), _p(drp), n, _p(tokens), _p(out), int(nthreads))
     return out
 
 
@@ -207,12 +219,13 @@ class Forward:
     tokens: np.ndarray
 
 
-def forward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=None, nthreads: int = 0) -> Forward:
+def forward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=None, nthreads: int = 0,
+            act: str = "gelu") -> Forward:
     """Whole layer: routing and dispatch over all tokens, FFN + combine for ``tokens`` (default: all)."""
     r = route(x, Wg, bg, k, dtype)
     aux, z = losses(r.p, r.lse, r.topk_idx)
     d = dispatch(r.topk_idx, Wg.shape[1], cf)
     T = x.shape[0]
     tokens = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
-    out = forward_tokens(x, W1, b1, W2, b2, r.topk_idx, r.topk_w, d.dropped, tokens, dtype, nthreads)
+    out = forward_tokens(x, W1, b1, W2, b2, r.topk_idx, r.topk_w, d.dropped, tokens, dtype, nthreads, act)
     return Forward(r, aux, z, d, out, tokens)

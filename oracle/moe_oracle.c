@@ -33,7 +33,8 @@
  *    assignment is kept iff its rank among earlier assignments to the same expert is < capacity,
  *    and that rank is also its row inside the expert's segment of the permuted buffer;
  *  - a dropped assignment contributes nothing and the kept weights are not renormalised again;
- *  - GELU is the exact erf form 0.5*u*(1 + erf(u/sqrt(2))) (nn.GELU() default);
+ *  - GELU is the exact erf form 0.5*u*(1 + erf(u/sqrt(2))) (nn.GELU() default); the Mixtral block's
+ *    variant uses SiLU u*sigmoid(u) and bias-free Linear layers (a NULL bias pointer means zeros);
  *  - for T = 0 both losses are defined as 0.
  *
  * Inputs are passed in their storage type (fp32 or bf16 bit patterns) and widened to double element
@@ -61,6 +62,15 @@ static double load(const void* base, int dtype, size_t i) {
 
 /* GELU, exact erf form (nn.GELU() default) -- [SKILL] Quick Start expert FFN */
 double oracle_gelu(double u) { return 0.5 * u * (1.0 + erf(u / sqrt(2.0))); }
+
+/* SiLU, u * sigmoid(u) (nn.SiLU()) -- [SKILL] Advanced Patterns, "Mixtral 8x7B Architecture" experts */
+double oracle_silu(double u) { return u / (1.0 + exp(-u)); }
+
+enum { ORACLE_ACT_GELU = 0, ORACLE_ACT_SILU = 1 };
+static double activation(int act, double u) { return act == ORACLE_ACT_SILU ? oracle_silu(u) : oracle_gelu(u); }
+
+/* a bias pointer may be NULL: the Mixtral block's Linear layers have bias=False */
+static double load_bias(const void* base, int dtype, size_t i) { return base ? load(base, dtype, i) : 0.0; }
 
 /* capacity of one expert: ceil(CF * T * k / E), or -1 for "unlimited" (CF = +inf).
  * [SKILL] Core Concepts 4 / Best Practices 2; the k factor and the ceiling follow the workload
@@ -93,7 +103,7 @@ void oracle_route(int64_t T, int64_t H, int64_t E, int64_t k, int dtype, const v
 #pragma omp for schedule(static)
     for (int64_t t = 0; t < T; ++t) {
       for (int64_t e = 0; e < E; ++e) {
-        double acc = load(bg, dtype, (size_t)e);
+        double acc = load_bias(bg, dtype, (size_t)e);
         for (int64_t h = 0; h < H; ++h) acc += load(x, dtype, (size_t)(t * H + h)) * load(Wg, dtype, (size_t)(h * E + e));
         logit[e] = acc;
       }
@@ -221,22 +231,23 @@ int64_t oracle_dispatch(int64_t T, int64_t E, int64_t k, int64_t cap, const int3
 }
 
 /*
- * One expert's FFN on one input row -- [SKILL] Quick Start expert: Linear(H, F) -> GELU -> Linear(F, H).
- *   u[f] = b1[e,f] + sum_h xrow[h] * W1[e,h,f]
- *   g[f] = GELU(u[f])
- *   y[h] = b2[e,h] + sum_f g[f] * W2[e,f,h]
+ * One expert's FFN on one input row -- [SKILL] Quick Start expert: Linear(H, F) -> GELU -> Linear(F, H);
+ * Advanced Patterns, Mixtral block: Linear(H, F, bias=False) -> SiLU -> Linear(F, H, bias=False).
+ *   u[f] = b1[e,f] + sum_h xrow[h] * W1[e,h,f]        (b1 = 0 when absent)
+ *   g[f] = act(u[f])                                   (GELU or SiLU)
+ *   y[h] = b2[e,h] + sum_f g[f] * W2[e,f,h]            (b2 = 0 when absent)
  * xrow is already double; u is scratch of length F.
  */
-static void expert_ffn_row(int64_t H, int64_t F, int dtype, const double* xrow, int32_t e, const void* W1,
+static void expert_ffn_row(int64_t H, int64_t F, int dtype, int act, const double* xrow, int32_t e, const void* W1,
                            const void* b1, const void* W2, const void* b2, double* u, double* y) {
-  for (int64_t f = 0; f < F; ++f) u[f] = load(b1, dtype, (size_t)(e * F + f));
+  for (int64_t f = 0; f < F; ++f) u[f] = load_bias(b1, dtype, (size_t)(e * F + f));
   for (int64_t h = 0; h < H; ++h) {
     double xh = xrow[h];
     size_t base = (size_t)((e * H + h) * F);
     for (int64_t f = 0; f < F; ++f) u[f] += xh * load(W1, dtype, base + (size_t)f);
   }
-  for (int64_t f = 0; f < F; ++f) u[f] = oracle_gelu(u[f]);
-  for (int64_t h = 0; h < H; ++h) y[h] = load(b2, dtype, (size_t)(e * H + h));
+  for (int64_t f = 0; f < F; ++f) u[f] = activation(act, u[f]);
+  for (int64_t h = 0; h < H; ++h) y[h] = load_bias(b2, dtype, (size_t)(e * H + h));
   for (int64_t f = 0; f < F; ++f) {
     double gf = u[f];
     size_t base = (size_t)((e * F + f) * H);
@@ -248,7 +259,7 @@ static void expert_ffn_row(int64_t H, int64_t F, int dtype, const double* xrow, 
  * Expert FFN for a list of (token, expert) pairs: y[i,:] = FFN_{experts[i]}(x[tokens[i],:]).
  * Used to check the grouped GEMM stage on its own, fed any dispatch.
  */
-void oracle_expert_rows(int64_t H, int64_t F, int dtype, const void* x, const void* W1, const void* b1,
+void oracle_expert_rows(int64_t H, int64_t F, int dtype, int act, const void* x, const void* W1, const void* b1,
                         const void* W2, const void* b2, int64_t n, const int32_t* tokens, const int32_t* experts,
                         double* y, int nthreads) {
 #ifdef _OPENMP
@@ -261,7 +272,7 @@ void oracle_expert_rows(int64_t H, int64_t F, int dtype, const void* x, const vo
 #pragma omp for schedule(dynamic, 1)
     for (int64_t i = 0; i < n; ++i) {
       for (int64_t h = 0; h < H; ++h) xrow[h] = load(x, dtype, (size_t)(tokens[i] * H + h));
-      expert_ffn_row(H, F, dtype, xrow, experts[i], W1, b1, W2, b2, u, y + i * H);
+      expert_ffn_row(H, F, dtype, act, xrow, experts[i], W1, b1, W2, b2, u, y + i * H);
     }
     free(xrow);
     free(u);
@@ -274,7 +285,7 @@ void oracle_expert_rows(int64_t H, int64_t F, int dtype, const void* x, const vo
  *   out[t,:] = sum over kept slots s (slot order) of topk_w[t,s] * FFN_{topk_idx[t,s]}(x[t,:])
  * A token whose every slot was dropped gets zeros.
  */
-void oracle_forward_tokens(int64_t H, int64_t F, int64_t k, int dtype, const void* x, const void* W1,
+void oracle_forward_tokens(int64_t H, int64_t F, int64_t k, int dtype, int act, const void* x, const void* W1,
                            const void* b1, const void* W2, const void* b2, const int32_t* topk_idx,
                            const double* topk_w, const uint8_t* dropped, int64_t n, const int32_t* tokens,
                            double* out, int nthreads) {
@@ -294,7 +305,7 @@ void oracle_forward_tokens(int64_t H, int64_t F, int64_t k, int dtype, const voi
       for (int64_t h = 0; h < H; ++h) xrow[h] = load(x, dtype, (size_t)(t * H + h));
       for (int64_t s = 0; s < k; ++s) {
         if (dropped && dropped[t * k + s]) continue;
-        expert_ffn_row(H, F, dtype, xrow, topk_idx[t * k + s], W1, b1, W2, b2, u, y);
+        expert_ffn_row(H, F, dtype, act, xrow, topk_idx[t * k + s], W1, b1, W2, b2, u, y);
         double w = topk_w[t * k + s];
         for (int64_t h = 0; h < H; ++h) o[h] += w * y[h];
       }

@@ -52,6 +52,25 @@ def test_gelu_matches_normal_cdf():
         assert oracle.gelu(u) == pytest.approx(u * stats.norm.cdf(u), rel=1e-14, abs=1e-15)
 
 
+# ---------------------------------------------------------------- SiLU ---------------------------
+
+def test_silu_textbook_values():
+    # SiLU(u) = u * sigmoid(u); sigmoid(1) = e/(1+e), sigmoid(2) = 1/(1+e^-2)
+    assert oracle.silu(0.0) == 0.0
+    assert oracle.silu(1.0) == pytest.approx(math.e / (1 + math.e), abs=1e-15)
+    assert oracle.silu(2.0) == pytest.approx(2 / (1 + math.exp(-2.0)), abs=1e-15)
+    assert oracle.silu(-1.0) == pytest.approx(-1 / (1 + math.e), abs=1e-15)
+    assert oracle.silu(40.0) == pytest.approx(40.0, rel=1e-16)
+    assert oracle.silu(-40.0) == pytest.approx(-40.0 * math.exp(-40.0), rel=1e-12)
+
+
+def test_silu_matches_expit_and_odd_part():
+    for u in np.linspace(-12, 12, 241):
+        assert oracle.silu(u) == pytest.approx(u * special.expit(u), rel=1e-14, abs=1e-300)
+        # sigmoid(u) + sigmoid(-u) = 1  =>  SiLU(u) - SiLU(-u) = u
+        assert oracle.silu(u) - oracle.silu(-u) == pytest.approx(u, abs=1e-14)
+
+
 # ---------------------------------------------------------------- router -------------------------
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
@@ -274,6 +293,50 @@ def test_expert_rows_vs_numpy_matmul(dtype):
         g = u * stats.norm.cdf(u)
         ref = g @ W2[e] + b2[e]
         np.testing.assert_allclose(y[i], ref, rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_expert_rows_silu_bias_free_vs_numpy_matmul(dtype):
+    """Mixtral block expert: Linear(bias=False) -> SiLU -> Linear(bias=False); None biases are zeros."""
+    inp = _rand_layer(T=11, H=24, E=3, F=40, seed=33, dtype=dtype)
+    tokens = np.array([1, 4, 9, 4, 0, 10], np.int32)
+    experts = np.array([0, 2, 1, 0, 2, 1], np.int32)
+    y = oracle.expert_rows(inp.x, inp.W1, None, inp.W2, None, tokens, experts, dtype, act="silu")
+    x, W1, W2 = (_f64(a, dtype) for a in (inp.x, inp.W1, inp.W2))
+    for i, (t, e) in enumerate(zip(tokens, experts)):
+        u = x[t] @ W1[e]
+        ref = (u * special.expit(u)) @ W2[e]
+        np.testing.assert_allclose(y[i], ref, rtol=1e-12, atol=1e-13)
+    # with the biases present the result changes (they are not silently ignored) ...
+    yb = oracle.expert_rows(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, tokens, experts, dtype, act="silu")
+    assert not np.allclose(yb, y)
+    # ... and the activation selector is honoured
+    yg = oracle.expert_rows(inp.x, inp.W1, None, inp.W2, None, tokens, experts, dtype, act="gelu")
+    assert not np.allclose(yg, y)
+
+
+def test_route_without_gate_bias_equals_zero_bias():
+    inp = _rand_layer(T=29, H=16, E=8, F=8, seed=37)
+    a = oracle.route(inp.x, inp.Wg, None, 2, "f32")
+    b = oracle.route(inp.x, inp.Wg, np.zeros(8, np.float32), 2, "f32")
+    np.testing.assert_array_equal(a.logits, b.logits)
+    np.testing.assert_array_equal(a.topk_idx, b.topk_idx)
+    np.testing.assert_allclose(a.logits, inp.x.astype(np.float64) @ inp.Wg.astype(np.float64), rtol=1e-13,
+                               atol=1e-14)
+
+
+def test_mixtral_block_k_equals_E_is_dense_softmax_silu_mixture():
+    """Bias-free gate and SiLU experts with k = E: out = sum_e softmax(x Wg)_e * FFN_e(x)."""
+    T, H, E, F = 17, 12, 4, 20
+    inp = _rand_layer(T=T, H=H, E=E, F=F, seed=45)
+    f = oracle.forward(inp.x, inp.Wg, None, inp.W1, None, inp.W2, None, E, math.inf, "f32", act="silu")
+    x = inp.x.astype(np.float64)
+    p = special.softmax(x @ inp.Wg.astype(np.float64), axis=1)
+    ref = np.zeros((T, H))
+    for e in range(E):
+        u = x @ inp.W1[e].astype(np.float64)
+        ref += p[:, e:e + 1] * ((u * special.expit(u)) @ inp.W2[e].astype(np.float64))
+    np.testing.assert_allclose(f.out, ref, rtol=1e-11, atol=1e-12)
 
 
 def test_identical_experts_equal_dense_ffn():
