@@ -38,7 +38,8 @@ METRIC = "MoE-layer fwd tokens/sec (Mixtral shape, 1 B200); grouped-GEMM % of BF
 
 def workload_config(cfg: synth.LayerConfig) -> str:
     cf = "dropless" if math.isinf(cfg.CF) else f"CF={cfg.CF}"
-    return (f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} F={cfg.F} {cf}, GELU FFN with biases, "
+    ffn = f"{cfg.act.upper()} FFN " + ("with biases" if cfg.bias else "without biases")
+    return (f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} F={cfg.F} {cf}, {ffn}, "
             f"{cfg.dtype} storage / fp32 accumulate")
 
 
@@ -49,7 +50,7 @@ def alg_flops(cfg: synth.LayerConfig, kept: int) -> float:
 
 def alg_bytes(cfg: synth.LayerConfig, touched_experts: int) -> float:
     es = 2 if cfg.dtype == "bf16" else 4
-    w = touched_experts * (2 * cfg.H * cfg.F + cfg.F + cfg.H) * es
+    w = touched_experts * (2 * cfg.H * cfg.F + (cfg.F + cfg.H if cfg.bias else 0)) * es
     return w + cfg.T * cfg.H * es + cfg.T * cfg.H * 4 + cfg.H * cfg.E * es
 
 
@@ -176,7 +177,7 @@ def cpu_oracle_rate(cfg: synth.LayerConfig, inp: synth.LayerInputs, budget_s: fl
     spent = 0.0
     while True:
         t0 = time.perf_counter()
-        oracle.forward(inp.x[:n], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+        oracle.forward(inp.x[:n], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
         dt = time.perf_counter() - t0
         spent += dt
         best = (n, dt)
@@ -200,16 +201,16 @@ def run_reference(args, cfg):
     threads = oracle.max_threads()
     # calibrate tokens per step so the whole run stays within about two minutes
     t0 = time.perf_counter()
-    oracle.forward(inp.x[:1], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+    oracle.forward(inp.x[:1], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
     t1 = time.perf_counter() - t0
     per_step = 120.0 / max(1, args.steps + args.warmup)
     S = int(max(1, min(cfg.T, per_step / max(t1, 1e-6))))
     for _ in range(args.warmup):
-        oracle.forward(inp.x[:S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+        oracle.forward(inp.x[:S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
     t0 = time.perf_counter()
     for i in range(args.steps):
         lo = (i * S) % max(1, cfg.T - S + 1)
-        oracle.forward(inp.x[lo:lo + S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype)
+        oracle.forward(inp.x[lo:lo + S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
     dt = time.perf_counter() - t0
     value = S * args.steps / dt
     line = {
@@ -255,7 +256,7 @@ def run_ours_impl(args, cfg):
 
     inp = replica_inputs(cfg, rank)
     dev = {n: _upload(a, cfg.dtype) for n, a in inp.arrays().items()}
-    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype)
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype, cfg.act)
     buf = moe.MoEBuffers(shape, dev)
     stream = torch.cuda.current_stream()
     peaks = load_peaks()

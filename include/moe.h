@@ -11,7 +11,8 @@
  *                   into expert-contiguous segments                        (Core Concepts 4;
  *                                                                           Best Practices 2)
  *   moe_expert_ffn  per-expert Linear(H,F) -> GELU -> Linear(F,H) as two grouped GEMMs
- *                   (Quick Start expert FFN), optionally with the weighted combine fused in
+ *                   (Quick Start expert FFN), optionally with the weighted combine fused in;
+ *                   SiLU and bias-free Linear layers for the Mixtral block's experts
  *   moe_combine     out[t] = sum over kept slots of w[t,s] * y[row(t,s)]     (Quick Start
  *                                                          "output[mask] += score * output";
  *                                                          Mixtral block index_add_)
@@ -22,13 +23,16 @@
  *    owned by the caller; the library never allocates device memory and never frees it.
  *  - Storage dtype (moe_shape_t.dtype) applies to x, Wg, bg, W1, b1, W2, b2: MOE_DTYPE_F32 or
  *    MOE_DTYPE_BF16.  Accumulation is fp32 everywhere.  out, topk_w and the losses are fp32.
+ *  - The biases bg, b1 and b2 are optional: a NULL pointer means the Linear layer has no bias
+ *    (the Mixtral block's gate and experts are Linear(..., bias=False)), computed as a zero bias.
  *  - All work is asynchronous on the given stream (0 = legacy default stream).  No entry point
  *    synchronises except moe_get_device_status.
  *  - Arguments are validated on the host before anything is launched:
  *      MOE_ERR_INVALID_ARG  null shape/io/workspace pointer, a needed io pointer that is null, a
  *                           device pointer of x/Wg/W1/W2/out/workspace not 16-byte aligned,
  *                           T < 0, H/E/F/k <= 0, k > E, k > 8, E > 256, capacity_factor <= 0 or
- *                           NaN, unknown dtype
+ *                           NaN, unknown dtype or activation, a non-null b1/b2 not 16-byte
+ *                           aligned
  *      MOE_ERR_UNSUPPORTED  bf16 with H or F not a multiple of 64; f32 with H or F not a multiple
  *                           of 4; T*k*max(H,F) beyond 2^31 elements
  *      MOE_ERR_WORKSPACE    ws_bytes < moe_workspace_size(shape)
@@ -74,6 +78,10 @@ typedef enum {
 
 typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 
+/* Activation between the two expert Linear layers.  GELU is the exact erf form (Quick Start
+ * expert, nn.GELU()); SiLU is u * sigmoid(u) (Advanced Patterns, Mixtral block experts). */
+typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SILU = 1 } moe_activation_t;
+
 /* Problem statement.  capacity_factor = +INFINITY means dropless.  Per-expert capacity is
  * ceil(capacity_factor * T * k / E) evaluated in double ("MoE Training" page, Core Concepts 4 and
  * Best Practices 2 give capacity = tokens * CF / E; k counts the assignments of top-k routing). */
@@ -85,10 +93,12 @@ typedef struct {
   int32_t k;              /* experts per token, 1..min(E, 8) */
   double capacity_factor; /* > 0; +INFINITY = no capacity limit */
   moe_dtype_t dtype;      /* storage type of x and all weights */
+  moe_activation_t activation; /* expert activation; a zero-initialised shape gets GELU */
 } moe_shape_t;
 
 /* Caller-owned device buffers.  Layouts (row-major):
- *   x[T,H] Wg[H,E] bg[E] W1[E,H,F] b1[E,F] W2[E,F,H] b2[E,H]       storage dtype, read only
+ *   x[T,H] Wg[H,E] bg[E] W1[E,H,F] b1[E,F] W2[E,F,H] b2[E,H]       storage dtype, read only;
+ *                                                                  bg, b1, b2 may be NULL
  *   out[T,H]           fp32  layer output
  *   topk_idx[T,k]      int32 chosen experts, slot s = rank s by (logit desc, expert index asc)
  *   topk_w[T,k]        fp32  softmax probabilities of the chosen experts divided by their sum
@@ -122,7 +132,7 @@ typedef struct {
   int32_t* row_token;  /* [T*k] token of each row (rows >= offsets[E] unused) */
   int32_t* row_slot;   /* [T*k] slot of each row */
   void* x_perm;        /* [T*k, H] storage dtype: x rows grouped by expert, (slot, token) order */
-  void* h;             /* [T*k, F] storage dtype: GELU(x_perm . W1[e] + b1[e]) */
+  void* h;             /* [T*k, F] storage dtype: act(x_perm . W1[e] + b1[e]) */
   float* y;            /* [T*k, H] fp32: h . W2[e] + b2[e] (only written when the combine is not fused) */
   size_t bytes;        /* total workspace size */
 } moe_ws_view_t;

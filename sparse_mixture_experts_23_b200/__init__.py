@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
 MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 DTYPES = {"f32": MOE_DTYPE_F32, "bf16": MOE_DTYPE_BF16}
+MOE_ACT_GELU, MOE_ACT_SILU = 0, 1
+ACTIVATIONS = {"gelu": MOE_ACT_GELU, "silu": MOE_ACT_SILU}
 
 ENTRY_POINTS = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
@@ -33,7 +35,8 @@ class MoEError(RuntimeError):
 
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32), ("F", ctypes.c_int32),
-                ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_double), ("dtype", ctypes.c_int)]
+                ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_double), ("dtype", ctypes.c_int),
+                ("activation", ctypes.c_int)]
 
 
 class IO(ctypes.Structure):
@@ -90,8 +93,9 @@ def status_string(status: int) -> str:
     return load_library().moe_status_string(status).decode()
 
 
-def make_shape(T: int, H: int, E: int, k: int, F: int, capacity_factor: float = math.inf, dtype: str = "bf16") -> Shape:
-    return Shape(T, H, E, F, k, float(capacity_factor), DTYPES[dtype])
+def make_shape(T: int, H: int, E: int, k: int, F: int, capacity_factor: float = math.inf, dtype: str = "bf16",
+               activation: str = "gelu") -> Shape:
+    return Shape(T, H, E, F, k, float(capacity_factor), DTYPES[dtype], ACTIVATIONS[activation])
 
 
 def _check(status: int, where: str) -> int:
@@ -161,7 +165,8 @@ class MoEBuffers:
     """Device buffers of one layer invocation, allocated with PyTorch (plumbing only).
 
     ``inputs`` maps x, Wg, bg, W1, b1, W2, b2 to device tensors of the storage dtype (bf16 as
-    torch.bfloat16, f32 as torch.float32).  Outputs and the workspace are allocated here.
+    torch.bfloat16, f32 as torch.float32); a bias that is missing or None is passed as NULL (no
+    bias).  Outputs and the workspace are allocated here.
     """
 
     def __init__(self, shape: Shape, inputs: dict, device="cuda"):

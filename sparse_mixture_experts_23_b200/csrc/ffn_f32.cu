@@ -2,7 +2,8 @@
 //
 // Expert ("MoE Training: Mixture of Experts" page, Quick Start: Linear(H, 4H) -> GELU ->
 // Linear(4H, H)) applied to every expert segment of the permuted rows:
-//   GEMM1: h[r,:] = GELU(x_perm[r,:] . W1[e] + b1[e])                (GELU exact erf form)
+//   GEMM1: h[r,:] = act(x_perm[r,:] . W1[e] + b1[e])   (GELU exact erf form, or SiLU for the
+//          Mixtral block's experts; a null b1 / b2 is a zero bias)
 //   GEMM2: fused   out[token(r),:] += w(r) * (h[r,:] . W2[e] + b2[e])
 //          unfused y[r,:]           =          h[r,:] . W2[e] + b2[e]
 // One block computes a 64x64 tile of one expert segment; the tile -> (expert, row block) map
@@ -17,9 +18,11 @@ namespace {
 
 constexpr int BM = 64, BN = 64, BK = 16;
 
-enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2 };
+enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2, EPI_SILU = 3 };
 
 __device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
+// u * sigmoid(u) with the accurate exponential and an IEEE divide (fp32 path)
+__device__ __forceinline__ float silu(float u) { return u / (1.f + expf(-u)); }
 
 template <int EPI>
 __global__ void __launch_bounds__(256) ffn_f32_kernel(FfnArgs a, const float* __restrict__ A, const float* __restrict__ W,
@@ -98,9 +101,11 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(FfnArgs a, const float* __
     for (int j = 0; j < 4; ++j) {
       int n = n0 + tx * 4 + j;
       if (n >= N) continue;
-      float v = acc[i][j] + bias[(size_t)e * N + n];
+      float v = acc[i][j] + (bias ? bias[(size_t)e * N + n] : 0.f);
       if (EPI == EPI_GELU) {
         reinterpret_cast<float*>(a.h)[(size_t)grow * N + n] = gelu_erf(v);
+      } else if (EPI == EPI_SILU) {
+        reinterpret_cast<float*>(a.h)[(size_t)grow * N + n] = silu(v);
       } else if (EPI == EPI_COMBINE) {
         atomicAdd(&a.out[(size_t)tok * N + n], w * v);
       } else {
@@ -117,9 +122,9 @@ cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t st, int* launches) {
   const int mt_max = (a.rows_cap + BM - 1) / BM + a.E;
   {
     dim3 grid(mt_max, (a.F + BN - 1) / BN);
-    ffn_f32_kernel<EPI_GELU><<<grid, 256, 0, st>>>(a, reinterpret_cast<const float*>(a.x_perm),
-                                                   reinterpret_cast<const float*>(a.W1),
-                                                   reinterpret_cast<const float*>(a.b1), a.F, a.H);
+    auto kern = a.act == MOE_ACT_SILU ? ffn_f32_kernel<EPI_SILU> : ffn_f32_kernel<EPI_GELU>;
+    kern<<<grid, 256, 0, st>>>(a, reinterpret_cast<const float*>(a.x_perm), reinterpret_cast<const float*>(a.W1),
+                               reinterpret_cast<const float*>(a.b1), a.F, a.H);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     ++*launches;

@@ -5,6 +5,7 @@
 // scale by the routing weight, index_add_ back to token order) over variable-length expert
 // segments of the permuted rows:
 //   GEMM1 (EPI_GELU):     h[r, n]   = bf16( GELU( sum_k x_perm[r,k] W1[e,k,n] + b1[e,n] ) )
+//   GEMM1 (EPI_SILU):     the same with SiLU (Mixtral block experts); b1 and b2 may be absent (zero)
 //   GEMM2 (EPI_COMBINE):  out[t, n] += w(t,s) * ( sum_k h[r,k] W2[e,k,n] + b2[e,n] ),  t,s = row r's
 //   GEMM2 (EPI_STORE_Y):  y[r, n]   = sum_k h[r,k] W2[e,k,n] + b2[e,n]
 //
@@ -48,7 +49,9 @@ constexpr int kStgStride = 36;                     // floats per staged row (32 
 constexpr int kStgWarpBytes = 5 * 1024;  // one warp's staging tile: 32 x 32 fp32 (padded rows) or a
                                           // 1024-aligned 32 x 64 bf16 box in 128-byte swizzle
 
-enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2 };
+enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2, EPI_SILU = 3 };
+// GEMM1 epilogues write h = act(acc + b1); GEMM2 epilogues combine or store y.
+__host__ __device__ constexpr bool epi_h(int epi) { return epi == EPI_GELU || epi == EPI_SILU; }
 
 template <int BN>
 struct Cfg {
@@ -266,6 +269,17 @@ __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
 }
 
 __device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
+// u * sigmoid(u); for u < -87 the fast divide returns 0 where the exact value is below 1e-35
+__device__ __forceinline__ float silu(float u) { return __fdividef(u, 1.f + __expf(-u)); }
+template <int EPI>
+__device__ __forceinline__ float act(float u) {
+  if constexpr (EPI == EPI_SILU) return silu(u);
+  else return gelu_erf(u);
+}
+// 8 bias values at brow[n0 .. n0+8) as 4 bf16 pairs, zeros when the layer has no bias
+__device__ __forceinline__ uint4 bias8(const __nv_bfloat16* brow, int n0) {
+  return brow ? __ldg(reinterpret_cast<const uint4*>(brow + n0)) : make_uint4(0u, 0u, 0u, 0u);
+}
 
 // tile -> (expert, m tile inside the expert, n tile); prefix[e] = tiles of experts < e
 __device__ __forceinline__ void decode_tile(int tile, const int* prefix, const int* offs, int E, int NT, int& e,
@@ -289,7 +303,7 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, const i
 // Epilogue of one 32 x 32 accumulator chunk of a warp (lane i holds row i of the chunk in r[]).
 // The chunk goes through the warp's shared staging tile so that, after the transpose, lane j owns
 // column j and every global store or reduction writes one contiguous row segment:
-//   EPI_GELU:    h[grow_i, n0 + j]   = bf16(GELU(acc + b1[n0 + j]))       (64 B per row)
+//   EPI_GELU:    h[grow_i, n0 + j]   = bf16(GELU(acc + b1[n0 + j]))       (64 B per row; SiLU alike)
 //   EPI_COMBINE: out[tok_i, n0 + j] += w_i * (acc + b2[n0 + j])           (128 B per row, fp32 red)
 //   EPI_STORE_Y: y[grow_i, n0 + j]   = acc + b2[n0 + j]                   (128 B per row)
 // Rows i >= nrows (past the expert's segment) are skipped.  grow_i = grow0 + i.
@@ -303,12 +317,12 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t
     mine[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
                           __uint_as_float(r[4 * q + 3]));
   __syncwarp();
-  const float bj = __bfloat162float(brow[n0 + lane]);
+  const float bj = brow ? __bfloat162float(brow[n0 + lane]) : 0.f;
   const int nr = nrows < 32 ? nrows : 32;
-  if (EPI == EPI_GELU) {
+  if constexpr (epi_h(EPI)) {
     for (int i = 0; i < nr; ++i) {
       const float v = stg[i * kStgStride + lane] + bj;
-      g.h_out[(size_t)(grow0 + i) * g.N + n0 + lane] = __float2bfloat16_rn(gelu_erf(v));
+      g.h_out[(size_t)(grow0 + i) * g.N + n0 + lane] = __float2bfloat16_rn(act<EPI>(v));
     }
   } else if (EPI == EPI_COMBINE) {
     for (int i = 0; i < nr; ++i) {
@@ -323,11 +337,12 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t
   __syncwarp();
 }
 
-// GEMM1 epilogue of a 64-column group of a warp's 32 rows (lane i owns row i): bias + GELU, bf16,
+// GEMM1 epilogue of a 64-column group of a warp's 32 rows (lane i owns row i): bias + activation, bf16,
 // written into the warp's staging box in the 128-byte swizzle a TMA store expects (16-byte piece
 // j of row i sits at piece j ^ (i % 8)), then stored with one TMA instruction.  Only used when all
 // 32 rows lie inside the expert's segment, so the box never touches the next expert's rows.
-__device__ __forceinline__ void epilogue_gelu_box(const CUtensorMap* tmC, const uint32_t (&r0)[32],
+template <int EPI>
+__device__ __forceinline__ void epilogue_h_box(const CUtensorMap* tmC, const uint32_t (&r0)[32],
                                                   const uint32_t (&r1)[32], uint8_t* stg, int lane,
                                                   const __nv_bfloat16* brow, int n0, int grow0) {
   if (lane == 0) bulk_wait_read0();  // the previous box has left the staging buffer
@@ -336,14 +351,14 @@ __device__ __forceinline__ void epilogue_gelu_box(const CUtensorMap* tmC, const 
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t* src = j < 4 ? &r0[8 * j] : &r1[8 * (j - 4)];
-    const uint4 bb = __ldg(reinterpret_cast<const uint4*>(brow + n0 + 8 * j));
+    const uint4 bb = bias8(brow, n0 + 8 * j);
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
     uint32_t w[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float2 f = __bfloat1622float2(b2[u]);
       const __nv_bfloat162 v =
-          __floats2bfloat162_rn(gelu_erf(__uint_as_float(src[2 * u]) + f.x), gelu_erf(__uint_as_float(src[2 * u + 1]) + f.y));
+          __floats2bfloat162_rn(act<EPI>(__uint_as_float(src[2 * u]) + f.x), act<EPI>(__uint_as_float(src[2 * u + 1]) + f.y));
       w[u] = *reinterpret_cast<const uint32_t*>(&v);
     }
     *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -357,21 +372,22 @@ __device__ __forceinline__ void epilogue_gelu_box(const CUtensorMap* tmC, const 
 }
 
 // The same values written row by row from registers (rows past the segment are skipped).
-__device__ __forceinline__ void epilogue_gelu_rows(const GemmArgs& g, const uint32_t (&r0)[32], const uint32_t (&r1)[32],
+template <int EPI>
+__device__ __forceinline__ void epilogue_h_rows(const GemmArgs& g, const uint32_t (&r0)[32], const uint32_t (&r1)[32],
                                                    int lane, int nrows, const __nv_bfloat16* brow, int n0, int grow0) {
   if (lane >= nrows) return;
   uint4* dst = reinterpret_cast<uint4*>(g.h_out + (size_t)(grow0 + lane) * g.N + n0);
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t* src = j < 4 ? &r0[8 * j] : &r1[8 * (j - 4)];
-    const uint4 bb = __ldg(reinterpret_cast<const uint4*>(brow + n0 + 8 * j));
+    const uint4 bb = bias8(brow, n0 + 8 * j);
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
     uint32_t w[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float2 f = __bfloat1622float2(b2[u]);
       const __nv_bfloat162 v =
-          __floats2bfloat162_rn(gelu_erf(__uint_as_float(src[2 * u]) + f.x), gelu_erf(__uint_as_float(src[2 * u + 1]) + f.y));
+          __floats2bfloat162_rn(act<EPI>(__uint_as_float(src[2 * u]) + f.x), act<EPI>(__uint_as_float(src[2 * u + 1]) + f.y));
       w[u] = *reinterpret_cast<const uint32_t*>(&v);
     }
     dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -542,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tok = g.row_token[grow];
         wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
       }
-      const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
+      const __nv_bfloat16* brow = g.bias ? g.bias + (size_t)e * g.N : nullptr;
       const int wrows = rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
       constexpr int kChunks = BN / 32 / (kEpiWarps / 4);  // 32-column chunks per epilogue warp
 #pragma unroll 1
@@ -812,20 +828,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tok = g.row_token[grow];
         wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
       }
-      const __nv_bfloat16* brow = g.bias + (size_t)e * g.N;
+      const __nv_bfloat16* brow = g.bias ? g.bias + (size_t)e * g.N : nullptr;
       const int wrows = my_rows - qr * 32;  // rows of this warp's 32 that lie inside the segment
       const int wrow0 = row0 + cta_rows * (int)rank + qr * 32;
       const int nch = (hm ? C::kTileN / 64 : C::kTileN / 32) / (kEpiWarps / 4);  // 32-column chunks per warp
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::kTileN);
-      if (EPI == EPI_GELU) {
+      if constexpr (epi_h(EPI)) {
 #pragma unroll 1
         for (int c = half * nch; c < (half + 1) * nch; c += 2) {
           uint32_t r0[32], r1[32];
           tmem_ld32(taddr + c * 32, r0);
           tmem_ld32(taddr + (c + 1) * 32, r1);
           const int n0 = n_idx * C::kTileN + colbase + c * 32;
-          if (wrows >= 32) epilogue_gelu_box(&tmC, r0, r1, reinterpret_cast<uint8_t*>(stg), lane, brow, n0, wrow0);
-          else if (wrows > 0) epilogue_gelu_rows(g, r0, r1, lane, wrows, brow, n0, wrow0);
+          if (wrows >= 32) epilogue_h_box<EPI>(&tmC, r0, r1, reinterpret_cast<uint8_t*>(stg), lane, brow, n0, wrow0);
+          else if (wrows > 0) epilogue_h_rows<EPI>(g, r0, r1, lane, wrows, brow, n0, wrow0);
         }
       } else {
 #pragma unroll 1
@@ -840,7 +856,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
     }
-    if (EPI == EPI_GELU && lane == 0) bulk_wait0();  // this warp's h boxes are written before exit
+    if (epi_h(EPI) && lane == 0) bulk_wait0();  // this warp's h boxes are written before exit
   }
 
   tc_fence_before();
@@ -982,7 +998,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
   const long long avg_rows = (long long)a.T * a.k / a.E;
-  cudaError_t err = launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st);
+  cudaError_t err = a.act == MOE_ACT_SILU ? launch_bn<EPI_SILU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st)
+                                          : launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st);
   if (err != cudaSuccess) return err;
   ++*launches;
 

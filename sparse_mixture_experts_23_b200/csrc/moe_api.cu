@@ -91,6 +91,7 @@ moe_status_t check_shape(const moe_shape_t* s) {
   if (s->k > s->E || s->k > 8 || s->E > 256) return MOE_ERR_INVALID_ARG;
   if (!(s->capacity_factor > 0.0)) return MOE_ERR_INVALID_ARG;  // also rejects NaN
   if (s->dtype != MOE_DTYPE_F32 && s->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if (s->activation != MOE_ACT_GELU && s->activation != MOE_ACT_SILU) return MOE_ERR_INVALID_ARG;
   if (s->dtype == MOE_DTYPE_BF16 && (s->H % 64 != 0 || s->F % 64 != 0)) return MOE_ERR_UNSUPPORTED;
   if (s->dtype == MOE_DTYPE_F32 && (s->H % 4 != 0 || s->F % 4 != 0)) return MOE_ERR_UNSUPPORTED;
   const long long rows = (long long)s->T * s->k;
@@ -224,6 +225,7 @@ moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse
   a.y = at<float>(ws, L.y);
   a.out = io->out;
   a.fuse_combine = fuse;
+  a.act = s->activation;
   a.status = at<int32_t>(ws, L.status);
   a.wait_limit = g_wait_limit;
   a.num_sms = num_sms();
@@ -272,7 +274,7 @@ moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, s
   if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
   if (null_any({io->aux_loss, io->z_loss})) return MOE_ERR_INVALID_ARG;
   if (shape->T == 0) return do_route(shape, io, ws, stream, true);
-  if (null_any({io->x, io->Wg, io->bg, io->topk_idx, io->topk_w})) return MOE_ERR_INVALID_ARG;
+  if (null_any({io->x, io->Wg, io->topk_idx, io->topk_w})) return MOE_ERR_INVALID_ARG;  // bg optional
   if (!aligned16(io->x) || !aligned16(io->Wg)) return MOE_ERR_INVALID_ARG;
   if ((st = do_route(shape, io, ws, stream, true)) != MOE_OK) return st;
   ++g_launches;
@@ -311,7 +313,7 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io, void* 
   if (io == nullptr) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
-  if (null_any({io->W1, io->b1, io->W2, io->b2, io->topk_w})) return MOE_ERR_INVALID_ARG;
+  if (null_any({io->W1, io->W2, io->topk_w})) return MOE_ERR_INVALID_ARG;  // b1, b2 optional
   if (fuse_combine && io->out == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(io->W1) || !aligned16(io->W2) || !aligned16(io->b1) || !aligned16(io->b2) ||
       (fuse_combine && !aligned16(io->out)))
@@ -345,8 +347,7 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws,
     ++g_launches;
     return cuda_status(launch_zero_outputs(io->expert_counts, shape->E, io->aux_loss, io->z_loss, stream));
   }
-  if (null_any({io->x, io->Wg, io->bg, io->W1, io->b1, io->W2, io->b2, io->out, io->topk_idx, io->topk_w,
-                io->dropped}))
+  if (null_any({io->x, io->Wg, io->W1, io->W2, io->out, io->topk_idx, io->topk_w, io->dropped}))
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(io->x) || !aligned16(io->Wg) || !aligned16(io->W1) || !aligned16(io->W2) || !aligned16(io->out) ||
       !aligned16(io->b1) || !aligned16(io->b2))

@@ -81,9 +81,10 @@ struct FfnArgs {
   const float* topk_w;
   const void* x_perm;
   const void* W1;
-  const void* b1;
+  const void* b1;  // may be null (no bias)
   const void* W2;
-  const void* b2;
+  const void* b2;  // may be null (no bias)
+  int act;         // moe_activation_t
   void* h;
   float* y;
   float* out;

@@ -75,7 +75,7 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   if (shape->T == 0) return moe::launch_zero_outputs(nullptr, 0, io->aux_loss, io->z_loss, stream) == cudaSuccess
                                 ? MOE_OK
                                 : MOE_ERR_CUDA;
-  if (io->x == nullptr || io->Wg == nullptr || io->bg == nullptr || io->topk_idx == nullptr || io->topk_w == nullptr)
+  if (io->x == nullptr || io->Wg == nullptr || io->topk_idx == nullptr || io->topk_w == nullptr)
     return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(io->x) & 15u) || (reinterpret_cast<uintptr_t>(io->Wg) & 15u))
     return MOE_ERR_INVALID_ARG;

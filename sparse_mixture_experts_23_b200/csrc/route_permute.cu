@@ -2,7 +2,7 @@
 //
 // Router ("MoE Training: Mixture of Experts" page, Quick Start MoELayer.forward; Core Concepts 2
 // "Routing Mechanisms" and 3 "Load Balancing"):
-//   logits = x.Wg + bg, p = softmax(logits), top-k by (logit desc, index asc), w = p_sel / sum p_sel,
+//   logits = x.Wg + bg (bg optional), p = softmax(logits), top-k by (logit desc, index asc), w = p_sel / sum p_sel,
 //   aux = E * sum_e f_e P_e (f from pre-drop counts / (T*k), P = mean_t p), z = mean_t lse_t^2.
 // Dispatch (Core Concepts 4 capacity_factor / drop_tokens; Best Practices 2 capacity tuning):
 //   capacity = ceil(CF*T*k/E) or unlimited; assignments ranked per expert in (slot, token) order;
@@ -284,7 +284,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           int e = eq * 4 + j;
-          logits[(tq + 8 * i) * L.epad + e] = acc[q][i * 4 + j] + (e < E ? to_f32(bg[e]) : 0.f);
+          logits[(tq + 8 * i) * L.epad + e] = acc[q][i * 4 + j] + (bg && e < E ? to_f32(bg[e]) : 0.f);
         }
     }
   } else {
@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
       float s = 0.f;
       for (int q = 0; q < KS; ++q) s += red[q * kChunk * L.epad + o];
       int e = o % L.epad;
-      logits[o] = s + (e < E ? to_f32(bg[e]) : 0.f);
+      logits[o] = s + (bg && e < E ? to_f32(bg[e]) : 0.f);
     }
   }
   __syncthreads();
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_stream_kernel(RouterArg
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int e = 0; e < EP; ++e) logits[(tl0 + i) * EP + e] = acc[i][e] + (e < E ? __bfloat162float(bg[e]) : 0.f);
+      for (int e = 0; e < EP; ++e) logits[(tl0 + i) * EP + e] = acc[i][e] + (bg && e < E ? __bfloat162float(bg[e]) : 0.f);
   }
   __syncthreads();
   router_finish(a, logits, EP, reinterpret_cast<float*>(smem + S::psum_off(H)), reinterpret_cast<int*>(smem + S::misc_off(H)),
@@ -602,7 +602,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_mma_kernel(RouterArgs a
           const int row = m * 16 + g + (q >= 2 ? 8 : 0);
           const int col = nt * 8 + t4 * 2 + (q & 1);
           if (P.ks > 1) red[(my_ks * 32 + row) * P.ep8 + col] = acc[j][m][q];
-          else logits[row * P.ep8 + col] = acc[j][m][q] + (col < E ? __bfloat162float(bg[col]) : 0.f);
+          else logits[row * P.ep8 + col] = acc[j][m][q] + (bg && col < E ? __bfloat162float(bg[col]) : 0.f);
         }
     }
   }
@@ -612,7 +612,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_mma_kernel(RouterArgs a
       float v = 0.f;
       for (int q = 0; q < P.ks; ++q) v += red[q * 32 * P.ep8 + o];
       const int col = o % P.ep8;
-      logits[o] = v + (col < E ? __bfloat162float(bg[col]) : 0.f);
+      logits[o] = v + (bg && col < E ? __bfloat162float(bg[col]) : 0.f);
     }
   }
   __syncthreads();
@@ -756,7 +756,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_direct_kernel(RouterArg
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += red[w * 32 * E + o];
-    logits[o] = v + __bfloat162float(bg[o % E]);
+    logits[o] = v + (bg ? __bfloat162float(bg[o % E]) : 0.f);
   }
   __syncthreads();
   router_finish(a, logits, E, reinterpret_cast<float*>(smem + S::psum_off(H)), reinterpret_cast<int*>(smem + S::misc_off(H)),

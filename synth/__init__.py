@@ -5,9 +5,10 @@ weights Wg[H,E], bg[E] and expert weights W1[E,H,F], b1[E,F], W2[E,F,H], b2[E,H]
 counter-based generator (``synth.c`` states the exact definition) and rounds them to the storage
 dtype.  Values are produced on the host so that the CUDA path and the oracle see the same bits.
 
-The workload recipes (``CONFIGS``) restate the five synthetic layer shapes used for parity and
+The workload recipes (``CONFIGS``) restate the synthetic layer shapes used for parity and
 measurement: a tiny fp32 layer, a decode-sized layer, a Switch-style training layer with a capacity
-factor, a Mixtral-shaped layer and a skewed-load layer.  Shapes follow the pages' DeepSpeed
+factor, a Mixtral-shaped layer, a skewed-load layer, and the Mixtral block's own expert variant
+(bias-free, SiLU) at the Mixtral shape.  Shapes follow the pages' DeepSpeed
 launch examples ("MoE Training" skill page, Quick Start / Training Script sections) where they give
 them.
 """
@@ -119,6 +120,8 @@ class LayerConfig:
     bias_std: float = 0.02
     bg_rule: str = "zero"  # "zero" or "zipf"  (bg[e] = 1.5 * ln(1/(e+1)))
     note: str = ""
+    act: str = "gelu"  # expert activation: "gelu" (Quick Start expert) or "silu" (Mixtral block)
+    bias: bool = True  # False: gate and experts have no bias at all (bg = b1 = b2 = None)
 
     @property
     def x_std(self) -> float:
@@ -144,6 +147,9 @@ CONFIGS = {
                            note="Mixtral-shaped layer, dropless (headline)"),
     "skew": LayerConfig("skew", T=16384, H=2048, E=64, k=2, F=8192, CF=math.inf, dtype="bf16", seed=5,
                         bg_rule="zipf", note="skewed expert load, dropless"),
+    "mixtral_block": LayerConfig("mixtral_block", T=4096, H=4096, E=8, k=2, F=14336, CF=math.inf, dtype="bf16",
+                                 seed=6, act="silu", bias=False,
+                                 note="the Mixtral block's own expert: bias-free gate and Linear layers, SiLU"),
 }
 
 
@@ -152,15 +158,17 @@ class LayerInputs:
     cfg: LayerConfig
     x: np.ndarray
     Wg: np.ndarray
-    bg: np.ndarray
+    bg: np.ndarray | None
     W1: np.ndarray
-    b1: np.ndarray
+    b1: np.ndarray | None
     W2: np.ndarray
-    b2: np.ndarray
+    b2: np.ndarray | None
     extra: dict = field(default_factory=dict)
 
     def arrays(self):
-        return dict(x=self.x, Wg=self.Wg, bg=self.bg, W1=self.W1, b1=self.b1, W2=self.W2, b2=self.b2)
+        """The inputs that are present (a bias-free layer has no bg / b1 / b2 entries)."""
+        d = dict(x=self.x, Wg=self.Wg, bg=self.bg, W1=self.W1, b1=self.b1, W2=self.W2, b2=self.b2)
+        return {n: a for n, a in d.items() if a is not None}
 
 
 def make_bg(cfg: LayerConfig) -> np.ndarray:
@@ -186,6 +194,8 @@ def make_inputs(cfg: LayerConfig, with_weights: bool = True) -> LayerInputs:
         W1 = W2 = None
     b1 = normal(s, STREAM["b1"], (E, F), 0.0, cfg.bias_std, dt)
     b2 = normal(s, STREAM["b2"], (E, H), 0.0, cfg.bias_std, dt)
+    if not cfg.bias:
+        bg = b1 = b2 = None
     return LayerInputs(cfg, x, Wg, bg, W1, b1, W2, b2)
 
 

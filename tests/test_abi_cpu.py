@@ -87,6 +87,24 @@ def test_bad_dtype_enum(lib):
     assert moe.moe_forward(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG
 
 
+def test_activation_field(lib):
+    """moe_shape_t keeps its 40-byte layout: the activation sits in the tail after dtype, and a
+    zero-initialised shape means GELU; unknown activations are rejected before any launch."""
+    assert ctypes.sizeof(moe.Shape) == 40 and moe.Shape.activation.offset == 36
+    assert moe.Shape().activation == moe.MOE_ACT_GELU
+    s = _shape()
+    assert moe.moe_workspace_size(s) > 0
+    s.activation = moe.MOE_ACT_SILU
+    assert moe.moe_workspace_size(s) > 0
+    s.activation = 2
+    assert moe.moe_workspace_size(s) == 0
+    for fn in (moe.moe_route, moe.moe_permute, moe.moe_combine, moe.moe_forward):
+        assert fn(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_expert_ffn(s, _io(), FAKE, 1 << 40, 1) == moe.MOE_ERR_INVALID_ARG
+    text = open(HEADER).read()
+    assert "MOE_ACT_GELU = 0" in text and "MOE_ACT_SILU = 1" in text
+
+
 def test_workspace_errors(lib):
     s = _shape()
     n = moe.moe_workspace_size(s)
@@ -96,7 +114,7 @@ def test_workspace_errors(lib):
     assert moe.moe_forward(s, _io(), FAKE + 16, n) == moe.MOE_ERR_INVALID_ARG  # not 256-aligned
 
 
-@pytest.mark.parametrize("field", ["x", "Wg", "bg", "W1", "b1", "W2", "b2", "out", "topk_idx", "topk_w",
+@pytest.mark.parametrize("field", ["x", "Wg", "W1", "W2", "out", "topk_idx", "topk_w",
                                    "expert_counts", "dropped", "aux_loss", "z_loss"])
 def test_null_pointers_rejected(lib, field):
     s = _shape()
@@ -104,7 +122,7 @@ def test_null_pointers_rejected(lib, field):
     assert moe.moe_forward(s, _io(**{field: None}), FAKE, n) == moe.MOE_ERR_INVALID_ARG
 
 
-@pytest.mark.parametrize("field", ["x", "Wg", "W1", "W2", "out"])
+@pytest.mark.parametrize("field", ["x", "Wg", "W1", "W2", "out", "b1", "b2"])
 def test_misaligned_pointers_rejected(lib, field):
     s = _shape()
     n = moe.moe_workspace_size(s)

@@ -56,7 +56,7 @@ def _check_against_oracle(cfg, r):
     assert abs(r["losses"][1] - z) <= TOL_LOSS * abs(z)
     toks = np.arange(cfg.T, dtype=np.int32)
     want = oracle.forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, r["topk_idx"],
-                                 r["topk_w"].astype(np.float64), r["dropped"], toks, cfg.dtype)
+                                 r["topk_w"].astype(np.float64), r["dropped"], toks, cfg.dtype, act=cfg.act)
     live = ~r["dropped"].astype(bool).all(axis=1)
     err, tol = out_error(r["out"].astype(np.float64), want, cfg.dtype, rows=live)
     assert err <= tol, (err, tol)
@@ -79,9 +79,27 @@ def _check_against_oracle(cfg, r):
     _cfg("long_segments", 1000, 128, 3, 2, 256, math.inf, "bf16", 26),
     # CTA-pair tiles in both GEMMs (N divisible by 256, K by 128), ragged tails, capacity drops
     _cfg("pair_tiles", 1500, 256, 4, 2, 512, 1.1, "bf16", 27),
+    # the Mixtral block's expert (SiLU, no bias anywhere) on the fp32 path, the single-CTA tiles
+    # (N = 192 -> 64-wide, 128 -> 128-wide) and the CTA-pair tiles with half tiles and drops
+    _cfg("silu_nobias_f32", 77, 20, 5, 2, 12, math.inf, "f32", 28, act="silu", bias=False),
+    _cfg("silu_nobias_bf16", 100, 128, 6, 3, 192, 1.0, "bf16", 29, act="silu", bias=False),
+    _cfg("silu_nobias_pair", 1500, 256, 4, 2, 512, 1.1, "bf16", 30, act="silu", bias=False),
+    # SiLU with biases present, k = 1 with drops
+    _cfg("silu_bias", 300, 256, 16, 1, 512, 1.25, "bf16", 33, act="silu"),
 ], ids=lambda c: c.name)
 def test_small_shapes_end_to_end(cfg):
     r = _run_forward(cfg)
+    _check_against_oracle(cfg, r)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_some_biases_absent(dtype):
+    """Each bias is optional on its own: no gate bias and no b2, but b1 present (GELU)."""
+    cfg = _cfg("partial_bias", 260, 128, 4, 2, 256, math.inf, dtype, 34)
+    inp = synth.make_inputs(cfg)
+    inp.bg = None
+    inp.b2 = None
+    r = _run_forward(cfg, inp=inp)
     _check_against_oracle(cfg, r)
 
 

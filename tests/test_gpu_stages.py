@@ -1,4 +1,4 @@
-"""Stage-wise parity of the CUDA path against the fp64 oracle on the five synthetic layer workloads.
+"""Stage-wise parity of the CUDA path against the fp64 oracle on the synthetic layer workloads.
 
 Each stage is fed the GPU's own upstream result, so a near-tie flip in routing cannot cascade:
   route    -> top-k indices bit-exact (near ties excluded and counted), weights 1e-4, losses 1e-3
@@ -20,7 +20,7 @@ from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, out_error,
 
 pytestmark = pytest.mark.gpu
 
-SAMPLES = {"tiny": 256, "decode": 32, "switch": 48, "mixtral": 24, "skew": 48}
+SAMPLES = {"tiny": 256, "decode": 32, "switch": 48, "mixtral": 24, "skew": 48, "mixtral_block": 24}
 
 
 @pytest.fixture(scope="module", params=list(synth.CONFIGS))
@@ -130,7 +130,7 @@ def test_ffn_combine_vs_oracle(run):
     cfg, inp = run["cfg"], run["inp"]
     toks = sample_tokens(cfg.T, SAMPLES[cfg.name], seed=cfg.seed)
     ref = oracle.forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, run["topk_idx"],
-                                run["topk_w"].astype(np.float64), run["dropped"], toks, cfg.dtype)
+                                run["topk_w"].astype(np.float64), run["dropped"], toks, cfg.dtype, act=cfg.act)
     got = run["out"][toks].astype(np.float64)
     live = ~run["dropped"][toks].astype(bool).all(axis=1)
     err, tol = out_error(got, ref, cfg.dtype, rows=live)
