@@ -13,6 +13,8 @@ documented steps:
   losses     -> Switch aux loss E*sum f*P (pre-drop counts / (T*k)), z-loss mean(lse^2)
   dispatch   -> capacity ceil(CF*T*k/E) or unlimited; slot-major then token-order ranks; rows
   forward    -> out[t] = sum over kept slots of w * FFN_e(x_t)
+  expert choice (ec_*) -> every expert takes its top-C tokens by logit; out[t] = sum over the
+                experts that chose t of p[t,e] * FFN_e(x_t)
 
 Parity status of each function is recorded in the test-suite pins (``tests/test_oracle_pins.py``);
 every function here is pinned there against closed forms, library routines or brute force.
@@ -69,6 +71,12 @@ def _load():
     lib.oracle_forward_tokens.argtypes = [i64, i64, i64, c_int, c_int, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp,
                                           vp, c_int]
     lib.oracle_forward_tokens.restype = None
+    lib.oracle_ec_capacity.argtypes = [dbl, i64, i64, i64]
+    lib.oracle_ec_capacity.restype = i64
+    lib.oracle_expert_choice.argtypes = [i64, i64, i64, vp, vp, vp]
+    lib.oracle_expert_choice.restype = None
+    lib.oracle_ec_losses.argtypes = [i64, i64, i64, vp, vp, vp, vp]
+    lib.oracle_ec_losses.restype = None
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     lib.oracle_set_threads.argtypes = [c_int]
@@ -229,3 +237,79 @@ def forward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=Non
     tokens = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
     out = forward_tokens(x, W1, b1, W2, b2, r.topk_idx, r.topk_w, d.dropped, tokens, dtype, nthreads, act)
     return Forward(r, aux, z, d, out, tokens)
+
+
+# ------------------------------------------------------------------ expert-choice routing -------
+
+def ec_capacity(cf: float, T: int, k: int, E: int) -> int:
+    """Tokens per expert under expert choice: min(T, ceil(CF*T*k/E)); T when CF = +inf."""
+    return int(_load().oracle_ec_capacity(float(cf), T, k, E))
+
+
+@dataclass
+class ExpertChoice:
+    C: int
+    chosen: np.ndarray  # [E, C] int32, ascending token order per expert
+    margin: np.ndarray  # [E] f64: gap between the C-th and (C+1)-th logit of each expert
+
+    def member(self, T: int) -> np.ndarray:
+        """[T, E] bool: token t chosen by expert e."""
+        E = self.chosen.shape[0]
+        m = np.zeros((T, E), bool)
+        for e in range(E):
+            m[self.chosen[e], e] = True
+        return m
+
+
+def expert_choice(logits, C: int) -> ExpertChoice:
+    lg = _c(logits, np.float64)
+    T, E = lg.shape
+    chosen = np.empty((E, max(C, 0)), np.int32)
+    margin = np.empty(E, np.float64)
+    _load().oracle_expert_choice(T, E, C, _p(lg), _p(chosen), _p(margin))
+    return ExpertChoice(C, chosen, margin)
+
+
+def ec_losses(p, lse, C: int):
+    p, lse = _c(p, np.float64), _c(lse, np.float64)
+    T, E = p.shape
+    aux = np.zeros(1, np.float64)
+    z = np.zeros(1, np.float64)
+    _load().oracle_ec_losses(T, E, C, _p(p), _p(lse), _p(aux), _p(z))
+    return float(aux[0]), float(z[0])
+
+
+def ec_forward_tokens(x, W1, b1, W2, b2, p, member, tokens, dtype: str, nthreads: int = 0,
+                      act: str = "gelu") -> np.ndarray:
+    """out[i] = sum over experts e that chose token tokens[i] of p[t,e] * FFN_e(x_t), experts in
+    ascending order: the token-choice combine with every expert as a slot and the unchosen ones
+    dropped."""
+    p = _c(p, np.float64)
+    T, E = p.shape
+    idx = np.tile(np.arange(E, dtype=np.int32), (T, 1))
+    dropped = (~np.asarray(member, bool)).astype(np.uint8)
+    return forward_tokens(x, W1, b1, W2, b2, idx, p, dropped, tokens, dtype, nthreads, act)
+
+
+@dataclass
+class ForwardEC:
+    routing: Routing
+    ec: ExpertChoice
+    aux: float
+    z: float
+    out: np.ndarray
+    tokens: np.ndarray
+
+
+def forward_ec(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=None, nthreads: int = 0,
+               act: str = "gelu") -> ForwardEC:
+    """Whole layer under expert-choice routing (Core Concepts 2)."""
+    T = x.shape[0]
+    E = Wg.shape[1]
+    r = route(x, Wg, bg, 1, dtype)
+    C = ec_capacity(cf, T, k, E)
+    ec = expert_choice(r.logits, C)
+    aux, z = ec_losses(r.p, r.lse, C)
+    tokens = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
+    out = ec_forward_tokens(x, W1, b1, W2, b2, r.p, ec.member(T), tokens, dtype, nthreads, act)
+    return ForwardEC(r, ec, aux, z, out, tokens)

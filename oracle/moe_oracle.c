@@ -316,6 +316,89 @@ void oracle_forward_tokens(int64_t H, int64_t F, int64_t k, int dtype, int act, 
   }
 }
 
+/* ----------------------------------------------------------------------------------------------
+ * Expert-choice routing -- [SKILL] Core Concepts 2, "Expert Choice Routing": the router scores
+ * are transposed to (experts, tokens) and every expert takes the top capacity_per_expert tokens
+ * of its row ("guarantees perfect load balancing").  Readings (listed in the design notes):
+ *  - the scores are the router's logits, as printed (no softmax before the per-expert top-k);
+ *  - capacity_per_expert C = min(T, ceil(CF * T * k / E)), k being the average number of experts
+ *    per token; CF = +inf gives C = T (every expert sees every token);
+ *  - ties go to the lower token index; an expert's chosen tokens are listed in ascending token
+ *    order, which is also their row order inside the expert's segment;
+ *  - a chosen (token, expert) pair is weighted by the token's softmax probability p[t,e] over the
+ *    experts, without renormalisation; a token chosen by no expert gets out = 0.
+ * ---------------------------------------------------------------------------------------------- */
+int64_t oracle_ec_capacity(double cf, int64_t T, int64_t k, int64_t E) {
+  if (isinf(cf) && cf > 0) return T;
+  int64_t c = (int64_t)ceil(cf * (double)T * (double)k / (double)E);
+  return c < T ? c : T;
+}
+
+typedef struct {
+  double v;
+  int32_t t;
+} scored_token;
+
+/* score descending, token index ascending */
+static int by_score_then_token(const void* pa, const void* pb) {
+  const scored_token* a = (const scored_token*)pa;
+  const scored_token* b = (const scored_token*)pb;
+  if (a->v > b->v) return -1;
+  if (a->v < b->v) return 1;
+  return (a->t > b->t) - (a->t < b->t);
+}
+
+/*
+ * chosen[e*C + j], j < C: the C tokens of expert e in ascending token order.
+ * margin[e]: logits gap between the C-th and (C+1)-th token of expert e in score order
+ *            (+inf when C == T).  margin may be NULL.
+ */
+void oracle_expert_choice(int64_t T, int64_t E, int64_t C, const double* logits, int32_t* chosen, double* margin) {
+#pragma omp parallel
+  {
+    scored_token* order = (scored_token*)malloc(sizeof(scored_token) * (size_t)(T > 0 ? T : 1));
+    char* mark = (char*)malloc((size_t)(T > 0 ? T : 1));
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t e = 0; e < E; ++e) {
+      for (int64_t t = 0; t < T; ++t) {
+        order[t].v = logits[t * E + e];
+        order[t].t = (int32_t)t;
+      }
+      qsort(order, (size_t)T, sizeof(scored_token), by_score_then_token);
+      for (int64_t t = 0; t < T; ++t) mark[t] = 0;
+      for (int64_t j = 0; j < C; ++j) mark[order[j].t] = 1;
+      int64_t j = 0;
+      for (int64_t t = 0; t < T; ++t)
+        if (mark[t]) chosen[e * C + j++] = (int32_t)t;
+      if (margin) margin[e] = (C < T && C > 0) ? order[C - 1].v - order[C].v : INFINITY;
+    }
+    free(order);
+    free(mark);
+  }
+}
+
+/* Losses under expert choice: every expert holds C of the E*C assignments, so f_e = 1/E and
+ * aux = E * sum_e f_e * P_e = sum_e P_e; z = mean_t lse_t^2 as for token choice (Core Concepts 3). */
+void oracle_ec_losses(int64_t T, int64_t E, int64_t C, const double* p, const double* lse, double* aux, double* z) {
+  if (T == 0) {
+    *aux = 0.0;
+    *z = 0.0;
+    return;
+  }
+  double a = 0.0;
+  for (int64_t e = 0; e < E; ++e) {
+    double P = 0.0;
+    for (int64_t t = 0; t < T; ++t) P += p[t * E + e];
+    P /= (double)T;
+    const double f = (double)C / ((double)E * (double)C);
+    a += f * P;
+  }
+  *aux = (double)E * a;
+  double zz = 0.0;
+  for (int64_t t = 0; t < T; ++t) zz += lse[t] * lse[t];
+  *z = zz / (double)T;
+}
+
 /* threads the OpenMP runtime will use for a parallel region (for reporting) */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -417,3 +417,113 @@ def test_planted_mistakes_are_caught():
     d = oracle.dispatch(idx, 2, 2 * 2 / 6)
     token_major_drop = [[0, 0], [1, 0], [0, 1]]  # what token-major order would give
     assert d.dropped.tolist() != token_major_drop
+
+
+# ---------------------------------------------------------------- expert-choice routing ---------
+
+def test_ec_capacity_values():
+    assert oracle.ec_capacity(1.0, 4096, 2, 8) == 1024
+    assert oracle.ec_capacity(1.25, 8192, 1, 128) == 80
+    assert oracle.ec_capacity(1.0, 10, 1, 3) == 4  # ceil(10/3)
+    assert oracle.ec_capacity(math.inf, 77, 2, 5) == 77
+    assert oracle.ec_capacity(50.0, 77, 2, 5) == 77  # never more than T
+
+
+def test_ec_brute_force_topC_per_expert():
+    """The chosen set of every expert is the unique C-subset whose worst member beats every other token
+    under (logit, -token); listed in ascending token order."""
+    rng = np.random.default_rng(5)
+    T, E, C = 8, 3, 3
+    logits = np.round(rng.normal(size=(T, E)), 1)  # rounding makes ties likely
+    ec = oracle.expert_choice(logits, C)
+    for e in range(E):
+        key = lambda t: (logits[t, e], -t)  # noqa: E731
+        winners = [S for S in itertools.combinations(range(T), C)
+                   if min(key(t) for t in S) > max(key(t) for t in range(T) if t not in S)]
+        assert len(winners) == 1
+        assert ec.chosen[e].tolist() == sorted(winners[0])
+        srt = sorted(range(T), key=key, reverse=True)
+        assert ec.margin[e] == logits[srt[C - 1], e] - logits[srt[C], e]
+
+
+def test_ec_perfect_balance_and_scalar_closed_form():
+    """H = 1 and Wg[0] = (+1, -1): expert 0 takes the C largest x, expert 1 the C smallest (numpy
+    argsort gives the closed form); every expert holds exactly C distinct tokens."""
+    T, C = 50, 7
+    x = synth.normal(7, 1, (T, 1))
+    Wg = np.array([[1.0, -1.0]], np.float32)
+    r = oracle.route(x, Wg, None, 1, "f32")
+    ec = oracle.expert_choice(r.logits, C)
+    xs = x[:, 0].astype(np.float64)
+    assert ec.chosen[0].tolist() == sorted(np.argsort(-xs, kind="stable")[:C].tolist())
+    assert ec.chosen[1].tolist() == sorted(np.argsort(xs, kind="stable")[:C].tolist())
+    for e in range(2):
+        assert len(set(ec.chosen[e].tolist())) == C and (np.diff(ec.chosen[e]) > 0).all()
+
+
+def test_ec_equal_scores_take_the_first_tokens():
+    """Wg = 0: every token has the same logit for a given expert, so each expert takes tokens 0..C-1."""
+    T, H, E, C = 20, 8, 4, 6
+    x = synth.normal(8, 1, (T, H))
+    bg = np.array([0.3, -1.0, 2.0, 0.0], np.float32)
+    r = oracle.route(x, np.zeros((H, E), np.float32), bg, 1, "f32")
+    ec = oracle.expert_choice(r.logits, C)
+    assert (ec.chosen == np.arange(C)).all()
+    assert (ec.margin == 0).all()
+
+
+def test_ec_losses_closed_form():
+    """f_e = 1/E under expert choice, so aux = sum_e P_e = 1 (softmax rows sum to 1); z as for top-k."""
+    inp = _rand_layer(T=31, H=16, E=6, F=8, seed=61)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, 1, "f32")
+    aux, z = oracle.ec_losses(r.p, r.lse, 9)
+    assert aux == pytest.approx(1.0, abs=1e-13)
+    assert z == pytest.approx(float(np.mean(special.logsumexp(r.logits, axis=1) ** 2)), rel=1e-13)
+    assert oracle.ec_losses(np.zeros((0, 6)), np.zeros(0), 1) == (0.0, 0.0)
+
+
+def test_ec_full_capacity_is_dense_softmax_mixture():
+    """C = T (CF = +inf): every expert processes every token, so out = sum_e p_e FFN_e(x), the same
+    dense mixture as token choice with k = E."""
+    T, H, E, F = 15, 12, 4, 20
+    inp = _rand_layer(T=T, H=H, E=E, F=F, seed=63)
+    f = oracle.forward_ec(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, 2, math.inf, "f32")
+    assert f.ec.C == T
+    x = inp.x.astype(np.float64)
+    p = special.softmax(x @ inp.Wg.astype(np.float64) + inp.bg, axis=1)
+    ref = np.zeros((T, H))
+    for e in range(E):
+        u = x @ inp.W1[e].astype(np.float64) + inp.b1[e]
+        ref += p[:, e:e + 1] * ((u * stats.norm.cdf(u)) @ inp.W2[e].astype(np.float64) + inp.b2[e])
+    np.testing.assert_allclose(f.out, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_ec_forward_per_token_sum_and_unchosen_tokens():
+    """out[t] = sum over the experts that chose t of p[t,e] * FFN_e(x_t), checked row by row with
+    expert_rows; tokens chosen by no expert are exactly zero."""
+    T, H, E, F = 40, 8, 4, 16
+    inp = _rand_layer(T=T, H=H, E=E, F=F, seed=65)
+    f = oracle.forward_ec(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, 1, 0.5, "f32", act="silu")
+    assert f.ec.C == 5
+    member = f.ec.member(T)
+    assert (member.sum(axis=0) == 5).all()
+    for t in range(T):
+        es = np.where(member[t])[0].astype(np.int32)
+        if len(es) == 0:
+            assert (f.out[t] == 0).all()
+            continue
+        ys = oracle.expert_rows(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, np.full(len(es), t, np.int32), es, "f32",
+                                act="silu")
+        ref = sum(f.routing.p[t, e] * ys[i] for i, e in enumerate(es))
+        np.testing.assert_allclose(f.out[t], ref, rtol=1e-13, atol=1e-14)
+    assert (~member.any(axis=1)).sum() > 0
+
+
+def test_ec_selects_on_logits_not_probabilities():
+    """The page's expert-choice scores are the router outputs themselves: token 1 has the larger logit
+    for expert 0 (3 > 2) but the smaller probability (0.5 < 0.88), and it is the one chosen."""
+    logits = np.array([[2.0, 0.0], [3.0, 3.0]])
+    ec = oracle.expert_choice(logits, 1)
+    assert ec.chosen[0].tolist() == [1]
+    assert ec.chosen[1].tolist() == [1]
+    assert special.softmax(logits, axis=1)[0, 0] > special.softmax(logits, axis=1)[1, 0]
