@@ -39,7 +39,8 @@ METRIC = "MoE-layer fwd tokens/sec (Mixtral shape, 1 B200); grouped-GEMM % of BF
 def workload_config(cfg: synth.LayerConfig) -> str:
     cf = "dropless" if math.isinf(cfg.CF) else f"CF={cfg.CF}"
     ffn = f"{cfg.act.upper()} FFN " + ("with biases" if cfg.bias else "without biases")
-    return (f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} F={cfg.F} {cf}, {ffn}, "
+    route = "" if cfg.routing == "token_choice" else f"{cfg.routing.replace('_', '-')} routing, "
+    return (f"{cfg.name}: T={cfg.T} H={cfg.H} E={cfg.E} k={cfg.k} F={cfg.F} {cf}, {route}{ffn}, "
             f"{cfg.dtype} storage / fp32 accumulate")
 
 
@@ -165,6 +166,16 @@ def aggregate_rate(world: int, tokens_per_rank: int, steps: int, ms_total_max: f
 
 
 # ------------------------------------------------------------------------------------------------
+def oracle_layer(cfg: synth.LayerConfig, inp: synth.LayerInputs, lo: int, n: int):
+    """The fp64 oracle's whole layer on tokens [lo, lo+n) taken as one batch, under the workload's
+    routing rule."""
+    import oracle
+
+    fwd = oracle.forward_ec if cfg.routing == "expert_choice" else oracle.forward
+    return fwd(inp.x[lo:lo + n], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype,
+               act=cfg.act)
+
+
 def cpu_oracle_rate(cfg: synth.LayerConfig, inp: synth.LayerInputs, budget_s: float, max_tokens: int = 4096):
     """Tokens/s of the fp64 oracle (routing + dispatch + FFN + combine) on a leading token sample,
     growing the sample until one run lasts at least budget_s / 3."""
@@ -177,7 +188,7 @@ def cpu_oracle_rate(cfg: synth.LayerConfig, inp: synth.LayerInputs, budget_s: fl
     spent = 0.0
     while True:
         t0 = time.perf_counter()
-        oracle.forward(inp.x[:n], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
+        oracle_layer(cfg, inp, 0, n)
         dt = time.perf_counter() - t0
         spent += dt
         best = (n, dt)
@@ -201,16 +212,16 @@ def run_reference(args, cfg):
     threads = oracle.max_threads()
     # calibrate tokens per step so the whole run stays within about two minutes
     t0 = time.perf_counter()
-    oracle.forward(inp.x[:1], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
+    oracle_layer(cfg, inp, 0, 1)
     t1 = time.perf_counter() - t0
     per_step = 120.0 / max(1, args.steps + args.warmup)
     S = int(max(1, min(cfg.T, per_step / max(t1, 1e-6))))
     for _ in range(args.warmup):
-        oracle.forward(inp.x[:S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
+        oracle_layer(cfg, inp, 0, S)
     t0 = time.perf_counter()
     for i in range(args.steps):
         lo = (i * S) % max(1, cfg.T - S + 1)
-        oracle.forward(inp.x[lo:lo + S], inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, act=cfg.act)
+        oracle_layer(cfg, inp, lo, S)
     dt = time.perf_counter() - t0
     value = S * args.steps / dt
     line = {
@@ -256,7 +267,7 @@ def run_ours_impl(args, cfg):
 
     inp = replica_inputs(cfg, rank)
     dev = {n: _upload(a, cfg.dtype) for n, a in inp.arrays().items()}
-    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype, cfg.act)
+    shape = moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype, cfg.act, cfg.routing)
     buf = moe.MoEBuffers(shape, dev)
     stream = torch.cuda.current_stream()
     peaks = load_peaks()

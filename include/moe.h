@@ -18,6 +18,11 @@
  *                                                          Mixtral block index_add_)
  *   moe_forward     the four chained on one stream (fused combine)
  *
+ * Two routing rules (moe_shape_t.routing): token choice, where every token takes its top-k experts
+ * (Quick Start; Core Concepts 2 top-1 / top-2), and expert choice, where every expert takes its
+ * top-C tokens (Core Concepts 2, "Expert Choice Routing").  The buffers whose meaning differs
+ * between the two are listed under moe_io_t.
+ *
  * Conventions shared by every entry point
  *  - All tensors are row-major and contiguous.  Every pointer in moe_io_t is a DEVICE pointer
  *    owned by the caller; the library never allocates device memory and never frees it.
@@ -31,10 +36,11 @@
  *      MOE_ERR_INVALID_ARG  null shape/io/workspace pointer, a needed io pointer that is null, a
  *                           device pointer of x/Wg/W1/W2/out/workspace not 16-byte aligned,
  *                           T < 0, H/E/F/k <= 0, k > E, k > 8, E > 256, capacity_factor <= 0 or
- *                           NaN, unknown dtype or activation, a non-null b1/b2 not 16-byte
+ *                           NaN, unknown dtype, activation or routing, a non-null b1/b2 not 16-byte
  *                           aligned
  *      MOE_ERR_UNSUPPORTED  bf16 with H or F not a multiple of 64; f32 with H or F not a multiple
- *                           of 4; T*k*max(H,F) beyond 2^31 elements
+ *                           of 4; rows*max(H,F) beyond 2^31 elements (rows = T*k, or E*C under
+ *                           expert choice)
  *      MOE_ERR_WORKSPACE    ws_bytes < moe_workspace_size(shape)
  *      MOE_ERR_CUDA         a launch or driver call failed (the CUDA error is not cleared)
  *    On any error nothing has been launched by that call.
@@ -78,6 +84,14 @@ typedef enum {
 
 typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 
+/* Routing rule.  Expert choice: the router's logits are read per expert (the page transposes
+ * them to (experts, tokens)) and every expert takes the C tokens with the largest logits, ties to
+ * the lower token index, C = min(T, ceil(capacity_factor * T * k / E)) -- k is then the average
+ * number of experts per token, and capacity_factor = +INFINITY gives C = T.  Each chosen
+ * (token, expert) pair is weighted by the token's softmax probability over the experts, not
+ * renormalised; a token chosen by no expert gets out = 0.  Every expert holds exactly C rows. */
+typedef enum { MOE_ROUTING_TOKEN_CHOICE = 0, MOE_ROUTING_EXPERT_CHOICE = 1 } moe_routing_t;
+
 /* Activation between the two expert Linear layers.  GELU is the exact erf form (Quick Start
  * expert, nn.GELU()); SiLU is u * sigmoid(u) (Advanced Patterns, Mixtral block experts). */
 typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SILU = 1 } moe_activation_t;
@@ -94,6 +108,7 @@ typedef struct {
   double capacity_factor; /* > 0; +INFINITY = no capacity limit */
   moe_dtype_t dtype;      /* storage type of x and all weights */
   moe_activation_t activation; /* expert activation; a zero-initialised shape gets GELU */
+  moe_routing_t routing;       /* a zero-initialised shape gets token choice */
 } moe_shape_t;
 
 /* Caller-owned device buffers.  Layouts (row-major):
@@ -105,7 +120,14 @@ typedef struct {
  *                            (pre-drop values; dropped slots keep their weight here)
  *   expert_counts[E]   int32 kept assignments per expert (after capacity)
  *   dropped[T,k]       uint8 1 = assignment dropped by capacity
- *   aux_loss, z_loss   fp32 scalars: E*sum_e f_e*P_e and mean_t logsumexp_t^2, no coefficients */
+ *   aux_loss, z_loss   fp32 scalars: E*sum_e f_e*P_e and mean_t logsumexp_t^2, no coefficients
+ * Under expert choice (C as above) four of them change shape and meaning:
+ *   topk_idx[E,C]      int32 the tokens each expert chose, in ascending token order
+ *   topk_w[T,E]        fp32  softmax probabilities of every token over all experts (the weight of
+ *                            (t,e) when e chose t)
+ *   expert_counts[E]   int32 C for every expert
+ *   dropped[T]         uint8 1 = token chosen by no expert
+ * and aux_loss = sum_e P_e (f_e = 1/E; 1 up to rounding). */
 typedef struct {
   const void* x;
   const void* Wg;
@@ -135,17 +157,28 @@ typedef struct {
   void* h;             /* [T*k, F] storage dtype: act(x_perm . W1[e] + b1[e]) */
   float* y;            /* [T*k, H] fp32: h . W2[e] + b2[e] (only written when the combine is not fused) */
   size_t bytes;        /* total workspace size */
+  float* scores;       /* expert choice only (else NULL): [E,T] fp32 router logits, expert-major */
 } moe_ws_view_t;
+/* Under expert choice the row buffers hold E*C rows instead of T*k, row e*C + j being the j-th token
+ * that expert e chose; row_slot holds the expert and row_of is unused. */
 
 /* Workspace bytes for a shape; 0 if the shape is invalid.  Host only, pure. */
 MOE_API size_t moe_workspace_size(const moe_shape_t* shape);
+
+/* Per-expert capacity the shape implies.  Token choice: ceil(capacity_factor * T * k / E), or -1
+ * when capacity_factor = +INFINITY (no limit).  Expert choice: C = min(T, ceil(capacity_factor *
+ * T * k / E)), the number of tokens every expert takes (the leading size of topk_idx[E,C]).
+ * -2 if the shape is invalid.  Host only, pure. */
+MOE_API int64_t moe_capacity(const moe_shape_t* shape);
 
 /* Pointers to each stage buffer inside `ws` for `shape`.  Host only, pure. */
 MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, moe_ws_view_t* view);
 
 /* Router ("MoE Training" page, Quick Start MoELayer.forward: gate, softmax, topk, renormalise;
  * Core Concepts 3: load_balancing_loss, router_z_loss).
- * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws). */
+ * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws).
+ * Expert choice: also the per-expert selection (Core Concepts 2), so it writes the chosen tokens
+ * to topk_idx[E,C], expert_counts and dropped[T] as well; 3 launches. */
 MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
@@ -162,14 +195,17 @@ MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, voi
  * routine it calls.  The first call on a device looks up the array's device address for that
  * device (cudaGetSymbolAddress, with the device current); make that first call before any stream
  * capture.  Every call, on every stream, shares the one array and leaves the last call's contents
- * in it: calls that overlap on the GPU race, so serialise them (one stream, or events). */
+ * in it: calls that overlap on the GPU race, so serialise them (one stream, or events).
+ * Token choice only: an expert-choice shape returns MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream);
 
 /* Dispatch (Core Concepts 4 "capacity_factor", "drop_tokens"; Best Practices 2; Advanced Patterns
  * Mixtral block gather by expert).  Assignments are visited slot-major then by token; an
  * assignment is kept iff fewer than `capacity` earlier assignments went to its expert.
  * Reads x, topk_idx.  Writes expert_counts, dropped, the row maps and x_perm in ws, and clears
- * out[T,H] to zero (the fused combine accumulates into it). */
+ * out[T,H] to zero (the fused combine accumulates into it).
+ * Expert choice: nothing is dropped (each expert already holds exactly C tokens); reads x and
+ * topk_idx[E,C], writes the row maps and x_perm, and clears out. */
 MOE_API moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
@@ -177,7 +213,8 @@ MOE_API moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, v
  * grouped GEMMs over the expert segments of x_perm.  bf16: tcgen05 tensor cores, h stored bf16;
  * f32: CUDA cores, h stored f32.  fuse_combine != 0: out[t] += topk_w[t,s]*(h.W2[e] + b2[e]) for
  * every kept row (out must hold zeros from moe_permute); at most k fp32 adds reach each element,
- * so for k <= 2 the result does not depend on their order.  fuse_combine == 0: y in ws is
+ * so for k <= 2 the result does not depend on their order (under expert choice up to E adds
+ * reach an element, in no fixed order).  fuse_combine == 0: y in ws is
  * written instead and out is untouched.  Reads W1, b1, W2, b2, topk_w and the ws state of
  * moe_permute. */
 MOE_API moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
@@ -185,11 +222,14 @@ MOE_API moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io
 
 /* Combine from a materialised y (Quick Start "output[mask] += expert_scores * expert_output"):
  * out[t] = sum over kept slots s, in slot order, of topk_w[t,s] * y[row_of(t,s)]; tokens with
- * every slot dropped get zeros.  Overwrites out.  Use after moe_expert_ffn(fuse_combine = 0). */
+ * every slot dropped get zeros.  Overwrites out.  Use after moe_expert_ffn(fuse_combine = 0).
+ * Expert choice: out[t] += topk_w[t,e] * y[row] for every row, with fp32 atomics into the zeros
+ * that moe_permute left in out. */
 MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
-/* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream. */
+/* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream (5 launches; 6
+ * under expert choice). */
 MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 

@@ -19,11 +19,13 @@ MOE_DTYPE_F32, MOE_DTYPE_BF16 = 0, 1
 DTYPES = {"f32": MOE_DTYPE_F32, "bf16": MOE_DTYPE_BF16}
 MOE_ACT_GELU, MOE_ACT_SILU = 0, 1
 ACTIVATIONS = {"gelu": MOE_ACT_GELU, "silu": MOE_ACT_SILU}
+MOE_ROUTING_TOKEN_CHOICE, MOE_ROUTING_EXPERT_CHOICE = 0, 1
+ROUTINGS = {"token_choice": MOE_ROUTING_TOKEN_CHOICE, "expert_choice": MOE_ROUTING_EXPERT_CHOICE}
 
 ENTRY_POINTS = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_forward_host", "moe_get_device_status", "moe_set_wait_limit", "moe_debug_timeout_probe",
-    "moe_last_launch_count", "moe_status_string", "moe_route_noalloc",
+    "moe_last_launch_count", "moe_status_string", "moe_route_noalloc", "moe_capacity",
 )
 
 
@@ -36,7 +38,7 @@ class MoEError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32), ("F", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_double), ("dtype", ctypes.c_int),
-                ("activation", ctypes.c_int)]
+                ("activation", ctypes.c_int), ("routing", ctypes.c_int)]
 
 
 class IO(ctypes.Structure):
@@ -46,7 +48,8 @@ class IO(ctypes.Structure):
 
 class WsView(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("status", "offsets", "cnt_pre", "row_of", "row_token", "row_slot",
-                                               "x_perm", "h", "y")] + [("bytes", ctypes.c_size_t)]
+                                               "x_perm", "h", "y")] + [("bytes", ctypes.c_size_t),
+                                                                        ("scores", ctypes.c_void_p)]
 
 
 _lib = None
@@ -63,6 +66,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P, vp, sz, st = ctypes.POINTER, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
     lib.moe_workspace_size.argtypes = [P(Shape)]
     lib.moe_workspace_size.restype = sz
+    lib.moe_capacity.argtypes = [P(Shape)]
+    lib.moe_capacity.restype = ctypes.c_int64
     lib.moe_workspace_layout.argtypes = [P(Shape), vp, P(WsView)]
     lib.moe_workspace_layout.restype = st
     for name in ("moe_route", "moe_permute", "moe_combine", "moe_forward"):
@@ -94,8 +99,12 @@ def status_string(status: int) -> str:
 
 
 def make_shape(T: int, H: int, E: int, k: int, F: int, capacity_factor: float = math.inf, dtype: str = "bf16",
-               activation: str = "gelu") -> Shape:
-    return Shape(T, H, E, F, k, float(capacity_factor), DTYPES[dtype], ACTIVATIONS[activation])
+               activation: str = "gelu", routing: str = "token_choice") -> Shape:
+    return Shape(T, H, E, F, k, float(capacity_factor), DTYPES[dtype], ACTIVATIONS[activation], ROUTINGS[routing])
+
+
+def moe_capacity(shape: Shape) -> int:
+    return load_library().moe_capacity(ctypes.byref(shape))
 
 
 def _check(status: int, where: str) -> int:
@@ -176,10 +185,18 @@ class MoEBuffers:
         T, H, E, k = shape.T, shape.H, shape.E, shape.k
         self.inputs = inputs
         self.out = torch.empty((T, H), dtype=torch.float32, device=device)
-        self.topk_idx = torch.empty((T, k), dtype=torch.int32, device=device)
-        self.topk_w = torch.empty((T, k), dtype=torch.float32, device=device)
+        if shape.routing == MOE_ROUTING_EXPERT_CHOICE:
+            # expert choice: chosen tokens [E, C], softmax over all experts [T, E], per-token flags [T]
+            C = moe_capacity(shape)
+            if C < 0:
+                raise MoEError(MOE_ERR_INVALID_ARG, "moe_capacity")
+            idx_shape, w_shape, drop_shape = (E, C), (T, E), (T,)
+        else:
+            idx_shape, w_shape, drop_shape = (T, k), (T, k), (T, k)
+        self.topk_idx = torch.empty(idx_shape, dtype=torch.int32, device=device)
+        self.topk_w = torch.empty(w_shape, dtype=torch.float32, device=device)
         self.expert_counts = torch.empty((E,), dtype=torch.int32, device=device)
-        self.dropped = torch.empty((T, k), dtype=torch.uint8, device=device)
+        self.dropped = torch.empty(drop_shape, dtype=torch.uint8, device=device)
         self.losses = torch.empty((2,), dtype=torch.float32, device=device)
         self.ws_bytes = moe_workspace_size(shape)
         if self.ws_bytes == 0:

@@ -1,0 +1,245 @@
+// Expert-choice routing ("MoE Training: Mixture of Experts" page, Core Concepts 2, "Expert Choice
+// Routing"): the router's logits are read per expert and every expert takes the C tokens with the
+// largest logits (ties to the lower token index), so every expert holds exactly C rows.
+//
+//   ec_select_kernel   one 1024-thread block per expert: radix select of the C-th largest logit
+//                      (four 8-bit passes over order-preserving integer keys), then a stable
+//                      compaction in token order -> chosen[e][0..C) ascending; per-token counts of
+//                      the experts that chose it; the last block to finish writes dropped[t]
+//   ec_gather_kernel   x rows into x_perm (row e*C + j = j-th token of expert e), row maps,
+//                      offsets e*C, and clearing of out
+//   ec_combine_kernel  unfused combine: out[t] += p[t,e] * y[row] with fp32 atomics
+//
+// The expert FFN that runs between gather and combine is the token-choice one: row_slot holds the
+// expert and the combine weight of row r is topk_w[t * E + e] = p[t,e].
+#include "moe_internal.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kSelThreads = 1024;  // the block scans below assume exactly 32 warps
+
+// fp32 -> uint32 with the same order (larger float, larger key); -0 sorts just below +0
+__device__ __forceinline__ uint32_t order_key(float v) {
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Exclusive count of `flag` over the block's threads in thread order; the block total goes to
+// `total`.  `buf` holds at least 65 ints of shared memory.
+__device__ __forceinline__ int block_excl_count(bool flag, int* buf, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) buf[warp] = __popc(bal);
+  __syncthreads();
+  if (warp == 0) {
+    const int v = buf[lane];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    buf[32 + lane] = incl - v;
+    if (lane == 31) buf[64] = incl;
+  }
+  __syncthreads();
+  const int r = buf[32 + warp] + __popc(bal & ((1u << lane) - 1u));
+  total = buf[64];
+  __syncthreads();  // buf is reused by the next call
+  return r;
+}
+
+__global__ void __launch_bounds__(kSelThreads) ec_select_kernel(EcSelectArgs a) {
+  __shared__ int hist[256];
+  __shared__ int buf[72];
+  __shared__ uint32_t sel_digit;
+  __shared__ int sel_need;
+  __shared__ int is_last;
+  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int T = a.T, C = a.C;
+  const float* sc = a.scores + (size_t)e * T;
+  const bool all = C >= T;
+
+  // Radix select, most significant digit first.  Invariant: at least `need` of the tokens whose key
+  // matches `prefix` under `mask` remain, and exactly C - need tokens have a larger key.
+  uint32_t prefix = 0, mask = 0;
+  int need = C;
+  if (!all) {
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
+      __syncthreads();
+      for (int t = tid; t < T; t += kSelThreads) {
+        const uint32_t key = order_key(sc[t]);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l holds digits 255-8l .. 248-8l (largest first); the first lane whose running
+        // count from the top reaches `need` holds the digit of the C-th largest key
+        int cnt[8], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          cnt[j] = hist[255 - 8 * lane - j];
+          sum += cnt[j];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += n;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+        if (lane == __ffs(hit) - 1) {
+          int run = incl - sum;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (run + cnt[j] >= need) {
+              sel_digit = (uint32_t)(255 - 8 * lane - j);
+              sel_need = need - run;
+              break;
+            }
+            run += cnt[j];
+          }
+        }
+      }
+      __syncthreads();
+      prefix |= sel_digit << shift;
+      mask |= 255u << shift;
+      need = sel_need;
+      __syncthreads();  // hist and sel_* are rewritten by the next pass
+    }
+  }
+  const uint32_t thr = prefix;  // the C-th largest key; `need` tokens equal to it are taken
+
+  // Stable compaction in token order: every key above thr, and the first `need` keys equal to it.
+  int base_eq = 0, base_sel = 0;
+  for (int t0 = 0; t0 < T; t0 += kSelThreads) {
+    const int t = t0 + tid;
+    const uint32_t key = t < T ? order_key(sc[t]) : 0u;
+    const bool gt = t < T && (all || key > thr);
+    const bool eq = t < T && !all && key == thr;
+    int tot_eq, tot_sel;
+    const int r_eq = base_eq + block_excl_count(eq, buf, tot_eq);
+    const bool take = gt || (eq && r_eq < need);
+    const int pos = base_sel + block_excl_count(take, buf, tot_sel);
+    if (take) {
+      a.chosen[(size_t)e * C + pos] = t;
+      atomicAdd(&a.tok_count[t], 1);
+    }
+    base_eq += tot_eq;
+    base_sel += tot_sel;
+  }
+  if (tid == 0) {
+    a.expert_counts[e] = C;
+    a.cnt_pre[e] = C;
+  }
+
+  // The last block to finish sees every expert's counts and writes the per-token flags.
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(a.done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    for (int t = tid; t < T; t += kSelThreads) a.dropped[t] = __ldcg(&a.tok_count[t]) == 0 ? 1 : 0;
+    if (tid == 0) *a.done = 0u;  // ready for the next call on this workspace
+  }
+}
+
+// 32 rows per 256-thread block: row maps, 16-byte copies of the x rows into x_perm (8 loads in
+// flight per thread), and a grid-stride clear of out.
+__global__ void __launch_bounds__(256) ec_gather_kernel(EcGatherArgs a) {
+  __shared__ int tok_s[32];
+  const int tid = threadIdx.x;
+  const long long rows = (long long)a.E * a.C;
+  const long long r0 = (long long)blockIdx.x * 32;
+  if (tid < 32) {
+    const long long r = r0 + tid;
+    int t = -1;
+    if (r < rows) {
+      t = a.chosen[r];
+      a.row_token[r] = t;
+      a.row_slot[r] = (int)(r / a.C);
+    }
+    tok_s[tid] = t;
+  }
+  if (blockIdx.x == 0)
+    for (int e = tid; e <= a.E; e += 256) a.offsets[e] = e * a.C;
+  __syncthreads();
+  const int nvec = a.H * a.esize / 16;
+  const uint4* xv = reinterpret_cast<const uint4*>(a.x);
+  uint4* pv = reinterpret_cast<uint4*>(a.x_perm);
+  const int total = 32 * nvec;
+  constexpr int U = 8;
+  for (int i = tid; i < total; i += 256 * U) {
+    uint4 v[U];
+    int ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int idx = i + u * 256;
+      ok[u] = 0;
+      if (idx < total) {
+        const int r = idx / nvec, c = idx % nvec;
+        if (tok_s[r] >= 0) {
+          v[u] = xv[(size_t)tok_s[r] * nvec + c];
+          ok[u] = 1;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u)
+      if (ok[u]) {
+        const int idx = i + u * 256;
+        const int r = idx / nvec, c = idx % nvec;
+        pv[(size_t)(r0 + r) * nvec + c] = v[u];
+      }
+  }
+  const long long ovec = (long long)a.T * a.H / 4;
+  float4* o = reinterpret_cast<float4*>(a.out);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long i = (long long)blockIdx.x * 256 + tid; i < ovec; i += (long long)gridDim.x * 256) o[i] = z;
+}
+
+// One block per row: out[t] += p[t,e] * y[row] (fp32 atomics; up to E rows meet in a token).
+__global__ void __launch_bounds__(256) ec_combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ row_token,
+                                                         const int32_t* __restrict__ row_slot,
+                                                         const float* __restrict__ topk_w, int E, int H,
+                                                         float* __restrict__ out) {
+  const int r = blockIdx.x;
+  const int t = row_token[r];
+  const float w = topk_w[(size_t)t * E + row_slot[r]];
+  const float4* yv = reinterpret_cast<const float4*>(y) + (size_t)r * (H / 4);
+  float* o = out + (size_t)t * H;
+  for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
+    const float4 v = yv[c];
+    atomicAdd(o + 4 * c + 0, w * v.x);
+    atomicAdd(o + 4 * c + 1, w * v.y);
+    atomicAdd(o + 4 * c + 2, w * v.z);
+    atomicAdd(o + 4 * c + 3, w * v.w);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st) {
+  ec_select_kernel<<<a.E, kSelThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st) {
+  const long long rows = (long long)a.E * a.C;
+  const int grid = (int)((rows + 31) / 32);
+  ec_gather_kernel<<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ec_combine(const float* y, const int32_t* row_token, const int32_t* row_slot, const float* topk_w,
+                              int rows, int E, int H, float* out, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  ec_combine_kernel<<<rows, 256, 0, st>>>(y, row_token, row_slot, topk_w, E, H, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -997,7 +997,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.k = a.k;
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
-  const long long avg_rows = (long long)a.T * a.k / a.E;
+  const long long avg_rows = a.avg_rows;
   cudaError_t err = a.act == MOE_ACT_SILU ? launch_bn<EPI_SILU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st)
                                           : launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st);
   if (err != cudaSuccess) return err;

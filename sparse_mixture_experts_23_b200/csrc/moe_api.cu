@@ -38,13 +38,23 @@ cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
   return err;
 }
 
+// Tokens per expert under expert choice: min(T, ceil(CF*T*k/E)), T when CF = +inf.
+long long ec_capacity(const moe_shape_t& s) {
+  if (isinf(s.capacity_factor)) return s.T;
+  const double c = ceil(s.capacity_factor * (double)s.T * (double)s.k / (double)s.E);
+  return c < (double)s.T ? (long long)c : (long long)s.T;
+}
+
 WsLayout ws_layout(const moe_shape_t& s) {
   WsLayout L{};
   const size_t T = (size_t)s.T, E = (size_t)s.E, k = (size_t)s.k;
   const size_t es = s.dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  const bool ec = s.routing == MOE_ROUTING_EXPERT_CHOICE;
   L.nblk = (int)((T + kChunk - 1) / kChunk);
   const size_t nblk = (size_t)L.nblk;
-  const size_t rows = T * k;
+  L.ec_cap = ec ? (int)ec_capacity(s) : 0;
+  const size_t rows = ec ? E * (size_t)L.ec_cap : T * k;
+  L.rows = (long long)rows;
   size_t o = 0;
   L.status = o;
   o = align256(o + 16);
@@ -70,6 +80,10 @@ WsLayout ws_layout(const moe_shape_t& s) {
   o = align256(o + rows * (size_t)s.F * es);
   L.y = o;
   o = align256(o + rows * (size_t)s.H * 4);
+  L.scores = o;  // expert choice: [E][T] fp32 logits, then [T] per-token expert counts
+  o = align256(o + (ec ? E * T * 4 : 0));
+  L.tok_count = o;
+  o = align256(o + (ec ? T * 4 : 0));
   L.total = o;
   return L;
 }
@@ -92,9 +106,11 @@ moe_status_t check_shape(const moe_shape_t* s) {
   if (!(s->capacity_factor > 0.0)) return MOE_ERR_INVALID_ARG;  // also rejects NaN
   if (s->dtype != MOE_DTYPE_F32 && s->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
   if (s->activation != MOE_ACT_GELU && s->activation != MOE_ACT_SILU) return MOE_ERR_INVALID_ARG;
+  if (s->routing != MOE_ROUTING_TOKEN_CHOICE && s->routing != MOE_ROUTING_EXPERT_CHOICE) return MOE_ERR_INVALID_ARG;
   if (s->dtype == MOE_DTYPE_BF16 && (s->H % 64 != 0 || s->F % 64 != 0)) return MOE_ERR_UNSUPPORTED;
   if (s->dtype == MOE_DTYPE_F32 && (s->H % 4 != 0 || s->F % 4 != 0)) return MOE_ERR_UNSUPPORTED;
-  const long long rows = (long long)s->T * s->k;
+  const long long rows =
+      s->routing == MOE_ROUTING_EXPERT_CHOICE ? (long long)s->E * ec_capacity(*s) : (long long)s->T * s->k;
   const long long widest = s->H > s->F ? s->H : s->F;
   if (rows * widest >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -133,6 +149,7 @@ int num_sms() {
 }
 
 // ---------------------------------------------------------------- stage bodies (validated) -------
+ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int do_losses, int do_dispatch);
 moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, bool emit_hist) {
   const WsLayout L = ws_layout(*s);
   if (s->T == 0) {
@@ -152,10 +169,56 @@ moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaSt
   r.loss_part = at<float>(ws, L.loss_part);
   r.chunk_hist = at<int32_t>(ws, L.chunk_hist);
   (void)emit_hist;
+  if (s->routing == MOE_ROUTING_EXPERT_CHOICE) {
+    r.chunk_hist = nullptr;
+    r.scores = at<float>(ws, L.scores);
+    r.tok_count = at<int32_t>(ws, L.tok_count);
+  }
   cudaError_t err = launch_router(r, s->dtype, st);
   ++g_launches;
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
+}
+
+// Expert choice, after the router: per-expert top-C selection, then the losses.
+moe_status_t do_ec_select_and_losses(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(*s);
+  EcSelectArgs a{};
+  a.scores = at<float>(ws, L.scores);
+  a.T = s->T;
+  a.E = s->E;
+  a.C = L.ec_cap;
+  a.chosen = io->topk_idx;
+  a.expert_counts = io->expert_counts;
+  a.cnt_pre = at<int32_t>(ws, L.cnt_pre);
+  a.tok_count = at<int32_t>(ws, L.tok_count);
+  a.dropped = io->dropped;
+  a.done = at<unsigned>(ws, L.status + kEcDoneOffset);
+  ++g_launches;
+  if (launch_ec_select(a, st) != cudaSuccess) return MOE_ERR_CUDA;
+  ReduceArgs ra = reduce_args(s, io, ws, 1, 0);
+  ra.ec_count = L.ec_cap;
+  ++g_launches;
+  return cuda_status(launch_reduce(ra, st));
+}
+
+moe_status_t do_ec_gather(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(*s);
+  EcGatherArgs a{};
+  a.x = io->x;
+  a.T = s->T;
+  a.H = s->H;
+  a.E = s->E;
+  a.C = L.ec_cap;
+  a.esize = s->dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  a.chosen = io->topk_idx;
+  a.offsets = at<int32_t>(ws, L.offsets);
+  a.row_token = at<int32_t>(ws, L.row_token);
+  a.row_slot = at<int32_t>(ws, L.row_slot);
+  a.x_perm = at<void>(ws, L.x_perm);
+  a.out = io->out;
+  ++g_launches;
+  return cuda_status(launch_ec_gather(a, st));
 }
 
 ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int do_losses, int do_dispatch) {
@@ -211,7 +274,11 @@ moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse
   a.E = s->E;
   a.F = s->F;
   a.k = s->k;
-  a.rows_cap = s->T * s->k;
+  const bool ec = s->routing == MOE_ROUTING_EXPERT_CHOICE;
+  a.rows_cap = (int)L.rows;
+  // under expert choice row_slot holds the expert, so the weight of row r is topk_w[t*E + e]
+  if (ec) a.k = s->E;
+  a.avg_rows = ec ? L.ec_cap : (long long)s->T * s->k / s->E;
   a.offsets = at<int32_t>(ws, L.offsets);
   a.row_token = at<int32_t>(ws, L.row_token);
   a.row_slot = at<int32_t>(ws, L.row_slot);
@@ -248,6 +315,13 @@ size_t moe_workspace_size(const moe_shape_t* shape) {
   return ws_layout(*shape).total;
 }
 
+int64_t moe_capacity(const moe_shape_t* shape) {
+  if (check_shape(shape) != MOE_OK) return -2;
+  if (shape->routing == MOE_ROUTING_EXPERT_CHOICE) return ec_capacity(*shape);
+  if (isinf(shape->capacity_factor)) return -1;
+  return (int64_t)ceil(shape->capacity_factor * (double)shape->T * (double)shape->k / (double)shape->E);
+}
+
 moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, moe_ws_view_t* view) {
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
@@ -263,6 +337,7 @@ moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, moe_ws_vie
   view->h = at<void>(ws, L.h);
   view->y = at<float>(ws, L.y);
   view->bytes = L.total;
+  view->scores = shape->routing == MOE_ROUTING_EXPERT_CHOICE ? at<float>(ws, L.scores) : nullptr;
   return MOE_OK;
 }
 
@@ -273,10 +348,18 @@ moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, s
   if (io == nullptr) return MOE_ERR_INVALID_ARG;
   if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
   if (null_any({io->aux_loss, io->z_loss})) return MOE_ERR_INVALID_ARG;
-  if (shape->T == 0) return do_route(shape, io, ws, stream, true);
+  const bool ec = shape->routing == MOE_ROUTING_EXPERT_CHOICE;
+  if (ec && null_any({io->expert_counts})) return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) {
+    if (!ec) return do_route(shape, io, ws, stream, true);
+    ++g_launches;
+    return cuda_status(launch_zero_outputs(io->expert_counts, shape->E, io->aux_loss, io->z_loss, stream));
+  }
   if (null_any({io->x, io->Wg, io->topk_idx, io->topk_w})) return MOE_ERR_INVALID_ARG;  // bg optional
+  if (ec && null_any({io->dropped})) return MOE_ERR_INVALID_ARG;
   if (!aligned16(io->x) || !aligned16(io->Wg)) return MOE_ERR_INVALID_ARG;
   if ((st = do_route(shape, io, ws, stream, true)) != MOE_OK) return st;
+  if (ec) return do_ec_select_and_losses(shape, io, ws, stream);
   ++g_launches;
   return cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 0), stream));
 }
@@ -292,6 +375,11 @@ moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   if (shape->T == 0) {
     ++g_launches;
     return cuda_status(launch_zero_outputs(io->expert_counts, shape->E, nullptr, nullptr, stream));
+  }
+  if (shape->routing == MOE_ROUTING_EXPERT_CHOICE) {
+    if (null_any({io->x, io->topk_idx, io->out})) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(io->x) || !aligned16(io->out)) return MOE_ERR_INVALID_ARG;
+    return do_ec_gather(shape, io, ws, stream);
   }
   if (null_any({io->x, io->topk_idx, io->dropped, io->out})) return MOE_ERR_INVALID_ARG;
   if (!aligned16(io->x) || !aligned16(io->out)) return MOE_ERR_INVALID_ARG;
@@ -332,6 +420,9 @@ moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   if (!aligned16(io->out)) return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*shape);
   ++g_launches;
+  if (shape->routing == MOE_ROUTING_EXPERT_CHOICE)
+    return cuda_status(launch_ec_combine(at<float>(ws, L.y), at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_slot),
+                                         io->topk_w, (int)L.rows, shape->E, shape->H, io->out, stream));
   return cuda_status(launch_combine(at<float>(ws, L.y), at<int32_t>(ws, L.row_of), io->topk_w, shape->T, shape->H,
                                     shape->k, io->out, stream));
 }
@@ -352,6 +443,13 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   if (!aligned16(io->x) || !aligned16(io->Wg) || !aligned16(io->W1) || !aligned16(io->W2) || !aligned16(io->out) ||
       !aligned16(io->b1) || !aligned16(io->b2))
     return MOE_ERR_INVALID_ARG;
+  if (shape->routing == MOE_ROUTING_EXPERT_CHOICE) {
+    // router, per-expert selection, losses, gather, GEMM1, GEMM2 (each call adds its launches)
+    if ((st = do_route(shape, io, ws, stream, false)) != MOE_OK) return st;
+    if ((st = do_ec_select_and_losses(shape, io, ws, stream)) != MOE_OK) return st;
+    if ((st = do_ec_gather(shape, io, ws, stream)) != MOE_OK) return st;
+    return do_ffn(shape, io, ws, 1, stream);
+  }
   int n = 0;
   // router emits the chunk histograms itself, so one reduction serves losses and dispatch
   if ((st = do_route(shape, io, ws, stream, true)) != MOE_OK) return st;

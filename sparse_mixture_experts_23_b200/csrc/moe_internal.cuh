@@ -26,9 +26,14 @@ enum DevError : int {
 // Workspace sections (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
   size_t status, offsets, cnt_pre, chunk_hist, chunk_base, loss_part, row_of, row_token, row_slot, x_perm, h, y,
-      total;
-  int nblk;  // router chunks = ceil(T / kChunk)
+      scores, tok_count, total;
+  int nblk;       // router chunks = ceil(T / kChunk)
+  long long rows; // rows of x_perm / h / y: T*k, or E*C under expert choice
+  int ec_cap;     // C under expert choice, else 0
 };
+
+// Workspace word (next to the device error word) counting finished expert-choice selection blocks.
+constexpr size_t kEcDoneOffset = 4;
 
 WsLayout ws_layout(const moe_shape_t& s);
 
@@ -41,10 +46,37 @@ struct RouterArgs {
   float* topk_w;
   float* loss_part;    // [nblk][E+1]: sum_t p[t,e] (E values) then sum_t lse_t^2
   int32_t* chunk_hist; // [k][nblk][E] or null
+  // expert choice (non-null scores): no top-k; p goes to topk_w[T,E], logits to scores[E,T], and
+  // tok_count[t] is cleared for the selection that follows
+  float* scores;
+  int32_t* tok_count;
+};
+
+struct EcSelectArgs {
+  const float* scores;  // [E][T] router logits
+  int T, E, C;
+  int32_t* chosen;      // [E][C] out: chosen tokens, ascending
+  int32_t* expert_counts;
+  int32_t* cnt_pre;
+  int32_t* tok_count;   // [T] experts that chose each token (cleared by the router)
+  uint8_t* dropped;     // [T] out: 1 = chosen by no expert
+  unsigned* done;       // finished-block counter, 0 between calls
+};
+
+struct EcGatherArgs {
+  const void* x;
+  int T, H, E, C, esize;
+  const int32_t* chosen;  // [E][C]
+  int32_t* offsets;       // [E+1] out: e*C
+  int32_t* row_token;     // [E*C] out
+  int32_t* row_slot;      // [E*C] out: the expert
+  void* x_perm;           // [E*C][H] out
+  float* out;             // [T][H] cleared
 };
 
 struct ReduceArgs {
   int T, E, k, nblk;
+  int ec_count;  // > 0: expert choice, every expert holds ec_count rows (no histogram, no dispatch)
   long long cap;  // < 0: unlimited
   const float* loss_part;
   int32_t* chunk_hist;  // [k][nblk][E]
@@ -74,7 +106,8 @@ struct ScatterArgs {
 
 struct FfnArgs {
   int T, H, E, F, k;
-  int rows_cap;  // T*k: height of x_perm / h / y
+  int rows_cap;  // height of x_perm / h / y: T*k, or E*C under expert choice
+  long long avg_rows;  // expected rows per expert (T*k/E, or C), for the tile-shape choice
   const int32_t* offsets;
   const int32_t* row_token;
   const int32_t* row_slot;
@@ -104,6 +137,10 @@ cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
 cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);
 cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t st, int* launches);
+cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st);
+cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st);
+cudaError_t launch_ec_combine(const float* y, const int32_t* row_token, const int32_t* row_slot, const float* topk_w,
+                              int rows, int E, int H, float* out, cudaStream_t st);
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int T, int H, int k, float* out,
                            cudaStream_t st);

@@ -64,10 +64,13 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   if (moe_workspace_size(shape) == 0) {
     if (shape->T < 0 || shape->H <= 0 || shape->E <= 0 || shape->F <= 0 || shape->k <= 0 || shape->k > shape->E ||
         shape->k > 8 || shape->E > 256 || !(shape->capacity_factor > 0.0) ||
-        (shape->dtype != MOE_DTYPE_F32 && shape->dtype != MOE_DTYPE_BF16))
+        (shape->dtype != MOE_DTYPE_F32 && shape->dtype != MOE_DTYPE_BF16) ||
+        (shape->activation != MOE_ACT_GELU && shape->activation != MOE_ACT_SILU) ||
+        (shape->routing != MOE_ROUTING_TOKEN_CHOICE && shape->routing != MOE_ROUTING_EXPERT_CHOICE))
       return MOE_ERR_INVALID_ARG;
     return MOE_ERR_UNSUPPORTED;
   }
+  if (shape->routing != MOE_ROUTING_TOKEN_CHOICE) return MOE_ERR_UNSUPPORTED;  // the selection needs a workspace
   if (io->aux_loss == nullptr || io->z_loss == nullptr) return MOE_ERR_INVALID_ARG;
   size_t hist_off = 0, cnt_off = 0;
   if (scratch_bytes(shape, &hist_off, &cnt_off) > kScratchBytes)

@@ -105,6 +105,20 @@ __device__ void router_finish(const RouterArgs& a, const float* logits, int epad
       if (j < NJ && lane + 32 * j < E) pacc[j] += expf(lv[j] - m) * inv_s;
     zacc += lse * lse;
 
+    if (a.scores != nullptr) {
+      // expert choice: every probability is a combine weight, the logits go out expert-major
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        if (j < NJ && e < E) {
+          a.topk_w[(size_t)t * E + e] = expf(lv[j] - m) * inv_s;
+          a.scores[(size_t)e * T + t] = lv[j];
+        }
+      }
+      if (lane == 0) a.tok_count[t] = 0;
+      continue;
+    }
+
     // top-k: k rounds of a warp arg-max with ties to the lower index
     unsigned taken = 0;
     float psel_sum = 0.f;
@@ -797,38 +811,47 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
   const int c0 = in ? (int)((long long)C * g / G) : 0;
   const int c1 = in ? (int)((long long)C * (g + 1) / G) : 0;
 
-  int s = 0;
-  for (int c = c0; c < c1; ++c) s += a.chunk_hist[(size_t)c * E + e];
-  if (in) gsum[g * E + e] = s;
-  __syncthreads();
-  // exclusive scan of the G group sums of each expert: warp w scans experts w, w+32, ...; lane l
-  // owns a contiguous run of groups, then a shuffle scan across the lanes (exact integer sums)
-  {
-    const int warp = tid >> 5, lane = tid & 31;
-    const int gpl = (G + 31) / 32;  // groups per lane
-    for (int ee = warp; ee < E; ee += 32) {
-      const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
-      int local = 0;
-      for (int q = q0; q < q1; ++q) local += gsum[q * E + ee];
-      int incl = local;
+  if (a.ec_count > 0) {
+    // expert choice: every expert holds exactly ec_count rows
+    for (int q = tid; q < E; q += 1024) {
+      cnt_s[q] = a.ec_count;
+      a.cnt_pre[q] = a.ec_count;
+    }
+    __syncthreads();
+  } else {
+    int s = 0;
+    for (int c = c0; c < c1; ++c) s += a.chunk_hist[(size_t)c * E + e];
+    if (in) gsum[g * E + e] = s;
+    __syncthreads();
+    // exclusive scan of the G group sums of each expert: warp w scans experts w, w+32, ...; lane l
+    // owns a contiguous run of groups, then a shuffle scan across the lanes (exact integer sums)
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      const int gpl = (G + 31) / 32;  // groups per lane
+      for (int ee = warp; ee < E; ee += 32) {
+        const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
+        int local = 0;
+        for (int q = q0; q < q1; ++q) local += gsum[q * E + ee];
+        int incl = local;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      int run = incl - local;
-      for (int q = q0; q < q1; ++q) {
-        const int v = gsum[q * E + ee];
-        gsum[q * E + ee] = run;
-        run += v;
-      }
-      if (lane == 31) {
-        cnt_s[ee] = incl;
-        a.cnt_pre[ee] = incl;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int q = q0; q < q1; ++q) {
+          const int v = gsum[q * E + ee];
+          gsum[q * E + ee] = run;
+          run += v;
+        }
+        if (lane == 31) {
+          cnt_s[ee] = incl;
+          a.cnt_pre[ee] = incl;
+        }
       }
     }
+    __syncthreads();
   }
-  __syncthreads();
   if (a.do_dispatch && in) {
     int run = gsum[g * E + e];
     for (int c = c0; c < c1; ++c) {
@@ -883,7 +906,9 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
         for (int q = q0; q < q1; ++q) P += pf[q * E + ee];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) P += __shfl_xor_sync(0xffffffffu, P, o);
-        if (lane == 0) term[ee] = ((double)cnt_s[ee] / ((double)a.T * a.k)) * ((double)P / (double)a.T);
+        // f_e = count_e / (all assignments): T*k, or E*C under expert choice
+        const double n_assign = a.ec_count > 0 ? (double)E * a.ec_count : (double)a.T * a.k;
+        if (lane == 0) term[ee] = ((double)cnt_s[ee] / n_assign) * ((double)P / (double)a.T);
       }
     }
     __syncthreads();

@@ -7,8 +7,8 @@ dtype.  Values are produced on the host so that the CUDA path and the oracle see
 
 The workload recipes (``CONFIGS``) restate the synthetic layer shapes used for parity and
 measurement: a tiny fp32 layer, a decode-sized layer, a Switch-style training layer with a capacity
-factor, a Mixtral-shaped layer, a skewed-load layer, and the Mixtral block's own expert variant
-(bias-free, SiLU) at the Mixtral shape.  Shapes follow the pages' DeepSpeed
+factor, a Mixtral-shaped layer, a skewed-load layer, the Mixtral block's own expert variant
+(bias-free, SiLU) and expert-choice routing, both at the Mixtral shape.  Shapes follow the pages' DeepSpeed
 launch examples ("MoE Training" skill page, Quick Start / Training Script sections) where they give
 them.
 """
@@ -122,6 +122,7 @@ class LayerConfig:
     note: str = ""
     act: str = "gelu"  # expert activation: "gelu" (Quick Start expert) or "silu" (Mixtral block)
     bias: bool = True  # False: gate and experts have no bias at all (bg = b1 = b2 = None)
+    routing: str = "token_choice"  # or "expert_choice" (every expert takes its top-C tokens)
 
     @property
     def x_std(self) -> float:
@@ -150,6 +151,9 @@ CONFIGS = {
     "mixtral_block": LayerConfig("mixtral_block", T=4096, H=4096, E=8, k=2, F=14336, CF=math.inf, dtype="bf16",
                                  seed=6, act="silu", bias=False,
                                  note="the Mixtral block's own expert: bias-free gate and Linear layers, SiLU"),
+    "mixtral_ec": LayerConfig("mixtral_ec", T=4096, H=4096, E=8, k=2, F=14336, CF=1.0, dtype="bf16", seed=7,
+                              routing="expert_choice",
+                              note="expert-choice routing at the Mixtral shape: C = T*k/E = 1024 tokens per expert"),
 }
 
 

@@ -88,9 +88,9 @@ def test_bad_dtype_enum(lib):
 
 
 def test_activation_field(lib):
-    """moe_shape_t keeps its 40-byte layout: the activation sits in the tail after dtype, and a
-    zero-initialised shape means GELU; unknown activations are rejected before any launch."""
-    assert ctypes.sizeof(moe.Shape) == 40 and moe.Shape.activation.offset == 36
+    """The activation sits right after dtype, and a zero-initialised shape means GELU; unknown
+    activations are rejected before any launch."""
+    assert ctypes.sizeof(moe.Shape) == 48 and moe.Shape.activation.offset == 36
     assert moe.Shape().activation == moe.MOE_ACT_GELU
     s = _shape()
     assert moe.moe_workspace_size(s) > 0
@@ -165,3 +165,43 @@ def test_missing_library_fails_loudly(tmp_path):
             m.load_library(str(tmp_path / "nope.so"))
     finally:
         m._lib = saved
+
+
+def test_routing_field_and_capacity(lib):
+    """moe_shape_t.routing follows activation; zero means token choice.  moe_capacity gives the
+    per-expert capacity of either rule; unknown rules are rejected before any launch."""
+    assert moe.Shape.routing.offset == 40 and moe.Shape().routing == moe.MOE_ROUTING_TOKEN_CHOICE
+    s = _shape(T=4096, H=64, E=8, k=2, F=64, capacity_factor=1.0)
+    assert moe.moe_capacity(s) == 1024
+    s.routing = moe.MOE_ROUTING_EXPERT_CHOICE
+    assert moe.moe_capacity(s) == 1024
+    s.capacity_factor = math.inf
+    assert moe.moe_capacity(s) == 4096  # every expert sees every token
+    s.routing = moe.MOE_ROUTING_TOKEN_CHOICE
+    assert moe.moe_capacity(s) == -1  # no limit
+    s.capacity_factor = 100.0
+    s.routing = moe.MOE_ROUTING_EXPERT_CHOICE
+    assert moe.moe_capacity(s) == 4096  # never more than T
+    s.routing = 2
+    assert moe.moe_capacity(s) == -2 and moe.moe_workspace_size(s) == 0
+    for fn in (moe.moe_route, moe.moe_permute, moe.moe_combine, moe.moe_forward):
+        assert fn(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_route_noalloc(s, _io()) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_expert_choice_workspace_and_layout(lib):
+    """Under expert choice the row buffers hold E*C rows and the workspace gains the [E,T] score
+    matrix; the view publishes it (NULL under token choice)."""
+    tc = _shape(T=100, H=128, E=8, k=2, F=512, dtype="bf16", capacity_factor=2.0)
+    ec = _shape(T=100, H=128, E=8, k=2, F=512, dtype="bf16", capacity_factor=2.0)
+    ec.routing = moe.MOE_ROUTING_EXPERT_CHOICE
+    C = moe.moe_capacity(ec)
+    assert C == 50
+    v_tc = moe.moe_workspace_layout(tc, FAKE)
+    v_ec = moe.moe_workspace_layout(ec, FAKE)
+    assert v_tc.scores is None and v_ec.scores is not None
+    assert v_ec.h - v_ec.x_perm >= 8 * C * 128 * 2 and v_ec.y - v_ec.h >= 8 * C * 512 * 2
+    assert v_ec.scores - v_ec.y >= 8 * C * 128 * 4
+    assert FAKE + v_ec.bytes - v_ec.scores >= 8 * 100 * 4 + 100 * 4
+    # the no-workspace router does not take expert choice
+    assert moe.moe_route_noalloc(ec, _io()) == moe.MOE_ERR_UNSUPPORTED

@@ -1,0 +1,228 @@
+"""Parity of expert-choice routing ("MoE Training: Mixture of Experts" page, Core Concepts 2, "Expert
+Choice Routing") on the GPU against the fp64 oracle, through the C ABI.
+
+Checks, per workload:
+  route    -> the router's fp32 logits (published in the workspace) against the oracle's, normwise
+              1e-4; the chosen tokens of every expert bit-exact against a top-C of those same fp32
+              logits (the integer decision taken in the kernel's precision), and bit-exact against
+              the oracle's fp64 choice for every expert whose C-th/(C+1)-th logit gap is >= 1e-4;
+              softmax weights 1e-4 relative; counts == C; per-token "chosen by none" flags exact;
+              losses 1e-3
+  permute  -> row maps, offsets and permuted rows bit-exact
+  ffn      -> out against the oracle's expert-choice combine of the GPU's choice, tolerance of the
+              storage dtype; tokens chosen by no expert exactly zero
+  forward  -> moe_forward (6 launches) gives the same choice and, up to the order of the fp32
+              atomic adds, the same out; the unfused FFN + moe_combine agrees as well
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from moe_testlib import NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, normwise_rel, out_error, sample_tokens, shape_of, upload
+
+pytestmark = pytest.mark.gpu
+
+
+def _cfg(name, T, H, E, k, F, CF, dtype, seed, **kw):
+    return synth.LayerConfig(name, T=T, H=H, E=E, k=k, F=F, CF=CF, dtype=dtype, seed=seed, routing="expert_choice",
+                             **kw)
+
+
+CASES = [
+    _cfg("ec_tiny_f32", 256, 64, 4, 2, 256, 1.0, "f32", 41),
+    _cfg("ec_ragged_bf16", 100, 128, 6, 3, 192, 1.0, "bf16", 42),       # C = 50, single-CTA tiles
+    _cfg("ec_pair_tiles", 1500, 256, 4, 2, 512, 1.1, "bf16", 43),        # C = 825: CTA-pair + half tiles
+    _cfg("ec_all_tokens", 77, 64, 5, 2, 64, math.inf, "bf16", 44),       # C = T: dense mixture
+    _cfg("ec_silu_nobias", 300, 256, 8, 2, 512, 1.25, "bf16", 45, act="silu", bias=False),
+    _cfg("ec_many_experts", 2048, 128, 64, 2, 128, 1.0, "bf16", 46),    # C = 64
+    synth.CONFIGS["mixtral_ec"],                                        # C = 1024 at the Mixtral shape
+]
+SAMPLES = {"mixtral_ec": 24}
+
+
+def _lib():
+    import sparse_mixture_experts_23_b200 as moe
+    from sparse_mixture_experts_23_b200 import build as moe_build
+
+    moe_build.build()
+    return moe
+
+
+def _topC_fp32(scores: np.ndarray, C: int) -> np.ndarray:
+    """Top-C tokens of every row of an [E, T] float32 matrix by (score desc, token asc), ascending."""
+    E, T = scores.shape
+    out = np.empty((E, C), np.int32)
+    for e in range(E):
+        order = np.lexsort((np.arange(T), -scores[e].astype(np.float64)))  # exact for float32 values
+        out[e] = np.sort(order[:C])
+    return out
+
+
+@pytest.fixture(scope="module", params=CASES, ids=lambda c: c.name)
+def run(request):
+    import torch
+
+    moe = _lib()
+    cfg = request.param
+    inp = synth.make_inputs(cfg)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    T, E, H = cfg.T, cfg.E, cfg.H
+    C = moe.moe_capacity(buf.shape)
+    res = {"cfg": cfg, "inp": inp, "C": C}
+    buf.route()
+    torch.cuda.synchronize()
+    v = buf.view()
+    wsb = buf.ws
+
+    def ws_arr(ptr, n, dt):
+        off = ptr - buf.ws_ptr
+        nb = n * torch.tensor([], dtype=dt).element_size()
+        return wsb[off:off + nb].view(dt).cpu().numpy()
+
+    res["scores"] = ws_arr(v.scores, E * T, torch.float32).reshape(E, T)
+    res["chosen"] = buf.topk_idx.cpu().numpy()
+    res["p"] = buf.topk_w.cpu().numpy()
+    res["dropped"] = buf.dropped.cpu().numpy()
+    res["counts"] = buf.expert_counts.cpu().numpy()
+    res["losses"] = buf.losses.cpu().numpy().copy()
+    buf.permute()
+    torch.cuda.synchronize()
+    rows = E * C
+    res["offsets"] = ws_arr(v.offsets, E + 1, torch.int32)
+    res["row_token"] = ws_arr(v.row_token, rows, torch.int32)
+    res["row_slot"] = ws_arr(v.row_slot, rows, torch.int32)
+    es = 2 if cfg.dtype == "bf16" else 4
+    off = v.x_perm - buf.ws_ptr
+    xp = wsb[off:off + rows * H * es].view(torch.bfloat16 if es == 2 else torch.float32)
+    res["x_perm"] = from_device_bits(xp, cfg.dtype).reshape(rows, H)
+    buf.expert_ffn(fuse_combine=True)
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+    res["out"] = buf.out.cpu().numpy().copy()
+    # unfused: y in the workspace, then the standalone combine into the zeros moe_permute leaves
+    buf.permute()
+    buf.expert_ffn(fuse_combine=False)
+    buf.combine()
+    torch.cuda.synchronize()
+    res["out_unfused"] = buf.out.cpu().numpy().copy()
+    # the whole pass in one call
+    buf.out.fill_(float("nan"))
+    buf.topk_idx.fill_(-1)
+    buf.forward()
+    torch.cuda.synchronize()
+    res["launches"] = moe.moe_last_launch_count()
+    assert buf.device_status() == moe.MOE_OK
+    res["out_forward"] = buf.out.cpu().numpy().copy()
+    res["chosen_forward"] = buf.topk_idx.cpu().numpy()
+    res["ref"] = oracle.route(inp.x, inp.Wg, inp.bg, 1, cfg.dtype)
+    del buf
+    torch.cuda.empty_cache()
+    return res
+
+
+def test_ec_scores_match_oracle_logits(run):
+    err = normwise_rel(run["scores"].T.astype(np.float64), run["ref"].logits)
+    assert err <= 1e-4, err
+
+
+def test_ec_choice_exact_in_kernel_precision(run):
+    assert np.array_equal(run["chosen"], _topC_fp32(run["scores"], run["C"]))
+
+
+def test_ec_choice_matches_oracle_except_near_ties(run):
+    cfg, C = run["cfg"], run["C"]
+    assert C == oracle.ec_capacity(cfg.CF, cfg.T, cfg.k, cfg.E)
+    ec = oracle.expert_choice(run["ref"].logits, C)
+    near = ec.margin < NEAR_TIE
+    same = (run["chosen"] == ec.chosen).all(axis=1)
+    print(f"{cfg.name}: C={C}, experts with a near tie at the boundary: {int(near.sum())} / {cfg.E}, "
+          f"differing among them: {int((~same & near).sum())}")
+    assert (same | near).all(), np.where(~same & ~near)[0]
+
+
+def test_ec_weights_counts_flags_losses(run):
+    cfg, C = run["cfg"], run["C"]
+    p, rp = run["p"].astype(np.float64), run["ref"].p
+    assert np.max(np.abs(p - rp) / rp) <= TOL_W
+    assert (run["counts"] == C).all()
+    member = np.zeros((cfg.T, cfg.E), bool)
+    for e in range(cfg.E):
+        member[run["chosen"][e], e] = True
+    assert (member.sum(axis=0) == C).all()
+    assert np.array_equal(run["dropped"].astype(bool), ~member.any(axis=1))
+    aux, z = oracle.ec_losses(run["ref"].p, run["ref"].lse, C)
+    assert abs(run["losses"][0] - aux) <= TOL_LOSS * abs(aux)
+    assert abs(run["losses"][1] - z) <= TOL_LOSS * abs(z)
+
+
+def test_ec_permute_bit_exact(run):
+    cfg, C = run["cfg"], run["C"]
+    assert np.array_equal(run["offsets"], np.arange(cfg.E + 1) * C)
+    assert np.array_equal(run["row_token"], run["chosen"].reshape(-1))
+    assert np.array_equal(run["row_slot"], np.repeat(np.arange(cfg.E), C))
+    assert np.array_equal(run["x_perm"], run["inp"].x[run["row_token"]])
+
+
+def test_ec_ffn_combine_vs_oracle(run):
+    cfg, inp = run["cfg"], run["inp"]
+    member = np.zeros((cfg.T, cfg.E), bool)
+    for e in range(cfg.E):
+        member[run["chosen"][e], e] = True
+    toks = sample_tokens(cfg.T, SAMPLES.get(cfg.name, cfg.T), seed=cfg.seed)
+    ref = oracle.ec_forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, run["p"].astype(np.float64), member, toks,
+                                   cfg.dtype, act=cfg.act)
+    live = member[toks].any(axis=1)
+    err, tol = out_error(run["out"][toks].astype(np.float64), ref, cfg.dtype, rows=live)
+    print(f"{cfg.name}: out error {err:.3e} (tol {tol:.0e}) over {len(toks)} tokens, "
+          f"{int((~member.any(axis=1)).sum())} tokens chosen by no expert")
+    assert err <= tol
+    assert (run["out"][~member.any(axis=1)] == 0).all()
+
+
+def test_ec_forward_and_unfused_agree(run):
+    assert np.array_equal(run["chosen_forward"], run["chosen"])
+    assert run["launches"] == 6
+    scale = float(np.max(np.abs(run["out"]))) or 1.0
+    assert np.max(np.abs(run["out_forward"] - run["out"])) <= 1e-5 * scale
+    assert np.max(np.abs(run["out_unfused"] - run["out"])) <= 1e-5 * scale
+
+
+def test_ec_equal_logits_take_the_first_tokens():
+    """Wg = 0: all tokens tie within each expert, so every expert takes tokens 0..C-1 (lower index
+    first), on the GPU exactly as in the oracle."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("ec_ties", 300, 64, 8, 2, 64, 1.0, "bf16", 47)
+    inp = synth.make_inputs(cfg)
+    inp.Wg = synth.to_storage(np.zeros((cfg.H, cfg.E)), "bf16")
+    inp.bg = synth.to_storage(np.linspace(-1, 1, cfg.E), "bf16")
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf.forward()
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+    C = moe.moe_capacity(buf.shape)
+    assert C == 75
+    assert (buf.topk_idx.cpu().numpy() == np.arange(C)).all()
+    dropped = buf.dropped.cpu().numpy()
+    assert (dropped[:C] == 0).all() and (dropped[C:] == 1).all()
+    out = buf.out.cpu().numpy()
+    assert (out[C:] == 0).all()
+
+
+def test_ec_empty_batch():
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("ec_empty", 0, 64, 4, 2, 64, 1.0, "bf16", 48)
+    dev = {n: upload_one for n, upload_one in upload(synth.make_inputs(cfg.with_(T=1))).items()}
+    buf = moe.MoEBuffers(shape_of(cfg), dev)
+    buf.losses.fill_(7.0)
+    buf.expert_counts.fill_(7)
+    buf.forward()
+    torch.cuda.synchronize()
+    assert (buf.losses.cpu().numpy() == 0).all()
+    assert (buf.expert_counts.cpu().numpy() == 0).all()

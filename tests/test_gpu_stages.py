@@ -23,7 +23,10 @@ pytestmark = pytest.mark.gpu
 SAMPLES = {"tiny": 256, "decode": 32, "switch": 48, "mixtral": 24, "skew": 48, "mixtral_block": 24}
 
 
-@pytest.fixture(scope="module", params=list(synth.CONFIGS))
+TOKEN_CHOICE = [n for n, c in synth.CONFIGS.items() if c.routing == "token_choice"]
+
+
+@pytest.fixture(scope="module", params=TOKEN_CHOICE)
 def run(request):
     import torch
 
