@@ -15,6 +15,8 @@ documented steps:
   forward    -> out[t] = sum over kept slots of w * FFN_e(x_t)
   expert choice (ec_*) -> every expert takes its top-C tokens by logit; out[t] = sum over the
                 experts that chose t of p[t,e] * FFN_e(x_t)
+  backward (bwd_*) -> gradients of L = sum dout*out + d_aux*aux + d_z*z with respect to x and every
+                weight, by the chain rule through the definitions above
 
 Parity status of each function is recorded in the test-suite pins (``tests/test_oracle_pins.py``);
 every function here is pinned there against closed forms, library routines or brute force.
@@ -77,6 +79,16 @@ def _load():
     lib.oracle_expert_choice.restype = None
     lib.oracle_ec_losses.argtypes = [i64, i64, i64, vp, vp, vp, vp]
     lib.oracle_ec_losses.restype = None
+    lib.oracle_act_grad.argtypes = [c_int, dbl]
+    lib.oracle_act_grad.restype = dbl
+    lib.oracle_bwd_slot.argtypes = [i64, i64, c_int, c_int, vp, i64, ctypes.c_int32, vp, vp, vp, vp, vp, dbl, vp,
+                                    vp, vp]
+    lib.oracle_bwd_slot.restype = None
+    lib.oracle_bwd_expert_weights.argtypes = [i64, i64, c_int, c_int, vp, ctypes.c_int32, vp, vp, vp, i64, vp, vp,
+                                              vp, i64, vp, vp, vp, vp, vp, c_int]
+    lib.oracle_bwd_expert_weights.restype = None
+    lib.oracle_bwd_router.argtypes = [i64, i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, dbl, dbl, vp, vp, vp, vp]
+    lib.oracle_bwd_router.restype = None
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     lib.oracle_set_threads.argtypes = [c_int]
@@ -313,3 +325,125 @@ def forward_ec(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=
     tokens = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
     out = ec_forward_tokens(x, W1, b1, W2, b2, r.p, ec.member(T), tokens, dtype, nthreads, act)
     return ForwardEC(r, ec, aux, z, out, tokens)
+
+
+# ------------------------------------------------------------------ backward pass ----------------
+
+def act_grad(u: float, act: str = "gelu") -> float:
+    return _load().oracle_act_grad(ACT[act], float(u))
+
+
+def bwd_slot(x, W1, b1, W2, b2, t: int, e: int, dout_t, w: float, dtype: str, act: str = "gelu"):
+    """One kept slot: (dx_part[H] = W1[e] du, dw = dout_t . y, du[F])."""
+    x, W1, b1, W2, b2 = _c(x), _c(W1), _opt(b1), _c(W2), _opt(b2)
+    E, H, F = W1.shape
+    d = _c(dout_t, np.float64)
+    dx = np.empty(H, np.float64)
+    du = np.empty(F, np.float64)
+    dw = np.zeros(1, np.float64)
+    _load().oracle_bwd_slot(H, F, _DT[dtype], ACT[act], _p(x), int(t), int(e), _p(W1), _p(b1), _p(W2), _p(b2), _p(d),
+                            float(w), _p(dx), _p(dw), _p(du))
+    return dx, float(dw[0]), du
+
+
+def bwd_expert_weights(x, W1, b1, W2, e: int, tokens, w, dout, fcols, dtype: str, act: str = "gelu",
+                       nthreads: int = 0):
+    """Expert e's weight gradients from its kept rows, at FFN columns fcols:
+    (dW2[e][fcols, :], dW1[e][:, fcols].T, db1[e][fcols], db2[e])."""
+    x, W1, b1, W2 = _c(x), _c(W1), _opt(b1), _c(W2)
+    E, H, F = W1.shape
+    tokens, w = _c(tokens, np.int32), _c(w, np.float64)
+    dout = _c(dout, np.float64)
+    fcols = _c(fcols, np.int32)
+    nf = fcols.shape[0]
+    dW2r = np.empty((nf, H), np.float64)
+    dW1c = np.empty((nf, H), np.float64)
+    db1 = np.empty(nf, np.float64)
+    db2 = np.empty(H, np.float64)
+    _load().oracle_bwd_expert_weights(H, F, _DT[dtype], ACT[act], _p(x), int(e), _p(W1), _p(b1), _p(W2),
+                                      tokens.shape[0], _p(tokens), _p(w), _p(dout), nf, _p(fcols), _p(dW2r), _p(dW1c),
+                                      _p(db1), _p(db2), int(nthreads))
+    return dW2r, dW1c, db1, db2
+
+
+def bwd_router(x, Wg, bg, topk_idx, cnt_pre, dw, d_aux: float, d_z: float, dtype: str):
+    """(dlogits[T,E], dWg[H,E], dbg[E], dx_router[T,H]) given dw[T,k] (0 on dropped slots)."""
+    x, Wg, bg = _c(x), _c(Wg), _opt(bg)
+    idx, cnt, dw = _c(topk_idx, np.int32), _c(cnt_pre, np.int32), _c(dw, np.float64)
+    T, H = x.shape
+    E = Wg.shape[1]
+    k = idx.shape[1]
+    dl = np.empty((T, E), np.float64)
+    dWg = np.empty((H, E), np.float64)
+    dbg = np.empty(E, np.float64)
+    dxr = np.empty((T, H), np.float64)
+    _load().oracle_bwd_router(T, H, E, k, _DT[dtype], _p(x), _p(Wg), _p(bg), _p(idx), _p(cnt), _p(dw), float(d_aux),
+                              float(d_z), _p(dl), _p(dWg), _p(dbg), _p(dxr))
+    return dl, dWg, dbg, dxr
+
+
+@dataclass
+class Grads:
+    dx: np.ndarray    # [T,H]
+    dWg: np.ndarray   # [H,E]
+    dbg: np.ndarray   # [E]
+    dW1: np.ndarray   # [E,H,F]
+    db1: np.ndarray   # [E,F]
+    dW2: np.ndarray   # [E,F,H]
+    db2: np.ndarray   # [E,H]
+    dw: np.ndarray    # [T,k] gradient of each slot's combine weight (0 when dropped)
+    dlogits: np.ndarray  # [T,E]
+
+
+def backward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_aux: float, d_z: float,
+             act: str = "gelu", topk_idx=None, dropped=None) -> Grads:
+    """All gradients of L = sum(dout*out) + d_aux*aux + d_z*z (small problems).  The routing is the
+    oracle's own unless topk_idx / dropped are given (e.g. the GPU's, to avoid near-tie flips)."""
+    T, H = x.shape
+    E, _, F = W1.shape
+    r = route(x, Wg, bg, k, dtype)
+    idx = r.topk_idx if topk_idx is None else np.asarray(topk_idx, np.int32)
+    w = r.topk_w if topk_idx is None else _renorm_weights(r.p, idx)
+    d = dispatch(idx, E, cf)
+    drp = d.dropped if dropped is None else np.asarray(dropped, np.uint8)
+    dout = _c(dout, np.float64)
+    dx = np.zeros((T, H))
+    dw = np.zeros((T, k))
+    rows = {e: ([], []) for e in range(E)}
+    for t in range(T):
+        for s in range(k):
+            if drp[t, s]:
+                continue
+            e = int(idx[t, s])
+            dxp, dws, _ = bwd_slot(x, W1, b1, W2, b2, t, e, dout[t], w[t, s], dtype, act)
+            dx[t] += dxp
+            dw[t, s] = dws
+            rows[e][0].append(t)
+            rows[e][1].append(w[t, s])
+    dW1 = np.zeros((E, H, F))
+    dW2 = np.zeros((E, F, H))
+    db1 = np.zeros((E, F))
+    db2 = np.zeros((E, H))
+    allf = np.arange(F, dtype=np.int32)
+    for e in range(E):
+        toks, ws = rows[e]
+        r2, c1, b1s, b2s = bwd_expert_weights(x, W1, b1, W2, e, np.array(toks, np.int32), np.array(ws), dout, allf,
+                                              dtype, act)
+        dW2[e] = r2
+        dW1[e] = c1.T
+        db1[e] = b1s
+        db2[e] = b2s
+    dl, dWg, dbg, dxr = bwd_router(x, Wg, bg, idx, d.cnt_pre, dw, d_aux, d_z, dtype)
+    return Grads(dx + dxr, dWg, dbg, dW1, db1, dW2, db2, dw, dl)
+
+
+def _renorm_weights(p, idx):
+    sel = np.take_along_axis(np.asarray(p, np.float64), np.asarray(idx, np.int64), axis=1)
+    return sel / sel.sum(axis=1, keepdims=True)
+
+
+def loss_of(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_aux: float, d_z: float,
+            act: str = "gelu") -> float:
+    """L = sum(dout * out) + d_aux * aux + d_z * z of the oracle's forward pass."""
+    f = forward(x, Wg, bg, W1, b1, W2, b2, k, cf, dtype, act=act)
+    return float(np.sum(np.asarray(dout, np.float64) * f.out)) + d_aux * f.aux + d_z * f.z

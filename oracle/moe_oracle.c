@@ -40,6 +40,7 @@
  * Inputs are passed in their storage type (fp32 or bf16 bit patterns) and widened to double element
  * by element (both widenings are exact), so the oracle never needs a double copy of the weights.
  */
+#define _USE_MATH_DEFINES
 #include <math.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -397,6 +398,166 @@ void oracle_ec_losses(int64_t T, int64_t E, int64_t C, const double* p, const do
   double zz = 0.0;
   for (int64_t t = 0; t < T; ++t) zz += lse[t] * lse[t];
   *z = zz / (double)T;
+}
+
+/* ----------------------------------------------------------------------------------------------
+ * Backward pass.  The pages train MoE layers (the skill's subject; Core Concepts 3 adds the two
+ * losses to the training loss), so the layer's gradients are the chain rule through the forward
+ * definition above.  Given dout[t,:] = dL/dout[t,:], d_aux = dL/daux and d_z = dL/dz:
+ *
+ * every kept slot (t, s) with expert e and weight w = topk_w[t,s]:
+ *   u = x_t.W1[e] + b1[e],  g = act(u),  y = g.W2[e] + b2[e]
+ *   dY = w dout_t                dw[t,s] = dout_t . y
+ *   dW2[e] += g^T dY             db2[e] += dY
+ *   du = (W2[e] dY) * act'(u)    dW1[e] += x_t^T du      db1[e] += du      dx_t += W1[e] du
+ * a dropped slot has dw = 0 and adds nothing;
+ *
+ * the router, per token (p = softmax(logits), lse, chosen experts e_s, S = sum_s p[e_s]):
+ *   dp[e_s]  = (dw[t,s] - sum_s' dw[t,s'] w[t,s']) / S          renormalisation w_s = p[e_s] / S
+ *   dp[e]   += d_aux * E * f_e / T                              aux = E sum_e f_e P_e (f fixed)
+ *   dlogit[e] = p[e] (dp[e] - sum_e' p[e'] dp[e']) + d_z * 2 lse p[e] / T
+ *   dWg += x_t^T dlogit          dbg += dlogit                  dx_t += Wg dlogit
+ * The top-k choice and the capacity drops are piecewise constant and carry no gradient.
+ * ---------------------------------------------------------------------------------------------- */
+
+/* d act / du: GELU' = Phi(u) + u phi(u); SiLU' = s(u) (1 + u (1 - s(u))) with s the logistic */
+double oracle_act_grad(int act, double u) {
+  if (act == ORACLE_ACT_SILU) {
+    const double sg = 1.0 / (1.0 + exp(-u));
+    return sg * (1.0 + u * (1.0 - sg));
+  }
+  return 0.5 * (1.0 + erf(u / sqrt(2.0))) + u * exp(-0.5 * u * u) / sqrt(2.0 * M_PI);
+}
+
+/*
+ * One kept slot: dx_part[H] = W1[e] du and dw = dout_t . y; du_out[F] (may be NULL) receives du.
+ * dout_t is the token's output gradient row (double, length H).
+ */
+void oracle_bwd_slot(int64_t H, int64_t F, int dtype, int act, const void* x, int64_t t, int32_t e, const void* W1,
+                     const void* b1, const void* W2, const void* b2, const double* dout_t, double w, double* dx_part,
+                     double* dw, double* du_out) {
+  double* u = (double*)malloc(sizeof(double) * (size_t)F);
+  double* du = (double*)malloc(sizeof(double) * (size_t)F);
+  for (int64_t f = 0; f < F; ++f) u[f] = load_bias(b1, dtype, (size_t)(e * F + f));
+  for (int64_t h = 0; h < H; ++h) {
+    const double xv = load(x, dtype, (size_t)(t * H + h));
+    const size_t base = (size_t)((e * H + h) * F);
+    for (int64_t f = 0; f < F; ++f) u[f] += xv * load(W1, dtype, base + (size_t)f);
+  }
+  /* dout . y = dout . b2[e] + sum_f g[f] (W2[e][f,:] . dout);  dg[f] = w (W2[e][f,:] . dout) */
+  double acc = 0.0;
+  for (int64_t h = 0; h < H; ++h) acc += dout_t[h] * load_bias(b2, dtype, (size_t)(e * H + h));
+  for (int64_t f = 0; f < F; ++f) {
+    const size_t base = (size_t)((e * F + f) * H);
+    double wd = 0.0;
+    for (int64_t h = 0; h < H; ++h) wd += load(W2, dtype, base + (size_t)h) * dout_t[h];
+    acc += activation(act, u[f]) * wd;
+    du[f] = w * wd * oracle_act_grad(act, u[f]);
+  }
+  *dw = acc;
+  for (int64_t h = 0; h < H; ++h) {
+    const size_t base = (size_t)((e * H + h) * F);
+    double s = 0.0;
+    for (int64_t f = 0; f < F; ++f) s += load(W1, dtype, base + (size_t)f) * du[f];
+    dx_part[h] = s;
+  }
+  if (du_out)
+    for (int64_t f = 0; f < F; ++f) du_out[f] = du[f];
+  free(u);
+  free(du);
+}
+
+/*
+ * Weight gradients of expert e from its kept rows (tokens[i], weight w[i]), restricted to the
+ * listed FFN columns fcols[j] (all F of them for the full gradient):
+ *   dW2_rows[j, :] = dW2[e][fcols[j], :]      dW1_cols[j, :] = dW1[e][:, fcols[j]]
+ *   db1_sel[j]     = db1[e][fcols[j]]          db2_e[:]       = db2[e][:]
+ * dout is [T,H] double.  Rows are visited in the order given.
+ */
+void oracle_bwd_expert_weights(int64_t H, int64_t F, int dtype, int act, const void* x, int32_t e, const void* W1,
+                               const void* b1, const void* W2, int64_t n, const int32_t* tokens, const double* w,
+                               const double* dout, int64_t nf, const int32_t* fcols, double* dW2_rows,
+                               double* dW1_cols, double* db1_sel, double* db2_e, int nthreads) {
+#ifdef _OPENMP
+  if (nthreads > 0) omp_set_num_threads(nthreads);
+#endif
+  for (int64_t h = 0; h < H; ++h) db2_e[h] = 0.0;
+  for (int64_t i = 0; i < n; ++i)
+    for (int64_t h = 0; h < H; ++h) db2_e[h] += w[i] * dout[tokens[i] * H + h];
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t j = 0; j < nf; ++j) {
+    const int64_t f = fcols[j];
+    double* r2 = dW2_rows + j * H;
+    double* c1 = dW1_cols + j * H;
+    for (int64_t h = 0; h < H; ++h) r2[h] = c1[h] = 0.0;
+    double db1 = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+      const int64_t t = tokens[i];
+      double u = load_bias(b1, dtype, (size_t)(e * F + f));
+      for (int64_t h = 0; h < H; ++h) u += load(x, dtype, (size_t)(t * H + h)) * load(W1, dtype, (size_t)((e * H + h) * F + f));
+      const double g = activation(act, u);
+      double wd = 0.0;
+      for (int64_t h = 0; h < H; ++h) wd += load(W2, dtype, (size_t)((e * F + f) * H + h)) * dout[t * H + h];
+      const double du = w[i] * wd * oracle_act_grad(act, u);
+      for (int64_t h = 0; h < H; ++h) {
+        r2[h] += g * w[i] * dout[t * H + h];
+        c1[h] += load(x, dtype, (size_t)(t * H + h)) * du;
+      }
+      db1 += du;
+    }
+    db1_sel[j] = db1;
+  }
+}
+
+/*
+ * Router backward for all tokens, given dw[T,k] (zero for dropped slots) and the pre-drop counts
+ * cnt_pre[E].  Outputs dlogits[T,E], dWg[H,E], dbg[E] and dx_router[T,H] (the gate's part of dx).
+ */
+void oracle_bwd_router(int64_t T, int64_t H, int64_t E, int64_t k, int dtype, const void* x, const void* Wg,
+                       const void* bg, const int32_t* topk_idx, const int32_t* cnt_pre, const double* dw,
+                       double d_aux, double d_z, double* dlogits, double* dWg, double* dbg, double* dx_router) {
+  double* lg = (double*)malloc(sizeof(double) * (size_t)E);
+  double* p = (double*)malloc(sizeof(double) * (size_t)E);
+  double* dp = (double*)malloc(sizeof(double) * (size_t)E);
+  for (int64_t i = 0; i < H * E; ++i) dWg[i] = 0.0;
+  for (int64_t e = 0; e < E; ++e) dbg[e] = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t e = 0; e < E; ++e) {
+      double acc = load_bias(bg, dtype, (size_t)e);
+      for (int64_t h = 0; h < H; ++h) acc += load(x, dtype, (size_t)(t * H + h)) * load(Wg, dtype, (size_t)(h * E + e));
+      lg[e] = acc;
+    }
+    double m = lg[0];
+    for (int64_t e = 1; e < E; ++e)
+      if (lg[e] > m) m = lg[e];
+    double se = 0.0;
+    for (int64_t e = 0; e < E; ++e) se += exp(lg[e] - m);
+    const double lse = m + log(se);
+    for (int64_t e = 0; e < E; ++e) p[e] = exp(lg[e] - lse);
+    double S = 0.0;
+    for (int64_t s = 0; s < k; ++s) S += p[topk_idx[t * k + s]];
+    double dww = 0.0;
+    for (int64_t s = 0; s < k; ++s) dww += dw[t * k + s] * p[topk_idx[t * k + s]] / S;
+    for (int64_t e = 0; e < E; ++e) dp[e] = d_aux * (double)E * ((double)cnt_pre[e] / ((double)T * (double)k)) / (double)T;
+    for (int64_t s = 0; s < k; ++s) dp[topk_idx[t * k + s]] += (dw[t * k + s] - dww) / S;
+    double pdp = 0.0;
+    for (int64_t e = 0; e < E; ++e) pdp += p[e] * dp[e];
+    double* dl = dlogits + t * E;
+    for (int64_t e = 0; e < E; ++e) dl[e] = p[e] * (dp[e] - pdp) + d_z * 2.0 * lse * p[e] / (double)T;
+    for (int64_t e = 0; e < E; ++e) dbg[e] += dl[e];
+    for (int64_t h = 0; h < H; ++h) {
+      const double xv = load(x, dtype, (size_t)(t * H + h));
+      double s = 0.0;
+      for (int64_t e = 0; e < E; ++e) {
+        dWg[h * E + e] += xv * dl[e];
+        s += load(Wg, dtype, (size_t)(h * E + e)) * dl[e];
+      }
+      dx_router[t * H + h] = s;
+    }
+  }
+  free(lg);
+  free(p);
+  free(dp);
 }
 
 /* threads the OpenMP runtime will use for a parallel region (for reporting) */

@@ -527,3 +527,99 @@ def test_ec_selects_on_logits_not_probabilities():
     assert ec.chosen[0].tolist() == [1]
     assert ec.chosen[1].tolist() == [1]
     assert special.softmax(logits, axis=1)[0, 0] > special.softmax(logits, axis=1)[1, 0]
+
+
+# ---------------------------------------------------------------- backward pass -----------------
+
+@pytest.mark.parametrize("act", ["gelu", "silu"])
+def test_act_grad_closed_forms_and_numeric_derivative(act):
+    f = oracle.gelu if act == "gelu" else oracle.silu
+    assert oracle.act_grad(0.0, act) == pytest.approx(0.5, abs=1e-15)  # Phi(0) = s(0) = 1/2
+    if act == "gelu":
+        # GELU'(1) = Phi(1) + phi(1)
+        assert oracle.act_grad(1.0, act) == pytest.approx(0.8413447460685429 + 0.24197072451914337, abs=1e-14)
+    else:
+        # SiLU'(1) = s(1) (1 + 1 - s(1)) with s(1) = e/(1+e)
+        s1 = math.e / (1 + math.e)
+        assert oracle.act_grad(1.0, act) == pytest.approx(s1 * (2 - s1), abs=1e-15)
+    for u in np.linspace(-6, 6, 49):
+        h = 1e-5
+        num = (f(u + h) - f(u - h)) / (2 * h)
+        assert oracle.act_grad(u, act) == pytest.approx(num, abs=1e-9)
+    assert oracle.act_grad(30.0, act) == pytest.approx(1.0, abs=1e-10)  # SiLU'(30) = 1 + 30 e^-30 + ...
+    assert oracle.act_grad(-40.0, act) == pytest.approx(0.0, abs=1e-12)
+
+
+def _fd_layer(seed, T=7, H=6, E=3, F=5, k=2, cf=math.inf, act="gelu", bias=True):
+    cfg = synth.LayerConfig("fd", T=T, H=H, E=E, k=k, F=F, CF=cf, dtype="f32", seed=seed, bias_std=0.3, act=act,
+                            bias=bias)
+    inp = synth.make_inputs(cfg)
+    if bias:
+        inp.bg = synth.normal(seed, 98, (E,), 0.0, 0.4)
+    dout = synth.normal(seed, 97, (T, H)).astype(np.float64)
+    return cfg, inp, dout
+
+
+@pytest.mark.parametrize("case", [
+    dict(seed=71),                                  # GELU, biases, top-2, dropless
+    dict(seed=72, act="silu", bias=False),          # the Mixtral block: SiLU, no biases
+    dict(seed=73, cf=0.75),                         # capacity drops
+    dict(seed=74, k=1, E=4),                        # top-1: the weight is constant, only the losses reach the gate
+], ids=["gelu_bias", "silu_nobias", "drops", "top1"])
+def test_backward_matches_central_differences(case):
+    """Every gradient of L = sum(dout*out) + d_aux*aux + d_z*z against central differences of the oracle's
+    own forward pass (fp64), at a few entries of every input; the step is the actual fp32 difference."""
+    case = dict(case)
+    seed = case.pop("seed")
+    cfg, inp, dout = _fd_layer(seed, **case)
+    d_aux, d_z = 0.37, -0.21
+    r = oracle.route(inp.x, inp.Wg, inp.bg, cfg.k, "f32")
+    assert r.margin.min() > 2e-2  # the routing cannot flip under the steps below
+    g = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, "f32", dout, d_aux, d_z,
+                        act=cfg.act)
+    if cfg.CF < math.inf:
+        assert oracle.dispatch(r.topk_idx, cfg.E, cfg.CF).dropped.sum() > 0
+    names = ["x", "Wg", "W1", "W2"] + (["bg", "b1", "b2"] if cfg.bias else [])
+    grads = dict(x=g.dx, Wg=g.dWg, bg=g.dbg, W1=g.dW1, b1=g.db1, W2=g.dW2, b2=g.db2)
+    rng = np.random.default_rng(seed)
+    for name in names:
+        base = getattr(inp, name)
+        for flat in rng.choice(base.size, size=min(6, base.size), replace=False):
+            idx = np.unravel_index(flat, base.shape)
+            lo, hi = base.copy(), base.copy()
+            lo[idx] = np.float32(base[idx] - 1e-3)
+            hi[idx] = np.float32(base[idx] + 1e-3)
+            step = float(hi[idx]) - float(lo[idx])
+            args = {n: getattr(inp, n) for n in ("x", "Wg", "bg", "W1", "b1", "W2", "b2")}
+            args[name] = hi
+            Lp = oracle.loss_of(args["x"], args["Wg"], args["bg"], args["W1"], args["b1"], args["W2"], args["b2"],
+                                cfg.k, cfg.CF, "f32", dout, d_aux, d_z, act=cfg.act)
+            args[name] = lo
+            Lm = oracle.loss_of(args["x"], args["Wg"], args["bg"], args["W1"], args["b1"], args["W2"], args["b2"],
+                                cfg.k, cfg.CF, "f32", dout, d_aux, d_z, act=cfg.act)
+            assert grads[name][idx] == pytest.approx((Lp - Lm) / step, rel=1e-5, abs=1e-7), (name, idx)
+
+
+def test_backward_top1_weight_gradient_does_not_reach_the_gate():
+    """k = 1: the renormalised weight is 1 whatever the logits, so without the two losses the gate gets
+    exactly zero gradient, while dw itself is not zero."""
+    cfg, inp, dout = _fd_layer(75, k=1, E=4)
+    g = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, 1, math.inf, "f32", dout, 0.0, 0.0)
+    assert np.abs(g.dw).max() > 0.1
+    assert np.abs(g.dlogits).max() < 1e-15 and np.abs(g.dWg).max() < 1e-15
+
+
+def test_backward_sampled_columns_match_full():
+    """bwd_expert_weights at a subset of FFN columns gives the same entries as the full gradient."""
+    cfg, inp, dout = _fd_layer(76, T=9, F=7)
+    g = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, 2, math.inf, "f32", dout, 0.1, 0.1)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, 2, "f32")
+    e = 1
+    toks, slots = np.where(r.topk_idx == e)
+    cols = np.array([6, 0, 3], np.int32)
+    r2, c1, b1s, b2s = oracle.bwd_expert_weights(inp.x, inp.W1, inp.b1, inp.W2, e, toks.astype(np.int32),
+                                                 r.topk_w[toks, slots], dout, cols, "f32")
+    np.testing.assert_allclose(r2, g.dW2[e][cols], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(c1, g.dW1[e][:, cols].T, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(b1s, g.db1[e][cols], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(b2s, g.db2[e], rtol=1e-13, atol=1e-15)
