@@ -377,6 +377,29 @@ def run_ours_impl(args, cfg):
     # permute: read the kept x rows, write them to x_perm, clear out (fp32), index traffic
     permute_bytes = kept * cfg.H * es * 2 + cfg.T * cfg.H * 4 + cfg.T * cfg.k * 8
     traffic = None
+    # ---------------- training step: forward that keeps state + backward (bf16 token choice) -----
+    train = None
+    if not args.no_train and cfg.dtype == "bf16" and cfg.routing == "token_choice":
+        tbuf = moe.MoEBuffers(shape, dev, train=True)
+        grads = tbuf.make_grads(with_dw=False)
+        dout = torch.randn((cfg.T, cfg.H), dtype=torch.float32, device="cuda",
+                           generator=torch.Generator(device="cuda").manual_seed(cfg.seed))
+        tbuf.forward_train()
+        ms_fwd_train = time_calls(tbuf.forward_train)
+        ms_bwd = time_calls(lambda: tbuf.backward(dout, grads, 0.01, 0.001))
+        bwd_launches = moe.moe_last_launch_count()
+        tkept = int(tbuf.expert_counts.sum().item())
+        bwd_flops = 8.0 * cfg.H * cfg.F * tkept + 4.0 * cfg.T * cfg.H * cfg.E
+        train = {"fwd_train_ms": ms_fwd_train, "bwd_ms": ms_bwd, "step_ms": ms_fwd_train + ms_bwd,
+                 "tokens_per_s": world * cfg.T / ((ms_fwd_train + ms_bwd) / 1000.0),
+                 "bwd_tflops": bwd_flops / (ms_bwd / 1000.0) / 1e12,
+                 "bwd_frac_sustained": bwd_flops / (ms_bwd / 1000.0) / 1e12 / peak,
+                 "bwd_launches": bwd_launches,
+                 "note": "backward = dout row gather, dgrad W2 (+du, dw), dgrad W1 (+dx), wgrad W2, wgrad W1, bias "
+                         "gradients, router backward, gate weight gradient; flops 8*H*F per kept row + 4*T*H*E"}
+        del tbuf, grads, dout
+        torch.cuda.empty_cache()
+
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         try:
@@ -412,6 +435,7 @@ def run_ours_impl(args, cfg):
             "layer_roofline_ms": 1000 * max(alg_flops(cfg, kept) / (peaks["bf16_tflops"] * 1e12),
                                             alg_bytes(cfg, touched) / (peaks["hbm_gbs"] * 1e9)),
         },
+        "train": train,
         "layer": {"kept": kept, "dropped": drops, "touched_experts": touched, "aux_loss": float(losses[0]),
                   "z_loss": float(losses[1]), "expert_counts_min_max": [int(counts.min()), int(counts.max())]},
     }
@@ -429,6 +453,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="mixtral", choices=list(synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-train", action="store_true", help="skip the training-step (forward + backward) timing")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
     for dim in ("T", "H", "E", "k", "F"):
         ap.add_argument(f"--{dim}", type=int, default=None, help=f"override {dim} of the workload (profiling)")

@@ -240,6 +240,48 @@ MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, v
 MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_io_t* io, const void* x_host,
                               float* out_host, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Training: forward pass that keeps what the backward pass needs, and the backward pass.
+ * The pages train MoE layers (Core Concepts 3 adds the two losses to the training loss); the
+ * gradients are the chain rule through the forward definition: for L with dL/dout = dout,
+ * dL/daux = d_aux and dL/dz = d_z, every input x, Wg, bg, W1, b1, W2, b2 gets dL/d(input).  The
+ * top-k choice and the capacity drops are piecewise constant and carry no gradient; a dropped
+ * slot contributes nothing.  Token choice with bf16 storage only (else MOE_ERR_UNSUPPORTED).
+ * ------------------------------------------------------------------------------------------- */
+
+/* Caller-owned device buffers of the backward pass, fp32, row-major. */
+typedef struct {
+  const float* dout; /* [T,H] dL/dout */
+  float d_aux;       /* dL/d aux_loss (its coefficient in the loss) */
+  float d_z;         /* dL/d z_loss */
+  float* dx;         /* [T,H] */
+  float* dWg;        /* [H,E] */
+  float* dbg;        /* [E]; must be NULL exactly when io->bg is NULL */
+  float* dW1;        /* [E,H,F] */
+  float* db1;        /* [E,F]; NULL exactly when io->b1 is NULL */
+  float* dW2;        /* [E,F,H] */
+  float* db2;        /* [E,H]; NULL exactly when io->b2 is NULL */
+  float* dw;         /* [T,k] optional (may be NULL): dL/d topk_w per slot, 0 for dropped slots */
+} moe_grad_t;
+
+/* Workspace bytes for moe_forward_train + moe_backward (the inference layout plus the saved router
+ * logits, the pre-activation u and the backward's row buffers); 0 if the shape is invalid.  A
+ * training workspace also serves every inference entry point. */
+MOE_API size_t moe_train_workspace_size(const moe_shape_t* shape);
+
+/* moe_forward (same outputs), also keeping the router logits and the pre-activation u in ws for
+ * moe_backward.  ws_bytes >= moe_train_workspace_size(shape).  5 launches. */
+MOE_API moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
+
+/* Gradients of the layer after moe_forward_train on the same ws, io and inputs.  Reads x, Wg, W1,
+ * W2, b2 (optional), topk_idx, topk_w, dropped from io and the saved state from ws; writes every
+ * buffer of grad (dx, dWg, dbg are cleared first; no output is accumulated across calls).
+ * Row order of the bf16 intermediates: the permuted (expert-major) rows of the forward pass.
+ * Order of fp32 additions in dx, dWg and dbg is not fixed (atomics).  7 or 8 launches. */
+MOE_API moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const moe_grad_t* grad, void* ws,
+                          size_t ws_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the workspace's device error word.
  * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out) or MOE_ERR_CUDA. */
 MOE_API moe_status_t moe_get_device_status(void* ws, cudaStream_t stream);

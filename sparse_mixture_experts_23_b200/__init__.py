@@ -26,6 +26,7 @@ ENTRY_POINTS = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_forward_host", "moe_get_device_status", "moe_set_wait_limit", "moe_debug_timeout_probe",
     "moe_last_launch_count", "moe_status_string", "moe_route_noalloc", "moe_capacity",
+    "moe_train_workspace_size", "moe_forward_train", "moe_backward",
 )
 
 
@@ -44,6 +45,11 @@ class Shape(ctypes.Structure):
 class IO(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("x", "Wg", "bg", "W1", "b1", "W2", "b2", "out", "topk_idx", "topk_w",
                                                "expert_counts", "dropped", "aux_loss", "z_loss")]
+
+
+class Grad(ctypes.Structure):
+    _fields_ = [("dout", ctypes.c_void_p), ("d_aux", ctypes.c_float), ("d_z", ctypes.c_float)] + [
+        (n, ctypes.c_void_p) for n in ("dx", "dWg", "dbg", "dW1", "db1", "dW2", "db2", "dw")]
 
 
 class WsView(ctypes.Structure):
@@ -79,6 +85,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_expert_ffn.argtypes = [P(Shape), P(IO), vp, sz, ctypes.c_int, vp]
     lib.moe_expert_ffn.restype = st
     lib.moe_forward_host.argtypes = [P(Shape), P(IO), vp, vp, vp, sz, vp]
+    lib.moe_train_workspace_size.argtypes = [P(Shape)]
+    lib.moe_train_workspace_size.restype = sz
+    lib.moe_forward_train.argtypes = [P(Shape), P(IO), vp, sz, vp]
+    lib.moe_forward_train.restype = st
+    lib.moe_backward.argtypes = [P(Shape), P(IO), P(Grad), vp, sz, vp]
+    lib.moe_backward.restype = st
     lib.moe_forward_host.restype = st
     lib.moe_get_device_status.argtypes = [vp, vp]
     lib.moe_get_device_status.restype = st
@@ -149,6 +161,18 @@ def moe_forward(shape, io, ws, ws_bytes, stream=0) -> int:
     return load_library().moe_forward(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, stream)
 
 
+def moe_train_workspace_size(shape: Shape) -> int:
+    return load_library().moe_train_workspace_size(ctypes.byref(shape))
+
+
+def moe_forward_train(shape, io, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_forward_train(ctypes.byref(shape), ctypes.byref(io), ws, ws_bytes, stream)
+
+
+def moe_backward(shape, io, grad, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_backward(ctypes.byref(shape), ctypes.byref(io), ctypes.byref(grad), ws, ws_bytes, stream)
+
+
 def moe_forward_host(shape, io, x_host, out_host, ws, ws_bytes, stream=0) -> int:
     return load_library().moe_forward_host(ctypes.byref(shape), ctypes.byref(io), x_host, out_host, ws, ws_bytes,
                                            stream)
@@ -178,7 +202,7 @@ class MoEBuffers:
     bias).  Outputs and the workspace are allocated here.
     """
 
-    def __init__(self, shape: Shape, inputs: dict, device="cuda"):
+    def __init__(self, shape: Shape, inputs: dict, device="cuda", train: bool = False):
         import torch
 
         self.shape = shape
@@ -198,7 +222,7 @@ class MoEBuffers:
         self.expert_counts = torch.empty((E,), dtype=torch.int32, device=device)
         self.dropped = torch.empty(drop_shape, dtype=torch.uint8, device=device)
         self.losses = torch.empty((2,), dtype=torch.float32, device=device)
-        self.ws_bytes = moe_workspace_size(shape)
+        self.ws_bytes = moe_train_workspace_size(shape) if train else moe_workspace_size(shape)
         if self.ws_bytes == 0:
             raise MoEError(MOE_ERR_INVALID_ARG, "moe_workspace_size")
         self.ws = torch.empty((self.ws_bytes,), dtype=torch.uint8, device=device)
@@ -252,3 +276,34 @@ class MoEBuffers:
 
     def device_status(self) -> int:
         return moe_get_device_status(self.ws_ptr, self.stream())
+
+    # ---- training (buffers built with train=True) ----
+    def forward_train(self):
+        return _check(moe_forward_train(self.shape, self.io, self.ws_ptr, self.ws_bytes, self.stream()),
+                      "moe_forward_train")
+
+    def make_grads(self, with_dw: bool = True) -> dict:
+        """fp32 gradient buffers for every input the layer has (bias gradients only where the bias exists)."""
+        import torch
+
+        s, dev = self.shape, self.out.device
+        T, H, E, F, k = s.T, s.H, s.E, s.F, s.k
+        g = {"dx": torch.empty((T, H), dtype=torch.float32, device=dev),
+             "dWg": torch.empty((H, E), dtype=torch.float32, device=dev),
+             "dW1": torch.empty((E, H, F), dtype=torch.float32, device=dev),
+             "dW2": torch.empty((E, F, H), dtype=torch.float32, device=dev)}
+        if self.inputs.get("bg") is not None:
+            g["dbg"] = torch.empty((E,), dtype=torch.float32, device=dev)
+        if self.inputs.get("b1") is not None:
+            g["db1"] = torch.empty((E, F), dtype=torch.float32, device=dev)
+        if self.inputs.get("b2") is not None:
+            g["db2"] = torch.empty((E, H), dtype=torch.float32, device=dev)
+        if with_dw:
+            g["dw"] = torch.empty((T, k), dtype=torch.float32, device=dev)
+        return g
+
+    def backward(self, dout, grads: dict, d_aux: float = 0.0, d_z: float = 0.0):
+        p = lambda n: None if grads.get(n) is None else grads[n].data_ptr()  # noqa: E731
+        g = Grad(dout.data_ptr(), float(d_aux), float(d_z), p("dx"), p("dWg"), p("dbg"), p("dW1"), p("db1"), p("dW2"),
+                 p("db2"), p("dw"))
+        return _check(moe_backward(self.shape, self.io, g, self.ws_ptr, self.ws_bytes, self.stream()), "moe_backward")

@@ -33,6 +33,7 @@
 #include <stdlib.h>
 
 #include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
@@ -49,9 +50,11 @@ constexpr int kStgStride = 36;                     // floats per staged row (32 
 constexpr int kStgWarpBytes = 5 * 1024;  // one warp's staging tile: 32 x 32 fp32 (padded rows) or a
                                           // 1024-aligned 32 x 64 bf16 box in 128-byte swizzle
 
-enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2, EPI_SILU = 3 };
-// GEMM1 epilogues write h = act(acc + b1); GEMM2 epilogues combine or store y.
+enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2, EPI_SILU = 3, EPI_DGRAD_GELU = 4, EPI_DGRAD_SILU = 5 };
+// GEMM1 epilogues write h = act(acc + b1); GEMM2 epilogues combine or store y; the backward's
+// first GEMM (G = dout_rows . W2[e]^T) writes du = w * G * act'(u) and accumulates dw = G . h.
 __host__ __device__ constexpr bool epi_h(int epi) { return epi == EPI_GELU || epi == EPI_SILU; }
+__host__ __device__ constexpr bool epi_dgrad(int epi) { return epi == EPI_DGRAD_GELU || epi == EPI_DGRAD_SILU; }
 
 template <int BN>
 struct Cfg {
@@ -77,7 +80,11 @@ struct GemmArgs {
   const int32_t* offsets;
   int E, N, K;
   const __nv_bfloat16* bias;
-  __nv_bfloat16* h_out;
+  __nv_bfloat16* h_out;           // GEMM1: h; backward GEMM: du
+  __nv_bfloat16* u_out;           // GEMM1 of a training forward: the pre-activation u (else null)
+  const __nv_bfloat16* h_in;      // backward GEMM: the forward's h and u
+  const __nv_bfloat16* u_in;
+  float* dwraw;                   // backward GEMM: per-row sum_n G * h (atomically accumulated)
   float* out;
   float* y;
   const int32_t* row_token;
@@ -88,185 +95,7 @@ struct GemmArgs {
   long long wait_limit;
 };
 
-// ------------------------------------------------------------------ PTX wrappers ----------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait. Returns false when the CTA is aborting or the bound ran out (then it aborts).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long long limit, volatile int* abort_flag,
-                                          int32_t* status, int code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
-    if (clock64() - t0 > limit) {
-      *abort_flag = 1;
-      atomicCAS(status, 0, code);
-      return false;
-    }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-// TMA store of a shared-memory box to global memory, tracked by this thread's bulk groups
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];\n" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(src), "r"(x), "r"(y)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
-
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
-  asm volatile("prefetch.tensormap [%0];\n" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-
-__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot), "r"(ncols) : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Shared-memory matrix descriptors (tcgen05 "matrix descriptor" format, version 1 for sm_100):
-// bits 0-13 start>>4, 16-29 leading byte offset>>4, 32-45 stride byte offset>>4, 46-47 version=1,
-// 49-51 base offset (0: atoms 1024-aligned), 61-63 layout (2 = 128-byte swizzle).
-// A, K-major 128B swizzle: rows of 128 bytes, 8-row atoms 1024 B apart (SBO); LBO unused (16 B).
-__device__ __forceinline__ uint64_t desc_a_kmajor(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-// B, MN-major 128B swizzle: each k row holds 64 n values (128 B); 8 k rows form a 1024 B atom
-// (SBO = 1024 between k groups); the next 64 n values sit one whole 64x64 box further (LBO).
-__device__ __forceinline__ uint64_t desc_b_mnmajor(uint32_t addr) {
-  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((BK * 128) >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-          d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
-        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
-        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-}
-
-// ---- CTA-pair (cta_group::2) helpers --------------------------------------------------------
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
-  return r;
-}
-// address of the same shared-memory offset in CTA `rank` of this cluster
-__device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
-}
-// TMA into this CTA's shared memory, completion bytes counted on a barrier of either CTA of the pair
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, "
-      "%4}], [%5];\n" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(slot), "r"(ncols) : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(taddr), "r"(ncols) : "memory");
-}
-__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                              uint32_t acc) {
-  asm volatile(
-      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\ntcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
-          d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-      : "memory");
-}
-// arrive (once the pair's prior MMAs complete) on the barrier at this offset in both CTAs of the pair
-__device__ __forceinline__ void mma_commit_both(uint32_t bar) {
-  const uint16_t both = 3;
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster"
-      ".multicast::cluster.b64 [%0], %1;\n" ::"r"(bar),
-      "h"(both)
-      : "memory");
-}
-// arrive (once the pair's prior MMAs complete) on the barrier at cluster address `bar`
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar) : "memory");
-}
+using namespace sm100;
 
 __device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
 // u * sigmoid(u); for u < -87 the fast divide returns 0 where the exact value is below 1e-35
@@ -275,6 +104,19 @@ template <int EPI>
 __device__ __forceinline__ float act(float u) {
   if constexpr (EPI == EPI_SILU) return silu(u);
   else return gelu_erf(u);
+}
+// derivatives: GELU'(u) = Phi(u) + u phi(u); SiLU'(u) = s (1 + u (1 - s)), s = sigmoid(u)
+__device__ __forceinline__ float gelu_grad(float u) {
+  return 0.5f * (1.f + erff(u * 0.70710678118654752f)) + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+}
+__device__ __forceinline__ float silu_grad(float u) {
+  const float sg = __fdividef(1.f, 1.f + __expf(-u));
+  return sg * (1.f + u * (1.f - sg));
+}
+template <int EPI>
+__device__ __forceinline__ float act_grad(float u) {
+  if constexpr (EPI == EPI_DGRAD_SILU) return silu_grad(u);
+  else return gelu_grad(u);
 }
 // 8 bias values at brow[n0 .. n0+8) as 4 bf16 pairs, zeros when the layer has no bias
 __device__ __forceinline__ uint4 bias8(const __nv_bfloat16* brow, int n0) {
@@ -323,6 +165,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t
     for (int i = 0; i < nr; ++i) {
       const float v = stg[i * kStgStride + lane] + bj;
       g.h_out[(size_t)(grow0 + i) * g.N + n0 + lane] = __float2bfloat16_rn(act<EPI>(v));
+      if (g.u_out) g.u_out[(size_t)(grow0 + i) * g.N + n0 + lane] = __float2bfloat16_rn(v);
     }
   } else if (EPI == EPI_COMBINE) {
     for (int i = 0; i < nr; ++i) {
@@ -344,24 +187,29 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t
 template <int EPI>
 __device__ __forceinline__ void epilogue_h_box(const CUtensorMap* tmC, const uint32_t (&r0)[32],
                                                   const uint32_t (&r1)[32], uint8_t* stg, int lane,
-                                                  const __nv_bfloat16* brow, int n0, int grow0) {
+                                                  const __nv_bfloat16* brow, int n0, int grow0,
+                                                  __nv_bfloat16* u_out, int ldu) {
   if (lane == 0) bulk_wait_read0();  // the previous box has left the staging buffer
   __syncwarp();
   uint8_t* row = stg + lane * 128;
+  uint4* urow = u_out ? reinterpret_cast<uint4*>(u_out + (size_t)(grow0 + lane) * ldu + n0) : nullptr;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t* src = j < 4 ? &r0[8 * j] : &r1[8 * (j - 4)];
     const uint4 bb = bias8(brow, n0 + 8 * j);
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
-    uint32_t w[4];
+    uint32_t w[4], uw[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float2 f = __bfloat1622float2(b2[u]);
-      const __nv_bfloat162 v =
-          __floats2bfloat162_rn(act<EPI>(__uint_as_float(src[2 * u]) + f.x), act<EPI>(__uint_as_float(src[2 * u + 1]) + f.y));
+      const float v0 = __uint_as_float(src[2 * u]) + f.x, v1 = __uint_as_float(src[2 * u + 1]) + f.y;
+      const __nv_bfloat162 v = __floats2bfloat162_rn(act<EPI>(v0), act<EPI>(v1));
       w[u] = *reinterpret_cast<const uint32_t*>(&v);
+      const __nv_bfloat162 pre = __floats2bfloat162_rn(v0, v1);
+      uw[u] = *reinterpret_cast<const uint32_t*>(&pre);
     }
     *reinterpret_cast<uint4*>(row + ((j ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
+    if (urow) urow[j] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
   }
   fence_async_smem();
   __syncwarp();
@@ -377,24 +225,55 @@ __device__ __forceinline__ void epilogue_h_rows(const GemmArgs& g, const uint32_
                                                    int lane, int nrows, const __nv_bfloat16* brow, int n0, int grow0) {
   if (lane >= nrows) return;
   uint4* dst = reinterpret_cast<uint4*>(g.h_out + (size_t)(grow0 + lane) * g.N + n0);
+  uint4* urow = g.u_out ? reinterpret_cast<uint4*>(g.u_out + (size_t)(grow0 + lane) * g.N + n0) : nullptr;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const uint32_t* src = j < 4 ? &r0[8 * j] : &r1[8 * (j - 4)];
     const uint4 bb = bias8(brow, n0 + 8 * j);
     const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&bb);
-    uint32_t w[4];
+    uint32_t w[4], uw[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float2 f = __bfloat1622float2(b2[u]);
-      const __nv_bfloat162 v =
-          __floats2bfloat162_rn(act<EPI>(__uint_as_float(src[2 * u]) + f.x), act<EPI>(__uint_as_float(src[2 * u + 1]) + f.y));
+      const float v0 = __uint_as_float(src[2 * u]) + f.x, v1 = __uint_as_float(src[2 * u + 1]) + f.y;
+      const __nv_bfloat162 v = __floats2bfloat162_rn(act<EPI>(v0), act<EPI>(v1));
       w[u] = *reinterpret_cast<const uint32_t*>(&v);
+      const __nv_bfloat162 pre = __floats2bfloat162_rn(v0, v1);
+      uw[u] = *reinterpret_cast<const uint32_t*>(&pre);
     }
     dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+    if (urow) urow[j] = make_uint4(uw[0], uw[1], uw[2], uw[3]);
   }
 }
 
-template <int BN, int EPI>
+// Backward epilogue of 32 accumulator columns of one row (lane = row): G = acc is the row's
+// dout . W2[e]^T at columns n0..n0+32; dw += G . h[row, cols]; du[row, cols] = bf16(w G act'(u)).
+// h, u and du rows are read and written as 64-byte runs.
+template <int EPI>
+__device__ __forceinline__ void epilogue_dgrad32(const GemmArgs& g, const uint32_t (&r)[32], int grow, int n0, float w,
+                                                 float& dw) {
+  const uint4* hp = reinterpret_cast<const uint4*>(g.h_in + (size_t)grow * g.N + n0);
+  const uint4* up = reinterpret_cast<const uint4*>(g.u_in + (size_t)grow * g.N + n0);
+  uint4* dp = reinterpret_cast<uint4*>(g.h_out + (size_t)grow * g.N + n0);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 hv = __ldg(hp + j), uv = __ldg(up + j);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hv);
+    const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&uv);
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 hf = __bfloat1622float2(h2[q]), uf = __bfloat1622float2(u2[q]);
+      const float g0 = __uint_as_float(r[8 * j + 2 * q]), g1 = __uint_as_float(r[8 * j + 2 * q + 1]);
+      dw = fmaf(g0, hf.x, fmaf(g1, hf.y, dw));
+      const __nv_bfloat162 d = __floats2bfloat162_rn(w * g0 * act_grad<EPI>(uf.x), w * g1 * act_grad<EPI>(uf.y));
+      o[q] = *reinterpret_cast<const uint32_t*>(&d);
+    }
+    dp[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <int BN, int EPI, bool BKM>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
   using C = Cfg<BN>;
@@ -470,9 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
           armed[stage] = (int)phase;
           tma_load_2d(a_dst, &tmA, kb * BK, row0, full_bar(stage));
+          if constexpr (BKM) {
+            // B stored [E][N][K]: one 64 k x BN rows box, k contiguous
+            tma_load_3d(b_dst, &tmB, kb * BK, n_idx * BN, e, full_bar(stage));
+          } else {
 #pragma unroll
-          for (int j = 0; j < BN / 64; ++j)
-            tma_load_3d(b_dst + j * (BK * 128), &tmB, n_idx * BN + j * 64, kb * BK, e, full_bar(stage));
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_3d(b_dst + j * (BK * 128), &tmB, n_idx * BN + j * 64, kb * BK, e, full_bar(stage));
+          }
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
@@ -515,7 +399,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t b_addr = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            mma_bf16(d_tmem, desc_a_kmajor(a_addr + kk * 32), desc_b_mnmajor(b_addr + kk * 16 * 128), C::kIdesc,
+            const uint64_t bdesc =
+                BKM ? desc_a_kmajor(b_addr + kk * 32) : desc_mnmajor(b_addr + kk * 16 * 128, BK * 128);
+            mma_bf16(d_tmem, desc_a_kmajor(a_addr + kk * 32), bdesc, BKM ? (C::kIdesc & ~(1u << 16)) : C::kIdesc,
                      (kb | kk) != 0 ? 1u : 0u);
           }
           issued = true;
@@ -554,18 +440,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int grow = row0 + r_in_tile;
       float wgt = 0.f;
       int tok = 0;
-      if (EPI == EPI_COMBINE && row_ok) {
+      if ((EPI == EPI_COMBINE || epi_dgrad(EPI)) && row_ok) {
         tok = g.row_token[grow];
-        wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
+        wgt = g.topk_w ? g.topk_w[(size_t)tok * g.k + g.row_slot[grow]] : 1.f;  // no weights: plain scatter-add
       }
       const __nv_bfloat16* brow = g.bias ? g.bias + (size_t)e * g.N : nullptr;
       const int wrows = rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
       constexpr int kChunks = BN / 32 / (kEpiWarps / 4);  // 32-column chunks per epilogue warp
+      float dw = 0.f;
 #pragma unroll 1
       for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN + c * 32), r);
-        if (wrows > 0) epilogue_chunk<EPI>(g, r, stg, lane, row0 + quarter * 32, wrows, tok, wgt, brow, n_idx * BN + c * 32);
+        if constexpr (epi_dgrad(EPI)) {
+          if (row_ok) epilogue_dgrad32<EPI>(g, r, grow, n_idx * BN + c * 32, wgt, dw);
+        } else {
+          if (wrows > 0)
+            epilogue_chunk<EPI>(g, r, stg, lane, row0 + quarter * 32, wrows, tok, wgt, brow, n_idx * BN + c * 32);
+        }
+      }
+      if constexpr (epi_dgrad(EPI)) {
+        if (row_ok) atomicAdd(g.dwraw + grow, dw);
       }
       tc_fence_before();
       __syncwarp();
@@ -639,7 +534,7 @@ __device__ __forceinline__ void decode_tile_m(int tile, const int* prefix, const
   rows = min(tile_m, cnt - m_local * tile_m);
 }
 
-template <int EPI>
+template <int EPI, bool BKM>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                              const __grid_constant__ CUtensorMap tmC, GemmArgs g) {
@@ -725,10 +620,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int sk = 0; sk < C::kSubK; ++sk) {
             const int k0 = kb * C::kStageK + sk * BK;
             tma_load_2d_pair(a_dst + sk * C::kASubBytes, &tmA, k0, row0 + cta_rows * (int)rank, fb);
+            if constexpr (BKM) {
+              // B stored [E][N][K]: this CTA's 128 columns as one 64 k x 128 rows box, k contiguous
+              tma_load_3d_pair(b_dst + sk * C::kBSubBytes, &tmB, k0, n_idx * C::kTileN + C::kHalfN * (int)rank, e, fb);
+            } else {
 #pragma unroll
-            for (int j = 0; j < C::kHalfN / 64; ++j)
-              tma_load_3d_pair(b_dst + sk * C::kBSubBytes + j * (BK * 128), &tmB,
-                               n_idx * C::kTileN + C::kHalfN * (int)rank + j * 64, k0, e, fb);
+              for (int j = 0; j < C::kHalfN / 64; ++j)
+                tma_load_3d_pair(b_dst + sk * C::kBSubBytes + j * (BK * 128), &tmB,
+                                 n_idx * C::kTileN + C::kHalfN * (int)rank + j * 64, k0, e, fb);
+            }
           }
           if (++stage == C::kStages) {
             stage = 0;
@@ -757,7 +657,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const uint32_t tphase = (uint32_t)((it >> 1) & 1);
         int e_, m_l, n_i, r0_, rows;
         decode_tile_m(tile, prefix, offs, E, NT, C::kTileM, e_, m_l, n_i, r0_, rows);
-        const uint32_t idesc = rows <= C::kTileM / 2 ? C::kIdescHalf : C::kIdesc;
+        const uint32_t idesc0 = rows <= C::kTileM / 2 ? C::kIdescHalf : C::kIdesc;
+        const uint32_t idesc = BKM ? (idesc0 & ~(1u << 16)) : idesc0;  // bit 16: B is MN-major
         if (!mbar_wait(tempty_bar(buf), tphase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutMma)) {
           ok = false;
           break;
@@ -775,8 +676,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < C::kStageK / 16; ++kk) {
             const int sk = kk / (BK / 16), ks = kk % (BK / 16);
-            mma_bf16_pair(d_tmem, desc_a_kmajor(a_addr + sk * C::kASubBytes + ks * 32),
-                          desc_b_mnmajor(b_addr + sk * C::kBSubBytes + ks * 16 * 128), idesc,
+            const uint64_t bdesc = BKM ? desc_a_kmajor(b_addr + sk * C::kBSubBytes + ks * 32)
+                                       : desc_mnmajor(b_addr + sk * C::kBSubBytes + ks * 16 * 128, BK * 128);
+            mma_bf16_pair(d_tmem, desc_a_kmajor(a_addr + sk * C::kASubBytes + ks * 32), bdesc, idesc,
                           (kb | kk) != 0 ? 1u : 0u);
           }
           issued = true;
@@ -824,9 +726,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const int grow = row0 + cta_rows * (int)rank + r_in;
       float wgt = 0.f;
       int tok = 0;
-      if (EPI == EPI_COMBINE && row_ok) {
+      if ((EPI == EPI_COMBINE || epi_dgrad(EPI)) && row_ok) {
         tok = g.row_token[grow];
-        wgt = g.topk_w[(size_t)tok * g.k + g.row_slot[grow]];
+        wgt = g.topk_w ? g.topk_w[(size_t)tok * g.k + g.row_slot[grow]] : 1.f;  // no weights: plain scatter-add
       }
       const __nv_bfloat16* brow = g.bias ? g.bias + (size_t)e * g.N : nullptr;
       const int wrows = my_rows - qr * 32;  // rows of this warp's 32 that lie inside the segment
@@ -840,9 +742,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           tmem_ld32(taddr + c * 32, r0);
           tmem_ld32(taddr + (c + 1) * 32, r1);
           const int n0 = n_idx * C::kTileN + colbase + c * 32;
-          if (wrows >= 32) epilogue_h_box<EPI>(&tmC, r0, r1, reinterpret_cast<uint8_t*>(stg), lane, brow, n0, wrow0);
+          if (wrows >= 32)
+            epilogue_h_box<EPI>(&tmC, r0, r1, reinterpret_cast<uint8_t*>(stg), lane, brow, n0, wrow0, g.u_out, g.N);
           else if (wrows > 0) epilogue_h_rows<EPI>(g, r0, r1, lane, wrows, brow, n0, wrow0);
         }
+      } else if constexpr (epi_dgrad(EPI)) {
+        float dw = 0.f;
+#pragma unroll 1
+        for (int c = half * nch; c < (half + 1) * nch; ++c) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          if (row_ok) epilogue_dgrad32<EPI>(g, r, grow, n_idx * C::kTileN + colbase + c * 32, wgt, dw);
+        }
+        if (row_ok) atomicAdd(g.dwraw + grow, dw);
       } else {
 #pragma unroll 1
         for (int c = half * nch; c < (half + 1) * nch; ++c) {
@@ -866,6 +778,251 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ weight gradients ----------
+// D[e] (M x N, fp32, row-major) = A_e^T . B_e for every expert, where A_e and B_e are the expert's
+// rows offs[e]..offs[e+1] of A [rows, M] and B [rows, N] (both stored row-major, so both operands
+// are MN-major).  The contraction runs over the expert's rows in 64-row blocks; rows of the last
+// block past the segment belong to the next expert (or were never written), so the MMA warp zeroes
+// them in shared memory after the TMA lands and before the MMAs read it.  Tiles are 128 x 256, m
+// fastest inside an n column, expert-major; an expert with no rows gets zeros.  M and N are
+// multiples of 64: partial tiles read zeros past the edge and the epilogue masks them.
+struct WgCfg {
+  static constexpr int kTileM = 128, kTileN = 256, kBK = 64;
+  static constexpr int kStages = 4;
+  static constexpr int kBoxBytes = 64 * kBK * 2;              // one 64 (m or n) x 64 (k) box: 8 KB
+  static constexpr int kABytes = (kTileM / 64) * kBoxBytes;   // 16 KB
+  static constexpr int kBBytes = (kTileN / 64) * kBoxBytes;   // 32 KB
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * kTileN;
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kNumBars = 2 * kStages + 4 + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kOffsOff = kMiscOff + 16;
+  static constexpr int kStgOff = (kOffsOff + 260 * 4 + 127) & ~127;
+  static constexpr int kSmemBytes = 1024 + kStgOff + kEpiWarps * kStgWarpBytes;
+  static_assert(kStgOff % 16 == 0 && kSmemBytes <= 232448, "shared-memory plan");
+  // kind::f16: D fp32, A and B bf16, both MN-major (bits 15, 16), N = 256, M = 128
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                     ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+};
+
+struct WgradArgs {
+  const int32_t* offsets;
+  int E, M, N;
+  float* out;  // [E][M][N]
+  int32_t* status;
+  long long wait_limit;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, WgradArgs g) {
+  using C = WgCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  int* offs = reinterpret_cast<int*>(smem + C::kOffsOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* stg = reinterpret_cast<float*>(smem + C::kStgOff + (warp >= 2 ? warp - 2 : 0) * kStgWarpBytes);
+  const int E = g.E;
+  const int MT = (g.M + C::kTileM - 1) / C::kTileM, NT = (g.N + C::kTileN - 1) / C::kTileN;
+  const int per_e = MT * NT;
+  const int total = E * per_e;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), kEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  for (int i = threadIdx.x; i <= E; i += kThreads) offs[i] = g.offsets[i];
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto decode = [&](int tile, int& e, int& m0, int& n0) {
+    e = tile / per_e;
+    const int local = tile - e * per_e;
+    n0 = (local / MT) * C::kTileN;
+    m0 = (local % MT) * C::kTileM;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer -----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, m0, n0;
+        decode(tile, e, m0, n0);
+        const int r0 = offs[e], KB = (offs[e + 1] - r0 + C::kBK - 1) / C::kBK;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = sbase + stage * C::kStageBytes;
+          const uint32_t b_dst = a_dst + C::kABytes;
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          armed[stage] = (int)phase;
+          const int k0 = r0 + kb * C::kBK;
+#pragma unroll
+          for (int j = 0; j < C::kTileM / 64; ++j) tma_load_2d(a_dst + j * C::kBoxBytes, &tmA, m0 + j * 64, k0, full_bar(stage));
+#pragma unroll
+          for (int j = 0; j < C::kTileN / 64; ++j) tma_load_2d(b_dst + j * C::kBoxBytes, &tmB, n0 + j * 64, k0, full_bar(stage));
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok || *abort_flag) {
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed[s] >= 0) {
+            volatile int dummy = 0;
+            mbar_wait(full_bar(s), (uint32_t)armed[s], g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (whole warp) -------
+    // All lanes wait on each stage; on a segment's last block they zero the rows past it, then
+    // lane 0 issues the MMAs.
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true;
+    bool issued = false;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      int e, m0, n0;
+      decode(tile, e, m0, n0);
+      const int r0 = offs[e], cnt = offs[e + 1] - r0, KB = (cnt + C::kBK - 1) / C::kBK;
+      const int buf = it & 1;
+      const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(buf), tphase ^ 1u, g.wait_limit, abort_flag, g.status,
+                                             kDevTimeoutMma))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kTileN);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status,
+                                               kDevTimeoutMma))) {
+          ok = false;
+          break;
+        }
+        const uint32_t a_addr = sbase + stage * C::kStageBytes;
+        const uint32_t b_addr = a_addr + C::kABytes;
+        const int valid = min(C::kBK, cnt - kb * C::kBK);
+        if (valid < C::kBK) {
+          // rows valid..63 of every box: whole 128-byte lines (the swizzle permutes within a line)
+          const int per_box = (C::kBK - valid) * 8;  // 16-byte pieces per box
+          const int nbox = (C::kTileM + C::kTileN) / 64;
+          for (int i = lane; i < nbox * per_box; i += 32) {
+            const int box = i / per_box, rem = i - box * per_box;
+            const uint32_t addr = a_addr + box * C::kBoxBytes + (valid + rem / 8) * 128 + (rem % 8) * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};\n" ::"r"(addr), "r"(0u) : "memory");
+          }
+          fence_async_smem();
+        }
+        __syncwarp();
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < C::kBK / 16; ++kk)
+            mma_bf16(d_tmem, desc_mnmajor(a_addr + kk * 16 * 128, C::kBoxBytes),
+                     desc_mnmajor(b_addr + kk * 16 * 128, C::kBoxBytes), C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+          mma_commit(empty_bar(stage));
+        }
+        issued = true;
+        __syncwarp();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (lane == 0) mma_commit(tfull_bar(buf));  // with no rows this arrives at once; the epilogue writes zeros
+      __syncwarp();
+    }
+    if ((!ok || *abort_flag) && issued && lane == 0) {
+      mma_commit(drain_bar);
+      volatile int dummy = 0;
+      mbar_wait(drain_bar, 0, g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5) --------
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      int e, m0, n0;
+      decode(tile, e, m0, n0);
+      const bool empty = offs[e + 1] == offs[e];
+      const int buf = it & 1;
+      const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+      const bool got = mbar_wait(tfull_bar(buf), tphase, g.wait_limit, abort_flag, g.status, kDevTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int row0 = m0 + quarter * 32;  // this warp's 32 rows of D
+      const int nrows = min(32, g.M - row0);
+      float* dst = g.out + (size_t)e * g.M * g.N;
+      constexpr int kChunks = C::kTileN / 32 / (kEpiWarps / 4);
+#pragma unroll 1
+      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::kTileN + c * 32), r);
+        const int col = n0 + c * 32;
+        if (nrows <= 0 || col >= g.N) continue;
+        // transpose through the warp's staging tile so that each store covers 128 contiguous bytes
+        float4* mine = reinterpret_cast<float4*>(stg + lane * kStgStride);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          mine[q] = empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                          : make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                        __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+        __syncwarp();
+        for (int i = 0; i < nrows; ++i) dst[(size_t)(row0 + i) * g.N + col + lane] = stg[i * kStgStride + lane];
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(buf));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -944,19 +1101,45 @@ bool make_map_b(CUtensorMap* m, const void* base, int E, int K, int N) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int EPI>
+// K-major B operand: W stored [E][N][K] (k contiguous); box = 64 k x box_rows n x 1 expert
+bool make_map_bk(CUtensorMap* m, const void* base, int E, int N, int K, int box_rows) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)N * K * 2};
+  cuuint32_t box[3] = {BK, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// MN-major operand of the weight gradients: [rows, C] bf16 row-major; box = 64 columns x 64 rows
+bool make_map_rows64(CUtensorMap* m, const void* base, int rows, int C) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)C * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)WgCfg::kBK};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, int EPI, bool BKM = false>
 cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid, cudaStream_t st) {
-  auto kern = grouped_gemm_kernel<BN, EPI>;
+  auto kern = grouped_gemm_kernel<BN, EPI, BKM>;
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(kern), Cfg<BN>::kSmemBytes);
   if (err != cudaSuccess) return err;
   kern<<<grid, kThreads, Cfg<BN>::kSmemBytes, st>>>(ma, mb, g);
   return cudaGetLastError();
 }
 
-template <int EPI>
+template <int EPI, bool BKM = false>
 cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmArgs& g, int grid,
                         cudaStream_t st) {
-  auto kern = grouped_gemm_pair_kernel<EPI>;
+  auto kern = grouped_gemm_pair_kernel<EPI, BKM>;
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(kern), PairCfg::kSmemBytes);
   if (err != cudaSuccess) return err;
   kern<<<grid & ~1, kThreads, PairCfg::kSmemBytes, st>>>(ma, mb, mc, g);
@@ -977,7 +1160,91 @@ cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const
   return launch_one<64, EPI>(ma, mb, g, grid, st);
 }
 
+// A [rows, K] . W[e]^T with W stored [E][N][K]: the backward's data-gradient GEMMs.
+template <int EPI>
+cudaError_t launch_dgrad(const void* A, int rows_cap, const void* W, int E, int N, int K, const GemmArgs& g, int grid,
+                         long long avg_rows, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map_a(&ma, A, rows_cap, K)) return cudaErrorInvalidValue;
+  if (N % 256 == 0 && K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled()) {
+    if (!make_map_bk(&mb, W, E, N, K, PairCfg::kHalfN)) return cudaErrorInvalidValue;
+    return launch_pair<EPI, true>(ma, mb, ma, g, grid, st);
+  }
+  const int BN = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
+  if (!make_map_bk(&mb, W, E, N, K, BN)) return cudaErrorInvalidValue;
+  if (BN == 256) return launch_one<256, EPI, true>(ma, mb, g, grid, st);
+  if (BN == 128) return launch_one<128, EPI, true>(ma, mb, g, grid, st);
+  return launch_one<64, EPI, true>(ma, mb, g, grid, st);
+}
+
+cudaError_t launch_wgrad(const void* A, const void* B, int rows_cap, int M, int N, const int32_t* offsets, int E,
+                         float* out, int32_t* status, long long wait_limit, int grid, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map_rows64(&ma, A, rows_cap, M) || !make_map_rows64(&mb, B, rows_cap, N)) return cudaErrorInvalidValue;
+  WgradArgs g{};
+  g.offsets = offsets;
+  g.E = E;
+  g.M = M;
+  g.N = N;
+  g.out = out;
+  g.status = status;
+  g.wait_limit = wait_limit;
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(wgrad_kernel), WgCfg::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  wgrad_kernel<<<grid, kThreads, WgCfg::kSmemBytes, st>>>(ma, mb, g);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_bwd_gemms_sm100(const BwdGemmArgs& a, cudaStream_t st, int* launches) {
+  const int grid = a.num_sms > 0 ? a.num_sms : 148;
+  // G = dout_rows . W2[e]^T (W2 stored [E][F][H]: N = F, K = H); epilogue -> du, dw partials
+  GemmArgs g{};
+  g.offsets = a.offsets;
+  g.E = a.E;
+  g.N = a.F;
+  g.K = a.H;
+  g.h_out = reinterpret_cast<__nv_bfloat16*>(a.du);
+  g.h_in = reinterpret_cast<const __nv_bfloat16*>(a.h);
+  g.u_in = reinterpret_cast<const __nv_bfloat16*>(a.u);
+  g.dwraw = a.dwraw;
+  g.row_token = a.row_token;
+  g.row_slot = a.row_slot;
+  g.topk_w = a.topk_w;
+  g.k = a.k;
+  g.status = a.status;
+  g.wait_limit = a.wait_limit;
+  cudaError_t err = a.act == MOE_ACT_SILU
+                        ? launch_dgrad<EPI_DGRAD_SILU>(a.dperm, a.rows_cap, a.W2, a.E, a.F, a.H, g, grid, a.avg_rows, st)
+                        : launch_dgrad<EPI_DGRAD_GELU>(a.dperm, a.rows_cap, a.W2, a.E, a.F, a.H, g, grid, a.avg_rows, st);
+  if (err != cudaSuccess) return err;
+  ++*launches;
+  // dx[t] += du . W1[e]^T (W1 stored [E][H][F]: N = H, K = F), scatter-added with weight 1
+  GemmArgs g2{};
+  g2.offsets = a.offsets;
+  g2.E = a.E;
+  g2.N = a.H;
+  g2.K = a.F;
+  g2.out = a.dx;
+  g2.row_token = a.row_token;
+  g2.row_slot = a.row_slot;
+  g2.topk_w = nullptr;
+  g2.k = a.k;
+  g2.status = a.status;
+  g2.wait_limit = a.wait_limit;
+  err = launch_dgrad<EPI_COMBINE>(a.du, a.rows_cap, a.W1, a.E, a.H, a.F, g2, grid, a.avg_rows, st);
+  if (err != cudaSuccess) return err;
+  ++*launches;
+  // dW2[e] = h_e^T . (w dout)_e  (F x H);  dW1[e] = x_e^T . du_e  (H x F)
+  err = launch_wgrad(a.h, a.dyperm, a.rows_cap, a.F, a.H, a.offsets, a.E, a.dW2, a.status, a.wait_limit, grid, st);
+  if (err != cudaSuccess) return err;
+  ++*launches;
+  err = launch_wgrad(a.x_perm, a.du, a.rows_cap, a.H, a.F, a.offsets, a.E, a.dW1, a.status, a.wait_limit, grid, st);
+  if (err != cudaSuccess) return err;
+  ++*launches;
+  return cudaSuccess;
+}
 
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches) {
   CUtensorMap ma1, mb1, ma2, mb2, mc1;
@@ -994,6 +1261,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.K = a.H;
   g1.bias = reinterpret_cast<const __nv_bfloat16*>(a.b1);
   g1.h_out = reinterpret_cast<__nv_bfloat16*>(a.h);
+  g1.u_out = reinterpret_cast<__nv_bfloat16*>(a.u_out);
   g1.k = a.k;
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
@@ -1008,6 +1276,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g2.K = a.F;
   g2.bias = reinterpret_cast<const __nv_bfloat16*>(a.b2);
   g2.h_out = nullptr;
+  g2.u_out = nullptr;
   g2.out = a.out;
   g2.y = a.y;
   g2.row_token = a.row_token;

@@ -85,6 +85,22 @@ WsLayout ws_layout(const moe_shape_t& s) {
   L.tok_count = o;
   o = align256(o + (ec ? T * 4 : 0));
   L.total = o;
+  // training sections (moe_forward_train / moe_backward), appended after the inference layout
+  L.logits = o;
+  o = align256(o + T * E * 4);
+  L.u = o;
+  o = align256(o + rows * (size_t)s.F * es);
+  L.dperm = o;
+  o = align256(o + rows * (size_t)s.H * es);
+  L.dyperm = o;
+  o = align256(o + rows * (size_t)s.H * es);
+  L.du = o;
+  o = align256(o + rows * (size_t)s.F * es);
+  L.dwraw = o;
+  o = align256(o + rows * 4);
+  L.dlogits = o;
+  o = align256(o + T * E * 4);
+  L.train_total = o;
   return L;
 }
 
@@ -150,7 +166,8 @@ int num_sms() {
 
 // ---------------------------------------------------------------- stage bodies (validated) -------
 ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int do_losses, int do_dispatch);
-moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, bool emit_hist) {
+moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, bool emit_hist,
+                      bool train = false) {
   const WsLayout L = ws_layout(*s);
   if (s->T == 0) {
     ++g_launches;
@@ -168,6 +185,7 @@ moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaSt
   r.topk_w = io->topk_w;
   r.loss_part = at<float>(ws, L.loss_part);
   r.chunk_hist = at<int32_t>(ws, L.chunk_hist);
+  r.logits_out = train ? at<float>(ws, L.logits) : nullptr;
   (void)emit_hist;
   if (s->routing == MOE_ROUTING_EXPERT_CHOICE) {
     r.chunk_hist = nullptr;
@@ -266,7 +284,7 @@ moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cuda
   return cuda_status(launch_scatter(a, st));
 }
 
-moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse, cudaStream_t st) {
+moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse, cudaStream_t st, bool train = false) {
   const WsLayout L = ws_layout(*s);
   FfnArgs a{};
   a.T = s->T;
@@ -292,6 +310,7 @@ moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse
   a.y = at<float>(ws, L.y);
   a.out = io->out;
   a.fuse_combine = fuse;
+  a.u_out = train ? at<void>(ws, L.u) : nullptr;
   a.act = s->activation;
   a.status = at<int32_t>(ws, L.status);
   a.wait_limit = g_wait_limit;
@@ -463,6 +482,165 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   st = do_ffn(shape, io, ws, 1, stream);
   g_launches += n;
   return st;
+}
+
+size_t moe_train_workspace_size(const moe_shape_t* shape) {
+  if (check_shape(shape) != MOE_OK) return 0;
+  return ws_layout(*shape).train_total;
+}
+
+static moe_status_t check_train(const moe_shape_t* shape, void* ws, size_t ws_bytes) {
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (shape->dtype != MOE_DTYPE_BF16 || shape->routing != MOE_ROUTING_TOKEN_CHOICE) return MOE_ERR_UNSUPPORTED;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < ws_layout(*shape).train_total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+  g_launches = 0;
+  moe_status_t st = check_train(shape, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (io == nullptr) return MOE_ERR_INVALID_ARG;
+  if (null_any({io->aux_loss, io->z_loss, io->expert_counts})) return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) {
+    ++g_launches;
+    return cuda_status(launch_zero_outputs(io->expert_counts, shape->E, io->aux_loss, io->z_loss, stream));
+  }
+  if (null_any({io->x, io->Wg, io->W1, io->W2, io->out, io->topk_idx, io->topk_w, io->dropped}))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(io->x) || !aligned16(io->Wg) || !aligned16(io->W1) || !aligned16(io->W2) || !aligned16(io->out) ||
+      !aligned16(io->b1) || !aligned16(io->b2))
+    return MOE_ERR_INVALID_ARG;
+  if ((st = do_route(shape, io, ws, stream, true, true)) != MOE_OK) return st;
+  ++g_launches;
+  if ((st = cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 1), stream))) != MOE_OK) return st;
+  if ((st = do_scatter(shape, io, ws, stream)) != MOE_OK) return st;
+  return do_ffn(shape, io, ws, 1, stream, true);
+}
+
+moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const moe_grad_t* grad, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
+  g_launches = 0;
+  moe_status_t st = check_train(shape, ws, ws_bytes);
+  if (st != MOE_OK) return st;
+  if (io == nullptr || grad == nullptr) return MOE_ERR_INVALID_ARG;
+  if (null_any({grad->dout, grad->dx, grad->dWg, grad->dW1, grad->dW2})) return MOE_ERR_INVALID_ARG;
+  // a bias gradient is wanted exactly when the layer has that bias
+  if ((io->bg == nullptr) != (grad->dbg == nullptr) || (io->b1 == nullptr) != (grad->db1 == nullptr) ||
+      (io->b2 == nullptr) != (grad->db2 == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if (shape->T == 0) return MOE_OK;
+  if (null_any({io->x, io->Wg, io->W1, io->W2, io->topk_idx, io->topk_w, io->dropped})) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(grad->dout) || !aligned16(grad->dx) || !aligned16(io->W1) || !aligned16(io->W2))
+    return MOE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(*shape);
+  const int32_t* offsets = at<int32_t>(ws, L.offsets);
+  const int32_t* row_token = at<int32_t>(ws, L.row_token);
+  const int32_t* row_slot = at<int32_t>(ws, L.row_slot);
+
+  BwdPrepArgs pa{};
+  pa.T = shape->T;
+  pa.H = shape->H;
+  pa.E = shape->E;
+  pa.k = shape->k;
+  pa.offsets = offsets;
+  pa.row_token = row_token;
+  pa.row_slot = row_slot;
+  pa.topk_w = io->topk_w;
+  pa.dout = grad->dout;
+  pa.dperm = at<void>(ws, L.dperm);
+  pa.dyperm = at<void>(ws, L.dyperm);
+  pa.dwraw = at<float>(ws, L.dwraw);
+  pa.dx = grad->dx;
+  pa.dWg = grad->dWg;
+  pa.dbg = grad->dbg;
+  ++g_launches;
+  if ((st = cuda_status(launch_bwd_prep(pa, stream))) != MOE_OK) return st;
+
+  BwdGemmArgs ga{};
+  ga.T = shape->T;
+  ga.H = shape->H;
+  ga.E = shape->E;
+  ga.F = shape->F;
+  ga.k = shape->k;
+  ga.rows_cap = (int)L.rows;
+  ga.act = shape->activation;
+  ga.avg_rows = (long long)shape->T * shape->k / shape->E;
+  ga.offsets = offsets;
+  ga.row_token = row_token;
+  ga.row_slot = row_slot;
+  ga.topk_w = io->topk_w;
+  ga.W1 = io->W1;
+  ga.W2 = io->W2;
+  ga.x_perm = at<void>(ws, L.x_perm);
+  ga.h = at<void>(ws, L.h);
+  ga.u = at<void>(ws, L.u);
+  ga.dperm = pa.dperm;
+  ga.dyperm = pa.dyperm;
+  ga.du = at<void>(ws, L.du);
+  ga.dwraw = pa.dwraw;
+  ga.dx = grad->dx;
+  ga.dW1 = grad->dW1;
+  ga.dW2 = grad->dW2;
+  ga.status = at<int32_t>(ws, L.status);
+  ga.wait_limit = g_wait_limit;
+  ga.num_sms = num_sms();
+  if ((st = cuda_status(launch_bwd_gemms_sm100(ga, stream, &g_launches))) != MOE_OK) return st;
+
+  if (grad->db1 || grad->db2) {
+    BiasGradArgs ba{};
+    ba.H = shape->H;
+    ba.F = shape->F;
+    ba.E = shape->E;
+    ba.k = shape->k;
+    ba.offsets = offsets;
+    ba.row_token = row_token;
+    ba.row_slot = row_slot;
+    ba.topk_w = io->topk_w;
+    ba.dout = grad->dout;
+    ba.du = ga.du;
+    ba.db1 = grad->db1;
+    ba.db2 = grad->db2;
+    ++g_launches;
+    if ((st = cuda_status(launch_bias_grad(ba, stream))) != MOE_OK) return st;
+  }
+
+  RouterBwdArgs ra{};
+  ra.T = shape->T;
+  ra.H = shape->H;
+  ra.E = shape->E;
+  ra.k = shape->k;
+  ra.logits = at<float>(ws, L.logits);
+  ra.topk_idx = io->topk_idx;
+  ra.topk_w = io->topk_w;
+  ra.dropped = io->dropped;
+  ra.row_of = at<int32_t>(ws, L.row_of);
+  ra.cnt_pre = at<int32_t>(ws, L.cnt_pre);
+  ra.dwraw = pa.dwraw;
+  ra.dout = grad->dout;
+  ra.b2 = reinterpret_cast<const __nv_bfloat16*>(io->b2);
+  ra.Wg = reinterpret_cast<const __nv_bfloat16*>(io->Wg);
+  ra.d_aux = grad->d_aux;
+  ra.d_z = grad->d_z;
+  ra.dlogits = at<float>(ws, L.dlogits);
+  ra.dw_out = grad->dw;
+  ra.dx = grad->dx;
+  ++g_launches;
+  if ((st = cuda_status(launch_router_bwd(ra, stream))) != MOE_OK) return st;
+
+  GateWgradArgs wa{};
+  wa.T = shape->T;
+  wa.H = shape->H;
+  wa.E = shape->E;
+  wa.x = reinterpret_cast<const __nv_bfloat16*>(io->x);
+  wa.dlogits = ra.dlogits;
+  wa.dWg = grad->dWg;
+  wa.dbg = grad->dbg;
+  ++g_launches;
+  return cuda_status(launch_gate_wgrad(wa, stream));
 }
 
 moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_io_t* io, const void* x_host, float* out_host,

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 #include "../../include/moe.h"
@@ -27,6 +28,9 @@ enum DevError : int {
 struct WsLayout {
   size_t status, offsets, cnt_pre, chunk_hist, chunk_base, loss_part, row_of, row_token, row_slot, x_perm, h, y,
       scores, tok_count, total;
+  // training sections, after the inference ones: router logits [T,E] f32, pre-activation u, dout rows
+  // (plain and weighted), du (all bf16), per-row dw partial sums, dlogits [T,E] f32
+  size_t logits, u, dperm, dyperm, du, dwraw, dlogits, train_total;
   int nblk;       // router chunks = ceil(T / kChunk)
   long long rows; // rows of x_perm / h / y: T*k, or E*C under expert choice
   int ec_cap;     // C under expert choice, else 0
@@ -50,6 +54,7 @@ struct RouterArgs {
   // tok_count[t] is cleared for the selection that follows
   float* scores;
   int32_t* tok_count;
+  float* logits_out;  // training forward: logits [T,E] for the backward pass (else null)
 };
 
 struct EcSelectArgs {
@@ -122,6 +127,7 @@ struct FfnArgs {
   float* y;
   float* out;
   int fuse_combine;
+  void* u_out;  // training forward: pre-activation u [rows, F] (bf16 path only; else null)
   int32_t* status;
   long long wait_limit;
   int num_sms;
@@ -138,6 +144,91 @@ cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
 cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);
 cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st);
+
+// ---- backward pass ----
+struct BwdPrepArgs {
+  int T, H, E, k;
+  const int32_t* offsets;
+  const int32_t* row_token;
+  const int32_t* row_slot;
+  const float* topk_w;
+  const float* dout;  // [T,H]
+  void* dperm;        // [rows,H] bf16 out
+  void* dyperm;       // [rows,H] bf16 out
+  float* dwraw;       // [rows] cleared
+  float* dx;          // [T,H] cleared
+  float* dWg;         // [H,E] cleared
+  float* dbg;         // [E] cleared, or null
+};
+
+struct BiasGradArgs {
+  int H, F, E, k;
+  const int32_t* offsets;
+  const int32_t* row_token;
+  const int32_t* row_slot;
+  const float* topk_w;
+  const float* dout;
+  const void* du;  // [rows,F] bf16
+  float* db1;      // [E,F] or null
+  float* db2;      // [E,H] or null
+};
+
+struct RouterBwdArgs {
+  int T, H, E, k;
+  const float* logits;  // [T,E] from the training forward
+  const int32_t* topk_idx;
+  const float* topk_w;
+  const uint8_t* dropped;
+  const int32_t* row_of;
+  const int32_t* cnt_pre;
+  const float* dwraw;
+  const float* dout;
+  const __nv_bfloat16* b2;  // [E,H] or null
+  const __nv_bfloat16* Wg;  // [H,E]
+  float d_aux, d_z;
+  float* dlogits;  // [T,E] out
+  float* dw_out;   // [T,k] out, or null
+  float* dx;       // [T,H] += Wg dlogits
+};
+
+struct GateWgradArgs {
+  int T, H, E, chunk;
+  const __nv_bfloat16* x;
+  const float* dlogits;
+  float* dWg;
+  float* dbg;  // or null
+};
+
+struct BwdGemmArgs {
+  int T, H, E, F, k, rows_cap, act;
+  long long avg_rows;
+  const int32_t* offsets;
+  const int32_t* row_token;
+  const int32_t* row_slot;
+  const float* topk_w;
+  const void* W1;
+  const void* W2;
+  const void* x_perm;
+  const void* h;
+  const void* u;
+  const void* dperm;
+  const void* dyperm;
+  void* du;
+  float* dwraw;
+  float* dx;
+  float* dW1;
+  float* dW2;
+  int32_t* status;
+  long long wait_limit;
+  int num_sms;
+};
+
+cudaError_t launch_bwd_prep(const BwdPrepArgs& a, cudaStream_t st);
+cudaError_t launch_bias_grad(const BiasGradArgs& a, cudaStream_t st);
+cudaError_t launch_router_bwd(const RouterBwdArgs& a, cudaStream_t st);
+cudaError_t launch_gate_wgrad(GateWgradArgs a, cudaStream_t st);
+// dgrad of W2 (du, dw partials), dgrad of W1 (scatter-add into dx), weight gradients of W2 and W1
+cudaError_t launch_bwd_gemms_sm100(const BwdGemmArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st);
 cudaError_t launch_ec_combine(const float* y, const int32_t* row_token, const int32_t* row_slot, const float* topk_w,
                               int rows, int E, int H, float* out, cudaStream_t st);

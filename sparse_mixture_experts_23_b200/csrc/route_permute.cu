@@ -119,6 +119,14 @@ __device__ void router_finish(const RouterArgs& a, const float* logits, int epad
       continue;
     }
 
+    if (a.logits_out != nullptr) {  // training forward: the backward pass recomputes p from these
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        if (j < NJ && e < E) a.logits_out[(size_t)t * E + e] = lv[j];
+      }
+    }
+
     // top-k: k rounds of a warp arg-max with ties to the lower index
     unsigned taken = 0;
     float psel_sum = 0.f;

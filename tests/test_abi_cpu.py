@@ -205,3 +205,33 @@ def test_expert_choice_workspace_and_layout(lib):
     assert FAKE + v_ec.bytes - v_ec.scores >= 8 * 100 * 4 + 100 * 4
     # the no-workspace router does not take expert choice
     assert moe.moe_route_noalloc(ec, _io()) == moe.MOE_ERR_UNSUPPORTED
+
+
+def _grad(**over):
+    g = moe.Grad(FAKE, 0.0, 0.0, *([FAKE] * 8))
+    for k, v in over.items():
+        setattr(g, k, v)
+    return g
+
+
+def test_training_entry_points_validate_before_launch(lib):
+    """moe_forward_train / moe_backward: bf16 token choice only, a training-sized workspace, and bias
+    gradients exactly where the layer has biases; every refusal happens before any launch."""
+    L = moe.load_library()
+    s = _shape(T=64, H=64, E=4, k=2, F=128, dtype="bf16")
+    n_inf, n_train = moe.moe_workspace_size(s), moe.moe_train_workspace_size(s)
+    assert n_train > n_inf > 0
+    assert moe.moe_forward_train(s, _io(), FAKE, n_inf) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_backward(s, _io(), _grad(), FAKE, n_inf) == moe.MOE_ERR_WORKSPACE
+    f32 = _shape(T=64, H=64, E=4, k=2, F=128, dtype="f32")
+    assert moe.moe_forward_train(f32, _io(), FAKE, 1 << 40) == moe.MOE_ERR_UNSUPPORTED
+    ec = _shape(T=64, H=64, E=4, k=2, F=128, dtype="bf16")
+    ec.routing = moe.MOE_ROUTING_EXPERT_CHOICE
+    assert moe.moe_backward(ec, _io(), _grad(), FAKE, 1 << 40) == moe.MOE_ERR_UNSUPPORTED
+    # bias gradient present without the bias, or missing with it
+    assert moe.moe_backward(s, _io(bg=None), _grad(), FAKE, n_train) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_backward(s, _io(), _grad(db1=None), FAKE, n_train) == moe.MOE_ERR_INVALID_ARG
+    for f in ("dout", "dx", "dWg", "dW1", "dW2"):
+        assert moe.moe_backward(s, _io(), _grad(**{f: None}), FAKE, n_train) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_backward(ctypes.byref(s), ctypes.byref(_io()), None, FAKE, n_train, None) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_train_workspace_size(_shape(T=-1)) == 0

@@ -1,0 +1,154 @@
+"""Parity of the backward pass on the GPU against the fp64 oracle's chain rule, through the C ABI.
+
+The GPU's own routing (top-k, drops) is fed to the oracle, so a near-tie flip cannot move a
+gradient.  Tolerance, per gradient tensor: max|d| <= 4e-2 * RMS(ref) and a relative Frobenius error
+<= 1e-2 (the GPU keeps dout rows, du, h and u in bf16 between the GEMMs, so each weight-gradient
+product carries two bf16 roundings; the oracle is fp64 throughout).
+
+  small layers   every gradient in full: dx, dWg, dbg, dW1, db1, dW2, db2 and the per-slot dw
+  Mixtral shape  dx and dw on sampled tokens, dW1 / dW2 / db1 on sampled FFN columns of every
+                 expert, db2 in full, dWg / dbg in full from the oracle's router backward fed the
+                 GPU's dw (every token's dw would need every token's expert output)
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from moe_testlib import TOL_BWD_FRO, TOL_BWD_MAX, fro_rel, rms_rel, sample_tokens, shape_of, upload
+
+pytestmark = pytest.mark.gpu
+
+D_AUX, D_Z = 0.01, 0.001  # the loss coefficients the pages quote (Core Concepts 3)
+
+
+def _cfg(name, T, H, E, k, F, CF, seed, **kw):
+    return synth.LayerConfig(name, T=T, H=H, E=E, k=k, F=F, CF=CF, dtype="bf16", seed=seed, **kw)
+
+
+SMALL = [
+    _cfg("bwd_single_tiles", 200, 128, 4, 2, 256, math.inf, 51),        # 128-row tiles, N = 128 / 256
+    _cfg("bwd_ragged", 100, 128, 6, 3, 192, 1.0, 52),                    # N = 192 -> 64-wide tiles, drops
+    _cfg("bwd_pair_tiles", 1500, 256, 4, 2, 512, 1.1, 53),               # CTA-pair dgrad, half tiles, drops
+    _cfg("bwd_silu_nobias", 600, 256, 4, 2, 512, 1.25, 54, act="silu", bias=False),
+    _cfg("bwd_top1", 300, 128, 8, 1, 256, 1.25, 55),
+]
+
+
+def _lib():
+    import sparse_mixture_experts_23_b200 as moe
+    from sparse_mixture_experts_23_b200 import build as moe_build
+
+    moe_build.build()
+    return moe
+
+
+def _run(cfg, dout):
+    import torch
+
+    moe = _lib()
+    inp = synth.make_inputs(cfg)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp), train=True)
+    buf.forward_train()
+    grads = buf.make_grads()
+    dout_d = torch.from_numpy(dout.astype(np.float32)).cuda()
+    buf.backward(dout_d, grads, D_AUX, D_Z)
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+    res = {n: t.cpu().numpy().astype(np.float64) for n, t in grads.items()}
+    res.update(inp=inp, topk_idx=buf.topk_idx.cpu().numpy(), dropped=buf.dropped.cpu().numpy(),
+               topk_w=buf.topk_w.cpu().numpy().astype(np.float64), launches=moe.moe_last_launch_count(),
+               out=buf.out.cpu().numpy())
+    # the training forward gives the same out as the inference forward
+    buf2 = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf2.forward()
+    torch.cuda.synchronize()
+    res["out_inference"] = buf2.out.cpu().numpy()
+    del buf, buf2
+    torch.cuda.empty_cache()
+    return res
+
+
+def _check(name, got, ref):
+    err, fro = rms_rel(got, ref), fro_rel(got, ref)
+    print(f"  {name}: max {err:.3e} x RMS, Frobenius {fro:.3e}")
+    assert err <= TOL_BWD_MAX and fro <= TOL_BWD_FRO, (name, err, fro)
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_backward_small_all_gradients(cfg):
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    r = _run(cfg, dout)
+    inp = r["inp"]
+    # same out as the inference forward: bit for bit when at most two fp32 adds meet in an element
+    if cfg.k <= 2:
+        assert np.array_equal(r["out"], r["out_inference"])
+    else:
+        np.testing.assert_allclose(r["out"], r["out_inference"], rtol=0, atol=1e-6 * np.abs(r["out"]).max())
+    ref = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, dout,
+                          D_AUX, D_Z, act=cfg.act, topk_idx=r["topk_idx"], dropped=r["dropped"])
+    print(cfg.name)
+    _check("dw", r["dw"], ref.dw)
+    assert (r["dw"][r["dropped"].astype(bool)] == 0).all()
+    _check("dx", r["dx"], ref.dx)
+    _check("dW1", r["dW1"], ref.dW1)
+    _check("dW2", r["dW2"], ref.dW2)
+    _check("dWg", r["dWg"], ref.dWg)
+    if cfg.bias:
+        _check("db1", r["db1"], ref.db1)
+        _check("db2", r["db2"], ref.db2)
+        _check("dbg", r["dbg"], ref.dbg)
+    else:
+        assert "db1" not in r and "dbg" not in r
+    assert r["launches"] == (8 if cfg.bias else 7)
+
+
+def test_backward_mixtral_shape_sampled():
+    cfg = synth.CONFIGS["mixtral"]
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    r = _run(cfg, dout)
+    inp = r["inp"]
+    idx, drp, w = r["topk_idx"], r["dropped"], r["topk_w"]
+    E, k = cfg.E, cfg.k
+    print("mixtral")
+    # dx and dw on sampled tokens: expert paths + router path (the latter from the GPU's dw)
+    toks = sample_tokens(cfg.T, 6, seed=cfg.seed)
+    ex_dx = np.zeros((len(toks), cfg.H))
+    ref_dw = np.zeros((len(toks), k))
+    for i, t in enumerate(toks):
+        for s in range(k):
+            if drp[t, s]:
+                continue
+            dxp, dws, _ = oracle.bwd_slot(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, t, idx[t, s], dout[t], w[t, s],
+                                          cfg.dtype, cfg.act)
+            ex_dx[i] += dxp
+            ref_dw[i, s] = dws
+    _check("dw (sampled tokens)", r["dw"][toks], ref_dw)
+    cnt_pre = np.bincount(idx.reshape(-1), minlength=E).astype(np.int32)
+    dl, dWg, dbg, dxr = oracle.bwd_router(inp.x, inp.Wg, inp.bg, idx, cnt_pre, r["dw"], D_AUX, D_Z, cfg.dtype)
+    _check("dWg (router fed the GPU's dw)", r["dWg"], dWg)
+    _check("dbg (router fed the GPU's dw)", r["dbg"], dbg)
+    _check("dx (sampled tokens)", r["dx"][toks], ex_dx + dxr[toks])
+    # weight gradients at sampled FFN columns of every expert
+    rng = np.random.default_rng(cfg.seed)
+    cols = np.sort(rng.choice(cfg.F, size=6, replace=False)).astype(np.int32)
+    g2, g1, gb1, gb2 = [], [], [], []
+    r2, r1, rb1, rb2 = [], [], [], []
+    for e in range(E):
+        tt, ss = np.where((idx == e) & (drp == 0))
+        dW2r, dW1c, db1s, db2e = oracle.bwd_expert_weights(inp.x, inp.W1, inp.b1, inp.W2, e, tt.astype(np.int32),
+                                                           w[tt, ss], dout, cols, cfg.dtype, cfg.act)
+        r2.append(dW2r)
+        r1.append(dW1c)
+        rb1.append(db1s)
+        rb2.append(db2e)
+        g2.append(r["dW2"][e][cols])
+        g1.append(r["dW1"][e][:, cols].T)
+        gb1.append(r["db1"][e][cols])
+        gb2.append(r["db2"][e])
+    _check("dW2 (sampled columns)", np.array(g2), np.array(r2))
+    _check("dW1 (sampled columns)", np.array(g1), np.array(r1))
+    _check("db1 (sampled columns)", np.array(gb1), np.array(rb1))
+    _check("db2", np.array(gb2), np.array(rb2))
