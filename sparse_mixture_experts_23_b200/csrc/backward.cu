@@ -5,8 +5,8 @@
 // row_slot[r], expert e, weight w = topk_w[t,s]; dout = dL/dout.
 //
 //   bwd_prep_kernel       dperm[r] = bf16(dout[t]), dyperm[r] = bf16(w * dout[t]), dwraw[r] = 0;
-//                         clears dx, dWg and dbg
-//   bias_grad_kernel      db2[e] = sum_r w_r dout[t_r] (fp32 dout), db1[e] = sum_r du_r
+//                         clears dx, dWg, dbg, db1 and db2
+//   bias_grad_kernel      db2[e] += sum_r w_r dout[t_r] (fp32 dout), db1[e] += sum_r du_r, by row chunks
 //   router_bwd_kernel     one warp per token: dw per slot (dwraw + dout . b2[e], 0 when dropped),
 //                         renormalisation, softmax, aux- and z-loss terms -> dlogits[t];
 //                         dx[t] += Wg dlogits[t]
@@ -49,33 +49,81 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
     a.dWg[i] = 0.f;
   if (a.dbg)
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < a.E; i += stride) a.dbg[i] = 0.f;
+  if (a.db1)
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (long long)a.E * a.F; i += stride)
+      a.db1[i] = 0.f;
+  if (a.db2)
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (long long)a.E * a.H; i += stride)
+      a.db2[i] = 0.f;
 }
 
-// grid (E, ceil(max(H, F/2) / 256)): thread j of block (e, b) owns column 256*b + j of db2[e] and
-// the column pair 2*(256*b + j) of db1[e]; rows of the expert's segment are summed in order.
+// Bias gradients over 64-row chunks of the permuted rows (a chunk may span experts; rows are
+// grouped by expert, so each thread flushes its running sums with one atomic add per expert met):
+//   db2[e] += sum_r w_r dout[t_r]   (fp32 dout, two columns per thread)
+//   db1[e] += sum_r du[r]           (bf16 du, two columns per thread)
+// grid (ceil(rows / 64), ceil(max(H, F) / 512)); the targets are cleared by bwd_prep_kernel.
+constexpr int kBgRows = 64;
+
 __global__ void __launch_bounds__(256) bias_grad_kernel(BiasGradArgs a) {
-  const int e = blockIdx.x;
-  const int j = blockIdx.y * 256 + threadIdx.x;
-  const int r0 = a.offsets[e], r1 = a.offsets[e + 1];
-  if (a.db2 && j < a.H) {
-    float acc = 0.f;
-    for (int r = r0; r < r1; ++r) {
-      const int t = a.row_token[r];
-      const float w = a.topk_w[(size_t)t * a.k + a.row_slot[r]];
-      acc = fmaf(w, a.dout[(size_t)t * a.H + j], acc);
+  __shared__ int tok_s[kBgRows];
+  __shared__ float w_s[kBgRows];
+  __shared__ int e_s[kBgRows];
+  __shared__ int offs_s[257];
+  const int kept = a.offsets[a.E];
+  const int r0 = blockIdx.x * kBgRows;
+  if (r0 >= kept) return;
+  const int nr = min(kBgRows, kept - r0);
+  for (int i = threadIdx.x; i <= a.E; i += 256) offs_s[i] = a.offsets[i];
+  __syncthreads();
+  if (threadIdx.x < nr) {
+    const int r = r0 + threadIdx.x;
+    const int t = a.row_token[r];
+    tok_s[threadIdx.x] = t;
+    w_s[threadIdx.x] = a.topk_w[(size_t)t * a.k + a.row_slot[r]];
+    int lo = 0, hi = a.E;  // expert of row r: the last e with offsets[e] <= r
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (offs_s[mid] <= r) lo = mid;
+      else hi = mid;
     }
-    a.db2[(size_t)e * a.H + j] = acc;
+    e_s[threadIdx.x] = lo;
   }
-  if (a.db1 && 2 * j < a.F) {
+  __syncthreads();
+  const int c = 2 * (blockIdx.y * 256 + threadIdx.x);  // first of this thread's two columns
+  if (a.db2 && c < a.H) {
     float2 acc = make_float2(0.f, 0.f);
+    int cur = e_s[0];
+    for (int i = 0; i < nr; ++i) {
+      if (e_s[i] != cur) {
+        atomicAdd(a.db2 + (size_t)cur * a.H + c, acc.x);
+        atomicAdd(a.db2 + (size_t)cur * a.H + c + 1, acc.y);
+        acc = make_float2(0.f, 0.f);
+        cur = e_s[i];
+      }
+      const float2 d = *reinterpret_cast<const float2*>(a.dout + (size_t)tok_s[i] * a.H + c);
+      acc.x = fmaf(w_s[i], d.x, acc.x);
+      acc.y = fmaf(w_s[i], d.y, acc.y);
+    }
+    atomicAdd(a.db2 + (size_t)cur * a.H + c, acc.x);
+    atomicAdd(a.db2 + (size_t)cur * a.H + c + 1, acc.y);
+  }
+  if (a.db1 && c < a.F) {
     const __nv_bfloat162* du = reinterpret_cast<const __nv_bfloat162*>(a.du);
-    for (int r = r0; r < r1; ++r) {
-      const float2 v = __bfloat1622float2(du[(size_t)r * (a.F / 2) + j]);
+    float2 acc = make_float2(0.f, 0.f);
+    int cur = e_s[0];
+    for (int i = 0; i < nr; ++i) {
+      if (e_s[i] != cur) {
+        atomicAdd(a.db1 + (size_t)cur * a.F + c, acc.x);
+        atomicAdd(a.db1 + (size_t)cur * a.F + c + 1, acc.y);
+        acc = make_float2(0.f, 0.f);
+        cur = e_s[i];
+      }
+      const float2 v = __bfloat1622float2(du[((size_t)(r0 + i) * a.F + c) / 2]);
       acc.x += v.x;
       acc.y += v.y;
     }
-    a.db1[(size_t)e * a.F + 2 * j] = acc.x;
-    a.db1[(size_t)e * a.F + 2 * j + 1] = acc.y;
+    atomicAdd(a.db1 + (size_t)cur * a.F + c, acc.x);
+    atomicAdd(a.db1 + (size_t)cur * a.F + c + 1, acc.y);
   }
 }
 
@@ -128,9 +176,15 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
     float d = 0.f;
     if (!a.dropped[(size_t)t * k + q]) {
       float bdot = 0.f;
-      if (a.b2) {
+      if (a.b2) {  // dout[t] . b2[e], four columns per lane per step (H is a multiple of 64)
         const __nv_bfloat16* b2 = a.b2 + (size_t)e * H;
-        for (int h = lane; h < H; h += 32) bdot = fmaf(a.dout[(size_t)t * H + h], __bfloat162float(b2[h]), bdot);
+        for (int h = 4 * lane; h < H; h += 128) {
+          const float4 d = *reinterpret_cast<const float4*>(a.dout + (size_t)t * H + h);
+          const uint2 bb = *reinterpret_cast<const uint2*>(b2 + h);
+          const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb.x));
+          const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb.y));
+          bdot = fmaf(d.x, b01.x, fmaf(d.y, b01.y, fmaf(d.z, b23.x, fmaf(d.w, b23.y, bdot))));
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) bdot += __shfl_xor_sync(0xffffffffu, bdot, o);
       }
@@ -175,58 +229,83 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
     }
   }
   __syncwarp();
-  // dx[t] += Wg dlogits[t]
-  for (int h = lane; h < H; h += 32) {
-    const __nv_bfloat16* wrow = a.Wg + (size_t)h * E;
-    float acc = 0.f;
-    for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(wrow[e]), dl_s[warp][e], acc);
-    a.dx[(size_t)t * H + h] += acc;
+  // dx[t] += Wg dlogits[t]: four rows of Wg per lane per step
+  for (int h = 4 * lane; h < H; h += 128) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    if (E % 8 == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4* wrow = reinterpret_cast<const uint4*>(a.Wg + (size_t)(h + i) * E);
+        for (int e8 = 0; e8 < E / 8; ++e8) {
+          const uint4 v = wrow[e8];
+          const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(w2[q]);
+            acc[i] = fmaf(f.x, dl_s[warp][8 * e8 + 2 * q], fmaf(f.y, dl_s[warp][8 * e8 + 2 * q + 1], acc[i]));
+          }
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        for (int e = 0; e < E; ++e) acc[i] = fmaf(__bfloat162float(a.Wg[(size_t)(h + i) * E + e]), dl_s[warp][e], acc[i]);
+    }
+    float4* dxp = reinterpret_cast<float4*>(a.dx + (size_t)t * H + h);
+    float4 v = *dxp;
+    v.x += acc[0];
+    v.y += acc[1];
+    v.z += acc[2];
+    v.w += acc[3];
+    *dxp = v;
   }
 }
 
-// grid (ceil(H / 256), token chunks): thread j owns h = 256*bx + j and accumulates x[t,h] dlogits[t,:]
-// over the chunk's tokens (staged in shared memory), then adds into dWg; block column 0 also adds
-// the chunk's dlogits sums into dbg.
-constexpr int kGwTokens = 32;
+// grid (ceil(H / 512), token chunks): thread j owns columns h, h+1 (h = 2 (256 bx + j)) and, for
+// every group of 8 experts, accumulates x[t, h..h+1] dlogits[t, group] over the chunk's tokens
+// (dlogits staged in shared memory), then adds into dWg; block column 0 also adds the chunk's sums
+// of dlogits into dbg.  dWg and dbg are cleared by bwd_prep_kernel.
+constexpr int kGwTokens = 128;
 
 __global__ void __launch_bounds__(256) gate_wgrad_kernel(GateWgradArgs a) {
-  __shared__ float dl[kGwTokens][32];
-  __shared__ __nv_bfloat16 xs[kGwTokens][256];
+  __shared__ float dl[kGwTokens][8];
   const int E = a.E, H = a.H;
-  const int h = blockIdx.x * 256 + threadIdx.x;
-  const int tc0 = blockIdx.y * a.chunk, tc1 = min(a.T, tc0 + a.chunk);
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    const int ne = min(32, E - e0);
-    float acc[32];
+  const int h = 2 * (blockIdx.x * 256 + threadIdx.x);
+  const int t0 = blockIdx.y * kGwTokens, nt = min(kGwTokens, a.T - t0);
+  const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(a.x);
+  for (int e0 = 0; e0 < E; e0 += 8) {
+    const int ne = min(8, E - e0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kGwTokens * 8; i += 256) {
+      const int tt = i / 8, q = i % 8;
+      dl[tt][q] = (tt < nt && q < ne) ? a.dlogits[(size_t)(t0 + tt) * E + e0 + q] : 0.f;
+    }
+    __syncthreads();
+    if (h < H) {
+      float acc0[8], acc1[8];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) acc[q] = 0.f;
-    float bsum = 0.f;
-    for (int t0 = tc0; t0 < tc1; t0 += kGwTokens) {
-      const int nt = min(kGwTokens, tc1 - t0);
-      __syncthreads();
-      for (int i = threadIdx.x; i < nt * ne; i += 256) {
-        const int tt = i / ne, q = i % ne;
-        dl[tt][q] = a.dlogits[(size_t)(t0 + tt) * E + e0 + q];
-      }
-      for (int tt = 0; tt < nt; ++tt) xs[tt][threadIdx.x] = h < H ? a.x[(size_t)(t0 + tt) * H + h] : __float2bfloat16(0.f);
-      __syncthreads();
-      if (h < H) {
-        for (int tt = 0; tt < nt; ++tt) {
-          const float xv = __bfloat162float(xs[tt][threadIdx.x]);
+      for (int q = 0; q < 8; ++q) acc0[q] = acc1[q] = 0.f;
+#pragma unroll 4
+      for (int tt = 0; tt < nt; ++tt) {
+        const float2 xv = __bfloat1622float2(x2[((size_t)(t0 + tt) * H + h) / 2]);
 #pragma unroll
-          for (int q = 0; q < 32; ++q)
-            if (q < ne) acc[q] = fmaf(xv, dl[tt][q], acc[q]);
+        for (int q = 0; q < 8; ++q) {
+          acc0[q] = fmaf(xv.x, dl[tt][q], acc0[q]);
+          acc1[q] = fmaf(xv.y, dl[tt][q], acc1[q]);
         }
       }
-      if (a.dbg && blockIdx.x == 0 && threadIdx.x < ne)
-        for (int tt = 0; tt < nt; ++tt) bsum += dl[tt][threadIdx.x];
-    }
-    if (h < H) {
 #pragma unroll
-      for (int q = 0; q < 32; ++q)
-        if (q < ne) atomicAdd(a.dWg + (size_t)h * E + e0 + q, acc[q]);
+      for (int q = 0; q < 8; ++q)
+        if (q < ne) {
+          atomicAdd(a.dWg + (size_t)h * E + e0 + q, acc0[q]);
+          atomicAdd(a.dWg + (size_t)(h + 1) * E + e0 + q, acc1[q]);
+        }
     }
-    if (a.dbg && blockIdx.x == 0 && threadIdx.x < ne) atomicAdd(a.dbg + e0 + threadIdx.x, bsum);
+    if (a.dbg && blockIdx.x == 0 && threadIdx.x < ne) {
+      float bsum = 0.f;
+      for (int tt = 0; tt < nt; ++tt) bsum += dl[tt][threadIdx.x];
+      atomicAdd(a.dbg + e0 + threadIdx.x, bsum);
+    }
   }
 }
 
@@ -238,8 +317,8 @@ cudaError_t launch_bwd_prep(const BwdPrepArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_bias_grad(const BiasGradArgs& a, cudaStream_t st) {
-  const int cols = a.H > a.F / 2 ? a.H : a.F / 2;
-  dim3 grid(a.E, (cols + 255) / 256);
+  const int cols = a.H > a.F ? a.H : a.F;
+  dim3 grid((a.rows_cap + kBgRows - 1) / kBgRows, (cols + 511) / 512);
   bias_grad_kernel<<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
@@ -250,14 +329,7 @@ cudaError_t launch_router_bwd(const RouterBwdArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_gate_wgrad(GateWgradArgs a, cudaStream_t st) {
-  // enough token chunks to fill the GPU about twice, given ceil(H / 256) column blocks
-  const int hb = (a.H + 255) / 256;
-  int chunks = (2 * 148 + hb - 1) / hb;
-  if (chunks < 1) chunks = 1;
-  a.chunk = (a.T + chunks - 1) / chunks;
-  if (a.chunk < kGwTokens) a.chunk = kGwTokens;
-  chunks = (a.T + a.chunk - 1) / a.chunk;
-  dim3 grid(hb, chunks);
+  dim3 grid((a.H + 511) / 512, (a.T + kGwTokens - 1) / kGwTokens);
   gate_wgrad_kernel<<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }

@@ -1026,6 +1026,266 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// The same weight gradients on CTA pairs (cta_group::2): 256 x 256 tiles of D[e], each CTA holding
+// 128 of the m rows (its A^T half) and 128 of the n columns (its B half), with stages of 128
+// contraction rows.  Each CTA's loads land on its own full barrier; on a segment's last stage each
+// CTA's MMA warp zeroes its own rows past the segment.  The peer then signals the leader through a
+// remote arrive on the leader's ready barrier, and the leader issues the pair's MMAs once both
+// halves are in place.  Commits free the stage (and hand the accumulator to the epilogue) in both
+// CTAs at once.
+struct WgPairCfg {
+  static constexpr int kTileM = 256, kTileN = 256, kStageK = 128;
+  static constexpr int kStages = 3;
+  static constexpr int kBoxBytes = 64 * kStageK * 2;  // one 64 (m or n) x 128 (k) box: 16 KB
+  static constexpr int kABytes = 2 * kBoxBytes;        // this CTA's 128 m values
+  static constexpr int kBBytes = 2 * kBoxBytes;        // this CTA's 128 n values
+  static constexpr int kStageBytes = kABytes + kBBytes;  // 64 KB per CTA
+  static constexpr int kTmemCols = 2 * kTileN;
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kNumBars = 3 * kStages + 4 + 1;  // full, empty, ready; tfull x2, tempty x2; drain
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kOffsOff = kMiscOff + 16;
+  static constexpr int kStgOff = (kOffsOff + 260 * 4 + 1023) & ~1023;
+  static constexpr int kSmemBytes = 1024 + kStgOff + kEpiWarps * kStgWarpBytes;
+  static_assert(kStgOff % 16 == 0 && kSmemBytes <= 232448, "shared-memory plan");
+  // kind::f16, D fp32, A and B bf16 MN-major, N = 256, M = 256 over the pair
+  static constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                     ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    wgrad_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmD, WgradArgs g) {
+  using C = WgPairCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto ready_bar = [&](int s) { return bar0 + 8u * (2 * C::kStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (3 * C::kStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  int* offs = reinterpret_cast<int*>(smem + C::kOffsOff);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* stg = reinterpret_cast<float*>(smem + C::kStgOff + (warp >= 2 ? warp - 2 : 0) * kStgWarpBytes);
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+  const int E = g.E;
+  const int MT = (g.M + C::kTileM - 1) / C::kTileM, NT = (g.N + C::kTileN - 1) / C::kTileN;
+  const int per_e = MT * NT;
+  const int total = E * per_e;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+      mbar_init(ready_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 2 * kEpiWarps);  // every epilogue warp of both CTAs
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  for (int i = threadIdx.x; i <= E; i += kThreads) offs[i] = g.offsets[i];
+  if (warp == 1) tmem_alloc_pair(smem_u32(tmem_slot), C::kTmemCols);
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before any cross-CTA signal
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto decode = [&](int tile, int& e, int& m0, int& n0) {
+    e = tile / per_e;
+    const int local = tile - e * per_e;
+    n0 = (local / MT) * C::kTileN;
+    m0 = (local % MT) * C::kTileM;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs) -----
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int armed[C::kStages];
+      for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
+      bool ok = true;
+      for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
+        int e, m0, n0;
+        decode(tile, e, m0, n0);
+        const int r0 = offs[e], KB = (offs[e + 1] - r0 + C::kStageK - 1) / C::kStageK;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = sbase + stage * C::kStageBytes;
+          const uint32_t b_dst = a_dst + C::kABytes;
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          armed[stage] = (int)phase;
+          const int k0 = r0 + kb * C::kStageK;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            tma_load_2d(a_dst + j * C::kBoxBytes, &tmA, m0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
+            tma_load_2d(b_dst + j * C::kBoxBytes, &tmB, n0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok || *abort_flag) {
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed[s] >= 0) {
+            volatile int dummy = 0;
+            mbar_wait(full_bar(s), (uint32_t)armed[s], g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ stage check (both) + MMA (leader)
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true;
+    bool issued = false;
+    const uint32_t leader_ready0 = peer_addr(ready_bar(0), 0);
+    for (int tile = cluster_id; tile < total && ok; tile += nclusters, ++it) {
+      int e, m0, n0;
+      decode(tile, e, m0, n0);
+      const int r0 = offs[e], cnt = offs[e + 1] - r0, KB = (cnt + C::kStageK - 1) / C::kStageK;
+      const int buf = it & 1;
+      const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+      if (leader) {
+        if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(buf), tphase ^ 1u, g.wait_limit, abort_flag, g.status,
+                                               kDevTimeoutMma))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kTileN);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status,
+                                               kDevTimeoutMma))) {
+          ok = false;
+          break;
+        }
+        const uint32_t a_addr = sbase + stage * C::kStageBytes;
+        const int valid = min(C::kStageK, cnt - kb * C::kStageK);
+        if (valid < C::kStageK) {
+          // this CTA's rows valid..127 of its four boxes: whole 128-byte lines
+          const int per_box = (C::kStageK - valid) * 8;
+          for (int i = lane; i < 4 * per_box; i += 32) {
+            const int box = i / per_box, rem = i - box * per_box;
+            const uint32_t addr = a_addr + box * C::kBoxBytes + (valid + rem / 8) * 128 + (rem % 8) * 16;
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};\n" ::"r"(addr), "r"(0u) : "memory");
+          }
+          fence_async_smem();
+        }
+        __syncwarp();
+        if (!leader) {
+          // this half is ready: tell the leader (its ready barrier of this stage)
+          if (lane == 0) mbar_arrive_cluster(leader_ready0 + 8u * stage);
+        } else {
+          if (!__all_sync(0xffffffffu, mbar_wait_cluster(ready_bar(stage), phase, g.wait_limit, abort_flag, g.status,
+                                                         kDevTimeoutMma))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+            for (int kk = 0; kk < C::kStageK / 16; ++kk)
+              mma_bf16_pair(d_tmem, desc_mnmajor(a_addr + kk * 16 * 128, C::kBoxBytes),
+                            desc_mnmajor(b_addr + kk * 16 * 128, C::kBoxBytes), C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+            mma_commit_both(empty_bar(stage));  // frees this stage in both CTAs once its MMAs are done
+          }
+          issued = true;
+        }
+        __syncwarp();
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      if (leader && lane == 0) mma_commit_both(tfull_bar(buf));  // with no rows this arrives at once
+      __syncwarp();
+    }
+    if (leader && (!ok || *abort_flag) && issued && lane == 0) {
+      mma_commit_pair(drain_bar);
+      volatile int dummy = 0;
+      mbar_wait(drain_bar, 0, g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5, both) --
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const uint32_t tempty_leader0 = peer_addr(tempty_bar(0), 0);
+    const uint32_t tempty_leader1 = peer_addr(tempty_bar(1), 0);
+    int it = 0;
+    for (int tile = cluster_id; tile < total; tile += nclusters, ++it) {
+      int e, m0, n0;
+      decode(tile, e, m0, n0);
+      const bool empty = offs[e + 1] == offs[e];
+      const int buf = it & 1;
+      const uint32_t tphase = (uint32_t)((it >> 1) & 1);
+      const bool got = mbar_wait(tfull_bar(buf), tphase, g.wait_limit, abort_flag, g.status, kDevTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int row0 = m0 + 128 * (int)rank + quarter * 32;  // this warp's 32 rows of D
+      constexpr int kChunks = C::kTileN / 32 / (kEpiWarps / 4);
+      uint8_t* box = reinterpret_cast<uint8_t*>(stg);  // 32 x 32 fp32, 128-byte rows, 128-byte swizzle
+#pragma unroll 1
+      for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::kTileN + c * 32), r);
+        const int col = n0 + c * 32;
+        if (row0 >= g.M || col >= g.N) continue;  // wholly past the edge (partial parts are clipped)
+        if (lane == 0) bulk_wait_read0();  // the previous box has left the staging buffer
+        __syncwarp();
+        uint8_t* row = box + lane * 128;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 v = empty ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+          *reinterpret_cast<uint4*>(row + ((q ^ (lane & 7)) * 16)) = v;
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tmD, smem_u32(box), col, row0, e);  // rows >= M and columns >= N are not written
+          bulk_commit();
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+    }
+    if (lane == 0) bulk_wait0();  // this warp's boxes are written before exit
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync_all();  // neither CTA frees TMEM or exits while the pair still uses it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
 // One thread waits on a barrier that nothing completes; the bound must end it.
 __global__ void timeout_probe_kernel(int32_t* status, long long limit) {
   __shared__ __align__(8) uint64_t bar;
@@ -1114,17 +1374,32 @@ bool make_map_bk(CUtensorMap* m, const void* base, int E, int N, int K, int box_
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// MN-major operand of the weight gradients: [rows, C] bf16 row-major; box = 64 columns x 64 rows
-bool make_map_rows64(CUtensorMap* m, const void* base, int rows, int C) {
+// MN-major operand of the weight gradients: [rows, C] bf16 row-major; box = 64 columns x box_rows rows
+bool make_map_rows(CUtensorMap* m, const void* base, int rows, int C, int box_rows) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)C * 2};
-  cuuint32_t box[2] = {64, (cuuint32_t)WgCfg::kBK};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Weight-gradient output D[E][M][N] fp32; stores of 32 columns x 32 rows, 128-byte swizzle.  Three
+// dimensions so that rows past M (or columns past N) of a partial tile are clipped, never written
+// into the next expert.
+bool make_map_dw(CUtensorMap* m, float* base, int E, int M, int N) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)N * 4, (cuuint64_t)M * N * 4};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 template <int BN, int EPI, bool BKM = false>
@@ -1179,8 +1454,11 @@ cudaError_t launch_dgrad(const void* A, int rows_cap, const void* W, int E, int 
 
 cudaError_t launch_wgrad(const void* A, const void* B, int rows_cap, int M, int N, const int32_t* offsets, int E,
                          float* out, int32_t* status, long long wait_limit, int grid, cudaStream_t st) {
+  const bool pair = pair_mode_enabled();
+  const int box_rows = pair ? WgPairCfg::kStageK : WgCfg::kBK;
   CUtensorMap ma, mb;
-  if (!make_map_rows64(&ma, A, rows_cap, M) || !make_map_rows64(&mb, B, rows_cap, N)) return cudaErrorInvalidValue;
+  if (!make_map_rows(&ma, A, rows_cap, M, box_rows) || !make_map_rows(&mb, B, rows_cap, N, box_rows))
+    return cudaErrorInvalidValue;
   WgradArgs g{};
   g.offsets = offsets;
   g.E = E;
@@ -1189,6 +1467,14 @@ cudaError_t launch_wgrad(const void* A, const void* B, int rows_cap, int M, int 
   g.out = out;
   g.status = status;
   g.wait_limit = wait_limit;
+  if (pair) {
+    CUtensorMap md;
+    if (!make_map_dw(&md, out, E, M, N)) return cudaErrorInvalidValue;
+    cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(wgrad_pair_kernel), WgPairCfg::kSmemBytes);
+    if (err != cudaSuccess) return err;
+    wgrad_pair_kernel<<<grid & ~1, kThreads, WgPairCfg::kSmemBytes, st>>>(ma, mb, md, g);
+    return cudaGetLastError();
+  }
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(wgrad_kernel), WgCfg::kSmemBytes);
   if (err != cudaSuccess) return err;
   wgrad_kernel<<<grid, kThreads, WgCfg::kSmemBytes, st>>>(ma, mb, g);

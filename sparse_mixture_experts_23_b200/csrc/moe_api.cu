@@ -557,6 +557,9 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   pa.dx = grad->dx;
   pa.dWg = grad->dWg;
   pa.dbg = grad->dbg;
+  pa.F = shape->F;
+  pa.db1 = grad->db1;
+  pa.db2 = grad->db2;
   ++g_launches;
   if ((st = cuda_status(launch_bwd_prep(pa, stream))) != MOE_OK) return st;
 
@@ -596,6 +599,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
     ba.F = shape->F;
     ba.E = shape->E;
     ba.k = shape->k;
+    ba.rows_cap = (int)L.rows;
     ba.offsets = offsets;
     ba.row_token = row_token;
     ba.row_slot = row_slot;

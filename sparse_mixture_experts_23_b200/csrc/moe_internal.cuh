@@ -147,7 +147,7 @@ cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st);
 
 // ---- backward pass ----
 struct BwdPrepArgs {
-  int T, H, E, k;
+  int T, H, E, F, k;
   const int32_t* offsets;
   const int32_t* row_token;
   const int32_t* row_slot;
@@ -159,10 +159,12 @@ struct BwdPrepArgs {
   float* dx;          // [T,H] cleared
   float* dWg;         // [H,E] cleared
   float* dbg;         // [E] cleared, or null
+  float* db1;         // [E,F] cleared, or null
+  float* db2;         // [E,H] cleared, or null
 };
 
 struct BiasGradArgs {
-  int H, F, E, k;
+  int H, F, E, k, rows_cap;
   const int32_t* offsets;
   const int32_t* row_token;
   const int32_t* row_slot;
