@@ -65,10 +65,10 @@ __host__ __device__ inline RouterSmem router_smem(int E, int esize) {
 // Softmax, top-k, renormalisation and the block's loss partials from logits[32][epad] in shared
 // memory (bias already added).  256 threads: warp w handles the chunk's tokens w, w+8, w+16, w+24.
 // psum: [8][epad] floats, hist: [k][E] ints, zw: [8] floats, all shared.
-__device__ void router_finish(const RouterArgs& a, const float* logits, int epad, float* psum, int* hist, float* zw) {
+__device__ void router_finish(const RouterArgs& a, const float* logits, int epad, float* psum, int* hist, float* zw,
+                              int blk) {
   const int E = a.E, T = a.T, k = a.k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int blk = blockIdx.x;
   const int t0 = blk * kChunk;
   for (int i = tid; i < k * E; i += kRouterThreads) hist[i] = 0;
   for (int i = tid; i < 8 * epad; i += kRouterThreads) psum[i] = 0.f;
@@ -187,7 +187,7 @@ __device__ void router_finish(const RouterArgs& a, const float* logits, int epad
     a.loss_part[(size_t)blk * (E + 1) + E] = s;
   }
   if (a.chunk_hist) {
-    const int nblk = gridDim.x;
+    const int nblk = (T + kChunk - 1) / kChunk;  // router chunks
     for (int i = tid; i < k * E; i += kRouterThreads) {
       int s = i / E, e = i % E;
       a.chunk_hist[((size_t)s * nblk + blk) * E + e] = hist[i];
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(RouterArgs a) {
   __syncthreads();
 
   router_finish(a, logits, L.epad, reinterpret_cast<float*>(smem + L.psum), reinterpret_cast<int*>(smem + L.misc),
-                reinterpret_cast<float*>(smem + L.misc + 8 * 256 * 4));
+                reinterpret_cast<float*>(smem + L.misc + 8 * 256 * 4), blockIdx.x);
 }
 
 // Streaming router for bf16 with few experts (E <= 16): memory-bound, so the gate weights stay in
@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_stream_kernel(RouterArg
   }
   __syncthreads();
   router_finish(a, logits, EP, reinterpret_cast<float*>(smem + S::psum_off(H)), reinterpret_cast<int*>(smem + S::misc_off(H)),
-                reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4));
+                reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4), blockIdx.x);
 }
 
 // Tensor-core router for bf16 with E a multiple of 8: the gate GEMM [32 tokens x H] x [H x E] of
@@ -639,7 +639,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_mma_kernel(RouterArgs a
   }
   __syncthreads();
   router_finish(a, logits, P.ep8, reinterpret_cast<float*>(smem + P.psum), reinterpret_cast<int*>(smem + P.misc),
-                reinterpret_cast<float*>(smem + P.misc + 8 * 256 * 4));
+                reinterpret_cast<float*>(smem + P.misc + 8 * 256 * 4), blockIdx.x);
 }
 
 // Register-direct tensor-core router for bf16 with E = 8, 16 or 32 (gate weights resident in
@@ -782,7 +782,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_direct_kernel(RouterArg
   }
   __syncthreads();
   router_finish(a, logits, E, reinterpret_cast<float*>(smem + S::psum_off(H)), reinterpret_cast<int*>(smem + S::misc_off(H)),
-                reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4));
+                reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4), blockIdx.x);
 }
 
 // Per-chunk, per-slot expert histogram from a given topk_idx (standalone permute).
