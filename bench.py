@@ -337,6 +337,10 @@ def run_ours_impl(args, cfg):
     ms_ffn = time_calls(lambda: buf.expert_ffn(True))
     ms_route = time_calls(buf.route)
     ms_permute = time_calls(buf.permute)
+    # standalone combine (the unfused path: y materialised by moe_expert_ffn(fuse_combine=0))
+    buf.permute()
+    buf.expert_ffn(False)
+    ms_combine = time_calls(buf.combine)
     buf.forward()
     torch.cuda.synchronize()
     counts = buf.expert_counts.cpu().numpy()
@@ -376,6 +380,8 @@ def run_ours_impl(args, cfg):
     router_bytes = cfg.T * cfg.H * es + cfg.H * cfg.E * es + cfg.T * cfg.k * 8
     # permute: read the kept x rows, write them to x_perm, clear out (fp32), index traffic
     permute_bytes = kept * cfg.H * es * 2 + cfg.T * cfg.H * 4 + cfg.T * cfg.k * 8
+    # combine: read every kept row of y (fp32), write out (fp32), index and weight traffic
+    combine_bytes = kept * cfg.H * 4 + cfg.T * cfg.H * 4 + cfg.T * cfg.k * 8
     traffic = None
     # ---------------- training step: forward that keeps state + backward (bf16 token choice) -----
     train = None
@@ -431,6 +437,8 @@ def run_ours_impl(args, cfg):
             "ffn_tflops": tflops, "ffn_frac_burst_peak": tflops / peaks["bf16_tflops"],
             "route_gbs": router_bytes / (ms_route / 1000.0) / 1e9,
             "permute_gbs": permute_bytes / (ms_permute / 1000.0) / 1e9,
+            "combine_ms": ms_combine,
+            "combine_gbs": combine_bytes / (ms_combine / 1000.0) / 1e9,
             "hbm_peak_gbs": peaks["hbm_gbs"],
             "layer_roofline_ms": 1000 * max(alg_flops(cfg, kept) / (peaks["bf16_tflops"] * 1e12),
                                             alg_bytes(cfg, touched) / (peaks["hbm_gbs"] * 1e9)),

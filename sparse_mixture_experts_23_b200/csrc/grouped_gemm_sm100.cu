@@ -91,6 +91,7 @@ struct GemmArgs {
   const int32_t* row_slot;
   const float* topk_w;
   int k;
+  int single_rows;  // offsets == null: one segment of this many rows (a plain dense GEMM)
   int32_t* status;
   long long wait_limit;
 };
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
   }
-  for (int i = threadIdx.x; i <= E; i += kThreads) offs[i] = g.offsets[i];
+  for (int i = threadIdx.x; i <= E; i += kThreads) offs[i] = g.offsets ? g.offsets[i] : (i == 0 ? 0 : g.single_rows);
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -1575,6 +1576,27 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   if (err != cudaSuccess) return err;
   ++*launches;
   return cudaSuccess;
+}
+
+// logits[T,E] (fp32) = x[T,H] . Wg[H,E] + bg on the tensor cores: one dense segment through the
+// single-CTA kernel with 128 x 64 tiles and the fp32 store epilogue (bias added there).
+cudaError_t launch_gate_logits_sm100(const void* x, const void* Wg, const void* bg, int T, int H, int E, float* logits,
+                                     int32_t* status, long long wait_limit, int num_sms, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map_a(&ma, x, T, H) || !make_map_b(&mb, Wg, 1, H, E)) return cudaErrorInvalidValue;
+  GemmArgs g{};
+  g.offsets = nullptr;
+  g.single_rows = T;
+  g.E = 1;
+  g.N = E;
+  g.K = H;
+  g.bias = reinterpret_cast<const __nv_bfloat16*>(bg);
+  g.y = logits;
+  g.status = status;
+  g.wait_limit = wait_limit;
+  const int tiles = ((T + BM - 1) / BM) * (E / 64);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  return launch_one<64, EPI_STORE_Y>(ma, mb, g, grid, st);
 }
 
 cudaError_t launch_timeout_probe(int32_t* status, long long limit, cudaStream_t st) {

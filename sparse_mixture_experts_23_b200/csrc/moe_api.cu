@@ -84,10 +84,10 @@ WsLayout ws_layout(const moe_shape_t& s) {
   o = align256(o + (ec ? E * T * 4 : 0));
   L.tok_count = o;
   o = align256(o + (ec ? T * 4 : 0));
+  L.logits = o;  // [T,E] fp32: gate logits (the tensor-core gate's output; saved for the backward pass)
+  o = align256(o + T * E * 4);
   L.total = o;
   // training sections (moe_forward_train / moe_backward), appended after the inference layout
-  L.logits = o;
-  o = align256(o + T * E * 4);
   L.u = o;
   o = align256(o + rows * (size_t)s.F * es);
   L.dperm = o;
@@ -192,8 +192,11 @@ moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaSt
     r.scores = at<float>(ws, L.scores);
     r.tok_count = at<int32_t>(ws, L.tok_count);
   }
-  cudaError_t err = launch_router(r, s->dtype, st);
-  ++g_launches;
+  r.gemm_logits = at<float>(ws, L.logits);
+  r.status = at<int32_t>(ws, L.status);
+  r.wait_limit = g_wait_limit;
+  r.num_sms = num_sms();
+  cudaError_t err = launch_router(r, s->dtype, st, &g_launches);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }

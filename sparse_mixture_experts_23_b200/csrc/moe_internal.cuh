@@ -55,6 +55,12 @@ struct RouterArgs {
   float* scores;
   int32_t* tok_count;
   float* logits_out;  // training forward: logits [T,E] for the backward pass (else null)
+  // [T,E] fp32 scratch: when given (bf16, E a multiple of 64) the gate is one tensor-core GEMM
+  // into it, followed by the per-chunk softmax / top-k / partials kernel
+  float* gemm_logits;
+  int32_t* status;
+  long long wait_limit;
+  int num_sms;
 };
 
 struct EcSelectArgs {
@@ -137,12 +143,14 @@ struct FfnArgs {
 // driver call is made once per (kernel, device) and size, so repeated launches cost nothing.
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 
-cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st);
+cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* launches);
 cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, cudaStream_t st);
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
 cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);
 cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t st, int* launches);
+cudaError_t launch_gate_logits_sm100(const void* x, const void* Wg, const void* bg, int T, int H, int E, float* logits,
+                                     int32_t* status, long long wait_limit, int num_sms, cudaStream_t st);
 cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st);
 
 // ---- backward pass ----

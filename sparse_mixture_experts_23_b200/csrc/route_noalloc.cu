@@ -104,7 +104,8 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   r.topk_w = io->topk_w;
   r.loss_part = loss_part;
   r.chunk_hist = chunk_hist;
-  if (moe::launch_router(r, shape->dtype, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  int launches = 0;  // no gate scratch here, so always the one-kernel router
+  if (moe::launch_router(r, shape->dtype, stream, &launches) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::ReduceArgs a{};
   a.T = shape->T;

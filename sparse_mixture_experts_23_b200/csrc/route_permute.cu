@@ -785,6 +785,23 @@ __global__ void __launch_bounds__(kRouterThreads) router_direct_kernel(RouterArg
                 reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4), blockIdx.x);
 }
 
+// Softmax, top-k, renormalisation and partials of one 32-token chunk from logits that a tensor-core
+// GEMM already wrote to global memory ([T,E] fp32, bias included).
+__global__ void __launch_bounds__(kRouterThreads) router_logits_finish_kernel(RouterArgs a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const int E = a.E;
+  float* logits = reinterpret_cast<float*>(smem);  // [32][E]
+  float* psum = logits + kChunk * E;                 // [8][E]
+  int* misc = reinterpret_cast<int*>(psum + 8 * E);  // [k][E] histogram, then 8 floats
+  const int t0 = blockIdx.x * kChunk;
+  const int n4 = min(kChunk, a.T - t0) * E / 4;
+  const float4* src = reinterpret_cast<const float4*>(a.gemm_logits + (size_t)t0 * E);
+  for (int i = threadIdx.x; i < kChunk * E / 4; i += kRouterThreads)
+    reinterpret_cast<float4*>(logits)[i] = i < n4 ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  router_finish(a, logits, E, psum, misc, reinterpret_cast<float*>(misc + 8 * 256), blockIdx.x);
+}
+
 // Per-chunk, per-slot expert histogram from a given topk_idx (standalone permute).
 __global__ void hist_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int32_t* __restrict__ chunk_hist) {
   __shared__ int hist[8 * 256];
@@ -1053,8 +1070,23 @@ cudaError_t launch_stream(const RouterArgs& a, int nblk, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st) {
+cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* launches) {
   const int nblk = (a.T + kChunk - 1) / kChunk;
+  // bf16, E a multiple of 64, scratch given: the gate is one dense tensor-core GEMM, then the
+  // per-chunk tail (the gate weights are read once per 128-token tile instead of once per chunk)
+  if (a.gemm_logits != nullptr && dtype == MOE_DTYPE_BF16 && a.E % 64 == 0 && a.H % 64 == 0 && !router_mma_disabled()) {
+    cudaError_t err = launch_gate_logits_sm100(a.x, a.Wg, a.bg, a.T, a.H, a.E, a.gemm_logits, a.status, a.wait_limit,
+                                               a.num_sms > 0 ? a.num_sms : 148, st);
+    if (err != cudaSuccess) return err;
+    ++*launches;
+    const int bytes = (kChunk * a.E + 8 * a.E) * 4 + (8 * 256 + 64) * 4;
+    err = ensure_smem_limit(reinterpret_cast<const void*>(router_logits_finish_kernel), bytes);
+    if (err != cudaSuccess) return err;
+    router_logits_finish_kernel<<<nblk, kRouterThreads, bytes, st>>>(a);
+    ++*launches;
+    return cudaGetLastError();
+  }
+  ++*launches;  // every other form is one kernel
   // bf16, E in {8, 16, 32}, Wg^T fits in shared memory: register-direct tensor-core stream over x
   if (dtype == MOE_DTYPE_BF16 && (a.E == 8 || a.E == 16 || a.E == 32) && a.H % 256 == 0 && !router_mma_disabled()) {
     const int bytes = a.E == 8 ? DirectSmem<1>::total(a.H) : (a.E == 16 ? DirectSmem<2>::total(a.H) : DirectSmem<4>::total(a.H));

@@ -104,3 +104,9 @@ def fro_rel(a: np.ndarray, ref: np.ndarray) -> float:
     den = float(np.linalg.norm(ref))
     num = float(np.linalg.norm(a - ref))
     return num / den if den > 0 else num
+
+
+def router_launches(cfg) -> int:
+    """Kernels of the gate: one, or two (tensor-core logits GEMM + per-chunk softmax/top-k) for bf16
+    layers whose expert count is a multiple of 64."""
+    return 2 if cfg.dtype == "bf16" and cfg.E % 64 == 0 else 1

@@ -15,8 +15,8 @@ import pytest
 
 import oracle
 import synth
-from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, out_error, sample_tokens, shape_of,
-                         upload)
+from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, out_error, router_launches, sample_tokens,
+                         shape_of, upload)
 
 pytestmark = pytest.mark.gpu
 
@@ -147,4 +147,4 @@ def test_forward_equals_stages(run):
     assert np.array_equal(run["topk_idx_forward"], run["topk_idx"])
     assert np.array_equal(run["losses_forward"], run["losses"])
     assert np.array_equal(run["out_forward"], run["out"])
-    assert run["launches"] == 5
+    assert run["launches"] == 4 + router_launches(run["cfg"])
