@@ -89,6 +89,8 @@ def _load():
     lib.oracle_bwd_expert_weights.restype = None
     lib.oracle_bwd_router.argtypes = [i64, i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, dbl, dbl, vp, vp, vp, vp]
     lib.oracle_bwd_router.restype = None
+    lib.oracle_bwd_router_ec.argtypes = [i64, i64, i64, c_int, vp, vp, vp, vp, dbl, dbl, vp, vp, vp, vp]
+    lib.oracle_bwd_router_ec.restype = None
     lib.oracle_max_threads.argtypes = []
     lib.oracle_max_threads.restype = c_int
     lib.oracle_set_threads.argtypes = [c_int]
@@ -446,4 +448,60 @@ def loss_of(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_au
             act: str = "gelu") -> float:
     """L = sum(dout * out) + d_aux * aux + d_z * z of the oracle's forward pass."""
     f = forward(x, Wg, bg, W1, b1, W2, b2, k, cf, dtype, act=act)
+    return float(np.sum(np.asarray(dout, np.float64) * f.out)) + d_aux * f.aux + d_z * f.z
+
+
+def bwd_router_ec(x, Wg, bg, dw, d_aux: float, d_z: float, dtype: str):
+    """Expert-choice router backward: (dlogits[T,E], dWg[H,E], dbg[E], dx_router[T,H]) given dw[T,E]
+    (dout_t . y for the chosen pairs, 0 elsewhere)."""
+    x, Wg, bg, dw = _c(x), _c(Wg), _opt(bg), _c(dw, np.float64)
+    T, H = x.shape
+    E = Wg.shape[1]
+    dl = np.empty((T, E), np.float64)
+    dWg = np.empty((H, E), np.float64)
+    dbg = np.empty(E, np.float64)
+    dxr = np.empty((T, H), np.float64)
+    _load().oracle_bwd_router_ec(T, H, E, _DT[dtype], _p(x), _p(Wg), _p(bg), _p(dw), float(d_aux), float(d_z), _p(dl),
+                                 _p(dWg), _p(dbg), _p(dxr))
+    return dl, dWg, dbg, dxr
+
+
+def backward_ec(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_aux: float, d_z: float,
+                act: str = "gelu", chosen=None) -> Grads:
+    """All gradients of L = sum(dout*out) + d_aux*aux + d_z*z under expert choice (small problems).
+    The selection is the oracle's own unless chosen[E,C] is given.  Grads.dw is [T,E] here."""
+    T, H = x.shape
+    E, _, F = W1.shape
+    r = route(x, Wg, bg, 1, dtype)
+    if chosen is None:
+        chosen = expert_choice(r.logits, ec_capacity(cf, T, k, E)).chosen
+    chosen = np.asarray(chosen, np.int32)
+    dout = _c(dout, np.float64)
+    dx = np.zeros((T, H))
+    dw = np.zeros((T, E))
+    dW1 = np.zeros((E, H, F))
+    dW2 = np.zeros((E, F, H))
+    db1 = np.zeros((E, F))
+    db2 = np.zeros((E, H))
+    allf = np.arange(F, dtype=np.int32)
+    for e in range(E):
+        toks = chosen[e]
+        ws = r.p[toks, e]
+        for t, w in zip(toks, ws):
+            dxp, dws, _ = bwd_slot(x, W1, b1, W2, b2, int(t), e, dout[t], float(w), dtype, act)
+            dx[t] += dxp
+            dw[t, e] = dws
+        r2, c1, b1s, b2s = bwd_expert_weights(x, W1, b1, W2, e, toks, ws, dout, allf, dtype, act)
+        dW2[e] = r2
+        dW1[e] = c1.T
+        db1[e] = b1s
+        db2[e] = b2s
+    dl, dWg, dbg, dxr = bwd_router_ec(x, Wg, bg, dw, d_aux, d_z, dtype)
+    return Grads(dx + dxr, dWg, dbg, dW1, db1, dW2, db2, dw, dl)
+
+
+def loss_of_ec(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_aux: float, d_z: float,
+               act: str = "gelu") -> float:
+    """L = sum(dout * out) + d_aux * aux + d_z * z of the oracle's expert-choice forward pass."""
+    f = forward_ec(x, Wg, bg, W1, b1, W2, b2, k, cf, dtype, act=act)
     return float(np.sum(np.asarray(dout, np.float64) * f.out)) + d_aux * f.aux + d_z * f.z

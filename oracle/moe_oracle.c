@@ -560,6 +560,56 @@ void oracle_bwd_router(int64_t T, int64_t H, int64_t E, int64_t k, int dtype, co
   free(dp);
 }
 
+/*
+ * Router backward under expert choice (Core Concepts 2): the weight of a chosen pair (t, e) is the
+ * token's softmax probability itself, so dp[t,e] = dw[t,e] for chosen pairs (0 elsewhere), plus the
+ * aux-loss term d_aux / T (f_e = 1/E is fixed), which the softmax backward cancels because the
+ * probabilities of a token sum to 1:
+ *   dlogit[e] = p[e] (dp[e] - sum_e' p[e'] dp[e']) + d_z * 2 lse p[e] / T
+ * dw[T,E] holds dout_t . y for every chosen pair.  Outputs as for oracle_bwd_router.
+ */
+void oracle_bwd_router_ec(int64_t T, int64_t H, int64_t E, int dtype, const void* x, const void* Wg, const void* bg,
+                          const double* dw, double d_aux, double d_z, double* dlogits, double* dWg, double* dbg,
+                          double* dx_router) {
+  double* lg = (double*)malloc(sizeof(double) * (size_t)E);
+  double* p = (double*)malloc(sizeof(double) * (size_t)E);
+  double* dp = (double*)malloc(sizeof(double) * (size_t)E);
+  for (int64_t i = 0; i < H * E; ++i) dWg[i] = 0.0;
+  for (int64_t e = 0; e < E; ++e) dbg[e] = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    for (int64_t e = 0; e < E; ++e) {
+      double acc = load_bias(bg, dtype, (size_t)e);
+      for (int64_t h = 0; h < H; ++h) acc += load(x, dtype, (size_t)(t * H + h)) * load(Wg, dtype, (size_t)(h * E + e));
+      lg[e] = acc;
+    }
+    double m = lg[0];
+    for (int64_t e = 1; e < E; ++e)
+      if (lg[e] > m) m = lg[e];
+    double se = 0.0;
+    for (int64_t e = 0; e < E; ++e) se += exp(lg[e] - m);
+    const double lse = m + log(se);
+    for (int64_t e = 0; e < E; ++e) p[e] = exp(lg[e] - lse);
+    for (int64_t e = 0; e < E; ++e) dp[e] = dw[t * E + e] + d_aux / (double)T;
+    double pdp = 0.0;
+    for (int64_t e = 0; e < E; ++e) pdp += p[e] * dp[e];
+    double* dl = dlogits + t * E;
+    for (int64_t e = 0; e < E; ++e) dl[e] = p[e] * (dp[e] - pdp) + d_z * 2.0 * lse * p[e] / (double)T;
+    for (int64_t e = 0; e < E; ++e) dbg[e] += dl[e];
+    for (int64_t h = 0; h < H; ++h) {
+      const double xv = load(x, dtype, (size_t)(t * H + h));
+      double s = 0.0;
+      for (int64_t e = 0; e < E; ++e) {
+        dWg[h * E + e] += xv * dl[e];
+        s += load(Wg, dtype, (size_t)(h * E + e)) * dl[e];
+      }
+      dx_router[t * H + h] = s;
+    }
+  }
+  free(lg);
+  free(p);
+  free(dp);
+}
+
 /* threads the OpenMP runtime will use for a parallel region (for reporting) */
 int oracle_max_threads(void) {
 #ifdef _OPENMP

@@ -623,3 +623,41 @@ def test_backward_sampled_columns_match_full():
     np.testing.assert_allclose(c1, g.dW1[e][:, cols].T, rtol=1e-13, atol=1e-15)
     np.testing.assert_allclose(b1s, g.db1[e][cols], rtol=1e-13, atol=1e-15)
     np.testing.assert_allclose(b2s, g.db2[e], rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("case", [
+    dict(seed=81, cf=1.0),                          # C = T k / E: some tokens unchosen, some chosen twice
+    dict(seed=82, cf=math.inf, act="silu", bias=False),  # C = T: every expert sees every token
+], ids=["ec_partial", "ec_all_tokens"])
+def test_backward_expert_choice_matches_central_differences(case):
+    """Expert-choice gradients against central differences of the oracle's expert-choice forward pass; the
+    per-expert selection margins exceed the steps, so the choice cannot change."""
+    case = dict(case)
+    seed, cf = case.pop("seed"), case.pop("cf")
+    cfg, inp, dout = _fd_layer(seed, T=9, **case)
+    d_aux, d_z = 0.37, -0.21
+    r = oracle.route(inp.x, inp.Wg, inp.bg, 1, "f32")
+    C = oracle.ec_capacity(cf, cfg.T, cfg.k, cfg.E)
+    ec = oracle.expert_choice(r.logits, C)
+    assert ec.margin.min() > 2e-2
+    g = oracle.backward_ec(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cf, "f32", dout, d_aux, d_z,
+                           act=cfg.act)
+    names = ["x", "Wg", "W1", "W2"] + (["bg", "b1", "b2"] if cfg.bias else [])
+    grads = dict(x=g.dx, Wg=g.dWg, bg=g.dbg, W1=g.dW1, b1=g.db1, W2=g.dW2, b2=g.db2)
+    rng = np.random.default_rng(seed)
+    for name in names:
+        base = getattr(inp, name)
+        for flat in rng.choice(base.size, size=min(6, base.size), replace=False):
+            idx = np.unravel_index(flat, base.shape)
+            lo, hi = base.copy(), base.copy()
+            lo[idx] = np.float32(base[idx] - 1e-3)
+            hi[idx] = np.float32(base[idx] + 1e-3)
+            step = float(hi[idx]) - float(lo[idx])
+            args = {n: getattr(inp, n) for n in ("x", "Wg", "bg", "W1", "b1", "W2", "b2")}
+            args[name] = hi
+            Lp = oracle.loss_of_ec(args["x"], args["Wg"], args["bg"], args["W1"], args["b1"], args["W2"], args["b2"],
+                                   cfg.k, cf, "f32", dout, d_aux, d_z, act=cfg.act)
+            args[name] = lo
+            Lm = oracle.loss_of_ec(args["x"], args["Wg"], args["bg"], args["W1"], args["b1"], args["W2"], args["b2"],
+                                   cfg.k, cf, "f32", dout, d_aux, d_z, act=cfg.act)
+            assert grads[name][idx] == pytest.approx((Lp - Lm) / step, rel=1e-5, abs=1e-7), (name, idx)
