@@ -246,7 +246,9 @@ MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_io_t* 
  * gradients are the chain rule through the forward definition: for L with dL/dout = dout,
  * dL/daux = d_aux and dL/dz = d_z, every input x, Wg, bg, W1, b1, W2, b2 gets dL/d(input).  The
  * top-k choice and the capacity drops are piecewise constant and carry no gradient; a dropped
- * slot contributes nothing.  Token choice with bf16 storage only (else MOE_ERR_UNSUPPORTED).
+ * slot contributes nothing.  bf16 storage only (else MOE_ERR_UNSUPPORTED); both routing rules.  Under
+ * expert choice the weight of a chosen pair is the softmax probability itself, so the gate receives
+ * p (dw - sum p dw) with no renormalisation term, and the aux-loss term cancels (f_e = 1/E).
  * ------------------------------------------------------------------------------------------- */
 
 /* Caller-owned device buffers of the backward pass, fp32, row-major. */
@@ -261,7 +263,8 @@ typedef struct {
   float* db1;        /* [E,F]; NULL exactly when io->b1 is NULL */
   float* dW2;        /* [E,F,H] */
   float* db2;        /* [E,H]; NULL exactly when io->b2 is NULL */
-  float* dw;         /* [T,k] optional (may be NULL): dL/d topk_w per slot, 0 for dropped slots */
+  float* dw;         /* optional (may be NULL): dL/d topk_w -- [T,k] per slot, 0 for dropped slots;
+                        under expert choice [T,E], 0 for pairs not chosen */
 } moe_grad_t;
 
 /* Workspace bytes for moe_forward_train + moe_backward (the inference layout plus the saved router
@@ -278,7 +281,8 @@ MOE_API moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t*
  * W2, b2 (optional), topk_idx, topk_w, dropped from io and the saved state from ws; writes every
  * buffer of grad (dx, dWg, dbg are cleared first; no output is accumulated across calls).
  * Row order of the bf16 intermediates: the permuted (expert-major) rows of the forward pass.
- * Order of fp32 additions in dx, dWg and dbg is not fixed (atomics).  7 or 8 launches. */
+ * Order of fp32 additions in dx, dWg and dbg is not fixed (atomics).  7 or 8 launches (one more
+ * under expert choice). */
 MOE_API moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const moe_grad_t* grad, void* ws,
                           size_t ws_bytes, cudaStream_t stream);
 

@@ -299,7 +299,8 @@ class MoEBuffers:
         if self.inputs.get("b2") is not None:
             g["db2"] = torch.empty((E, H), dtype=torch.float32, device=dev)
         if with_dw:
-            g["dw"] = torch.empty((T, k), dtype=torch.float32, device=dev)
+            ec = s.routing == MOE_ROUTING_EXPERT_CHOICE
+            g["dw"] = torch.empty((T, E if ec else k), dtype=torch.float32, device=dev)
         return g
 
     def backward(self, dout, grads: dict, d_aux: float = 0.0, d_z: float = 0.0):

@@ -55,6 +55,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
   if (a.db2)
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (long long)a.E * a.H; i += stride)
       a.db2[i] = 0.f;
+  if (a.dwmat)
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (long long)a.T * a.E; i += stride)
+      a.dwmat[i] = 0.f;
 }
 
 // Bias gradients over 64-row chunks of the permuted rows (a chunk may span experts; rows are
@@ -127,6 +130,28 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(BiasGradArgs a) {
   }
 }
 
+// Expert choice: one warp per row r (token t, expert e): dwmat[t,e] = dwraw[r] + dout[t] . b2[e].
+__global__ void __launch_bounds__(256) ec_dw_scatter_kernel(EcDwArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  if (r >= a.rows) return;
+  const int t = a.row_token[r], e = a.row_slot[r];
+  float bdot = 0.f;
+  if (a.b2) {
+    const __nv_bfloat16* b2 = a.b2 + (size_t)e * a.H;
+    for (int h = 4 * lane; h < a.H; h += 128) {
+      const float4 d = *reinterpret_cast<const float4*>(a.dout + (size_t)t * a.H + h);
+      const uint2 bb = *reinterpret_cast<const uint2*>(b2 + h);
+      const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb.x));
+      const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb.y));
+      bdot = fmaf(d.x, b01.x, fmaf(d.y, b01.y, fmaf(d.z, b23.x, fmaf(d.w, b23.y, bdot))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) bdot += __shfl_xor_sync(0xffffffffu, bdot, o);
+  }
+  if (lane == 0) a.dwmat[(size_t)t * a.E + e] = a.dwraw[r] + bdot;
+}
+
 constexpr int kRbWarps = 8;  // tokens per block
 
 __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs a) {
@@ -156,6 +181,30 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
 #pragma unroll
   for (int j = 0; j < 8; ++j) p[j] = (j < NJ && lane + 32 * j < E) ? expf(lv[j] - m) * inv_s : 0.f;
 
+  if (a.dwmat != nullptr) {
+    // expert choice: the weight of a chosen pair is p itself, so dp = dw (0 for pairs not chosen);
+    // the aux term is the same for every expert of a token and cancels in the softmax backward
+    float pdp = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      dp[j] = (j < NJ && e < E) ? a.dwmat[(size_t)t * E + e] : 0.f;
+      if (a.dw_out && j < NJ && e < E) a.dw_out[(size_t)t * E + e] = dp[j];
+      pdp += p[j] * dp[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pdp += __shfl_xor_sync(0xffffffffu, pdp, o);
+    const float zc = a.d_z * 2.f * lse / (float)a.T;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (j < NJ && e < E) {
+        const float d = p[j] * (dp[j] - pdp) + zc * p[j];
+        a.dlogits[(size_t)t * E + e] = d;
+        dl_s[warp][e] = d;
+      }
+    }
+  } else {
   // dw per slot: the GEMM's sum_n G h (already in dwraw) plus dout . b2[e]; 0 when dropped
   float dws[8], ws[8];
   int es[8];
@@ -227,6 +276,7 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
       a.dlogits[(size_t)t * E + e] = d;
       dl_s[warp][e] = d;
     }
+  }
   }
   __syncwarp();
   // dx[t] += Wg dlogits[t]: four rows of Wg per lane per step
@@ -320,6 +370,12 @@ cudaError_t launch_bias_grad(const BiasGradArgs& a, cudaStream_t st) {
   const int cols = a.H > a.F ? a.H : a.F;
   dim3 grid((a.rows_cap + kBgRows - 1) / kBgRows, (cols + 511) / 512);
   bias_grad_kernel<<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ec_dw_scatter(const EcDwArgs& a, cudaStream_t st) {
+  if (a.rows <= 0) return cudaSuccess;
+  ec_dw_scatter_kernel<<<(a.rows + 7) / 8, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

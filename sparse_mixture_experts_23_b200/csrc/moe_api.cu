@@ -495,7 +495,7 @@ size_t moe_train_workspace_size(const moe_shape_t* shape) {
 static moe_status_t check_train(const moe_shape_t* shape, void* ws, size_t ws_bytes) {
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
-  if (shape->dtype != MOE_DTYPE_BF16 || shape->routing != MOE_ROUTING_TOKEN_CHOICE) return MOE_ERR_UNSUPPORTED;
+  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < ws_layout(*shape).train_total) return MOE_ERR_WORKSPACE;
   return MOE_OK;
@@ -518,6 +518,11 @@ moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, voi
       !aligned16(io->b1) || !aligned16(io->b2))
     return MOE_ERR_INVALID_ARG;
   if ((st = do_route(shape, io, ws, stream, true, true)) != MOE_OK) return st;
+  if (shape->routing == MOE_ROUTING_EXPERT_CHOICE) {
+    if ((st = do_ec_select_and_losses(shape, io, ws, stream)) != MOE_OK) return st;
+    if ((st = do_ec_gather(shape, io, ws, stream)) != MOE_OK) return st;
+    return do_ffn(shape, io, ws, 1, stream, true);
+  }
   ++g_launches;
   if ((st = cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 1), stream))) != MOE_OK) return st;
   if ((st = do_scatter(shape, io, ws, stream)) != MOE_OK) return st;
@@ -540,15 +545,18 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   if (!aligned16(grad->dout) || !aligned16(grad->dx) || !aligned16(io->W1) || !aligned16(io->W2))
     return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*shape);
+  const bool ec = shape->routing == MOE_ROUTING_EXPERT_CHOICE;
+  const int kw = ec ? shape->E : shape->k;  // stride of the combine weights in topk_w
   const int32_t* offsets = at<int32_t>(ws, L.offsets);
   const int32_t* row_token = at<int32_t>(ws, L.row_token);
   const int32_t* row_slot = at<int32_t>(ws, L.row_slot);
+  float* dlogits = at<float>(ws, L.dlogits);  // under expert choice it first holds dL/dp of the chosen pairs
 
   BwdPrepArgs pa{};
   pa.T = shape->T;
   pa.H = shape->H;
   pa.E = shape->E;
-  pa.k = shape->k;
+  pa.k = kw;
   pa.offsets = offsets;
   pa.row_token = row_token;
   pa.row_slot = row_slot;
@@ -563,6 +571,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   pa.F = shape->F;
   pa.db1 = grad->db1;
   pa.db2 = grad->db2;
+  pa.dwmat = ec ? dlogits : nullptr;
   ++g_launches;
   if ((st = cuda_status(launch_bwd_prep(pa, stream))) != MOE_OK) return st;
 
@@ -571,10 +580,10 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   ga.H = shape->H;
   ga.E = shape->E;
   ga.F = shape->F;
-  ga.k = shape->k;
+  ga.k = kw;
   ga.rows_cap = (int)L.rows;
   ga.act = shape->activation;
-  ga.avg_rows = (long long)shape->T * shape->k / shape->E;
+  ga.avg_rows = ec ? L.ec_cap : (long long)shape->T * shape->k / shape->E;
   ga.offsets = offsets;
   ga.row_token = row_token;
   ga.row_slot = row_slot;
@@ -601,7 +610,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
     ba.H = shape->H;
     ba.F = shape->F;
     ba.E = shape->E;
-    ba.k = shape->k;
+    ba.k = kw;
     ba.rows_cap = (int)L.rows;
     ba.offsets = offsets;
     ba.row_token = row_token;
@@ -613,6 +622,21 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
     ba.db2 = grad->db2;
     ++g_launches;
     if ((st = cuda_status(launch_bias_grad(ba, stream))) != MOE_OK) return st;
+  }
+
+  if (ec) {
+    EcDwArgs da{};
+    da.rows = (int)L.rows;
+    da.H = shape->H;
+    da.E = shape->E;
+    da.row_token = row_token;
+    da.row_slot = row_slot;
+    da.dwraw = pa.dwraw;
+    da.dout = grad->dout;
+    da.b2 = reinterpret_cast<const __nv_bfloat16*>(io->b2);
+    da.dwmat = dlogits;
+    ++g_launches;
+    if ((st = cuda_status(launch_ec_dw_scatter(da, stream))) != MOE_OK) return st;
   }
 
   RouterBwdArgs ra{};
@@ -632,7 +656,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   ra.Wg = reinterpret_cast<const __nv_bfloat16*>(io->Wg);
   ra.d_aux = grad->d_aux;
   ra.d_z = grad->d_z;
-  ra.dlogits = at<float>(ws, L.dlogits);
+  ra.dlogits = dlogits;
+  ra.dwmat = ec ? dlogits : nullptr;
   ra.dw_out = grad->dw;
   ra.dx = grad->dx;
   ++g_launches;

@@ -169,6 +169,7 @@ struct BwdPrepArgs {
   float* dbg;         // [E] cleared, or null
   float* db1;         // [E,F] cleared, or null
   float* db2;         // [E,H] cleared, or null
+  float* dwmat;       // expert choice: [T,E] cleared, or null
 };
 
 struct BiasGradArgs {
@@ -197,7 +198,8 @@ struct RouterBwdArgs {
   const __nv_bfloat16* Wg;  // [H,E]
   float d_aux, d_z;
   float* dlogits;  // [T,E] out
-  float* dw_out;   // [T,k] out, or null
+  float* dw_out;   // [T,k] out (token choice) or [T,E] (expert choice), or null
+  const float* dwmat;  // expert choice: [T,E] dL/dp of the chosen pairs (may alias dlogits), else null
   float* dx;       // [T,H] += Wg dlogits
 };
 
@@ -233,7 +235,18 @@ struct BwdGemmArgs {
   int num_sms;
 };
 
+struct EcDwArgs {
+  int rows, H, E;
+  const int32_t* row_token;
+  const int32_t* row_slot;
+  const float* dwraw;
+  const float* dout;
+  const __nv_bfloat16* b2;  // or null
+  float* dwmat;             // [T,E]
+};
+
 cudaError_t launch_bwd_prep(const BwdPrepArgs& a, cudaStream_t st);
+cudaError_t launch_ec_dw_scatter(const EcDwArgs& a, cudaStream_t st);
 cudaError_t launch_bias_grad(const BiasGradArgs& a, cudaStream_t st);
 cudaError_t launch_router_bwd(const RouterBwdArgs& a, cudaStream_t st);
 cudaError_t launch_gate_wgrad(GateWgradArgs a, cudaStream_t st);

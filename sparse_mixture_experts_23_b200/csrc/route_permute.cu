@@ -113,6 +113,7 @@ __device__ void router_finish(const RouterArgs& a, const float* logits, int epad
         if (j < NJ && e < E) {
           a.topk_w[(size_t)t * E + e] = expf(lv[j] - m) * inv_s;
           a.scores[(size_t)e * T + t] = lv[j];
+          if (a.logits_out != nullptr) a.logits_out[(size_t)t * E + e] = lv[j];
         }
       }
       if (lane == 0) a.tok_count[t] = 0;

@@ -13,7 +13,8 @@ Tolerances (written here once, used by every parity test):
     weighted dout rows, or x and du), where the forward GEMMs round one (h); a rounding of 2^-9
     relative on each operand gives a bulk (Frobenius) error of a few 1e-3, and the largest of ~1e5
     elements reaches 4-5 standard deviations of it.  A wrong or missing term moves the Frobenius
-    error to O(1).
+    error to O(1).  The per-expert weight and bias gradients are checked per expert (each is its
+    own GEMM over its own rows, and the experts' scales differ): max|d_e| <= 4e-2 * RMS(ref_e).
 """
 from __future__ import annotations
 
