@@ -60,7 +60,7 @@ def _load():
     lib.oracle_gelu.restype = dbl
     lib.oracle_silu.argtypes = [dbl]
     lib.oracle_silu.restype = dbl
-    lib.oracle_capacity.argtypes = [dbl, i64, i64, i64]
+    lib.oracle_capacity.argtypes = [dbl, i64, i64, i64, i64]
     lib.oracle_capacity.restype = i64
     lib.oracle_route.argtypes = [i64, i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.oracle_route.restype = None
@@ -73,7 +73,7 @@ def _load():
     lib.oracle_forward_tokens.argtypes = [i64, i64, i64, c_int, c_int, vp, vp, vp, vp, vp, vp, vp, vp, i64, vp,
                                           vp, c_int]
     lib.oracle_forward_tokens.restype = None
-    lib.oracle_ec_capacity.argtypes = [dbl, i64, i64, i64]
+    lib.oracle_ec_capacity.argtypes = [dbl, i64, i64, i64, i64]
     lib.oracle_ec_capacity.restype = i64
     lib.oracle_expert_choice.argtypes = [i64, i64, i64, vp, vp, vp]
     lib.oracle_expert_choice.restype = None
@@ -129,9 +129,9 @@ def _opt(a):
     return None if a is None else _c(a)
 
 
-def capacity(cf: float, T: int, k: int, E: int):
-    """Per-expert capacity, or None when unlimited (CF = +inf)."""
-    c = _load().oracle_capacity(float(cf), T, k, E)
+def capacity(cf: float, T: int, k: int, E: int, min_capacity: int = 0):
+    """Per-expert capacity max(ceil(CF*T*k/E), min_capacity), or None when unlimited (CF = +inf)."""
+    c = _load().oracle_capacity(float(cf), T, k, E, int(min_capacity))
     return None if c < 0 else int(c)
 
 
@@ -186,10 +186,10 @@ class Dispatch:
         return int(self.offsets[-1])
 
 
-def dispatch(topk_idx, E: int, cf: float) -> Dispatch:
+def dispatch(topk_idx, E: int, cf: float, min_capacity: int = 0) -> Dispatch:
     idx = _c(topk_idx, np.int32)
     T, k = idx.shape
-    cap = capacity(cf, T, k, E)
+    cap = capacity(cf, T, k, E, min_capacity)
     cnt_pre = np.empty(E, np.int32)
     counts = np.empty(E, np.int32)
     offsets = np.empty(E + 1, np.int32)
@@ -242,11 +242,11 @@ class Forward:
 
 
 def forward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=None, nthreads: int = 0,
-            act: str = "gelu") -> Forward:
+            act: str = "gelu", min_capacity: int = 0) -> Forward:
     """Whole layer: routing and dispatch over all tokens, FFN + combine for ``tokens`` (default: all)."""
     r = route(x, Wg, bg, k, dtype)
     aux, z = losses(r.p, r.lse, r.topk_idx)
-    d = dispatch(r.topk_idx, Wg.shape[1], cf)
+    d = dispatch(r.topk_idx, Wg.shape[1], cf, min_capacity)
     T = x.shape[0]
     tokens = np.arange(T, dtype=np.int32) if tokens is None else np.asarray(tokens, np.int32)
     out = forward_tokens(x, W1, b1, W2, b2, r.topk_idx, r.topk_w, d.dropped, tokens, dtype, nthreads, act)
@@ -255,9 +255,9 @@ def forward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, tokens=Non
 
 # ------------------------------------------------------------------ expert-choice routing -------
 
-def ec_capacity(cf: float, T: int, k: int, E: int) -> int:
-    """Tokens per expert under expert choice: min(T, ceil(CF*T*k/E)); T when CF = +inf."""
-    return int(_load().oracle_ec_capacity(float(cf), T, k, E))
+def ec_capacity(cf: float, T: int, k: int, E: int, min_capacity: int = 0) -> int:
+    """Tokens per expert under expert choice: min(T, max(ceil(CF*T*k/E), min_capacity)); T when CF = +inf."""
+    return int(_load().oracle_ec_capacity(float(cf), T, k, E, int(min_capacity)))
 
 
 @dataclass

@@ -73,12 +73,14 @@ static double activation(int act, double u) { return act == ORACLE_ACT_SILU ? or
 /* a bias pointer may be NULL: the Mixtral block's Linear layers have bias=False */
 static double load_bias(const void* base, int dtype, size_t i) { return base ? load(base, dtype, i) : 0.0; }
 
-/* capacity of one expert: ceil(CF * T * k / E), or -1 for "unlimited" (CF = +inf).
+/* capacity of one expert: max(ceil(CF * T * k / E), min_capacity), or -1 for "unlimited" (CF = +inf).
  * [SKILL] Core Concepts 4 / Best Practices 2; the k factor and the ceiling follow the workload
- * statement (the pages' formulas differ only in rounding and in whether k appears). */
-int64_t oracle_capacity(double cf, int64_t T, int64_t k, int64_t E) {
+ * statement (the pages' formulas differ only in rounding and in whether k appears); the lower
+ * bound is the "min_capacity" of the Core Concepts 4 configuration (0 = none). */
+int64_t oracle_capacity(double cf, int64_t T, int64_t k, int64_t E, int64_t min_capacity) {
   if (isinf(cf) && cf > 0) return -1;
-  return (int64_t)ceil(cf * (double)T * (double)k / (double)E);
+  const int64_t c = (int64_t)ceil(cf * (double)T * (double)k / (double)E);
+  return c > min_capacity ? c : min_capacity;
 }
 
 /*
@@ -322,16 +324,17 @@ void oracle_forward_tokens(int64_t H, int64_t F, int64_t k, int dtype, int act, 
  * are transposed to (experts, tokens) and every expert takes the top capacity_per_expert tokens
  * of its row ("guarantees perfect load balancing").  Readings (listed in the design notes):
  *  - the scores are the router's logits, as printed (no softmax before the per-expert top-k);
- *  - capacity_per_expert C = min(T, ceil(CF * T * k / E)), k being the average number of experts
+ *  - capacity_per_expert C = min(T, max(ceil(CF * T * k / E), min_capacity)), k being the average number of experts
  *    per token; CF = +inf gives C = T (every expert sees every token);
  *  - ties go to the lower token index; an expert's chosen tokens are listed in ascending token
  *    order, which is also their row order inside the expert's segment;
  *  - a chosen (token, expert) pair is weighted by the token's softmax probability p[t,e] over the
  *    experts, without renormalisation; a token chosen by no expert gets out = 0.
  * ---------------------------------------------------------------------------------------------- */
-int64_t oracle_ec_capacity(double cf, int64_t T, int64_t k, int64_t E) {
+int64_t oracle_ec_capacity(double cf, int64_t T, int64_t k, int64_t E, int64_t min_capacity) {
   if (isinf(cf) && cf > 0) return T;
   int64_t c = (int64_t)ceil(cf * (double)T * (double)k / (double)E);
+  if (c < min_capacity) c = min_capacity;
   return c < T ? c : T;
 }
 

@@ -661,3 +661,17 @@ def test_backward_expert_choice_matches_central_differences(case):
             Lm = oracle.loss_of_ec(args["x"], args["Wg"], args["bg"], args["W1"], args["b1"], args["W2"], args["b2"],
                                    cfg.k, cf, "f32", dout, d_aux, d_z, act=cfg.act)
             assert grads[name][idx] == pytest.approx((Lp - Lm) / step, rel=1e-5, abs=1e-7), (name, idx)
+
+
+def test_min_capacity_lower_bound():
+    """Core Concepts 4's "min_capacity": the capacity never falls below it (0 = no bound); dispatch keeps
+    exactly min(count, max(ceil(CF*T*k/E), min_capacity)) per expert, first in slot-major order."""
+    assert oracle.capacity(0.25, 40, 1, 4) == 3 and oracle.capacity(0.25, 40, 1, 4, min_capacity=4) == 4
+    assert oracle.capacity(2.0, 40, 1, 4, min_capacity=4) == 20  # the bound does not bind
+    assert oracle.capacity(math.inf, 40, 1, 4, min_capacity=4) is None
+    assert oracle.ec_capacity(0.02, 100, 1, 4, min_capacity=6) == 6
+    assert oracle.ec_capacity(0.5, 10, 1, 1, min_capacity=50) == 10  # never more than T
+    idx = np.zeros((40, 1), np.int32)  # every token picks expert 0
+    d = oracle.dispatch(idx, 4, 0.25, min_capacity=4)
+    assert d.cap == 4 and d.expert_counts.tolist() == [4, 0, 0, 0]
+    assert d.dropped[:4].sum() == 0 and d.dropped[4:].all()
