@@ -36,7 +36,7 @@
  *      MOE_ERR_INVALID_ARG  null shape/io/workspace pointer, a needed io pointer that is null, a
  *                           device pointer of x/Wg/W1/W2/out/workspace not 16-byte aligned,
  *                           T < 0, H/E/F/k <= 0, k > E, k > 8, E > 256, capacity_factor <= 0 or
- *                           NaN, unknown dtype, activation or routing, a non-null b1/b2 not 16-byte
+ *                           NaN, min_capacity < 0, unknown dtype, activation or routing, a non-null b1/b2 not 16-byte
  *                           aligned
  *      MOE_ERR_UNSUPPORTED  bf16 with H or F not a multiple of 64; f32 with H or F not a multiple
  *                           of 4; rows*max(H,F) beyond 2^31 elements (rows = T*k, or E*C under
@@ -86,7 +86,7 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 
 /* Routing rule.  Expert choice: the router's logits are read per expert (the page transposes
  * them to (experts, tokens)) and every expert takes the C tokens with the largest logits, ties to
- * the lower token index, C = min(T, ceil(capacity_factor * T * k / E)) -- k is then the average
+ * the lower token index, C = min(T, max(ceil(capacity_factor * T * k / E), min_capacity)) -- k is then the average
  * number of experts per token, and capacity_factor = +INFINITY gives C = T.  Each chosen
  * (token, expert) pair is weighted by the token's softmax probability over the experts, not
  * renormalised; a token chosen by no expert gets out = 0.  Every expert holds exactly C rows. */
@@ -97,8 +97,9 @@ typedef enum { MOE_ROUTING_TOKEN_CHOICE = 0, MOE_ROUTING_EXPERT_CHOICE = 1 } moe
 typedef enum { MOE_ACT_GELU = 0, MOE_ACT_SILU = 1 } moe_activation_t;
 
 /* Problem statement.  capacity_factor = +INFINITY means dropless.  Per-expert capacity is
- * ceil(capacity_factor * T * k / E) evaluated in double ("MoE Training" page, Core Concepts 4 and
- * Best Practices 2 give capacity = tokens * CF / E; k counts the assignments of top-k routing). */
+ * max(ceil(capacity_factor * T * k / E), min_capacity) evaluated in double ("MoE Training" page,
+ * Core Concepts 4 and Best Practices 2 give capacity = tokens * CF / E; k counts the assignments of
+ * top-k routing). */
 typedef struct {
   int32_t T;              /* tokens (batch * sequence), >= 0 */
   int32_t H;              /* hidden size */
@@ -109,6 +110,8 @@ typedef struct {
   moe_dtype_t dtype;      /* storage type of x and all weights */
   moe_activation_t activation; /* expert activation; a zero-initialised shape gets GELU */
   moe_routing_t routing;       /* a zero-initialised shape gets token choice */
+  int32_t min_capacity;        /* lower bound on the per-expert capacity ("min_capacity" of the page's
+                                  Core Concepts 4 configuration); 0 = none, < 0 invalid */
 } moe_shape_t;
 
 /* Caller-owned device buffers.  Layouts (row-major):
@@ -165,9 +168,10 @@ typedef struct {
 /* Workspace bytes for a shape; 0 if the shape is invalid.  Host only, pure. */
 MOE_API size_t moe_workspace_size(const moe_shape_t* shape);
 
-/* Per-expert capacity the shape implies.  Token choice: ceil(capacity_factor * T * k / E), or -1
- * when capacity_factor = +INFINITY (no limit).  Expert choice: C = min(T, ceil(capacity_factor *
- * T * k / E)), the number of tokens every expert takes (the leading size of topk_idx[E,C]).
+/* Per-expert capacity the shape implies.  Token choice: max(ceil(capacity_factor * T * k / E),
+ * min_capacity), or -1 when capacity_factor = +INFINITY (no limit).  Expert choice: C = min(T,
+ * max(ceil(capacity_factor * T * k / E), min_capacity)), the number of tokens every expert takes
+ * (the leading size of topk_idx[E,C]).
  * -2 if the shape is invalid.  Host only, pure. */
 MOE_API int64_t moe_capacity(const moe_shape_t* shape);
 

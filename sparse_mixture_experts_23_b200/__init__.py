@@ -39,7 +39,7 @@ class MoEError(RuntimeError):
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("E", ctypes.c_int32), ("F", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("capacity_factor", ctypes.c_double), ("dtype", ctypes.c_int),
-                ("activation", ctypes.c_int), ("routing", ctypes.c_int)]
+                ("activation", ctypes.c_int), ("routing", ctypes.c_int), ("min_capacity", ctypes.c_int32)]
 
 
 class IO(ctypes.Structure):
@@ -111,8 +111,9 @@ def status_string(status: int) -> str:
 
 
 def make_shape(T: int, H: int, E: int, k: int, F: int, capacity_factor: float = math.inf, dtype: str = "bf16",
-               activation: str = "gelu", routing: str = "token_choice") -> Shape:
-    return Shape(T, H, E, F, k, float(capacity_factor), DTYPES[dtype], ACTIVATIONS[activation], ROUTINGS[routing])
+               activation: str = "gelu", routing: str = "token_choice", min_capacity: int = 0) -> Shape:
+    return Shape(T, H, E, F, k, float(capacity_factor), DTYPES[dtype], ACTIVATIONS[activation], ROUTINGS[routing],
+                 int(min_capacity))
 
 
 def moe_capacity(shape: Shape) -> int:

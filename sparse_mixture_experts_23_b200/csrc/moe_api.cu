@@ -41,7 +41,8 @@ cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
 // Tokens per expert under expert choice: min(T, ceil(CF*T*k/E)), T when CF = +inf.
 long long ec_capacity(const moe_shape_t& s) {
   if (isinf(s.capacity_factor)) return s.T;
-  const double c = ceil(s.capacity_factor * (double)s.T * (double)s.k / (double)s.E);
+  double c = ceil(s.capacity_factor * (double)s.T * (double)s.k / (double)s.E);
+  if (c < (double)s.min_capacity) c = (double)s.min_capacity;
   return c < (double)s.T ? (long long)c : (long long)s.T;
 }
 
@@ -123,6 +124,7 @@ moe_status_t check_shape(const moe_shape_t* s) {
   if (s->dtype != MOE_DTYPE_F32 && s->dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
   if (s->activation != MOE_ACT_GELU && s->activation != MOE_ACT_SILU) return MOE_ERR_INVALID_ARG;
   if (s->routing != MOE_ROUTING_TOKEN_CHOICE && s->routing != MOE_ROUTING_EXPERT_CHOICE) return MOE_ERR_INVALID_ARG;
+  if (s->min_capacity < 0) return MOE_ERR_INVALID_ARG;
   if (s->dtype == MOE_DTYPE_BF16 && (s->H % 64 != 0 || s->F % 64 != 0)) return MOE_ERR_UNSUPPORTED;
   if (s->dtype == MOE_DTYPE_F32 && (s->H % 4 != 0 || s->F % 4 != 0)) return MOE_ERR_UNSUPPORTED;
   const long long rows =
@@ -135,6 +137,7 @@ moe_status_t check_shape(const moe_shape_t* s) {
 long long capacity_of(const moe_shape_t* s) {
   if (isinf(s->capacity_factor)) return -1;
   double c = ceil(s->capacity_factor * (double)s->T * (double)s->k / (double)s->E);
+  if (c < (double)s->min_capacity) c = (double)s->min_capacity;
   if (c >= (double)((long long)s->T * s->k)) return -1;  // never binding
   return (long long)c;
 }
@@ -341,7 +344,8 @@ int64_t moe_capacity(const moe_shape_t* shape) {
   if (check_shape(shape) != MOE_OK) return -2;
   if (shape->routing == MOE_ROUTING_EXPERT_CHOICE) return ec_capacity(*shape);
   if (isinf(shape->capacity_factor)) return -1;
-  return (int64_t)ceil(shape->capacity_factor * (double)shape->T * (double)shape->k / (double)shape->E);
+  const int64_t c = (int64_t)ceil(shape->capacity_factor * (double)shape->T * (double)shape->k / (double)shape->E);
+  return c > shape->min_capacity ? c : (int64_t)shape->min_capacity;
 }
 
 moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, moe_ws_view_t* view) {

@@ -123,6 +123,7 @@ class LayerConfig:
     act: str = "gelu"  # expert activation: "gelu" (Quick Start expert) or "silu" (Mixtral block)
     bias: bool = True  # False: gate and experts have no bias at all (bg = b1 = b2 = None)
     routing: str = "token_choice"  # or "expert_choice" (every expert takes its top-C tokens)
+    min_capacity: int = 0  # lower bound on the per-expert capacity (0 = none)
 
     @property
     def x_std(self) -> float:

@@ -56,7 +56,7 @@ def upload(inp: synth.LayerInputs, device="cuda") -> dict:
 def shape_of(cfg: synth.LayerConfig):
     import sparse_mixture_experts_23_b200 as moe
 
-    return moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype, cfg.act, cfg.routing)
+    return moe.make_shape(cfg.T, cfg.H, cfg.E, cfg.k, cfg.F, cfg.CF, cfg.dtype, cfg.act, cfg.routing, cfg.min_capacity)
 
 
 def from_device_bits(t, dtype: str) -> np.ndarray:

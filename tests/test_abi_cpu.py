@@ -90,7 +90,7 @@ def test_bad_dtype_enum(lib):
 def test_activation_field(lib):
     """The activation sits right after dtype, and a zero-initialised shape means GELU; unknown
     activations are rejected before any launch."""
-    assert ctypes.sizeof(moe.Shape) == 48 and moe.Shape.activation.offset == 36
+    assert ctypes.sizeof(moe.Shape) == 48 and moe.Shape.activation.offset == 36 and moe.Shape.min_capacity.offset == 44
     assert moe.Shape().activation == moe.MOE_ACT_GELU
     s = _shape()
     assert moe.moe_workspace_size(s) > 0
@@ -235,3 +235,17 @@ def test_training_entry_points_validate_before_launch(lib):
         assert moe.moe_backward(s, _io(), _grad(**{f: None}), FAKE, n_train) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_backward(ctypes.byref(s), ctypes.byref(_io()), None, FAKE, n_train, None) == moe.MOE_ERR_INVALID_ARG
     assert moe.moe_train_workspace_size(_shape(T=-1)) == 0
+
+
+def test_min_capacity_field(lib):
+    s = _shape(T=40, H=64, E=4, k=1, F=64, capacity_factor=0.25)
+    assert moe.moe_capacity(s) == 3
+    s.min_capacity = 4
+    assert moe.moe_capacity(s) == 4
+    s.routing = moe.MOE_ROUTING_EXPERT_CHOICE
+    assert moe.moe_capacity(s) == 4
+    s.min_capacity = 100
+    assert moe.moe_capacity(s) == 40  # expert choice never takes more than T
+    s.min_capacity = -1
+    assert moe.moe_capacity(s) == -2 and moe.moe_workspace_size(s) == 0
+    assert moe.moe_forward(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG

@@ -48,7 +48,7 @@ def _check_against_oracle(cfg, r):
     ref = oracle.route(inp.x, inp.Wg, inp.bg, cfg.k, cfg.dtype)
     ok = ref.margin >= NEAR_TIE
     assert (r["topk_idx"][ok] == ref.topk_idx[ok]).all()
-    d = oracle.dispatch(r["topk_idx"], cfg.E, cfg.CF)
+    d = oracle.dispatch(r["topk_idx"], cfg.E, cfg.CF, cfg.min_capacity)
     assert (r["dropped"] == d.dropped).all()
     assert (r["counts"] == d.expert_counts).all()
     aux, z = oracle.losses(ref.p, ref.lse, r["topk_idx"])
@@ -86,6 +86,8 @@ def _check_against_oracle(cfg, r):
     _cfg("silu_nobias_pair", 1500, 256, 4, 2, 512, 1.1, "bf16", 30, act="silu", bias=False),
     # SiLU with biases present, k = 1 with drops
     _cfg("silu_bias", 300, 256, 16, 1, 512, 1.25, "bf16", 33, act="silu"),
+    # min_capacity binding: ceil(0.02 * 256 * 2 / 8) = 2 < 6
+    _cfg("min_capacity", 256, 128, 8, 2, 128, 0.02, "bf16", 36, min_capacity=6),
 ], ids=lambda c: c.name)
 def test_small_shapes_end_to_end(cfg):
     r = _run_forward(cfg)
