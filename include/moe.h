@@ -182,7 +182,9 @@ MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, mo
  * Core Concepts 3: load_balancing_loss, router_z_loss).
  * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws).
  * Expert choice: also the per-expert selection (Core Concepts 2), so it writes the chosen tokens
- * to topk_idx[E,C], expert_counts and dropped[T] as well; 3 launches. */
+ * to topk_idx[E,C], expert_counts and dropped[T] as well; 3 launches.
+ * bf16 layers whose expert count is a multiple of 64 compute the gate as one tensor-core GEMM into
+ * the workspace, then the per-chunk softmax/top-k, which adds one launch. */
 MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
@@ -232,8 +234,9 @@ MOE_API moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io
 MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
-/* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream (5 launches; 6
- * under expert choice). */
+/* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream (5 launches; one
+ * more under expert choice, and one more for the tensor-core gate of bf16 layers with a multiple of
+ * 64 experts). */
 MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
@@ -277,7 +280,7 @@ typedef struct {
 MOE_API size_t moe_train_workspace_size(const moe_shape_t* shape);
 
 /* moe_forward (same outputs), also keeping the router logits and the pre-activation u in ws for
- * moe_backward.  ws_bytes >= moe_train_workspace_size(shape).  5 launches. */
+ * moe_backward.  ws_bytes >= moe_train_workspace_size(shape).  Launches as moe_forward. */
 MOE_API moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                                cudaStream_t stream);
 
