@@ -980,40 +980,49 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
   const int nvec = a.H * a.esize / 16;  // 16-byte vectors per row
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* pv = reinterpret_cast<uint4*>(a.x_perm);
-  const int total = kChunk * nvec;
+  // this thread's (row, vector) walk over the chunk's 32 rows in steps of 256 vectors, with the
+  // row / column split kept incrementally (no division per element)
+  const int step_r = 256 / nvec, step_c = 256 % nvec;
   constexpr int U = 8;  // 16-byte loads in flight per thread
-  for (int i = tid; i < total; i += 256 * U) {
+  int r = tid / nvec, c = tid % nvec;
+  while (r < kChunk) {
     uint4 v[U];
-    int rr[U];
+    int dst[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      int idx = i + u * 256;
-      rr[u] = -1;
-      if (idx < total) {
-        int r = idx / nvec, c = idx % nvec;
-        int row = rows_s[r];
+      dst[u] = -1;
+      if (r < kChunk) {
+        const int row = rows_s[r];
         if (row >= 0) {
           v[u] = xv[(size_t)tok_s[r] * nvec + c];
-          rr[u] = idx;
+          dst[u] = row * nvec + c;  // < T*k*nvec < 2^31 (checked on the host)
         }
+      }
+      r += step_r;
+      c += step_c;
+      if (c >= nvec) {
+        c -= nvec;
+        ++r;
       }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      if (rr[u] >= 0) {
-        int idx = rr[u];
-        int r = idx / nvec, c = idx % nvec;
-        pv[(size_t)rows_s[r] * nvec + c] = v[u];
-      }
-    }
+    for (int u = 0; u < U; ++u)
+      if (dst[u] >= 0) pv[dst[u]] = v[u];
   }
   if (s == 0 && a.out != nullptr) {
     const int ovec = a.H / 4;
     float4* o = reinterpret_cast<float4*>(a.out);
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = tid; i < kChunk * ovec; i += 256) {
-      int r = i / ovec, c = i % ovec;
-      if (tok_s[r] >= 0) o[(size_t)tok_s[r] * ovec + c] = z;
+    const int sr = 256 / ovec, sc = 256 % ovec;
+    int orow = tid / ovec, oc = tid % ovec;
+    while (orow < kChunk) {
+      if (tok_s[orow] >= 0) o[(size_t)tok_s[orow] * ovec + oc] = z;
+      orow += sr;
+      oc += sc;
+      if (oc >= ovec) {
+        oc -= ovec;
+        ++orow;
+      }
     }
   }
 }
