@@ -193,3 +193,104 @@ def test_backward_expert_choice_all_gradients(cfg):
         _check("db2", r["db2"], ref.db2, per_expert=True)
         _check("dbg", r["dbg"], ref.dbg)
     assert r["launches"] == (9 if cfg.bias else 8)
+
+
+def _run_bg(cfg, dout, bg_override=None):
+    """_run with an optional gate-bias override (to force empty experts or drops)."""
+    import torch
+
+    moe = _lib()
+    inp = synth.make_inputs(cfg)
+    if bg_override is not None:
+        inp.bg = synth.to_storage(bg_override, cfg.dtype)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp), train=True)
+    buf.forward_train()
+    grads = buf.make_grads()
+    buf.backward(torch.from_numpy(dout.astype(np.float32)).cuda(), grads, D_AUX, D_Z)
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+    res = {n: t.cpu().numpy().astype(np.float64) for n, t in grads.items()}
+    res.update(inp=inp, topk_idx=buf.topk_idx.cpu().numpy(), dropped=buf.dropped.cpu().numpy(),
+               counts=buf.expert_counts.cpu().numpy())
+    return res
+
+
+def _ref_tc(cfg, r, dout):
+    inp = r["inp"]
+    return oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, dout,
+                           D_AUX, D_Z, act=cfg.act, topk_idx=r["topk_idx"], dropped=r["dropped"])
+
+
+def test_backward_empty_experts_get_zero_weight_gradients():
+    """Experts 4..7 are never chosen: their dW1, dW2, db1, db2 are exactly zero (the weight-gradient
+    kernel's empty-segment path), the others match the oracle."""
+    cfg = _cfg("bwd_empty", 200, 128, 8, 2, 256, math.inf, 71)
+    bg = np.zeros(8)
+    bg[4:] = -30.0
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    r = _run_bg(cfg, dout, bg)
+    assert (r["counts"][4:] == 0).all()
+    for n in ("dW1", "dW2", "db1", "db2"):
+        assert (r[n][4:] == 0).all(), n
+    ref = _ref_tc(cfg, r, dout)
+    for n in ("dx", "dWg", "dbg"):
+        _check(n, r[n], getattr(ref, n))
+    for n in ("dW1", "dW2", "db1", "db2"):
+        _check(n, r[n][:4], getattr(ref, n)[:4], per_expert=True)
+
+
+def test_backward_heavy_drops():
+    """cap = 16 with everyone wanting experts 0 and 1: most slots are dropped (dw = 0 there) and tokens with
+    every slot dropped get only the router's part of dx."""
+    cfg = _cfg("bwd_drops", 256, 64, 4, 2, 128, 0.125, 72)
+    bg = np.array([3.0, 2.5, -5.0, -5.0])
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    r = _run_bg(cfg, dout, bg)
+    assert r["dropped"].sum() > cfg.T
+    assert (r["dw"][r["dropped"].astype(bool)] == 0).all()
+    ref = _ref_tc(cfg, r, dout)
+    live = ~r["dropped"].astype(bool)
+    _check("dw (kept slots)", r["dw"][live], ref.dw[live])
+    for n in ("dx", "dWg", "dbg"):
+        _check(n, r[n], getattr(ref, n))
+    for n in ("dW1", "dW2", "db1", "db2"):
+        _check(n, r[n], getattr(ref, n), per_expert=True)
+
+
+def test_backward_one_token():
+    cfg = _cfg("bwd_one_token", 1, 64, 4, 2, 64, math.inf, 73)
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    r = _run_bg(cfg, dout)
+    ref = _ref_tc(cfg, r, dout)
+    for n in ("dx", "dWg", "dw"):
+        _check(n, r[n], getattr(ref, n))
+    used = sorted(set(r["topk_idx"][0].tolist()))
+    for n in ("dW1", "dW2"):
+        _check(n, r[n][used], getattr(ref, n)[used], per_expert=True)
+        unused = [e for e in range(cfg.E) if e not in used]
+        assert (r[n][unused] == 0).all()
+
+
+def test_backward_deterministic_parts_repeat_bitwise():
+    """dW1, dW2 (tensor-core accumulation in a fixed order), db1/db2 over one expert-major chunk order and
+    the per-slot dw repeat bit for bit; dx, dWg and dbg use fp32 atomics and are compared within 1e-6."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("bwd_repeat", 600, 256, 4, 2, 512, 1.25, 74)
+    inp = synth.make_inputs(cfg)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp), train=True)
+    dout = torch.from_numpy(synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float32)).cuda()
+    outs = []
+    for _ in range(3):
+        buf.forward_train()
+        g = buf.make_grads()
+        buf.backward(dout, g, D_AUX, D_Z)
+        torch.cuda.synchronize()
+        outs.append({n: t.cpu().numpy() for n, t in g.items()})
+    for o in outs[1:]:
+        for n in ("dW1", "dW2"):
+            assert np.array_equal(o[n], outs[0][n]), n
+        for n in ("dx", "dWg", "dbg", "db1", "db2", "dw"):
+            scale = float(np.abs(outs[0][n]).max()) or 1.0
+            assert np.max(np.abs(o[n] - outs[0][n])) <= 1e-6 * scale, n
