@@ -253,7 +253,8 @@ MOE_API moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_io_t* 
  * gradients are the chain rule through the forward definition: for L with dL/dout = dout,
  * dL/daux = d_aux and dL/dz = d_z, every input x, Wg, bg, W1, b1, W2, b2 gets dL/d(input).  The
  * top-k choice and the capacity drops are piecewise constant and carry no gradient; a dropped
- * slot contributes nothing.  bf16 storage only (else MOE_ERR_UNSUPPORTED); both routing rules.  Under
+ * slot contributes nothing.  Both storage types (bf16: tensor cores, intermediates in bf16; fp32:
+ * CUDA cores, intermediates in fp32) and both routing rules.  Under
  * expert choice the weight of a chosen pair is the softmax probability itself, so the gate receives
  * p (dw - sum p dw) with no renormalisation term, and the aux-loss term cancels (f_e = 1/E).
  * ------------------------------------------------------------------------------------------- */

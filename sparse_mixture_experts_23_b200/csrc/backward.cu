@@ -19,6 +19,10 @@
 namespace moe {
 namespace {
 
+__device__ __forceinline__ float ld_store(const void* p, size_t i, int f32) {
+  return f32 ? reinterpret_cast<const float*>(p)[i] : __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+}
+
 __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
   const int kept = a.offsets[a.E];
   const int nv = a.H / 4;  // float4 per dout row
@@ -30,6 +34,11 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdPrepArgs a) {
     const int t = a.row_token[r];
     const float w = a.topk_w[(size_t)t * a.k + a.row_slot[r]];
     const float4 v = dv[(size_t)t * nv + c];
+    if (a.f32) {
+      reinterpret_cast<float4*>(a.dperm)[(size_t)r * nv + c] = v;
+      reinterpret_cast<float4*>(a.dyperm)[(size_t)r * nv + c] = make_float4(w * v.x, w * v.y, w * v.z, w * v.w);
+      continue;
+    }
     const __nv_bfloat162 d01 = __floats2bfloat162_rn(v.x, v.y), d23 = __floats2bfloat162_rn(v.z, v.w);
     const __nv_bfloat162 y01 = __floats2bfloat162_rn(w * v.x, w * v.y), y23 = __floats2bfloat162_rn(w * v.z, w * v.w);
     uint2 dd, yy;
@@ -112,6 +121,7 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(BiasGradArgs a) {
   }
   if (a.db1 && c < a.F) {
     const __nv_bfloat162* du = reinterpret_cast<const __nv_bfloat162*>(a.du);
+    const float2* duf = reinterpret_cast<const float2*>(a.du);
     float2 acc = make_float2(0.f, 0.f);
     int cur = e_s[0];
     for (int i = 0; i < nr; ++i) {
@@ -121,7 +131,8 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(BiasGradArgs a) {
         acc = make_float2(0.f, 0.f);
         cur = e_s[i];
       }
-      const float2 v = __bfloat1622float2(du[((size_t)(r0 + i) * a.F + c) / 2]);
+      const size_t o = ((size_t)(r0 + i) * a.F + c) / 2;
+      const float2 v = a.f32 ? duf[o] : __bfloat1622float2(du[o]);
       acc.x += v.x;
       acc.y += v.y;
     }
@@ -138,14 +149,8 @@ __global__ void __launch_bounds__(256) ec_dw_scatter_kernel(EcDwArgs a) {
   const int t = a.row_token[r], e = a.row_slot[r];
   float bdot = 0.f;
   if (a.b2) {
-    const __nv_bfloat16* b2 = a.b2 + (size_t)e * a.H;
-    for (int h = 4 * lane; h < a.H; h += 128) {
-      const float4 d = *reinterpret_cast<const float4*>(a.dout + (size_t)t * a.H + h);
-      const uint2 bb = *reinterpret_cast<const uint2*>(b2 + h);
-      const float2 b01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb.x));
-      const float2 b23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bb.y));
-      bdot = fmaf(d.x, b01.x, fmaf(d.y, b01.y, fmaf(d.z, b23.x, fmaf(d.w, b23.y, bdot))));
-    }
+    for (int h = lane; h < a.H; h += 32)
+      bdot = fmaf(a.dout[(size_t)t * a.H + h], ld_store(a.b2, (size_t)e * a.H + h, a.f32), bdot);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) bdot += __shfl_xor_sync(0xffffffffu, bdot, o);
   }
@@ -225,8 +230,13 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
     float d = 0.f;
     if (!a.dropped[(size_t)t * k + q]) {
       float bdot = 0.f;
-      if (a.b2) {  // dout[t] . b2[e], four columns per lane per step (H is a multiple of 64)
-        const __nv_bfloat16* b2 = a.b2 + (size_t)e * H;
+      if (a.b2 && a.f32) {
+        for (int h = lane; h < H; h += 32)
+          bdot = fmaf(a.dout[(size_t)t * H + h], reinterpret_cast<const float*>(a.b2)[(size_t)e * H + h], bdot);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) bdot += __shfl_xor_sync(0xffffffffu, bdot, o);
+      } else if (a.b2) {  // dout[t] . b2[e], four columns per lane per step (H is a multiple of 64)
+        const __nv_bfloat16* b2 = reinterpret_cast<const __nv_bfloat16*>(a.b2) + (size_t)e * H;
         for (int h = 4 * lane; h < H; h += 128) {
           const float4 d = *reinterpret_cast<const float4*>(a.dout + (size_t)t * H + h);
           const uint2 bb = *reinterpret_cast<const uint2*>(b2 + h);
@@ -280,12 +290,22 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
   }
   __syncwarp();
   // dx[t] += Wg dlogits[t]: four rows of Wg per lane per step
+  if (a.f32) {  // fp32 gate: one row of Wg per lane per step
+    const float* wg = reinterpret_cast<const float*>(a.Wg);
+    for (int h = lane; h < H; h += 32) {
+      float acc = 0.f;
+      for (int e = 0; e < E; ++e) acc = fmaf(wg[(size_t)h * E + e], dl_s[warp][e], acc);
+      a.dx[(size_t)t * H + h] += acc;
+    }
+    return;
+  }
+  const __nv_bfloat16* Wgb = reinterpret_cast<const __nv_bfloat16*>(a.Wg);
   for (int h = 4 * lane; h < H; h += 128) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (E % 8 == 0) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint4* wrow = reinterpret_cast<const uint4*>(a.Wg + (size_t)(h + i) * E);
+        const uint4* wrow = reinterpret_cast<const uint4*>(Wgb + (size_t)(h + i) * E);
         for (int e8 = 0; e8 < E / 8; ++e8) {
           const uint4 v = wrow[e8];
           const __nv_bfloat162* w2 = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -299,7 +319,7 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
     } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        for (int e = 0; e < E; ++e) acc[i] = fmaf(__bfloat162float(a.Wg[(size_t)(h + i) * E + e]), dl_s[warp][e], acc[i]);
+        for (int e = 0; e < E; ++e) acc[i] = fmaf(__bfloat162float(Wgb[(size_t)(h + i) * E + e]), dl_s[warp][e], acc[i]);
     }
     float4* dxp = reinterpret_cast<float4*>(a.dx + (size_t)t * H + h);
     float4 v = *dxp;
@@ -323,6 +343,7 @@ __global__ void __launch_bounds__(256) gate_wgrad_kernel(GateWgradArgs a) {
   const int h = 2 * (blockIdx.x * 256 + threadIdx.x);
   const int t0 = blockIdx.y * kGwTokens, nt = min(kGwTokens, a.T - t0);
   const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(a.x);
+  const float2* xf2 = reinterpret_cast<const float2*>(a.x);
   for (int e0 = 0; e0 < E; e0 += 8) {
     const int ne = min(8, E - e0);
     __syncthreads();
@@ -337,7 +358,8 @@ __global__ void __launch_bounds__(256) gate_wgrad_kernel(GateWgradArgs a) {
       for (int q = 0; q < 8; ++q) acc0[q] = acc1[q] = 0.f;
 #pragma unroll 4
       for (int tt = 0; tt < nt; ++tt) {
-        const float2 xv = __bfloat1622float2(x2[((size_t)(t0 + tt) * H + h) / 2]);
+        const size_t xo = ((size_t)(t0 + tt) * H + h) / 2;
+        const float2 xv = a.f32 ? xf2[xo] : __bfloat1622float2(x2[xo]);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           acc0[q] = fmaf(xv.x, dl[tt][q], acc0[q]);

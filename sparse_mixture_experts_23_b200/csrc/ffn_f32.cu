@@ -102,10 +102,9 @@ __global__ void __launch_bounds__(256) ffn_f32_kernel(FfnArgs a, const float* __
       int n = n0 + tx * 4 + j;
       if (n >= N) continue;
       float v = acc[i][j] + (bias ? bias[(size_t)e * N + n] : 0.f);
-      if (EPI == EPI_GELU) {
-        reinterpret_cast<float*>(a.h)[(size_t)grow * N + n] = gelu_erf(v);
-      } else if (EPI == EPI_SILU) {
-        reinterpret_cast<float*>(a.h)[(size_t)grow * N + n] = silu(v);
+      if (EPI == EPI_GELU || EPI == EPI_SILU) {
+        reinterpret_cast<float*>(a.h)[(size_t)grow * N + n] = EPI == EPI_GELU ? gelu_erf(v) : silu(v);
+        if (a.u_out) reinterpret_cast<float*>(a.u_out)[(size_t)grow * N + n] = v;  // training forward
       } else if (EPI == EPI_COMBINE) {
         atomicAdd(&a.out[(size_t)tok * N + n], w * v);
       } else {

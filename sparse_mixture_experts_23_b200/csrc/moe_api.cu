@@ -499,7 +499,6 @@ size_t moe_train_workspace_size(const moe_shape_t* shape) {
 static moe_status_t check_train(const moe_shape_t* shape, void* ws, size_t ws_bytes) {
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
-  if (shape->dtype != MOE_DTYPE_BF16) return MOE_ERR_UNSUPPORTED;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;
   if (ws_bytes < ws_layout(*shape).train_total) return MOE_ERR_WORKSPACE;
   return MOE_OK;
@@ -550,6 +549,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
     return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*shape);
   const bool ec = shape->routing == MOE_ROUTING_EXPERT_CHOICE;
+  const int f32 = shape->dtype == MOE_DTYPE_F32 ? 1 : 0;
   const int kw = ec ? shape->E : shape->k;  // stride of the combine weights in topk_w
   const int32_t* offsets = at<int32_t>(ws, L.offsets);
   const int32_t* row_token = at<int32_t>(ws, L.row_token);
@@ -561,6 +561,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   pa.H = shape->H;
   pa.E = shape->E;
   pa.k = kw;
+  pa.f32 = f32;
   pa.offsets = offsets;
   pa.row_token = row_token;
   pa.row_slot = row_slot;
@@ -607,7 +608,9 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   ga.status = at<int32_t>(ws, L.status);
   ga.wait_limit = g_wait_limit;
   ga.num_sms = num_sms();
-  if ((st = cuda_status(launch_bwd_gemms_sm100(ga, stream, &g_launches))) != MOE_OK) return st;
+  if ((st = cuda_status(f32 ? launch_bwd_gemms_f32(ga, stream, &g_launches)
+                            : launch_bwd_gemms_sm100(ga, stream, &g_launches))) != MOE_OK)
+    return st;
 
   if (grad->db1 || grad->db2) {
     BiasGradArgs ba{};
@@ -615,6 +618,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
     ba.F = shape->F;
     ba.E = shape->E;
     ba.k = kw;
+    ba.f32 = f32;
     ba.rows_cap = (int)L.rows;
     ba.offsets = offsets;
     ba.row_token = row_token;
@@ -637,7 +641,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
     da.row_slot = row_slot;
     da.dwraw = pa.dwraw;
     da.dout = grad->dout;
-    da.b2 = reinterpret_cast<const __nv_bfloat16*>(io->b2);
+    da.b2 = io->b2;
+    da.f32 = f32;
     da.dwmat = dlogits;
     ++g_launches;
     if ((st = cuda_status(launch_ec_dw_scatter(da, stream))) != MOE_OK) return st;
@@ -656,8 +661,9 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   ra.cnt_pre = at<int32_t>(ws, L.cnt_pre);
   ra.dwraw = pa.dwraw;
   ra.dout = grad->dout;
-  ra.b2 = reinterpret_cast<const __nv_bfloat16*>(io->b2);
-  ra.Wg = reinterpret_cast<const __nv_bfloat16*>(io->Wg);
+  ra.b2 = io->b2;
+  ra.Wg = io->Wg;
+  ra.f32 = f32;
   ra.d_aux = grad->d_aux;
   ra.d_z = grad->d_z;
   ra.dlogits = dlogits;
@@ -671,7 +677,8 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
   wa.T = shape->T;
   wa.H = shape->H;
   wa.E = shape->E;
-  wa.x = reinterpret_cast<const __nv_bfloat16*>(io->x);
+  wa.x = io->x;
+  wa.f32 = f32;
   wa.dlogits = ra.dlogits;
   wa.dWg = grad->dWg;
   wa.dbg = grad->dbg;

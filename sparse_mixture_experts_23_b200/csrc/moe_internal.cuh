@@ -156,6 +156,7 @@ cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st);
 // ---- backward pass ----
 struct BwdPrepArgs {
   int T, H, E, F, k;
+  int f32;            // storage dtype fp32: dperm / dyperm are written as fp32
   const int32_t* offsets;
   const int32_t* row_token;
   const int32_t* row_slot;
@@ -174,6 +175,7 @@ struct BwdPrepArgs {
 
 struct BiasGradArgs {
   int H, F, E, k, rows_cap;
+  int f32;         // du is fp32
   const int32_t* offsets;
   const int32_t* row_token;
   const int32_t* row_slot;
@@ -194,8 +196,9 @@ struct RouterBwdArgs {
   const int32_t* cnt_pre;
   const float* dwraw;
   const float* dout;
-  const __nv_bfloat16* b2;  // [E,H] or null
-  const __nv_bfloat16* Wg;  // [H,E]
+  const void* b2;  // [E,H] storage dtype, or null
+  const void* Wg;  // [H,E] storage dtype
+  int f32;         // storage dtype fp32
   float d_aux, d_z;
   float* dlogits;  // [T,E] out
   float* dw_out;   // [T,k] out (token choice) or [T,E] (expert choice), or null
@@ -205,7 +208,8 @@ struct RouterBwdArgs {
 
 struct GateWgradArgs {
   int T, H, E, chunk;
-  const __nv_bfloat16* x;
+  int f32;  // x is fp32
+  const void* x;
   const float* dlogits;
   float* dWg;
   float* dbg;  // or null
@@ -241,8 +245,9 @@ struct EcDwArgs {
   const int32_t* row_slot;
   const float* dwraw;
   const float* dout;
-  const __nv_bfloat16* b2;  // or null
-  float* dwmat;             // [T,E]
+  const void* b2;  // storage dtype, or null
+  int f32;
+  float* dwmat;    // [T,E]
 };
 
 cudaError_t launch_bwd_prep(const BwdPrepArgs& a, cudaStream_t st);
@@ -252,6 +257,8 @@ cudaError_t launch_router_bwd(const RouterBwdArgs& a, cudaStream_t st);
 cudaError_t launch_gate_wgrad(GateWgradArgs a, cudaStream_t st);
 // dgrad of W2 (du, dw partials), dgrad of W1 (scatter-add into dx), weight gradients of W2 and W1
 cudaError_t launch_bwd_gemms_sm100(const BwdGemmArgs& a, cudaStream_t st, int* launches);
+// the same four GEMMs for fp32 storage, on CUDA cores
+cudaError_t launch_bwd_gemms_f32(const BwdGemmArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st);
 cudaError_t launch_ec_combine(const float* y, const int32_t* row_token, const int32_t* row_slot, const float* topk_w,
                               int rows, int E, int H, float* out, cudaStream_t st);

@@ -294,3 +294,35 @@ def test_backward_deterministic_parts_repeat_bitwise():
         for n in ("dx", "dWg", "dbg", "db1", "db2", "dw"):
             scale = float(np.abs(outs[0][n]).max()) or 1.0
             assert np.max(np.abs(o[n] - outs[0][n])) <= 1e-6 * scale, n
+
+
+F32_CASES = [
+    synth.LayerConfig("bwd_f32_ragged", T=77, H=20, E=5, k=2, F=12, CF=math.inf, dtype="f32", seed=81),
+    synth.LayerConfig("bwd_f32_drops", T=256, H=64, E=4, k=2, F=256, CF=1.0, dtype="f32", seed=82),
+    synth.LayerConfig("bwd_f32_silu_nobias", T=100, H=32, E=4, k=1, F=64, CF=1.25, dtype="f32", seed=83, act="silu",
+                      bias=False),
+    synth.LayerConfig("bwd_f32_expert_choice", T=96, H=32, E=4, k=2, F=48, CF=1.0, dtype="f32", seed=84,
+                      routing="expert_choice"),
+]
+
+
+@pytest.mark.parametrize("cfg", F32_CASES, ids=lambda c: c.name)
+def test_backward_f32_all_gradients(cfg):
+    """fp32 storage: every gradient on CUDA cores with fp32 intermediates, within the fp32 rule
+    (max|d| <= 1e-4 max|ref| per tensor) of the oracle's chain rule fed the GPU's routing."""
+    from moe_testlib import TOL_F32, normwise_rel
+
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    r = _run(cfg, dout)
+    inp = r["inp"]
+    if cfg.routing == "expert_choice":
+        ref = oracle.backward_ec(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype,
+                                 dout, D_AUX, D_Z, act=cfg.act, chosen=r["topk_idx"])
+    else:
+        ref = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, dout,
+                              D_AUX, D_Z, act=cfg.act, topk_idx=r["topk_idx"], dropped=r["dropped"])
+    names = ["dx", "dWg", "dW1", "dW2", "dw"] + (["dbg", "db1", "db2"] if cfg.bias else [])
+    for n in names:
+        err = normwise_rel(r[n], getattr(ref, n))
+        print(f"  {cfg.name} {n}: {err:.3e}")
+        assert err <= TOL_F32, (n, err)
