@@ -209,7 +209,8 @@ MOE_API moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t*
  * Mixtral block gather by expert).  Assignments are visited slot-major then by token; an
  * assignment is kept iff fewer than `capacity` earlier assignments went to its expert.
  * Reads x, topk_idx.  Writes expert_counts, dropped, the row maps and x_perm in ws, and clears
- * out[T,H] to zero (the fused combine accumulates into it).
+ * out[T,H] to zero (the fused combine accumulates into it).  The kernels check every index they
+ * read from topk_idx (see moe_get_device_status); nothing outside the buffers is touched.
  * Expert choice: nothing is dropped (each expert already holds exactly C tokens); reads x and
  * topk_idx[E,C], writes the row maps and x_perm, and clears out. */
 MOE_API moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
@@ -295,7 +296,10 @@ MOE_API moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, 
                           size_t ws_bytes, cudaStream_t stream);
 
 /* Synchronises `stream`, then reads and clears the workspace's device error word.
- * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out) or MOE_ERR_CUDA. */
+ * Returns MOE_OK, MOE_ERR_TIMEOUT (a bounded device wait ran out), MOE_ERR_INVALID_ARG (a kernel met
+ * an out-of-range entry in a caller-supplied index array -- an expert outside [0, E) in topk_idx, or
+ * a token outside [0, T) in an expert-choice topk_idx -- and skipped it: such a slot counts as dropped,
+ * such a row computes on zeros for token 0; results are then not meaningful) or MOE_ERR_CUDA. */
 MOE_API moe_status_t moe_get_device_status(void* ws, cudaStream_t stream);
 
 /* Bound on device-side waits, in GPU clock cycles (default 2e9, about one second).  Applies to

@@ -160,7 +160,11 @@ __global__ void __launch_bounds__(256) ec_gather_kernel(EcGatherArgs a) {
     int t = -1;
     if (r < rows) {
       t = a.chosen[r];
-      a.row_token[r] = t;
+      if (t < 0 || t >= a.T) {  // caller-supplied token outside [0, T): a zero row for token 0, error recorded
+        atomicCAS(a.status, 0, kDevBadIndex);
+        t = -1;
+      }
+      a.row_token[r] = t < 0 ? 0 : t;
       a.row_slot[r] = (int)(r / a.C);
     }
     tok_s[tid] = t;
@@ -189,12 +193,13 @@ __global__ void __launch_bounds__(256) ec_gather_kernel(EcGatherArgs a) {
       }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u)
-      if (ok[u]) {
-        const int idx = i + u * 256;
-        const int r = idx / nvec, c = idx % nvec;
-        pv[(size_t)(r0 + r) * nvec + c] = v[u];
-      }
+    for (int u = 0; u < U; ++u) {
+      const int idx = i + u * 256;
+      if (idx >= total) continue;
+      const int r = idx / nvec, c = idx % nvec;
+      if (ok[u]) pv[(size_t)(r0 + r) * nvec + c] = v[u];
+      else if (r0 + r < rows) pv[(size_t)(r0 + r) * nvec + c] = make_uint4(0u, 0u, 0u, 0u);  // invalid token
+    }
   }
   const long long ovec = (long long)a.T * a.H / 4;
   float4* o = reinterpret_cast<float4*>(a.out);

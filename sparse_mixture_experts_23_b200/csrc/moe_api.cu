@@ -8,6 +8,8 @@
 #include <mutex>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>  // header-only; the calls cost nothing unless a profiler is attached
+
 #include "moe_internal.cuh"
 
 namespace moe {
@@ -112,6 +114,13 @@ using namespace moe;
 namespace {
 
 thread_local int g_launches = 0;
+
+// One NVTX range per entry-point call ("moe_route", "moe_forward", ...), so that a timeline shows the
+// stages of a layer call around its kernels.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 long long g_wait_limit = 2000000000LL;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -229,6 +238,7 @@ moe_status_t do_ec_select_and_losses(const moe_shape_t* s, const moe_io_t* io, v
 moe_status_t do_ec_gather(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st) {
   const WsLayout L = ws_layout(*s);
   EcGatherArgs a{};
+  a.status = at<int32_t>(ws, L.status);
   a.x = io->x;
   a.T = s->T;
   a.H = s->H;
@@ -269,6 +279,7 @@ ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int d
 moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st) {
   const WsLayout L = ws_layout(*s);
   ScatterArgs a{};
+  a.status = at<int32_t>(ws, L.status);
   a.x = io->x;
   a.T = s->T;
   a.H = s->H;
@@ -368,6 +379,7 @@ moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, moe_ws_vie
 }
 
 moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_route");
   g_launches = 0;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
@@ -392,6 +404,7 @@ moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, s
 
 moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_permute");
   g_launches = 0;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
@@ -412,6 +425,7 @@ moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   const WsLayout L = ws_layout(*shape);
   ++g_launches;
   if ((st = cuda_status(launch_hist(io->topk_idx, shape->T, shape->E, shape->k, L.nblk, at<int32_t>(ws, L.chunk_hist),
+                                    at<int32_t>(ws, L.status),
                                     stream))) != MOE_OK)
     return st;
   ++g_launches;
@@ -421,6 +435,7 @@ moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws,
 
 moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, int fuse_combine,
                             cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_expert_ffn");
   g_launches = 0;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
@@ -436,6 +451,7 @@ moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io, void* 
 }
 
 moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_combine");
   g_launches = 0;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
@@ -454,6 +470,7 @@ moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws,
 }
 
 moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_forward");
   g_launches = 0;
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
@@ -506,6 +523,7 @@ static moe_status_t check_train(const moe_shape_t* shape, void* ws, size_t ws_by
 
 moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                                cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_forward_train");
   g_launches = 0;
   moe_status_t st = check_train(shape, ws, ws_bytes);
   if (st != MOE_OK) return st;
@@ -534,6 +552,7 @@ moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, voi
 
 moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const moe_grad_t* grad, void* ws,
                           size_t ws_bytes, cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_backward");
   g_launches = 0;
   moe_status_t st = check_train(shape, ws, ws_bytes);
   if (st != MOE_OK) return st;
@@ -688,6 +707,7 @@ moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const mo
 
 moe_status_t moe_forward_host(const moe_shape_t* shape, const moe_io_t* io, const void* x_host, float* out_host,
                               void* ws, size_t ws_bytes, cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_forward_host");
   moe_status_t st = check_shape(shape);
   if (st != MOE_OK) return st;
   if (io == nullptr || x_host == nullptr || out_host == nullptr || io->x == nullptr || io->out == nullptr)
@@ -712,7 +732,7 @@ moe_status_t moe_get_device_status(void* ws, cudaStream_t stream) {
   if (word != 0) {
     const int32_t zero = 0;
     if (cudaMemcpy(ws, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return MOE_ERR_CUDA;
-    return MOE_ERR_TIMEOUT;
+    return word == kDevBadIndex ? MOE_ERR_INVALID_ARG : MOE_ERR_TIMEOUT;
   }
   return MOE_OK;
 }

@@ -22,6 +22,7 @@ enum DevError : int {
   kDevTimeoutEpilogue = 0x103,
   kDevTimeoutProbe = 0x104,
   kDevTimeoutDrain = 0x105,
+  kDevBadIndex = 0x201,  // an index array given by the caller held an out-of-range entry (it was skipped)
 };
 
 // Workspace sections (byte offsets from the workspace base, 256-aligned).
@@ -75,6 +76,7 @@ struct EcSelectArgs {
 };
 
 struct EcGatherArgs {
+  int32_t* status;  // device error word
   const void* x;
   int T, H, E, C, esize;
   const int32_t* chosen;  // [E][C]
@@ -101,6 +103,7 @@ struct ReduceArgs {
 };
 
 struct ScatterArgs {
+  int32_t* status;  // device error word
   const void* x;
   int T, H, E, k, nblk, esize;
   long long cap;
@@ -144,7 +147,8 @@ struct FfnArgs {
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 
 cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* launches);
-cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, cudaStream_t st);
+cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, int32_t* status,
+                        cudaStream_t st);
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
 cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);

@@ -804,14 +804,21 @@ __global__ void __launch_bounds__(kRouterThreads) router_logits_finish_kernel(Ro
 }
 
 // Per-chunk, per-slot expert histogram from a given topk_idx (standalone permute).
-__global__ void hist_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int32_t* __restrict__ chunk_hist) {
+// An expert index outside [0, E) (from a caller-supplied topk_idx) is not counted; the error word
+// records it and moe_get_device_status reports it.
+__global__ void hist_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int32_t* __restrict__ chunk_hist,
+                            int32_t* status) {
   __shared__ int hist[8 * 256];
   const int blk = blockIdx.x, nblk = gridDim.x, tid = threadIdx.x;
   for (int i = tid; i < k * E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
   if (tid < kChunk * k) {
     int s = tid / kChunk, t = blk * kChunk + (tid % kChunk);
-    if (t < T) atomicAdd(&hist[s * E + topk_idx[(size_t)t * k + s]], 1);
+    if (t < T) {
+      const int e = topk_idx[(size_t)t * k + s];
+      if (e >= 0 && e < E) atomicAdd(&hist[s * E + e], 1);
+      else atomicCAS(status, 0, kDevBadIndex);
+    }
   }
   __syncthreads();
   for (int i = tid; i < k * E; i += blockDim.x) {
@@ -957,11 +964,17 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
   if (tid < 32) {
     const int lane = tid;
     const int t = b * kChunk + lane;
-    const bool valid = t < a.T;
-    const int e = valid ? a.topk_idx[(size_t)t * a.k + s] : -1 - lane;  // invalid lanes never match
+    int e = t < a.T ? a.topk_idx[(size_t)t * a.k + s] : -1;
+    if (t < a.T && (e < 0 || e >= a.E)) atomicCAS(a.status, 0, kDevBadIndex);  // dropped below, never copied
+    const bool valid = t < a.T && e >= 0 && e < a.E;
+    if (!valid) e = -1 - lane;  // invalid lanes never match
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank_local = __popc(peers & ((1u << lane) - 1u));
     int row = -1;
+    if (t < a.T && !valid) {
+      a.dropped[(size_t)t * a.k + s] = 1;
+      a.row_of[(size_t)t * a.k + s] = -1;
+    }
     if (valid) {
       const long long rank = (long long)a.chunk_base[((size_t)s * nblk + b) * a.E + e] + rank_local;
       const bool keep = a.cap < 0 || rank < a.cap;
@@ -1145,8 +1158,9 @@ cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, cudaStream_t st) {
-  hist_kernel<<<nblk, 256, 0, st>>>(topk_idx, T, E, k, chunk_hist);
+cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, int32_t* status,
+                        cudaStream_t st) {
+  hist_kernel<<<nblk, 256, 0, st>>>(topk_idx, T, E, k, chunk_hist, status);
   return cudaGetLastError();
 }
 

@@ -247,3 +247,41 @@ def test_stream_ordering_on_side_stream():
              topk_w=buf.topk_w.cpu().numpy(), dropped=buf.dropped.cpu().numpy(),
              counts=buf.expert_counts.cpu().numpy(), losses=buf.losses.cpu().numpy())
     _check_against_oracle(cfg, r)
+
+
+def test_out_of_range_indices_are_reported_not_followed():
+    """A caller-supplied topk_idx with an expert outside [0, E) (token choice), or a chosen token outside
+    [0, T) (expert choice): the kernels skip the entry, touch nothing outside the buffers, and the device
+    status reports MOE_ERR_INVALID_ARG once; the next call on the same workspace is clean."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("bad_index", 96, 128, 4, 2, 128, math.inf, "bf16", 37)
+    inp = synth.make_inputs(cfg)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf.route()
+    bad = buf.topk_idx.clone()
+    buf.topk_idx[5, 1] = 1000
+    buf.topk_idx[9, 0] = -3
+    buf.permute()
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_ERR_INVALID_ARG
+    dropped = buf.dropped.cpu().numpy()
+    assert dropped[5, 1] == 1 and dropped[9, 0] == 1
+    assert int(buf.expert_counts.sum().item()) == cfg.T * cfg.k - 2
+    buf.topk_idx.copy_(bad)
+    buf.forward()
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+
+    ec = _cfg("bad_token_ec", 96, 128, 4, 2, 128, 1.0, "bf16", 38, routing="expert_choice")
+    inp = synth.make_inputs(ec)
+    buf = moe.MoEBuffers(shape_of(ec), upload(inp))
+    buf.route()
+    buf.topk_idx[2, 3] = ec.T + 7
+    buf.permute()
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_ERR_INVALID_ARG
+    buf.forward()
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
