@@ -92,6 +92,7 @@ struct GemmArgs {
   const float* topk_w;
   int k;
   int single_rows;  // offsets == null: one segment of this many rows (a plain dense GEMM)
+  int a_box_rows;   // single-CTA kernel: > 0 loads only ceil(rows / a_box_rows) boxes of that many A rows
   int32_t* status;
   long long wait_limit;
 };
@@ -276,7 +277,8 @@ __device__ __forceinline__ void epilogue_dgrad32(const GemmArgs& g, const uint32
 
 template <int BN, int EPI, bool BKM>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, GemmArgs g) {
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmA16, GemmArgs g) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -347,9 +349,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t a_dst = sbase + stage * C::kABytes;
           const uint32_t b_dst = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
-          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
           armed[stage] = (int)phase;
-          tma_load_2d(a_dst, &tmA, kb * BK, row0, full_bar(stage));
+          if (g.a_box_rows > 0) {
+            // small segments: only the boxes that hold the tile's rows (the MMA's other A rows are
+            // stale shared memory; their accumulator rows are never stored)
+            const int nb = (rows + g.a_box_rows - 1) / g.a_box_rows;
+            mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(nb * g.a_box_rows * BK * 2 + C::kBBytes));
+            for (int j = 0; j < nb; ++j)
+              tma_load_2d(a_dst + j * g.a_box_rows * 128, &tmA16, kb * BK, row0 + j * g.a_box_rows, full_bar(stage));
+          } else {
+            mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+            tma_load_2d(a_dst, &tmA, kb * BK, row0, full_bar(stage));
+          }
           if constexpr (BKM) {
             // B stored [E][N][K]: one 64 k x BN rows box, k contiguous
             tma_load_3d(b_dst, &tmB, kb * BK, n_idx * BN, e, full_bar(stage));
@@ -1336,6 +1347,19 @@ bool make_map_a(CUtensorMap* m, const void* base, int rows, int K) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A operand in 16-row boxes (box = 64 k x 16 rows) for segments of a few rows
+bool make_map_a16(CUtensorMap* m, const void* base, int rows, int K) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {BK, 16};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // GEMM1 output h: [rows, N] bf16 row-major; stores of 64 columns x 32 rows, 128-byte swizzle
 bool make_map_store(CUtensorMap* m, void* base, int rows, int N) {
   auto enc = get_encode_fn();
@@ -1403,12 +1427,14 @@ bool make_map_dw(CUtensorMap* m, float* base, int E, int M, int N) {
          CUDA_SUCCESS;
 }
 
+// ma16: the same A operand in 16-row boxes, used when g.a_box_rows = 16 (else any valid map)
 template <int BN, int EPI, bool BKM = false>
-cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid, cudaStream_t st) {
+cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mb, const GemmArgs& g, int grid, cudaStream_t st,
+                       const CUtensorMap* ma16 = nullptr) {
   auto kern = grouped_gemm_kernel<BN, EPI, BKM>;
   cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(kern), Cfg<BN>::kSmemBytes);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, Cfg<BN>::kSmemBytes, st>>>(ma, mb, g);
+  kern<<<grid, kThreads, Cfg<BN>::kSmemBytes, st>>>(ma, mb, ma16 ? *ma16 : ma, g);
   return cudaGetLastError();
 }
 
@@ -1426,11 +1452,35 @@ cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUte
 // shorter segments (many experts, or few tokens) most of a 256-row tile would be padding, and the
 // 128-row single-CTA tiles waste half as much.  The host sees only the expected rows per expert
 // (T*k/E); the actual counts stay on the device.
+// Small segments (a few rows per expert, e.g. decode): the GEMM streams the weights, and every tile
+// loads only the 16-row A boxes that hold its rows.  The tile width is then chosen for the fewest
+// weight-streaming waves: cost = waves x (16 + BN), ties to the widest.
+int pick_bn_small(int N, int E, int grid) {
+  int best = 0;
+  long long best_cost = -1;
+  for (int bn = 256; bn >= 64; bn >>= 1) {
+    if (N % bn != 0) continue;
+    const long long tiles = (long long)E * (N / bn);
+    const long long cost = ((tiles + grid - 1) / grid) * (16 + bn);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
 template <int EPI>
 cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmArgs& g,
-                      int grid, long long avg_rows, cudaStream_t st) {
+                      int grid, long long avg_rows, cudaStream_t st, const CUtensorMap* ma16 = nullptr) {
   if (N % 256 == 0 && g.K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled())
     return launch_pair<EPI>(ma, mb, mc, g, grid, st);
+  if (ma16 != nullptr && g.a_box_rows > 0) {
+    const int bn = pick_bn_small(N, g.E, grid);
+    if (bn == 256) return launch_one<256, EPI>(ma, mb, g, grid, st, ma16);
+    if (bn == 128) return launch_one<128, EPI>(ma, mb, g, grid, st, ma16);
+    return launch_one<64, EPI>(ma, mb, g, grid, st, ma16);
+  }
   if (N % 256 == 0) return launch_one<256, EPI>(ma, mb, g, grid, st);
   if (N % 128 == 0) return launch_one<128, EPI>(ma, mb, g, grid, st);
   return launch_one<64, EPI>(ma, mb, g, grid, st);
@@ -1540,6 +1590,11 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
       !make_map_store(&mc1, a.h, a.rows_cap, a.F))
     return cudaErrorInvalidValue;
   const int grid = a.num_sms > 0 ? a.num_sms : 148;
+  // a few rows per expert on average: 16-row A boxes (decode-sized batches)
+  const bool small = a.avg_rows < 32;
+  CUtensorMap ma1s, ma2s;
+  if (small && (!make_map_a16(&ma1s, a.x_perm, a.rows_cap, a.H) || !make_map_a16(&ma2s, a.h, a.rows_cap, a.F)))
+    return cudaErrorInvalidValue;
 
   GemmArgs g1{};
   g1.offsets = a.offsets;
@@ -1550,11 +1605,13 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.h_out = reinterpret_cast<__nv_bfloat16*>(a.h);
   g1.u_out = reinterpret_cast<__nv_bfloat16*>(a.u_out);
   g1.k = a.k;
+  g1.a_box_rows = small ? 16 : 0;
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
   const long long avg_rows = a.avg_rows;
-  cudaError_t err = a.act == MOE_ACT_SILU ? launch_bn<EPI_SILU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st)
-                                          : launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st);
+  cudaError_t err = a.act == MOE_ACT_SILU
+                        ? launch_bn<EPI_SILU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st, small ? &ma1s : nullptr)
+                        : launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st, small ? &ma1s : nullptr);
   if (err != cudaSuccess) return err;
   ++*launches;
 
@@ -1570,9 +1627,9 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g2.row_slot = a.row_slot;
   g2.topk_w = a.topk_w;
   if (a.fuse_combine)
-    err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st);
+    err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, small ? &ma2s : nullptr);
   else
-    err = launch_bn<EPI_STORE_Y>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st);
+    err = launch_bn<EPI_STORE_Y>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, small ? &ma2s : nullptr);
   if (err != cudaSuccess) return err;
   ++*launches;
   return cudaSuccess;
