@@ -425,6 +425,10 @@ def run_ours_impl(args, cfg):
     out_diff = float((hosts[0][1] - hosts[1][1]).abs().max())  # both buffer sets ran the same x
     e2e_status = max(buf.device_status(), buf2.device_status())
     del buf2, inputs2
+    # losses of the whole job's batch: every replica's loss sums all-reduced (one small collective,
+    # outside the timed regions; with one GPU these are this batch's own losses)
+    buf.forward()
+    global_losses = buf.global_losses().cpu().numpy()
 
     if rank != 0:
         if world > 1:
@@ -500,7 +504,8 @@ def run_ours_impl(args, cfg):
         },
         "train": train,
         "layer": {"kept": kept, "dropped": drops, "touched_experts": touched, "aux_loss": float(losses[0]),
-                  "z_loss": float(losses[1]), "expert_counts_min_max": [int(counts.min()), int(counts.max())]},
+                  "z_loss": float(losses[1]), "expert_counts_min_max": [int(counts.min()), int(counts.max())],
+                  "global_aux_loss": float(global_losses[0]), "global_z_loss": float(global_losses[1])},
     }
     print(json.dumps(line), flush=True)
     if world > 1:

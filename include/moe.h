@@ -205,6 +205,29 @@ MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, voi
  * Token choice only: an expert-choice shape returns MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream);
 
+/* Losses of a batch split over data-parallel replicas ("MoE Training" page, Core Concepts 3:
+ * load_balancing_loss, router_z_loss).  Both losses are built from sums over tokens:
+ *   aux = E * sum_e (cnt_e / sum_e' cnt_e') * (Psum_e / T),   z = Zsum / T,
+ * with cnt_e the assignments routed to expert e before any drop (T*k in all under token choice,
+ * E*C under expert choice), Psum_e = sum_t p[t,e] and Zsum = sum_t lse_t^2.  Each sum is additive
+ * over disjoint token sets, so adding the replicas' sums (an all-reduce) and applying the formula
+ * gives the losses of the whole batch -- which a mean of the replicas' own aux values does not,
+ * as aux is a product of two means.
+ *
+ * moe_loss_sums: after moe_route, moe_forward or moe_forward_train on ws (same shape, same stream),
+ * writes the 2E+2 fp32 sums of this call's batch to the device buffer sums (caller-owned, 4-byte
+ * aligned): sums[0..E) = cnt_e, sums[E..2E) = Psum_e, sums[2E] = Zsum, sums[2E+1] = T.  Counts and
+ * T are exact below 2^24.  T = 0 gives zeros.  Errors: MOE_ERR_INVALID_ARG (null sums or bad
+ * shape), MOE_ERR_WORKSPACE, MOE_ERR_CUDA.  One launch.
+ *
+ * moe_losses_from_sums: aux_loss and z_loss (device fp32 scalars) from 2E+2 sums laid out as above
+ * -- one replica's, or their element-wise total over replicas.  A total of T = 0 gives zeros.
+ * Errors: MOE_ERR_INVALID_ARG (E outside [1, 256] or a null pointer), MOE_ERR_CUDA.  One launch. */
+MOE_API moe_status_t moe_loss_sums(const moe_shape_t* shape, void* ws, size_t ws_bytes, float* sums,
+                           cudaStream_t stream);
+MOE_API moe_status_t moe_losses_from_sums(int E, const float* sums, float* aux_loss, float* z_loss,
+                                  cudaStream_t stream);
+
 /* Dispatch (Core Concepts 4 "capacity_factor", "drop_tokens"; Best Practices 2; Advanced Patterns
  * Mixtral block gather by expert).  Assignments are visited slot-major then by token; an
  * assignment is kept iff fewer than `capacity` earlier assignments went to its expert.

@@ -26,7 +26,7 @@ ENTRY_POINTS = (
     "moe_workspace_size", "moe_workspace_layout", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
     "moe_forward", "moe_forward_host", "moe_get_device_status", "moe_set_wait_limit", "moe_debug_timeout_probe",
     "moe_last_launch_count", "moe_status_string", "moe_route_noalloc", "moe_capacity",
-    "moe_train_workspace_size", "moe_forward_train", "moe_backward",
+    "moe_train_workspace_size", "moe_forward_train", "moe_backward", "moe_loss_sums", "moe_losses_from_sums",
 )
 
 
@@ -92,6 +92,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_backward.argtypes = [P(Shape), P(IO), P(Grad), vp, sz, vp]
     lib.moe_backward.restype = st
     lib.moe_forward_host.restype = st
+    lib.moe_loss_sums.argtypes = [P(Shape), vp, sz, vp, vp]
+    lib.moe_loss_sums.restype = st
+    lib.moe_losses_from_sums.argtypes = [ctypes.c_int, vp, vp, vp, vp]
+    lib.moe_losses_from_sums.restype = st
     lib.moe_get_device_status.argtypes = [vp, vp]
     lib.moe_get_device_status.restype = st
     lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
@@ -177,6 +181,40 @@ def moe_backward(shape, io, grad, ws, ws_bytes, stream=0) -> int:
 def moe_forward_host(shape, io, x_host, out_host, ws, ws_bytes, stream=0) -> int:
     return load_library().moe_forward_host(ctypes.byref(shape), ctypes.byref(io), x_host, out_host, ws, ws_bytes,
                                            stream)
+
+
+def moe_loss_sums(shape, ws, ws_bytes, sums, stream=0) -> int:
+    return load_library().moe_loss_sums(ctypes.byref(shape), ws, ws_bytes, sums, stream)
+
+
+def moe_losses_from_sums(E, sums, aux_loss, z_loss, stream=0) -> int:
+    return load_library().moe_losses_from_sums(int(E), sums, aux_loss, z_loss, stream)
+
+
+def loss_sums_size(E: int) -> int:
+    """Length of the loss-sum vector: [cnt_e (E)][Psum_e (E)][Zsum][T]."""
+    return 2 * E + 2
+
+
+def allreduce_sums(sums, group=None):
+    """Element-wise total of every replica's loss sums (in place) over the torch.distributed process
+    group, when one is initialised; a single process keeps its own.  Host plumbing only: the sums
+    and the losses are computed by moe_loss_sums / moe_losses_from_sums."""
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(sums, op=dist.ReduceOp.SUM, group=group)
+    return sums
+
+
+def losses_from_sums(E: int, sums):
+    """[aux_loss, z_loss] (fp32 CUDA tensor) from a CUDA tensor of 2E+2 loss sums."""
+    import torch
+
+    out = torch.empty((2,), dtype=torch.float32, device=sums.device)
+    _check(moe_losses_from_sums(E, sums.data_ptr(), out.data_ptr(), out.data_ptr() + 4,
+                                torch.cuda.current_stream().cuda_stream), "moe_losses_from_sums")
+    return out
 
 
 def moe_get_device_status(ws, stream=0) -> int:
@@ -277,6 +315,20 @@ class MoEBuffers:
 
     def device_status(self) -> int:
         return moe_get_device_status(self.ws_ptr, self.stream())
+
+    def loss_sums(self):
+        """The 2E+2 additive loss sums of the last routed batch (fp32 CUDA tensor)."""
+        import torch
+
+        sums = torch.empty((loss_sums_size(self.shape.E),), dtype=torch.float32, device=self.out.device)
+        _check(moe_loss_sums(self.shape, self.ws_ptr, self.ws_bytes, sums.data_ptr(), self.stream()), "moe_loss_sums")
+        return sums
+
+    def global_losses(self, group=None):
+        """[aux_loss, z_loss] of the whole batch across data-parallel replicas: every rank's loss sums
+        all-reduced over `group`, then the losses from the totals.  Call on every rank after the
+        forward pass, in the same order (it is a collective)."""
+        return losses_from_sums(self.shape.E, allreduce_sums(self.loss_sums(), group))
 
     # ---- training (buffers built with train=True) ----
     def forward_train(self):

@@ -402,6 +402,28 @@ moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, s
   return cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 0), stream));
 }
 
+moe_status_t moe_loss_sums(const moe_shape_t* shape, void* ws, size_t ws_bytes, float* sums, cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_loss_sums");
+  g_launches = 0;
+  moe_status_t st = check_shape(shape);
+  if (st != MOE_OK) return st;
+  if (sums == nullptr || (reinterpret_cast<uintptr_t>(sums) & 3u) != 0) return MOE_ERR_INVALID_ARG;
+  if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
+  const WsLayout L = ws_layout(*shape);
+  ++g_launches;
+  return cuda_status(launch_loss_sums(at<float>(ws, L.loss_part), at<int32_t>(ws, L.cnt_pre), L.nblk, shape->E,
+                                      shape->T, sums, stream));
+}
+
+moe_status_t moe_losses_from_sums(int E, const float* sums, float* aux_loss, float* z_loss, cudaStream_t stream) {
+  NvtxRange nvtx_range("moe_losses_from_sums");
+  g_launches = 0;
+  if (E < 1 || E > 256) return MOE_ERR_INVALID_ARG;
+  if (null_any({sums, aux_loss, z_loss})) return MOE_ERR_INVALID_ARG;
+  ++g_launches;
+  return cuda_status(launch_losses_from_sums(sums, E, aux_loss, z_loss, stream));
+}
+
 moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream) {
   NvtxRange nvtx_range("moe_permute");

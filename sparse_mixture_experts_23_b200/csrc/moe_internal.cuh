@@ -152,6 +152,9 @@ cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, 
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
 cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);
+cudaError_t launch_loss_sums(const float* loss_part, const int32_t* cnt_pre, int nblk, int E, int T, float* sums,
+                             cudaStream_t st);
+cudaError_t launch_losses_from_sums(const float* sums, int E, float* aux, float* z, cudaStream_t st);
 cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_gate_logits_sm100(const void* x, const void* Wg, const void* bg, int T, int H, int E, float* logits,
                                      int32_t* status, long long wait_limit, int num_sms, cudaStream_t st);

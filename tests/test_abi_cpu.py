@@ -249,3 +249,22 @@ def test_min_capacity_field(lib):
     s.min_capacity = -1
     assert moe.moe_capacity(s) == -2 and moe.moe_workspace_size(s) == 0
     assert moe.moe_forward(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_loss_sum_entry_points_validate_before_launch(lib):
+    s = _shape()
+    need = moe.moe_workspace_size(s)
+    E = s.E
+    # moe_loss_sums: null or misaligned sums, missing or short workspace, bad shape
+    assert moe.moe_loss_sums(s, FAKE, need, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_loss_sums(s, FAKE, need, FAKE + 2) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_loss_sums(s, 0, need, FAKE) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_loss_sums(s, FAKE, need - 1, FAKE) == moe.MOE_ERR_WORKSPACE
+    assert moe.moe_loss_sums(_shape(k=5), FAKE, need, FAKE) == moe.MOE_ERR_INVALID_ARG
+    # moe_losses_from_sums: expert count outside [1, 256], null pointers
+    for bad_e in (0, -1, 257):
+        assert moe.moe_losses_from_sums(bad_e, FAKE, FAKE, FAKE) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_losses_from_sums(E, 0, FAKE, FAKE) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_losses_from_sums(E, FAKE, 0, FAKE) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_losses_from_sums(E, FAKE, FAKE, 0) == moe.MOE_ERR_INVALID_ARG
+    assert moe.loss_sums_size(E) == 2 * E + 2
