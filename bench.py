@@ -522,7 +522,7 @@ def main():
     ap.add_argument("--config", default="mixtral", choices=list(synth.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-train", action="store_true", help="skip the training-step (forward + backward) timing")
-    ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle time for cpu_baseline")
+    ap.add_argument("--cpu-budget", type=float, default=30.0, help="seconds of oracle time for cpu_baseline")
     for dim in ("T", "H", "E", "k", "F"):
         ap.add_argument(f"--{dim}", type=int, default=None, help=f"override {dim} of the workload (profiling)")
     args = ap.parse_args()
