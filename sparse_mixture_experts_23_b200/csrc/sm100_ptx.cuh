@@ -214,11 +214,9 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, u
 // arrive (once the pair's prior MMAs complete) on the barrier at this offset in both CTAs of the pair
 __device__ __forceinline__ void mma_commit_both(uint32_t bar) {
   const uint16_t both = 3;
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster"
-      ".multicast::cluster.b64 [%0], %1;\n" ::"r"(bar),
-      "h"(both)
-      : "memory");
+  // (an MMA-completion arrive, not a copy: no data moves between the CTAs here)
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n"
+               ::"r"(bar), "h"(both) : "memory");
 }
 // arrive (once the pair's prior MMAs complete) on the barrier at cluster address `bar`
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
