@@ -1,5 +1,6 @@
 /*
- * moe.h -- C ABI of the B200 (sm_100a) sparse top-k Mixture-of-Experts layer forward pass.
+ * moe.h -- C ABI of the B200 (sm_100a) sparse top-k Mixture-of-Experts layer: its forward pass,
+ * its backward pass, and its losses over a batch split across data-parallel replicas.
  *
  * The layer (web page "MoE Training: Mixture of Experts", Quick Start "Basic MoE Architecture",
  * class MoELayer; Core Concepts 2-4; Advanced Patterns "Mixtral 8x7B Architecture") maps
@@ -17,6 +18,10 @@
  *                                                          "output[mask] += score * output";
  *                                                          Mixtral block index_add_)
  *   moe_forward     the four chained on one stream (fused combine)
+ *
+ * Around them: moe_forward_host (the same pass on host buffers, copies included), moe_route_noalloc
+ * (the router without a workspace), moe_forward_train + moe_backward (every gradient of the layer),
+ * moe_loss_sums + moe_losses_from_sums (the losses of a batch spread over replicas).
  *
  * Two routing rules (moe_shape_t.routing): token choice, where every token takes its top-k experts
  * (Quick Start; Core Concepts 2 top-1 / top-2), and expert choice, where every expert takes its
