@@ -1,0 +1,67 @@
+"""Host-side pieces of bench.py that the JSON line depends on, checked on the CPU: the whole-job
+rate, the workload description, and the rule that reports the captured DRAM traffic only while
+the GEMM sources still match the ones it was captured on."""
+import hashlib
+import json
+import math
+import os
+
+import pytest
+
+import bench
+import synth
+
+
+def test_aggregate_rate_counts_every_rank():
+    assert bench.aggregate_rate(1, 4096, 10, 20.0) == pytest.approx(4096 * 10 / 0.020)
+    assert bench.aggregate_rate(8, 4096, 10, 20.0) == pytest.approx(8 * 4096 * 10 / 0.020)
+
+
+def test_max_over_ranks_single_process():
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_workload_config_names_the_shape():
+    w = bench.workload_config(synth.CONFIGS["mixtral"])
+    for part in ("T=4096", "H=4096", "E=8", "k=2", "F=14336", "dropless", "GELU"):
+        assert part in w
+    assert "CF=1.25" in bench.workload_config(synth.CONFIGS["switch"])
+
+
+def test_alg_flops_and_bytes_of_the_headline_workload():
+    cfg = synth.CONFIGS["mixtral"]
+    kept = cfg.T * cfg.k
+    assert bench.alg_flops(cfg, kept) == pytest.approx(4.0 * cfg.H * cfg.F * kept + 2.0 * cfg.T * cfg.H * cfg.E)
+    # every expert's W1 and W2 (bf16) dominate the algorithmic bytes
+    assert bench.alg_bytes(cfg, cfg.E) > 2 * cfg.E * cfg.H * cfg.F * 2
+
+
+def test_captured_traffic_follows_the_source_hashes(tmp_path, monkeypatch):
+    src = tmp_path / "kernel.cu"
+    src.write_text("// kernel v1\n")
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    entry = {"grouped_gemm_bytes_per_launch": 123,
+             "sources_sha256": {"kernel.cu": hashlib.sha256(b"// kernel v1\n").hexdigest()}}
+    (prof / "traffic.json").write_text(json.dumps({"note": "test", "w": entry}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.captured_traffic("w") == 123
+    assert bench.captured_traffic("other") is None
+    src.write_text("// kernel v2\n")  # the kernel changed since the capture
+    assert bench.captured_traffic("w") is None
+    os.remove(src)
+    assert bench.captured_traffic("w") is None
+
+
+def test_committed_traffic_record_is_consistent():
+    """The committed record names existing sources and a per-launch byte count near the
+    algorithmic bytes of one moe_expert_ffn call (between 1x and 2x)."""
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))["mixtral"]
+    for rel in rec["sources_sha256"]:
+        assert os.path.exists(os.path.join(bench.ROOT, rel)), rel
+    cfg = synth.CONFIGS["mixtral"]
+    rows = cfg.T * cfg.k
+    alg = 2 * cfg.E * cfg.H * cfg.F * 2 + rows * cfg.H * 2 + 2 * rows * cfg.F * 2 + 2 * cfg.T * cfg.H * 4
+    assert alg <= rec["grouped_gemm_bytes_per_launch"] <= 2 * alg
+    assert math.isclose(sum(v["dram_read"] + v["dram_write"] for v in rec["per_kernel"].values()),
+                        rec["grouped_gemm_bytes_per_launch"])
