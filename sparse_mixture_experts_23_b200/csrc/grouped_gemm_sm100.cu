@@ -58,7 +58,7 @@ __host__ __device__ constexpr bool epi_dgrad(int epi) { return epi == EPI_DGRAD_
 
 template <int BN>
 struct Cfg {
-  static constexpr int kStages = BN == 256 ? 3 : (BN == 128 ? 5 : 6);
+  static constexpr int kStages = BN == 256 ? 4 : (BN == 128 ? 6 : 8);  // as deep as shared memory allows
   static constexpr int kABytes = BM * BK * 2;
   static constexpr int kBBytes = BK * BN * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
