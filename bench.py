@@ -56,6 +56,35 @@ def alg_bytes(cfg: synth.LayerConfig, touched_experts: int) -> float:
     return w + cfg.T * cfg.H * es + cfg.T * cfg.H * 4 + cfg.H * cfg.E * es
 
 
+def ffn_alg_bytes(cfg: synth.LayerConfig, kept: int, touched_experts: int) -> float:
+    """Algorithmic DRAM bytes of one moe_expert_ffn call: the touched experts' W1, W2 (and biases)
+    once, x_perm read, h written and read back (storage dtype), out read and written (fp32)."""
+    es = 2 if cfg.dtype == "bf16" else 4
+    w = touched_experts * (2 * cfg.H * cfg.F + (cfg.F + cfg.H if cfg.bias else 0)) * es
+    return w + kept * cfg.H * es + 2 * kept * cfg.F * es + 2 * cfg.T * cfg.H * 4
+
+
+def ffn_roofline(cfg: synth.LayerConfig, kept: int, touched_experts: int, ms_ffn: float, peaks: dict) -> dict:
+    """Roofline object of the dominant kernel pair (one moe_expert_ffn call): tensor-bound when its
+    FLOPs take longer at the sustained bf16 peak than its algorithmic bytes at the copy bandwidth,
+    else HBM-bound (weight streaming: decode, the Switch shape)."""
+    flops = 4.0 * cfg.H * cfg.F * kept
+    nbytes = ffn_alg_bytes(cfg, kept, touched_experts)
+    t_tensor = flops / (peaks["bf16_tflops_sustained"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    sec = ms_ffn / 1000.0
+    if t_tensor >= t_hbm:
+        a, pk = flops / sec / 1e12, peaks["bf16_tflops_sustained"]
+        r = {"bound": "tensor", "achieved": a, "peak": pk, "unit": "TFLOP/s", "frac": a / pk,
+             "peak_source": f"{peaks['source']} bf16 sustained"}
+    else:
+        a, pk = nbytes / sec / 1e9, peaks["hbm_gbs"]
+        r = {"bound": "hbm", "achieved": a, "peak": pk, "unit": "GB/s", "frac": a / pk,
+             "peak_source": f"{peaks['source']} HBM copy"}
+    r["algorithmic"] = {"flops": flops, "bytes": nbytes}
+    return r
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -459,7 +488,7 @@ def run_ours_impl(args, cfg):
         tkept = int(tbuf.expert_counts.sum().item())
         bwd_flops = 8.0 * cfg.H * cfg.F * tkept + 4.0 * cfg.T * cfg.H * cfg.E
         train = {"fwd_train_ms": ms_fwd_train, "bwd_ms": ms_bwd, "step_ms": ms_fwd_train + ms_bwd,
-                 "tokens_per_s": world * cfg.T / ((ms_fwd_train + ms_bwd) / 1000.0),
+                 "tokens_per_s": cfg.T / ((ms_fwd_train + ms_bwd) / 1000.0),  # rank 0's replica
                  "bwd_tflops": bwd_flops / (ms_bwd / 1000.0) / 1e12,
                  "bwd_frac_sustained": bwd_flops / (ms_bwd / 1000.0) / 1e12 / peak,
                  "bwd_launches": bwd_launches,
@@ -480,10 +509,8 @@ def run_ours_impl(args, cfg):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2: the expert weights (%.2f GB) stream every step" %
                          (cfg.E * 2 * cfg.H * cfg.F * es / 1e9)},
-        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
-                     "traffic": traffic,
-                     "kernel": "grouped GEMM pair (GEMM1 bias+GELU, GEMM2 scale+combine), one moe_expert_ffn call",
-                     "peak_source": f"{peaks['source']} bf16 sustained"},
+        "roofline": dict(ffn_roofline(cfg, kept, touched, ms_ffn, peaks), traffic=traffic,
+                         kernel="grouped GEMMs (GEMM1 bias+act, GEMM2 scale+combine), one moe_expert_ffn call"),
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": cfg.T * cfg.H * es,
                 "d2h_bytes_per_step": cfg.T * cfg.H * 4, "api": "moe_forward_host",

@@ -65,3 +65,22 @@ def test_committed_traffic_record_is_consistent():
     assert alg <= rec["grouped_gemm_bytes_per_launch"] <= 2 * alg
     assert math.isclose(sum(v["dram_read"] + v["dram_write"] for v in rec["per_kernel"].values()),
                         rec["grouped_gemm_bytes_per_launch"])
+
+
+PEAKS = {"hbm_gbs": 6548.8, "bf16_tflops": 1661.1, "bf16_tflops_sustained": 1383.9, "source": "measured"}
+
+
+def test_roofline_bound_follows_arithmetic_intensity():
+    mix = synth.CONFIGS["mixtral"]
+    r = bench.ffn_roofline(mix, mix.T * mix.k, mix.E, 1.75, PEAKS)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(4.0 * mix.H * mix.F * mix.T * mix.k / 1.75e-3 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops_sustained"])
+    dec = synth.CONFIGS["decode"]
+    r = bench.ffn_roofline(dec, dec.T * dec.k, dec.E, 0.35, PEAKS)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    weights = dec.E * (2 * dec.H * dec.F + dec.F + dec.H) * 2
+    assert weights < r["algorithmic"]["bytes"] < 1.05 * weights  # weight streaming dominates
+    assert r["frac"] == pytest.approx(r["algorithmic"]["bytes"] / 0.35e-3 / 1e9 / PEAKS["hbm_gbs"])
+    sw = synth.CONFIGS["switch"]
+    assert bench.ffn_roofline(sw, 8104, sw.E, 0.56, PEAKS)["bound"] == "hbm"
