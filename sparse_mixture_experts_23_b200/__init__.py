@@ -1,4 +1,5 @@
-"""Python binding of the B200 sparse top-k MoE forward library (``libmoe.so``, C ABI in include/moe.h).
+"""Python binding of the B200 sparse top-k MoE layer library (``libmoe.so``, C ABI in include/moe.h):
+the forward pass, the backward pass and the losses across data-parallel replicas.
 
 This module only marshals arguments: it mirrors the C structs with ctypes and calls the entry
 points by the same names.  Every step of the layer runs in the CUDA kernels of ``libmoe.so``;
