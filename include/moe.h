@@ -205,8 +205,10 @@ MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, voi
  * before anything is launched.  No device memory is allocated or freed, by this call or by any
  * routine it calls.  The first call on a device looks up the array's device address for that
  * device (cudaGetSymbolAddress, with the device current); make that first call before any stream
- * capture.  Every call, on every stream, shares the one array and leaves the last call's contents
- * in it: calls that overlap on the GPU race, so serialise them (one stream, or events).
+ * capture.  Later calls made outside stream capture look the address up again, so a context that
+ * was reset and rebuilt (cudaDeviceReset) is served its new address.  Every call, on every stream,
+ * shares the one array and leaves the last call's contents in it: calls that overlap on the GPU
+ * race, so serialise them (one stream, or events).  2 launches (1 when T = 0); one NVTX range.
  * Token choice only: an expert-choice shape returns MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream);
 
@@ -333,6 +335,17 @@ MOE_API moe_status_t moe_get_device_status(void* ws, cudaStream_t stream);
 /* Bound on device-side waits, in GPU clock cycles (default 2e9, about one second).  Applies to
  * launches made after the call.  Values <= 0 restore the default. */
 MOE_API void moe_set_wait_limit(long long cycles);
+
+/* Kernel-selection switches for side-by-side comparisons of the kernels; normal use needs none.
+ *   MOE_KERNEL_NO_CTA_PAIR  single-CTA 128-row grouped-GEMM tiles everywhere, instead of the CTA-pair
+ *                           256 x 256 tiles the long-segment shapes use (forward and backward GEMMs)
+ *   MOE_KERNEL_NO_TC_GATE   the CUDA-core gate kernels instead of the tensor-core ones (mma.sync for
+ *                           8/16/32 experts, the tcgen05 GEMM for multiples of 64)
+ * Default 0.  Process-wide; applies to launches made after the call, from any host thread.  Results
+ * stay within the same tolerances of the definition either way; unknown bits are ignored. */
+typedef enum { MOE_KERNEL_DEFAULT = 0, MOE_KERNEL_NO_CTA_PAIR = 1, MOE_KERNEL_NO_TC_GATE = 2 } moe_kernel_flags_t;
+MOE_API void moe_set_kernel_options(int flags);
+MOE_API int moe_get_kernel_options(void);
 
 /* Launches one block that waits on a pipeline barrier nothing will ever complete, with the
  * current wait bound; it must come back with the error word set.  For testing the timeout path. */

@@ -405,7 +405,7 @@ def backward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_a
     E, _, F = W1.shape
     r = route(x, Wg, bg, k, dtype)
     idx = r.topk_idx if topk_idx is None else np.asarray(topk_idx, np.int32)
-    w = r.topk_w if topk_idx is None else _renorm_weights(r.p, idx)
+    w = r.topk_w if topk_idx is None else renorm_weights(r.p, idx)
     d = dispatch(idx, E, cf)
     drp = d.dropped if dropped is None else np.asarray(dropped, np.uint8)
     dout = _c(dout, np.float64)
@@ -439,9 +439,28 @@ def backward(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_a
     return Grads(dx + dxr, dWg, dbg, dW1, db1, dW2, db2, dw, dl)
 
 
-def _renorm_weights(p, idx):
+def renorm_weights(p, idx):
+    """w[t,s] = p[t, idx[t,s]] / sum_s' p[t, idx[t,s']]: the Quick Start's division of the selected
+    softmax scores by their sum, for a given selection (not necessarily the top-k of p).  The
+    weights are pre-drop values: a dropped slot keeps its weight and contributes nothing."""
     sel = np.take_along_axis(np.asarray(p, np.float64), np.asarray(idx, np.int64), axis=1)
     return sel / sel.sum(axis=1, keepdims=True)
+
+
+def loss_of_given(x, Wg, bg, W1, b1, W2, b2, topk_idx, dropped, dtype: str, dout, d_aux: float, d_z: float,
+                  act: str = "gelu") -> float:
+    """L = sum(dout * out) + d_aux * aux + d_z * z with the routing held fixed at (topk_idx, dropped):
+    p and lse from the gate as usual, the weights renormalised over the given selection, out from
+    the kept slots only, aux from the given selection's pre-drop counts.  This is the function whose
+    gradient backward(..., topk_idx=, dropped=) returns."""
+    idx = np.asarray(topk_idx, np.int32)
+    k = idx.shape[1]
+    r = route(x, Wg, bg, k, dtype)
+    w = renorm_weights(r.p, idx)
+    aux, z = losses(r.p, r.lse, idx)
+    T = x.shape[0]
+    out = forward_tokens(x, W1, b1, W2, b2, idx, w, dropped, np.arange(T, dtype=np.int32), dtype, act=act)
+    return float(np.sum(np.asarray(dout, np.float64) * out)) + d_aux * aux + d_z * z
 
 
 def loss_of(x, Wg, bg, W1, b1, W2, b2, k: int, cf: float, dtype: str, dout, d_aux: float, d_z: float,

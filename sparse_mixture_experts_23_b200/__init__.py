@@ -28,7 +28,9 @@ ENTRY_POINTS = (
     "moe_forward", "moe_forward_host", "moe_get_device_status", "moe_set_wait_limit", "moe_debug_timeout_probe",
     "moe_last_launch_count", "moe_status_string", "moe_route_noalloc", "moe_capacity",
     "moe_train_workspace_size", "moe_forward_train", "moe_backward", "moe_loss_sums", "moe_losses_from_sums",
+    "moe_set_kernel_options", "moe_get_kernel_options",
 )
+MOE_KERNEL_DEFAULT, MOE_KERNEL_NO_CTA_PAIR, MOE_KERNEL_NO_TC_GATE = 0, 1, 2
 
 
 class MoEError(RuntimeError):
@@ -101,6 +103,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_get_device_status.restype = st
     lib.moe_set_wait_limit.argtypes = [ctypes.c_longlong]
     lib.moe_set_wait_limit.restype = None
+    lib.moe_set_kernel_options.argtypes = [ctypes.c_int]
+    lib.moe_set_kernel_options.restype = None
+    lib.moe_get_kernel_options.argtypes = []
+    lib.moe_get_kernel_options.restype = ctypes.c_int
     lib.moe_debug_timeout_probe.argtypes = [vp, sz, vp]
     lib.moe_debug_timeout_probe.restype = st
     lib.moe_last_launch_count.argtypes = []
@@ -224,6 +230,14 @@ def moe_get_device_status(ws, stream=0) -> int:
 
 def moe_set_wait_limit(cycles: int) -> None:
     load_library().moe_set_wait_limit(int(cycles))
+
+
+def moe_set_kernel_options(flags: int) -> None:
+    load_library().moe_set_kernel_options(int(flags))
+
+
+def moe_get_kernel_options() -> int:
+    return load_library().moe_get_kernel_options()
 
 
 def moe_debug_timeout_probe(ws, ws_bytes, stream=0) -> int:

@@ -9,15 +9,16 @@
 //   GEMM2 (EPI_COMBINE):  out[t, n] += w(t,s) * ( sum_k h[r,k] W2[e,k,n] + b2[e,n] ),  t,s = row r's
 //   GEMM2 (EPI_STORE_Y):  y[r, n]   = sum_k h[r,k] W2[e,k,n] + b2[e,n]
 //
-// Design (one persistent CTA per SM, 320 threads):
+// Design (one persistent CTA per SM, 64 + 32 * kEpiWarps threads: 192 with the default 4 epilogue warps):
 //   warp 0      TMA producer: A tile [128 rows x 64 k] (K-major, 128B swizzle) and B tile
 //               [64 k x BN n] (weights are stored n-contiguous, i.e. MN-major, 128B swizzle, loaded
 //               as BN/64 boxes of 64x64) into a kStages-deep shared-memory ring.
 //   warp 1      allocates 2*BN TMEM columns (two fp32 accumulators), one elected lane issues
 //               tcgen05.mma kind::f16 (M=128, N=BN, K=16, bf16 x bf16 -> fp32) and tcgen05.commit
 //               to release smem stages and to hand a finished accumulator to the epilogue.
-//   warps 2..9  epilogue: tcgen05.ld 32 lanes x 32 columns per step (each thread owns one row; two
-//               warps share each TMEM lane quarter and split the tile's columns),
+//   warps 2..   epilogue (kEpiWarps = 4: warps 2..5, one per TMEM lane quarter; 8: two warps share
+//               each quarter and split the tile's columns): tcgen05.ld 32 lanes x 32 columns per step
+//               (each thread owns one row),
 //               fused bias + GELU -> bf16 store, or bias + gate-weight scale + vector fp32 red.add
 //               into out (at most k adds per element, so k <= 2 is order independent).
 // Tiles run expert-major, then n-tile, then m-tile, so the CTAs in flight share one expert's
@@ -1324,15 +1325,9 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 // CTA-pair tiles are used for N divisible by 256 and K by 128 when segments are long enough;
-// MOE_GEMM_PAIR=0 in the environment selects the single-CTA kernel everywhere (for comparison).
-bool pair_mode_enabled() {
-  static int mode = -1;
-  if (mode < 0) {
-    const char* v = getenv("MOE_GEMM_PAIR");
-    mode = (v != nullptr && v[0] == '0') ? 0 : 1;
-  }
-  return mode == 1;
-}
+// moe_set_kernel_options(MOE_KERNEL_NO_CTA_PAIR) selects the single-CTA kernel everywhere (for
+// comparisons).
+bool pair_mode_enabled() { return (kernel_options() & MOE_KERNEL_NO_CTA_PAIR) == 0; }
 
 // A operand: [rows, K] bf16 row-major; box = 64 k x 128 rows
 bool make_map_a(CUtensorMap* m, const void* base, int rows, int K) {

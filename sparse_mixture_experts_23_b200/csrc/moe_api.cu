@@ -116,16 +116,24 @@ namespace {
 
 thread_local int g_launches = 0;
 
-// One NVTX range per entry-point call ("moe_route", "moe_forward", ...), so that a timeline shows the
-// stages of a layer call around its kernels.
-struct NvtxRange {
-  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-  ~NvtxRange() { nvtxRangePop(); }
-};
 // bound on device-side waits for launches made after moe_set_wait_limit (any host thread may set it)
 std::atomic<long long> g_wait_limit{2000000000LL};
+// kernel-selection flags of moe_set_kernel_options (any host thread may set them)
+std::atomic<int> g_kernel_options{0};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+namespace moe {
+
+int& launch_count() { return g_launches; }
+int kernel_options() { return g_kernel_options.load(std::memory_order_relaxed); }
+
+// One NVTX range per entry-point call ("moe_route", "moe_forward", ...), so that a timeline shows the
+// stages of a layer call around its kernels.
+NvtxRange::NvtxRange(const char* name) { nvtxRangePushA(name); }
+NvtxRange::~NvtxRange() { nvtxRangePop(); }
 
 moe_status_t check_shape(const moe_shape_t* s) {
   if (s == nullptr) return MOE_ERR_INVALID_ARG;
@@ -144,6 +152,10 @@ moe_status_t check_shape(const moe_shape_t* s) {
   if (rows * widest >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
+
+}  // namespace moe
+
+namespace {
 
 long long capacity_of(const moe_shape_t* s) {
   if (isinf(s->capacity_factor)) return -1;
@@ -762,6 +774,12 @@ moe_status_t moe_get_device_status(void* ws, cudaStream_t stream) {
 }
 
 void moe_set_wait_limit(long long cycles) { g_wait_limit = cycles > 0 ? cycles : 2000000000LL; }
+
+void moe_set_kernel_options(int flags) {
+  g_kernel_options.store(flags & (MOE_KERNEL_NO_CTA_PAIR | MOE_KERNEL_NO_TC_GATE), std::memory_order_relaxed);
+}
+
+int moe_get_kernel_options(void) { return g_kernel_options.load(std::memory_order_relaxed); }
 
 moe_status_t moe_debug_timeout_probe(void* ws, size_t ws_bytes, cudaStream_t stream) {
   g_launches = 0;

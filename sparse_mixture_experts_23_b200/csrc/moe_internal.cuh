@@ -142,6 +142,21 @@ struct FfnArgs {
   int num_sms;
 };
 
+// ---- host-side helpers shared by the entry points (defined in moe_api.cu) ----
+// Argument rules every entry point applies to a shape (the MOE_ERR_* codes of include/moe.h).
+moe_status_t check_shape(const moe_shape_t* s);
+// This host thread's count of kernels launched by the current moe_* call (moe_last_launch_count).
+int& launch_count();
+// Flags of moe_set_kernel_options (MOE_KERNEL_*), read at each launch.
+int kernel_options();
+// One NVTX range per entry-point call, named after the entry point.
+struct NvtxRange {
+  explicit NvtxRange(const char* name);
+  ~NvtxRange();
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 // Raises a kernel's dynamic shared-memory limit to at least `bytes` on the current device; the
 // driver call is made once per (kernel, device) and size, so repeated launches cost nothing.
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);

@@ -9,8 +9,11 @@
 //
 // The array is a file-scope __device__ object, so every GPU that loads the library holds it
 // until the process exits.  Host code must not use the array's name as a device address: it only
-// names a host-side stand-in.  The device address is looked up once per device, with that device
-// current, by cudaGetSymbolAddress, and handed to the kernels as a plain pointer.
+// names a host-side stand-in.  The device address comes from cudaGetSymbolAddress with the device
+// current and is handed to the kernels as a plain pointer.  It is looked up again on every call
+// made outside stream capture, so a context torn down and rebuilt (cudaDeviceReset) gets the
+// array's new address; a call made while its stream is capturing uses the address of the last
+// uncaptured call on that device, and fails if there was none.
 #include <mutex>
 
 #include "moe_internal.cuh"
@@ -24,18 +27,24 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
-// Device address of g_route_scratch on the current device; looked up on first use per device.
-cudaError_t scratch_for_current_device(void** out) {
+// Device address of g_route_scratch on the current device: looked up now when `stream` is not
+// capturing (and remembered for the device), else the remembered one.
+cudaError_t scratch_for_current_device(cudaStream_t stream, void** out) {
   int dev = 0;
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  err = cudaStreamIsCapturing(stream, &cap);
+  if (err != cudaSuccess) return err;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* p = nullptr;
     err = cudaGetSymbolAddress(&p, g_route_scratch);
     if (err != cudaSuccess) return err;
     g_scratch_ptr[dev] = p;
+  } else if (g_scratch_ptr[dev] == nullptr) {
+    return cudaErrorStreamCaptureUnsupported;  // no uncaptured call on this device yet
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;
@@ -59,32 +68,29 @@ size_t scratch_bytes(const moe_shape_t* s, size_t* hist_off, size_t* cnt_off) {
 extern "C" {
 
 moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream) {
-  if (shape == nullptr || io == nullptr) return MOE_ERR_INVALID_ARG;
-  // same argument rules as moe_route, checked through a zero-size workspace probe of the shape
-  if (moe_workspace_size(shape) == 0) {
-    if (shape->T < 0 || shape->H <= 0 || shape->E <= 0 || shape->F <= 0 || shape->k <= 0 || shape->k > shape->E ||
-        shape->k > 8 || shape->E > 256 || !(shape->capacity_factor > 0.0) ||
-        (shape->dtype != MOE_DTYPE_F32 && shape->dtype != MOE_DTYPE_BF16) ||
-        (shape->activation != MOE_ACT_GELU && shape->activation != MOE_ACT_SILU) ||
-        (shape->routing != MOE_ROUTING_TOKEN_CHOICE && shape->routing != MOE_ROUTING_EXPERT_CHOICE))
-      return MOE_ERR_INVALID_ARG;
-    return MOE_ERR_UNSUPPORTED;
-  }
+  moe::NvtxRange nvtx_range("moe_route_noalloc");
+  int& launches = moe::launch_count();
+  launches = 0;
+  moe_status_t st = moe::check_shape(shape);  // the same argument rules as moe_route
+  if (st != MOE_OK) return st;
+  if (io == nullptr) return MOE_ERR_INVALID_ARG;
   if (shape->routing != MOE_ROUTING_TOKEN_CHOICE) return MOE_ERR_UNSUPPORTED;  // the selection needs a workspace
   if (io->aux_loss == nullptr || io->z_loss == nullptr) return MOE_ERR_INVALID_ARG;
   size_t hist_off = 0, cnt_off = 0;
   if (scratch_bytes(shape, &hist_off, &cnt_off) > kScratchBytes)
     return MOE_ERR_WORKSPACE;  // shape too large for the built-in scratch
-  if (shape->T == 0) return moe::launch_zero_outputs(nullptr, 0, io->aux_loss, io->z_loss, stream) == cudaSuccess
-                                ? MOE_OK
-                                : MOE_ERR_CUDA;
+  if (shape->T == 0) {
+    ++launches;
+    return moe::launch_zero_outputs(nullptr, 0, io->aux_loss, io->z_loss, stream) == cudaSuccess ? MOE_OK
+                                                                                                  : MOE_ERR_CUDA;
+  }
   if (io->x == nullptr || io->Wg == nullptr || io->topk_idx == nullptr || io->topk_w == nullptr)
     return MOE_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(io->x) & 15u) || (reinterpret_cast<uintptr_t>(io->Wg) & 15u))
     return MOE_ERR_INVALID_ARG;
 
   void* base = nullptr;
-  if (scratch_for_current_device(&base) != cudaSuccess) return MOE_ERR_CUDA;
+  if (scratch_for_current_device(stream, &base) != cudaSuccess) return MOE_ERR_CUDA;
   const int nblk = (shape->T + moe::kChunk - 1) / moe::kChunk;
   float* loss_part = static_cast<float*>(base);
   int32_t* chunk_hist = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + hist_off);
@@ -104,7 +110,7 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   r.topk_w = io->topk_w;
   r.loss_part = loss_part;
   r.chunk_hist = chunk_hist;
-  int launches = 0;  // no gate scratch here, so always the one-kernel router
+  // no gate scratch here, so always the one-kernel router
   if (moe::launch_router(r, shape->dtype, stream, &launches) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::ReduceArgs a{};
@@ -123,6 +129,7 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   a.z_loss = io->z_loss;
   a.do_losses = 1;
   a.do_dispatch = 0;
+  ++launches;
   return moe::launch_reduce(a, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -1074,15 +1074,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 
 }  // namespace
 
-// MOE_ROUTER_MMA=0 in the environment selects the CUDA-core routers instead (for comparison).
-bool router_mma_disabled() {
-  static int v = -1;
-  if (v < 0) {
-    const char* e = getenv("MOE_ROUTER_MMA");
-    v = (e != nullptr && e[0] == '0') ? 1 : 0;
-  }
-  return v == 1;
-}
+// moe_set_kernel_options(MOE_KERNEL_NO_TC_GATE) selects the CUDA-core routers (for comparisons).
+bool router_mma_disabled() { return (kernel_options() & MOE_KERNEL_NO_TC_GATE) != 0; }
 
 template <int EP>
 cudaError_t launch_stream(const RouterArgs& a, int nblk, cudaStream_t st) {

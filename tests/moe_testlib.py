@@ -101,6 +101,41 @@ def sample_tokens(T: int, n: int, seed: int = 0) -> np.ndarray:
     return np.unique(np.concatenate([fixed, rest])).astype(np.int32)
 
 
+def stratified_rows(offsets, tile: int = 128, seed: int = 0) -> np.ndarray:
+    """Rows of the permuted layout chosen so that every GEMM tile of every expert segment is checked:
+    the first and last row of each non-empty segment, one random row in each 128-row block (every
+    128-row and 256-row m-tile starts on a block boundary inside its segment), and every row of each
+    segment's last block (the expert's tail tile: a half pair tile when it holds <= 128 rows)."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    offsets = np.asarray(offsets)
+    for e in range(len(offsets) - 1):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if b <= a:
+            continue
+        rows += [a, b - 1]
+        rows += [int(rng.integers(m0, min(b, m0 + tile))) for m0 in range(a, b, tile)]
+        rows += range(a + ((b - a - 1) // tile) * tile, b)
+    return np.unique(np.asarray(rows, np.int64))
+
+
+def stratified_tokens(offsets, row_token, tile: int = 128, seed: int = 0) -> np.ndarray:
+    """Tokens owning the stratified rows (each token's whole output row, every slot, is then checked)."""
+    rows = stratified_rows(offsets, tile, seed)
+    return np.unique(np.asarray(row_token)[rows]).astype(np.int32)
+
+
+def stratified_columns(n: int, block: int = 256, extra_last: int = 8, seed: int = 0) -> np.ndarray:
+    """One random column in every `block`-wide block of n columns (every N tile of the GEMMs that produce
+    or consume them), plus `extra_last` more from the last block, whole or partial."""
+    rng = np.random.default_rng(seed)
+    cols = [int(rng.integers(c0, min(n, c0 + block))) for c0 in range(0, n, block)]
+    last0 = ((n - 1) // block) * block
+    cols += rng.choice(np.arange(last0, n), size=min(extra_last, n - last0), replace=False).tolist()
+    cols.append(n - 1)
+    return np.unique(np.asarray(cols, np.int32))
+
+
 def fro_rel(a: np.ndarray, ref: np.ndarray) -> float:
     den = float(np.linalg.norm(ref))
     num = float(np.linalg.norm(a - ref))

@@ -249,6 +249,22 @@ def test_min_capacity_field(lib):
     s.min_capacity = -1
     assert moe.moe_capacity(s) == -2 and moe.moe_workspace_size(s) == 0
     assert moe.moe_forward(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG
+    # the no-workspace router applies the same shape rules as moe_route, and launches nothing
+    s.routing = moe.MOE_ROUTING_TOKEN_CHOICE
+    assert moe.moe_route(s, _io(), FAKE, 1 << 40) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_route_noalloc(s, _io()) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_last_launch_count() == 0
+
+
+def test_kernel_options_round_trip(lib):
+    """moe_set_kernel_options keeps the known flags, drops unknown bits, and 0 restores the default."""
+    assert moe.moe_get_kernel_options() == moe.MOE_KERNEL_DEFAULT
+    try:
+        moe.moe_set_kernel_options(moe.MOE_KERNEL_NO_CTA_PAIR | moe.MOE_KERNEL_NO_TC_GATE | 0x40)
+        assert moe.moe_get_kernel_options() == moe.MOE_KERNEL_NO_CTA_PAIR | moe.MOE_KERNEL_NO_TC_GATE
+    finally:
+        moe.moe_set_kernel_options(moe.MOE_KERNEL_DEFAULT)
+    assert moe.moe_get_kernel_options() == 0
 
 
 def test_loss_sum_entry_points_validate_before_launch(lib):

@@ -6,6 +6,8 @@ import json
 import math
 import os
 
+import numpy as np
+
 import pytest
 
 import bench
@@ -75,7 +77,14 @@ def test_roofline_bound_follows_arithmetic_intensity():
     r = bench.ffn_roofline(mix, mix.T * mix.k, mix.E, 1.75, PEAKS)
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(4.0 * mix.H * mix.F * mix.T * mix.k / 1.75e-3 / 1e12)
-    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops_sustained"])
+    # the call is timed alone: the burst peak is the denominator, the sustained fraction rides along
+    assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
+    assert r["frac_of_sustained"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops_sustained"])
+    assert "tensor_flop_per_sm_clk" not in r
+    clk = bench.ffn_roofline(mix, mix.T * mix.k, mix.E, 1.75, PEAKS, {"sm_mhz": 1500.0}, 148)
+    per_clk = 4.0 * mix.H * mix.F * mix.T * mix.k / (1.75e-3 * 1500e6 * 148)
+    assert clk["tensor_flop_per_sm_clk"]["value"] == pytest.approx(per_clk)
+    assert clk["tensor_flop_per_sm_clk"]["of_nominal"] == pytest.approx(per_clk / 8192)
     dec = synth.CONFIGS["decode"]
     r = bench.ffn_roofline(dec, dec.T * dec.k, dec.E, 0.35, PEAKS)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
@@ -84,3 +93,32 @@ def test_roofline_bound_follows_arithmetic_intensity():
     assert r["frac"] == pytest.approx(r["algorithmic"]["bytes"] / 0.35e-3 / 1e9 / PEAKS["hbm_gbs"])
     sw = synth.CONFIGS["switch"]
     assert bench.ffn_roofline(sw, 8104, sw.E, 0.56, PEAKS)["bound"] == "hbm"
+
+
+def test_stratified_rows_cover_every_tile():
+    """The full-size parity rows: both ends of every segment, a row in every 128-row block of every
+    segment, and every row of each segment's last block; empty segments contribute nothing."""
+    from moe_testlib import stratified_columns, stratified_rows, stratified_tokens
+
+    counts = np.array([1000, 0, 1, 128, 129, 256, 300, 0])
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    rows = stratified_rows(offsets, seed=3)
+    for e, c in enumerate(counts):
+        a, b = offsets[e], offsets[e + 1]
+        mine = rows[(rows >= a) & (rows < b)]
+        if c == 0:
+            assert mine.size == 0
+            continue
+        assert a in mine and b - 1 in mine
+        for m0 in range(a, b, 128):
+            assert ((mine >= m0) & (mine < min(b, m0 + 128))).any()
+        tail0 = a + ((c - 1) // 128) * 128
+        assert set(range(tail0, b)) <= set(mine.tolist())
+    row_token = np.arange(offsets[-1])[::-1] % 700
+    toks = stratified_tokens(offsets, row_token, seed=3)
+    assert set(toks.tolist()) == set(row_token[rows].tolist())
+    cols = stratified_columns(14336, seed=1)
+    assert len(cols) >= 56 and cols.max() == 14335
+    for c0 in range(0, 14336, 256):
+        assert ((cols >= c0) & (cols < c0 + 256)).any()
+    assert ((cols >= 14080)).sum() >= 8

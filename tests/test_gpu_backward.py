@@ -6,9 +6,10 @@ gradient.  Tolerance, per gradient tensor: max|d| <= 4e-2 * RMS(ref) and a relat
 product carries two bf16 roundings; the oracle is fp64 throughout).
 
   small layers   every gradient in full: dx, dWg, dbg, dW1, db1, dW2, db2 and the per-slot dw
-  Mixtral shape  dx and dw on sampled tokens, dW1 / dW2 / db1 on sampled FFN columns of every
-                 expert, db2 in full, dWg / dbg in full from the oracle's router backward fed the
-                 GPU's dw (every token's dw would need every token's expert output)
+  Mixtral shape  dx and dw on tokens of every expert segment, dW1 / dW2 / db1 on one FFN column in
+                 every 256-column tile of every expert plus the last tile's, db2 in full, dWg / dbg
+                 in full from the oracle's router backward fed the GPU's dw (every token's dw
+                 would need every token's expert output)
 """
 import math
 
@@ -17,7 +18,7 @@ import pytest
 
 import oracle
 import synth
-from moe_testlib import TOL_BWD_FRO, TOL_BWD_MAX, fro_rel, rms_rel, sample_tokens, shape_of, upload
+from moe_testlib import TOL_BWD_FRO, TOL_BWD_MAX, fro_rel, rms_rel, shape_of, stratified_columns, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -72,13 +73,26 @@ def _run(cfg, dout):
 
 
 def _check(name, got, ref, per_expert: bool = False):
-    """max|d| <= 4e-2 RMS(ref) (per leading index when per_expert) and Frobenius <= 1e-2 overall."""
+    """max|d| <= 4e-2 RMS(ref) (per leading index when per_expert) and Frobenius <= 1e-2 overall.  The
+    error against one RMS over the whole tensor is printed beside the per-expert one."""
+    glob = rms_rel(got, ref)
     if per_expert:
         err = max(rms_rel(got[e], ref[e]) for e in range(ref.shape[0]) if np.any(ref[e]))
     else:
-        err = rms_rel(got, ref)
+        err = glob
     fro = fro_rel(got, ref)
-    print(f"  {name}: max {err:.3e} x RMS{' (per expert)' if per_expert else ''}, Frobenius {fro:.3e}")
+    print(f"  {name}: max {err:.3e} x RMS{' (per expert)' if per_expert else ''}, global-RMS {glob:.3e}, "
+          f"Frobenius {fro:.3e}")
+    assert err <= TOL_BWD_MAX and fro <= TOL_BWD_FRO, (name, err, fro)
+
+
+def _check_experts(name, gots, refs):
+    """The per-expert rule over per-expert arrays of different sizes (each expert's own column set)."""
+    err = max(rms_rel(g, r) for g, r in zip(gots, refs) if np.any(r))
+    cat_g = np.concatenate([np.ravel(g) for g in gots])
+    cat_r = np.concatenate([np.ravel(r) for r in refs])
+    glob, fro = rms_rel(cat_g, cat_r), fro_rel(cat_g, cat_r)
+    print(f"  {name}: max {err:.3e} x RMS (per expert), global-RMS {glob:.3e}, Frobenius {fro:.3e}")
     assert err <= TOL_BWD_MAX and fro <= TOL_BWD_FRO, (name, err, fro)
 
 
@@ -110,7 +124,26 @@ def test_backward_small_all_gradients(cfg):
     assert r["launches"] == (8 if cfg.bias else 7)
 
 
-def test_backward_mixtral_shape_sampled():
+def _slots_parallel(inp, cfg, pairs, dout, w):
+    """oracle.bwd_slot over (token, slot, expert) triples on a thread pool (the ctypes calls release the
+    GIL): returns {(t, s): (dx part, dw)}."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(p):
+        t, s, e = p
+        dxp, dws, _ = oracle.bwd_slot(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, t, e, dout[t], w[t, s], cfg.dtype, cfg.act)
+        return (t, s), (dxp, dws)
+
+    with ThreadPoolExecutor(max_workers=oracle.max_threads()) as ex:
+        return dict(ex.map(one, pairs))
+
+
+def test_backward_mixtral_shape_stratified():
+    """Mixtral shape, every expert covered.  dx and dw on the tokens of the first, last and a random row of
+    every expert segment; dW1 / dW2 / db1 on one FFN column in every 256-column tile of every expert (so
+    every N tile of the dgrad GEMM, every M tile of dW2 and every N tile of dW1) plus the last tile's
+    columns, each over all H; db2 in full; dWg / dbg in full from the oracle's router backward fed the
+    GPU's dw (every token's dw would need every token's expert output)."""
     cfg = synth.CONFIGS["mixtral"]
     dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
     r = _run(cfg, dout)
@@ -118,30 +151,34 @@ def test_backward_mixtral_shape_sampled():
     idx, drp, w = r["topk_idx"], r["dropped"], r["topk_w"]
     E, k = cfg.E, cfg.k
     print("mixtral")
-    # dx and dw on sampled tokens: expert paths + router path (the latter from the GPU's dw)
-    toks = sample_tokens(cfg.T, 6, seed=cfg.seed)
+    rng = np.random.default_rng(cfg.seed)
+    toks = set()
+    for e in range(E):
+        tt, _ = np.where((idx == e) & (drp == 0))
+        tt = np.sort(tt)  # the segment's rows are in (slot, token) order; any three of its tokens will do
+        if tt.size:
+            toks.update([int(tt[0]), int(tt[-1]), int(rng.choice(tt))])
+    toks = np.array(sorted(toks), np.int32)
+    pairs = [(int(t), s, int(idx[t, s])) for t in toks for s in range(k) if not drp[t, s]]
+    assert {e for _, _, e in pairs} == set(range(E))
+    parts = _slots_parallel(inp, cfg, pairs, dout, w)
     ex_dx = np.zeros((len(toks), cfg.H))
     ref_dw = np.zeros((len(toks), k))
     for i, t in enumerate(toks):
         for s in range(k):
-            if drp[t, s]:
-                continue
-            dxp, dws, _ = oracle.bwd_slot(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, t, idx[t, s], dout[t], w[t, s],
-                                          cfg.dtype, cfg.act)
-            ex_dx[i] += dxp
-            ref_dw[i, s] = dws
-    _check("dw (sampled tokens)", r["dw"][toks], ref_dw)
+            if (int(t), s) in parts:
+                ex_dx[i] += parts[(int(t), s)][0]
+                ref_dw[i, s] = parts[(int(t), s)][1]
+    _check("dw (tokens of every expert)", r["dw"][toks], ref_dw)
     cnt_pre = np.bincount(idx.reshape(-1), minlength=E).astype(np.int32)
     dl, dWg, dbg, dxr = oracle.bwd_router(inp.x, inp.Wg, inp.bg, idx, cnt_pre, r["dw"], D_AUX, D_Z, cfg.dtype)
     _check("dWg (router fed the GPU's dw)", r["dWg"], dWg)
     _check("dbg (router fed the GPU's dw)", r["dbg"], dbg)
-    _check("dx (sampled tokens)", r["dx"][toks], ex_dx + dxr[toks])
-    # weight gradients at sampled FFN columns of every expert
-    rng = np.random.default_rng(cfg.seed)
-    cols = np.sort(rng.choice(cfg.F, size=6, replace=False)).astype(np.int32)
+    _check("dx (tokens of every expert)", r["dx"][toks], ex_dx + dxr[toks])
     g2, g1, gb1, gb2 = [], [], [], []
     r2, r1, rb1, rb2 = [], [], [], []
     for e in range(E):
+        cols = stratified_columns(cfg.F, seed=cfg.seed + e)
         tt, ss = np.where((idx == e) & (drp == 0))
         dW2r, dW1c, db1s, db2e = oracle.bwd_expert_weights(inp.x, inp.W1, inp.b1, inp.W2, e, tt.astype(np.int32),
                                                            w[tt, ss], dout, cols, cfg.dtype, cfg.act)
@@ -153,9 +190,10 @@ def test_backward_mixtral_shape_sampled():
         g1.append(r["dW1"][e][:, cols].T)
         gb1.append(r["db1"][e][cols])
         gb2.append(r["db2"][e])
-    _check("dW2 (sampled columns)", np.array(g2), np.array(r2), per_expert=True)
-    _check("dW1 (sampled columns)", np.array(g1), np.array(r1), per_expert=True)
-    _check("db1 (sampled columns)", np.array(gb1), np.array(rb1), per_expert=True)
+    print(f"  {len(toks)} tokens, {sum(len(c) for c in r1)} FFN columns over {E} experts")
+    _check_experts("dW2 (stratified columns)", g2, r2)
+    _check_experts("dW1 (stratified columns)", g1, r1)
+    _check_experts("db1 (stratified columns)", gb1, rb1)
     _check("db2", np.array(gb2), np.array(rb2), per_expert=True)
 
 

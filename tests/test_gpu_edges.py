@@ -285,3 +285,38 @@ def test_out_of_range_indices_are_reported_not_followed():
     buf.forward()
     torch.cuda.synchronize()
     assert buf.device_status() == moe.MOE_OK
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3], ids=["no_cta_pair", "no_tc_gate", "both"])
+def test_kernel_options_select_other_kernels_same_results(flags):
+    """moe_set_kernel_options: the single-CTA GEMM tiles in place of CTA pairs and the CUDA-core gate in
+    place of the tensor-core ones give results that meet the same oracle rules (forward and backward)."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg("options", 1500, 256, 8, 2, 512, 1.1, "bf16", 37)       # pair tiles and the E = 8 mma gate
+    wide = _cfg("options_gemm_gate", 600, 128, 64, 2, 128, 1.0, "bf16", 38)  # the tcgen05 gate (E = 64)
+    try:
+        moe.moe_set_kernel_options(flags)
+        for c in (cfg, wide):
+            r = _run_forward(c)
+            _check_against_oracle(c, r)
+        # backward through the single-CTA dgrad / wgrad kernels as well
+        inp = synth.make_inputs(cfg)
+        buf = moe.MoEBuffers(shape_of(cfg), upload(inp), train=True)
+        buf.forward_train()
+        grads = buf.make_grads()
+        dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+        buf.backward(torch.from_numpy(dout.astype(np.float32)).cuda(), grads, 0.01, 0.001)
+        torch.cuda.synchronize()
+        assert buf.device_status() == moe.MOE_OK
+        ref = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, dout,
+                              0.01, 0.001, topk_idx=buf.topk_idx.cpu().numpy(), dropped=buf.dropped.cpu().numpy())
+        from moe_testlib import TOL_BWD_FRO, TOL_BWD_MAX, fro_rel, rms_rel
+        for n in ("dx", "dWg", "dW1", "dW2"):
+            got = grads[n].cpu().numpy().astype(np.float64)
+            want = getattr(ref, n)
+            per = [rms_rel(got[e], want[e]) for e in range(cfg.E)] if n in ("dW1", "dW2") else [rms_rel(got, want)]
+            assert max(per) <= TOL_BWD_MAX and fro_rel(got, want) <= TOL_BWD_FRO, (n, max(per))
+    finally:
+        moe.moe_set_kernel_options(0)

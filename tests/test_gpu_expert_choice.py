@@ -10,7 +10,9 @@ Checks, per workload:
               losses 1e-3
   permute  -> row maps, offsets and permuted rows bit-exact
   ffn      -> out against the oracle's expert-choice combine of the GPU's choice, tolerance of the
-              storage dtype; tokens chosen by no expert exactly zero
+              storage dtype, on every token (small cases) or on stratified rows at the Mixtral shape
+              (both ends and a row in every 128-row block of every expert, and each expert's last
+              block); tokens chosen by no expert exactly zero
   forward  -> moe_forward (6 launches) gives the same choice and, up to the order of the fp32
               atomic adds, the same out; the unfused FFN + moe_combine agrees as well
 """
@@ -22,7 +24,7 @@ import pytest
 import oracle
 import synth
 from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, normwise_rel, out_error, router_launches,
-                         sample_tokens, shape_of, upload)
+                         shape_of, stratified_tokens, upload)
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +43,7 @@ CASES = [
     _cfg("ec_many_experts", 2048, 128, 64, 2, 128, 1.0, "bf16", 46),    # C = 64
     synth.CONFIGS["mixtral_ec"],                                        # C = 1024 at the Mixtral shape
 ]
-SAMPLES = {"mixtral_ec": 24}
+STRATIFIED = {"mixtral_ec"}  # full size: stratified rows (every m-tile of every expert), else every token
 
 
 def _lib():
@@ -172,7 +174,10 @@ def test_ec_ffn_combine_vs_oracle(run):
     member = np.zeros((cfg.T, cfg.E), bool)
     for e in range(cfg.E):
         member[run["chosen"][e], e] = True
-    toks = sample_tokens(cfg.T, SAMPLES.get(cfg.name, cfg.T), seed=cfg.seed)
+    if cfg.name in STRATIFIED:
+        toks = stratified_tokens(run["offsets"], run["row_token"], seed=cfg.seed)
+    else:
+        toks = np.arange(cfg.T, dtype=np.int32)
     ref = oracle.ec_forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, run["p"].astype(np.float64), member, toks,
                                    cfg.dtype, act=cfg.act)
     live = member[toks].any(axis=1)

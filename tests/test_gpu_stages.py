@@ -4,8 +4,11 @@ Each stage is fed the GPU's own upstream result, so a near-tie flip in routing c
   route    -> top-k indices bit-exact (near ties excluded and counted), weights 1e-4, losses 1e-3
   permute  -> counts, offsets, drop flags, row maps bit-exact against the oracle's dispatch of the
               GPU's top-k; permuted rows equal the source token rows bit for bit
-  ffn      -> out against the oracle's weighted expert FFN of the GPU's routing and drops, on all
-              tokens (tiny) or a sample (full-size workloads)
+  ffn      -> out against the oracle's weighted expert FFN of the GPU's routing and drops, on every
+              token (tiny, decode, switch) or on stratified rows (mixtral, mixtral_block, skew): both
+              ends of every expert segment, a row in every 128-row block (so every 128- and 256-row
+              m-tile of both grouped GEMMs) and every row of each expert's tail tile; every column
+              of each checked row, so every n-tile too
   forward  -> moe_forward (fused, one call) equals the staged result bit for bit
 """
 import math
@@ -15,12 +18,12 @@ import pytest
 
 import oracle
 import synth
-from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, out_error, router_launches, sample_tokens,
-                         shape_of, upload)
+from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, out_error, router_launches, shape_of,
+                         stratified_tokens, upload)
 
 pytestmark = pytest.mark.gpu
 
-SAMPLES = {"tiny": 256, "decode": 32, "switch": 48, "mixtral": 24, "skew": 48, "mixtral_block": 24}
+ALL_TOKENS = {"tiny", "decode", "switch"}  # cheap enough for the oracle on every token
 
 
 TOKEN_CHOICE = [n for n, c in synth.CONFIGS.items() if c.routing == "token_choice"]
@@ -131,7 +134,10 @@ def test_permute_bit_exact(run):
 
 def test_ffn_combine_vs_oracle(run):
     cfg, inp = run["cfg"], run["inp"]
-    toks = sample_tokens(cfg.T, SAMPLES[cfg.name], seed=cfg.seed)
+    if cfg.name in ALL_TOKENS:
+        toks = np.arange(cfg.T, dtype=np.int32)
+    else:
+        toks = stratified_tokens(run["offsets"], run["row_token"], seed=cfg.seed)
     ref = oracle.forward_tokens(inp.x, inp.W1, inp.b1, inp.W2, inp.b2, run["topk_idx"],
                                 run["topk_w"].astype(np.float64), run["dropped"], toks, cfg.dtype, act=cfg.act)
     got = run["out"][toks].astype(np.float64)

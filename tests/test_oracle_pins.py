@@ -675,3 +675,90 @@ def test_min_capacity_lower_bound():
     d = oracle.dispatch(idx, 4, 0.25, min_capacity=4)
     assert d.cap == 4 and d.expert_counts.tolist() == [4, 0, 0, 0]
     assert d.dropped[:4].sum() == 0 and d.dropped[4:].all()
+
+
+# ------------------------------------------------------------------ backward with a given routing -------------
+def test_renorm_weights_closed_forms():
+    """The Quick Start's renormalisation over a given selection: hand-computed values, the slot order kept,
+    any selection (not only the top-k), and the sum-to-one and ratio invariants."""
+    p = np.array([[0.5, 0.3, 0.2], [0.1, 0.6, 0.3]])
+    w = oracle.renorm_weights(p, np.array([[2, 0], [0, 2]], np.int32))
+    assert w[0, 0] == pytest.approx(0.2 / 0.7, abs=1e-16) and w[0, 1] == pytest.approx(0.5 / 0.7, abs=1e-16)
+    assert w[1, 0] == pytest.approx(0.1 / 0.4, abs=1e-16) and w[1, 1] == pytest.approx(0.3 / 0.4, abs=1e-16)
+    rng = np.random.default_rng(5)
+    q = rng.dirichlet(np.ones(7), size=50)
+    idx = np.array([rng.choice(7, size=3, replace=False) for _ in range(50)], np.int32)
+    w = oracle.renorm_weights(q, idx)
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    sel = np.take_along_axis(q, idx.astype(np.int64), axis=1)
+    np.testing.assert_allclose(w[:, 0] / w[:, 1], sel[:, 0] / sel[:, 1], rtol=1e-13)
+    # k = 1: the weight is exactly one whatever the selection
+    assert (oracle.renorm_weights(q, idx[:, :1]) == 1.0).all()
+
+
+def test_renorm_weights_equal_the_routers_own():
+    """Fed the oracle's own top-k, the given-routing weights equal route()'s renormalised weights (two
+    statements of the same division: numpy here, the C loop there)."""
+    cfg = synth.LayerConfig("rw", T=64, H=16, E=6, k=3, F=8, CF=math.inf, dtype="f32", seed=31)
+    inp = synth.make_inputs(cfg)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, cfg.k, "f32")
+    np.testing.assert_allclose(oracle.renorm_weights(r.p, r.topk_idx), r.topk_w, rtol=1e-14, atol=1e-16)
+
+
+@pytest.mark.parametrize("cf", [math.inf, 0.75], ids=["dropless", "drops"])
+def test_backward_given_own_routing_equals_default(cf):
+    """backward(..., topk_idx=, dropped=) fed the oracle's own routing and drops gives every gradient of the
+    default call, to rounding."""
+    cfg, inp, dout = _fd_layer(91, T=11, cf=cf)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, cfg.k, "f32")
+    d = oracle.dispatch(r.topk_idx, cfg.E, cf)
+    if cf < math.inf:
+        assert d.dropped.sum() > 0
+    a = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cf, "f32", dout, 0.3, 0.2)
+    b = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cf, "f32", dout, 0.3, 0.2,
+                        topk_idx=r.topk_idx, dropped=d.dropped)
+    for n in ("dx", "dWg", "dbg", "dW1", "db1", "dW2", "db2", "dw", "dlogits"):
+        np.testing.assert_allclose(getattr(b, n), getattr(a, n), rtol=1e-15, atol=1e-15, err_msg=n)
+
+
+def test_backward_given_routing_matches_central_differences():
+    """The branch the GPU parity tests take: a given selection that is NOT the top-k (slots reversed for some
+    tokens, a lower-ranked expert for others) and a given drop mask that is not the capacity rule's.  Every
+    gradient must equal central differences of the loss with that routing held fixed; renormalising over
+    the wrong axis, using the top-k weights, or letting a dropped slot contribute each fails here."""
+    cfg, inp, dout = _fd_layer(92, T=9, E=4)
+    r = oracle.route(inp.x, inp.Wg, inp.bg, 3, "f32")  # top-3 order, to take a lower-ranked expert from
+    idx = r.topk_idx[:, :2].copy()
+    idx[0::3] = idx[0::3, ::-1]          # reversed slot order
+    idx[1::3, 1] = r.topk_idx[1::3, 2]   # the third-best expert in slot 1
+    dropped = np.zeros((cfg.T, 2), np.uint8)
+    dropped[2, 0] = dropped[5, 1] = 1
+    dropped[7] = 1                       # every slot of token 7 dropped
+    d_aux, d_z = 0.37, -0.21
+    g = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, 2, math.inf, "f32", dout, d_aux, d_z,
+                        topk_idx=idx, dropped=dropped)
+    assert (g.dw[dropped.astype(bool)] == 0).all()
+    grads = dict(x=g.dx, Wg=g.dWg, bg=g.dbg, W1=g.dW1, b1=g.db1, W2=g.dW2, b2=g.db2)
+    rng = np.random.default_rng(92)
+    for name in ("x", "Wg", "bg", "W1", "b1", "W2", "b2"):
+        base = getattr(inp, name)
+        for flat in rng.choice(base.size, size=min(6, base.size), replace=False):
+            at = np.unravel_index(flat, base.shape)
+            lo, hi = base.copy(), base.copy()
+            lo[at] = np.float32(base[at] - 1e-3)
+            hi[at] = np.float32(base[at] + 1e-3)
+            step = float(hi[at]) - float(lo[at])
+            args = {n: getattr(inp, n) for n in ("x", "Wg", "bg", "W1", "b1", "W2", "b2")}
+            vals = []
+            for v in (hi, lo):
+                args[name] = v
+                vals.append(oracle.loss_of_given(args["x"], args["Wg"], args["bg"], args["W1"], args["b1"], args["W2"],
+                                                 args["b2"], idx, dropped, "f32", dout, d_aux, d_z))
+            assert grads[name][at] == pytest.approx((vals[0] - vals[1]) / step, rel=1e-5, abs=1e-7), (name, at)
+    # the fixed-routing loss itself reduces to the oracle's forward when fed the oracle's own routing
+    own = oracle.route(inp.x, inp.Wg, inp.bg, 2, "f32")
+    dd = oracle.dispatch(own.topk_idx, cfg.E, math.inf)
+    assert oracle.loss_of_given(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, own.topk_idx, dd.dropped,
+                                "f32", dout, d_aux, d_z) == pytest.approx(
+        oracle.loss_of(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, 2, math.inf, "f32", dout, d_aux, d_z),
+        rel=1e-14)
