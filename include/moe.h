@@ -186,10 +186,14 @@ MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, mo
 /* Router ("MoE Training" page, Quick Start MoELayer.forward: gate, softmax, topk, renormalise;
  * Core Concepts 3: load_balancing_loss, router_z_loss).
  * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws).
+ * Token choice: 2 launches (the gate with its softmax / top-k tail, then the loss reduction).  bf16
+ * layers with 8, 16 or 32 experts run the gate as register-fed mma.sync over x, the hidden dimension
+ * split over a cluster of up to 8 CTAs per 32-token chunk; bf16 layers with 64, 128 or 256 experts
+ * run it as one tcgen05 GEMM whose epilogue does the softmax / top-k tail.
  * Expert choice: also the per-expert selection (Core Concepts 2), so it writes the chosen tokens
- * to topk_idx[E,C], expert_counts and dropped[T] as well; 3 launches.
- * bf16 layers whose expert count is a multiple of 64 compute the gate as one tensor-core GEMM into
- * the workspace, then the per-chunk softmax/top-k, which adds one launch. */
+ * to topk_idx[E,C], expert_counts and dropped[T] as well; 3 launches, one more for bf16 layers whose
+ * expert count is a multiple of 64 (the gate as a tensor-core GEMM into the workspace, then the
+ * per-chunk softmax). */
 MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
@@ -266,8 +270,8 @@ MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, v
                          cudaStream_t stream);
 
 /* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream (5 launches; one
- * more under expert choice, and one more for the tensor-core gate of bf16 layers with a multiple of
- * 64 experts). */
+ * more under expert choice, and one more again for the expert-choice tensor-core gate of bf16 layers
+ * with a multiple of 64 experts). */
 MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
@@ -335,6 +339,55 @@ MOE_API moe_status_t moe_get_device_status(void* ws, cudaStream_t stream);
 /* Bound on device-side waits, in GPU clock cycles (default 2e9, about one second).  Applies to
  * launches made after the call.  Values <= 0 restore the default. */
 MOE_API void moe_set_wait_limit(long long cycles);
+
+/* ---- expert parallelism ("MoE Training" page, Core Concepts 4, "Expert Parallelism": the experts
+ * are spread over workers, every kept assignment's row travels to the worker that holds its expert,
+ * and the expert outputs travel back to be combined where the token lives).  Each worker routes and
+ * permutes its own tokens with moe_route / moe_permute over all E experts; the rows of expert e then
+ * form the contiguous segment [offsets[e], offsets[e+1]) of its x_perm (moe_workspace_layout).  The
+ * two calls below move those segments and run the owner's experts on what it received; the worker
+ * that sent them writes the returned rows into its y and finishes with moe_combine.  A segment
+ * table is the whole exchange plan, so the same calls serve any placement of experts on workers. */
+
+/* One contiguous run of rows to copy: `rows` rows of the call's row_bytes each, from src to dst.
+ * src and dst are device pointers, 16-byte aligned; either may be another GPU's memory mapped into
+ * this one (a peer-accessible allocation), which makes the copy a pull or a push over NVLink. */
+typedef struct {
+  const void* src;
+  void* dst;
+  int64_t rows;
+} moe_row_segment_t;
+
+/* Copies every segment of segs[nsegs] (a DEVICE array of moe_row_segment_t, 16-byte aligned) in one
+ * launch: the dispatch of every row a worker receives, or the return of every row it sends back.
+ * row_bytes: bytes per row, a positive multiple of 16 (H * 2 for bf16 x rows, H * 4 for fp32 y rows).
+ * max_rows: an upper bound on any segment's rows (it sizes the grid; longer segments are still copied
+ * whole).  Segments must not overlap each other's destinations.  A segment whose src or dst is not
+ * 16-byte aligned is skipped and, when status is not NULL, recorded there as MOE_ERR_INVALID_ARG's
+ * device code (status: a device int32, e.g. a workspace's error word).  Returns MOE_ERR_INVALID_ARG
+ * for nsegs < 0 or > 65535, a bad row_bytes or max_rows, or a NULL / misaligned table with nsegs > 0;
+ * nothing is launched for nsegs = 0.  1 launch. */
+MOE_API moe_status_t moe_copy_row_segments(const moe_row_segment_t* segs, int nsegs, int64_t row_bytes,
+                                           int64_t max_rows, int32_t* status, cudaStream_t stream);
+
+/* The grouped expert FFN over caller-given rows (Quick Start expert Linear(H,F) -> act -> Linear(F,H),
+ * every expert on its own segment): for each expert e < shape->E and each row r in
+ * [offsets[e], offsets[e+1]),
+ *     y[r,:] = act(x_rows[r,:] . W1[e] + b1[e]) . W2[e] + b2[e]      (fp32, not weighted)
+ * shape: H, F, E (the experts held in W1[E,H,F], b1[E,F], W2[E,F,H], b2[E,H], e.g. one worker's
+ * share of the layer's experts), dtype and activation are used; T, k, capacity and routing are not.
+ * x_rows[rows_cap,H] (storage dtype) and y[rows_cap,H] are device buffers; offsets[E+1] is a device
+ * int32 array, non-decreasing from 0, offsets[E] <= rows_cap.  Offsets that break this are clamped
+ * on the device (and recorded in the workspace's error word, reported by moe_get_device_status),
+ * so no row outside [0, rows_cap) is read or written.  Rows in [offsets[E], rows_cap) of y are not
+ * written.  Workspace: moe_expert_ffn_rows_workspace_size(shape, rows_cap) bytes, 256-byte aligned,
+ * first 256 bytes zero before its first use; it holds the bf16 / fp32 h rows.  Validation as for
+ * moe_expert_ffn (H, F, E, dtype, activation; rows_cap >= 0; rows_cap * max(H, F) < 2^31).
+ * 3 launches (offsets check, GEMM1, GEMM2). */
+MOE_API size_t moe_expert_ffn_rows_workspace_size(const moe_shape_t* shape, int64_t rows_cap);
+MOE_API moe_status_t moe_expert_ffn_rows(const moe_shape_t* shape, int64_t rows_cap, const int32_t* offsets,
+                                         const void* x_rows, const void* W1, const void* b1, const void* W2,
+                                         const void* b2, float* y, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Kernel-selection switches for side-by-side comparisons of the kernels; normal use needs none.
  *   MOE_KERNEL_NO_CTA_PAIR  single-CTA 128-row grouped-GEMM tiles everywhere, instead of the CTA-pair

@@ -28,7 +28,8 @@ ENTRY_POINTS = (
     "moe_forward", "moe_forward_host", "moe_get_device_status", "moe_set_wait_limit", "moe_debug_timeout_probe",
     "moe_last_launch_count", "moe_status_string", "moe_route_noalloc", "moe_capacity",
     "moe_train_workspace_size", "moe_forward_train", "moe_backward", "moe_loss_sums", "moe_losses_from_sums",
-    "moe_set_kernel_options", "moe_get_kernel_options",
+    "moe_set_kernel_options", "moe_get_kernel_options", "moe_copy_row_segments", "moe_expert_ffn_rows",
+    "moe_expert_ffn_rows_workspace_size",
 )
 MOE_KERNEL_DEFAULT, MOE_KERNEL_NO_CTA_PAIR, MOE_KERNEL_NO_TC_GATE = 0, 1, 2
 
@@ -59,6 +60,11 @@ class WsView(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("status", "offsets", "cnt_pre", "row_of", "row_token", "row_slot",
                                                "x_perm", "h", "y")] + [("bytes", ctypes.c_size_t),
                                                                         ("scores", ctypes.c_void_p)]
+
+
+class RowSegment(ctypes.Structure):
+    """moe_row_segment_t: `rows` rows from device pointer src to device pointer dst."""
+    _fields_ = [("src", ctypes.c_void_p), ("dst", ctypes.c_void_p), ("rows", ctypes.c_int64)]
 
 
 _lib = None
@@ -107,6 +113,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_set_kernel_options.restype = None
     lib.moe_get_kernel_options.argtypes = []
     lib.moe_get_kernel_options.restype = ctypes.c_int
+    lib.moe_copy_row_segments.argtypes = [vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, vp, vp]
+    lib.moe_copy_row_segments.restype = st
+    lib.moe_expert_ffn_rows_workspace_size.argtypes = [P(Shape), ctypes.c_int64]
+    lib.moe_expert_ffn_rows_workspace_size.restype = sz
+    lib.moe_expert_ffn_rows.argtypes = [P(Shape), ctypes.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_expert_ffn_rows.restype = st
     lib.moe_debug_timeout_probe.argtypes = [vp, sz, vp]
     lib.moe_debug_timeout_probe.restype = st
     lib.moe_last_launch_count.argtypes = []
@@ -238,6 +250,20 @@ def moe_set_kernel_options(flags: int) -> None:
 
 def moe_get_kernel_options() -> int:
     return load_library().moe_get_kernel_options()
+
+
+def moe_copy_row_segments(segs, nsegs: int, row_bytes: int, max_rows: int, status=None, stream=0) -> int:
+    """segs: device address of a moe_row_segment_t array (see RowSegment)."""
+    return load_library().moe_copy_row_segments(segs, nsegs, row_bytes, max_rows, status, stream)
+
+
+def moe_expert_ffn_rows_workspace_size(shape, rows_cap: int) -> int:
+    return load_library().moe_expert_ffn_rows_workspace_size(ctypes.byref(shape), rows_cap)
+
+
+def moe_expert_ffn_rows(shape, rows_cap, offsets, x_rows, W1, b1, W2, b2, y, ws, ws_bytes, stream=0) -> int:
+    return load_library().moe_expert_ffn_rows(ctypes.byref(shape), rows_cap, offsets, x_rows, W1, b1, W2, b2, y, ws,
+                                              ws_bytes, stream)
 
 
 def moe_debug_timeout_probe(ws, ws_bytes, stream=0) -> int:

@@ -51,7 +51,15 @@ constexpr int kStgStride = 36;                     // floats per staged row (32 
 constexpr int kStgWarpBytes = 5 * 1024;  // one warp's staging tile: 32 x 32 fp32 (padded rows) or a
                                           // 1024-aligned 32 x 64 bf16 box in 128-byte swizzle
 
-enum { EPI_GELU = 0, EPI_COMBINE = 1, EPI_STORE_Y = 2, EPI_SILU = 3, EPI_DGRAD_GELU = 4, EPI_DGRAD_SILU = 5 };
+enum {
+  EPI_GELU = 0,
+  EPI_COMBINE = 1,
+  EPI_STORE_Y = 2,
+  EPI_SILU = 3,
+  EPI_DGRAD_GELU = 4,
+  EPI_DGRAD_SILU = 5,
+  EPI_ROUTER = 6  // the gate: softmax, top-k, renormalised weights and a chunk's loss partials
+};
 // GEMM1 epilogues write h = act(acc + b1); GEMM2 epilogues combine or store y; the backward's
 // first GEMM (G = dout_rows . W2[e]^T) writes du = w * G * act'(u) and accumulates dw = G . h.
 __host__ __device__ constexpr bool epi_h(int epi) { return epi == EPI_GELU || epi == EPI_SILU; }
@@ -93,6 +101,12 @@ struct GemmArgs {
   const float* topk_w;
   int k;
   int single_rows;  // offsets == null: one segment of this many rows (a plain dense GEMM)
+  // EPI_ROUTER outputs (N = E experts in one tile; each epilogue warp's 32 rows are one 32-token chunk)
+  int32_t* r_topk_idx;    // [T,k]
+  float* r_topk_w;        // [T,k]
+  float* r_loss_part;     // [nchunk][E+1]: sum_t p[t,e], then sum_t lse_t^2
+  int32_t* r_chunk_hist;  // [k][nchunk][E]
+  float* r_logits;        // [T,E] logits (training forward), or null
   int a_box_rows;   // single-CTA kernel: > 0 loads only ceil(rows / a_box_rows) boxes of that many A rows
   int32_t* status;
   long long wait_limit;
@@ -273,6 +287,133 @@ __device__ __forceinline__ void epilogue_dgrad32(const GemmArgs& g, const uint32
       o[q] = *reinterpret_cast<const uint32_t*>(&d);
     }
     dp[j] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Gate tail of one epilogue warp: lane i owns token row_base + i, whose BN logits sit in TMEM
+// columns [0, BN) of the warp's lane quarter (bias added here).  Three passes over TMEM: the max and
+// the top-k by (logit desc, index asc: a later expert displaces a candidate only when strictly
+// larger); the sum of exp(l - max); the probabilities, whose column sums over the warp's 32 tokens go
+// through the warp's staging tile.  Writes topk_idx / topk_w (renormalised over the k selected), the
+// chunk's loss partials (sum_t p[t,e] for every expert, then sum_t lse^2) and its per-slot expert
+// histograms -- the same quantities, in the same layout, as the CUDA-core router tail.
+template <int BN>
+__device__ __forceinline__ void router_epilogue(const GemmArgs& g, uint32_t taddr, float* stg, int lane, int row_base,
+                                                int wrows) {
+  constexpr int E = BN;
+  const int k = g.k;
+  const int t = row_base + lane;
+  const bool ok = lane < wrows;
+  const int chunk = row_base / 32;
+  const int nchunk = (g.single_rows + 31) / 32;
+  const __nv_bfloat16* bg = g.bias;
+  float cv[8];
+  int ci[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    cv[i] = -INFINITY;
+    ci[i] = 0x7fffffff;
+  }
+  float m = -INFINITY, kth = -INFINITY;
+  // pass 1: max and the top-k candidates (experts visited in increasing order)
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = c * 32 + j;
+      const float v = __uint_as_float(r[j]) + (bg ? __bfloat162float(bg[e]) : 0.f);
+      m = fmaxf(m, v);
+      if (v > kth) {  // k <= 8: insert, keeping (value desc, index asc)
+        float nv = v;
+        int ne = e;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q < k && nv > cv[q]) {
+            const float tv = cv[q];
+            const int te = ci[q];
+            cv[q] = nv;
+            ci[q] = ne;
+            nv = tv;
+            ne = te;
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (q == k - 1) kth = cv[q];  // static indices keep the candidates in registers
+      }
+    }
+  }
+  // pass 2: sum of exp(l - max)
+  float ssum = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int e = c * 32 + j;
+      ssum += expf(__uint_as_float(r[j]) + (bg ? __bfloat162float(bg[e]) : 0.f) - m);
+    }
+  }
+  const float inv_s = 1.f / ssum;
+  const float lse = m + logf(ssum);
+  if (ok) {
+    float psel = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < k) psel += expf(cv[q] - m) * inv_s;
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (q < k) {
+        g.r_topk_idx[(size_t)t * k + q] = ci[q];
+        g.r_topk_w[(size_t)t * k + q] = expf(cv[q] - m) * inv_s / psel;
+      }
+  }
+  // pass 3: probabilities -> per-expert sums over the chunk's tokens (column sums in a fixed order)
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    tmem_ld32(taddr + c * 32, r);
+    float4* mine = reinterpret_cast<float4*>(stg + lane * kStgStride);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float v4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = c * 32 + 4 * q + u;
+        const float l = __uint_as_float(r[4 * q + u]) + (bg ? __bfloat162float(bg[e]) : 0.f);
+        v4[u] = l;
+        r[4 * q + u] = __float_as_uint(ok ? expf(l - m) * inv_s : 0.f);
+      }
+      if (ok && g.r_logits) reinterpret_cast<float4*>(g.r_logits + (size_t)t * E + c * 32)[q] =
+          make_float4(v4[0], v4[1], v4[2], v4[3]);
+      mine[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                            __uint_as_float(r[4 * q + 3]));
+    }
+    __syncwarp();
+    float col = 0.f;
+    for (int i = 0; i < 32; ++i) col += stg[i * kStgStride + lane];
+    g.r_loss_part[(size_t)chunk * (E + 1) + c * 32 + lane] = col;
+    __syncwarp();
+  }
+  float z = ok ? lse * lse : 0.f;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  if (lane == 0) g.r_loss_part[(size_t)chunk * (E + 1) + E] = z;
+  // per-slot expert histograms of the chunk: clear the rows, then one write per distinct expert
+  for (int q = 0; q < k; ++q)
+    for (int e = lane; e < E; e += 32) g.r_chunk_hist[((size_t)q * nchunk + chunk) * E + e] = 0;
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    if (q < k) {
+      const int key = ok ? ci[q] : -1 - lane;  // rows past the tokens never match
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      if (ok && (__ffs(peers) - 1) == lane)
+        g.r_chunk_hist[((size_t)q * nchunk + chunk) * E + ci[q]] = __popc(peers);
+    }
   }
 }
 
@@ -461,6 +602,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int wrows = rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
       constexpr int kChunks = BN / 32 / (kEpiWarps / 4);  // 32-column chunks per epilogue warp
       float dw = 0.f;
+      if constexpr (EPI == EPI_ROUTER) {
+        // one 32-token chunk per warp (the tile's rows start at a multiple of 128); with 8 epilogue
+        // warps the second warp of each lane quarter has nothing to do
+        if (half == 0 && wrows > 0)
+          router_epilogue<BN>(g, tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN), stg, lane,
+                              row0 + quarter * 32, wrows);
+      } else
 #pragma unroll 1
       for (int c = half * kChunks; c < (half + 1) * kChunks; ++c) {
         uint32_t r[32];
@@ -1649,6 +1797,36 @@ cudaError_t launch_gate_logits_sm100(const void* x, const void* Wg, const void* 
   const int tiles = ((T + BM - 1) / BM) * (E / 64);
   const int grid = tiles < num_sms ? tiles : num_sms;
   return launch_one<64, EPI_STORE_Y>(ma, mb, g, grid, st);
+}
+
+// The whole gate of a bf16 layer with E = 64, 128 or 256 experts in one launch: logits = x.Wg + bg
+// on the tensor cores (128-token x E tiles, one dense segment) and, in the epilogue, the softmax,
+// top-k, renormalised weights, per-chunk loss partials and per-slot chunk histograms.
+cudaError_t launch_gate_router_sm100(const RouterArgs& a, cudaStream_t st) {
+  CUtensorMap ma, mb;
+  if (!make_map_a(&ma, a.x, a.T, a.H) || !make_map_b(&mb, a.Wg, 1, a.H, a.E)) return cudaErrorInvalidValue;
+  GemmArgs g{};
+  g.offsets = nullptr;
+  g.single_rows = a.T;
+  g.E = 1;
+  g.N = a.E;
+  g.K = a.H;
+  g.k = a.k;
+  g.bias = reinterpret_cast<const __nv_bfloat16*>(a.bg);
+  g.r_topk_idx = a.topk_idx;
+  g.r_topk_w = a.topk_w;
+  g.r_loss_part = a.loss_part;
+  g.r_chunk_hist = a.chunk_hist;
+  g.r_logits = a.logits_out;
+  g.status = a.status;
+  g.wait_limit = a.wait_limit;
+  const int tiles = (a.T + BM - 1) / BM;
+  const int sms = a.num_sms > 0 ? a.num_sms : 148;
+  const int grid = tiles < sms ? tiles : sms;
+  if (a.E == 64) return launch_one<64, EPI_ROUTER>(ma, mb, g, grid, st);
+  if (a.E == 128) return launch_one<128, EPI_ROUTER>(ma, mb, g, grid, st);
+  if (a.E == 256) return launch_one<256, EPI_ROUTER>(ma, mb, g, grid, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_timeout_probe(int32_t* status, long long limit, cudaStream_t st) {

@@ -129,6 +129,7 @@ namespace moe {
 
 int& launch_count() { return g_launches; }
 int kernel_options() { return g_kernel_options.load(std::memory_order_relaxed); }
+long long wait_limit() { return g_wait_limit.load(); }
 
 // One NVTX range per entry-point call ("moe_route", "moe_forward", ...), so that a timeline shows the
 // stages of a layer call around its kernels.

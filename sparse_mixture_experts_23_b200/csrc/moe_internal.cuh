@@ -149,6 +149,8 @@ moe_status_t check_shape(const moe_shape_t* s);
 int& launch_count();
 // Flags of moe_set_kernel_options (MOE_KERNEL_*), read at each launch.
 int kernel_options();
+// Bound on device-side waits (moe_set_wait_limit), read at each launch.
+long long wait_limit();
 // One NVTX range per entry-point call, named after the entry point.
 struct NvtxRange {
   explicit NvtxRange(const char* name);
@@ -174,6 +176,8 @@ cudaError_t launch_ffn_f32(const FfnArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_gate_logits_sm100(const void* x, const void* Wg, const void* bg, int T, int H, int E, float* logits,
                                      int32_t* status, long long wait_limit, int num_sms, cudaStream_t st);
 cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st);
+// bf16, E in {64, 128, 256}, token choice: the gate GEMM with the softmax / top-k tail in its epilogue
+cudaError_t launch_gate_router_sm100(const RouterArgs& a, cudaStream_t st);
 
 // ---- backward pass ----
 struct BwdPrepArgs {

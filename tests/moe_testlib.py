@@ -143,6 +143,9 @@ def fro_rel(a: np.ndarray, ref: np.ndarray) -> float:
 
 
 def router_launches(cfg) -> int:
-    """Kernels of the gate: one, or two (tensor-core logits GEMM + per-chunk softmax/top-k) for bf16
-    layers whose expert count is a multiple of 64."""
-    return 2 if cfg.dtype == "bf16" and cfg.E % 64 == 0 else 1
+    """Kernels of the gate: one, except under expert choice with a bf16 layer whose expert count is a
+    multiple of 64, where a tensor-core logits GEMM is followed by the per-chunk softmax kernel (under
+    token choice the 64/128/256-expert gate does its softmax and top-k in the GEMM's epilogue)."""
+    if cfg.dtype == "bf16" and cfg.E % 64 == 0 and cfg.routing == "expert_choice":
+        return 2
+    return 1
