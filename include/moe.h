@@ -264,8 +264,10 @@ MOE_API moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io
 /* Combine from a materialised y (Quick Start "output[mask] += expert_scores * expert_output"):
  * out[t] = sum over kept slots s, in slot order, of topk_w[t,s] * y[row_of(t,s)]; tokens with
  * every slot dropped get zeros.  Overwrites out.  Use after moe_expert_ffn(fuse_combine = 0).
- * Expert choice: out[t] += topk_w[t,e] * y[row] for every row, with fp32 atomics into the zeros
- * that moe_permute left in out. */
+ * Expert choice: out[t] = sum over the experts that chose t, in ascending expert order, of
+ * topk_w[t,e] * y[row(t,e)], the row found in the expert's ascending topk_idx[e,:]; a token that no
+ * expert chose gets zeros.  Overwrites out, with no atomics: both rules give the same bits on every
+ * run.  Reads topk_idx as well. */
 MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 

@@ -8,7 +8,8 @@
 //                      the experts that chose it; the last block to finish writes dropped[t]
 //   ec_gather_kernel   x rows into x_perm (row e*C + j = j-th token of expert e), row maps,
 //                      offsets e*C, and clearing of out
-//   ec_combine_kernel  unfused combine: out[t] += p[t,e] * y[row] with fp32 atomics
+//   ec_combine_kernel  unfused combine, token-major: out[t] = sum over the experts that chose t, in
+//                      ascending order, of p[t,e] * y[row] (no atomics; the same bits on every run)
 //
 // The expert FFN that runs between gather and combine is the token-choice one: row_slot holds the
 // expert and the combine weight of row r is topk_w[t * E + e] = p[t,e].
@@ -208,21 +209,45 @@ __global__ void __launch_bounds__(256) ec_gather_kernel(EcGatherArgs a) {
 }
 
 // One block per row: out[t] += p[t,e] * y[row] (fp32 atomics; up to E rows meet in a token).
-__global__ void __launch_bounds__(256) ec_combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ row_token,
-                                                         const int32_t* __restrict__ row_slot,
-                                                         const float* __restrict__ topk_w, int E, int H,
+// Token-major combine without atomics: block t finds, for every expert e, the row holding token t
+// (binary search of the expert's ascending chosen list; -1 when e did not choose t), then writes
+// out[t] = sum over those experts, in ascending order, of p[t,e] * y[row] -- one fixed order, so the
+// result repeats bit for bit, and every out row is written exactly once (0 for a token no expert chose).
+__global__ void __launch_bounds__(256) ec_combine_kernel(const float* __restrict__ y, const int32_t* __restrict__ chosen,
+                                                         const float* __restrict__ topk_w, int E, int C, int H,
                                                          float* __restrict__ out) {
-  const int r = blockIdx.x;
-  const int t = row_token[r];
-  const float w = topk_w[(size_t)t * E + row_slot[r]];
-  const float4* yv = reinterpret_cast<const float4*>(y) + (size_t)r * (H / 4);
-  float* o = out + (size_t)t * H;
-  for (int c = threadIdx.x; c < H / 4; c += blockDim.x) {
-    const float4 v = yv[c];
-    atomicAdd(o + 4 * c + 0, w * v.x);
-    atomicAdd(o + 4 * c + 1, w * v.y);
-    atomicAdd(o + 4 * c + 2, w * v.z);
-    atomicAdd(o + 4 * c + 3, w * v.w);
+  __shared__ int rows_s[256];
+  __shared__ float w_s[256];
+  const int t = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int32_t* ch = chosen + (size_t)e * C;
+    int lo = 0, hi = C;  // first position with ch[pos] >= t
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (ch[mid] < t) lo = mid + 1;
+      else hi = mid;
+    }
+    const bool hit = lo < C && ch[lo] == t;
+    rows_s[e] = hit ? e * C + lo : -1;
+    w_s[e] = hit ? topk_w[(size_t)t * E + e] : 0.f;
+  }
+  __syncthreads();
+  const int nv = H / 4;
+  const float4* yv = reinterpret_cast<const float4*>(y);
+  float4* ov = reinterpret_cast<float4*>(out) + (size_t)t * nv;
+  for (int c = threadIdx.x; c < nv; c += blockDim.x) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < E; ++e) {
+      const int r = rows_s[e];
+      if (r < 0) continue;
+      const float w = w_s[e];
+      const float4 v = yv[(size_t)r * nv + c];
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    ov[c] = acc;
   }
 }
 
@@ -240,10 +265,10 @@ cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_ec_combine(const float* y, const int32_t* row_token, const int32_t* row_slot, const float* topk_w,
-                              int rows, int E, int H, float* out, cudaStream_t st) {
-  if (rows <= 0) return cudaSuccess;
-  ec_combine_kernel<<<rows, 256, 0, st>>>(y, row_token, row_slot, topk_w, E, H, out);
+cudaError_t launch_ec_combine(const float* y, const int32_t* chosen, const float* topk_w, int T, int E, int C, int H,
+                              float* out, cudaStream_t st) {
+  if (T <= 0) return cudaSuccess;
+  ec_combine_kernel<<<T, 256, 0, st>>>(y, chosen, topk_w, E, C, H, out);
   return cudaGetLastError();
 }
 

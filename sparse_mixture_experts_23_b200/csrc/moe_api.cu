@@ -496,12 +496,13 @@ moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   if ((st = check_ws(shape, ws, ws_bytes)) != MOE_OK) return st;
   if (shape->T == 0) return MOE_OK;
   if (null_any({io->out, io->topk_w})) return MOE_ERR_INVALID_ARG;
+  if (shape->routing == MOE_ROUTING_EXPERT_CHOICE && io->topk_idx == nullptr) return MOE_ERR_INVALID_ARG;
   if (!aligned16(io->out)) return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*shape);
   ++g_launches;
   if (shape->routing == MOE_ROUTING_EXPERT_CHOICE)
-    return cuda_status(launch_ec_combine(at<float>(ws, L.y), at<int32_t>(ws, L.row_token), at<int32_t>(ws, L.row_slot),
-                                         io->topk_w, (int)L.rows, shape->E, shape->H, io->out, stream));
+    return cuda_status(launch_ec_combine(at<float>(ws, L.y), io->topk_idx, io->topk_w, shape->T, shape->E, L.ec_cap,
+                                         shape->H, io->out, stream));
   return cuda_status(launch_combine(at<float>(ws, L.y), at<int32_t>(ws, L.row_of), io->topk_w, shape->T, shape->H,
                                     shape->k, io->out, stream));
 }

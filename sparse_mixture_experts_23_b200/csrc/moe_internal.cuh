@@ -286,8 +286,8 @@ cudaError_t launch_bwd_gemms_sm100(const BwdGemmArgs& a, cudaStream_t st, int* l
 // the same four GEMMs for fp32 storage, on CUDA cores
 cudaError_t launch_bwd_gemms_f32(const BwdGemmArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st);
-cudaError_t launch_ec_combine(const float* y, const int32_t* row_token, const int32_t* row_slot, const float* topk_w,
-                              int rows, int E, int H, float* out, cudaStream_t st);
+cudaError_t launch_ec_combine(const float* y, const int32_t* chosen, const float* topk_w, int T, int E, int C, int H,
+                              float* out, cudaStream_t st);
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int T, int H, int k, float* out,
                            cudaStream_t st);

@@ -111,6 +111,10 @@ def run(request):
     buf.combine()
     torch.cuda.synchronize()
     res["out_unfused"] = buf.out.cpu().numpy().copy()
+    buf.out.fill_(float("nan"))  # the standalone combine overwrites every row, with no atomics
+    buf.combine()
+    torch.cuda.synchronize()
+    res["out_unfused_again"] = buf.out.cpu().numpy().copy()
     # the whole pass in one call
     buf.out.fill_(float("nan"))
     buf.topk_idx.fill_(-1)
@@ -194,6 +198,7 @@ def test_ec_forward_and_unfused_agree(run):
     scale = float(np.max(np.abs(run["out"]))) or 1.0
     assert np.max(np.abs(run["out_forward"] - run["out"])) <= 1e-5 * scale
     assert np.max(np.abs(run["out_unfused"] - run["out"])) <= 1e-5 * scale
+    assert np.array_equal(run["out_unfused"], run["out_unfused_again"])  # fixed expert order: same bits
 
 
 def test_ec_equal_logits_take_the_first_tokens():

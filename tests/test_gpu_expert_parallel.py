@@ -77,7 +77,7 @@ def _rows_case(name, H, F, E, counts, dtype, act="gelu", bias=True, seed=0):
 
 
 @pytest.mark.parametrize("case", [
-    _rows_case("rows_pair", 256, 512, 4, [300, 0, 520, 77], "bf16", seed=61),          # CTA-pair tiles, empty expert
+    _rows_case("rows_pair", 256, 512, 4, [300, 0, 700, 77], "bf16", seed=61),          # CTA-pair tiles (269 rows per expert), empty expert
     _rows_case("rows_single", 128, 192, 5, [40, 3, 0, 90, 17], "bf16", seed=62),       # single-CTA, 64-wide N tiles
     _rows_case("rows_silu_nobias", 256, 256, 2, [200, 180], "bf16", "silu", False, 63),
     _rows_case("rows_f32", 20, 12, 3, [7, 0, 11], "f32", seed=64),
