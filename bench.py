@@ -99,6 +99,21 @@ def ffn_roofline(cfg: synth.LayerConfig, kept: int, touched_experts: int, ms_ffn
     return r
 
 
+def sustained_roofline(cfg: synth.LayerConfig, kept: int, ms: float, peaks: dict, clocks: dict | None,
+                       sms: int = 148) -> dict:
+    """The same call timed in a loop of about 0.3 s, long enough for the power cap to set the clock: its
+    rate against the measured sustained (power-capped) bf16 peak, and per SM-cycle at that clock."""
+    flops = 4.0 * cfg.H * cfg.F * kept
+    a = flops / (ms / 1000.0) / 1e12
+    r = {"ms": ms, "achieved": a, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+         "frac": a / peaks["bf16_tflops_sustained"], "clocks": clocks}
+    mhz = (clocks or {}).get("sm_mhz")
+    if mhz:
+        per_clk = flops / (ms / 1000.0 * mhz * 1e6 * sms)
+        r["tensor_flop_per_sm_clk"] = {"value": per_clk, "of_nominal": per_clk / TC_FLOP_PER_CLK_SM}
+    return r
+
+
 def load_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -109,19 +124,40 @@ def load_peaks() -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 50 ms while running."""
+    """SM clock, power and throttle reasons sampled while running: NVML polled every `interval_ms`
+    (fine enough to resolve a loop of a few tens of milliseconds), else nvidia-smi every 50 ms.  Only
+    readings are taken; no setting of the GPU is touched."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap,power.limit,temperature.gpu")
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20), ("hw_thermal_slowdown", 0x40),
+               ("sw_power_cap", 0x4))
 
-    def __init__(self, gpu_id: str | None):
+    def __init__(self, gpu_id: str | None, interval_ms: float = 2.0):
         self.gpu_id = gpu_id
+        self.interval = interval_ms / 1000.0
         self.proc = None
-        self.lines = []
         self.thread = None
+        self.stop_flag = False
+        self.samples = []  # (time, sm_mhz, sm_max_mhz, power_w, reasons bitmask, power_limit_w, temp_c)
+        self.window = None  # host-time bounds of the measured region (mark), else every sample
+        self.lines = []
+        self.source = None
 
     def start(self):
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id) if self.gpu_id
+                 else pynvml.nvmlDeviceGetHandleByIndex(0))
+            self._nvml, self._h = pynvml, h
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.plimit = pynvml.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0
+            self.source = "nvml"
+            self.thread = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self._nvml = None
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.gpu_id:
             cmd.insert(1, f"--id={self.gpu_id}")
@@ -130,49 +166,92 @@ class ClockSampler:
         except Exception:
             self.proc = None
             return
+        self.source = "nvidia-smi"
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap,power.limit,temperature.gpu")
+
+    def mark(self, t0: float, t1: float):
+        """Keep only the samples taken between host times t0 and t1 (the region being measured)."""
+        self.window = (t0, t1)
+
+    def _poll_nvml(self):
+        nv, h = self._nvml, self._h
+        while not self.stop_flag:
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                tc = nv.nvmlDeviceGetTemperature(h, nv.NVML_TEMPERATURE_GPU)
+                self.samples.append((time.time(), float(sm), float(self.smax), pw, rs, self.plimit, float(tc)))
+            except Exception:
+                pass
+            time.sleep(self.interval)
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def stop(self) -> dict:
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampler unavailable"]}
+        self.stop_flag = True
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
         sm, smax, power, reasons, plimit, temp = [], [], [], set(), [], []
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-                power.append(float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-            try:
-                plimit.append(float(parts[8]))
-                temp.append(float(parts[9]))
-            except (ValueError, IndexError):
-                pass
+        if self.source == "nvml":
+            rows = self.samples
+            if self.window is not None:
+                inside = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
+                rows = inside or rows
+            for _, s_, mx, pw, rs, pl, tc in rows:
+                sm.append(s_)
+                smax.append(mx)
+                power.append(pw)
+                plimit.append(pl)
+                temp.append(tc)
+                for n, bit in self.REASONS:
+                    if rs & bit:
+                        reasons.add(n)
+        else:
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for ln in self.lines:
+                parts = [p.strip() for p in ln.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                    power.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+                try:
+                    plimit.append(float(parts[8]))
+                    temp.append(float(parts[9]))
+                except (ValueError, IndexError):
+                    pass
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        thr = max(power) * 0.5 if power else 0
-        loaded = [s for s, p in zip(sm, power) if p >= thr] or sm
+        if self.source == "nvml" and self.window is not None:
+            loaded = sm  # already the samples of the measured region
+        else:
+            thr = max(power) * 0.5 if power else 0
+            loaded = [s for s, p in zip(sm, power) if p >= thr] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm), "samples_loaded": len(loaded), "power_w_max": max(power) if power else None,
+                "samples": len(sm), "samples_loaded": len(loaded), "source": self.source,
+                "power_w_max": max(power) if power else None,
                 "power_w_median": statistics.median(power) if power else None,
                 "power_limit_w": max(plimit) if plimit else None, "temp_c_max": max(temp) if temp else None}
 
@@ -350,15 +429,18 @@ def run_ours_impl(args, cfg):
         buf.forward()
     if rank == 0:
         sampler.start()
-        time.sleep(0.5)  # let the sampler take its first reading
+        time.sleep(0.1)  # let the sampler take its first readings
     # ---------------- timed region: K whole forward passes -----------------------------------
     sync_all()
+    t_host0 = time.time()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
     for _ in range(args.steps):
         buf.forward()
     ev1.record(stream)
     sync_all()
+    if rank == 0:
+        sampler.mark(t_host0, time.time())
     clocks = sampler.stop() if rank == 0 else None
     launches_per_step = moe.moe_last_launch_count()
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world, "cuda")
@@ -368,7 +450,8 @@ def run_ours_impl(args, cfg):
     # ---------------- per-kernel timing (same stream, CUDA events, inputs > L2) ---------------
     reps = min(max(args.steps, 20), 200)
 
-    def time_calls(fn, min_seconds: float = 0.0, clock_name: str | None = None, reps: int = reps) -> float:
+    def time_calls(fn, min_seconds: float = 0.0, clock_name: str | None = None, reps: int = reps,
+                   settle: float = 0.0) -> float:
         """Average device time of one call: `reps` calls captured in a CUDA graph and replayed, so
         host-side launch cost does not enter (plain back-to-back calls when capture fails).  With
         min_seconds, the graph is replayed until that much device time has passed and the average
@@ -397,10 +480,13 @@ def run_ours_impl(args, cfg):
                 for _ in range(reps):
                     fn()
 
+        if settle > 0:
+            time.sleep(settle)  # an idle pause, so a short (burst) measurement starts from rested clocks
         smp = ClockSampler(uuid) if (clock_name and rank == 0) else None
         if smp is not None:
             smp.start()
-            time.sleep(0.5)  # the sampler's first reading
+            time.sleep(0.05)  # the sampler's first readings
+        th0 = time.time()
         a.record(stream)
         run_once()
         b.record(stream)
@@ -417,13 +503,17 @@ def run_ours_impl(args, cfg):
                 total_ms += a.elapsed_time(b)
                 n += more
         if smp is not None:
+            smp.mark(th0, time.time())
             kernel_clocks[clock_name] = smp.stop()
         del g
         return total_ms / (reps * n)
 
     kernel_clocks = {}
-    # the dominant kernel pair, timed alone (burst regime, about 0.3 s) with its own clock record
-    ms_ffn = time_calls(lambda: buf.expert_ffn(True), clock_name="ffn", reps=200)
+    # the dominant kernel pair, timed alone with its own clock record: as many back-to-back calls as
+    # the timed region has steps (burst regime, against the burst peak), and a 200-call loop of about
+    # 0.3 s (the power-capped regime, against the sustained peak)
+    ms_ffn = time_calls(lambda: buf.expert_ffn(True), clock_name="ffn", reps=max(20, args.steps), settle=0.5)
+    ms_ffn_sus = time_calls(lambda: buf.expert_ffn(True), clock_name="ffn_sustained", reps=200)
     ms_route = time_calls(buf.route)
     ms_permute = time_calls(buf.permute)
     # standalone combine (the unfused path: y materialised by moe_expert_ffn(fuse_combine=0))
@@ -553,7 +643,9 @@ def run_ours_impl(args, cfg):
                    "l2": "inputs larger than L2: the expert weights (%.2f GB) stream every step" %
                          (cfg.E * 2 * cfg.H * cfg.F * es / 1e9)},
         "roofline": dict(ffn_roofline(cfg, kept, touched, ms_ffn, peaks, kernel_clocks.get("ffn"), sms),
-                         traffic=traffic, clocks=kernel_clocks.get("ffn"),
+                         traffic=traffic, clocks=kernel_clocks.get("ffn"), calls_timed=max(20, args.steps),
+                         sustained=sustained_roofline(cfg, kept, ms_ffn_sus, peaks, kernel_clocks.get("ffn_sustained"),
+                                                      sms),
                          kernel="grouped GEMMs (GEMM1 bias+act, GEMM2 scale+combine), one moe_expert_ffn call"),
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": cfg.T * cfg.H * es,
