@@ -202,9 +202,10 @@ MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, voi
  * allocation after start-up, plugins whose host framework owns every allocation.  The pages
  * have no counterpart; it exists for these callers only.
  * Same inputs, outputs, validation and results as moe_route.  The router's scratch (per-block
- * sums and per-chunk histograms) lives in a 1 MiB array built into the library, which every GPU
- * that loads the library keeps until the process exits.  It needs
- *   align256(ceil(T/32)*(E+1)*4) + align256(k*ceil(T/32)*E*4) + align256(E*4) <= 1 MiB
+ * sums, per-chunk histograms, and a device error word where a bounded wait of the tensor-core gate
+ * would record a timeout, which this call has no way to report) lives in a 1 MiB array built into
+ * the library, which every GPU that loads the library keeps until the process exits.  It needs
+ *   256 + align256(ceil(T/32)*(E+1)*4) + align256(k*ceil(T/32)*E*4) + align256(E*4) <= 1 MiB
  * (for example T = 16384 with E = 64, k = 2 uses 395 KB); larger shapes return MOE_ERR_WORKSPACE
  * before anything is launched.  No device memory is allocated or freed, by this call or by any
  * routine it calls.  The first call on a device looks up the array's device address for that

@@ -1733,8 +1733,10 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
       !make_map_store(&mc1, a.h, a.rows_cap, a.F))
     return cudaErrorInvalidValue;
   const int grid = a.num_sms > 0 ? a.num_sms : 148;
-  // a few rows per expert on average: 16-row A boxes (decode-sized batches)
-  const bool small = a.avg_rows < 32;
+  // segments shorter than one 128-row tile on average (decode-sized batches; the Switch shape's ~64
+  // rows per expert): 16-row A boxes, so a tile loads only the boxes that hold its own rows and not
+  // the next expert's, and the tile width is chosen for the fewest weight-streaming waves
+  const bool small = a.avg_rows < BM;
   CUtensorMap ma1s, ma2s;
   if (small && (!make_map_a16(&ma1s, a.x_perm, a.rows_cap, a.H) || !make_map_a16(&ma2s, a.h, a.rows_cap, a.F)))
     return cudaErrorInvalidValue;

@@ -52,15 +52,26 @@ cudaError_t scratch_for_current_device(cudaStream_t stream, void** out) {
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Scratch layout for a shape: router partials [nblk][E+1] fp32, chunk histograms [k][nblk][E]
-// int32, per-expert totals [E] int32, each section 256-byte aligned.
-size_t scratch_bytes(const moe_shape_t* s, size_t* hist_off, size_t* cnt_off) {
+// Scratch layout for a shape: a device error word (256 bytes; the tensor-core gate's bounded waits
+// record a timeout there), router partials [nblk][E+1] fp32, chunk histograms [k][nblk][E] int32,
+// per-expert totals [E] int32, each section 256-byte aligned.
+constexpr size_t kStatusBytes = 256;
+size_t scratch_bytes(const moe_shape_t* s, size_t* part_off, size_t* hist_off, size_t* cnt_off) {
   const size_t nblk = ((size_t)s->T + moe::kChunk - 1) / moe::kChunk;
   const size_t part = align256(nblk * ((size_t)s->E + 1) * 4);
   const size_t hist = align256((size_t)s->k * nblk * (size_t)s->E * 4);
-  *hist_off = part;
-  *cnt_off = part + hist;
-  return part + hist + align256((size_t)s->E * 4);
+  *part_off = kStatusBytes;
+  *hist_off = kStatusBytes + part;
+  *cnt_off = kStatusBytes + part + hist;
+  return kStatusBytes + part + hist + align256((size_t)s->E * 4);
+}
+
+int device_sms() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      v <= 0)
+    v = 148;
+  return v;
 }
 
 }  // namespace
@@ -76,8 +87,8 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   if (io == nullptr) return MOE_ERR_INVALID_ARG;
   if (shape->routing != MOE_ROUTING_TOKEN_CHOICE) return MOE_ERR_UNSUPPORTED;  // the selection needs a workspace
   if (io->aux_loss == nullptr || io->z_loss == nullptr) return MOE_ERR_INVALID_ARG;
-  size_t hist_off = 0, cnt_off = 0;
-  if (scratch_bytes(shape, &hist_off, &cnt_off) > kScratchBytes)
+  size_t part_off = 0, hist_off = 0, cnt_off = 0;
+  if (scratch_bytes(shape, &part_off, &hist_off, &cnt_off) > kScratchBytes)
     return MOE_ERR_WORKSPACE;  // shape too large for the built-in scratch
   if (shape->T == 0) {
     ++launches;
@@ -92,12 +103,14 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   void* base = nullptr;
   if (scratch_for_current_device(stream, &base) != cudaSuccess) return MOE_ERR_CUDA;
   const int nblk = (shape->T + moe::kChunk - 1) / moe::kChunk;
-  float* loss_part = static_cast<float*>(base);
+  int32_t* status = static_cast<int32_t*>(base);
+  float* loss_part = reinterpret_cast<float*>(static_cast<unsigned char*>(base) + part_off);
   int32_t* chunk_hist = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + hist_off);
   int32_t* cnt_pre = reinterpret_cast<int32_t*>(static_cast<unsigned char*>(base) + cnt_off);
   // Every element the kernels read from the scratch is written earlier in the same call (each
   // router block writes its whole partial row and histogram rows; the reduction writes the
-  // per-expert totals before reading them), so nothing needs clearing between calls.
+  // per-expert totals before reading them), so nothing needs clearing between calls.  The error
+  // word is only ever written (on a timeout), never read by a kernel.
   moe::RouterArgs r{};
   r.x = io->x;
   r.Wg = io->Wg;
@@ -110,7 +123,11 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   r.topk_w = io->topk_w;
   r.loss_part = loss_part;
   r.chunk_hist = chunk_hist;
-  // no gate scratch here, so always the one-kernel router
+  r.status = status;  // a bounded wait of the tensor-core gate records a timeout here
+  r.wait_limit = moe::wait_limit();
+  r.num_sms = device_sms();
+  // no [T,E] gate scratch here: the router is one kernel (the tensor-core gate of 64 / 128 / 256
+  // experts keeps its softmax / top-k tail in the GEMM epilogue and needs none)
   if (moe::launch_router(r, shape->dtype, stream, &launches) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::ReduceArgs a{};

@@ -1205,16 +1205,19 @@ cudaError_t launch_stream(const RouterArgs& a, int nblk, cudaStream_t st) {
 
 cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* launches) {
   const int nblk = (a.T + kChunk - 1) / kChunk;
+  // the tcgen05 gate kernels wait on pipeline barriers with a bound, and record a wait that ran out
+  // in a device error word: without one (or without a bound) they are not used
+  const bool tc_gate_ok = a.status != nullptr && a.wait_limit > 0 && !router_mma_disabled();
   // bf16, token choice, E = 64, 128 or 256: one tensor-core GEMM whose epilogue does the whole
   // softmax / top-k / partials tail (the logits never leave the SM)
   if (dtype == MOE_DTYPE_BF16 && a.scores == nullptr && (a.E == 64 || a.E == 128 || a.E == 256) && a.H % 64 == 0 &&
-      a.k <= 8 && !router_mma_disabled()) {
+      a.k <= 8 && tc_gate_ok) {
     ++*launches;
     return launch_gate_router_sm100(a, st);
   }
   // bf16, E a multiple of 64, scratch given: the gate is one dense tensor-core GEMM, then the
   // per-chunk tail (the gate weights are read once per 128-token tile instead of once per chunk)
-  if (a.gemm_logits != nullptr && dtype == MOE_DTYPE_BF16 && a.E % 64 == 0 && a.H % 64 == 0 && !router_mma_disabled()) {
+  if (a.gemm_logits != nullptr && dtype == MOE_DTYPE_BF16 && a.E % 64 == 0 && a.H % 64 == 0 && tc_gate_ok) {
     cudaError_t err = launch_gate_logits_sm100(a.x, a.Wg, a.bg, a.T, a.H, a.E, a.gemm_logits, a.status, a.wait_limit,
                                                a.num_sms > 0 ? a.num_sms : 148, st);
     if (err != cudaSuccess) return err;

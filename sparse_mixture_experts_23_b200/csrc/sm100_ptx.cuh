@@ -54,7 +54,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
     if (*abort_flag) return false;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
-      atomicCAS(status, 0, code);
+      if (status != nullptr) atomicCAS(status, 0, code);  // a caller without an error word only aborts
       return false;
     }
   }
@@ -69,7 +69,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
     if (*abort_flag) return false;
     if (clock64() - t0 > limit) {
       *abort_flag = 1;
-      atomicCAS(status, 0, code);
+      if (status != nullptr) atomicCAS(status, 0, code);  // a caller without an error word only aborts
       return false;
     }
   }
