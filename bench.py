@@ -315,13 +315,26 @@ def cpu_oracle_rate(cfg: synth.LayerConfig, inp: synth.LayerInputs, budget_s: fl
         dt = time.perf_counter() - t0
         spent += dt
         best = (n, dt)
-        if dt >= budget_s / 3 or n >= max_tokens or spent + 2.2 * dt > budget_s:
+        if dt >= budget_s / 3 or n >= min(max_tokens, cfg.T) or spent + 2.2 * dt > budget_s:
             break
-        n *= 2
+        n = min(n * 2, cfg.T)  # the sample never runs past the batch
     n, dt = best
+    # one core on a small leading sample, for the single-core figure (extrapolated to the whole batch)
+    n1 = max(1, min(n, 8))
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle_layer(cfg, inp, 0, n1)
+        dt1 = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(threads)
     return {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": f"first {n} tokens of the {cfg.name} workload as one layer call (routing, dispatch, "
-                      f"expert FFN, combine in fp64), {dt:.2f} s"}
+                      f"expert FFN, combine in fp64), {dt:.2f} s",
+            "full_batch_estimate_s": cfg.T * dt / n,
+            "single_core": {"value": n1 / dt1, "unit": "tokens/s", "cores": 1, "extrapolated": True,
+                            "sample": f"first {n1} tokens on one thread, {dt1:.2f} s; the whole {cfg.T}-token "
+                                      f"batch would take about {cfg.T * dt1 / n1:.0f} s"}}
 
 
 def run_reference(args, cfg):
