@@ -291,22 +291,29 @@ __device__ __forceinline__ void epilogue_dgrad32(const GemmArgs& g, const uint32
 }
 
 // Gate tail of one epilogue warp: lane i owns token row_base + i, whose BN logits sit in TMEM
-// columns [0, BN) of the warp's lane quarter (bias added here).  Three passes over TMEM: the max and
-// the top-k by (logit desc, index asc: a later expert displaces a candidate only when strictly
-// larger); the sum of exp(l - max); the probabilities, whose column sums over the warp's 32 tokens go
-// through the warp's staging tile.  Writes topk_idx / topk_w (renormalised over the k selected), the
-// chunk's loss partials (sum_t p[t,e] for every expert, then sum_t lse^2) and its per-slot expert
-// histograms -- the same quantities, in the same layout, as the CUDA-core router tail.
+// columns [0, BN) of the warp's lane quarter.  The bias goes to the warp's staging area once (read
+// back by broadcast); then three passes over TMEM: (1) the max and the top-k by (logit desc, index
+// asc: a later expert displaces a candidate only when strictly larger), plus the logits themselves
+// for a training forward; (2) e = exp(l - max) and their sum, the e written back over the
+// accumulator; (3) p = e / sum, whose column sums over the warp's 32 tokens go through the staging
+// tile (stored with a rotation so both the row writes and the column reads spread over the banks).
+// Writes topk_idx / topk_w (renormalised over the k selected), the chunk's loss partials (sum_t
+// p[t,e] for every expert, then sum_t lse^2) and its per-slot expert histograms -- the same
+// quantities, in the same layout, as the CUDA-core router tail.
 template <int BN>
 __device__ __forceinline__ void router_epilogue(const GemmArgs& g, uint32_t taddr, float* stg, int lane, int row_base,
                                                 int wrows) {
   constexpr int E = BN;
+  constexpr float kLog2e = 1.4426950408889634f;
   const int k = g.k;
   const int t = row_base + lane;
   const bool ok = lane < wrows;
   const int chunk = row_base / 32;
   const int nchunk = (g.single_rows + 31) / 32;
-  const __nv_bfloat16* bg = g.bias;
+  float* tile = stg;          // [32][32] fp32, rotated by row
+  float* bias = stg + 1024;   // [E] fp32
+  for (int e = lane; e < E; e += 32) bias[e] = g.bias ? __bfloat162float(g.bias[e]) : 0.f;
+  __syncwarp();
   float cv[8];
   int ci[8];
 #pragma unroll
@@ -323,9 +330,10 @@ __device__ __forceinline__ void router_epilogue(const GemmArgs& g, uint32_t tadd
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const int e = c * 32 + j;
-      const float v = __uint_as_float(r[j]) + (bg ? __bfloat162float(bg[e]) : 0.f);
+      const float v = __uint_as_float(r[j]) + bias[e];
+      r[j] = __float_as_uint(v);
       m = fmaxf(m, v);
-      if (v > kth) {  // k <= 8: insert, keeping (value desc, index asc)
+      if (v > kth) {
         float nv = v;
         int ne = e;
 #pragma unroll
@@ -341,11 +349,18 @@ __device__ __forceinline__ void router_epilogue(const GemmArgs& g, uint32_t tadd
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          if (q == k - 1) kth = cv[q];  // static indices keep the candidates in registers
+          if (q == k - 1) kth = cv[q];
       }
     }
+    if (ok && g.r_logits) {
+      float4* dst = reinterpret_cast<float4*>(g.r_logits + (size_t)t * E + c * 32);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
+                             __uint_as_float(r[4 * q + 3]));
+    }
   }
-  // pass 2: sum of exp(l - max)
+  // pass 2: e = exp(l - max) written back over the accumulator, and their sum
   float ssum = 0.f;
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
@@ -353,48 +368,41 @@ __device__ __forceinline__ void router_epilogue(const GemmArgs& g, uint32_t tadd
     tmem_ld32(taddr + c * 32, r);
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
-      const int e = c * 32 + j;
-      ssum += expf(__uint_as_float(r[j]) + (bg ? __bfloat162float(bg[e]) : 0.f) - m);
+      const float ev = __expf(__uint_as_float(r[j]) + bias[c * 32 + j] - m);
+      ssum += ev;
+      r[j] = __float_as_uint(ev);
     }
+    tmem_st32(taddr + c * 32, r);
   }
   const float inv_s = 1.f / ssum;
-  const float lse = m + logf(ssum);
+  const float lse = m + __logf(ssum);
   if (ok) {
     float psel = 0.f;
 #pragma unroll
     for (int q = 0; q < 8; ++q)
-      if (q < k) psel += expf(cv[q] - m) * inv_s;
+      if (q < k) psel += __expf(cv[q] - m);
 #pragma unroll
     for (int q = 0; q < 8; ++q)
       if (q < k) {
         g.r_topk_idx[(size_t)t * k + q] = ci[q];
-        g.r_topk_w[(size_t)t * k + q] = expf(cv[q] - m) * inv_s / psel;
+        g.r_topk_w[(size_t)t * k + q] = __expf(cv[q] - m) / psel;
       }
   }
-  // pass 3: probabilities -> per-expert sums over the chunk's tokens (column sums in a fixed order)
+  // pass 3: p = e / sum -> per-expert sums over the chunk's tokens (column sums in a fixed order)
 #pragma unroll 1
   for (int c = 0; c < BN / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
-    float4* mine = reinterpret_cast<float4*>(stg + lane * kStgStride);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      float v4[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = c * 32 + 4 * q + u;
-        const float l = __uint_as_float(r[4 * q + u]) + (bg ? __bfloat162float(bg[e]) : 0.f);
-        v4[u] = l;
-        r[4 * q + u] = __float_as_uint(ok ? expf(l - m) * inv_s : 0.f);
-      }
-      if (ok && g.r_logits) reinterpret_cast<float4*>(g.r_logits + (size_t)t * E + c * 32)[q] =
-          make_float4(v4[0], v4[1], v4[2], v4[3]);
-      mine[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]), __uint_as_float(r[4 * q + 2]),
-                            __uint_as_float(r[4 * q + 3]));
+      const float s4 = ok ? inv_s : 0.f;
+      reinterpret_cast<float4*>(tile + lane * 32)[(q + lane) & 7] =
+          make_float4(__uint_as_float(r[4 * q]) * s4, __uint_as_float(r[4 * q + 1]) * s4,
+                      __uint_as_float(r[4 * q + 2]) * s4, __uint_as_float(r[4 * q + 3]) * s4);
     }
     __syncwarp();
     float col = 0.f;
-    for (int i = 0; i < 32; ++i) col += stg[i * kStgStride + lane];
+    for (int i = 0; i < 32; ++i) col += tile[i * 32 + ((((lane >> 2) + i) & 7) << 2) + (lane & 3)];
     g.r_loss_part[(size_t)chunk * (E + 1) + c * 32 + lane] = col;
     __syncwarp();
   }
@@ -416,6 +424,7 @@ __device__ __forceinline__ void router_epilogue(const GemmArgs& g, uint32_t tadd
     }
   }
 }
+
 
 template <int BN, int EPI, bool BKM>
 __global__ void __launch_bounds__(kThreads, 1)
