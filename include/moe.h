@@ -187,13 +187,13 @@ MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, mo
  * Core Concepts 3: load_balancing_loss, router_z_loss).
  * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws).
  * Token choice: 2 launches (the gate with its softmax / top-k tail, then the loss reduction).  bf16
- * layers with 8, 16 or 32 experts run the gate as register-fed mma.sync over x, the hidden dimension
- * split over a cluster of up to 8 CTAs per 32-token chunk; bf16 layers with 64, 128 or 256 experts
- * run it as one tcgen05 GEMM whose epilogue does the softmax / top-k tail.
+ * layers with 8, 16 or 32 experts run the gate as register-fed mma.sync over x; bf16 layers whose
+ * expert count is a multiple of 64 run it as a tcgen05 GEMM into the workspace followed by the
+ * per-chunk softmax / top-k (one launch more), or -- with 64, 128 or 256 experts and at least one
+ * 128-token tile per two SMs -- as one tcgen05 GEMM whose epilogue does the softmax / top-k.
  * Expert choice: also the per-expert selection (Core Concepts 2), so it writes the chosen tokens
  * to topk_idx[E,C], expert_counts and dropped[T] as well; 3 launches, one more for bf16 layers whose
- * expert count is a multiple of 64 (the gate as a tensor-core GEMM into the workspace, then the
- * per-chunk softmax). */
+ * expert count is a multiple of 64. */
 MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
@@ -273,8 +273,7 @@ MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, v
                          cudaStream_t stream);
 
 /* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream (5 launches; one
- * more under expert choice, and one more again for the expert-choice tensor-core gate of bf16 layers
- * with a multiple of 64 experts). */
+ * more under expert choice, and one more for the two-kernel tensor-core gate described at moe_route). */
 MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 

@@ -304,7 +304,6 @@ template <int BN>
 __device__ __forceinline__ void router_epilogue(const GemmArgs& g, uint32_t taddr, float* stg, int lane, int row_base,
                                                 int wrows) {
   constexpr int E = BN;
-  constexpr float kLog2e = 1.4426950408889634f;
   const int k = g.k;
   const int t = row_base + lane;
   const bool ok = lane < wrows;
@@ -1742,10 +1741,10 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
       !make_map_store(&mc1, a.h, a.rows_cap, a.F))
     return cudaErrorInvalidValue;
   const int grid = a.num_sms > 0 ? a.num_sms : 148;
-  // segments shorter than one 128-row tile on average (decode-sized batches; the Switch shape's ~64
-  // rows per expert): 16-row A boxes, so a tile loads only the boxes that hold its own rows and not
-  // the next expert's, and the tile width is chosen for the fewest weight-streaming waves
-  const bool small = a.avg_rows < BM;
+  // a few rows per expert on average (decode-sized batches): 16-row A boxes, and the tile width chosen
+  // for the fewest weight-streaming waves.  (At the Switch shape's ~64 rows per expert this mode measured
+  // slower: its narrower GEMM2 tiles read shorter runs of each weight row.)
+  const bool small = a.avg_rows < 32;
   CUtensorMap ma1s, ma2s;
   if (small && (!make_map_a16(&ma1s, a.x_perm, a.rows_cap, a.H) || !make_map_a16(&ma2s, a.h, a.rows_cap, a.F)))
     return cudaErrorInvalidValue;

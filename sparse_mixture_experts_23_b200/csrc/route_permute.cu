@@ -643,69 +643,39 @@ __global__ void __launch_bounds__(kRouterThreads) router_mma_kernel(RouterArgs a
                 reinterpret_cast<float*>(smem + P.misc + 8 * 256 * 4), blockIdx.x);
 }
 
-// Register-direct tensor-core router for bf16 with E = 8, 16 or 32, split over the hidden
-// dimension.  A cluster of S CTAs serves one 32-token chunk; CTA r of the cluster owns the hidden
-// columns [r*HS, (r+1)*HS), HS = H/S, and keeps only that slice of the gate weights (transposed,
-// Wg^T [E][HS]) in shared memory, so CTAs stay small and many of them stream x at once.  Lanes load
-// 16-byte vectors of x straight from HBM and feed them to mma.sync m16n8k16 without staging.  Lane
-// (g = lane/4, t = lane%4) loads the 8 columns [8t, 8t+8) of a 32-column block for token rows g and
-// g+8; the sum over h does not depend on its order, so the fragments use a permuted k (virtual pair
-// {2t, 2t+1} <-> columns {8t, 8t+1}, {2t+8, 2t+9} <-> {8t+2, 8t+3} in the first MMA; columns
-// 8t+4..8t+7 in the second) and the matching Wg^T vector (row e, columns 8t..8t+7) supplies both B
-// fragments.  The 8 warps split the slice; their partial logits are added in warp order, and the
-// S slices' partials are added in slice order in the leader CTA (rank 0), through distributed shared
-// memory, before the softmax / top-k tail.  Every sum runs in a fixed order, so results repeat bit
-// for bit and do not depend on S's scheduling.
+// Register-direct tensor-core router for bf16 with E = 8, 16 or 32 (gate weights resident in
+// shared memory): lanes load 16-byte vectors of x straight from HBM, deeply unrolled, and feed
+// them to mma.sync m16n8k16 without staging.  Lane (g = lane/4, t = lane%4) loads the 8 columns
+// [8t, 8t+8) of a 32-column block for token rows g and g+8; the sum over h does not depend on its
+// order, so the fragments use a permuted k (virtual pair {2t, 2t+1} <-> columns {8t, 8t+1},
+// {2t+8, 2t+9} <-> {8t+2, 8t+3} in the first MMA; columns 8t+4..8t+7 in the second) and the
+// matching Wg^T vector (row e, columns 8t..8t+7) supplies both B fragments.  Warps split H and
+// their partial logits are added in warp order.
 template <int NT8>
-struct SplitSmem {
+struct DirectSmem {
   static constexpr int E = NT8 * 8;
-  static __host__ __device__ int row_bytes(int HS) { return HS * 2 + 16; }  // Wg^T slice row, padded
-  static __host__ __device__ int red_off(int HS) { return E * row_bytes(HS); }
-  static __host__ __device__ int part_off(int HS) { return red_off(HS) + 8 * 32 * E * 4; }  // [S][32][E]
-  static __host__ __device__ int logits_off(int HS, int S) { return part_off(HS) + S * 32 * E * 4; }
-  static __host__ __device__ int psum_off(int HS, int S) { return logits_off(HS, S) + 32 * E * 4; }
-  static __host__ __device__ int misc_off(int HS, int S) { return psum_off(HS, S) + 8 * E * 4; }
-  static __host__ __device__ int total(int HS, int S) { return misc_off(HS, S) + (8 * 256 + 64) * 4; }
+  static __host__ __device__ int row_bytes(int H) { return H * 2 + 16; }  // Wg^T row, padded
+  static __host__ __device__ int red_off(int H) { return E * row_bytes(H); }
+  static __host__ __device__ int logits_off(int H) { return red_off(H) + 8 * 32 * E * 4; }
+  static __host__ __device__ int psum_off(int H) { return logits_off(H) + 32 * E * 4; }
+  static __host__ __device__ int misc_off(int H) { return psum_off(H) + 8 * E * 4; }
+  static __host__ __device__ int total(int H) { return misc_off(H) + (8 * 256 + 64) * 4; }
 };
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
-}
-// store v at the same shared-memory offset `addr` (this CTA's address space) in cluster CTA `rank`
-__device__ __forceinline__ void st_cluster_f32(uint32_t addr, uint32_t rank, float v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(addr), "r"(rank));
-  asm volatile("st.shared::cluster.f32 [%0], %1;\n" ::"r"(remote), "f"(v) : "memory");
-}
-
 template <int NT8>
-__global__ void __launch_bounds__(kRouterThreads) router_split_kernel(RouterArgs a, int S) {
-  using L = SplitSmem<NT8>;
-  constexpr int E = L::E;
+__global__ void __launch_bounds__(kRouterThreads) router_direct_kernel(RouterArgs a) {
+  using S = DirectSmem<NT8>;
+  constexpr int E = S::E;
   extern __shared__ __align__(16) unsigned char smem[];
   const int H = a.H, T = a.T;
-  const int HS = H / S;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;
-  const int RB = L::row_bytes(HS);
-  const int rank = S > 1 ? (int)cluster_rank() : 0;
-  const int chunk = blockIdx.x / S;
-  if (S > 1) cluster_arrive_relaxed();  // paired with the wait before the first remote store
+  const int RB = S::row_bytes(H);
 
-  const int t0 = chunk * kChunk;
+  const int t0 = blockIdx.x * kChunk;
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   const int rowvec = H / 8;  // 16-byte vectors per token row
+  // this lane's token rows: m-tile m, row g (+8)
   int rows[4];
   bool rvalid[4];
 #pragma unroll
@@ -724,9 +694,9 @@ __global__ void __launch_bounds__(kRouterThreads) router_split_kernel(RouterArgs
 #pragma unroll
       for (int q = 0; q < 4; ++q) acc[m][n][q] = 0.f;
 
-  const int nblk32 = HS / 32 / 8;                  // 32-column blocks per warp
-  const int b0 = rank * (HS / 32) + warp * nblk32; // first block (global, in 32-column units)
-  constexpr int U = 2;
+  const int nblk32 = H / 32 / 8;  // 32-column blocks per warp
+  const int b0 = warp * nblk32;
+  constexpr int U = 4;
   auto load_x = [&](uint4 (&xr)[U][4], int bb) {
 #pragma unroll
     for (int u = 0; u < U; ++u)
@@ -737,14 +707,13 @@ __global__ void __launch_bounds__(kRouterThreads) router_split_kernel(RouterArgs
                                                   : make_uint4(0, 0, 0, 0);
       }
   };
-  uint4 xr[U][4], xr2[U][4];
-  load_x(xr, 0);  // the first x loads go out before the gate slice is staged
-  if (U < nblk32) load_x(xr2, U);
+  uint4 xr[U][4];
+  load_x(xr, 0);  // first x loads go out before the gate weights are staged
 
-  // Wg [H][E] rows of this slice -> Wg^T [E][HS] (bf16); each thread issues all its loads first
+  // Wg [H][E] -> Wg^T [E][H] (bf16) in shared memory; each thread issues all its loads first
   {
-    const uint4* src = reinterpret_cast<const uint4*>(a.Wg) + (size_t)rank * HS * E / 8;
-    const int nvec = HS * E / 8;
+    const uint4* src = reinterpret_cast<const uint4*>(a.Wg);
+    const int nvec = H * E / 8;
     for (int i0 = tid; i0 < nvec; i0 += kRouterThreads * 8) {
       uint4 v[8];
 #pragma unroll
@@ -766,17 +735,17 @@ __global__ void __launch_bounds__(kRouterThreads) router_split_kernel(RouterArgs
   }
   __syncthreads();
 
-  auto compute = [&](const uint4 (&xr_)[U][4], int bb) {
+  auto compute = [&](const uint4 (&xr)[U][4], int bb) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       if (bb + u >= nblk32) break;
-      const int h0 = (warp * nblk32 + bb + u) * 32;  // column inside the slice
+      const int h0 = (b0 + bb + u) * 32;
 #pragma unroll
       for (int n = 0; n < NT8; ++n) {
         const uint4 w = *reinterpret_cast<const uint4*>(smem + (n * 8 + g) * RB + (h0 + 8 * t4) * 2);
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
-          const uint4 xa = xr_[u][2 * m], xb = xr_[u][2 * m + 1];
+          const uint4 xa = xr[u][2 * m], xb = xr[u][2 * m + 1];
           mma_16816(acc[m][n], xa.x, xb.x, xa.y, xb.y, w.x, w.y);
           mma_16816(acc[m][n], xa.z, xb.z, xa.w, xb.w, w.z, w.w);
         }
@@ -784,14 +753,15 @@ __global__ void __launch_bounds__(kRouterThreads) router_split_kernel(RouterArgs
     }
   };
   // two register groups alternate: the next group's loads are in flight while one is computed
+  uint4 xr2[U][4];
   for (int bb = 0; bb < nblk32; bb += 2 * U) {
+    if (bb + U < nblk32) load_x(xr2, bb + U);
     compute(xr, bb);
     if (bb + 2 * U < nblk32) load_x(xr, bb + 2 * U);
     if (bb + U < nblk32) compute(xr2, bb + U);
-    if (bb + 3 * U < nblk32) load_x(xr2, bb + 3 * U);
   }
-  // per-warp partials -> shared, then a fixed-order sum over warps
-  float* red = reinterpret_cast<float*>(smem + L::red_off(HS));
+  // per-warp partials -> shared, then a fixed-order sum over warps (+ bias)
+  float* red = reinterpret_cast<float*>(smem + S::red_off(H));
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -803,32 +773,17 @@ __global__ void __launch_bounds__(kRouterThreads) router_split_kernel(RouterArgs
         red[(warp * 32 + row) * E + col] = acc[m][n][q];
       }
   __syncthreads();
-  float* part = reinterpret_cast<float*>(smem + L::part_off(HS));  // [S][32][E], filled in the leader
-  if (S > 1) cluster_wait_acquire();  // every CTA of the cluster has started: remote stores are safe
+  float* logits = reinterpret_cast<float*>(smem + S::logits_off(H));
+  const __nv_bfloat16* bg = reinterpret_cast<const __nv_bfloat16*>(a.bg);
   for (int o = tid; o < 32 * E; o += kRouterThreads) {
     float v = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) v += red[w * 32 * E + o];
-    if (S > 1) st_cluster_f32((uint32_t)__cvta_generic_to_shared(part + rank * 32 * E + o), 0, v);
-    else part[o] = v;
-  }
-  if (S > 1) {
-    cluster_arrive_release();  // this slice's partial is in the leader
-    cluster_wait_acquire();
-    if (rank != 0) return;     // nothing of a non-leader is read after this point
-  }
-  float* logits = reinterpret_cast<float*>(smem + L::logits_off(HS, S));
-  const __nv_bfloat16* bg = reinterpret_cast<const __nv_bfloat16*>(a.bg);
-  __syncthreads();
-  for (int o = tid; o < 32 * E; o += kRouterThreads) {
-    float v = 0.f;
-    for (int r = 0; r < S; ++r) v += part[r * 32 * E + o];
     logits[o] = v + (bg ? __bfloat162float(bg[o % E]) : 0.f);
   }
   __syncthreads();
-  router_finish(a, logits, E, reinterpret_cast<float*>(smem + L::psum_off(HS, S)),
-                reinterpret_cast<int*>(smem + L::misc_off(HS, S)),
-                reinterpret_cast<float*>(smem + L::misc_off(HS, S) + 8 * 256 * 4), chunk);
+  router_finish(a, logits, E, reinterpret_cast<float*>(smem + S::psum_off(H)), reinterpret_cast<int*>(smem + S::misc_off(H)),
+                reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4), blockIdx.x);
 }
 
 // Softmax, top-k, renormalisation and partials of one 32-token chunk from logits that a tensor-core
@@ -872,26 +827,8 @@ __global__ void hist_kernel(const int32_t* __restrict__ topk_idx, int T, int E, 
   }
 }
 
-// Sum of v[(c0 + i) * stride] for i < n, loaded in batches of kBatch independent loads so that a
-// thread's chain of L2 round trips is n / kBatch long, not n.
-constexpr int kBatch = 16;
-template <typename V>
-__device__ __forceinline__ V strided_sum(const V* __restrict__ v, long long c0, int n, int stride) {
-  V s = V(0);
-  for (int i0 = 0; i0 < n; i0 += kBatch) {
-    V r[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) r[u] = i0 + u < n ? v[(size_t)(c0 + i0 + u) * stride] : V(0);
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) s += r[u];  // fixed order: the same sum on every run
-  }
-  return s;
-}
-
 // One block: losses from the router partials, per-expert totals, capacity, offsets and the
-// exclusive scan of the chunk histograms in (slot, chunk) order.  Thread (g, e) owns a contiguous
-// range of chunks (and of router blocks) for expert e; every range is read with batched
-// independent loads, and the cross-group scans and sums run in shared memory.
+// exclusive scan of the chunk histograms in (slot, chunk) order.
 __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
   __shared__ int gsum[1024];
   __shared__ int cnt_s[256];
@@ -915,7 +852,8 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
     }
     __syncthreads();
   } else {
-    const int s = in ? strided_sum(a.chunk_hist + e, c0, c1 - c0, E) : 0;
+    int s = 0;
+    for (int c = c0; c < c1; ++c) s += a.chunk_hist[(size_t)c * E + e];
     if (in) gsum[g * E + e] = s;
     __syncthreads();
     // exclusive scan of the G group sums of each expert: warp w scans experts w, w+32, ...; lane l
@@ -948,55 +886,36 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
     __syncthreads();
   }
   if (a.do_dispatch && in) {
-    // the group's chunk bases: its values again, batch by batch, with the running prefix
     int run = gsum[g * E + e];
-    for (int i0 = c0; i0 < c1; i0 += kBatch) {
-      int r[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) r[u] = i0 + u < c1 ? a.chunk_hist[(size_t)(i0 + u) * E + e] : 0;
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-        if (i0 + u < c1) {
-          a.chunk_base[(size_t)(i0 + u) * E + e] = run;
-          run += r[u];
-        }
+    for (int c = c0; c < c1; ++c) {
+      int v = a.chunk_hist[(size_t)c * E + e];
+      a.chunk_base[(size_t)c * E + e] = run;
+      run += v;
     }
   }
-  if (a.do_dispatch && tid < 32) {
-    // offsets: exclusive scan of the kept counts over the experts, lane l owning a run of experts
-    const int lane = tid, epl = (E + 31) / 32;
-    const int q0 = min(E, lane * epl), q1 = min(E, q0 + epl);
-    int local = 0;
-    for (int q = q0; q < q1; ++q) {
-      const long long c = cnt_s[q];
-      local += (a.cap >= 0 && c > a.cap) ? (int)a.cap : (int)c;
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    int run = incl - local;
-    for (int q = q0; q < q1; ++q) {
-      const long long c = cnt_s[q];
-      const int kept = (a.cap >= 0 && c > a.cap) ? (int)a.cap : (int)c;
+  if (a.do_dispatch && tid == 0) {
+    int run = 0;
+    for (int q = 0; q < E; ++q) {
+      long long c = cnt_s[q];
+      int kept = (a.cap >= 0 && c > a.cap) ? (int)a.cap : (int)c;
       a.expert_counts[q] = kept;
       a.offsets[q] = run;
       run += kept;
     }
-    if (lane == 31) a.offsets[E] = incl;
+    a.offsets[E] = run;
   }
   if (a.do_losses) {
     // P_e: thread (g, e) sums a fixed range of router blocks, then the group sums are added in
-    // group order; z: each thread a fixed contiguous range, then a fixed tree.  Same order on every run.
+    // group order; z: thread-strided sums then a fixed tree.  Same order on every run.
     {
       const int b0 = in ? (int)((long long)a.nblk * g / G) : 0;
       const int b1 = in ? (int)((long long)a.nblk * (g + 1) / G) : 0;
-      const float ps = in ? strided_sum(a.loss_part + e, b0, b1 - b0, E + 1) : 0.f;
+      float ps = 0.f;
+      for (int b = b0; b < b1; ++b) ps += a.loss_part[(size_t)b * (E + 1) + e];
       if (in) pf[g * E + e] = ps;
-      const int z0 = (int)((long long)a.nblk * tid / 1024), z1 = (int)((long long)a.nblk * (tid + 1) / 1024);
-      zf[tid] = strided_sum(a.loss_part + E, z0, z1 - z0, E + 1);
+      float zs = 0.f;
+      for (int b = tid; b < a.nblk; b += 1024) zs += a.loss_part[(size_t)b * (E + 1) + E];
+      zf[tid] = zs;
     }
     __syncthreads();
     for (int w = 512; w >= 32; w >>= 1) {
@@ -1026,18 +945,11 @@ __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
       }
     }
     __syncthreads();
-    if (tid < 32) {
-      // aux = E * sum_e term[e]: lane l sums its run of experts, then a fixed tree
-      const int lane = tid, epl = (E + 31) / 32;
-      const int q0 = min(E, lane * epl), q1 = min(E, q0 + epl);
+    if (tid == 0) {
       double sum = 0.0;
-      for (int q = q0; q < q1; ++q) sum += term[q];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) {
-        *a.aux_loss = (float)((double)E * sum);
-        *a.z_loss = (float)((double)zred[0] / (double)a.T);
-      }
+      for (int q = 0; q < E; ++q) sum += term[q];
+      *a.aux_loss = (float)((double)E * sum);
+      *a.z_loss = (float)((double)zred[0] / (double)a.T);
     }
   }
 }
@@ -1165,35 +1077,6 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 // moe_set_kernel_options(MOE_KERNEL_NO_TC_GATE) selects the CUDA-core routers (for comparisons).
 bool router_mma_disabled() { return (kernel_options() & MOE_KERNEL_NO_TC_GATE) != 0; }
 
-// Hidden-dimension slices per chunk for the split router: the smallest power of two S that leaves each
-// warp at most 4 blocks of 32 columns (so a lane's x loads are all in flight at once), then doubled
-// while the grid is below two CTAs per SM; at most 8 (a portable cluster), H divisible by 256*S.
-int split_router_slices(int H, int nchunk, int num_sms) {
-  int S = 1;
-  while (S < 8 && H % (512 * S) == 0 && H / (256 * S) > 4) S *= 2;
-  while (S < 8 && H % (512 * S) == 0 && (long long)nchunk * S < 2LL * num_sms) S *= 2;
-  return S;
-}
-
-template <int NT8>
-cudaError_t launch_split(const RouterArgs& a, int nchunk, int S, int bytes, cudaStream_t st) {
-  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(router_split_kernel<NT8>), bytes);
-  if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3((unsigned)(nchunk * S), 1, 1);
-  cfg.blockDim = dim3(kRouterThreads, 1, 1);
-  cfg.dynamicSmemBytes = (size_t)bytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, router_split_kernel<NT8>, a, S);
-}
-
 template <int EP>
 cudaError_t launch_stream(const RouterArgs& a, int nblk, cudaStream_t st) {
   const int bytes = StreamSmem<EP>::total(a.H);
@@ -1208,10 +1091,14 @@ cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* 
   // the tcgen05 gate kernels wait on pipeline barriers with a bound, and record a wait that ran out
   // in a device error word: without one (or without a bound) they are not used
   const bool tc_gate_ok = a.status != nullptr && a.wait_limit > 0 && !router_mma_disabled();
-  // bf16, token choice, E = 64, 128 or 256: one tensor-core GEMM whose epilogue does the whole
-  // softmax / top-k / partials tail (the logits never leave the SM)
+  const int sms = a.num_sms > 0 ? a.num_sms : 148;
+  // bf16, token choice, E = 64, 128 or 256, and enough 128-token tiles to fill at least half the SMs:
+  // one tensor-core GEMM whose epilogue does the whole softmax / top-k / partials tail (the logits
+  // never leave the SM).  With fewer tiles each CTA's short k-loop is latency-bound (the Switch shape:
+  // 64 tiles of K = 1024 took 36.5 us against 23 us for the two-kernel form below), so the
+  // 64-column-tile GEMM + per-chunk tail keeps more SMs streaming.
   if (dtype == MOE_DTYPE_BF16 && a.scores == nullptr && (a.E == 64 || a.E == 128 || a.E == 256) && a.H % 64 == 0 &&
-      a.k <= 8 && tc_gate_ok) {
+      a.k <= 8 && tc_gate_ok && 2 * ((a.T + 127) / 128) >= sms) {
     ++*launches;
     return launch_gate_router_sm100(a, st);
   }
@@ -1230,16 +1117,19 @@ cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* 
     return cudaGetLastError();
   }
   ++*launches;  // every other form is one kernel
-  // bf16, E in {8, 16, 32}: register-direct tensor-core stream over x, the hidden dimension split
-  // over a cluster of S CTAs per chunk
+  // bf16, E in {8, 16, 32}, Wg^T fits in shared memory: register-direct tensor-core stream over x
   if (dtype == MOE_DTYPE_BF16 && (a.E == 8 || a.E == 16 || a.E == 32) && a.H % 256 == 0 && !router_mma_disabled()) {
-    const int S = split_router_slices(a.H, nblk, a.num_sms > 0 ? a.num_sms : 148);
-    const int HS = a.H / S;
-    const int bytes = a.E == 8 ? SplitSmem<1>::total(HS, S) : (a.E == 16 ? SplitSmem<2>::total(HS, S) : SplitSmem<4>::total(HS, S));
+    const int bytes = a.E == 8 ? DirectSmem<1>::total(a.H) : (a.E == 16 ? DirectSmem<2>::total(a.H) : DirectSmem<4>::total(a.H));
     if (bytes <= 200 * 1024) {
-      if (a.E == 8) return launch_split<1>(a, nblk, S, bytes, st);
-      if (a.E == 16) return launch_split<2>(a, nblk, S, bytes, st);
-      return launch_split<4>(a, nblk, S, bytes, st);
+      const void* kern = a.E == 8 ? reinterpret_cast<const void*>(router_direct_kernel<1>)
+                                  : (a.E == 16 ? reinterpret_cast<const void*>(router_direct_kernel<2>)
+                                               : reinterpret_cast<const void*>(router_direct_kernel<4>));
+      cudaError_t err = ensure_smem_limit(kern, bytes);
+      if (err != cudaSuccess) return err;
+      if (a.E == 8) router_direct_kernel<1><<<nblk, kRouterThreads, bytes, st>>>(a);
+      else if (a.E == 16) router_direct_kernel<2><<<nblk, kRouterThreads, bytes, st>>>(a);
+      else router_direct_kernel<4><<<nblk, kRouterThreads, bytes, st>>>(a);
+      return cudaGetLastError();
     }
   }
   // bf16 with E a multiple of 8: tensor-core gate tile staged through shared memory

@@ -142,10 +142,12 @@ def fro_rel(a: np.ndarray, ref: np.ndarray) -> float:
     return num / den if den > 0 else num
 
 
-def router_launches(cfg) -> int:
-    """Kernels of the gate: one, except under expert choice with a bf16 layer whose expert count is a
-    multiple of 64, where a tensor-core logits GEMM is followed by the per-chunk softmax kernel (under
-    token choice the 64/128/256-expert gate does its softmax and top-k in the GEMM's epilogue)."""
-    if cfg.dtype == "bf16" and cfg.E % 64 == 0 and cfg.routing == "expert_choice":
-        return 2
-    return 1
+def router_launches(cfg, sms: int = 148) -> int:
+    """Kernels of the gate: one, or two (a tensor-core logits GEMM, then the per-chunk softmax / top-k
+    kernel) for bf16 layers whose expert count is a multiple of 64 -- except under token choice with 64,
+    128 or 256 experts and at least sms/2 tiles of 128 tokens, where the softmax / top-k runs in the
+    GEMM's epilogue (one kernel)."""
+    if cfg.dtype != "bf16" or cfg.E % 64 != 0:
+        return 1
+    fused = cfg.routing == "token_choice" and cfg.E in (64, 128, 256) and 2 * ((cfg.T + 127) // 128) >= sms
+    return 1 if fused else 2
