@@ -559,7 +559,8 @@ def run_ours_impl(args, cfg):
             xh = xh.view(torch.bfloat16)
         return xh.pin_memory(), torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
 
-    hosts = [host_pair(), host_pair()]
+    NBUF = 3  # buffer sets for the pipelined figure (triple buffering)
+    hosts = [host_pair() for _ in range(NBUF)]
     for _ in range(2):
         buf.forward_host(*hosts[0])
     sync_all()
@@ -571,20 +572,24 @@ def run_ours_impl(args, cfg):
     sync_all()
     ms_e2e_serial = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
 
-    inputs2 = dict(buf.inputs)
-    inputs2["x"] = torch.empty_like(buf.inputs["x"])  # moe_forward_host writes the step's x here
-    buf2 = moe.MoEBuffers(shape, inputs2)
-    bufs = (buf, buf2)
-    streams = (torch.cuda.Stream(), torch.cuda.Stream())
+    extra = []
+    for _ in range(NBUF - 1):
+        inputs_j = dict(buf.inputs)
+        inputs_j["x"] = torch.empty_like(buf.inputs["x"])  # moe_forward_host writes the step's x here
+        extra.append(moe.MoEBuffers(shape, inputs_j))
+    bufs = [buf] + extra
+    streams = [torch.cuda.Stream() for _ in range(NBUF)]
 
     def pipelined(n):
+        # step i runs on buffer set i % NBUF and its own stream: the copies of one step overlap the
+        # kernels of the others, and a set's next input copy waits only for its own previous output
         for i in range(n):
-            with torch.cuda.stream(streams[i % 2]):
-                bufs[i % 2].forward_host(*hosts[i % 2])
+            with torch.cuda.stream(streams[i % NBUF]):
+                bufs[i % NBUF].forward_host(*hosts[i % NBUF])
 
     for s_ in streams:
         s_.wait_stream(torch.cuda.current_stream())
-    pipelined(4)
+    pipelined(2 * NBUF)
     sync_all()
     e0.record(stream)
     for s_ in streams:
@@ -597,9 +602,9 @@ def run_ours_impl(args, cfg):
     ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
     e2e_value = aggregate_rate(world, cfg.T, args.steps, ms_e2e)
     e2e_serial = aggregate_rate(world, cfg.T, args.steps, ms_e2e_serial)
-    out_diff = float((hosts[0][1] - hosts[1][1]).abs().max())  # both buffer sets ran the same x
-    e2e_status = max(buf.device_status(), buf2.device_status())
-    del buf2, inputs2
+    out_diff = max(float((hosts[0][1] - h[1]).abs().max()) for h in hosts[1:])  # every set ran the same x
+    e2e_status = max(b.device_status() for b in bufs)
+    del extra, bufs
     # losses of the whole job's batch: every replica's loss sums all-reduced (one small collective,
     # outside the timed regions; with one GPU these are this batch's own losses)
     buf.forward()
@@ -669,7 +674,7 @@ def run_ours_impl(args, cfg):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": cfg.T * cfg.H * es,
                 "d2h_bytes_per_step": cfg.T * cfg.H * 4, "api": "moe_forward_host",
-                "mode": "pipelined: 2 buffer sets on 2 streams, steps alternate", "serial_value": e2e_serial,
+                "mode": f"pipelined: {NBUF} buffer sets on {NBUF} streams, steps rotate", "serial_value": e2e_serial,
                 "max_abs_diff_across_buffer_sets": out_diff, "device_status": e2e_status},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
