@@ -8,8 +8,8 @@ whole forward pass (router, permutation, both grouped GEMMs with the fused combi
 C-ABI call moe_forward; inputs are resident in HBM when the timed region starts.  The expert
 weights (1.88 GB) stream through L2 every step, so the inputs are larger than L2 and no flush is
 needed.  ``e2e`` times moe_forward_host: per step it copies x from pinned host memory to the device
-and out back to pinned host memory; two buffer sets on two streams let one step's copies overlap the
-other's kernels (the one-stream figure is reported beside it).  With N GPUs (torchrun), every rank runs its own replica on its
+and out back to pinned host memory; three buffer sets on three streams let one step's copies overlap
+the other steps' kernels (the one-stream figure is reported beside it).  With N GPUs (torchrun), every rank runs its own replica on its
 own batch (no data-path collective; the layer shards by tokens), timing is the max over ranks.
 
 ``--impl reference`` times the fp64 CPU oracle on the host cores on a bounded token sample of the
@@ -463,13 +463,11 @@ def run_ours_impl(args, cfg):
     # ---------------- per-kernel timing (same stream, CUDA events, inputs > L2) ---------------
     reps = min(max(args.steps, 20), 200)
 
-    def time_calls(fn, min_seconds: float = 0.0, clock_name: str | None = None, reps: int = reps,
-                   settle: float = 0.0) -> float:
-        """Average device time of one call: `reps` calls captured in a CUDA graph and replayed, so
+    def time_calls(fn, clock_name: str | None = None, reps: int = reps, settle: float = 0.0) -> float:
+        """Average device time of one call: `reps` calls captured in a CUDA graph and replayed once, so
         host-side launch cost does not enter (plain back-to-back calls when capture fails).  With
-        min_seconds, the graph is replayed until that much device time has passed and the average
-        covers every replay; with clock_name, nvidia-smi samples the clocks over exactly those
-        replays (rank 0) and the summary is kept in kernel_clocks[clock_name]."""
+        settle, an idle pause comes first; with clock_name, the clocks are sampled over exactly that
+        replay (rank 0) and the summary is kept in kernel_clocks[clock_name]."""
         for _ in range(2):
             fn()
         torch.cuda.synchronize()
@@ -504,22 +502,12 @@ def run_ours_impl(args, cfg):
         run_once()
         b.record(stream)
         torch.cuda.synchronize()
-        total_ms, n = a.elapsed_time(b), 1
-        if min_seconds > 0:
-            more = max(0, int(math.ceil(min_seconds * 1000.0 / max(total_ms, 1e-3))) - 1)
-            a.record(stream)
-            for _ in range(more):
-                run_once()
-            b.record(stream)
-            torch.cuda.synchronize()
-            if more:
-                total_ms += a.elapsed_time(b)
-                n += more
+        total_ms = a.elapsed_time(b)
         if smp is not None:
             smp.mark(th0, time.time())
             kernel_clocks[clock_name] = smp.stop()
         del g
-        return total_ms / (reps * n)
+        return total_ms / reps
 
     kernel_clocks = {}
     # the dominant kernel pair, timed alone with its own clock record: as many back-to-back calls as
