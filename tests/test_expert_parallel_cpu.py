@@ -6,7 +6,6 @@ the counts all-gather, the plan, both all-to-alls and the regrouping between the
 expert-major layouts.  Every rank's output must equal the oracle's whole layer on that rank's own batch
 (capacity per rank) -- the statement that expert placement changes where the arithmetic runs, not what
 it computes."""
-import math
 import os
 import socket
 

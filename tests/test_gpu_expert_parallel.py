@@ -18,7 +18,7 @@ import pytest
 
 import oracle
 import synth
-from moe_testlib import NEAR_TIE, TOL_BF16_RMS, out_error, rms_rel, shape_of, to_device, upload
+from moe_testlib import NEAR_TIE, out_error, rms_rel, shape_of, to_device, upload
 
 pytestmark = pytest.mark.gpu
 
