@@ -460,6 +460,72 @@ def run_ours_impl(args, cfg):
     ms_step = ms_total / args.steps
     value = aggregate_rate(world, cfg.T, args.steps, ms_total)
 
+    # ---------------- e2e: host buffers through moe_forward_host ----------------------------
+    # Every step copies its x from pinned host memory, runs the layer and copies out back to pinned
+    # host memory, all inside the timed region.  "serial": one stream, so each step's copies wait for
+    # the previous step's kernels.  "pipelined" (the reported value): three device buffer sets on
+    # three streams, steps rotating between them, so the host copies of some steps run on the copy
+    # engines while another step's kernels run -- what a caller streaming batches through the layer
+    # does (calls on distinct workspaces may run concurrently on distinct streams).  Both run right
+    # after the device-timed region and an idle pause, before the power-capped GEMM loops below.
+    es = 2 if cfg.dtype == "bf16" else 4
+    x_np = np.ascontiguousarray(inp.x).view(np.int16 if es == 2 else np.float32)
+
+    def host_pair():
+        xh = torch.from_numpy(x_np.copy())
+        if es == 2:
+            xh = xh.view(torch.bfloat16)
+        return xh.pin_memory(), torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
+
+    NBUF = 3  # buffer sets for the pipelined figure (triple buffering)
+    hosts = [host_pair() for _ in range(NBUF)]
+    for _ in range(2):
+        buf.forward_host(*hosts[0])
+    sync_all()
+    time.sleep(0.5)  # rested clocks, as for the device-timed region
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        buf.forward_host(*hosts[0])
+    e1.record(stream)
+    sync_all()
+    ms_e2e_serial = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+
+    extra = []
+    for _ in range(NBUF - 1):
+        inputs_j = dict(buf.inputs)
+        inputs_j["x"] = torch.empty_like(buf.inputs["x"])  # moe_forward_host writes the step's x here
+        extra.append(moe.MoEBuffers(shape, inputs_j))
+    bufs = [buf] + extra
+    streams = [torch.cuda.Stream() for _ in range(NBUF)]
+
+    def pipelined(n):
+        # step i runs on buffer set i % NBUF and its own stream: the copies of one step overlap the
+        # kernels of the others, and a set's next input copy waits only for its own previous output
+        for i in range(n):
+            with torch.cuda.stream(streams[i % NBUF]):
+                bufs[i % NBUF].forward_host(*hosts[i % NBUF])
+
+    for s_ in streams:
+        s_.wait_stream(torch.cuda.current_stream())
+    pipelined(2 * NBUF)
+    sync_all()
+    time.sleep(0.5)
+    e0.record(stream)
+    for s_ in streams:
+        s_.wait_event(e0)
+    pipelined(args.steps)
+    for s_ in streams:
+        stream.wait_stream(s_)
+    e1.record(stream)
+    sync_all()
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
+    e2e_value = aggregate_rate(world, cfg.T, args.steps, ms_e2e)
+    e2e_serial = aggregate_rate(world, cfg.T, args.steps, ms_e2e_serial)
+    out_diff = max(float((hosts[0][1] - h[1]).abs().max()) for h in hosts[1:])  # every set ran the same x
+    e2e_status = max(b.device_status() for b in bufs)
+    del extra, bufs
+
     # ---------------- per-kernel timing (same stream, CUDA events, inputs > L2) ---------------
     reps = min(max(args.steps, 20), 200)
 
@@ -531,68 +597,6 @@ def run_ours_impl(args, cfg):
     drops = int(buf.dropped.cpu().numpy().sum())
     losses = buf.losses.cpu().numpy()
 
-    # ---------------- e2e: host buffers through moe_forward_host ----------------------------
-    # Every step copies its x from pinned host memory, runs the layer and copies out back to pinned
-    # host memory, all inside the timed region.  "serial": one stream, so each step's copies wait for
-    # the previous step's kernels.  "pipelined" (the reported value): two device buffer sets on two
-    # streams, steps alternating between them, so one step's host copies run on the copy engines
-    # while the other step's kernels run -- what a caller streaming batches through the layer does
-    # (calls on distinct workspaces may run concurrently on distinct streams).
-    es = 2 if cfg.dtype == "bf16" else 4
-    x_np = np.ascontiguousarray(inp.x).view(np.int16 if es == 2 else np.float32)
-
-    def host_pair():
-        xh = torch.from_numpy(x_np.copy())
-        if es == 2:
-            xh = xh.view(torch.bfloat16)
-        return xh.pin_memory(), torch.empty((cfg.T, cfg.H), dtype=torch.float32).pin_memory()
-
-    NBUF = 3  # buffer sets for the pipelined figure (triple buffering)
-    hosts = [host_pair() for _ in range(NBUF)]
-    for _ in range(2):
-        buf.forward_host(*hosts[0])
-    sync_all()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        buf.forward_host(*hosts[0])
-    e1.record(stream)
-    sync_all()
-    ms_e2e_serial = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
-
-    extra = []
-    for _ in range(NBUF - 1):
-        inputs_j = dict(buf.inputs)
-        inputs_j["x"] = torch.empty_like(buf.inputs["x"])  # moe_forward_host writes the step's x here
-        extra.append(moe.MoEBuffers(shape, inputs_j))
-    bufs = [buf] + extra
-    streams = [torch.cuda.Stream() for _ in range(NBUF)]
-
-    def pipelined(n):
-        # step i runs on buffer set i % NBUF and its own stream: the copies of one step overlap the
-        # kernels of the others, and a set's next input copy waits only for its own previous output
-        for i in range(n):
-            with torch.cuda.stream(streams[i % NBUF]):
-                bufs[i % NBUF].forward_host(*hosts[i % NBUF])
-
-    for s_ in streams:
-        s_.wait_stream(torch.cuda.current_stream())
-    pipelined(2 * NBUF)
-    sync_all()
-    e0.record(stream)
-    for s_ in streams:
-        s_.wait_event(e0)
-    pipelined(args.steps)
-    for s_ in streams:
-        stream.wait_stream(s_)
-    e1.record(stream)
-    sync_all()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world, "cuda")
-    e2e_value = aggregate_rate(world, cfg.T, args.steps, ms_e2e)
-    e2e_serial = aggregate_rate(world, cfg.T, args.steps, ms_e2e_serial)
-    out_diff = max(float((hosts[0][1] - h[1]).abs().max()) for h in hosts[1:])  # every set ran the same x
-    e2e_status = max(b.device_status() for b in bufs)
-    del extra, bufs
     # losses of the whole job's batch: every replica's loss sums all-reduced (one small collective,
     # outside the timed regions; with one GPU these are this batch's own losses)
     buf.forward()

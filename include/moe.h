@@ -186,11 +186,13 @@ MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, mo
 /* Router ("MoE Training" page, Quick Start MoELayer.forward: gate, softmax, topk, renormalise;
  * Core Concepts 3: load_balancing_loss, router_z_loss).
  * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws).
- * Token choice: 2 launches (the gate with its softmax / top-k tail, then the loss reduction).  bf16
- * layers with 8, 16 or 32 experts run the gate as register-fed mma.sync over x; bf16 layers whose
- * expert count is a multiple of 64 run it as a tcgen05 GEMM into the workspace followed by the
- * per-chunk softmax / top-k (one launch more), or -- with 64, 128 or 256 experts and at least one
- * 128-token tile per two SMs -- as one tcgen05 GEMM whose epilogue does the softmax / top-k.
+ * Token choice: 1 launch, the gate with its softmax / top-k tail, whose last block to finish also
+ * reduces the loss partials (a workspace counter beside the error word picks that block).  bf16
+ * layers with 8 or 16 experts stream x through a shared-memory ring of bulk copies into mma.sync
+ * (32 experts: register-fed mma.sync); bf16 layers whose expert count is a multiple of 64 run the
+ * gate as a tcgen05 GEMM into the workspace followed by the per-chunk softmax / top-k (one launch
+ * more), or -- with 64, 128 or 256 experts and at least one 128-token tile per two SMs -- as one
+ * tcgen05 GEMM whose epilogue does the softmax / top-k, followed by one reduce launch.
  * Expert choice: also the per-expert selection (Core Concepts 2), so it writes the chosen tokens
  * to topk_idx[E,C], expert_counts and dropped[T] as well; 3 launches, one more for bf16 layers whose
  * expert count is a multiple of 64. */
@@ -213,7 +215,8 @@ MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, voi
  * capture.  Later calls made outside stream capture look the address up again, so a context that
  * was reset and rebuilt (cudaDeviceReset) is served its new address.  Every call, on every stream,
  * shares the one array and leaves the last call's contents in it: calls that overlap on the GPU
- * race, so serialise them (one stream, or events).  2 launches (1 when T = 0); one NVTX range.
+ * race, so serialise them (one stream, or events).  1 launch (2 with the one-GEMM gate of 64, 128
+ * or 256 experts, whose reduction is a launch of its own); one NVTX range.
  * Token choice only: an expert-choice shape returns MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream);
 
@@ -244,7 +247,8 @@ MOE_API moe_status_t moe_losses_from_sums(int E, const float* sums, float* aux_l
  * Mixtral block gather by expert).  Assignments are visited slot-major then by token; an
  * assignment is kept iff fewer than `capacity` earlier assignments went to its expert.
  * Reads x, topk_idx.  Writes expert_counts, dropped, the row maps and x_perm in ws, and clears
- * out[T,H] to zero (the fused combine accumulates into it).  The kernels check every index they
+ * out[T,H] to zero (the fused combine accumulates into it).  Token choice: 2 launches, per-chunk
+ * histograms (the last block also scans them into offsets) and the scatter; expert choice: 1.  The kernels check every index they
  * read from topk_idx (see moe_get_device_status); nothing outside the buffers is touched.
  * Expert choice: nothing is dropped (each expert already holds exactly C tokens); reads x and
  * topk_idx[E,C], writes the row maps and x_perm, and clears out. */
@@ -272,8 +276,10 @@ MOE_API moe_status_t moe_expert_ffn(const moe_shape_t* shape, const moe_io_t* io
 MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
-/* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream (5 launches; one
- * more under expert choice, and one more for the two-kernel tensor-core gate described at moe_route). */
+/* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream.  Token choice: the gate
+ * (whose last block reduces the losses and the dispatch), the scatter, GEMM1 and GEMM2: 4 launches,
+ * 5 with either tensor-core gate form of moe_route.  Expert choice: 6 launches, 7 with the
+ * two-kernel tensor-core gate. */
 MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);
 
@@ -396,9 +402,17 @@ MOE_API moe_status_t moe_expert_ffn_rows(const moe_shape_t* shape, int64_t rows_
  *                           256 x 256 tiles the long-segment shapes use (forward and backward GEMMs)
  *   MOE_KERNEL_NO_TC_GATE   the CUDA-core gate kernels instead of the tensor-core ones (mma.sync for
  *                           8/16/32 experts, the tcgen05 GEMM for multiples of 64)
+ *   MOE_KERNEL_NO_TMA_ROUTER  for bf16 with 8 or 16 experts, the register-direct mma.sync gate (x loaded
+ *                           into registers) instead of the one that streams x through a shared-memory
+ *                           ring of bulk copies
  * Default 0.  Process-wide; applies to launches made after the call, from any host thread.  Results
  * stay within the same tolerances of the definition either way; unknown bits are ignored. */
-typedef enum { MOE_KERNEL_DEFAULT = 0, MOE_KERNEL_NO_CTA_PAIR = 1, MOE_KERNEL_NO_TC_GATE = 2 } moe_kernel_flags_t;
+typedef enum {
+  MOE_KERNEL_DEFAULT = 0,
+  MOE_KERNEL_NO_CTA_PAIR = 1,
+  MOE_KERNEL_NO_TC_GATE = 2,
+  MOE_KERNEL_NO_TMA_ROUTER = 4
+} moe_kernel_flags_t;
 MOE_API void moe_set_kernel_options(int flags);
 MOE_API int moe_get_kernel_options(void);
 

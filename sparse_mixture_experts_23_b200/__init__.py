@@ -31,7 +31,7 @@ ENTRY_POINTS = (
     "moe_set_kernel_options", "moe_get_kernel_options", "moe_copy_row_segments", "moe_expert_ffn_rows",
     "moe_expert_ffn_rows_workspace_size",
 )
-MOE_KERNEL_DEFAULT, MOE_KERNEL_NO_CTA_PAIR, MOE_KERNEL_NO_TC_GATE = 0, 1, 2
+MOE_KERNEL_DEFAULT, MOE_KERNEL_NO_CTA_PAIR, MOE_KERNEL_NO_TC_GATE, MOE_KERNEL_NO_TMA_ROUTER = 0, 1, 2, 4
 
 
 class MoEError(RuntimeError):

@@ -193,7 +193,10 @@ int num_sms() {
 
 // ---------------------------------------------------------------- stage bodies (validated) -------
 ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int do_losses, int do_dispatch);
-moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, bool emit_hist,
+// reduce: which reductions follow the router (kReduceLosses, kReduceDispatch; token choice only).  The
+// router's last block runs them when the chosen router kernel can, else one reduce launch follows.
+constexpr int kReduceLosses = 1, kReduceDispatch = 2;
+moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, int reduce,
                       bool train = false) {
   const WsLayout L = ws_layout(*s);
   if (s->T == 0) {
@@ -213,7 +216,6 @@ moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaSt
   r.loss_part = at<float>(ws, L.loss_part);
   r.chunk_hist = at<int32_t>(ws, L.chunk_hist);
   r.logits_out = train ? at<float>(ws, L.logits) : nullptr;
-  (void)emit_hist;
   if (s->routing == MOE_ROUTING_EXPERT_CHOICE) {
     r.chunk_hist = nullptr;
     r.scores = at<float>(ws, L.scores);
@@ -223,8 +225,17 @@ moe_status_t do_route(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaSt
   r.status = at<int32_t>(ws, L.status);
   r.wait_limit = g_wait_limit;
   r.num_sms = num_sms();
-  cudaError_t err = launch_router(r, s->dtype, st, &g_launches);
+  if (reduce != 0 && s->routing != MOE_ROUTING_EXPERT_CHOICE) {
+    r.red = reduce_args(s, io, ws, (reduce & kReduceLosses) != 0, (reduce & kReduceDispatch) != 0);
+    r.done = at<unsigned>(ws, L.status + kRouterDoneOffset);
+  }
+  bool reduced = false;
+  cudaError_t err = launch_router(r, s->dtype, st, &g_launches, &reduced);
   if (err != cudaSuccess) return MOE_ERR_CUDA;
+  if (r.done != nullptr && !reduced) {
+    ++g_launches;
+    return cuda_status(launch_reduce(r.red, st));
+  }
   return MOE_OK;
 }
 
@@ -404,17 +415,16 @@ moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, void* ws, s
   const bool ec = shape->routing == MOE_ROUTING_EXPERT_CHOICE;
   if (ec && null_any({io->expert_counts})) return MOE_ERR_INVALID_ARG;
   if (shape->T == 0) {
-    if (!ec) return do_route(shape, io, ws, stream, true);
+    if (!ec) return do_route(shape, io, ws, stream, kReduceLosses);
     ++g_launches;
     return cuda_status(launch_zero_outputs(io->expert_counts, shape->E, io->aux_loss, io->z_loss, stream));
   }
   if (null_any({io->x, io->Wg, io->topk_idx, io->topk_w})) return MOE_ERR_INVALID_ARG;  // bg optional
   if (ec && null_any({io->dropped})) return MOE_ERR_INVALID_ARG;
   if (!aligned16(io->x) || !aligned16(io->Wg)) return MOE_ERR_INVALID_ARG;
-  if ((st = do_route(shape, io, ws, stream, true)) != MOE_OK) return st;
+  if ((st = do_route(shape, io, ws, stream, ec ? 0 : kReduceLosses)) != MOE_OK) return st;
   if (ec) return do_ec_select_and_losses(shape, io, ws, stream);
-  ++g_launches;
-  return cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 0), stream));
+  return MOE_OK;
 }
 
 moe_status_t moe_loss_sums(const moe_shape_t* shape, void* ws, size_t ws_bytes, float* sums, cudaStream_t stream) {
@@ -460,13 +470,18 @@ moe_status_t moe_permute(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   if (null_any({io->x, io->topk_idx, io->dropped, io->out})) return MOE_ERR_INVALID_ARG;
   if (!aligned16(io->x) || !aligned16(io->out)) return MOE_ERR_INVALID_ARG;
   const WsLayout L = ws_layout(*shape);
+  // histograms, with the dispatch reduction in the last histogram block when it fits there
+  const ReduceArgs red = reduce_args(shape, io, ws, 0, 1);
+  bool reduced = false;
   ++g_launches;
   if ((st = cuda_status(launch_hist(io->topk_idx, shape->T, shape->E, shape->k, L.nblk, at<int32_t>(ws, L.chunk_hist),
-                                    at<int32_t>(ws, L.status),
-                                    stream))) != MOE_OK)
+                                    at<int32_t>(ws, L.status), red, at<unsigned>(ws, L.status + kRouterDoneOffset),
+                                    stream, &reduced))) != MOE_OK)
     return st;
-  ++g_launches;
-  if ((st = cuda_status(launch_reduce(reduce_args(shape, io, ws, 0, 1), stream))) != MOE_OK) return st;
+  if (!reduced) {
+    ++g_launches;
+    if ((st = cuda_status(launch_reduce(red, stream))) != MOE_OK) return st;
+  }
   return do_scatter(shape, io, ws, stream);
 }
 
@@ -526,17 +541,15 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws,
     return MOE_ERR_INVALID_ARG;
   if (shape->routing == MOE_ROUTING_EXPERT_CHOICE) {
     // router, per-expert selection, losses, gather, GEMM1, GEMM2 (each call adds its launches)
-    if ((st = do_route(shape, io, ws, stream, false)) != MOE_OK) return st;
+    if ((st = do_route(shape, io, ws, stream, 0)) != MOE_OK) return st;
     if ((st = do_ec_select_and_losses(shape, io, ws, stream)) != MOE_OK) return st;
     if ((st = do_ec_gather(shape, io, ws, stream)) != MOE_OK) return st;
     return do_ffn(shape, io, ws, 1, stream);
   }
   int n = 0;
-  // router emits the chunk histograms itself, so one reduction serves losses and dispatch
-  if ((st = do_route(shape, io, ws, stream, true)) != MOE_OK) return st;
+  // the router emits the chunk histograms itself, so one reduction serves losses and dispatch
+  if ((st = do_route(shape, io, ws, stream, kReduceLosses | kReduceDispatch)) != MOE_OK) return st;
   n += g_launches;
-  ++n;
-  if ((st = cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 1), stream))) != MOE_OK) return st;
   g_launches = 0;
   if ((st = do_scatter(shape, io, ws, stream)) != MOE_OK) return st;
   n += g_launches;
@@ -576,14 +589,13 @@ moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, voi
   if (!aligned16(io->x) || !aligned16(io->Wg) || !aligned16(io->W1) || !aligned16(io->W2) || !aligned16(io->out) ||
       !aligned16(io->b1) || !aligned16(io->b2))
     return MOE_ERR_INVALID_ARG;
-  if ((st = do_route(shape, io, ws, stream, true, true)) != MOE_OK) return st;
-  if (shape->routing == MOE_ROUTING_EXPERT_CHOICE) {
+  const bool ec = shape->routing == MOE_ROUTING_EXPERT_CHOICE;
+  if ((st = do_route(shape, io, ws, stream, ec ? 0 : kReduceLosses | kReduceDispatch, true)) != MOE_OK) return st;
+  if (ec) {
     if ((st = do_ec_select_and_losses(shape, io, ws, stream)) != MOE_OK) return st;
     if ((st = do_ec_gather(shape, io, ws, stream)) != MOE_OK) return st;
     return do_ffn(shape, io, ws, 1, stream, true);
   }
-  ++g_launches;
-  if ((st = cuda_status(launch_reduce(reduce_args(shape, io, ws, 1, 1), stream))) != MOE_OK) return st;
   if ((st = do_scatter(shape, io, ws, stream)) != MOE_OK) return st;
   return do_ffn(shape, io, ws, 1, stream, true);
 }
@@ -778,7 +790,8 @@ moe_status_t moe_get_device_status(void* ws, cudaStream_t stream) {
 void moe_set_wait_limit(long long cycles) { g_wait_limit = cycles > 0 ? cycles : 2000000000LL; }
 
 void moe_set_kernel_options(int flags) {
-  g_kernel_options.store(flags & (MOE_KERNEL_NO_CTA_PAIR | MOE_KERNEL_NO_TC_GATE), std::memory_order_relaxed);
+  g_kernel_options.store(flags & (MOE_KERNEL_NO_CTA_PAIR | MOE_KERNEL_NO_TC_GATE | MOE_KERNEL_NO_TMA_ROUTER),
+                         std::memory_order_relaxed);
 }
 
 int moe_get_kernel_options(void) { return g_kernel_options.load(std::memory_order_relaxed); }

@@ -39,8 +39,25 @@ struct WsLayout {
 
 // Workspace word (next to the device error word) counting finished expert-choice selection blocks.
 constexpr size_t kEcDoneOffset = 4;
+// The same for the router (and histogram) blocks, whose last block runs the loss / dispatch reduction.
+constexpr size_t kRouterDoneOffset = 8;
 
 WsLayout ws_layout(const moe_shape_t& s);
+
+struct ReduceArgs {
+  int T, E, k, nblk;
+  int ec_count;  // > 0: expert choice, every expert holds ec_count rows (no histogram, no dispatch)
+  long long cap;  // < 0: unlimited
+  const float* loss_part;
+  int32_t* chunk_hist;  // [k][nblk][E]
+  int32_t* chunk_base;  // [k][nblk][E] out: first rank of each chunk's assignments in its expert
+  int32_t* cnt_pre;     // [E]
+  int32_t* expert_counts;
+  int32_t* offsets;     // [E+1]
+  float* aux_loss;
+  float* z_loss;
+  int do_losses, do_dispatch;
+};
 
 struct RouterArgs {
   const void* x;
@@ -62,6 +79,11 @@ struct RouterArgs {
   int32_t* status;
   long long wait_limit;
   int num_sms;
+  // When done is given, the last chunk block to finish also runs the loss / dispatch reduction of
+  // red (in the router kernels that work chunk by chunk; launch_router reports whether it did).
+  // done is a workspace counter that is 0 between calls.
+  ReduceArgs red;
+  unsigned* done;
 };
 
 struct EcSelectArgs {
@@ -87,20 +109,6 @@ struct EcGatherArgs {
   float* out;             // [T][H] cleared
 };
 
-struct ReduceArgs {
-  int T, E, k, nblk;
-  int ec_count;  // > 0: expert choice, every expert holds ec_count rows (no histogram, no dispatch)
-  long long cap;  // < 0: unlimited
-  const float* loss_part;
-  int32_t* chunk_hist;  // [k][nblk][E]
-  int32_t* chunk_base;  // [k][nblk][E] out: first rank of each chunk's assignments in its expert
-  int32_t* cnt_pre;     // [E]
-  int32_t* expert_counts;
-  int32_t* offsets;     // [E+1]
-  float* aux_loss;
-  float* z_loss;
-  int do_losses, do_dispatch;
-};
 
 struct ScatterArgs {
   int32_t* status;  // device error word
@@ -163,9 +171,14 @@ struct NvtxRange {
 // driver call is made once per (kernel, device) and size, so repeated launches cost nothing.
 cudaError_t ensure_smem_limit(const void* kernel, int bytes);
 
-cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* launches);
+// *reduced: whether the router's last block ran the reduction of a.red (a.done given), so that no
+// separate reduce launch is needed
+cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* launches, bool* reduced);
+// Per-chunk histograms of a given topk_idx; with done given, the last block also runs the
+// reduction of red when it fits one router-sized block (*reduced says whether it did; if not, a
+// reduce launch must follow).
 cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, int32_t* status,
-                        cudaStream_t st);
+                        const ReduceArgs& red, unsigned* done, cudaStream_t st, bool* reduced);
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);
 cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
 cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);

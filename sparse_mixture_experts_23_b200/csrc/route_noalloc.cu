@@ -110,7 +110,8 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   // Every element the kernels read from the scratch is written earlier in the same call (each
   // router block writes its whole partial row and histogram rows; the reduction writes the
   // per-expert totals before reading them), so nothing needs clearing between calls.  The error
-  // word is only ever written (on a timeout), never read by a kernel.
+  // word is only ever written (on a timeout), never read by a kernel; the finished-block counter
+  // beside it starts at 0 (static device memory) and every call leaves it at 0.
   moe::RouterArgs r{};
   r.x = io->x;
   r.Wg = io->Wg;
@@ -126,10 +127,6 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   r.status = status;  // a bounded wait of the tensor-core gate records a timeout here
   r.wait_limit = moe::wait_limit();
   r.num_sms = device_sms();
-  // no [T,E] gate scratch here: the router is one kernel (the tensor-core gate of 64 / 128 / 256
-  // experts keeps its softmax / top-k tail in the GEMM epilogue and needs none)
-  if (moe::launch_router(r, shape->dtype, stream, &launches) != cudaSuccess) return MOE_ERR_CUDA;
-
   moe::ReduceArgs a{};
   a.T = shape->T;
   a.E = shape->E;
@@ -146,6 +143,14 @@ moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cud
   a.z_loss = io->z_loss;
   a.do_losses = 1;
   a.do_dispatch = 0;
+  // the losses are reduced by the router's last block (its counter sits next to the error word and
+  // is back at 0 after every call), or by one reduce launch after the one-GEMM gate of 64 / 128 / 256
+  // experts, which keeps its softmax / top-k tail in the GEMM epilogue.  No [T,E] gate scratch here.
+  r.red = a;
+  r.done = reinterpret_cast<unsigned*>(static_cast<unsigned char*>(base) + moe::kRouterDoneOffset);
+  bool reduced = false;
+  if (moe::launch_router(r, shape->dtype, stream, &launches, &reduced) != cudaSuccess) return MOE_ERR_CUDA;
+  if (reduced) return MOE_OK;
   ++launches;
   return moe::launch_reduce(a, stream) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -13,6 +13,7 @@
 #include <stdlib.h>
 
 #include "moe_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace moe {
 
@@ -62,11 +63,344 @@ __host__ __device__ inline RouterSmem router_smem(int E, int esize) {
   return s;
 }
 
+constexpr int kRB = 16;  // loads per batch in the reduction below
+
+// Shared memory of the reduction below, for a block of NT threads.
+template <int NT>
+struct ReduceSmem {
+  int gsum[NT];
+  int cnt_s[256];
+  double term[256];
+  float zred[32];
+  float pf[NT];
+  float zf[NT];
+};
+
+// One block of NT threads (E <= NT): losses from the router partials, per-expert totals, capacity,
+// offsets and the exclusive scan of the chunk histograms in (slot, chunk) order.  The partials are
+// read through L2 (__ldcg): in the fused form other blocks of the same grid wrote them.  Every sum
+// runs in a fixed order, so a given NT gives the same bits on every run.
+template <int NT>
+__device__ void reduce_body(const ReduceArgs& a, ReduceSmem<NT>& sm) {
+  int* gsum = sm.gsum;
+  int* cnt_s = sm.cnt_s;
+  double* term = sm.term;
+  float* zred = sm.zred;
+  float* pf = sm.pf;
+  float* zf = sm.zf;
+  const int tid = threadIdx.x, E = a.E;
+  const int C = a.k * a.nblk;  // chunks in (slot, token-chunk) order
+  const int G = NT / E;        // groups of chunks
+  const int g = tid / E, e = tid % E;
+  const bool in = tid < G * E;
+  const bool tc = a.ec_count <= 0;
+  const int c0 = in ? (int)((long long)C * g / G) : 0;
+  const int c1 = in ? (int)((long long)C * (g + 1) / G) : 0;
+  const int b0 = in ? (int)((long long)a.nblk * g / G) : 0;
+  const int b1 = in ? (int)((long long)a.nblk * (g + 1) / G) : 0;
+
+  // The first kRB values of every range this thread reads, all loads issued together (with short
+  // ranges that is every load: one L2 round trip); longer ranges continue in batches of kRB
+  // independent loads.  The additions keep their order (index ascending).
+  int hv[kRB];
+  float pv[kRB], zv[kRB];
+#pragma unroll
+  for (int u = 0; u < kRB; ++u) {
+    hv[u] = tc && c0 + u < c1 ? __ldcg(&a.chunk_hist[(size_t)(c0 + u) * E + e]) : 0;
+    pv[u] = a.do_losses && b0 + u < b1 ? __ldcg(&a.loss_part[(size_t)(b0 + u) * (E + 1) + e]) : 0.f;
+    zv[u] = a.do_losses && tid + u * NT < a.nblk ? __ldcg(&a.loss_part[(size_t)(tid + u * NT) * (E + 1) + E]) : 0.f;
+  }
+  if (a.do_losses) {
+    // P_e: thread (g, e) sums a fixed range of router blocks, then the group sums are added in
+    // group order; z: thread-strided sums then a fixed tree.  Same order on every run.
+    float ps = 0.f;
+#pragma unroll
+    for (int u = 0; u < kRB; ++u)
+      if (b0 + u < b1) ps += pv[u];
+    for (int b = b0 + kRB; b < b1; b += kRB) {
+      float v[kRB];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) v[u] = b + u < b1 ? __ldcg(&a.loss_part[(size_t)(b + u) * (E + 1) + e]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < kRB; ++u)
+        if (b + u < b1) ps += v[u];
+    }
+    if (in) pf[g * E + e] = ps;
+    float zs = 0.f;
+#pragma unroll
+    for (int u = 0; u < kRB; ++u)
+      if (tid + u * NT < a.nblk) zs += zv[u];
+    for (int b = tid + kRB * NT; b < a.nblk; b += kRB * NT) {
+      float v[kRB];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) {
+        const int bb = b + u * NT;
+        v[u] = bb < a.nblk ? __ldcg(&a.loss_part[(size_t)bb * (E + 1) + E]) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kRB; ++u)
+        if (b + u * NT < a.nblk) zs += v[u];
+    }
+    zf[tid] = zs;
+  }
+
+  if (!tc) {
+    // expert choice: every expert holds exactly ec_count rows
+    for (int q = tid; q < E; q += NT) {
+      cnt_s[q] = a.ec_count;
+      a.cnt_pre[q] = a.ec_count;
+    }
+    __syncthreads();
+  } else {
+    int hs = 0;
+#pragma unroll
+    for (int u = 0; u < kRB; ++u) hs += hv[u];
+    for (int c = c0 + kRB; c < c1; c += kRB) {
+      int v[kRB];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) v[u] = c + u < c1 ? __ldcg(&a.chunk_hist[(size_t)(c + u) * E + e]) : 0;
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) hs += v[u];
+    }
+    if (in) gsum[g * E + e] = hs;
+    __syncthreads();
+    // exclusive scan of the G group sums of each expert: warp w scans experts w, w + NT/32, ...; lane
+    // l owns a contiguous run of groups, then a shuffle scan across the lanes (exact integer sums)
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      const int gpl = (G + 31) / 32;  // groups per lane
+      for (int ee = warp; ee < E; ee += NT / 32) {
+        const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
+        int local = 0;
+        for (int q = q0; q < q1; ++q) local += gsum[q * E + ee];
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int run = incl - local;
+        for (int q = q0; q < q1; ++q) {
+          const int v = gsum[q * E + ee];
+          gsum[q * E + ee] = run;
+          run += v;
+        }
+        if (lane == 31) {
+          cnt_s[ee] = incl;
+          a.cnt_pre[ee] = incl;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  if (a.do_dispatch && in) {
+    // chunk bases: the first kRB histogram values are still in registers
+    int run = gsum[g * E + e];
+#pragma unroll
+    for (int u = 0; u < kRB; ++u)
+      if (c0 + u < c1) {
+        a.chunk_base[(size_t)(c0 + u) * E + e] = run;
+        run += hv[u];
+      }
+    for (int c = c0 + kRB; c < c1; c += kRB) {
+      int v[kRB];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) v[u] = c + u < c1 ? __ldcg(&a.chunk_hist[(size_t)(c + u) * E + e]) : 0;
+#pragma unroll
+      for (int u = 0; u < kRB; ++u)
+        if (c + u < c1) {
+          a.chunk_base[(size_t)(c + u) * E + e] = run;
+          run += v[u];
+        }
+    }
+  }
+  if (a.do_dispatch && tid == 0) {
+    int run = 0;
+    for (int q = 0; q < E; ++q) {
+      long long c = cnt_s[q];
+      int kept = (a.cap >= 0 && c > a.cap) ? (int)a.cap : (int)c;
+      a.expert_counts[q] = kept;
+      a.offsets[q] = run;
+      run += kept;
+    }
+    a.offsets[E] = run;
+  }
+  if (a.do_losses) {
+    __syncthreads();
+    for (int w = NT / 2; w >= 32; w >>= 1) {
+      if (tid < w) zf[tid] += zf[tid + w];
+      __syncthreads();
+    }
+    if (tid < 32) {
+      float z = zf[tid];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      if (tid == 0) zred[0] = z;
+    }
+    // P_e: warp w reduces experts w, w + NT/32, ...: lane l sums its contiguous groups, then a fixed
+    // shuffle tree (the same order on every run)
+    {
+      const int warp = tid >> 5, lane = tid & 31;
+      const int gpl = (G + 31) / 32;
+      for (int ee = warp; ee < E; ee += NT / 32) {
+        const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
+        float P = 0.f;
+        for (int q = q0; q < q1; ++q) P += pf[q * E + ee];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) P += __shfl_xor_sync(0xffffffffu, P, o);
+        // f_e = count_e / (all assignments): T*k, or E*C under expert choice
+        const double n_assign = a.ec_count > 0 ? (double)E * a.ec_count : (double)a.T * a.k;
+        if (lane == 0) term[ee] = ((double)cnt_s[ee] / n_assign) * ((double)P / (double)a.T);
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double sum = 0.0;
+      for (int q = 0; q < E; ++q) sum += term[q];
+      *a.aux_loss = (float)((double)E * sum);
+      *a.z_loss = (float)((double)zred[0] / (double)a.T);
+    }
+  }
+}
+
+// Called by every thread of a block once the block's partial results are written: true in the last
+// block of the grid to get here, to which every block's writes are then visible.  That block also
+// returns the counter to 0 for the next call on the workspace.
+__device__ bool last_block_to_finish(unsigned* done) {
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_last = atomicAdd(done, 1u) == gridDim.x - 1;
+    if (s_last) atomicExch(done, 0u);
+  }
+  __syncthreads();
+  const bool last = s_last != 0;
+  if (last) __threadfence();
+  return last;
+}
+
+// The reduction fits the last chunk block (256 threads) when each thread reads at most one batch
+// of histogram values: k * nblk * E <= kRB * 256.  Larger partials (many experts, long batches) go to
+// the one-block reduce kernel of 1024 threads.
+bool reduce_fits_router_block(int k, int nblk, int E) {
+  return (long long)k * nblk * E <= (long long)kRB * kRouterThreads;
+}
+
+// The reduction in the last chunk block of a router (or histogram) grid, when the caller asked for it.
+__device__ void fused_reduce_tail(const ReduceArgs& red, unsigned* done) {
+  if (done == nullptr) return;
+  __shared__ ReduceSmem<kRouterThreads> rs;
+  if (last_block_to_finish(done)) reduce_body<kRouterThreads>(red, rs);
+}
+
+__global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
+  __shared__ ReduceSmem<1024> sm;
+  reduce_body<1024>(a, sm);
+}
+
+// The tail below for token choice with E <= 16: L = 8 or 16 lanes per token (lane e of a group holds
+// expert e), so a warp takes 32 / L of its 4 tokens at once and every per-token reduction is an
+// L-lane shuffle.  Max, sum-exp, lse, p and the top-k come out bitwise as in the 32-lane form (the
+// lanes that form holds beyond E add nothing).  Warp w takes the chunk's tokens 4w .. 4w+3.
+template <int L>
+__device__ void router_finish_narrow(const RouterArgs& a, const float* logits, int epad, float* psum, int* hist,
+                                     float* zw, int blk) {
+  constexpr int G = 32 / L;  // tokens per pass
+  const int E = a.E, T = a.T, k = a.k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int sub = lane / L, e = lane % L;
+  const int t0 = blk * kChunk;
+  for (int i = tid; i < k * E; i += kRouterThreads) hist[i] = 0;
+  __syncthreads();
+  float pacc = 0.f, zacc = 0.f;
+#pragma unroll
+  for (int pass = 0; pass < 4 / G; ++pass) {
+    const int tl = warp * 4 + pass * G + sub;
+    const int t = t0 + tl;
+    const bool valid = t < T;  // a token past T still takes part in its group's shuffles
+    const bool live = e < E;
+    const float lv = live ? logits[tl * epad + e] : -INFINITY;
+    float m = lv;
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float ssum = live ? expf(lv - m) : 0.f;
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
+    const float inv_s = 1.f / ssum;
+    const float lse = m + logf(ssum);
+    if (valid && live) pacc += expf(lv - m) * inv_s;
+    if (valid && e == 0) zacc += lse * lse;
+    if (a.logits_out != nullptr && valid && live) a.logits_out[(size_t)t * E + e] = lv;
+    // top-k: k rounds of a group arg-max with ties to the lower index
+    bool taken = false;
+    float psel_sum = 0.f, my_p = 0.f;
+    int my_e = -1;
+    for (int rr = 0; rr < k; ++rr) {
+      float bv = (live && !taken) ? lv : -INFINITY;
+      int be = (live && !taken) ? e : 0x7fffffff;
+#pragma unroll
+      for (int o = L / 2; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) {
+          bv = ov;
+          be = oe;
+        }
+      }
+      if (be == e) taken = true;
+      const float pv = expf(bv - m) * inv_s;
+      psel_sum += pv;
+      if (e == rr) {
+        my_p = pv;
+        my_e = be;
+      }
+    }
+    if (valid && e < k) {
+      a.topk_idx[(size_t)t * k + e] = my_e;
+      a.topk_w[(size_t)t * k + e] = my_p / psel_sum;
+      if (a.chunk_hist) atomicAdd(&hist[e * E + my_e], 1);
+    }
+  }
+  // the warp's groups -> lane e (fixed order), then per-warp partials -> smem
+#pragma unroll
+  for (int o = L; o < 32; o <<= 1) {
+    pacc += __shfl_xor_sync(0xffffffffu, pacc, o);
+    zacc += __shfl_xor_sync(0xffffffffu, zacc, o);
+  }
+  if (lane < E) psum[warp * epad + lane] = pacc;
+  if (lane == 0) zw[warp] = zacc;
+  __syncthreads();
+  for (int q = tid; q < E; q += kRouterThreads) {
+    float v = 0.f;
+    for (int w = 0; w < 8; ++w) v += psum[w * epad + q];
+    a.loss_part[(size_t)blk * (E + 1) + q] = v;
+  }
+  if (tid == 0) {
+    float v = 0.f;
+    for (int w = 0; w < 8; ++w) v += zw[w];
+    a.loss_part[(size_t)blk * (E + 1) + E] = v;
+  }
+  if (a.chunk_hist) {
+    const int nblk = (T + kChunk - 1) / kChunk;
+    for (int i = tid; i < k * E; i += kRouterThreads) {
+      const int sl = i / E, ex = i % E;
+      a.chunk_hist[((size_t)sl * nblk + blk) * E + ex] = hist[i];
+    }
+  }
+  fused_reduce_tail(a.red, a.done);
+}
+
 // Softmax, top-k, renormalisation and the block's loss partials from logits[32][epad] in shared
 // memory (bias already added).  256 threads: warp w handles the chunk's tokens w, w+8, w+16, w+24.
 // psum: [8][epad] floats, hist: [k][E] ints, zw: [8] floats, all shared.
 __device__ void router_finish(const RouterArgs& a, const float* logits, int epad, float* psum, int* hist, float* zw,
                               int blk) {
+  if (a.scores == nullptr && a.E <= 16) {
+    if (a.E <= 8) router_finish_narrow<8>(a, logits, epad, psum, hist, zw, blk);
+    else router_finish_narrow<16>(a, logits, epad, psum, hist, zw, blk);
+    return;
+  }
   const int E = a.E, T = a.T, k = a.k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = blk * kChunk;
@@ -194,6 +528,7 @@ __device__ void router_finish(const RouterArgs& a, const float* logits, int epad
       a.chunk_hist[((size_t)s * nblk + blk) * E + e] = hist[i];
     }
   }
+  fused_reduce_tail(a.red, a.done);
 }
 
 template <typename TIn>
@@ -786,6 +1121,164 @@ __global__ void __launch_bounds__(kRouterThreads) router_direct_kernel(RouterArg
                 reinterpret_cast<float*>(smem + S::misc_off(H) + 8 * 256 * 4), blockIdx.x);
 }
 
+// Bulk-copy-streamed tensor-core router for bf16 with E = 8 or 16.  The chunk's 32 token rows and
+// the matching rows of the gate stream together through an 8-slot shared-memory ring
+// (cp.async.bulk, completing on the slot's mbarrier): stage s brings x[t0..t0+32, s*SC..(s+1)*SC)
+// (one copy per token row, one per lane) and Wg[s*SC..(s+1)*SC, :] (one contiguous copy per 8-expert
+// plane), so each SM keeps up to 8 stages in flight and nothing is staged before the stream starts.
+// Warp w owns slot w and the stages w, w + 8, ...; after computing a stage it refills the slot
+// with its next one.  Both operands go to mma.sync m16n8k16 through ldmatrix in the natural k order:
+//   - A (x rows): ldmatrix.x4 per 16-column step and 16-row m-tile.  Staged rows are SC*2 + 16 bytes
+//     apart (16 mod 128), so the 8 rows of each 8x8 matrix fall in 8 different bank groups.
+//   - B (the gate, stored [H][E]): a plane holds 16 bytes (8 experts) per h, so 8 consecutive h are
+//     one 128-byte line, and one ldmatrix.x4.trans over 32 consecutive h gives the B registers of
+//     two 16-column steps without conflicts.
+// Warps' partial logits are added in warp order.  A ring wait is bounded: one that runs out records
+// the error word, the CTA stops streaming, waits (bounded) for its copy in flight and finishes on
+// what it has (the results are then invalid and the error word says so).
+template <int NT8>
+struct TmaRouterSmem {
+  static constexpr int E = NT8 * 8;
+  static constexpr int SC = NT8 == 1 ? 256 : 128;   // x columns (= gate rows) per stage
+  static constexpr int kPitch = SC * 2 + 16;         // bytes per staged x row
+  static constexpr int kXBytes = kChunk * kPitch;
+  static constexpr int kWBytes = SC * 16;            // one plane's gate rows of a stage
+  static constexpr int kStage = kXBytes + NT8 * kWBytes;
+  static constexpr int kSlots = 8;                   // one per warp
+  // [ring][barriers][psum [8][E] f32][hist [8][E] i32][z [64] f32]; red [8][32][E] and logits
+  // [32][E] (f32) reuse the ring once every stage is consumed
+  static constexpr int kBarOff = kSlots * kStage;
+  static constexpr int kPsumOff = kBarOff + kSlots * 8;
+  static constexpr int kHistOff = kPsumOff + 8 * E * 4;
+  static constexpr int kZwOff = kHistOff + 8 * E * 4;
+  static constexpr int kTotal = kZwOff + 64 * 4;
+  static constexpr int kRedOff = 0;
+  static constexpr int kLogitsOff = 8 * kChunk * E * 4;
+  static_assert(kLogitsOff + kChunk * E * 4 <= kBarOff && kStage % 16 == 0 && kXBytes % 16 == 0, "layout");
+};
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+template <int NT8>
+__global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a) {
+  using S = TmaRouterSmem<NT8>;
+  constexpr int E = S::E, SC = S::SC, P = S::kPitch;
+  extern __shared__ __align__(16) unsigned char smem[];
+  __shared__ int abort_flag;
+  const int H = a.H, T = a.T;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t4 = lane & 3;
+  const int t0 = blockIdx.x * kChunk;
+  const int rows = min(kChunk, T - t0);
+  const int nst = H / SC;  // stages of the chunk
+  const uint32_t ring = sm100::smem_u32(smem);
+  const uint32_t slot = ring + warp * S::kStage;
+  const uint32_t wslot = slot + S::kXBytes;
+  const uint32_t bar = ring + S::kBarOff + warp * 8;
+  const char* xg = static_cast<const char*>(a.x) + (size_t)t0 * H * 2;
+  const char* wg = static_cast<const char*>(a.Wg);
+
+  if (lane == 0) sm100::mbar_init(bar, 1);
+  if (tid == 0) abort_flag = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  __syncthreads();
+  // stage s -> this warp's slot: lane r copies token row r (rows past T are not copied; their logits
+  // are never used), lanes 32 - NT8 .. 31 copy the gate planes
+  auto issue = [&](int s) {
+    if (lane == 0) sm100::mbar_arrive_expect_tx(bar, (uint32_t)(rows * SC * 2 + NT8 * S::kWBytes));
+    __syncwarp();
+    if (lane < rows) bulk_g2s(slot + lane * P, xg + (size_t)lane * H * 2 + (size_t)s * SC * 2, SC * 2, bar);
+    // the stage's gate rows [s*SC, (s+1)*SC) x E, contiguous in global memory: one copy
+    if (lane == 31) bulk_g2s(wslot, wg + (size_t)s * SC * E * 2, NT8 * S::kWBytes, bar);
+  };
+  if (warp < nst) issue(warp);
+
+  float acc[2][NT8][4];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < NT8; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) acc[m][n][q] = 0.f;
+  // ldmatrix row addresses of this lane: matrix i = lane/8, row j = lane%8
+  const int mi = lane >> 3, mj = lane & 7;
+  // A (x.4, non-transposed): matrices (rows 0-7, k 0-7), (rows 8-15, k 0-7), (rows 0-7, k 8-15),
+  // (rows 8-15, k 8-15) of a 16 x 16 block -> a0..a3 of m16n8k16
+  const uint32_t a_off = (uint32_t)(((mi & 1) * 8 + mj) * P + (mi >> 1) * 16);
+  // B (x.4, transposed): matrix i = gate rows h0 + 8i .. h0 + 8i + 7 of one 8-expert plane -> b0, b1 of
+  // the first 16-column step (i = 0, 1) and of the second (i = 2, 3)
+  const uint32_t b_off = (uint32_t)((8 * mi + mj) * (E * 2));
+  int pending = -1;  // a stage whose copies are in flight and not yet waited for
+  for (int s = warp; s < nst; s += 8) {
+    pending = s;
+    const bool landed =
+        sm100::mbar_wait(bar, (uint32_t)((s >> 3) & 1), a.wait_limit, &abort_flag, a.status, kDevTimeoutProducer);
+    if (!__all_sync(0xffffffffu, landed)) break;  // the whole warp leaves together
+    pending = -1;
+#pragma unroll 2
+    for (int blk = 0; blk < SC / 32; ++blk) {
+      uint32_t bq[NT8][4];
+#pragma unroll
+      for (int n = 0; n < NT8; ++n)
+        ldsm_x4_trans(wslot + (uint32_t)(blk * 32 * E * 2) + b_off + n * 16, bq[n][0], bq[n][1], bq[n][2], bq[n][3]);
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks) {
+        uint32_t af[2][4];
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+          ldsm_x4(slot + (uint32_t)(m * 16 * P + (blk * 32 + ks * 16) * 2) + a_off, af[m][0], af[m][1], af[m][2], af[m][3]);
+#pragma unroll
+        for (int n = 0; n < NT8; ++n)
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+            mma_16816(acc[m][n], af[m][0], af[m][1], af[m][2], af[m][3], bq[n][2 * ks], bq[n][2 * ks + 1]);
+      }
+    }
+    __syncwarp();
+    if (s + 8 < nst) {
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      issue(s + 8);
+    }
+  }
+  if (pending >= 0) {  // a wait ran out: let the copies in flight land before the ring is reused
+    int dummy = 0;
+    sm100::mbar_wait(bar, (uint32_t)((pending >> 3) & 1), a.wait_limit, &dummy, nullptr, 0);
+  }
+  __syncthreads();  // every slot consumed: the ring becomes red / logits
+  float* red = reinterpret_cast<float*>(smem + S::kRedOff);
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int n = 0; n < NT8; ++n)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = 16 * m + g + (q >= 2 ? 8 : 0);
+        const int col = n * 8 + t4 * 2 + (q & 1);
+        red[(warp * 32 + row) * E + col] = acc[m][n][q];
+      }
+  __syncthreads();
+  float* logits = reinterpret_cast<float*>(smem + S::kLogitsOff);
+  const __nv_bfloat16* bg = reinterpret_cast<const __nv_bfloat16*>(a.bg);
+  for (int o = tid; o < 32 * E; o += kRouterThreads) {
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[w * 32 * E + o];
+    logits[o] = v + (bg ? __bfloat162float(bg[o % E]) : 0.f);
+  }
+  __syncthreads();
+  router_finish(a, logits, E, reinterpret_cast<float*>(smem + S::kPsumOff), reinterpret_cast<int*>(smem + S::kHistOff),
+                reinterpret_cast<float*>(smem + S::kZwOff), blockIdx.x);
+}
+
 // Softmax, top-k, renormalisation and partials of one 32-token chunk from logits that a tensor-core
 // GEMM already wrote to global memory ([T,E] fp32, bias included).
 __global__ void __launch_bounds__(kRouterThreads) router_logits_finish_kernel(RouterArgs a) {
@@ -806,8 +1299,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_logits_finish_kernel(Ro
 // Per-chunk, per-slot expert histogram from a given topk_idx (standalone permute).
 // An expert index outside [0, E) (from a caller-supplied topk_idx) is not counted; the error word
 // records it and moe_get_device_status reports it.
-__global__ void hist_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k, int32_t* __restrict__ chunk_hist,
-                            int32_t* status) {
+// With done given, the last block also runs the dispatch reduction of red (as the routers do).
+__global__ void __launch_bounds__(kRouterThreads) hist_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int k,
+                                                          int32_t* __restrict__ chunk_hist, int32_t* status,
+                                                          ReduceArgs red, unsigned* done) {
   __shared__ int hist[8 * 256];
   const int blk = blockIdx.x, nblk = gridDim.x, tid = threadIdx.x;
   for (int i = tid; i < k * E; i += blockDim.x) hist[i] = 0;
@@ -825,133 +1320,7 @@ __global__ void hist_kernel(const int32_t* __restrict__ topk_idx, int T, int E, 
     int s = i / E, e = i % E;
     chunk_hist[((size_t)s * nblk + blk) * E + e] = hist[i];
   }
-}
-
-// One block: losses from the router partials, per-expert totals, capacity, offsets and the
-// exclusive scan of the chunk histograms in (slot, chunk) order.
-__global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
-  __shared__ int gsum[1024];
-  __shared__ int cnt_s[256];
-  __shared__ double term[256];
-  __shared__ float zred[32];
-  __shared__ float pf[1024];
-  __shared__ float zf[1024];
-  const int tid = threadIdx.x, E = a.E;
-  const int C = a.k * a.nblk;  // chunks in (slot, token-chunk) order
-  const int G = 1024 / E;      // groups of chunks
-  const int g = tid / E, e = tid % E;
-  const bool in = tid < G * E;
-  const int c0 = in ? (int)((long long)C * g / G) : 0;
-  const int c1 = in ? (int)((long long)C * (g + 1) / G) : 0;
-
-  if (a.ec_count > 0) {
-    // expert choice: every expert holds exactly ec_count rows
-    for (int q = tid; q < E; q += 1024) {
-      cnt_s[q] = a.ec_count;
-      a.cnt_pre[q] = a.ec_count;
-    }
-    __syncthreads();
-  } else {
-    int s = 0;
-    for (int c = c0; c < c1; ++c) s += a.chunk_hist[(size_t)c * E + e];
-    if (in) gsum[g * E + e] = s;
-    __syncthreads();
-    // exclusive scan of the G group sums of each expert: warp w scans experts w, w+32, ...; lane l
-    // owns a contiguous run of groups, then a shuffle scan across the lanes (exact integer sums)
-    {
-      const int warp = tid >> 5, lane = tid & 31;
-      const int gpl = (G + 31) / 32;  // groups per lane
-      for (int ee = warp; ee < E; ee += 32) {
-        const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
-        int local = 0;
-        for (int q = q0; q < q1; ++q) local += gsum[q * E + ee];
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += v;
-        }
-        int run = incl - local;
-        for (int q = q0; q < q1; ++q) {
-          const int v = gsum[q * E + ee];
-          gsum[q * E + ee] = run;
-          run += v;
-        }
-        if (lane == 31) {
-          cnt_s[ee] = incl;
-          a.cnt_pre[ee] = incl;
-        }
-      }
-    }
-    __syncthreads();
-  }
-  if (a.do_dispatch && in) {
-    int run = gsum[g * E + e];
-    for (int c = c0; c < c1; ++c) {
-      int v = a.chunk_hist[(size_t)c * E + e];
-      a.chunk_base[(size_t)c * E + e] = run;
-      run += v;
-    }
-  }
-  if (a.do_dispatch && tid == 0) {
-    int run = 0;
-    for (int q = 0; q < E; ++q) {
-      long long c = cnt_s[q];
-      int kept = (a.cap >= 0 && c > a.cap) ? (int)a.cap : (int)c;
-      a.expert_counts[q] = kept;
-      a.offsets[q] = run;
-      run += kept;
-    }
-    a.offsets[E] = run;
-  }
-  if (a.do_losses) {
-    // P_e: thread (g, e) sums a fixed range of router blocks, then the group sums are added in
-    // group order; z: thread-strided sums then a fixed tree.  Same order on every run.
-    {
-      const int b0 = in ? (int)((long long)a.nblk * g / G) : 0;
-      const int b1 = in ? (int)((long long)a.nblk * (g + 1) / G) : 0;
-      float ps = 0.f;
-      for (int b = b0; b < b1; ++b) ps += a.loss_part[(size_t)b * (E + 1) + e];
-      if (in) pf[g * E + e] = ps;
-      float zs = 0.f;
-      for (int b = tid; b < a.nblk; b += 1024) zs += a.loss_part[(size_t)b * (E + 1) + E];
-      zf[tid] = zs;
-    }
-    __syncthreads();
-    for (int w = 512; w >= 32; w >>= 1) {
-      if (tid < w) zf[tid] += zf[tid + w];
-      __syncthreads();
-    }
-    if (tid < 32) {
-      float z = zf[tid];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-      if (tid == 0) zred[0] = z;
-    }
-    // P_e: warp w reduces experts w, w+32, ...: lane l sums its contiguous groups, then a fixed
-    // shuffle tree (the same order on every run)
-    {
-      const int warp = tid >> 5, lane = tid & 31;
-      const int gpl = (G + 31) / 32;
-      for (int ee = warp; ee < E; ee += 32) {
-        const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
-        float P = 0.f;
-        for (int q = q0; q < q1; ++q) P += pf[q * E + ee];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) P += __shfl_xor_sync(0xffffffffu, P, o);
-        // f_e = count_e / (all assignments): T*k, or E*C under expert choice
-        const double n_assign = a.ec_count > 0 ? (double)E * a.ec_count : (double)a.T * a.k;
-        if (lane == 0) term[ee] = ((double)cnt_s[ee] / n_assign) * ((double)P / (double)a.T);
-      }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      double sum = 0.0;
-      for (int q = 0; q < E; ++q) sum += term[q];
-      *a.aux_loss = (float)((double)E * sum);
-      *a.z_loss = (float)((double)zred[0] / (double)a.T);
-    }
-  }
+  fused_reduce_tail(red, done);
 }
 
 // Block (chunk b, slot s): stable in-chunk ranks by warp match, rows, drop flags, row maps,
@@ -1086,8 +1455,22 @@ cudaError_t launch_stream(const RouterArgs& a, int nblk, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* launches) {
-  const int nblk = (a.T + kChunk - 1) / kChunk;
+template <int NT8>
+cudaError_t launch_tma_router(const RouterArgs& a, int nblk, cudaStream_t st) {
+  const int bytes = TmaRouterSmem<NT8>::kTotal;
+  cudaError_t err = ensure_smem_limit(reinterpret_cast<const void*>(router_tma_kernel<NT8>), bytes);
+  if (err != cudaSuccess) return err;
+  router_tma_kernel<NT8><<<nblk, kRouterThreads, bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router(const RouterArgs& a_in, int dtype, cudaStream_t st, int* launches, bool* reduced) {
+  const int nblk = (a_in.T + kChunk - 1) / kChunk;
+  // every chunk-by-chunk router below runs the reduction in its last block when done is given and
+  // the partials are small enough; the one-GEMM gate (its epilogue covers 128 tokens per tile) does not
+  RouterArgs a = a_in;
+  if (a.done != nullptr && !reduce_fits_router_block(a.k, nblk, a.E)) a.done = nullptr;
+  *reduced = a.done != nullptr;
   // the tcgen05 gate kernels wait on pipeline barriers with a bound, and record a wait that ran out
   // in a device error word: without one (or without a bound) they are not used
   const bool tc_gate_ok = a.status != nullptr && a.wait_limit > 0 && !router_mma_disabled();
@@ -1100,6 +1483,7 @@ cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* 
   if (dtype == MOE_DTYPE_BF16 && a.scores == nullptr && (a.E == 64 || a.E == 128 || a.E == 256) && a.H % 64 == 0 &&
       a.k <= 8 && tc_gate_ok && 2 * ((a.T + 127) / 128) >= sms) {
     ++*launches;
+    *reduced = false;
     return launch_gate_router_sm100(a, st);
   }
   // bf16, E a multiple of 64, scratch given: the gate is one dense tensor-core GEMM, then the
@@ -1117,6 +1501,14 @@ cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* 
     return cudaGetLastError();
   }
   ++*launches;  // every other form is one kernel
+  // bf16, E = 8 or 16: x streamed by bulk copies through a shared-memory ring (bounded waits, so an
+  // error word and a bound are needed), the gate weights resident
+  if (dtype == MOE_DTYPE_BF16 && (a.E == 8 || a.E == 16) && a.status != nullptr && a.wait_limit > 0 &&
+      !router_mma_disabled() && (kernel_options() & MOE_KERNEL_NO_TMA_ROUTER) == 0) {
+    // (the ring does not depend on H: the gate rows travel with the x stages)
+    if (a.E == 8 && a.H % TmaRouterSmem<1>::SC == 0) return launch_tma_router<1>(a, nblk, st);
+    if (a.E == 16 && a.H % TmaRouterSmem<2>::SC == 0) return launch_tma_router<2>(a, nblk, st);
+  }
   // bf16, E in {8, 16, 32}, Wg^T fits in shared memory: register-direct tensor-core stream over x
   if (dtype == MOE_DTYPE_BF16 && (a.E == 8 || a.E == 16 || a.E == 32) && a.H % 256 == 0 && !router_mma_disabled()) {
     const int bytes = a.E == 8 ? DirectSmem<1>::total(a.H) : (a.E == 16 ? DirectSmem<2>::total(a.H) : DirectSmem<4>::total(a.H));
@@ -1166,8 +1558,10 @@ cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* 
 }
 
 cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, int32_t* status,
-                        cudaStream_t st) {
-  hist_kernel<<<nblk, 256, 0, st>>>(topk_idx, T, E, k, chunk_hist, status);
+                        const ReduceArgs& red, unsigned* done, cudaStream_t st, bool* reduced) {
+  if (done != nullptr && !reduce_fits_router_block(k, nblk, E)) done = nullptr;
+  *reduced = done != nullptr;
+  hist_kernel<<<nblk, kRouterThreads, 0, st>>>(topk_idx, T, E, k, chunk_hist, status, red, done);
   return cudaGetLastError();
 }
 

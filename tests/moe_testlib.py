@@ -142,12 +142,25 @@ def fro_rel(a: np.ndarray, ref: np.ndarray) -> float:
     return num / den if den > 0 else num
 
 
+def gate_in_gemm_epilogue(cfg, sms: int = 148) -> bool:
+    """Whether the gate is one tensor-core GEMM with the softmax / top-k in its epilogue: bf16 token
+    choice with 64, 128 or 256 experts and at least sms/2 tiles of 128 tokens."""
+    return (cfg.dtype == "bf16" and cfg.routing == "token_choice" and cfg.E in (64, 128, 256)
+            and 2 * ((cfg.T + 127) // 128) >= sms)
+
+
 def router_launches(cfg, sms: int = 148) -> int:
     """Kernels of the gate: one, or two (a tensor-core logits GEMM, then the per-chunk softmax / top-k
-    kernel) for bf16 layers whose expert count is a multiple of 64 -- except under token choice with 64,
-    128 or 256 experts and at least sms/2 tiles of 128 tokens, where the softmax / top-k runs in the
-    GEMM's epilogue (one kernel)."""
+    kernel) for bf16 layers whose expert count is a multiple of 64 -- except when the softmax / top-k
+    runs in the GEMM's epilogue (one kernel)."""
     if cfg.dtype != "bf16" or cfg.E % 64 != 0:
         return 1
-    fused = cfg.routing == "token_choice" and cfg.E in (64, 128, 256) and 2 * ((cfg.T + 127) // 128) >= sms
-    return 1 if fused else 2
+    return 1 if gate_in_gemm_epilogue(cfg, sms) else 2
+
+
+def reduce_launches(cfg, sms: int = 148) -> int:
+    """Separate reduce kernels after the gate under token choice: none when the gate works chunk by
+    chunk and the partials fit its last block (k * ceil(T/32) * E <= 16 * 256 values; that block then
+    reduces the losses and the dispatch), else one (also after the GEMM-epilogue gate)."""
+    fits = cfg.k * ((cfg.T + 31) // 32) * cfg.E <= 16 * 256
+    return 1 if gate_in_gemm_epilogue(cfg, sms) or not fits else 0

@@ -260,8 +260,9 @@ def test_kernel_options_round_trip(lib):
     """moe_set_kernel_options keeps the known flags, drops unknown bits, and 0 restores the default."""
     assert moe.moe_get_kernel_options() == moe.MOE_KERNEL_DEFAULT
     try:
-        moe.moe_set_kernel_options(moe.MOE_KERNEL_NO_CTA_PAIR | moe.MOE_KERNEL_NO_TC_GATE | 0x40)
-        assert moe.moe_get_kernel_options() == moe.MOE_KERNEL_NO_CTA_PAIR | moe.MOE_KERNEL_NO_TC_GATE
+        known = moe.MOE_KERNEL_NO_CTA_PAIR | moe.MOE_KERNEL_NO_TC_GATE | moe.MOE_KERNEL_NO_TMA_ROUTER
+        moe.moe_set_kernel_options(known | 0x40)
+        assert moe.moe_get_kernel_options() == known
     finally:
         moe.moe_set_kernel_options(moe.MOE_KERNEL_DEFAULT)
     assert moe.moe_get_kernel_options() == 0

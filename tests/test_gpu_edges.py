@@ -307,10 +307,37 @@ def test_out_of_range_indices_are_reported_not_followed():
     assert buf.device_status() == moe.MOE_OK
 
 
-@pytest.mark.parametrize("flags", [1, 2, 3], ids=["no_cta_pair", "no_tc_gate", "both"])
+@pytest.mark.parametrize("T,H,E,k", [(1000, 256, 8, 2), (77, 2304, 8, 2), (333, 1152, 16, 2), (4100, 4096, 8, 1)],
+                         ids=["one_stage_ragged", "nine_stages", "e16_nine_stages", "two_rounds_ragged"])
+def test_streamed_gate_stage_counts_and_ragged_chunks(T, H, E, k):
+    """The bulk-copy gate (bf16, 8 or 16 experts) with stage counts below, at and past one per warp,
+    a last chunk of fewer than 32 tokens, and its last block's fused loss / dispatch reduction: routing,
+    dispatch and losses against the oracle, and the same results as the register-direct gate."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg(f"stream_gate_{T}_{H}_{E}", T, H, E, k, 128, 1.25, "bf16", 51 + E)
+    inp = synth.make_inputs(cfg)
+    r = _run_forward(cfg, inp)
+    _check_against_oracle(cfg, r)
+    try:
+        moe.moe_set_kernel_options(moe.MOE_KERNEL_NO_TMA_ROUTER)
+        r2 = _run_forward(cfg, inp)
+    finally:
+        moe.moe_set_kernel_options(0)
+    ref = oracle.route(inp.x, inp.Wg, inp.bg, cfg.k, cfg.dtype)
+    ok = ref.margin >= NEAR_TIE
+    assert (r["topk_idx"][ok] == r2["topk_idx"][ok]).all()
+    np.testing.assert_allclose(r["topk_w"][ok], r2["topk_w"][ok], rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(r["losses"], r2["losses"], rtol=1e-5)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("flags", [1, 2, 3, 4], ids=["no_cta_pair", "no_tc_gate", "both", "no_tma_router"])
 def test_kernel_options_select_other_kernels_same_results(flags):
-    """moe_set_kernel_options: the single-CTA GEMM tiles in place of CTA pairs and the CUDA-core gate in
-    place of the tensor-core ones give results that meet the same oracle rules (forward and backward)."""
+    """moe_set_kernel_options: the single-CTA GEMM tiles in place of CTA pairs, the CUDA-core gate in
+    place of the tensor-core ones, and the register-direct gate in place of the bulk-copy stream give
+    results that meet the same oracle rules (forward and backward)."""
     import torch
 
     moe = _lib()

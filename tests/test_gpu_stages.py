@@ -18,7 +18,7 @@ import pytest
 
 import oracle
 import synth
-from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, out_error, router_launches, shape_of,
+from moe_testlib import (NEAR_TIE, TOL_LOSS, TOL_W, from_device_bits, out_error, reduce_launches, router_launches, shape_of,
                          stratified_tokens, upload)
 
 pytestmark = pytest.mark.gpu
@@ -153,4 +153,5 @@ def test_forward_equals_stages(run):
     assert np.array_equal(run["topk_idx_forward"], run["topk_idx"])
     assert np.array_equal(run["losses_forward"], run["losses"])
     assert np.array_equal(run["out_forward"], run["out"])
-    assert run["launches"] == 4 + router_launches(run["cfg"])
+    # gate (+ a reduce after the GEMM-epilogue gate), scatter, GEMM1, GEMM2
+    assert run["launches"] == 3 + router_launches(run["cfg"]) + reduce_launches(run["cfg"])

@@ -18,7 +18,7 @@ import pytest
 
 import oracle
 import synth
-from moe_testlib import NEAR_TIE, TOL_LOSS, TOL_W, shape_of, upload
+from moe_testlib import NEAR_TIE, TOL_LOSS, TOL_W, reduce_launches, shape_of, upload
 
 pytestmark = pytest.mark.gpu
 
@@ -70,7 +70,8 @@ def test_route_noalloc_matches_workspace_route_and_oracle(name):
         w.fill_(float("nan"))
         losses.fill_(float("nan"))
         assert moe.moe_route_noalloc(shape, io, stream) == moe.MOE_OK
-        assert moe.moe_last_launch_count() == 2
+        # one gate kernel (no [T,E] scratch here), plus a reduce only after the GEMM-epilogue gate
+        assert moe.moe_last_launch_count() == 1 + reduce_launches(cfg)
         torch.cuda.synchronize()
         got_idx, got_w, got_l = idx.cpu().numpy(), w.cpu().numpy().astype(np.float64), losses.cpu().numpy()
         # against the workspace router (the same kernels, or the tensor-core gate for 64 experts)
