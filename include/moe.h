@@ -416,6 +416,13 @@ typedef enum {
 MOE_API void moe_set_kernel_options(int flags);
 MOE_API int moe_get_kernel_options(void);
 
+/* The bf16 tensor-core epilogues' activation arithmetic on n given fp32 values: out[i] = act(u[i])
+ * and out[n + i] = act'(u[i]), with act the shape's GELU (u Phi(u), Phi from Abramowitz & Stegun
+ * 7.1.26) or SiLU.  For tests of that arithmetic against its definition.  u: n floats, out: 2n
+ * floats, both device memory.  Errors: MOE_ERR_INVALID_ARG (unknown activation, n < 0, a null
+ * pointer with n > 0), MOE_ERR_CUDA.  One launch (none for n = 0). */
+MOE_API moe_status_t moe_debug_activation(int activation, const float* u, float* out, int64_t n, cudaStream_t stream);
+
 /* Launches one block that waits on a pipeline barrier nothing will ever complete, with the
  * current wait bound; it must come back with the error word set.  For testing the timeout path. */
 MOE_API moe_status_t moe_debug_timeout_probe(void* ws, size_t ws_bytes, cudaStream_t stream);

@@ -29,7 +29,7 @@ ENTRY_POINTS = (
     "moe_last_launch_count", "moe_status_string", "moe_route_noalloc", "moe_capacity",
     "moe_train_workspace_size", "moe_forward_train", "moe_backward", "moe_loss_sums", "moe_losses_from_sums",
     "moe_set_kernel_options", "moe_get_kernel_options", "moe_copy_row_segments", "moe_expert_ffn_rows",
-    "moe_expert_ffn_rows_workspace_size",
+    "moe_expert_ffn_rows_workspace_size", "moe_debug_activation",
 )
 MOE_KERNEL_DEFAULT, MOE_KERNEL_NO_CTA_PAIR, MOE_KERNEL_NO_TC_GATE, MOE_KERNEL_NO_TMA_ROUTER = 0, 1, 2, 4
 
@@ -119,6 +119,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.moe_expert_ffn_rows_workspace_size.restype = sz
     lib.moe_expert_ffn_rows.argtypes = [P(Shape), ctypes.c_int64, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_expert_ffn_rows.restype = st
+    lib.moe_debug_activation.argtypes = [ctypes.c_int, vp, vp, ctypes.c_int64, vp]
+    lib.moe_debug_activation.restype = st
     lib.moe_debug_timeout_probe.argtypes = [vp, sz, vp]
     lib.moe_debug_timeout_probe.restype = st
     lib.moe_last_launch_count.argtypes = []
@@ -264,6 +266,10 @@ def moe_expert_ffn_rows_workspace_size(shape, rows_cap: int) -> int:
 def moe_expert_ffn_rows(shape, rows_cap, offsets, x_rows, W1, b1, W2, b2, y, ws, ws_bytes, stream=0) -> int:
     return load_library().moe_expert_ffn_rows(ctypes.byref(shape), rows_cap, offsets, x_rows, W1, b1, W2, b2, y, ws,
                                               ws_bytes, stream)
+
+
+def moe_debug_activation(activation: int, u, out, n: int, stream=0) -> int:
+    return load_library().moe_debug_activation(int(activation), u, out, int(n), stream)
 
 
 def moe_debug_timeout_probe(ws, ws_bytes, stream=0) -> int:

@@ -114,7 +114,23 @@ struct GemmArgs {
 
 using namespace sm100;
 
-__device__ __forceinline__ float gelu_erf(float u) { return 0.5f * u * (1.f + erff(u * 0.70710678118654752f)); }
+// Phi(u) = P(Z <= u) for a standard normal Z, so that GELU(u) = u Phi(u) = 0.5 u (1 + erf(u / sqrt 2)).
+// erfc(x) for x >= 0 from Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.26 (Hastings):
+//   erfc(x) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-x^2) + e(x),  t = 1 / (1 + p x),  |e(x)| <= 1.5e-7,
+// at x = |u| / sqrt 2; Phi = 1 - erfc/2 for u >= 0 and erfc/2 below.  Two special-function-unit
+// operations (reciprocal, exponential) and five FMAs: the GEMM1 epilogue evaluates this for every
+// element of h, and on short-K tiles (the Switch shape) the epilogue sets the pace.
+__device__ __forceinline__ float normal_cdf(float u) {
+  const float x = fabsf(u) * 0.70710678118654752f;
+  const float t = __fdividef(1.f, fmaf(0.3275911f, x, 1.f));
+  float poly = fmaf(t, 1.061405429f, -1.453152027f);
+  poly = fmaf(t, poly, 1.421413741f);
+  poly = fmaf(t, poly, -0.284496736f);
+  poly = fmaf(t, poly, 0.254829592f);
+  const float half_erfc = 0.5f * poly * t * __expf(-x * x);
+  return u >= 0.f ? 1.f - half_erfc : half_erfc;
+}
+__device__ __forceinline__ float gelu_erf(float u) { return u * normal_cdf(u); }
 // u * sigmoid(u); for u < -87 the fast divide returns 0 where the exact value is below 1e-35
 __device__ __forceinline__ float silu(float u) { return __fdividef(u, 1.f + __expf(-u)); }
 template <int EPI>
@@ -124,7 +140,7 @@ __device__ __forceinline__ float act(float u) {
 }
 // derivatives: GELU'(u) = Phi(u) + u phi(u); SiLU'(u) = s (1 + u (1 - s)), s = sigmoid(u)
 __device__ __forceinline__ float gelu_grad(float u) {
-  return 0.5f * (1.f + erff(u * 0.70710678118654752f)) + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+  return normal_cdf(u) + u * 0.3989422804014327f * __expf(-0.5f * u * u);
 }
 __device__ __forceinline__ float silu_grad(float u) {
   const float sg = __fdividef(1.f, 1.f + __expf(-u));
@@ -1456,6 +1472,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // One thread waits on a barrier that nothing completes; the bound must end it.
+// The tensor-core epilogues' activation and its derivative on given values: out[i] = act(u[i]),
+// out[n + i] = act'(u[i]) (GELU or SiLU), for tests of the epilogue arithmetic.
+__global__ void activation_probe_kernel(int silu_act, const float* u, float* out, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = u[i];
+    out[i] = silu_act ? silu(v) : gelu_erf(v);
+    out[n + i] = silu_act ? silu_grad(v) : gelu_grad(v);
+  }
+}
+
 __global__ void timeout_probe_kernel(int32_t* status, long long limit) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
@@ -1837,6 +1863,13 @@ cudaError_t launch_gate_router_sm100(const RouterArgs& a, cudaStream_t st) {
   if (a.E == 128) return launch_one<128, EPI_ROUTER>(ma, mb, g, grid, st);
   if (a.E == 256) return launch_one<256, EPI_ROUTER>(ma, mb, g, grid, st);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_activation_probe(int act, const float* u, float* out, long long n, cudaStream_t st) {
+  const long long blocks = (n + 255) / 256;
+  activation_probe_kernel<<<(int)(blocks < 1024 ? (blocks > 0 ? blocks : 1) : 1024), 256, 0, st>>>(
+      act == MOE_ACT_SILU ? 1 : 0, u, out, n);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_timeout_probe(int32_t* status, long long limit, cudaStream_t st) {

@@ -796,6 +796,16 @@ void moe_set_kernel_options(int flags) {
 
 int moe_get_kernel_options(void) { return g_kernel_options.load(std::memory_order_relaxed); }
 
+moe_status_t moe_debug_activation(int activation, const float* u, float* out, int64_t n, cudaStream_t stream) {
+  g_launches = 0;
+  if (activation != MOE_ACT_GELU && activation != MOE_ACT_SILU) return MOE_ERR_INVALID_ARG;
+  if (n < 0) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (u == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
+  ++g_launches;
+  return cuda_status(launch_activation_probe(activation, u, out, n, stream));
+}
+
 moe_status_t moe_debug_timeout_probe(void* ws, size_t ws_bytes, cudaStream_t stream) {
   g_launches = 0;
   if (ws == nullptr || ws_bytes < 256 || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MOE_ERR_INVALID_ARG;

@@ -305,5 +305,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int T, int H, int k, float* out,
                            cudaStream_t st);
 cudaError_t launch_timeout_probe(int32_t* status, long long limit, cudaStream_t st);
+// out[i] = act(u[i]), out[n + i] = act'(u[i]) with the tensor-core epilogues' arithmetic
+cudaError_t launch_activation_probe(int act, const float* u, float* out, long long n, cudaStream_t st);
 
 }  // namespace moe

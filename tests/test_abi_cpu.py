@@ -256,6 +256,18 @@ def test_min_capacity_field(lib):
     assert moe.moe_last_launch_count() == 0
 
 
+def test_debug_activation_validates_before_launch(lib):
+    """moe_debug_activation refuses an unknown activation, a negative count and null buffers without
+    launching, and does nothing for n = 0."""
+    assert moe.moe_debug_activation(7, FAKE, FAKE, 4) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_debug_activation(moe.MOE_ACT_GELU, FAKE, FAKE, -1) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_debug_activation(moe.MOE_ACT_SILU, None, FAKE, 4) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_debug_activation(moe.MOE_ACT_GELU, FAKE, None, 4) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_last_launch_count() == 0
+    assert moe.moe_debug_activation(moe.MOE_ACT_GELU, None, None, 0) == moe.MOE_OK
+    assert moe.moe_last_launch_count() == 0
+
+
 def test_kernel_options_round_trip(lib):
     """moe_set_kernel_options keeps the known flags, drops unknown bits, and 0 restores the default."""
     assert moe.moe_get_kernel_options() == moe.MOE_KERNEL_DEFAULT

@@ -307,6 +307,52 @@ def test_out_of_range_indices_are_reported_not_followed():
     assert buf.device_status() == moe.MOE_OK
 
 
+def test_epilogue_activations_match_their_definitions():
+    """The bf16 epilogues' GELU and SiLU (and their derivatives), run on the device through
+    moe_debug_activation, against the fp64 definitions on a dense grid of [-12, 12] and special values.
+    GELU(u) = u Phi(u) with Phi from Abramowitz & Stegun 7.1.26, whose error in erfc is at most 1.5e-7,
+    so |Phi error| <= 0.75e-7 plus fp32 evaluation (a few ulp of quantities <= 1): the bound used is
+    |dGELU| <= 4e-7 |u| + 2^-22 |GELU| and |dGELU'| <= 6e-7 + 2^-20 |GELU'|.  SiLU uses the fast
+    exponential and division: relative error <= 2^-20 + |u| 2^-22."""
+    import torch
+    from scipy.special import erf
+
+    moe = _lib()
+    grid = np.linspace(-12.0, 12.0, 1 << 20)
+    special = np.array([0.0, -0.0, 1e-30, -1e-30, 1e-8, -1e-8, 0.5, -0.5, 1.0, -1.0, 3.0, -3.0, 6.0, -6.0])
+    u = np.concatenate([grid, special]).astype(np.float32)
+    n = u.size
+    ud = torch.from_numpy(u).cuda()
+    out = torch.empty(2 * n, dtype=torch.float32, device="cuda")
+    u64 = u.astype(np.float64)
+    phi = 0.5 * (1.0 + erf(u64 / np.sqrt(2.0)))
+    dens = np.exp(-0.5 * u64 * u64) / np.sqrt(2.0 * np.pi)
+    sig = 1.0 / (1.0 + np.exp(-u64))
+    refs = {moe.MOE_ACT_GELU: (u64 * phi, phi + u64 * dens), moe.MOE_ACT_SILU: (u64 * sig, sig * (1.0 + u64 * (1.0 - sig)))}
+    stream = torch.cuda.current_stream().cuda_stream
+    for act, (f, df) in refs.items():
+        assert moe.moe_debug_activation(act, ud.data_ptr(), out.data_ptr(), n, stream) == moe.MOE_OK
+        assert moe.moe_last_launch_count() == 1
+        torch.cuda.synchronize()
+        got = out.cpu().numpy().astype(np.float64)
+        g, dg = got[:n], got[n:]
+        if act == moe.MOE_ACT_GELU:
+            tol_f = 4e-7 * np.abs(u64) + 2.0 ** -22 * np.abs(f) + 1e-37
+            tol_d = 6e-7 + 2.0 ** -20 * np.abs(df)
+        else:
+            # the fast exponential's relative error grows with its argument (|u| log2 e rounded to
+            # fp32 before the base-2 power); SiLU' crosses zero near u = -1.28, where its two terms of
+            # size ~0.2 cancel, hence the error is bounded against |ref| + 1 there
+            rel = 2.0 ** -20 + np.abs(u64) * 2.0 ** -22
+            tol_f = rel * np.abs(f) + 1e-37
+            tol_d = rel * (np.abs(df) + 1.0)
+        ef, ed = np.abs(g - f), np.abs(dg - df)
+        print(f"act {act}: max |d act| {ef.max():.3e} (worst ratio to bound {np.max(ef / tol_f):.3f}), "
+              f"max |d act'| {ed.max():.3e} (ratio {np.max(ed / tol_d):.3f})")
+        assert np.all(ef <= tol_f), (act, u[np.argmax(ef / tol_f)])
+        assert np.all(ed <= tol_d), (act, u[np.argmax(ed / tol_d)])
+
+
 @pytest.mark.parametrize("T,H,E,k", [(1000, 256, 8, 2), (77, 2304, 8, 2), (333, 1152, 16, 2), (4100, 4096, 8, 1)],
                          ids=["one_stage_ragged", "nine_stages", "e16_nine_stages", "two_rounds_ragged"])
 def test_streamed_gate_stage_counts_and_ragged_chunks(T, H, E, k):
