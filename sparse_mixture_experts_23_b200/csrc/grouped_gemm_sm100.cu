@@ -108,6 +108,10 @@ struct GemmArgs {
   int32_t* r_chunk_hist;  // [k][nchunk][E]
   float* r_logits;        // [T,E] logits (training forward), or null
   int a_box_rows;   // single-CTA kernel: > 0 loads only ceil(rows / a_box_rows) boxes of that many A rows
+  // single-CTA kernel, with a_box_rows = 8: segment rows 8j .. 8j+7 of a tile go to tile rows
+  // 32*(j%4) + 8*(j/4) .., so the rows of a short segment spread over all four TMEM lane quarters and
+  // every epilogue warp gets a share of them (else a 64-row segment leaves two of the four idle)
+  int spread_rows;
   int32_t* status;
   long long wait_limit;
 };
@@ -181,8 +185,10 @@ __device__ __forceinline__ void decode_tile(int tile, const int* prefix, const i
 //   EPI_GELU:    h[grow_i, n0 + j]   = bf16(GELU(acc + b1[n0 + j]))       (64 B per row; SiLU alike)
 //   EPI_COMBINE: out[tok_i, n0 + j] += w_i * (acc + b2[n0 + j])           (128 B per row, fp32 red)
 //   EPI_STORE_Y: y[grow_i, n0 + j]   = acc + b2[n0 + j]                   (128 B per row)
-// Rows i >= nrows (past the expert's segment) are skipped.  grow_i = grow0 + i.
-template <int EPI>
+// Lane i's row is grow_i = grow0 + off_i with off_i = i, or with SPREAD (rows spread over the lane
+// quarters in groups of 8) off_i = 32*(i/8) + i%8; rows with off_i >= nrows (past the expert's
+// segment) are skipped.
+template <int EPI, bool SPREAD = false>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t (&r)[32], float* stg, int lane,
                                                int grow0, int nrows, int my_tok, float my_w, const __nv_bfloat16* brow,
                                                int n0) {
@@ -194,21 +200,33 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t
   __syncwarp();
   const float bj = brow ? __bfloat162float(brow[n0 + lane]) : 0.f;
   const int nr = nrows < 32 ? nrows : 32;
-  if constexpr (epi_h(EPI)) {
-    for (int i = 0; i < nr; ++i) {
-      const float v = stg[i * kStgStride + lane] + bj;
-      g.h_out[(size_t)(grow0 + i) * g.N + n0 + lane] = __float2bfloat16_rn(act<EPI>(v));
-      if (g.u_out) g.u_out[(size_t)(grow0 + i) * g.N + n0 + lane] = __float2bfloat16_rn(v);
+  // 8 rows at a time: their values (and activations) are independent, so the latency of one row's
+  // chain overlaps the others' (one warp per SM sub-partition runs this loop)
+#pragma unroll 1
+  for (int i0 = 0; i0 < 32; i0 += 8) {
+    const int off0 = SPREAD ? 4 * i0 : i0;  // offset of row i0: 32 * (i0 / 8) with SPREAD
+    if (off0 >= (SPREAD ? nrows : nr)) break;  // warp-uniform; later groups lie further out
+    float v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = stg[(i0 + q) * kStgStride + lane] + bj;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int i = i0 + q, off = off0 + q;
+      const bool ok = SPREAD ? off < nrows : i < nr;
+      if constexpr (epi_h(EPI)) {
+        const __nv_bfloat16 hv = __float2bfloat16_rn(act<EPI>(v[q]));
+        if (ok) {
+          g.h_out[(size_t)(grow0 + off) * g.N + n0 + lane] = hv;
+          if (g.u_out) g.u_out[(size_t)(grow0 + off) * g.N + n0 + lane] = __float2bfloat16_rn(v[q]);
+        }
+      } else if (EPI == EPI_COMBINE) {
+        const int tok = __shfl_sync(0xffffffffu, my_tok, i);
+        const float w = __shfl_sync(0xffffffffu, my_w, i);
+        if (ok) atomicAdd(g.out + (size_t)tok * g.N + n0 + lane, w * v[q]);
+      } else {
+        if (ok) g.y[(size_t)(grow0 + off) * g.N + n0 + lane] = v[q];
+      }
     }
-  } else if (EPI == EPI_COMBINE) {
-    for (int i = 0; i < nr; ++i) {
-      const int tok = __shfl_sync(0xffffffffu, my_tok, i);
-      const float w = __shfl_sync(0xffffffffu, my_w, i);
-      const float v = stg[i * kStgStride + lane] + bj;
-      atomicAdd(g.out + (size_t)tok * g.N + n0 + lane, w * v);
-    }
-  } else {
-    for (int i = 0; i < nr; ++i) g.y[(size_t)(grow0 + i) * g.N + n0 + lane] = stg[i * kStgStride + lane] + bj;
   }
   __syncwarp();
 }
@@ -521,8 +539,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // stale shared memory; their accumulator rows are never stored)
             const int nb = (rows + g.a_box_rows - 1) / g.a_box_rows;
             mbar_arrive_expect_tx(full_bar(stage), (uint32_t)(nb * g.a_box_rows * BK * 2 + C::kBBytes));
-            for (int j = 0; j < nb; ++j)
-              tma_load_2d(a_dst + j * g.a_box_rows * 128, &tmA16, kb * BK, row0 + j * g.a_box_rows, full_bar(stage));
+            for (int j = 0; j < nb; ++j) {
+              // spread: 8-row group j at tile row 32*(j%4) + 8*(j/4) (a multiple of 8 rows, so the
+              // 128-byte swizzle phase of every row is unchanged)
+              const int trow = g.spread_rows ? 32 * (j & 3) + 8 * (j >> 2) : j * g.a_box_rows;
+              tma_load_2d(a_dst + trow * 128, &tmA16, kb * BK, row0 + j * g.a_box_rows, full_bar(stage));
+            }
           } else {
             mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
             tma_load_2d(a_dst, &tmA, kb * BK, row0, full_bar(stage));
@@ -603,7 +625,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (warps 2..5) --------
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const int half = (warp - 2) >> 2;  // which half of the tile's columns this warp handles
-    const int r_in_tile = quarter * 32 + lane;
+    const bool spread = g.spread_rows != 0;
+    // the tile row (segment row inside the tile) whose accumulator sits in this lane
+    const int r_in_tile = spread ? 8 * quarter + 32 * (lane >> 3) + (lane & 7) : quarter * 32 + lane;
+    const int wbase = spread ? 8 * quarter : 32 * quarter;  // epilogue_chunk's grow0 offset for this warp
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int e, m_local, n_idx, row0, rows;
@@ -623,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         wgt = g.topk_w ? g.topk_w[(size_t)tok * g.k + g.row_slot[grow]] : 1.f;  // no weights: plain scatter-add
       }
       const __nv_bfloat16* brow = g.bias ? g.bias + (size_t)e * g.N : nullptr;
-      const int wrows = rows - quarter * 32;  // rows of this warp's 32 that lie inside the segment
+      const int wrows = rows - wbase;  // > 0: some of this warp's 32 rows lie inside the segment
       constexpr int kChunks = BN / 32 / (kEpiWarps / 4);  // 32-column chunks per epilogue warp
       float dw = 0.f;
       if constexpr (EPI == EPI_ROUTER) {
@@ -640,8 +665,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (epi_dgrad(EPI)) {
           if (row_ok) epilogue_dgrad32<EPI>(g, r, grow, n_idx * BN + c * 32, wgt, dw);
         } else {
-          if (wrows > 0)
-            epilogue_chunk<EPI>(g, r, stg, lane, row0 + quarter * 32, wrows, tok, wgt, brow, n_idx * BN + c * 32);
+          if (wrows > 0) {
+            if (spread)
+              epilogue_chunk<EPI, true>(g, r, stg, lane, row0 + wbase, wrows, tok, wgt, brow, n_idx * BN + c * 32);
+            else
+              epilogue_chunk<EPI>(g, r, stg, lane, row0 + wbase, wrows, tok, wgt, brow, n_idx * BN + c * 32);
+          }
         }
       }
       if constexpr (epi_dgrad(EPI)) {
@@ -1524,13 +1553,14 @@ bool make_map_a(CUtensorMap* m, const void* base, int rows, int K) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A operand in 16-row boxes (box = 64 k x 16 rows) for segments of a few rows
-bool make_map_a16(CUtensorMap* m, const void* base, int rows, int K) {
+// A operand in boxes of box_rows rows (box = 64 k x box_rows): 16 for segments of a few rows, 8 for
+// the spread placement of mid-length segments
+bool make_map_a_rows(CUtensorMap* m, const void* base, int rows, int K, int box_rows) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-  cuuint32_t box[2] = {BK, 16};
+  cuuint32_t box[2] = {BK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1652,15 +1682,15 @@ cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const
                       int grid, long long avg_rows, cudaStream_t st, const CUtensorMap* ma16 = nullptr) {
   if (N % 256 == 0 && g.K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled())
     return launch_pair<EPI>(ma, mb, mc, g, grid, st);
-  if (ma16 != nullptr && g.a_box_rows > 0) {
+  if (ma16 != nullptr && g.a_box_rows > 0 && !g.spread_rows) {
     const int bn = pick_bn_small(N, g.E, grid);
     if (bn == 256) return launch_one<256, EPI>(ma, mb, g, grid, st, ma16);
     if (bn == 128) return launch_one<128, EPI>(ma, mb, g, grid, st, ma16);
     return launch_one<64, EPI>(ma, mb, g, grid, st, ma16);
   }
-  if (N % 256 == 0) return launch_one<256, EPI>(ma, mb, g, grid, st);
-  if (N % 128 == 0) return launch_one<128, EPI>(ma, mb, g, grid, st);
-  return launch_one<64, EPI>(ma, mb, g, grid, st);
+  if (N % 256 == 0) return launch_one<256, EPI>(ma, mb, g, grid, st, ma16);
+  if (N % 128 == 0) return launch_one<128, EPI>(ma, mb, g, grid, st, ma16);
+  return launch_one<64, EPI>(ma, mb, g, grid, st, ma16);
 }
 
 // A [rows, K] . W[e]^T with W stored [E][N][K]: the backward's data-gradient GEMMs.
@@ -1771,8 +1801,14 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   // for the fewest weight-streaming waves.  (At the Switch shape's ~64 rows per expert this mode measured
   // slower: its narrower GEMM2 tiles read shorter runs of each weight row.)
   const bool small = a.avg_rows < 32;
+  // 32 .. 127 rows per expert on average (the Switch shape: ~64): a tile holds one short segment, and
+  // its rows are spread over all four TMEM lane quarters in 8-row groups, so that every epilogue warp
+  // (and every SM sub-partition) shares the bias + activation work instead of two of the four
+  const bool spread = !small && a.avg_rows < BM;
+  const int box_rows = small ? 16 : 8;
   CUtensorMap ma1s, ma2s;
-  if (small && (!make_map_a16(&ma1s, a.x_perm, a.rows_cap, a.H) || !make_map_a16(&ma2s, a.h, a.rows_cap, a.F)))
+  if ((small || spread) && (!make_map_a_rows(&ma1s, a.x_perm, a.rows_cap, a.H, box_rows) ||
+                            !make_map_a_rows(&ma2s, a.h, a.rows_cap, a.F, box_rows)))
     return cudaErrorInvalidValue;
 
   GemmArgs g1{};
@@ -1784,13 +1820,14 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.h_out = reinterpret_cast<__nv_bfloat16*>(a.h);
   g1.u_out = reinterpret_cast<__nv_bfloat16*>(a.u_out);
   g1.k = a.k;
-  g1.a_box_rows = small ? 16 : 0;
+  g1.a_box_rows = small ? 16 : (spread ? 8 : 0);
+  g1.spread_rows = spread ? 1 : 0;
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
   const long long avg_rows = a.avg_rows;
   cudaError_t err = a.act == MOE_ACT_SILU
-                        ? launch_bn<EPI_SILU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st, small ? &ma1s : nullptr)
-                        : launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st, small ? &ma1s : nullptr);
+                        ? launch_bn<EPI_SILU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st, (small || spread) ? &ma1s : nullptr)
+                        : launch_bn<EPI_GELU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st, (small || spread) ? &ma1s : nullptr);
   if (err != cudaSuccess) return err;
   ++*launches;
 
@@ -1806,9 +1843,9 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g2.row_slot = a.row_slot;
   g2.topk_w = a.topk_w;
   if (a.fuse_combine)
-    err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, small ? &ma2s : nullptr);
+    err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, (small || spread) ? &ma2s : nullptr);
   else
-    err = launch_bn<EPI_STORE_Y>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, small ? &ma2s : nullptr);
+    err = launch_bn<EPI_STORE_Y>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, (small || spread) ? &ma2s : nullptr);
   if (err != cudaSuccess) return err;
   ++*launches;
   return cudaSuccess;

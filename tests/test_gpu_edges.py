@@ -307,6 +307,42 @@ def test_out_of_range_indices_are_reported_not_followed():
     assert buf.device_status() == moe.MOE_OK
 
 
+@pytest.mark.parametrize("T,H,E,k,F,CF,extra", [
+    (1000, 256, 16, 2, 512, math.inf, {}),
+    (640, 128, 16, 1, 256, 1.25, {}),
+    (777, 192, 8, 1, 384, 1.1, {"act": "silu", "bias": False}),
+], ids=["avg125_dropless", "avg40_drops", "avg97_silu_nobias"])
+def test_spread_rows_every_row_against_oracle(T, H, E, k, F, CF, extra):
+    """32 to 127 rows per expert on average: the single-CTA GEMM tiles place each 8-row group of a
+    segment in a different TMEM lane quarter.  Routing, dispatch and every output row against the
+    oracle; then a training forward (u and h written through the same placement) and the backward."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg(f"spread_{T}_{E}", T, H, E, k, F, CF, "bf16", 61 + E, **extra)
+    inp = synth.make_inputs(cfg)
+    r = _run_forward(cfg, inp)
+    _check_against_oracle(cfg, r)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp), train=True)
+    buf.forward_train()
+    grads = buf.make_grads()
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    buf.backward(torch.from_numpy(dout.astype(np.float32)).cuda(), grads, 0.01, 0.001)
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+    assert np.array_equal(buf.out.cpu().numpy(), r["out"])  # the training forward gives the same out
+    ref = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, dout,
+                          0.01, 0.001, act=cfg.act, topk_idx=buf.topk_idx.cpu().numpy(),
+                          dropped=buf.dropped.cpu().numpy())
+    from moe_testlib import TOL_BWD_FRO, TOL_BWD_MAX, fro_rel, rms_rel
+    for n in ("dx", "dWg", "dW1", "dW2"):
+        got = grads[n].cpu().numpy().astype(np.float64)
+        want = getattr(ref, n)
+        per = [rms_rel(got[e], want[e]) for e in range(cfg.E) if np.any(want[e])] if n in ("dW1", "dW2") \
+            else [rms_rel(got, want)]
+        assert max(per) <= TOL_BWD_MAX and fro_rel(got, want) <= TOL_BWD_FRO, (n, max(per))
+
+
 def test_epilogue_activations_match_their_definitions():
     """The bf16 epilogues' GELU and SiLU (and their derivatives), run on the device through
     moe_debug_activation, against the fp64 definitions on a dense grid of [-12, 12] and special values.
