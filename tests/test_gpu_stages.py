@@ -153,5 +153,5 @@ def test_forward_equals_stages(run):
     assert np.array_equal(run["topk_idx_forward"], run["topk_idx"])
     assert np.array_equal(run["losses_forward"], run["losses"])
     assert np.array_equal(run["out_forward"], run["out"])
-    # gate (+ a reduce after the GEMM-epilogue gate), scatter, GEMM1, GEMM2
+    # gate (+ a reduce when the gate's last block cannot take it), scatter, GEMM1, GEMM2
     assert run["launches"] == 3 + router_launches(run["cfg"]) + reduce_launches(run["cfg"])
