@@ -268,16 +268,17 @@ __device__ void reduce_body(const ReduceArgs& a, ReduceSmem<NT>& sm) {
 // returns the counter to 0 for the next call on the workspace.
 __device__ bool last_block_to_finish(unsigned* done) {
   __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
+  __syncthreads();  // the block's writes happen before thread 0's fence below (CTA scope)
   if (threadIdx.x == 0) {
+    __threadfence();  // ... and, cumulatively, before its ticket at GPU scope
     s_last = atomicAdd(done, 1u) == gridDim.x - 1;
-    if (s_last) atomicExch(done, 0u);
+    if (s_last) {
+      __threadfence();  // every earlier block's ticket, and the writes before it, are seen from here on
+      atomicExch(done, 0u);
+    }
   }
   __syncthreads();
-  const bool last = s_last != 0;
-  if (last) __threadfence();
-  return last;
+  return s_last != 0;
 }
 
 // The reduction fits the last chunk block (256 threads) when each thread reads at most one batch
