@@ -187,7 +187,8 @@ MOE_API moe_status_t moe_workspace_layout(const moe_shape_t* shape, void* ws, mo
  * Core Concepts 3: load_balancing_loss, router_z_loss).
  * Reads x, Wg, bg.  Writes topk_idx, topk_w, aux_loss, z_loss (and router partials in ws).
  * Token choice: 1 launch, the gate with its softmax / top-k tail, whose last block to finish also
- * reduces the loss partials (a workspace counter beside the error word picks that block).  bf16
+ * reduces the loss partials (a workspace counter beside the error word picks that block) when they
+ * are small enough, k*ceil(T/32)*E <= 4096; else one reduce launch follows.  bf16
  * layers with 8 or 16 experts stream x through a shared-memory ring of bulk copies into mma.sync
  * (32 experts: register-fed mma.sync); bf16 layers whose expert count is a multiple of 64 run the
  * gate as a tcgen05 GEMM into the workspace followed by the per-chunk softmax / top-k (one launch
@@ -216,7 +217,8 @@ MOE_API moe_status_t moe_route(const moe_shape_t* shape, const moe_io_t* io, voi
  * was reset and rebuilt (cudaDeviceReset) is served its new address.  Every call, on every stream,
  * shares the one array and leaves the last call's contents in it: calls that overlap on the GPU
  * race, so serialise them (one stream, or events).  1 launch (2 with the one-GEMM gate of 64, 128
- * or 256 experts, whose reduction is a launch of its own); one NVTX range.
+ * or 256 experts, or when k*ceil(T/32)*E > 4096: the reduction is then a launch of its own); one
+ * NVTX range.
  * Token choice only: an expert-choice shape returns MOE_ERR_UNSUPPORTED. */
 MOE_API moe_status_t moe_route_noalloc(const moe_shape_t* shape, const moe_io_t* io, cudaStream_t stream);
 
@@ -248,7 +250,8 @@ MOE_API moe_status_t moe_losses_from_sums(int E, const float* sums, float* aux_l
  * assignment is kept iff fewer than `capacity` earlier assignments went to its expert.
  * Reads x, topk_idx.  Writes expert_counts, dropped, the row maps and x_perm in ws, and clears
  * out[T,H] to zero (the fused combine accumulates into it).  Token choice: 2 launches, per-chunk
- * histograms (the last block also scans them into offsets) and the scatter; expert choice: 1.  The kernels check every index they
+ * histograms (the last block also scans them into offsets, when k*ceil(T/32)*E <= 4096; else a
+ * reduce launch follows) and the scatter; expert choice: 1.  The kernels check every index they
  * read from topk_idx (see moe_get_device_status); nothing outside the buffers is touched.
  * Expert choice: nothing is dropped (each expert already holds exactly C tokens); reads x and
  * topk_idx[E,C], writes the row maps and x_perm, and clears out. */
@@ -278,7 +281,8 @@ MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, v
 
 /* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream.  Token choice: the gate
  * (whose last block reduces the losses and the dispatch), the scatter, GEMM1 and GEMM2: 4 launches,
- * 5 with either tensor-core gate form of moe_route.  Expert choice: 6 launches, 7 with the
+ * one more for either tensor-core gate form of moe_route or when the reduction does not fit the
+ * gate's last block (k*ceil(T/32)*E > 4096).  Expert choice: 6 launches, 7 with the
  * two-kernel tensor-core gate. */
 MOE_API moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws, size_t ws_bytes,
                          cudaStream_t stream);

@@ -1500,7 +1500,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   }
 }
 
-// One thread waits on a barrier that nothing completes; the bound must end it.
 // The tensor-core epilogues' activation and its derivative on given values: out[i] = act(u[i]),
 // out[n + i] = act'(u[i]) (GELU or SiLU), for tests of the epilogue arithmetic.
 __global__ void activation_probe_kernel(int silu_act, const float* u, float* out, long long n) {
@@ -1511,6 +1510,7 @@ __global__ void activation_probe_kernel(int silu_act, const float* u, float* out
   }
 }
 
+// One thread waits on a barrier that nothing completes; the bound must end it.
 __global__ void timeout_probe_kernel(int32_t* status, long long limit) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
