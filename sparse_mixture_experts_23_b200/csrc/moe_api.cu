@@ -90,6 +90,8 @@ WsLayout ws_layout(const moe_shape_t& s) {
   o = align256(o + (ec ? T * 4 : 0));
   L.logits = o;  // [T,E] fp32: gate logits (the tensor-core gate's output; saved for the backward pass)
   o = align256(o + T * E * 4);
+  L.red_scratch = o;  // the multi-block reduction's per-expert terms (fp64) and per-block z partials
+  o = align256(o + 256 * 8 + 256 * 4);
   L.total = o;
   // training sections (moe_forward_train / moe_backward), appended after the inference layout
   L.u = o;
@@ -299,6 +301,9 @@ ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int d
   a.z_loss = io->z_loss;
   a.do_losses = do_losses;
   a.do_dispatch = do_dispatch;
+  a.terms = at<double>(ws, L.red_scratch);
+  a.zpart = at<float>(ws, L.red_scratch + 256 * 8);
+  a.done = at<unsigned>(ws, L.status + kReduceDoneOffset);
   return a;
 }
 

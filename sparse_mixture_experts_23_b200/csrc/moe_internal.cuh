@@ -28,7 +28,7 @@ enum DevError : int {
 // Workspace sections (byte offsets from the workspace base, 256-aligned).
 struct WsLayout {
   size_t status, offsets, cnt_pre, chunk_hist, chunk_base, loss_part, row_of, row_token, row_slot, x_perm, h, y,
-      scores, tok_count, total;
+      scores, tok_count, red_scratch, total;
   // training sections, after the inference ones: router logits [T,E] f32, pre-activation u, dout rows
   // (plain and weighted), du (all bf16), per-row dw partial sums, dlogits [T,E] f32
   size_t logits, u, dperm, dyperm, du, dwraw, dlogits, train_total;
@@ -41,6 +41,8 @@ struct WsLayout {
 constexpr size_t kEcDoneOffset = 4;
 // The same for the router (and histogram) blocks, whose last block runs the loss / dispatch reduction.
 constexpr size_t kRouterDoneOffset = 8;
+// ... and for the blocks of the multi-block reduction.
+constexpr size_t kReduceDoneOffset = 12;
 
 WsLayout ws_layout(const moe_shape_t& s);
 
@@ -57,6 +59,12 @@ struct ReduceArgs {
   float* aux_loss;
   float* z_loss;
   int do_losses, do_dispatch;
+  // scratch of the multi-block form (launch_reduce picks it for large k*nblk*E when these are given):
+  // per-expert aux terms [E] (fp64), per-block z partials [256] and a finished-block counter (0
+  // between calls)
+  double* terms;
+  float* zpart;
+  unsigned* done;
 };
 
 struct RouterArgs {

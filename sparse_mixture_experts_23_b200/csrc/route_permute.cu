@@ -295,6 +295,193 @@ __device__ void fused_reduce_tail(const ReduceArgs& red, unsigned* done) {
   if (last_block_to_finish(done)) reduce_body<kRouterThreads>(red, rs);
 }
 
+// The same reduction spread over blocks of experts, for large k * nblk * E (many experts, long
+// batches), where one block would walk long ranges: block b takes experts [b*EB, (b+1)*EB).  Each
+// block scans its experts' chunk histograms into chunk bases and totals, sums their P_e into the
+// aux terms, and sums one slice of the router blocks' lse^2.  The last block to finish (a ticket on
+// a workspace counter) adds the terms and slices in a fixed order and writes the offsets.  Every
+// sum has a fixed order, so the results repeat bit for bit.
+constexpr int kRedMultiThreads = 256;
+struct ReduceMultiSmem {
+  int gsum[kRedMultiThreads];
+  int cnt_s[16];
+  float pf[kRedMultiThreads];
+  float zf[kRedMultiThreads];
+  double tv[kRedMultiThreads];  // the last block's copy of the per-expert terms
+};
+
+__global__ void __launch_bounds__(kRedMultiThreads) reduce_multi_kernel(ReduceArgs a, int EB) {
+  constexpr int NT = kRedMultiThreads;
+  __shared__ ReduceMultiSmem sm;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, E = a.E;
+  const int C = a.k * a.nblk;
+  const int G = NT / EB;  // groups of chunks (EB is a power of 2, at most 16)
+  const int g = tid / EB, j = tid % EB;
+  const int e = blockIdx.x * EB + j;
+  const bool in = e < E;
+  const int c0 = (int)((long long)C * g / G), c1 = (int)((long long)C * (g + 1) / G);
+  const int b0 = (int)((long long)a.nblk * g / G), b1 = (int)((long long)a.nblk * (g + 1) / G);
+  // this block's slice of router blocks for the lse^2 sum
+  const int z0 = (int)((long long)a.nblk * blockIdx.x / gridDim.x);
+  const int z1 = (int)((long long)a.nblk * (blockIdx.x + 1) / gridDim.x);
+
+  int hv[kRB];
+  float pv[kRB];
+#pragma unroll
+  for (int u = 0; u < kRB; ++u) {
+    hv[u] = in && c0 + u < c1 ? __ldcg(&a.chunk_hist[(size_t)(c0 + u) * E + e]) : 0;
+    pv[u] = a.do_losses && in && b0 + u < b1 ? __ldcg(&a.loss_part[(size_t)(b0 + u) * (E + 1) + e]) : 0.f;
+  }
+  int hs = 0;
+#pragma unroll
+  for (int u = 0; u < kRB; ++u) hs += hv[u];
+  for (int c = c0 + kRB; c < c1; c += kRB) {
+    int v[kRB];
+#pragma unroll
+    for (int u = 0; u < kRB; ++u) v[u] = in && c + u < c1 ? __ldcg(&a.chunk_hist[(size_t)(c + u) * E + e]) : 0;
+#pragma unroll
+    for (int u = 0; u < kRB; ++u) hs += v[u];
+  }
+  sm.gsum[g * EB + j] = hs;
+  if (a.do_losses) {
+    float ps = 0.f;
+#pragma unroll
+    for (int u = 0; u < kRB; ++u)
+      if (b0 + u < b1) ps += pv[u];
+    for (int b = b0 + kRB; b < b1; b += kRB) {
+      float v[kRB];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) v[u] = in && b + u < b1 ? __ldcg(&a.loss_part[(size_t)(b + u) * (E + 1) + e]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < kRB; ++u)
+        if (b + u < b1) ps += v[u];
+    }
+    sm.pf[g * EB + j] = ps;
+    float zs = 0.f;
+    for (int b = z0 + tid; b < z1; b += NT) zs += __ldcg(&a.loss_part[(size_t)b * (E + 1) + E]);
+    sm.zf[tid] = zs;
+  }
+  __syncthreads();
+  // per expert of the block (warp w takes experts w, w + 8, ...): exclusive scan of the G group sums
+  // (lane l owns a contiguous run of groups, then a shuffle scan), total, and P_e in the same order
+  const double n_assign = (double)a.T * a.k;
+  for (int jj = warp; jj < EB; jj += NT / 32) {
+    const int ee = blockIdx.x * EB + jj;
+    const int gpl = (G + 31) / 32;
+    const int q0 = min(G, lane * gpl), q1 = min(G, q0 + gpl);
+    int local = 0;
+    float P = 0.f;
+    for (int q = q0; q < q1; ++q) {
+      local += sm.gsum[q * EB + jj];
+      if (a.do_losses) P += sm.pf[q * EB + jj];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) P += __shfl_xor_sync(0xffffffffu, P, o);
+    int run = incl - local;
+    for (int q = q0; q < q1; ++q) {
+      const int v = sm.gsum[q * EB + jj];
+      sm.gsum[q * EB + jj] = run;
+      run += v;
+    }
+    if (lane == 31 && ee < E) {
+      sm.cnt_s[jj] = incl;
+      a.cnt_pre[ee] = incl;
+      if (a.do_dispatch) a.expert_counts[ee] = (a.cap >= 0 && incl > a.cap) ? (int)a.cap : incl;
+    }
+    // every lane holds the full P after the xor tree; lane 31 has the total count
+    if (a.do_losses && lane == 31 && ee < E) a.terms[ee] = ((double)incl / n_assign) * ((double)P / (double)a.T);
+  }
+  __syncthreads();
+  if (a.do_dispatch && in) {
+    int run = sm.gsum[g * EB + j];
+#pragma unroll
+    for (int u = 0; u < kRB; ++u)
+      if (c0 + u < c1) {
+        a.chunk_base[(size_t)(c0 + u) * E + e] = run;
+        run += hv[u];
+      }
+    for (int c = c0 + kRB; c < c1; c += kRB) {
+      int v[kRB];
+#pragma unroll
+      for (int u = 0; u < kRB; ++u) v[u] = c + u < c1 ? __ldcg(&a.chunk_hist[(size_t)(c + u) * E + e]) : 0;
+#pragma unroll
+      for (int u = 0; u < kRB; ++u)
+        if (c + u < c1) {
+          a.chunk_base[(size_t)(c + u) * E + e] = run;
+          run += v[u];
+        }
+    }
+  }
+  if (a.do_losses) {
+    for (int w = NT / 2; w >= 32; w >>= 1) {
+      if (tid < w) sm.zf[tid] += sm.zf[tid + w];
+      __syncthreads();
+    }
+    if (tid < 32) {
+      float z = sm.zf[tid];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      if (tid == 0) a.zpart[blockIdx.x] = z;
+    }
+  }
+  if (!last_block_to_finish(a.done)) return;
+  // the last block: every thread loads one value of each list (E <= 256, blocks <= 256), then warp 0
+  // scans the kept counts into offsets, warp 1 adds the terms and warp 2 the z partials, each lane
+  // over 8 consecutive entries and then a fixed shuffle tree
+  const int nb = gridDim.x;
+  if (tid < E) {
+    sm.gsum[tid] = a.do_dispatch ? __ldcg(&a.expert_counts[tid]) : 0;
+    sm.tv[tid] = a.do_losses ? __ldcg(&a.terms[tid]) : 0.0;
+  } else {
+    sm.gsum[tid] = 0;
+    sm.tv[tid] = 0.0;
+  }
+  sm.zf[tid] = (a.do_losses && tid < nb) ? __ldcg(&a.zpart[tid]) : 0.f;
+  __syncthreads();
+  if (warp == 0 && a.do_dispatch) {
+    int v[8], local = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      v[u] = sm.gsum[lane * 8 + u];
+      local += v[u];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int run = incl - local;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int q = lane * 8 + u;
+      if (q <= E) a.offsets[q] = run;  // offsets[E] = the total (the counts past E are 0)
+      run += v[u];
+    }
+    if (lane == 31 && E == kRedMultiThreads) a.offsets[E] = run;  // E = 256: the total is past the lanes' range
+  } else if (warp == 1 && a.do_losses) {
+    double sum = 0.0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sum += sm.tv[lane * 8 + u];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) *a.aux_loss = (float)((double)E * sum);
+  } else if (warp == 2 && a.do_losses) {
+    double z = 0.0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) z += (double)sm.zf[lane * 8 + u];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) *a.z_loss = (float)(z / (double)a.T);
+  }
+}
+
 __global__ void __launch_bounds__(1024) reduce_kernel(ReduceArgs a) {
   __shared__ ReduceSmem<1024> sm;
   reduce_body<1024>(a, sm);
@@ -1567,6 +1754,18 @@ cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, 
 }
 
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st) {
+  // token choice with more histogram values than one 1024-thread batch: spread over blocks of experts
+  const long long C = (long long)a.k * a.nblk;
+  if (a.ec_count <= 0 && a.terms != nullptr && a.zpart != nullptr && a.done != nullptr &&
+      C * a.E > (long long)kRB * 1024) {
+    int EB = 16;  // experts per block: the largest power of 2 (at most 16) with C * EB / 256 <= kRB
+    while (EB > 1 && C * EB > (long long)kRB * kRedMultiThreads) EB >>= 1;
+    const int nb = (a.E + EB - 1) / EB;
+    if (nb <= 256) {
+      reduce_multi_kernel<<<nb, kRedMultiThreads, 0, st>>>(a, EB);
+      return cudaGetLastError();
+    }
+  }
   reduce_kernel<<<1, 1024, 0, st>>>(a);
   return cudaGetLastError();
 }

@@ -343,6 +343,32 @@ def test_spread_rows_every_row_against_oracle(T, H, E, k, F, CF, extra):
         assert max(per) <= TOL_BWD_MAX and fro_rel(got, want) <= TOL_BWD_FRO, (n, max(per))
 
 
+@pytest.mark.parametrize("T,H,E,k,CF", [(1536, 64, 256, 2, math.inf), (4096, 128, 200, 1, 1.25), (4096, 64, 96, 3, 1.1)],
+                         ids=["E256", "E200_partial_block_drops", "E96_k3"])
+def test_multi_block_reduction_against_oracle(T, H, E, k, CF):
+    """k * ceil(T/32) * E past one 1024-thread batch: the loss / dispatch reduction runs over blocks of
+    experts (up to 16 per block; 256 experts exercise the last offset, 200 a partial last block).  Forward
+    and the standalone route + permute: routing, drops, counts, losses and every output row against the
+    oracle."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg(f"multi_reduce_{E}", T, H, E, k, 64, CF, "bf16", 71 + E)
+    inp = synth.make_inputs(cfg)
+    r = _run_forward(cfg, inp)
+    _check_against_oracle(cfg, r)
+    buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf.route()
+    buf.permute()
+    torch.cuda.synchronize()
+    assert buf.device_status() == moe.MOE_OK
+    idx = buf.topk_idx.cpu().numpy()
+    d = oracle.dispatch(idx, cfg.E, cfg.CF, cfg.min_capacity)
+    assert (buf.expert_counts.cpu().numpy() == d.expert_counts).all()
+    assert (buf.dropped.cpu().numpy() == d.dropped).all()
+    np.testing.assert_array_equal(buf.losses.cpu().numpy(), r["losses"])  # the same reduction, the same bits
+
+
 def test_epilogue_activations_match_their_definitions():
     """The bf16 epilogues' GELU and SiLU (and their derivatives), run on the device through
     moe_debug_activation, against the fp64 definitions on a dense grid of [-12, 12] and special values.
