@@ -329,7 +329,7 @@ moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cuda
   a.x_perm = at<void>(ws, L.x_perm);
   a.out = io->out;
   ++g_launches;
-  return cuda_status(launch_scatter(a, st));
+  return cuda_status(launch_scatter(a, num_sms(), st));
 }
 
 moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse, cudaStream_t st, bool train = false) {

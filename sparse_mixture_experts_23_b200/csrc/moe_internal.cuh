@@ -188,7 +188,7 @@ cudaError_t launch_router(const RouterArgs& a, int dtype, cudaStream_t st, int* 
 cudaError_t launch_hist(const int32_t* topk_idx, int T, int E, int k, int nblk, int32_t* chunk_hist, int32_t* status,
                         const ReduceArgs& red, unsigned* done, cudaStream_t st, bool* reduced);
 cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st);
-cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st);
+cudaError_t launch_scatter(const ScatterArgs& a, int num_sms, cudaStream_t st);
 cudaError_t launch_zero_outputs(int32_t* expert_counts, int E, float* aux, float* z, cudaStream_t st);
 cudaError_t launch_loss_sums(const float* loss_part, const int32_t* cnt_pre, int nblk, int E, int T, float* sums,
                              cudaStream_t st);

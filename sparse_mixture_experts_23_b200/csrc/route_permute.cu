@@ -264,14 +264,14 @@ __device__ void reduce_body(const ReduceArgs& a, ReduceSmem<NT>& sm) {
 }
 
 // Called by every thread of a block once the block's partial results are written: true in the last
-// block of the grid to get here, to which every block's writes are then visible.  That block also
-// returns the counter to 0 for the next call on the workspace.
-__device__ bool last_block_to_finish(unsigned* done) {
+// of `blocks` blocks to get here (the whole grid, or a chunk's CTAs), to which all their writes are then
+// visible.  That block also returns the counter to 0 for the next call on the workspace.
+__device__ bool last_block_to_finish(unsigned* done, unsigned blocks) {
   __shared__ int s_last;
   __syncthreads();  // the block's writes happen before thread 0's fence below (CTA scope)
   if (threadIdx.x == 0) {
     __threadfence();  // ... and, cumulatively, before its ticket at GPU scope
-    s_last = atomicAdd(done, 1u) == gridDim.x - 1;
+    s_last = atomicAdd(done, 1u) == blocks - 1;
     if (s_last) {
       __threadfence();  // every earlier block's ticket, and the writes before it, are seen from here on
       atomicExch(done, 0u);
@@ -292,7 +292,7 @@ bool reduce_fits_router_block(int k, int nblk, int E) {
 __device__ void fused_reduce_tail(const ReduceArgs& red, unsigned* done) {
   if (done == nullptr) return;
   __shared__ ReduceSmem<kRouterThreads> rs;
-  if (last_block_to_finish(done)) reduce_body<kRouterThreads>(red, rs);
+  if (last_block_to_finish(done, gridDim.x)) reduce_body<kRouterThreads>(red, rs);
 }
 
 // The same reduction spread over blocks of experts, for large k * nblk * E (many experts, long
@@ -430,7 +430,7 @@ __global__ void __launch_bounds__(kRedMultiThreads) reduce_multi_kernel(ReduceAr
       if (tid == 0) a.zpart[blockIdx.x] = z;
     }
   }
-  if (!last_block_to_finish(a.done)) return;
+  if (!last_block_to_finish(a.done, gridDim.x)) return;
   // the last block: every thread loads one value of each list (E <= 256, blocks <= 256), then warp 0
   // scans the kept counts into offsets, warp 1 adds the terms and warp 2 the z partials, each lane
   // over 8 consecutive entries and then a fixed shuffle tree
@@ -1358,8 +1358,8 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint3
 
 template <int NT8>
 __global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a) {
-  using S = TmaRouterSmem<NT8>;
-  constexpr int E = S::E, SC = S::SC, P = S::kPitch;
+  using L = TmaRouterSmem<NT8>;
+  constexpr int E = L::E, SC = L::SC, P = L::kPitch;
   extern __shared__ __align__(16) unsigned char smem[];
   __shared__ int abort_flag;
   const int H = a.H, T = a.T;
@@ -1369,9 +1369,9 @@ __global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a
   const int rows = min(kChunk, T - t0);
   const int nst = H / SC;  // stages of the chunk
   const uint32_t ring = sm100::smem_u32(smem);
-  const uint32_t slot = ring + warp * S::kStage;
-  const uint32_t wslot = slot + S::kXBytes;
-  const uint32_t bar = ring + S::kBarOff + warp * 8;
+  const uint32_t slot = ring + warp * L::kStage;
+  const uint32_t wslot = slot + L::kXBytes;
+  const uint32_t bar = ring + L::kBarOff + warp * 8;
   const char* xg = static_cast<const char*>(a.x) + (size_t)t0 * H * 2;
   const char* wg = static_cast<const char*>(a.Wg);
 
@@ -1382,11 +1382,11 @@ __global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a
   // stage s -> this warp's slot: lane r copies token row r (rows past T are not copied; their logits
   // are never used), lanes 32 - NT8 .. 31 copy the gate planes
   auto issue = [&](int s) {
-    if (lane == 0) sm100::mbar_arrive_expect_tx(bar, (uint32_t)(rows * SC * 2 + NT8 * S::kWBytes));
+    if (lane == 0) sm100::mbar_arrive_expect_tx(bar, (uint32_t)(rows * SC * 2 + NT8 * L::kWBytes));
     __syncwarp();
     if (lane < rows) bulk_g2s(slot + lane * P, xg + (size_t)lane * H * 2 + (size_t)s * SC * 2, SC * 2, bar);
     // the stage's gate rows [s*SC, (s+1)*SC) x E, contiguous in global memory: one copy
-    if (lane == 31) bulk_g2s(wslot, wg + (size_t)s * SC * E * 2, NT8 * S::kWBytes, bar);
+    if (lane == 31) bulk_g2s(wslot, wg + (size_t)s * SC * E * 2, NT8 * L::kWBytes, bar);
   };
   if (warp < nst) issue(warp);
 
@@ -1405,11 +1405,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a
   // B (x.4, transposed): matrix i = gate rows h0 + 8i .. h0 + 8i + 7 of one 8-expert plane -> b0, b1 of
   // the first 16-column step (i = 0, 1) and of the second (i = 2, 3)
   const uint32_t b_off = (uint32_t)((8 * mi + mj) * (E * 2));
-  int pending = -1;  // a stage whose copies are in flight and not yet waited for
-  for (int s = warp; s < nst; s += 8) {
-    pending = s;
+  int pending = -1;  // the use of this warp's slot whose copies are in flight and not yet waited for
+  int use = 0;       // uses of this warp's slot so far: the barrier phase parity
+  for (int s = warp; s < nst; s += 8, ++use) {
+    pending = use;
     const bool landed =
-        sm100::mbar_wait(bar, (uint32_t)((s >> 3) & 1), a.wait_limit, &abort_flag, a.status, kDevTimeoutProducer);
+        sm100::mbar_wait(bar, (uint32_t)(use & 1), a.wait_limit, &abort_flag, a.status, kDevTimeoutProducer);
     if (!__all_sync(0xffffffffu, landed)) break;  // the whole warp leaves together
     pending = -1;
 #pragma unroll 2
@@ -1439,10 +1440,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a
   }
   if (pending >= 0) {  // a wait ran out: let the copies in flight land before the ring is reused
     int dummy = 0;
-    sm100::mbar_wait(bar, (uint32_t)((pending >> 3) & 1), a.wait_limit, &dummy, nullptr, 0);
+    sm100::mbar_wait(bar, (uint32_t)(pending & 1), a.wait_limit, &dummy, nullptr, 0);
   }
   __syncthreads();  // every slot consumed: the ring becomes red / logits
-  float* red = reinterpret_cast<float*>(smem + S::kRedOff);
+  float* red = reinterpret_cast<float*>(smem + L::kRedOff);
 #pragma unroll
   for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -1454,7 +1455,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a
         red[(warp * 32 + row) * E + col] = acc[m][n][q];
       }
   __syncthreads();
-  float* logits = reinterpret_cast<float*>(smem + S::kLogitsOff);
+  float* logits = reinterpret_cast<float*>(smem + L::kLogitsOff);
   const __nv_bfloat16* bg = reinterpret_cast<const __nv_bfloat16*>(a.bg);
   for (int o = tid; o < 32 * E; o += kRouterThreads) {
     float v = 0.f;
@@ -1463,8 +1464,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_tma_kernel(RouterArgs a
     logits[o] = v + (bg ? __bfloat162float(bg[o % E]) : 0.f);
   }
   __syncthreads();
-  router_finish(a, logits, E, reinterpret_cast<float*>(smem + S::kPsumOff), reinterpret_cast<int*>(smem + S::kHistOff),
-                reinterpret_cast<float*>(smem + S::kZwOff), blockIdx.x);
+  router_finish(a, logits, E, reinterpret_cast<float*>(smem + L::kPsumOff), reinterpret_cast<int*>(smem + L::kHistOff),
+                reinterpret_cast<float*>(smem + L::kZwOff), blockIdx.x);
 }
 
 // Softmax, top-k, renormalisation and partials of one 32-token chunk from logits that a tensor-core
@@ -1518,17 +1519,20 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
   __shared__ int tok_s[kChunk];
   const int b = blockIdx.x, s = blockIdx.y, tid = threadIdx.x;
   const int nblk = a.nblk;
+  // gridDim.z > 1 (few chunks): block z copies and clears only its slice of the columns; every slice
+  // ranks the chunk itself (one warp, cheap) and slice 0 writes the row maps
+  const bool maps = blockIdx.z == 0;
   if (tid < 32) {
     const int lane = tid;
     const int t = b * kChunk + lane;
     int e = t < a.T ? a.topk_idx[(size_t)t * a.k + s] : -1;
-    if (t < a.T && (e < 0 || e >= a.E)) atomicCAS(a.status, 0, kDevBadIndex);  // dropped below, never copied
+    if (maps && t < a.T && (e < 0 || e >= a.E)) atomicCAS(a.status, 0, kDevBadIndex);  // dropped below, never copied
     const bool valid = t < a.T && e >= 0 && e < a.E;
     if (!valid) e = -1 - lane;  // invalid lanes never match
     const unsigned peers = __match_any_sync(0xffffffffu, e);
     const int rank_local = __popc(peers & ((1u << lane) - 1u));
     int row = -1;
-    if (t < a.T && !valid) {
+    if (maps && t < a.T && !valid) {
       a.dropped[(size_t)t * a.k + s] = 1;
       a.row_of[(size_t)t * a.k + s] = -1;
     }
@@ -1536,11 +1540,13 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
       const long long rank = (long long)a.chunk_base[((size_t)s * nblk + b) * a.E + e] + rank_local;
       const bool keep = a.cap < 0 || rank < a.cap;
       if (keep) row = a.offsets[e] + (int)rank;
-      a.dropped[(size_t)t * a.k + s] = keep ? 0 : 1;
-      a.row_of[(size_t)t * a.k + s] = row;
-      if (keep) {
-        a.row_token[row] = t;
-        a.row_slot[row] = s;
+      if (maps) {
+        a.dropped[(size_t)t * a.k + s] = keep ? 0 : 1;
+        a.row_of[(size_t)t * a.k + s] = row;
+        if (keep) {
+          a.row_token[row] = t;
+          a.row_slot[row] = s;
+        }
       }
     }
     rows_s[lane] = row;
@@ -1550,11 +1556,14 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
   const int nvec = a.H * a.esize / 16;  // 16-byte vectors per row
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* pv = reinterpret_cast<uint4*>(a.x_perm);
+  // this block's columns [c_lo, c_lo + w) of each row, in 16-byte vectors
+  const int c_lo = (int)((long long)nvec * blockIdx.z / gridDim.z);
+  const int w = (int)((long long)nvec * (blockIdx.z + 1) / gridDim.z) - c_lo;
   // this thread's (row, vector) walk over the chunk's 32 rows in steps of 256 vectors, with the
   // row / column split kept incrementally (no division per element)
-  const int step_r = 256 / nvec, step_c = 256 % nvec;
+  const int step_r = 256 / w, step_c = 256 % w;
   constexpr int U = 8;  // 16-byte loads in flight per thread
-  int r = tid / nvec, c = tid % nvec;
+  int r = tid / w, c = tid % w;
   while (r < kChunk) {
     uint4 v[U];
     int dst[U];
@@ -1564,14 +1573,14 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
       if (r < kChunk) {
         const int row = rows_s[r];
         if (row >= 0) {
-          v[u] = xv[(size_t)tok_s[r] * nvec + c];
-          dst[u] = row * nvec + c;  // < T*k*nvec < 2^31 (checked on the host)
+          v[u] = xv[(size_t)tok_s[r] * nvec + c_lo + c];
+          dst[u] = row * nvec + c_lo + c;  // < T*k*nvec < 2^31 (checked on the host)
         }
       }
       r += step_r;
       c += step_c;
-      if (c >= nvec) {
-        c -= nvec;
+      if (c >= w) {
+        c -= w;
         ++r;
       }
     }
@@ -1581,16 +1590,18 @@ __global__ void __launch_bounds__(256) scatter_kernel(ScatterArgs a) {
   }
   if (s == 0 && a.out != nullptr) {
     const int ovec = a.H / 4;
+    const int o_lo = (int)((long long)ovec * blockIdx.z / gridDim.z);
+    const int ow = (int)((long long)ovec * (blockIdx.z + 1) / gridDim.z) - o_lo;
     float4* o = reinterpret_cast<float4*>(a.out);
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int sr = 256 / ovec, sc = 256 % ovec;
-    int orow = tid / ovec, oc = tid % ovec;
+    const int sr = 256 / ow, sc = 256 % ow;
+    int orow = tid / ow, oc = tid % ow;
     while (orow < kChunk) {
-      if (tok_s[orow] >= 0) o[(size_t)tok_s[orow] * ovec + oc] = z;
+      if (tok_s[orow] >= 0) o[(size_t)tok_s[orow] * ovec + o_lo + oc] = z;
       orow += sr;
       oc += sc;
-      if (oc >= ovec) {
-        oc -= ovec;
+      if (oc >= ow) {
+        oc -= ow;
         ++orow;
       }
     }
@@ -1770,8 +1781,15 @@ cudaError_t launch_reduce(const ReduceArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_scatter(const ScatterArgs& a, cudaStream_t st) {
-  dim3 grid(a.nblk, a.k);
+cudaError_t launch_scatter(const ScatterArgs& a, int num_sms, cudaStream_t st) {
+  // fewer (chunk, slot) blocks than SMs (decode-sized batches): split the rows' columns over up to 16
+  // blocks each, while the grid stays within the SMs; each slice keeps at least 8 vectors (128 B) of
+  // a row and of an out row
+  const long long blocks = (long long)a.nblk * a.k;
+  int S = 1;
+  const int nvec = a.H * a.esize / 16, ovec = a.H / 4;
+  while (S < 16 && blocks * 2 * S <= (long long)num_sms && nvec / (2 * S) >= 8 && ovec / (2 * S) >= 8) S *= 2;
+  dim3 grid(a.nblk, a.k, S);
   scatter_kernel<<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }

@@ -415,12 +415,14 @@ def test_epilogue_activations_match_their_definitions():
         assert np.all(ed <= tol_d), (act, u[np.argmax(ed / tol_d)])
 
 
-@pytest.mark.parametrize("T,H,E,k", [(1000, 256, 8, 2), (77, 2304, 8, 2), (333, 1152, 16, 2), (4100, 4096, 8, 1)],
-                         ids=["one_stage_ragged", "nine_stages", "e16_nine_stages", "two_rounds_ragged"])
+@pytest.mark.parametrize("T,H,E,k", [(1000, 256, 8, 2), (77, 2304, 8, 2), (333, 1152, 16, 2), (4100, 4096, 8, 1),
+                                     (32, 4096, 16, 2)],
+                         ids=["one_stage_ragged", "nine_stages", "e16_nine_stages", "two_rounds_ragged", "decode_e16"])
 def test_streamed_gate_stage_counts_and_ragged_chunks(T, H, E, k):
     """The bulk-copy gate (bf16, 8 or 16 experts) with stage counts below, at and past one per warp,
-    a last chunk of fewer than 32 tokens, and its last block's fused loss / dispatch reduction: routing,
-    dispatch and losses against the oracle, and the same results as the register-direct gate."""
+    a last chunk of fewer than 32 tokens, a single chunk, and its last block's fused loss / dispatch
+    reduction: routing, dispatch and losses against the oracle, and the same results as the register-
+    direct gate."""
     import torch
 
     moe = _lib()

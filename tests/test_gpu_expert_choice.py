@@ -41,6 +41,7 @@ CASES = [
     _cfg("ec_all_tokens", 77, 64, 5, 2, 64, math.inf, "bf16", 44),       # C = T: dense mixture
     _cfg("ec_silu_nobias", 300, 256, 8, 2, 512, 1.25, "bf16", 45, act="silu", bias=False),
     _cfg("ec_many_experts", 2048, 128, 64, 2, 128, 1.0, "bf16", 46),    # C = 64
+    _cfg("ec_streamed_gate", 96, 1024, 8, 2, 256, 1.0, "bf16", 49),     # C = 24: the bulk-copy gate, 3 chunks
     synth.CONFIGS["mixtral_ec"],                                        # C = 1024 at the Mixtral shape
 ]
 STRATIFIED = {"mixtral_ec"}  # full size: stratified rows (every m-tile of every expert), else every token
