@@ -1312,15 +1312,16 @@ __global__ void __launch_bounds__(kRouterThreads) router_direct_kernel(RouterArg
 // Bulk-copy-streamed tensor-core router for bf16 with E = 8 or 16.  The chunk's 32 token rows and
 // the matching rows of the gate stream together through an 8-slot shared-memory ring
 // (cp.async.bulk, completing on the slot's mbarrier): stage s brings x[t0..t0+32, s*SC..(s+1)*SC)
-// (one copy per token row, one per lane) and Wg[s*SC..(s+1)*SC, :] (one contiguous copy per 8-expert
-// plane), so each SM keeps up to 8 stages in flight and nothing is staged before the stream starts.
+// (one copy per token row, one per lane) and Wg[s*SC..(s+1)*SC, :] (contiguous in [H][E]: one copy),
+// so each SM keeps up to 8 stages in flight and nothing is staged before the stream starts.
 // Warp w owns slot w and the stages w, w + 8, ...; after computing a stage it refills the slot
 // with its next one.  Both operands go to mma.sync m16n8k16 through ldmatrix in the natural k order:
 //   - A (x rows): ldmatrix.x4 per 16-column step and 16-row m-tile.  Staged rows are SC*2 + 16 bytes
 //     apart (16 mod 128), so the 8 rows of each 8x8 matrix fall in 8 different bank groups.
-//   - B (the gate, stored [H][E]): a plane holds 16 bytes (8 experts) per h, so 8 consecutive h are
-//     one 128-byte line, and one ldmatrix.x4.trans over 32 consecutive h gives the B registers of
-//     two 16-column steps without conflicts.
+//   - B (the gate rows as stored, [h][E]): for each 8-expert n-tile, one ldmatrix.x4.trans over 32
+//     consecutive h (16 bytes of each row) gives the B registers of two 16-column steps.  With E = 8 a
+//     row is 16 bytes, so 8 consecutive h fill one 128-byte line and the reads are conflict-free; with
+//     E = 16 (32-byte rows) each 8x8 matrix meets a 2-way bank conflict.
 // Warps' partial logits are added in warp order.  A ring wait is bounded: one that runs out records
 // the error word, the CTA stops streaming, waits (bounded) for its copy in flight and finishes on
 // what it has (the results are then invalid and the error word says so).
