@@ -269,6 +269,38 @@ def test_stream_ordering_on_side_stream():
     _check_against_oracle(cfg, r)
 
 
+@pytest.mark.parametrize("T,H,E,k,F", [(640, 256, 8, 2, 256), (8192, 128, 128, 1, 128), (32, 512, 8, 2, 256)],
+                         ids=["fused_gate_reduce", "multi_block_reduce", "decode_scatter_slices"])
+def test_concurrent_calls_on_distinct_workspaces(T, H, E, k, F):
+    """Calls on distinct workspaces may run concurrently on different streams: three layers (each with
+    its own batch and workspace, so its own finished-block counters) are enqueued on three streams
+    without waits between them, twice over, and every result must equal the same call run alone."""
+    import torch
+
+    moe = _lib()
+    bufs, serial = [], []
+    for i in range(3):
+        cfg = _cfg(f"concurrent_{E}_{i}", T, H, E, k, F, 1.25, "bf16", 81 + i)
+        buf = moe.MoEBuffers(shape_of(cfg), upload(synth.make_inputs(cfg)))
+        buf.forward()
+        torch.cuda.synchronize()
+        serial.append((buf.out.clone(), buf.topk_idx.clone(), buf.losses.clone(), buf.expert_counts.clone()))
+        bufs.append(buf)
+    streams = [torch.cuda.Stream() for _ in bufs]
+    for s_ in streams:
+        s_.wait_stream(torch.cuda.current_stream())
+    for _ in range(2):
+        for buf, s_ in zip(bufs, streams):
+            with torch.cuda.stream(s_):
+                buf.forward()
+    torch.cuda.synchronize()
+    for buf, (out, idx, losses, counts) in zip(bufs, serial):
+        assert buf.device_status() == moe.MOE_OK
+        assert torch.equal(buf.topk_idx, idx) and torch.equal(buf.expert_counts, counts)
+        assert torch.equal(buf.losses, losses)
+        assert torch.equal(buf.out, out)  # k <= 2: the fp32 adds into out do not depend on their order
+
+
 def test_out_of_range_indices_are_reported_not_followed():
     """A caller-supplied topk_idx with an expert outside [0, E) (token choice), or a chosen token outside
     [0, T) (expert choice): the kernels skip the entry, touch nothing outside the buffers, and the device
