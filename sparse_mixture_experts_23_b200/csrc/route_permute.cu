@@ -304,7 +304,6 @@ __device__ void fused_reduce_tail(const ReduceArgs& red, unsigned* done) {
 constexpr int kRedMultiThreads = 256;
 struct ReduceMultiSmem {
   int gsum[kRedMultiThreads];
-  int cnt_s[16];
   float pf[kRedMultiThreads];
   float zf[kRedMultiThreads];
   double tv[kRedMultiThreads];  // the last block's copy of the per-expert terms
@@ -390,7 +389,6 @@ __global__ void __launch_bounds__(kRedMultiThreads) reduce_multi_kernel(ReduceAr
       run += v;
     }
     if (lane == 31 && ee < E) {
-      sm.cnt_s[jj] = incl;
       a.cnt_pre[ee] = incl;
       if (a.do_dispatch) a.expert_counts[ee] = (a.cap >= 0 && incl > a.cap) ? (int)a.cap : incl;
     }
