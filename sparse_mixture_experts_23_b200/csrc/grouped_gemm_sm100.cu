@@ -1660,22 +1660,10 @@ cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUte
 // 128-row single-CTA tiles waste half as much.  The host sees only the expected rows per expert
 // (T*k/E); the actual counts stay on the device.
 // Small segments (a few rows per expert, e.g. decode): the GEMM streams the weights, and every tile
-// loads only the 16-row A boxes that hold its rows.  The tile width is then chosen for the fewest
-// weight-streaming waves: cost = waves x (16 + BN), ties to the widest.
-int pick_bn_small(int N, int E, int grid) {
-  int best = 0;
-  long long best_cost = -1;
-  for (int bn = 256; bn >= 64; bn >>= 1) {
-    if (N % bn != 0) continue;
-    const long long tiles = (long long)E * (N / bn);
-    const long long cost = ((tiles + grid - 1) / grid) * (16 + bn);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = bn;
-    }
-  }
-  return best;
-}
+// loads only the 16-row A boxes that hold its rows.  The widest tile that divides N streams best:
+// the longer contiguous run of each weight row outweighs a ragged last wave (decode's GEMM1 at
+// 256-wide tiles, 3.03 waves, beat 128-wide, 6.05 waves; 64-wide was far slower).
+int pick_bn_small(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
 
 template <int EPI>
 cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmArgs& g,
@@ -1683,7 +1671,7 @@ cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const
   if (N % 256 == 0 && g.K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled())
     return launch_pair<EPI>(ma, mb, mc, g, grid, st);
   if (ma16 != nullptr && g.a_box_rows > 0 && !g.spread_rows) {
-    const int bn = pick_bn_small(N, g.E, grid);
+    const int bn = pick_bn_small(N);
     if (bn == 256) return launch_one<256, EPI>(ma, mb, g, grid, st, ma16);
     if (bn == 128) return launch_one<128, EPI>(ma, mb, g, grid, st, ma16);
     return launch_one<64, EPI>(ma, mb, g, grid, st, ma16);
