@@ -108,6 +108,10 @@ struct GemmArgs {
   int32_t* r_chunk_hist;  // [k][nchunk][E]
   float* r_logits;        // [T,E] logits (training forward), or null
   int a_box_rows;   // single-CTA kernel: > 0 loads only ceil(rows / a_box_rows) boxes of that many A rows
+  // single-CTA kernel, GEMM2 with the fused combine of a top-1 layer: > 1 splits every tile's K range
+  // into that many parts, each its own work item adding its partial product into out (the bias with
+  // part 0).  With k = 1 an element of out then receives exactly 2 adds, whose order does not matter.
+  int k_splits;
   // single-CTA kernel, with a_box_rows = 8: segment rows 8j .. 8j+7 of a tile go to tile rows
   // 32*(j%4) + 8*(j/4) .., so the rows of a short segment spread over all four TMEM lane quarters and
   // every epilogue warp gets a share of them (else a 64-row segment leaves two of the four idle)
@@ -513,7 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = prefix[E];
+  // work items: every tile, or every (tile, K part) with split K
+  const int KS = g.k_splits > 1 ? g.k_splits : 1;
+  const int total = prefix[E] * KS;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer -----------------
@@ -525,8 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         int e, m_local, n_idx, row0, rows;
-        decode_tile(tile, prefix, offs, E, NT, e, m_local, n_idx, row0, rows);
-        for (int kb = 0; kb < KB; ++kb) {
+        decode_tile(tile / KS, prefix, offs, E, NT, e, m_local, n_idx, row0, rows);
+        const int kb0 = KB * (tile % KS) / KS, kb1 = KB * (tile % KS + 1) / KS;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutProducer)) {
             ok = false;
             break;
@@ -589,7 +596,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
-        for (int kb = 0; kb < KB; ++kb) {
+        const int kb0 = KB * (tile % KS) / KS, kb1 = KB * (tile % KS + 1) / KS;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status, kDevTimeoutMma)) {
             ok = false;
             break;
@@ -602,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bdesc =
                 BKM ? desc_a_kmajor(b_addr + kk * 32) : desc_mnmajor(b_addr + kk * 16 * 128, BK * 128);
             mma_bf16(d_tmem, desc_a_kmajor(a_addr + kk * 32), bdesc, BKM ? (C::kIdesc & ~(1u << 16)) : C::kIdesc,
-                     (kb | kk) != 0 ? 1u : 0u);
+                     (kb != kb0 || kk != 0) ? 1u : 0u);
           }
           issued = true;
           mma_commit(empty_bar(stage));
@@ -632,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int e, m_local, n_idx, row0, rows;
-      decode_tile(tile, prefix, offs, E, NT, e, m_local, n_idx, row0, rows);
+      decode_tile(tile / KS, prefix, offs, E, NT, e, m_local, n_idx, row0, rows);
       const int buf = it & 1;
       const uint32_t tphase = (uint32_t)((it >> 1) & 1);
       // every lane waits; the warp leaves together if any lane gave up (tcgen05.ld is warp-wide)
@@ -647,7 +655,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tok = g.row_token[grow];
         wgt = g.topk_w ? g.topk_w[(size_t)tok * g.k + g.row_slot[grow]] : 1.f;  // no weights: plain scatter-add
       }
-      const __nv_bfloat16* brow = g.bias ? g.bias + (size_t)e * g.N : nullptr;
+      const __nv_bfloat16* brow = (g.bias && tile % KS == 0) ? g.bias + (size_t)e * g.N : nullptr;  // part 0 adds it
       const int wrows = rows - wbase;  // > 0: some of this warp's 32 rows lie inside the segment
       constexpr int kChunks = BN / 32 / (kEpiWarps / 4);  // 32-column chunks per epilogue warp
       float dw = 0.f;
@@ -1830,6 +1838,12 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g2.row_token = a.row_token;
   g2.row_slot = a.row_slot;
   g2.topk_w = a.topk_w;
+  // top-1 layers on single-CTA tiles with a long K (the Switch shape: 512 tiles of K = 4096 are 3.46
+  // waves on 148 SMs): two K halves per tile even out the last wave; with one slot per token each
+  // element of out still receives a fixed pair of adds
+  const bool pair2 = a.H % PairCfg::kTileN == 0 && a.F % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM &&
+                     pair_mode_enabled();
+  if (a.fuse_combine && a.k == 1 && !small && !pair2 && a.F / BK >= 32) g2.k_splits = 2;
   if (a.fuse_combine)
     err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, (small || spread) ? &ma2s : nullptr);
   else

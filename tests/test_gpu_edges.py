@@ -401,6 +401,30 @@ def test_multi_block_reduction_against_oracle(T, H, E, k, CF):
     np.testing.assert_array_equal(buf.losses.cpu().numpy(), r["losses"])  # the same reduction, the same bits
 
 
+@pytest.mark.parametrize("T,H,E,F,CF", [(4096, 256, 64, 2048, 1.25), (3000, 128, 16, 4096, math.inf)],
+                         ids=["spread_drops", "ragged_dropless"])
+def test_top1_split_k_every_row_and_bitwise_repeatable(T, H, E, F, CF):
+    """Top-1 layers on single-CTA tiles with a long GEMM2 K split each GEMM2 tile into two K halves,
+    each adding its partial product into out (the bias with the first).  Every output row against the
+    oracle, and three runs give the same bits: with k = 1 each element receives exactly two adds."""
+    import torch
+
+    moe = _lib()
+    cfg = _cfg(f"split_k_{E}_{F}", T, H, E, 1, F, CF, "bf16", 91 + E)
+    inp = synth.make_inputs(cfg)
+    r = _run_forward(cfg, inp)
+    _check_against_oracle(cfg, r)
+    buf = r["buf"]
+    outs = []
+    for _ in range(3):
+        buf.forward()
+        torch.cuda.synchronize()
+        outs.append(buf.out.clone())
+    assert buf.device_status() == moe.MOE_OK
+    assert all(torch.equal(outs[0], o) for o in outs[1:])
+    assert np.array_equal(outs[0].cpu().numpy(), r["out"])
+
+
 def test_epilogue_activations_match_their_definitions():
     """The bf16 epilogues' GELU and SiLU (and their derivatives), run on the device through
     moe_debug_activation, against the fp64 definitions on a dense grid of [-12, 12] and special values.
