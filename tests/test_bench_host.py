@@ -81,6 +81,13 @@ def test_roofline_bound_follows_arithmetic_intensity():
     assert r["frac"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops"])
     assert r["frac_of_sustained"] == pytest.approx(r["achieved"] / PEAKS["bf16_tflops_sustained"])
     assert "tensor_flop_per_sm_clk" not in r
+    # a loop of 20 calls (35 ms) ends before the power cap's onset: burst peak; 500 calls (0.9 s): sustained
+    short = bench.ffn_roofline(mix, mix.T * mix.k, mix.E, 1.75, PEAKS, None, 148, 20 * 1.75e-3)
+    assert short["peak"] == PEAKS["bf16_tflops"] and short["frac"] == pytest.approx(r["frac"])
+    long = bench.ffn_roofline(mix, mix.T * mix.k, mix.E, 1.75, PEAKS, None, 148, 500 * 1.75e-3)
+    assert long["peak"] == PEAKS["bf16_tflops_sustained"] and "sustained" in long["peak_source"]
+    assert long["frac"] == pytest.approx(r["frac_of_sustained"])
+    assert long["frac_of_burst"] == pytest.approx(r["frac"])
     clk = bench.ffn_roofline(mix, mix.T * mix.k, mix.E, 1.75, PEAKS, {"sm_mhz": 1500.0}, 148)
     per_clk = 4.0 * mix.H * mix.F * mix.T * mix.k / (1.75e-3 * 1500e6 * 148)
     assert clk["tensor_flop_per_sm_clk"]["value"] == pytest.approx(per_clk)
