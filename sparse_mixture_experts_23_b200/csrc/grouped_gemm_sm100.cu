@@ -1250,11 +1250,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // The same weight gradients on CTA pairs (cta_group::2): 256 x 256 tiles of D[e], each CTA holding
 // 128 of the m rows (its A^T half) and 128 of the n columns (its B half), with stages of 128
-// contraction rows.  Each CTA's loads land on its own full barrier; on a segment's last stage each
-// CTA's MMA warp zeroes its own rows past the segment.  The peer then signals the leader through a
-// remote arrive on the leader's ready barrier, and the leader issues the pair's MMAs once both
-// halves are in place.  Commits free the stage (and hand the accumulator to the epilogue) in both
-// CTAs at once.
+// contraction rows.  A whole stage's loads from both CTAs complete on the leader's full barrier,
+// which the leader arms with both halves' bytes, and the leader issues the pair's MMAs once it
+// completes.  A segment's ragged last stage goes the long way: each CTA's loads land on its own full
+// barrier, each CTA's MMA warp zeroes its own rows past the segment, the peer then signals the leader
+// through a remote arrive on the leader's ready barrier, and the leader issues the MMAs once both
+// halves are in place.  (The peer's full barriers and the leader's ready barriers thus complete only
+// on ragged stages; each side tracks their parity per slot.)  Commits free the stage (and hand the
+// accumulator to the epilogue) in both CTAs at once.
 struct WgPairCfg {
   static constexpr int kTileM = 256, kTileN = 256, kStageK = 128;
   static constexpr int kStages = 3;
@@ -1341,10 +1344,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int armed[C::kStages];
       for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
       bool ok = true;
+      uint32_t own_par = 0;  // the peer's own full barriers complete only on ragged stages: their parity per slot
       for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
         int e, m0, n0;
         decode(tile, e, m0, n0);
-        const int r0 = offs[e], KB = (offs[e + 1] - r0 + C::kStageK - 1) / C::kStageK;
+        const int r0 = offs[e], cnt = offs[e + 1] - r0, KB = (cnt + C::kStageK - 1) / C::kStageK;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, g.wait_limit, abort_flag, g.status, kDevTimeoutProducer)) {
             ok = false;
@@ -1352,13 +1356,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const uint32_t a_dst = sbase + stage * C::kStageBytes;
           const uint32_t b_dst = a_dst + C::kABytes;
-          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-          armed[stage] = (int)phase;
           const int k0 = r0 + kb * C::kStageK;
+          if (kb == KB - 1 && cnt % C::kStageK != 0) {
+            // ragged last stage: each CTA counts its own bytes, so that its MMA warp can zero the rows past
+            // the segment once they land
+            mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+            armed[stage] = leader ? (int)phase : (int)((own_par >> stage) & 1u);
+            if (!leader) own_par ^= 1u << stage;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            tma_load_2d(a_dst + j * C::kBoxBytes, &tmA, m0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
-            tma_load_2d(b_dst + j * C::kBoxBytes, &tmB, n0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
+            for (int j = 0; j < 2; ++j) {
+              tma_load_2d(a_dst + j * C::kBoxBytes, &tmA, m0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
+              tma_load_2d(b_dst + j * C::kBoxBytes, &tmB, n0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
+            }
+          } else {
+            // whole stage: both CTAs' bytes complete on the leader's full barrier, which the leader arms
+            if (leader) {
+              mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
+              armed[stage] = (int)phase;
+            }
+            const uint32_t fb = peer_addr(full_bar(stage), 0);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              tma_load_2d_pair(a_dst + j * C::kBoxBytes, &tmA, m0 + 128 * (int)rank + 64 * j, k0, fb);
+              tma_load_2d_pair(b_dst + j * C::kBoxBytes, &tmB, n0 + 128 * (int)rank + 64 * j, k0, fb);
+            }
           }
           if (++stage == C::kStages) {
             stage = 0;
@@ -1378,6 +1399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ stage check (both) + MMA (leader)
     int stage = 0;
     uint32_t phase = 0;
+    uint32_t own_par = 0, ready_par = 0;  // per slot: the peer's full barrier, the leader's ready barrier
     int it = 0;
     bool ok = true;
     bool issued = false;
@@ -1398,13 +1420,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kTileN);
       for (int kb = 0; kb < KB; ++kb) {
-        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status,
+        const uint32_t a_addr = sbase + stage * C::kStageBytes;
+        const int valid = min(C::kStageK, cnt - kb * C::kStageK);
+        if (valid == C::kStageK) {
+          // whole stage: the leader's full barrier has both CTAs' bytes; the peer's MMA warp has nothing to do
+          if (leader) {
+            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status,
+                                                   kDevTimeoutMma))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t b_addr = a_addr + C::kABytes;
+#pragma unroll
+              for (int kk = 0; kk < C::kStageK / 16; ++kk)
+                mma_bf16_pair(d_tmem, desc_mnmajor(a_addr + kk * 16 * 128, C::kBoxBytes),
+                              desc_mnmajor(b_addr + kk * 16 * 128, C::kBoxBytes), C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              mma_commit_both(empty_bar(stage));  // frees this stage in both CTAs once its MMAs are done
+            }
+            issued = true;
+          }
+          __syncwarp();
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
+        }
+        const uint32_t fpar = leader ? phase : ((own_par >> stage) & 1u);
+        if (!leader) own_par ^= 1u << stage;
+        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), fpar, g.wait_limit, abort_flag, g.status,
                                                kDevTimeoutMma))) {
           ok = false;
           break;
         }
-        const uint32_t a_addr = sbase + stage * C::kStageBytes;
-        const int valid = min(C::kStageK, cnt - kb * C::kStageK);
         if (valid < C::kStageK) {
           // this CTA's rows valid..127 of its four boxes: whole 128-byte lines
           const int per_box = (C::kStageK - valid) * 8;
@@ -1420,7 +1470,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // this half is ready: tell the leader (its ready barrier of this stage)
           if (lane == 0) mbar_arrive_cluster(leader_ready0 + 8u * stage);
         } else {
-          if (!__all_sync(0xffffffffu, mbar_wait_cluster(ready_bar(stage), phase, g.wait_limit, abort_flag, g.status,
+          const uint32_t rpar = (ready_par >> stage) & 1u;
+          ready_par ^= 1u << stage;
+          if (!__all_sync(0xffffffffu, mbar_wait_cluster(ready_bar(stage), rpar, g.wait_limit, abort_flag, g.status,
                                                          kDevTimeoutMma))) {
             ok = false;
             break;
