@@ -102,42 +102,67 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(BiasGradArgs a) {
   }
   __syncthreads();
   const int c = 2 * (blockIdx.y * 256 + threadIdx.x);  // first of this thread's two columns
+  // The rows are grouped by expert.  Each run of one expert's rows is summed in row order, with the
+  // loads of eight rows issued together before their adds, then added into the expert's bias gradient.
   if (a.db2 && c < a.H) {
-    float2 acc = make_float2(0.f, 0.f);
-    int cur = e_s[0];
-    for (int i = 0; i < nr; ++i) {
-      if (e_s[i] != cur) {
-        atomicAdd(a.db2 + (size_t)cur * a.H + c, acc.x);
-        atomicAdd(a.db2 + (size_t)cur * a.H + c + 1, acc.y);
-        acc = make_float2(0.f, 0.f);
-        cur = e_s[i];
+    for (int i = 0; i < nr;) {
+      const int cur = e_s[i];
+      int iend = i + 1;
+      while (iend < nr && e_s[iend] == cur) ++iend;
+      float2 acc = make_float2(0.f, 0.f);
+      int j = i;
+      for (; j + 8 <= iend; j += 8) {
+        float2 d[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) d[q] = *reinterpret_cast<const float2*>(a.dout + (size_t)tok_s[j + q] * a.H + c);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          acc.x = fmaf(w_s[j + q], d[q].x, acc.x);
+          acc.y = fmaf(w_s[j + q], d[q].y, acc.y);
+        }
       }
-      const float2 d = *reinterpret_cast<const float2*>(a.dout + (size_t)tok_s[i] * a.H + c);
-      acc.x = fmaf(w_s[i], d.x, acc.x);
-      acc.y = fmaf(w_s[i], d.y, acc.y);
+      for (; j < iend; ++j) {
+        const float2 d = *reinterpret_cast<const float2*>(a.dout + (size_t)tok_s[j] * a.H + c);
+        acc.x = fmaf(w_s[j], d.x, acc.x);
+        acc.y = fmaf(w_s[j], d.y, acc.y);
+      }
+      atomicAdd(a.db2 + (size_t)cur * a.H + c, acc.x);
+      atomicAdd(a.db2 + (size_t)cur * a.H + c + 1, acc.y);
+      i = iend;
     }
-    atomicAdd(a.db2 + (size_t)cur * a.H + c, acc.x);
-    atomicAdd(a.db2 + (size_t)cur * a.H + c + 1, acc.y);
   }
   if (a.db1 && c < a.F) {
     const __nv_bfloat162* du = reinterpret_cast<const __nv_bfloat162*>(a.du);
     const float2* duf = reinterpret_cast<const float2*>(a.du);
-    float2 acc = make_float2(0.f, 0.f);
-    int cur = e_s[0];
-    for (int i = 0; i < nr; ++i) {
-      if (e_s[i] != cur) {
-        atomicAdd(a.db1 + (size_t)cur * a.F + c, acc.x);
-        atomicAdd(a.db1 + (size_t)cur * a.F + c + 1, acc.y);
-        acc = make_float2(0.f, 0.f);
-        cur = e_s[i];
-      }
+    auto load = [&](int i) -> float2 {
       const size_t o = ((size_t)(r0 + i) * a.F + c) / 2;
-      const float2 v = a.f32 ? duf[o] : __bfloat1622float2(du[o]);
-      acc.x += v.x;
-      acc.y += v.y;
+      return a.f32 ? duf[o] : __bfloat1622float2(du[o]);
+    };
+    for (int i = 0; i < nr;) {
+      const int cur = e_s[i];
+      int iend = i + 1;
+      while (iend < nr && e_s[iend] == cur) ++iend;
+      float2 acc = make_float2(0.f, 0.f);
+      int j = i;
+      for (; j + 8 <= iend; j += 8) {
+        float2 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = load(j + q);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          acc.x += v[q].x;
+          acc.y += v[q].y;
+        }
+      }
+      for (; j < iend; ++j) {
+        const float2 v = load(j);
+        acc.x += v.x;
+        acc.y += v.y;
+      }
+      atomicAdd(a.db1 + (size_t)cur * a.F + c, acc.x);
+      atomicAdd(a.db1 + (size_t)cur * a.F + c + 1, acc.y);
+      i = iend;
     }
-    atomicAdd(a.db1 + (size_t)cur * a.F + c, acc.x);
-    atomicAdd(a.db1 + (size_t)cur * a.F + c + 1, acc.y);
   }
 }
 
@@ -237,6 +262,7 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
         for (int o = 16; o > 0; o >>= 1) bdot += __shfl_xor_sync(0xffffffffu, bdot, o);
       } else if (a.b2) {  // dout[t] . b2[e], four columns per lane per step (H is a multiple of 64)
         const __nv_bfloat16* b2 = reinterpret_cast<const __nv_bfloat16*>(a.b2) + (size_t)e * H;
+#pragma unroll 4
         for (int h = 4 * lane; h < H; h += 128) {
           const float4 d = *reinterpret_cast<const float4*>(a.dout + (size_t)t * H + h);
           const uint2 bb = *reinterpret_cast<const uint2*>(b2 + h);
@@ -300,6 +326,7 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
     return;
   }
   const __nv_bfloat16* Wgb = reinterpret_cast<const __nv_bfloat16*>(a.Wg);
+#pragma unroll 4
   for (int h = 4 * lane; h < H; h += 128) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (E % 8 == 0) {
