@@ -262,7 +262,6 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
         for (int o = 16; o > 0; o >>= 1) bdot += __shfl_xor_sync(0xffffffffu, bdot, o);
       } else if (a.b2) {  // dout[t] . b2[e], four columns per lane per step (H is a multiple of 64)
         const __nv_bfloat16* b2 = reinterpret_cast<const __nv_bfloat16*>(a.b2) + (size_t)e * H;
-#pragma unroll 4
         for (int h = 4 * lane; h < H; h += 128) {
           const float4 d = *reinterpret_cast<const float4*>(a.dout + (size_t)t * H + h);
           const uint2 bb = *reinterpret_cast<const uint2*>(b2 + h);
@@ -326,7 +325,6 @@ __global__ void __launch_bounds__(32 * kRbWarps) router_bwd_kernel(RouterBwdArgs
     return;
   }
   const __nv_bfloat16* Wgb = reinterpret_cast<const __nv_bfloat16*>(a.Wg);
-#pragma unroll 4
   for (int h = 4 * lane; h < H; h += 128) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     if (E % 8 == 0) {
