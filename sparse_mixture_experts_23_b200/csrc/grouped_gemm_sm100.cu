@@ -1250,14 +1250,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // The same weight gradients on CTA pairs (cta_group::2): 256 x 256 tiles of D[e], each CTA holding
 // 128 of the m rows (its A^T half) and 128 of the n columns (its B half), with stages of 128
-// contraction rows.  A whole stage's loads from both CTAs complete on the leader's full barrier,
-// which the leader arms with both halves' bytes, and the leader issues the pair's MMAs once it
-// completes.  A segment's ragged last stage goes the long way: each CTA's loads land on its own full
-// barrier, each CTA's MMA warp zeroes its own rows past the segment, the peer then signals the leader
-// through a remote arrive on the leader's ready barrier, and the leader issues the MMAs once both
-// halves are in place.  (The peer's full barriers and the leader's ready barriers thus complete only
-// on ragged stages; each side tracks their parity per slot.)  Commits free the stage (and hand the
-// accumulator to the epilogue) in both CTAs at once.
+// contraction rows.  Both CTAs' loads of a stage complete on the leader's full barrier, which the
+// leader arms with both halves' bytes, and the leader issues the pair's MMAs once it completes.  A
+// segment's ragged last stage runs only the 16-row MMA steps that hold segment rows; the leader's MMA
+// warp first zeroes the rows past the segment inside the last of those steps, in its own shared memory
+// and (through the cluster window) in the peer's.  Commits free the stage (and hand the accumulator to
+// the epilogue) in both CTAs at once.
 struct WgPairCfg {
   static constexpr int kTileM = 256, kTileN = 256, kStageK = 128;
   static constexpr int kStages = 3;
@@ -1267,7 +1265,7 @@ struct WgPairCfg {
   static constexpr int kStageBytes = kABytes + kBBytes;  // 64 KB per CTA
   static constexpr int kTmemCols = 2 * kTileN;
   static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kNumBars = 3 * kStages + 4 + 1;  // full, empty, ready; tfull x2, tempty x2; drain
+  static constexpr int kNumBars = 2 * kStages + 4 + 1;  // full, empty; tfull x2, tempty x2; drain
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kOffsOff = kMiscOff + 16;
   static constexpr int kStgOff = (kOffsOff + 260 * 4 + 1023) & ~1023;
@@ -1288,10 +1286,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t bar0 = sbase + C::kBarOff;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
-  auto ready_bar = [&](int s) { return bar0 + 8u * (2 * C::kStages + s); };
-  auto tfull_bar = [&](int b) { return bar0 + 8u * (3 * C::kStages + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (3 * C::kStages + 2 + b); };
-  const uint32_t drain_bar = bar0 + 8u * (3 * C::kStages + 4);
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * C::kStages + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   int* offs = reinterpret_cast<int*>(smem + C::kOffsOff);
@@ -1310,7 +1307,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
-      mbar_init(ready_bar(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
@@ -1344,7 +1340,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       int armed[C::kStages];
       for (int s = 0; s < C::kStages; ++s) armed[s] = -1;
       bool ok = true;
-      uint32_t own_par = 0;  // the peer's own full barriers complete only on ragged stages: their parity per slot
       for (int tile = cluster_id; tile < total && ok; tile += nclusters) {
         int e, m0, n0;
         decode(tile, e, m0, n0);
@@ -1357,29 +1352,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t a_dst = sbase + stage * C::kStageBytes;
           const uint32_t b_dst = a_dst + C::kABytes;
           const int k0 = r0 + kb * C::kStageK;
-          if (kb == KB - 1 && cnt % C::kStageK != 0) {
-            // ragged last stage: each CTA counts its own bytes, so that its MMA warp can zero the rows past
-            // the segment once they land
-            mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-            armed[stage] = leader ? (int)phase : (int)((own_par >> stage) & 1u);
-            if (!leader) own_par ^= 1u << stage;
+          // both CTAs' bytes complete on the leader's full barrier, which the leader arms; rows of a
+          // ragged last stage past the segment are zeroed by the leader's MMA warp once they land
+          if (leader) {
+            mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
+            armed[stage] = (int)phase;
+          }
+          const uint32_t fb = peer_addr(full_bar(stage), 0);
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              tma_load_2d(a_dst + j * C::kBoxBytes, &tmA, m0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
-              tma_load_2d(b_dst + j * C::kBoxBytes, &tmB, n0 + 128 * (int)rank + 64 * j, k0, full_bar(stage));
-            }
-          } else {
-            // whole stage: both CTAs' bytes complete on the leader's full barrier, which the leader arms
-            if (leader) {
-              mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
-              armed[stage] = (int)phase;
-            }
-            const uint32_t fb = peer_addr(full_bar(stage), 0);
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-              tma_load_2d_pair(a_dst + j * C::kBoxBytes, &tmA, m0 + 128 * (int)rank + 64 * j, k0, fb);
-              tma_load_2d_pair(b_dst + j * C::kBoxBytes, &tmB, n0 + 128 * (int)rank + 64 * j, k0, fb);
-            }
+          for (int j = 0; j < 2; ++j) {
+            tma_load_2d_pair(a_dst + j * C::kBoxBytes, &tmA, m0 + 128 * (int)rank + 64 * j, k0, fb);
+            tma_load_2d_pair(b_dst + j * C::kBoxBytes, &tmB, n0 + 128 * (int)rank + 64 * j, k0, fb);
           }
           if (++stage == C::kStages) {
             stage = 0;
@@ -1396,112 +1379,80 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ stage check (both) + MMA (leader)
-    int stage = 0;
-    uint32_t phase = 0;
-    uint32_t own_par = 0, ready_par = 0;  // per slot: the peer's full barrier, the leader's ready barrier
-    int it = 0;
-    bool ok = true;
-    bool issued = false;
-    const uint32_t leader_ready0 = peer_addr(ready_bar(0), 0);
-    for (int tile = cluster_id; tile < total && ok; tile += nclusters, ++it) {
-      int e, m0, n0;
-      decode(tile, e, m0, n0);
-      const int r0 = offs[e], cnt = offs[e + 1] - r0, KB = (cnt + C::kStageK - 1) / C::kStageK;
-      const int buf = it & 1;
-      const uint32_t tphase = (uint32_t)((it >> 1) & 1);
-      if (leader) {
+    // ------------------------------------------------------------ MMA (leader) ---------------
+    if (leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = cluster_id; tile < total && ok; tile += nclusters, ++it) {
+        int e, m0, n0;
+        decode(tile, e, m0, n0);
+        const int r0 = offs[e], cnt = offs[e + 1] - r0, KB = (cnt + C::kStageK - 1) / C::kStageK;
+        const int buf = it & 1;
+        const uint32_t tphase = (uint32_t)((it >> 1) & 1);
         if (!__all_sync(0xffffffffu, mbar_wait(tempty_bar(buf), tphase ^ 1u, g.wait_limit, abort_flag, g.status,
                                                kDevTimeoutMma))) {
           ok = false;
           break;
         }
         tc_fence_after();
-      }
-      const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kTileN);
-      for (int kb = 0; kb < KB; ++kb) {
-        const uint32_t a_addr = sbase + stage * C::kStageBytes;
-        const int valid = min(C::kStageK, cnt - kb * C::kStageK);
-        if (valid == C::kStageK) {
-          // whole stage: the leader's full barrier has both CTAs' bytes; the peer's MMA warp has nothing to do
-          if (leader) {
-            if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status,
-                                                   kDevTimeoutMma))) {
-              ok = false;
-              break;
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * C::kTileN);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), phase, g.wait_limit, abort_flag, g.status,
+                                                 kDevTimeoutMma))) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_addr = sbase + stage * C::kStageBytes;
+          const int valid = min(C::kStageK, cnt - kb * C::kStageK);
+          // a ragged last stage runs only the 16-row MMA steps that hold segment rows; the rows past the
+          // segment inside the last of them are zeroed first, in this CTA's four boxes and the peer's
+          // (whole 128-byte lines, which the swizzle leaves in place)
+          const int nk = (valid + 15) / 16;
+          if (valid < 16 * nk) {
+            const int per_box = (16 * nk - valid) * 8;  // 16-byte pieces per box
+            for (int i = lane; i < 8 * per_box; i += 32) {
+              const int box = (i / per_box) & 3, rem = i % per_box;
+              const uint32_t addr = a_addr + box * C::kBoxBytes + (valid + rem / 8) * 128 + (rem % 8) * 16;
+              if (i < 4 * per_box) asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};\n" ::"r"(addr), "r"(0u) : "memory");
+              else asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %1, %1, %1};\n" ::"r"(peer_addr(addr, 1)), "r"(0u) : "memory");
             }
-            tc_fence_after();
-            if (lane == 0) {
-              const uint32_t b_addr = a_addr + C::kABytes;
+            asm volatile("fence.proxy.async.shared::cluster;\n" ::: "memory");
+          }
+          __syncwarp();
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t b_addr = a_addr + C::kABytes;
+            if (nk == C::kStageK / 16) {
 #pragma unroll
               for (int kk = 0; kk < C::kStageK / 16; ++kk)
                 mma_bf16_pair(d_tmem, desc_mnmajor(a_addr + kk * 16 * 128, C::kBoxBytes),
                               desc_mnmajor(b_addr + kk * 16 * 128, C::kBoxBytes), C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
-              mma_commit_both(empty_bar(stage));  // frees this stage in both CTAs once its MMAs are done
+            } else {
+              for (int kk = 0; kk < nk; ++kk)
+                mma_bf16_pair(d_tmem, desc_mnmajor(a_addr + kk * 16 * 128, C::kBoxBytes),
+                              desc_mnmajor(b_addr + kk * 16 * 128, C::kBoxBytes), C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
             }
-            issued = true;
+            mma_commit_both(empty_bar(stage));  // frees this stage in both CTAs once its MMAs are done
           }
+          issued = true;
           __syncwarp();
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
-          continue;
         }
-        const uint32_t fpar = leader ? phase : ((own_par >> stage) & 1u);
-        if (!leader) own_par ^= 1u << stage;
-        if (!__all_sync(0xffffffffu, mbar_wait(full_bar(stage), fpar, g.wait_limit, abort_flag, g.status,
-                                               kDevTimeoutMma))) {
-          ok = false;
-          break;
-        }
-        if (valid < C::kStageK) {
-          // this CTA's rows valid..127 of its four boxes: whole 128-byte lines
-          const int per_box = (C::kStageK - valid) * 8;
-          for (int i = lane; i < 4 * per_box; i += 32) {
-            const int box = i / per_box, rem = i - box * per_box;
-            const uint32_t addr = a_addr + box * C::kBoxBytes + (valid + rem / 8) * 128 + (rem % 8) * 16;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};\n" ::"r"(addr), "r"(0u) : "memory");
-          }
-          fence_async_smem();
-        }
+        if (!ok) break;
+        if (lane == 0) mma_commit_both(tfull_bar(buf));  // with no rows this arrives at once
         __syncwarp();
-        if (!leader) {
-          // this half is ready: tell the leader (its ready barrier of this stage)
-          if (lane == 0) mbar_arrive_cluster(leader_ready0 + 8u * stage);
-        } else {
-          const uint32_t rpar = (ready_par >> stage) & 1u;
-          ready_par ^= 1u << stage;
-          if (!__all_sync(0xffffffffu, mbar_wait_cluster(ready_bar(stage), rpar, g.wait_limit, abort_flag, g.status,
-                                                         kDevTimeoutMma))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t b_addr = a_addr + C::kABytes;
-#pragma unroll
-            for (int kk = 0; kk < C::kStageK / 16; ++kk)
-              mma_bf16_pair(d_tmem, desc_mnmajor(a_addr + kk * 16 * 128, C::kBoxBytes),
-                            desc_mnmajor(b_addr + kk * 16 * 128, C::kBoxBytes), C::kIdesc, (kb | kk) != 0 ? 1u : 0u);
-            mma_commit_both(empty_bar(stage));  // frees this stage in both CTAs once its MMAs are done
-          }
-          issued = true;
-        }
-        __syncwarp();
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1u;
-        }
       }
-      if (!ok) break;
-      if (leader && lane == 0) mma_commit_both(tfull_bar(buf));  // with no rows this arrives at once
-      __syncwarp();
-    }
-    if (leader && (!ok || *abort_flag) && issued && lane == 0) {
-      mma_commit_pair(drain_bar);
-      volatile int dummy = 0;
-      mbar_wait(drain_bar, 0, g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+      if ((!ok || *abort_flag) && issued && lane == 0) {
+        mma_commit_pair(drain_bar);
+        volatile int dummy = 0;
+        mbar_wait(drain_bar, 0, g.wait_limit, &dummy, g.status, kDevTimeoutDrain);
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5, both) --
