@@ -46,11 +46,11 @@ def _lib():
     return moe
 
 
-def _run(cfg, dout):
+def _run(cfg, dout, inp=None):
     import torch
 
     moe = _lib()
-    inp = synth.make_inputs(cfg)
+    inp = inp or synth.make_inputs(cfg)
     buf = moe.MoEBuffers(shape_of(cfg), upload(inp), train=True)
     buf.forward_train()
     grads = buf.make_grads()
@@ -364,3 +364,25 @@ def test_backward_f32_all_gradients(cfg):
         err = normwise_rel(r[n], getattr(ref, n))
         print(f"  {cfg.name} {n}: {err:.3e}")
         assert err <= TOL_F32, (n, err)
+
+
+@pytest.mark.parametrize("T", [256, 272, 263, 300, 9])
+def test_weight_gradient_segment_tails(T):
+    """The weight-gradient GEMM's last stage of a segment: with a zero gate matrix every token picks the
+    same two experts (the two largest gate biases), so both hold exactly T rows.  T = 256 leaves no ragged
+    stage; 272 ends on a whole 16-row MMA step (nothing to zero); 263 and 300 zero 9 and 4 rows past the
+    segment; 9 is a segment shorter than one MMA step.  dW1 and dW2 in full against the oracle, fed the
+    GPU's routing."""
+    cfg = _cfg(f"bwd_tail_{T}", T, 128, 4, 2, 256, math.inf, 57)
+    inp = synth.make_inputs(cfg)
+    inp.Wg = synth.to_storage(np.zeros((cfg.H, cfg.E)), cfg.dtype)
+    inp.bg = synth.to_storage(np.array([0.5, 0.25, -0.25, -0.5]), cfg.dtype)
+    dout = synth.normal(cfg.seed, 96, (cfg.T, cfg.H)).astype(np.float64)
+    r = _run(cfg, dout, inp)
+    assert (np.sort(r["topk_idx"], axis=1) == np.array([0, 1])).all()
+    ref = oracle.backward(inp.x, inp.Wg, inp.bg, inp.W1, inp.b1, inp.W2, inp.b2, cfg.k, cfg.CF, cfg.dtype, dout,
+                          D_AUX, D_Z, act=cfg.act, topk_idx=r["topk_idx"], dropped=r["dropped"])
+    print(cfg.name)
+    _check("dW1", r["dW1"], ref.dW1, per_expert=True)
+    _check("dW2", r["dW2"], ref.dW2, per_expert=True)
+    assert not r["dW1"][2:].any() and not r["dW2"][2:].any()  # experts without rows get zeros
