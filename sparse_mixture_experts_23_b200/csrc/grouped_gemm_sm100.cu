@@ -118,9 +118,20 @@ struct GemmArgs {
   int spread_rows;
   int32_t* status;
   long long wait_limit;
+  // GEMM1 on CTA pairs: the epilogue warps zero clear[0, clear_n) before their first tile, while the
+  // MMA warp runs that tile's main loop (the forward's out, which GEMM2 then accumulates into)
+  float4* clear;
+  long long clear_n;
 };
 
 using namespace sm100;
+
+// Zeroes p[0, n) in 16-byte stores, the CTAs' 2 KB runs interleaved across the grid.
+__device__ __noinline__ void clear_f4(float4* p, long long n, int cta, int ncta, int t) {
+  const long long stride = (long long)ncta * (32 * kEpiWarps);
+  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (long long i = (long long)cta * (32 * kEpiWarps) + t; i < n; i += stride) p[i] = z;
+}
 
 // Phi(u) = P(Z <= u) for a standard normal Z, so that GELU(u) = u Phi(u) = 0.5 u (1 + erf(u / sqrt 2)).
 // erfc(x) for x >= 0 from Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.26 (Hastings):
@@ -921,6 +932,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5, both) --
+    if constexpr (epi_h(EPI)) {
+      if (g.clear != nullptr) clear_f4(g.clear, g.clear_n, (int)blockIdx.x, (int)gridDim.x, (int)threadIdx.x - 64);
+    }
     const int quarter = warp & 3;
     const int half = (warp - 2) >> 2;
     const uint32_t tempty_leader0 = peer_addr(tempty_bar(0), 0);
@@ -1789,6 +1803,10 @@ cudaError_t launch_bwd_gemms_sm100(const BwdGemmArgs& a, cudaStream_t st, int* l
   return cudaSuccess;
 }
 
+bool ffn_gemm1_on_pairs(int H, int F, long long avg_rows) {
+  return F % 256 == 0 && H % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled();
+}
+
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches) {
   CUtensorMap ma1, mb1, ma2, mb2, mc1;
   if (!make_map_a(&ma1, a.x_perm, a.rows_cap, a.H) || !make_map_b(&mb1, a.W1, a.E, a.H, a.F) ||
@@ -1823,6 +1841,10 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.spread_rows = spread ? 1 : 0;
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
+  if (a.clear_out != nullptr) {
+    g1.clear = reinterpret_cast<float4*>(a.clear_out);
+    g1.clear_n = (long long)a.T * a.H / 4;
+  }
   const long long avg_rows = a.avg_rows;
   cudaError_t err = a.act == MOE_ACT_SILU
                         ? launch_bn<EPI_SILU>(a.F, ma1, mb1, mc1, g1, grid, avg_rows, st, (small || spread) ? &ma1s : nullptr)
@@ -1831,6 +1853,8 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   ++*launches;
 
   GemmArgs g2 = g1;
+  g2.clear = nullptr;
+  g2.clear_n = 0;
   g2.N = a.H;
   g2.K = a.F;
   g2.bias = reinterpret_cast<const __nv_bfloat16*>(a.b2);

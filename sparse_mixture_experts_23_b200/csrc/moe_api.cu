@@ -307,7 +307,7 @@ ReduceArgs reduce_args(const moe_shape_t* s, const moe_io_t* io, void* ws, int d
   return a;
 }
 
-moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st) {
+moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, bool clear_out = true) {
   const WsLayout L = ws_layout(*s);
   ScatterArgs a{};
   a.status = at<int32_t>(ws, L.status);
@@ -327,12 +327,19 @@ moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cuda
   a.row_token = at<int32_t>(ws, L.row_token);
   a.row_slot = at<int32_t>(ws, L.row_slot);
   a.x_perm = at<void>(ws, L.x_perm);
-  a.out = io->out;
+  a.out = clear_out ? io->out : nullptr;
   ++g_launches;
   return cuda_status(launch_scatter(a, num_sms(), st));
 }
 
-moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse, cudaStream_t st, bool train = false) {
+// Token choice, whole forward: whether GEMM1 zeroes out (its CTA-pair form, whose epilogue warps
+// are idle during the first tile) in place of the scatter, which then only copies rows.
+bool gemm1_clears_out(const moe_shape_t* s) {
+  return s->dtype == MOE_DTYPE_BF16 && ffn_gemm1_on_pairs(s->H, s->F, (long long)s->T * s->k / s->E);
+}
+
+moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse, cudaStream_t st, bool train = false,
+                    bool clear_out = false) {
   const WsLayout L = ws_layout(*s);
   FfnArgs a{};
   a.T = s->T;
@@ -363,6 +370,7 @@ moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse
   a.status = at<int32_t>(ws, L.status);
   a.wait_limit = g_wait_limit;
   a.num_sms = num_sms();
+  a.clear_out = clear_out ? io->out : nullptr;
   cudaError_t err = s->dtype == MOE_DTYPE_BF16 ? launch_ffn_bf16_sm100(a, st, &g_launches) : launch_ffn_f32(a, st, &g_launches);
   return cuda_status(err);
 }
@@ -556,10 +564,11 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws,
   if ((st = do_route(shape, io, ws, stream, kReduceLosses | kReduceDispatch)) != MOE_OK) return st;
   n += g_launches;
   g_launches = 0;
-  if ((st = do_scatter(shape, io, ws, stream)) != MOE_OK) return st;
+  const bool gc = gemm1_clears_out(shape);
+  if ((st = do_scatter(shape, io, ws, stream, !gc)) != MOE_OK) return st;
   n += g_launches;
   g_launches = 0;
-  st = do_ffn(shape, io, ws, 1, stream);
+  st = do_ffn(shape, io, ws, 1, stream, false, gc);
   g_launches += n;
   return st;
 }
@@ -601,8 +610,9 @@ moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, voi
     if ((st = do_ec_gather(shape, io, ws, stream)) != MOE_OK) return st;
     return do_ffn(shape, io, ws, 1, stream, true);
   }
-  if ((st = do_scatter(shape, io, ws, stream)) != MOE_OK) return st;
-  return do_ffn(shape, io, ws, 1, stream, true);
+  const bool gc = gemm1_clears_out(shape);
+  if ((st = do_scatter(shape, io, ws, stream, !gc)) != MOE_OK) return st;
+  return do_ffn(shape, io, ws, 1, stream, true, gc);
 }
 
 moe_status_t moe_backward(const moe_shape_t* shape, const moe_io_t* io, const moe_grad_t* grad, void* ws,

@@ -131,7 +131,7 @@ struct ScatterArgs {
   int32_t* row_token;
   int32_t* row_slot;
   void* x_perm;
-  float* out;  // cleared for this chunk's tokens (slot 0 blocks); may be null
+  float* out;  // the chunk's rows cleared, split over its k slot blocks; null: left alone (GEMM1 clears it)
 };
 
 struct FfnArgs {
@@ -156,6 +156,7 @@ struct FfnArgs {
   int32_t* status;
   long long wait_limit;
   int num_sms;
+  float* clear_out;  // [T, H] zeroed by GEMM1 (bf16, CTA-pair GEMM1 only: ffn_gemm1_on_pairs), or null
 };
 
 // ---- host-side helpers shared by the entry points (defined in moe_api.cu) ----
@@ -310,6 +311,9 @@ cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st);
 cudaError_t launch_ec_combine(const float* y, const int32_t* chosen, const float* topk_w, int T, int E, int C, int H,
                               float* out, cudaStream_t st);
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches);
+// Whether the bf16 FFN runs GEMM1 on CTA pairs (N = F, K = H, avg_rows rows per expert); its epilogue
+// warps can then zero out during their first tile, in place of the scatter.
+bool ffn_gemm1_on_pairs(int H, int F, long long avg_rows);
 cudaError_t launch_combine(const float* y, const int32_t* row_of, const float* topk_w, int T, int H, int k, float* out,
                            cudaStream_t st);
 cudaError_t launch_timeout_probe(int32_t* status, long long limit, cudaStream_t st);

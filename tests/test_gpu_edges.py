@@ -34,6 +34,7 @@ def _run_forward(cfg, inp=None, bg_override=None):
     if bg_override is not None:
         inp.bg = synth.to_storage(bg_override, cfg.dtype)
     buf = moe.MoEBuffers(shape_of(cfg), upload(inp))
+    buf.out.fill_(float("nan"))  # the forward must write (or clear) every element of out
     buf.forward()
     torch.cuda.synchronize()
     assert buf.device_status() == moe.MOE_OK
