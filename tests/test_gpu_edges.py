@@ -115,12 +115,16 @@ def test_empty_experts():
     assert (d.expert_counts[4:] == 0).all()
 
 
-def test_heavy_drops_and_all_dropped_tokens():
-    cfg = _cfg("drops", 256, 64, 4, 2, 128, 0.125, "bf16", 32)  # cap = ceil(0.125*256*2/4) = 16
+@pytest.mark.parametrize("T,H,F,CF,seed,cap", [
+    (256, 64, 128, 0.125, 32, 16),    # cap = ceil(0.125*256*2/4); single-CTA GEMMs, the scatter clears out
+    (1024, 128, 256, 0.15, 35, 77),   # T*k/E = 512 rows per expert on average: GEMM1 on CTA pairs zeroes out
+], ids=["single_cta", "cta_pair"])
+def test_heavy_drops_and_all_dropped_tokens(T, H, F, CF, seed, cap):
+    cfg = _cfg("drops", T, H, 4, 2, F, CF, "bf16", seed)
     bg = np.array([3.0, 2.5, -5.0, -5.0])  # everyone wants experts 0 and 1
-    r = _run_forward(cfg, bg_override=bg)
+    r = _run_forward(cfg, bg_override=bg)  # out starts as NaN
     d = _check_against_oracle(cfg, r)
-    assert d.cap == 16
+    assert d.cap == cap
     all_dropped = r["dropped"].all(axis=1)
     assert all_dropped.sum() > 100
     assert (r["out"][all_dropped] == 0).all()
