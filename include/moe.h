@@ -280,9 +280,9 @@ MOE_API moe_status_t moe_combine(const moe_shape_t* shape, const moe_io_t* io, v
                          cudaStream_t stream);
 
 /* moe_route, moe_permute and moe_expert_ffn(fuse_combine = 1) on one stream.  Where bf16 GEMM1 runs
- * on CTA pairs (F a multiple of 256, H of 128, T*k/E >= 256, pairs not switched off with
- * moe_set_kernel_options), its epilogue warps zero out during their first tile and the scatter
- * leaves out alone; the result is the same.  Token choice: the gate
+ * on CTA pairs (F a multiple of 256, H of 128, T*k/E >= 256 or under expert choice C >= 256, pairs
+ * not switched off with moe_set_kernel_options), its epilogue warps zero out during their first
+ * tile and the scatter (or gather) leaves out alone; the result is the same.  Token choice: the gate
  * (whose last block reduces the losses and the dispatch), the scatter, GEMM1 and GEMM2: 4 launches,
  * one more for either tensor-core gate form of moe_route or when the reduction does not fit the
  * gate's last block (k*ceil(T/32)*E > 4096).  Expert choice: 6 launches, 7 with the

@@ -7,7 +7,7 @@
 //                      compaction in token order -> chosen[e][0..C) ascending; per-token counts of
 //                      the experts that chose it; the last block to finish writes dropped[t]
 //   ec_gather_kernel   x rows into x_perm (row e*C + j = j-th token of expert e), row maps,
-//                      offsets e*C, and clearing of out
+//                      offsets e*C, and clearing of out where the forward's GEMM1 does not zero it
 //   ec_combine_kernel  unfused combine, token-major: out[t] = sum over the experts that chose t, in
 //                      ascending order, of p[t,e] * y[row] (no atomics; the same bits on every run)
 //
@@ -156,27 +156,42 @@ __global__ void __launch_bounds__(256) ec_gather_kernel(EcGatherArgs a) {
   const int tid = threadIdx.x;
   const long long rows = (long long)a.E * a.C;
   const long long r0 = (long long)blockIdx.x * 32;
+  // block (x, z) copies columns slice z of rows 32x..32x+31; slice 0 writes the row maps
+  const bool maps = blockIdx.y == 0;
   if (tid < 32) {
     const long long r = r0 + tid;
     int t = -1;
     if (r < rows) {
       t = a.chosen[r];
       if (t < 0 || t >= a.T) {  // caller-supplied token outside [0, T): a zero row for token 0, error recorded
-        atomicCAS(a.status, 0, kDevBadIndex);
+        if (maps) atomicCAS(a.status, 0, kDevBadIndex);
         t = -1;
       }
-      a.row_token[r] = t < 0 ? 0 : t;
-      a.row_slot[r] = (int)(r / a.C);
+      if (maps) {
+        a.row_token[r] = t < 0 ? 0 : t;
+        a.row_slot[r] = (int)(r / a.C);
+      }
     }
     tok_s[tid] = t;
   }
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0 && maps)
     for (int e = tid; e <= a.E; e += 256) a.offsets[e] = e * a.C;
   __syncthreads();
+  if (a.out != nullptr) {
+    // this block's share of out, interleaved over the grid; the stores go out before the copies
+    const long long ovec = (long long)a.T * a.H / 4;
+    const long long nb = (long long)gridDim.x * gridDim.y;
+    const long long b = (long long)blockIdx.y * gridDim.x + blockIdx.x;
+    float4* o = reinterpret_cast<float4*>(a.out);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (long long i = b * 256 + tid; i < ovec; i += nb * 256) o[i] = z;
+  }
   const int nvec = a.H * a.esize / 16;
+  const int c_lo = (int)((long long)nvec * blockIdx.y / gridDim.y);
+  const int w = (int)((long long)nvec * (blockIdx.y + 1) / gridDim.y) - c_lo;
   const uint4* xv = reinterpret_cast<const uint4*>(a.x);
   uint4* pv = reinterpret_cast<uint4*>(a.x_perm);
-  const int total = 32 * nvec;
+  const int total = 32 * w;
   constexpr int U = 8;
   for (int i = tid; i < total; i += 256 * U) {
     uint4 v[U];
@@ -186,7 +201,7 @@ __global__ void __launch_bounds__(256) ec_gather_kernel(EcGatherArgs a) {
       const int idx = i + u * 256;
       ok[u] = 0;
       if (idx < total) {
-        const int r = idx / nvec, c = idx % nvec;
+        const int r = idx / w, c = c_lo + idx % w;
         if (tok_s[r] >= 0) {
           v[u] = xv[(size_t)tok_s[r] * nvec + c];
           ok[u] = 1;
@@ -197,15 +212,11 @@ __global__ void __launch_bounds__(256) ec_gather_kernel(EcGatherArgs a) {
     for (int u = 0; u < U; ++u) {
       const int idx = i + u * 256;
       if (idx >= total) continue;
-      const int r = idx / nvec, c = idx % nvec;
+      const int r = idx / w, c = c_lo + idx % w;
       if (ok[u]) pv[(size_t)(r0 + r) * nvec + c] = v[u];
       else if (r0 + r < rows) pv[(size_t)(r0 + r) * nvec + c] = make_uint4(0u, 0u, 0u, 0u);  // invalid token
     }
   }
-  const long long ovec = (long long)a.T * a.H / 4;
-  float4* o = reinterpret_cast<float4*>(a.out);
-  const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (long long i = (long long)blockIdx.x * 256 + tid; i < ovec; i += (long long)gridDim.x * 256) o[i] = z;
 }
 
 // One block per row: out[t] += p[t,e] * y[row] (fp32 atomics; up to E rows meet in a token).
@@ -260,7 +271,12 @@ cudaError_t launch_ec_select(const EcSelectArgs& a, cudaStream_t st) {
 
 cudaError_t launch_ec_gather(const EcGatherArgs& a, cudaStream_t st) {
   const long long rows = (long long)a.E * a.C;
-  const int grid = (int)((rows + 31) / 32);
+  // each 32-row block's columns split over up to 4 slices of at least 8 vectors (128 B): one or two
+  // rounds of loads in flight per thread, as in the token-choice scatter
+  const int nvec = a.H * a.esize / 16;
+  int S = 1;
+  while (S < 4 && nvec / (2 * S) >= 8) S *= 2;
+  dim3 grid((unsigned)((rows + 31) / 32), (unsigned)S);
   ec_gather_kernel<<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }

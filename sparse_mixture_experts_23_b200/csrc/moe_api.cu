@@ -263,7 +263,7 @@ moe_status_t do_ec_select_and_losses(const moe_shape_t* s, const moe_io_t* io, v
   return cuda_status(launch_reduce(ra, st));
 }
 
-moe_status_t do_ec_gather(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st) {
+moe_status_t do_ec_gather(const moe_shape_t* s, const moe_io_t* io, void* ws, cudaStream_t st, bool clear_out = true) {
   const WsLayout L = ws_layout(*s);
   EcGatherArgs a{};
   a.status = at<int32_t>(ws, L.status);
@@ -278,7 +278,7 @@ moe_status_t do_ec_gather(const moe_shape_t* s, const moe_io_t* io, void* ws, cu
   a.row_token = at<int32_t>(ws, L.row_token);
   a.row_slot = at<int32_t>(ws, L.row_slot);
   a.x_perm = at<void>(ws, L.x_perm);
-  a.out = io->out;
+  a.out = clear_out ? io->out : nullptr;
   ++g_launches;
   return cuda_status(launch_ec_gather(a, st));
 }
@@ -332,10 +332,15 @@ moe_status_t do_scatter(const moe_shape_t* s, const moe_io_t* io, void* ws, cuda
   return cuda_status(launch_scatter(a, num_sms(), st));
 }
 
-// Token choice, whole forward: whether GEMM1 zeroes out (its CTA-pair form, whose epilogue warps
-// are idle during the first tile) in place of the scatter, which then only copies rows.
+// Expected rows per expert, for the FFN's tile-shape choice: T*k/E, or C under expert choice.
+long long ffn_avg_rows(const moe_shape_t* s) {
+  return s->routing == MOE_ROUTING_EXPERT_CHOICE ? ws_layout(*s).ec_cap : (long long)s->T * s->k / s->E;
+}
+
+// Whole forward: whether GEMM1 zeroes out (its CTA-pair form, whose epilogue warps are idle during
+// the first tile) in place of the scatter or gather, which then only copy rows.
 bool gemm1_clears_out(const moe_shape_t* s) {
-  return s->dtype == MOE_DTYPE_BF16 && ffn_gemm1_on_pairs(s->H, s->F, (long long)s->T * s->k / s->E);
+  return s->dtype == MOE_DTYPE_BF16 && ffn_gemm1_on_pairs(s->H, s->F, ffn_avg_rows(s));
 }
 
 moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse, cudaStream_t st, bool train = false,
@@ -351,7 +356,7 @@ moe_status_t do_ffn(const moe_shape_t* s, const moe_io_t* io, void* ws, int fuse
   a.rows_cap = (int)L.rows;
   // under expert choice row_slot holds the expert, so the weight of row r is topk_w[t*E + e]
   if (ec) a.k = s->E;
-  a.avg_rows = ec ? L.ec_cap : (long long)s->T * s->k / s->E;
+  a.avg_rows = ffn_avg_rows(s);
   a.offsets = at<int32_t>(ws, L.offsets);
   a.row_token = at<int32_t>(ws, L.row_token);
   a.row_slot = at<int32_t>(ws, L.row_slot);
@@ -556,8 +561,9 @@ moe_status_t moe_forward(const moe_shape_t* shape, const moe_io_t* io, void* ws,
     // router, per-expert selection, losses, gather, GEMM1, GEMM2 (each call adds its launches)
     if ((st = do_route(shape, io, ws, stream, 0)) != MOE_OK) return st;
     if ((st = do_ec_select_and_losses(shape, io, ws, stream)) != MOE_OK) return st;
-    if ((st = do_ec_gather(shape, io, ws, stream)) != MOE_OK) return st;
-    return do_ffn(shape, io, ws, 1, stream);
+    const bool gc = gemm1_clears_out(shape);
+    if ((st = do_ec_gather(shape, io, ws, stream, !gc)) != MOE_OK) return st;
+    return do_ffn(shape, io, ws, 1, stream, false, gc);
   }
   int n = 0;
   // the router emits the chunk histograms itself, so one reduction serves losses and dispatch
@@ -607,8 +613,9 @@ moe_status_t moe_forward_train(const moe_shape_t* shape, const moe_io_t* io, voi
   if ((st = do_route(shape, io, ws, stream, ec ? 0 : kReduceLosses | kReduceDispatch, true)) != MOE_OK) return st;
   if (ec) {
     if ((st = do_ec_select_and_losses(shape, io, ws, stream)) != MOE_OK) return st;
-    if ((st = do_ec_gather(shape, io, ws, stream)) != MOE_OK) return st;
-    return do_ffn(shape, io, ws, 1, stream, true);
+    const bool gc = gemm1_clears_out(shape);
+    if ((st = do_ec_gather(shape, io, ws, stream, !gc)) != MOE_OK) return st;
+    return do_ffn(shape, io, ws, 1, stream, true, gc);
   }
   const bool gc = gemm1_clears_out(shape);
   if ((st = do_scatter(shape, io, ws, stream, !gc)) != MOE_OK) return st;

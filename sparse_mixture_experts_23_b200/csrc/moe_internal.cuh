@@ -114,7 +114,7 @@ struct EcGatherArgs {
   int32_t* row_token;     // [E*C] out
   int32_t* row_slot;      // [E*C] out: the expert
   void* x_perm;           // [E*C][H] out
-  float* out;             // [T][H] cleared
+  float* out;             // [T][H] cleared; null: left alone (GEMM1 zeroes it)
 };
 
 
