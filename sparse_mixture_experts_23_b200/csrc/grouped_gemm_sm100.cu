@@ -1690,11 +1690,16 @@ cudaError_t launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUte
 // 256-wide tiles, 3.03 waves, beat 128-wide, 6.05 waves; 64-wide was far slower).
 int pick_bn_small(int N) { return N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64); }
 
+// Whether a grouped GEMM with N output columns, contraction K and avg_rows rows per expert runs on
+// CTA pairs (256 x 256 tiles) rather than single-CTA tiles.
+bool pair_tiles_fit(int N, int K, long long avg_rows) {
+  return N % 256 == 0 && K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled();
+}
+
 template <int EPI>
 cudaError_t launch_bn(int N, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmArgs& g,
                       int grid, long long avg_rows, cudaStream_t st, const CUtensorMap* ma16 = nullptr) {
-  if (N % 256 == 0 && g.K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled())
-    return launch_pair<EPI>(ma, mb, mc, g, grid, st);
+  if (pair_tiles_fit(N, g.K, avg_rows)) return launch_pair<EPI>(ma, mb, mc, g, grid, st);
   if (ma16 != nullptr && g.a_box_rows > 0 && !g.spread_rows) {
     const int bn = pick_bn_small(N);
     if (bn == 256) return launch_one<256, EPI>(ma, mb, g, grid, st, ma16);
@@ -1712,7 +1717,7 @@ cudaError_t launch_dgrad(const void* A, int rows_cap, const void* W, int E, int 
                          long long avg_rows, cudaStream_t st) {
   CUtensorMap ma, mb;
   if (!make_map_a(&ma, A, rows_cap, K)) return cudaErrorInvalidValue;
-  if (N % 256 == 0 && K % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled()) {
+  if (pair_tiles_fit(N, K, avg_rows)) {
     if (!make_map_bk(&mb, W, E, N, K, PairCfg::kHalfN)) return cudaErrorInvalidValue;
     return launch_pair<EPI, true>(ma, mb, ma, g, grid, st);
   }
@@ -1803,9 +1808,7 @@ cudaError_t launch_bwd_gemms_sm100(const BwdGemmArgs& a, cudaStream_t st, int* l
   return cudaSuccess;
 }
 
-bool ffn_gemm1_on_pairs(int H, int F, long long avg_rows) {
-  return F % 256 == 0 && H % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM && pair_mode_enabled();
-}
+bool ffn_gemm1_on_pairs(int H, int F, long long avg_rows) { return pair_tiles_fit(F, H, avg_rows); }
 
 cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launches) {
   CUtensorMap ma1, mb1, ma2, mb2, mc1;
@@ -1842,8 +1845,15 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   g1.status = a.status;
   g1.wait_limit = a.wait_limit;
   if (a.clear_out != nullptr) {
-    g1.clear = reinterpret_cast<float4*>(a.clear_out);
-    g1.clear_n = (long long)a.T * a.H / 4;
+    if (ffn_gemm1_on_pairs(a.H, a.F, a.avg_rows)) {
+      g1.clear = reinterpret_cast<float4*>(a.clear_out);
+      g1.clear_n = (long long)a.T * a.H / 4;
+    } else {
+      // only the CTA-pair GEMM1 zeroes out; callers ask for it only then, but out must hold zeros
+      // before GEMM2 whichever kernel runs
+      const cudaError_t e = cudaMemsetAsync(a.clear_out, 0, (size_t)a.T * a.H * sizeof(float), st);
+      if (e != cudaSuccess) return e;
+    }
   }
   const long long avg_rows = a.avg_rows;
   cudaError_t err = a.act == MOE_ACT_SILU
@@ -1868,8 +1878,7 @@ cudaError_t launch_ffn_bf16_sm100(const FfnArgs& a, cudaStream_t st, int* launch
   // top-1 layers on single-CTA tiles with a long K (the Switch shape: 512 tiles of K = 4096 are 3.46
   // waves on 148 SMs): two K halves per tile even out the last wave; with one slot per token each
   // element of out still receives a fixed pair of adds
-  const bool pair2 = a.H % PairCfg::kTileN == 0 && a.F % PairCfg::kStageK == 0 && avg_rows >= PairCfg::kTileM &&
-                     pair_mode_enabled();
+  const bool pair2 = pair_tiles_fit(a.H, a.F, avg_rows);
   if (a.fuse_combine && a.k == 1 && !small && !pair2 && a.F / BK >= 32) g2.k_splits = 2;
   if (a.fuse_combine)
     err = launch_bn<EPI_COMBINE>(a.H, ma2, mb2, ma2, g2, grid, avg_rows, st, (small || spread) ? &ma2s : nullptr);
